@@ -1,0 +1,238 @@
+/*
+ * wq.h -- C ABI of the weight-only quantized linear layer for LLM decode on
+ * NVIDIA B200 (sm_100a).
+ *
+ *     y[M][N] = x[M][K] . dequant(Wq)^T        (bf16 in, bf16 out)
+ *
+ * Two weight formats:
+ *   W8A16  int8 weights, one bf16 scale per output channel, no zero point:
+ *          w[n][k] = s[n] * q[n][k]
+ *          ("Per-channel W8A16 quantization", tileInfer README, Features
+ *          table.)
+ *   W4A16  unsigned 4-bit weights q in [0,15] with a bf16 scale and a 4-bit
+ *          zero point per (group of `group` consecutive k, output channel):
+ *          w[n][k] = s[n][k/group] * (q[n][k] - z[n][k/group])
+ *          (A WnA16 kernel shared by several checkpoint formats needs the same
+ *          layout, scales, zero points and group size. This is the review of
+ *          Figure 4 in "Toward a Cleaner Quantization Stack in SGLang".)
+ *
+ * Two kernel families sit behind one call:
+ *   - a GEMV for decode-sized M, with register-level dequantization and
+ *     128-bit weight loads ("BitBLAS-style GEMV", tileInfer README, Features
+ *     table). Its fp32 dot products run on mma.sync tensor-core fragments.
+ *   - a small-M GEMM (tcgen05 tensor cores, accumulators in tensor memory)
+ *     with split-K and a fixed-order fp32 reduction ("split_k" auto-tuning,
+ *     Mit han lab Llm awq Kernel Selection Thresholds, The Insight).
+ * A per-(M,K,N,bits,group) dispatcher picks the kernel and split factor. It
+ * starts from the pages' rule (fewer than 8 tokens -> GEMV, else GEMM with
+ * split 8; same page) and is overridden by measured timings (wq_tune).
+ *
+ * Conventions for every entry point:
+ *   - The return value is a wq_status: 0 on success, negative on error.
+ *     No call aborts, traps or throws.
+ *   - "device" pointers are CUDA device pointers on the current device.
+ *     "host" pointers are ordinary host memory.
+ *   - The caller owns every buffer. No call allocates device memory, except
+ *     wq_tune. wq_tune allocates and frees only its timing events.
+ *   - Work is enqueued on `stream` (0 = legacy default stream). Calls return
+ *     after the enqueue, with no implicit synchronization, unless the entry
+ *     says "synchronizes".
+ *   - bf16 values are passed as their uint16_t bit patterns.
+ *   - Shape rules: 1 <= N, N % 16 == 0. W8A16: K % 32 == 0.
+ *     W4A16: group == 128, K % 128 == 0. 1 <= M <= 128.
+ *     x, y and every packed buffer must be 16-byte aligned.
+ *   - Packed buffers are written by wq_pack_int8 / wq_pack_int4 and are
+ *     opaque. wq_packed_bytes gives their sizes. Their layout is described
+ *     in the library's design notes.
+ */
+#ifndef WQ_H
+#define WQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WQ_OK = 0,
+    WQ_ERR_NULL = -1,      /* a required pointer is NULL */
+    WQ_ERR_SHAPE = -2,     /* M, K or N outside the shape rules */
+    WQ_ERR_ALIGN = -3,     /* a pointer is not 16-byte aligned */
+    WQ_ERR_GROUP = -4,     /* unsupported bits / group combination */
+    WQ_ERR_HEADER = -5,    /* packed trailer does not match the arguments */
+    WQ_ERR_WORKSPACE = -6, /* split > 1 needs a larger split-K workspace */
+    WQ_ERR_CUDA = -7,      /* a CUDA runtime call or a launch failed */
+    WQ_ERR_TUNING = -8,    /* tuning file unreadable or malformed */
+    WQ_ERR_TIMEOUT = -9,   /* a bounded device-side wait gave up */
+    WQ_ERR_ARCH = -10,     /* device is not sm_100 (B200 class) */
+    WQ_ERR_VARIANT = -11   /* forced variant / split not valid for the shape */
+} wq_status;
+
+/* Kernel variants (wq_linear_forced, wq_get_choice). */
+#define WQ_VARIANT_AUTO (-1)
+#define WQ_VARIANT_GEMV 0 /* mma.sync register-dequant GEMV, M <= 32 */
+#define WQ_VARIANT_GEMM 1 /* tcgen05 split-K GEMM, M <= 128 */
+
+/* Static description of a status code. Host. Never NULL. */
+const char *wq_strerror(int status);
+
+/* Library version: major * 10000 + minor * 100 + patch. Host. */
+int wq_version(void);
+
+/* Byte sizes of the three packed buffers for a weight of shape [N][K].
+ * bits = 8 (group must be 0) or 4 (group must be 128). zero_bytes is 0 for
+ * INT8. Any output pointer may be NULL. Host, no device work. */
+int wq_packed_bytes(int bits, int K, int N, int group, size_t *wq_bytes,
+                    size_t *scale_bytes, size_t *zero_bytes);
+
+/* ---------------------------------------------------------------------
+ * Quantizers: fp32 source weights -> canonical quantized tensors.
+ * These are how the workloads' weights are made. They are not the layer
+ * itself. Every decision is taken in binary64, as in the CPU oracle, so
+ * the codes are bit-exact with it.
+ * ------------------------------------------------------------------- */
+
+/* Symmetric per-output-channel INT8 (per-channel W8A16, tileInfer README,
+ * Features table).
+ *   W       device, fp32 [N][K], row-major
+ *   q_out   device, int8 [N][K]
+ *   s_out   device, bf16 [N]:  s = bf16_rne(max_k |W[n][k]| / 127)
+ *   q = clamp(rint(W / s), -127, 127), ties to even. A row with s == 0 gets q = 0.
+ * One CUDA block per row. */
+int wq_quantize_int8(const float *W, int K, int N, int8_t *q_out, uint16_t *s_out,
+                     cudaStream_t stream);
+
+/* Asymmetric INT4 with `group` consecutive k per scale / zero point.
+ *   W       device, fp32 [N][K]
+ *   q_out   device, uint32 [N][K/8]; nibble j of word (n,c) = q[n][8c+j]
+ *   s_out   device, bf16 [N][K/group]: s = bf16 rounded toward +inf of
+ *           (hi - lo) / 15, where lo = min(min W, 0) and hi = max(max W, 0)
+ *   z_out   device, uint32 [N][ceil(K/group/8)]; nibble j of word (n,c) is
+ *           z[n][8c+j] = clamp(rint(-lo / s), 0, 15). Unused nibbles are 0.
+ *   q = clamp(rint(W / s) + z, 0, 15). A group with hi == lo gets s = z = q = 0. */
+int wq_quantize_int4(const float *W, int K, int N, int group, uint32_t *q_out,
+                     uint16_t *s_out, uint32_t *z_out, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------
+ * Packers: canonical tensors -> the GPU layout read by every kernel.
+ * Packing is a separate step from running the layer: the scheme-vs-kernel
+ * split of "Toward a Cleaner Quantization Stack in SGLang", Figure 1.
+ * ------------------------------------------------------------------- */
+
+/* q: device int8 [N][K]; scales: device bf16 [N].
+ * wq_out / scales_out: device buffers of wq_packed_bytes(8, K, N, 0, ...). */
+int wq_pack_int8(const int8_t *q, const uint16_t *scales, int K, int N, void *wq_out,
+                 void *scales_out, cudaStream_t stream);
+
+/* q: device uint32 [N][K/8] (low nibble first); scales: device bf16
+ * [N][K/group]; zeros: device uint32 [N][ceil(K/group/8)].
+ * Outputs sized by wq_packed_bytes(4, K, N, group, ...). */
+int wq_pack_int4(const uint32_t *q, const uint16_t *scales, const uint32_t *zeros, int K,
+                 int N, int group, void *wq_out, void *scales_out, void *zeros_out,
+                 cudaStream_t stream);
+
+/* Reads the 64-byte trailer that the packers write after the packed weights
+ * and checks it against (bits, K, N, group). Returns WQ_ERR_HEADER on a
+ * mismatch. Synchronizes `stream`, so call it once at load time, not per
+ * step. */
+int wq_check_packed(const void *Wq, int bits, int K, int N, int group, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------
+ * The layer.
+ * ------------------------------------------------------------------- */
+
+/* y = x . dequant(Wq)^T.
+ *   x       device, bf16 [M][K], row-major, 16-byte aligned
+ *   Wq, scales, zeros   device, packed by wq_pack_int8 / wq_pack_int4
+ *           (zeros = NULL for INT8)
+ *   group   0 for INT8 per-channel, 128 for INT4
+ *   y       device, bf16 [M][N], row-major, 16-byte aligned. Every element
+ *           is written: bf16_rne of the fp32-accumulated sum.
+ * The kernel and split factor come from the dispatcher (tuned table, else
+ * the default rule). A split factor > 1 uses the workspace registered with
+ * wq_set_workspace for the current device. Calls that share that workspace
+ * must not overlap on the GPU (keep them on one stream). */
+int wq_linear(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
+              const void *zeros, int group, int N, uint16_t *y, cudaStream_t stream);
+
+/* wq_linear with an explicit kernel variant (WQ_VARIANT_*) and split factor.
+ * variant = WQ_VARIANT_AUTO, or split = 0, leaves that choice to the dispatcher.
+ * GEMV: split = K-slices per 16-row block, one of 1, 2, 4, 8.
+ * GEMM: split = K-splits, 1 <= split <= min(32, ceil(K/128)).
+ * Returns WQ_ERR_VARIANT if the pair does not fit the shape. */
+int wq_linear_forced(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
+                     const void *zeros, int group, int N, uint16_t *y, int variant, int split,
+                     cudaStream_t stream);
+
+/* wq_linear_forced with an explicit split-K workspace, for callers that run
+ * several layers on concurrent streams (ws = NULL: the registered one). */
+int wq_linear_ex(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
+                 const void *zeros, int group, int N, uint16_t *y, int variant, int split,
+                 void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Bytes of split-K workspace for M tokens, N channels and up to max_split
+ * splits: the fp32 partial sums [split][M][N] and one ticket counter per
+ * 128-channel panel. Host. */
+size_t wq_workspace_bytes(int M, int N, int max_split);
+
+/* Registers a caller-owned device workspace for the current device, used by
+ * wq_linear. Zeroes its counters with a synchronous cudaMemset. The kernels
+ * leave the counters at zero after every call. ws = NULL unregisters. */
+int wq_set_workspace(void *ws, size_t bytes);
+
+/* ---------------------------------------------------------------------
+ * Dispatcher / tuner. The table is keyed by (device name, SM count, M, K, N,
+ * bits, group) and guarded by a mutex.
+ * ------------------------------------------------------------------- */
+
+/* Times every valid (variant, split) for the shape on the caller's own
+ * buffers with CUDA events: `warmup` untimed and `iters` timed calls each.
+ * It keeps the fastest by median time. On an exact tie the later, larger
+ * split wins, as in the split_k auto-tune loop of Mit han lab Llm awq Kernel
+ * Selection Thresholds, The Insight. Overwrites y. Synchronizes `stream`.
+ * Needs a registered workspace that fits split 32 to try every split. */
+int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
+            const void *zeros, int group, int N, uint16_t *y, int warmup, int iters,
+            cudaStream_t stream);
+
+/* The (variant, split) that wq_linear would use for this shape now. Host. */
+int wq_get_choice(int M, int K, int N, int bits, int group, int *variant, int *split);
+
+/* Sets one table entry by hand (for tests and offline tables). Host. */
+int wq_set_choice(int M, int K, int N, int bits, int group, int variant, int split);
+
+/* Drops every tuned entry. Host. */
+int wq_clear_tuning(void);
+
+/* Text file, one entry per line. Host. WQ_ERR_TUNING on a malformed line;
+ * in that case the table is left unchanged. */
+int wq_save_tuning(const char *path);
+int wq_load_tuning(const char *path);
+
+/* ---------------------------------------------------------------------
+ * Debug views of the packed layout (for the bit-exact tests).
+ * ------------------------------------------------------------------- */
+
+/* Unpacks the packed weights to integers: q_out int8 [N][K] (INT4: 0..15;
+ * INT8: -128..127) and, for INT4, z_out int8 [N][K/group]. Device pointers. */
+int wq_unpack_debug(const void *Wq, const void *zeros, int bits, int K, int N, int group,
+                    int8_t *q_out, int8_t *z_out, cudaStream_t stream);
+
+/* Dequantized weights in fp32, w_out [N][K]. s*(q - z) is exact in fp32. */
+int wq_dequant_debug(const void *Wq, const void *scales, const void *zeros, int bits, int K,
+                     int N, int group, float *w_out, cudaStream_t stream);
+
+/* Reads and clears the device-side error word that a kernel sets when a
+ * bounded wait gives up. Returns WQ_OK or WQ_ERR_TIMEOUT. Synchronizes
+ * `stream`. */
+int wq_device_error(cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H */

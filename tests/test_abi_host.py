@@ -1,0 +1,107 @@
+"""Host-side checks of the C ABI (no GPU needed, no compute calls).
+
+libwq.so must load, export every function include/wq.h declares, and its
+host-only entry points (status strings, sizes, tuning-file parsing) must
+behave as documented.
+"""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import weight_only_quantized_02_b200 as wq
+
+
+def test_library_exports_every_header_symbol():
+    names = wq.header_functions()
+    assert "wq_linear" in names and "wq_pack_int4" in names and "wq_pack_int8" in names
+    missing = [n for n in names if not hasattr(wq.lib, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_every_header_symbol():
+    missing = [n for n in wq.header_functions() if not callable(getattr(wq, n, None))]
+    assert not missing, missing
+
+
+def test_exports_with_nm():
+    out = subprocess.run(["nm", "-D", "--defined-only", wq.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in wq.header_functions():
+        assert n in exported, n
+
+
+def test_strerror_is_defined_for_every_status():
+    for code in list(wq.STATUS) + [-99, 7]:
+        s = wq.strerror(code)
+        assert isinstance(s, str) and s
+    assert wq.strerror(0) == "ok"
+
+
+def test_packed_bytes():
+    wb, sb, zb = wq.wq_packed_bytes(8, 5120, 17408, 0)
+    assert wb == 5120 * 17408 + 64 and sb == 17408 * 2 and zb == 0
+    wb, sb, zb = wq.wq_packed_bytes(4, 5120, 25600, 128)
+    assert wb == 5120 * 25600 // 2 + 64
+    assert sb == 25600 * 40 * 2 and zb == 25600 * 40 // 2
+    # ragged: N not a multiple of the 128-row panel, K not a multiple of the 128-k block
+    wb, sb, zb = wq.wq_packed_bytes(8, 1120, 400, 0)
+    assert wb == 512 * 1152 + 64 and sb == 512 * 2
+
+
+@pytest.mark.parametrize("bits,K,N,group,status", [
+    (8, 1024, 1024, 128, -4),   # INT8 takes no group
+    (4, 1024, 1024, 64, -4),    # only group 128
+    (4, 1000, 1024, 128, -2),   # K not a multiple of the group
+    (8, 1000, 1024, 0, -2),     # K not a multiple of 32
+    (8, 1024, 1000, 0, -2),     # N not a multiple of 16
+    (8, 0, 1024, 0, -2),
+    (3, 1024, 1024, 0, -4),
+])
+def test_packed_bytes_rejects(bits, K, N, group, status):
+    a = ctypes.c_size_t()
+    assert wq.lib.wq_packed_bytes(bits, K, N, group, ctypes.byref(a), None, None) == status
+
+
+def test_workspace_bytes():
+    # 40 panel tickets padded to 256 bytes + fp32 partials
+    assert wq.wq_workspace_bytes(128, 5120, 32) == 256 + 32 * 128 * 5120 * 4
+    assert wq.wq_workspace_bytes(16, 5120, 1) == 256
+    assert wq.wq_workspace_bytes(0, 5120, 4) == 0
+
+
+def test_null_pointer_checks_need_no_device():
+    assert wq.lib.wq_linear(None, 1, 1024, None, None, None, 0, 1024, None, None) == -1
+    assert wq.lib.wq_pack_int8(None, None, 1024, 1024, None, None, None) == -1
+    assert wq.lib.wq_quantize_int4(None, 1024, 16, 128, None, None, None, None) == -1
+
+
+def test_tuning_file_parse_errors(tmp_path):
+    good = tmp_path / "good.txt"
+    good.write_text("# comment\nNVIDIA B200|148 1 5120 17408 8 0 0 4 12.500\n")
+    assert wq.wq_load_tuning(str(good)) == 0
+    for bad_line in [
+        "NVIDIA B200|148 1 5120 17408 8 0 0 3 12.5\n",      # GEMV split must be 1/2/4/8
+        "NVIDIA B200|148 200 5120 17408 8 0 1 4 12.5\n",    # M > 128
+        "NVIDIA B200|148 1 5120 17408 8 64 0 4 12.5\n",     # bad group
+        "NVIDIA B200 1 5120 17408 8 0 0 4 12.5\n",          # no device key separator
+        "NVIDIA B200|148 1 5120 17408 8 0 0\n",             # truncated
+        "NVIDIA B200|148 1 5120 17408 8 0 0 4 12.5 extra\n",
+        "NVIDIA B200|148 64 17408 5120 4 128 1 64 1.0\n",   # split above 32
+    ]:
+        p = tmp_path / "bad.txt"
+        p.write_text(bad_line)
+        assert wq.wq_load_tuning(str(p)) == -8, bad_line
+    assert wq.wq_load_tuning(str(tmp_path / "missing.txt")) == -8
+    assert wq.lib.wq_load_tuning(None) == -1
+
+
+def test_no_oracle_in_product():
+    """The product package never imports or links the oracle."""
+    here = os.path.dirname(wq.__file__)
+    for root, _, files in os.walk(here):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(root, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text and "liboracle" not in text, f

@@ -1,0 +1,306 @@
+"""Parity of the CUDA layer with the CPU oracle, element by element.
+
+Shapes span several 16-row blocks, 128-row panels and 128-k blocks with a
+ragged tail (N not a multiple of 128, INT8 K not a multiple of 128), every
+token-tile boundary of both kernels (M = 1, 7, 8, 9, 16, 17, 32, 33, 64, 65,
+100, 128), every GEMV K-slice count and every GEMM split factor.
+Tolerance: |y_gpu - y_ref| <= 1e-2 * max(|y_ref|, 1).  Closed-form special
+cases (one-hot activations, one-hot and identity weights, zero scales,
+power-of-two scaling) are compared bit for bit.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import wq_inputs as gen
+import weight_only_quantized_02_b200 as wq
+from wqtest_helpers import (assert_parity, bf16_dev, dev, oracle_linear, pack_canonical_int4, pack_canonical_int8,
+                            quantize_and_pack, to_dev, workspace, y_host)
+
+pytestmark = pytest.mark.gpu
+
+GEMV, GEMM = wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM
+SHAPES = {8: (1120, 400), 4: (1152, 400)}  # (K, N): 3 full panels + a 16-row tail
+M_ALL = [1, 7, 8, 9, 16, 17, 32, 33, 64, 65, 100, 128]
+
+
+@pytest.fixture(scope="module")
+def ws():
+    t = workspace(128, 1024, 32)
+    wq.wq_set_workspace(t)
+    yield t
+    wq.wq_set_workspace(None)
+
+
+@pytest.fixture(scope="module", params=[8, 4], ids=["w8", "w4g128"])
+def weight(request):
+    bits = request.param
+    K, N = SHAPES[bits]
+    W = gen.W_f32(0, N, K)
+    pw, canon = quantize_and_pack(W, bits)
+    return bits, K, N, pw, canon
+
+
+def _cases(M, K):
+    kb = (K + 127) // 128
+    out = []
+    if M <= 32:
+        out += [(GEMV, ks) for ks in (1, 2, 4, 8)]
+    out += [(GEMM, s) for s in (1, 2, 4, 8, 16, 32) if s <= kb]
+    return out
+
+
+@pytest.mark.parametrize("M", M_ALL)
+def test_linear_parity_all_variants(weight, ws, M):
+    bits, K, N, pw, canon = weight
+    x = gen.x_bf16(M, K)
+    y_ref = oracle_linear(x, canon, bits)
+    xd = bf16_dev(x)
+    for variant, split in _cases(M, K):
+        y = wq.wq_linear_forced(xd, pw, variant, split)
+        assert_parity(y_host(y), y_ref, f"bits={bits} M={M} variant={variant} split={split}")
+    # the dispatcher's own choice
+    assert_parity(y_host(wq.wq_linear(xd, pw)), y_ref, f"bits={bits} M={M} auto")
+
+
+def test_deterministic_and_splits_agree(weight, ws):
+    bits, K, N, pw, canon = weight
+    x = bf16_dev(gen.x_bf16(24, K))
+    for variant, split in _cases(24, K):
+        a = wq.wq_linear_forced(x, pw, variant, split)
+        b = wq.wq_linear_forced(x, pw, variant, split)
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), (variant, split)
+
+
+def test_repeated_dispatch_resets_tickets(weight, ws):
+    """Many split-K calls in a row reuse the workspace tickets; each must
+    leave them at zero for the next (different split, different M)."""
+    bits, K, N, pw, canon = weight
+    for M, split in [(16, 2), (16, 8), (40, 4), (128, 9), (16, 2)]:
+        x = gen.x_bf16(M, K)
+        y = wq.wq_linear_forced(bf16_dev(x), pw, GEMM, split)
+        assert_parity(y_host(y), oracle_linear(x, canon, bits), f"M={M} split={split}")
+    ticket = ws[: 4 * ((N + 127) // 128)].view(torch.int32)
+    assert int(ticket.abs().sum()) == 0
+
+
+# ---------------------------------------------------------------------------
+# closed-form special cases, bit for bit
+# ---------------------------------------------------------------------------
+
+def _all_cases(M, K):
+    return _cases(M, K)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_one_hot_activations_pick_weights_exactly(bits, ws):
+    K, N = SHAPES[bits]
+    M = 5
+    g = gen.generator("misc", 21)
+    W = gen.W_f32(0, N, K)
+    pw, canon = quantize_and_pack(W, bits)
+    ks = [0, 127, 128, 641, K - 1]
+    x = np.zeros((M, K), np.uint16)
+    for m, k in enumerate(ks):
+        x[m, k] = 0x3F80  # 1.0
+    want = oracle.bf16_to_f64(oracle.bf16_rne_of(oracle_linear(x, canon, bits)))
+    for variant, split in _all_cases(M, K):
+        y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
+        assert np.array_equal(y, want), (variant, split)
+
+
+def test_one_hot_int8_weights_exact(ws):
+    K, N, M = 1120, 400, 9
+    g = gen.generator("misc", 22)
+    q = np.zeros((N, K), np.int8)
+    cols = g.integers(0, K, N)
+    q[np.arange(N), cols] = g.integers(-128, 128, N).astype(np.int8)
+    s = gen.f32_to_bf16_bits(g.uniform(1e-3, 2e-2, N).astype(np.float32))
+    pw = pack_canonical_int8(q, s)
+    x = gen.x_bf16(M, K)
+    want = oracle.bf16_to_f64(oracle.bf16_rne_of(oracle.linear_int8(x, q, s)))
+    for variant, split in _all_cases(M, K):
+        y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
+        assert np.array_equal(y, want), (variant, split)
+
+
+def test_one_hot_int4_weights_exact(ws):
+    """q = z except one (n, k) per row.  Power-of-two scales keep s*(q - z)
+    exact in bf16, so the GEMM's bf16 weight tile is exact too."""
+    K, N, M = 1152, 400, 9
+    G = 128
+    g = gen.generator("misc", 23)
+    zn = g.integers(0, 16, size=(N, K // G))
+    qn = np.repeat(zn, G, axis=1).astype(np.int64)
+    cols = g.integers(0, K, N)
+    qn[np.arange(N), cols] = g.integers(0, 16, N)
+    q = np.zeros((N, K // 8), np.uint32)
+    for k in range(K):
+        q[:, k // 8] |= qn[:, k].astype(np.uint32) << np.uint32(4 * (k % 8))
+    z = np.zeros((N, oracle.zero_words_per_row(K)), np.uint32)
+    for gi in range(K // G):
+        z[:, gi // 8] |= zn[:, gi].astype(np.uint32) << np.uint32(4 * (gi % 8))
+    s = (0x3F80 + (g.integers(-9, 3, size=(N, K // G)) << 7)).astype(np.uint16)  # 2^e
+    pw = pack_canonical_int4(q, s, z)
+    x = gen.x_bf16(M, K)
+    want = oracle.bf16_to_f64(oracle.bf16_rne_of(oracle.linear_int4(x, q, s, z)))
+    for variant, split in _all_cases(M, K):
+        y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
+        assert np.array_equal(y, want), (variant, split)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_identity_weights_reproduce_x(bits, ws):
+    K = N = 384 if bits == 8 else 512
+    M = 33
+    x = gen.x_bf16(M, K)
+    if bits == 8:
+        pw = pack_canonical_int8((np.eye(N) * 64).astype(np.int8), np.full(N, 0x3C80, np.uint16))
+    else:
+        qn = np.full((N, K), 8, np.uint32)
+        np.fill_diagonal(qn, 9)
+        q = np.zeros((N, K // 8), np.uint32)
+        for k in range(K):
+            q[:, k // 8] |= qn[:, k] << np.uint32(4 * (k % 8))
+        z = np.zeros((N, oracle.zero_words_per_row(K)), np.uint32)
+        for gi in range(K // 128):
+            z[:, gi // 8] |= np.uint32(8) << np.uint32(4 * (gi % 8))
+        pw = pack_canonical_int4(q, np.full((N, K // 128), 0x3F80, np.uint16), z)
+    want = oracle.bf16_to_f64(x)
+    for variant, split in _all_cases(M, K):
+        y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
+        assert np.array_equal(y, want), (variant, split)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_zero_scales_give_zero(bits, ws):
+    K, N = SHAPES[bits]
+    g = gen.generator("misc", 24)
+    if bits == 8:
+        pw = pack_canonical_int8(g.integers(-127, 128, (N, K), dtype=np.int8), np.zeros(N, np.uint16))
+    else:
+        q = g.integers(0, 2**32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
+        z = g.integers(0, 2**32, size=(N, oracle.zero_words_per_row(K)), dtype=np.uint64).astype(np.uint32)
+        pw = pack_canonical_int4(q, np.zeros((N, K // 128), np.uint16), z)
+    x = bf16_dev(gen.x_bf16(17, K))
+    for variant, split in _all_cases(17, K):
+        y = y_host(wq.wq_linear_forced(x, pw, variant, split))
+        assert np.all(y == 0), (variant, split)
+
+
+def test_power_of_two_scaling_is_exact(weight, ws):
+    bits, K, N, pw, canon = weight
+    x = gen.x_bf16(9, K)
+    xd = bf16_dev(x)
+    x2 = bf16_dev((x.astype(np.uint32) + (1 << 7)).astype(np.uint16))  # 2x exactly (no zeros in x)
+    assert np.all((x & 0x7F80) != 0)
+    for variant, split in _cases(9, K):
+        a = y_host(wq.wq_linear_forced(xd, pw, variant, split))
+        b = y_host(wq.wq_linear_forced(x2, pw, variant, split))
+        assert np.array_equal(2 * a, b), (variant, split)
+
+
+# ---------------------------------------------------------------------------
+# boundary behaviour: canaries, argument errors, graphs, tuner
+# ---------------------------------------------------------------------------
+
+def test_output_canaries_untouched(weight, ws):
+    bits, K, N, pw, canon = weight
+    for M in (1, 17, 100):
+        x = gen.x_bf16(M, K)
+        pad = 4096
+        buf = torch.full((M * N + 2 * pad,), -1234, dtype=torch.int16, device=dev())
+        y = buf[pad:pad + M * N].view(torch.bfloat16).view(M, N)
+        for variant, split in _cases(M, K):
+            wq.wq_linear_forced(bf16_dev(x), pw, variant, split, y=y)
+            torch.cuda.synchronize()
+            assert int((buf[:pad] != -1234).sum()) == 0 and int((buf[-pad:] != -1234).sum()) == 0, (variant, split)
+            assert_parity(y_host(y), oracle_linear(x, canon, bits), f"canary M={M} {variant}/{split}")
+
+
+def test_argument_errors(weight, ws):
+    bits, K, N, pw, canon = weight
+    x = bf16_dev(gen.x_bf16(4, K))
+    y = torch.empty((4, N), dtype=torch.bfloat16, device=dev())
+    assert wq.wq_linear_status(x, pw, y, GEMV, 3) == -11          # split not 1/2/4/8
+    assert wq.wq_linear_status(x, pw, y, GEMM, 33) == -11         # split above 32
+    assert wq.wq_linear_status(x, pw, y, 7, 1) == -11             # unknown variant
+    xb = bf16_dev(gen.x_bf16(40, K))
+    yb = torch.empty((40, N), dtype=torch.bfloat16, device=dev())
+    assert wq.wq_linear_status(xb, pw, yb, GEMV, 1) == -11        # GEMV takes M <= 32
+    # misaligned output pointer
+    raw = torch.empty(4 * N + 8, dtype=torch.bfloat16, device=dev())
+    assert wq.wq_linear_status(x, pw, raw[1:1 + 4 * N].view(4, N), GEMV, 1) == -3
+    # split > 1 without a workspace
+    wq.wq_set_workspace(None)
+    try:
+        assert wq.wq_linear_status(x, pw, y, GEMM, 4) == -6
+        assert wq.wq_linear_status(x, pw, y, GEMM, 1) == 0
+    finally:
+        wq.wq_set_workspace(ws)
+    small = torch.zeros(512, dtype=torch.uint8, device=dev())
+    with pytest.raises(wq.WQError):
+        wq.wq_linear_ex(x, pw, GEMM, 4, small)
+    torch.cuda.synchronize()
+    assert wq.wq_device_error() == 0
+
+
+def test_explicit_workspace_on_two_streams(weight):
+    bits, K, N, pw, canon = weight
+    x = gen.x_bf16(48, K)
+    xd = bf16_dev(x)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    w1, w2 = workspace(48, N, 8), workspace(48, N, 8)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s1):
+        y1 = wq.wq_linear_ex(xd, pw, GEMM, 8, w1, stream=s1)
+    with torch.cuda.stream(s2):
+        y2 = wq.wq_linear_ex(xd, pw, GEMM, 4, w2, stream=s2)
+    torch.cuda.synchronize()
+    ref = oracle_linear(x, canon, bits)
+    assert_parity(y_host(y1), ref, "stream 1")
+    assert_parity(y_host(y2), ref, "stream 2")
+
+
+def test_cuda_graph_replay(weight, ws):
+    bits, K, N, pw, canon = weight
+    for M, variant, split in [(1, GEMV, 4), (16, GEMM, 4), (128, GEMM, 2)]:
+        x = gen.x_bf16(M, K)
+        xd = bf16_dev(x)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            wq.wq_linear_forced(xd, pw, variant, split, y=y, stream=s)  # warm (attributes, tensor map fn)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            wq.wq_linear_forced(xd, pw, variant, split, y=y)
+        y.zero_()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        assert_parity(y_host(y), oracle_linear(x, canon, bits), f"graph M={M}")
+
+
+def test_tuner_and_table_roundtrip(weight, ws, tmp_path):
+    bits, K, N, pw, canon = weight
+    wq.wq_clear_tuning()
+    M = 16
+    x = gen.x_bf16(M, K)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
+    v, s = wq.wq_tune(bf16_dev(x), pw, y, warmup=1, iters=3)
+    assert (v, s) in _cases(M, K)
+    assert_parity(y_host(wq.wq_linear(bf16_dev(x), pw)), oracle_linear(x, canon, bits), "tuned")
+    path = str(tmp_path / "table.txt")
+    wq.wq_save_tuning(path)
+    wq.wq_clear_tuning()
+    assert wq.wq_load_tuning(path) == 0
+    assert wq.wq_get_choice(M, K, N, bits, 0 if bits == 8 else 128) == (v, s)
+    wq.wq_set_choice(M, K, N, bits, 0 if bits == 8 else 128, GEMV, 8)
+    assert wq.wq_get_choice(M, K, N, bits, 0 if bits == 8 else 128) == (GEMV, 8)
+    wq.wq_clear_tuning()

@@ -1,0 +1,90 @@
+"""Shared helpers of the GPU tests: moving seeded inputs to the device,
+building packed weights through the library, and the parity check.
+
+The expected values always come from the CPU oracle (``oracle``) on inputs
+from ``wq_inputs``; nothing expected is ever read back from the CUDA path.
+"""
+import numpy as np
+import torch
+
+import oracle
+import weight_only_quantized_02_b200 as wq
+
+# The layer's parity bar: |y_gpu - y_ref| <= 1e-2 * max(|y_ref|, 1) elementwise,
+# y_ref the fp64 oracle, y_gpu the bf16 output (fp32 accumulation).
+REL_TOL = 1e-2
+
+
+def dev():
+    return torch.device("cuda:0")
+
+
+def bf16_dev(x_bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).view(torch.bfloat16).to(dev())
+
+
+def to_dev(a: np.ndarray) -> torch.Tensor:
+    a = np.ascontiguousarray(a)
+    view = {np.dtype(np.uint16): np.int16, np.dtype(np.uint32): np.int32, np.dtype(np.uint8): np.uint8}
+    if a.dtype in view:
+        a = a.view(view[a.dtype])
+    return torch.from_numpy(a).to(dev())
+
+
+def y_host(y: torch.Tensor) -> np.ndarray:
+    return y.float().cpu().numpy().astype(np.float64)
+
+
+def bits_u16(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint16)
+
+
+def bits_u32(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint32)
+
+
+def assert_parity(y_gpu: np.ndarray, y_ref: np.ndarray, what: str = "") -> float:
+    assert y_gpu.shape == y_ref.shape, (y_gpu.shape, y_ref.shape)
+    err = np.abs(y_gpu - y_ref)
+    bound = REL_TOL * np.maximum(np.abs(y_ref), 1.0)
+    bad = err > bound
+    if bad.any():
+        i = np.argwhere(bad)[0]
+        raise AssertionError(f"{what}: {bad.sum()} elements out of tolerance; first at {tuple(i)}: "
+                             f"gpu {y_gpu[tuple(i)]} ref {y_ref[tuple(i)]}")
+    return float(np.sqrt(np.mean((y_gpu - y_ref) ** 2) / max(np.mean(y_ref ** 2), 1e-300)))
+
+
+def pack_canonical_int8(q: np.ndarray, s: np.ndarray) -> wq.PackedWeight:
+    return wq.wq_pack_int8(to_dev(q), to_dev(s))
+
+
+def pack_canonical_int4(q: np.ndarray, s: np.ndarray, z: np.ndarray) -> wq.PackedWeight:
+    return wq.wq_pack_int4(to_dev(q), to_dev(s), to_dev(z))
+
+
+def quantize_and_pack(W: np.ndarray, bits: int):
+    """fp32 W [N][K] -> device quantizer -> packer.  Returns the packed weight
+    and the device's canonical codes (host copies) for the bit-exact checks."""
+    Wd = torch.from_numpy(np.ascontiguousarray(W)).to(dev())
+    if bits == 8:
+        q, s = wq.wq_quantize_int8(Wd)
+        pw = wq.wq_pack_int8(q, s)
+        canon = (q.cpu().numpy(), bits_u16(s))
+    else:
+        q, s, z = wq.wq_quantize_int4(Wd)
+        pw = wq.wq_pack_int4(q, s, z)
+        canon = (bits_u32(q), bits_u16(s), bits_u32(z))
+    del Wd
+    return pw, canon
+
+
+def oracle_linear(x_bits: np.ndarray, canon, bits: int, rows=None) -> np.ndarray:
+    if bits == 8:
+        return oracle.linear_int8(x_bits, canon[0], canon[1], rows=rows)
+    return oracle.linear_int4(x_bits, canon[0], canon[1], canon[2], 128, rows=rows)
+
+
+def workspace(M: int, N: int, max_split: int = 32) -> torch.Tensor:
+    nbytes = wq.wq_workspace_bytes(M, N, max_split)
+    return torch.zeros(nbytes, dtype=torch.uint8, device=dev())

@@ -1,0 +1,593 @@
+// wq_api.cu -- the C ABI (include/wq.h): argument checks, the dispatcher
+// table and tuner, the split-K workspace registry and the debug views.
+#include <algorithm>
+#include <cerrno>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "wq.h"
+#include "wq_internal.h"
+#include "wq_layout.h"
+
+using namespace wq;
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Device facts (cached per device)
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+    bool ok = false;
+    int sm_count = 0, major = 0, minor = 0;
+    std::string name;
+};
+
+std::mutex g_mu;
+std::map<int, DeviceInfo> g_dev;
+std::map<int, std::pair<void *, size_t>> g_ws; // registered workspace per device
+
+int current_device_info(DeviceInfo *out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return WQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_dev.find(dev);
+    if (it == g_dev.end()) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess)
+            return WQ_ERR_CUDA;
+        DeviceInfo d;
+        d.ok = true;
+        d.sm_count = prop.multiProcessorCount;
+        d.major = prop.major;
+        d.minor = prop.minor;
+        d.name = prop.name;
+        it = g_dev.emplace(dev, d).first;
+    }
+    *out = it->second;
+    return WQ_OK;
+}
+
+std::string device_key(const DeviceInfo &d)
+{
+    std::string n = d.name;
+    std::replace(n.begin(), n.end(), '|', '_');
+    return n + "|" + std::to_string(d.sm_count);
+}
+
+// ---------------------------------------------------------------------------
+// Dispatcher table
+// ---------------------------------------------------------------------------
+using Key = std::tuple<std::string, int, int, int, int, int>; // device, M, K, N, bits, group
+struct Choice {
+    int variant, split;
+    float us;
+};
+std::map<Key, Choice> g_table;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int bits_of_group(int group, int *bits)
+{
+    if (group == 0) {
+        *bits = 8;
+        return WQ_OK;
+    }
+    if (group == 128) {
+        *bits = 4;
+        return WQ_OK;
+    }
+    return WQ_ERR_GROUP;
+}
+
+int check_weight_shape(int bits, int K, int N, int group)
+{
+    if (bits == 8 && group != 0)
+        return WQ_ERR_GROUP;
+    if (bits == 4 && group != 128)
+        return WQ_ERR_GROUP;
+    if (bits != 4 && bits != 8)
+        return WQ_ERR_GROUP;
+    if (K <= 0 || N <= 0 || N % 16 != 0)
+        return WQ_ERR_SHAPE;
+    if (bits == 8 && K % 32 != 0)
+        return WQ_ERR_SHAPE;
+    if (bits == 4 && K % 128 != 0)
+        return WQ_ERR_SHAPE;
+    if ((long long)K * N > (1LL << 40))
+        return WQ_ERR_SHAPE;
+    return WQ_OK;
+}
+
+int max_gemm_split(int K) { return std::min(32, (K + kBlockK - 1) / kBlockK); }
+
+bool choice_valid(int variant, int split, int M, int K)
+{
+    if (variant == WQ_VARIANT_GEMV)
+        return M <= 32 && (split == 1 || split == 2 || split == 4 || split == 8);
+    if (variant == WQ_VARIANT_GEMM)
+        return M <= 128 && split >= 1 && split <= max_gemm_split(K);
+    return false;
+}
+
+// The pages' untuned rule: fewer than 8 tokens -> GEMV, otherwise the GEMM
+// with split_k = 8 (Mit han lab Llm awq Kernel Selection Thresholds, The
+// Insight).  The GEMV's K-slice count keeps about 32 warps per SM busy.
+Choice default_choice(int M, int K, int N, int sm_count)
+{
+    if (M < 8) {
+        const long long rbs = N / 16;
+        int ks = 1;
+        while (ks < 8 && rbs * ks < (long long)sm_count * 32)
+            ks *= 2;
+        if (K / 128 < ks)
+            ks = std::max(1, K / 128);
+        while (ks > 1 && (ks & (ks - 1)))
+            --ks;
+        return {WQ_VARIANT_GEMV, ks, 0.f};
+    }
+    return {WQ_VARIANT_GEMM, std::min(8, max_gemm_split(K)), 0.f};
+}
+
+int lookup_choice(const DeviceInfo &d, int M, int K, int N, int bits, int group, Choice *c)
+{
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_table.find(Key{device_key(d), M, K, N, bits, group});
+        if (it != g_table.end()) {
+            *c = it->second;
+            return WQ_OK;
+        }
+    }
+    *c = default_choice(M, K, N, d.sm_count);
+    return WQ_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
+
+int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros, int group,
+                int N, uint16_t *y, int variant, int split, void *ws, size_t ws_bytes_given, cudaStream_t stream)
+{
+    int bits = 0;
+    int st = bits_of_group(group, &bits);
+    if (st != WQ_OK)
+        return st;
+    if (!x || !Wq || !scales || !y || (bits == 4 && !zeros))
+        return WQ_ERR_NULL;
+    if ((st = check_weight_shape(bits, K, N, group)) != WQ_OK)
+        return st;
+    if (M < 1 || M > 128)
+        return WQ_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(Wq) || !aligned16(scales) || (zeros && !aligned16(zeros)))
+        return WQ_ERR_ALIGN;
+    DeviceInfo d;
+    if ((st = current_device_info(&d)) != WQ_OK)
+        return st;
+    if (d.major != 10)
+        return WQ_ERR_ARCH;
+
+    Choice c;
+    lookup_choice(d, M, K, N, bits, group, &c);
+    if (variant != WQ_VARIANT_AUTO) {
+        c.variant = variant;
+        if (split <= 0)
+            c.split = default_choice(variant == WQ_VARIANT_GEMV ? 1 : 8, K, N, d.sm_count).split;
+    }
+    if (split > 0)
+        c.split = split;
+    if (variant == WQ_VARIANT_AUTO && !choice_valid(c.variant, c.split, M, K))
+        c = default_choice(M, K, N, d.sm_count);
+    if (!choice_valid(c.variant, c.split, M, K))
+        return WQ_ERR_VARIANT;
+
+    LinearArgs a{x, M, K, N, Wq, scales, zeros, bits, group, y};
+    if (c.variant == WQ_VARIANT_GEMV)
+        return cuda_status(launch_gemv(a, c.split, d.sm_count, stream));
+
+    void *w = nullptr;
+    if (c.split > 1) {
+        size_t have = 0;
+        if (ws) {
+            w = ws;
+            have = ws_bytes_given;
+        } else {
+            int dev = 0;
+            cudaGetDevice(&dev);
+            std::lock_guard<std::mutex> lk(g_mu);
+            auto it = g_ws.find(dev);
+            if (it != g_ws.end()) {
+                w = it->second.first;
+                have = it->second.second;
+            }
+        }
+        if (!w || have < ws_bytes(M, N, c.split))
+            return WQ_ERR_WORKSPACE;
+        if (!aligned16(w))
+            return WQ_ERR_ALIGN;
+    }
+    return cuda_status(launch_gemm(a, c.split, w, d.sm_count, stream));
+}
+
+} // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char *wq_strerror(int status)
+{
+    switch (status) {
+    case WQ_OK: return "ok";
+    case WQ_ERR_NULL: return "a required pointer is NULL";
+    case WQ_ERR_SHAPE: return "M, K or N outside the supported shape rules";
+    case WQ_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case WQ_ERR_GROUP: return "unsupported bits/group combination (INT8: group 0, INT4: group 128)";
+    case WQ_ERR_HEADER: return "packed-weight trailer does not match the arguments";
+    case WQ_ERR_WORKSPACE: return "split-K workspace missing or too small";
+    case WQ_ERR_CUDA: return "CUDA runtime error";
+    case WQ_ERR_TUNING: return "tuning file unreadable or malformed";
+    case WQ_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    case WQ_ERR_ARCH: return "device is not sm_100 (B200 class)";
+    case WQ_ERR_VARIANT: return "forced variant/split not valid for this shape";
+    default: return "unknown status";
+    }
+}
+
+int wq_version(void) { return 100; }
+
+int wq_packed_bytes(int bits, int K, int N, int group, size_t *wq_bytes, size_t *scale_bytes, size_t *zero_bytes)
+{
+    const int st = check_weight_shape(bits, K, N, group);
+    if (st != WQ_OK)
+        return st;
+    const Shape sh{bits, K, N, group};
+    if (wq_bytes)
+        *wq_bytes = sh.wq_bytes();
+    if (scale_bytes)
+        *scale_bytes = sh.scale_bytes();
+    if (zero_bytes)
+        *zero_bytes = sh.zero_bytes();
+    return WQ_OK;
+}
+
+int wq_quantize_int8(const float *W, int K, int N, int8_t *q_out, uint16_t *s_out, cudaStream_t stream)
+{
+    if (!W || !q_out || !s_out)
+        return WQ_ERR_NULL;
+    if (K <= 0 || N <= 0)
+        return WQ_ERR_SHAPE;
+    return cuda_status(launch_quantize_int8(W, K, N, q_out, s_out, stream));
+}
+
+int wq_quantize_int4(const float *W, int K, int N, int group, uint32_t *q_out, uint16_t *s_out, uint32_t *z_out,
+                     cudaStream_t stream)
+{
+    if (!W || !q_out || !s_out || !z_out)
+        return WQ_ERR_NULL;
+    if (group != 128)
+        return WQ_ERR_GROUP;
+    if (K <= 0 || N <= 0 || K % 128 != 0)
+        return WQ_ERR_SHAPE;
+    return cuda_status(launch_quantize_int4(W, K, N, q_out, s_out, z_out, stream));
+}
+
+int wq_pack_int8(const int8_t *q, const uint16_t *scales, int K, int N, void *wq_out, void *scales_out,
+                 cudaStream_t stream)
+{
+    if (!q || !scales || !wq_out || !scales_out)
+        return WQ_ERR_NULL;
+    const int st = check_weight_shape(8, K, N, 0);
+    if (st != WQ_OK)
+        return st;
+    if (!aligned16(q) || !aligned16(wq_out) || !aligned16(scales_out))
+        return WQ_ERR_ALIGN;
+    return cuda_status(launch_pack_int8(q, scales, K, N, wq_out, scales_out, stream));
+}
+
+int wq_pack_int4(const uint32_t *q, const uint16_t *scales, const uint32_t *zeros, int K, int N, int group,
+                 void *wq_out, void *scales_out, void *zeros_out, cudaStream_t stream)
+{
+    if (!q || !scales || !zeros || !wq_out || !scales_out || !zeros_out)
+        return WQ_ERR_NULL;
+    const int st = check_weight_shape(4, K, N, group);
+    if (st != WQ_OK)
+        return st;
+    if (!aligned16(wq_out) || !aligned16(scales_out) || !aligned16(zeros_out))
+        return WQ_ERR_ALIGN;
+    return cuda_status(launch_pack_int4(q, scales, zeros, K, N, wq_out, scales_out, zeros_out, stream));
+}
+
+int wq_check_packed(const void *Wq, int bits, int K, int N, int group, cudaStream_t stream)
+{
+    if (!Wq)
+        return WQ_ERR_NULL;
+    int st = check_weight_shape(bits, K, N, group);
+    if (st != WQ_OK)
+        return st;
+    const Shape sh{bits, K, N, group};
+    Trailer t;
+    if (cudaMemcpyAsync(&t, (const uint8_t *)Wq + sh.weight_bytes(), sizeof t, cudaMemcpyDeviceToHost, stream) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return WQ_ERR_CUDA;
+    const size_t wb = sh.weight_bytes();
+    if (t.magic != kMagic || t.version != kLayoutVersion || t.bits != (uint32_t)bits || t.K != (uint32_t)K ||
+        t.N != (uint32_t)N || t.group != (uint32_t)group || t.layout_bytes_lo != (uint32_t)(wb & 0xffffffffu) ||
+        t.layout_bytes_hi != (uint32_t)(wb >> 32))
+        return WQ_ERR_HEADER;
+    return WQ_OK;
+}
+
+int wq_linear(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros, int group,
+              int N, uint16_t *y, cudaStream_t stream)
+{
+    return linear_impl(x, M, K, Wq, scales, zeros, group, N, y, WQ_VARIANT_AUTO, 0, nullptr, 0, stream);
+}
+
+int wq_linear_forced(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros,
+                     int group, int N, uint16_t *y, int variant, int split, cudaStream_t stream)
+{
+    return linear_impl(x, M, K, Wq, scales, zeros, group, N, y, variant, split, nullptr, 0, stream);
+}
+
+int wq_linear_ex(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros, int group,
+                 int N, uint16_t *y, int variant, int split, void *ws, size_t ws_bytes_given, cudaStream_t stream)
+{
+    return linear_impl(x, M, K, Wq, scales, zeros, group, N, y, variant, split, ws, ws_bytes_given, stream);
+}
+
+size_t wq_workspace_bytes(int M, int N, int max_split)
+{
+    if (M < 1 || N < 1 || max_split < 1)
+        return 0;
+    return ws_bytes(M, N, max_split);
+}
+
+int wq_set_workspace(void *ws, size_t bytes)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return WQ_ERR_CUDA;
+    if (ws && !aligned16(ws))
+        return WQ_ERR_ALIGN;
+    if (ws && bytes > 0) {
+        if (cudaMemset(ws, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+            return WQ_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!ws)
+        g_ws.erase(dev);
+    else
+        g_ws[dev] = {ws, bytes};
+    return WQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Tuner
+// ---------------------------------------------------------------------------
+int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros, int group,
+            int N, uint16_t *y, int warmup, int iters, cudaStream_t stream)
+{
+    int bits = 0;
+    int st = bits_of_group(group, &bits);
+    if (st != WQ_OK)
+        return st;
+    DeviceInfo d;
+    if ((st = current_device_info(&d)) != WQ_OK)
+        return st;
+    if (warmup < 0 || iters < 1)
+        return WQ_ERR_SHAPE;
+    std::vector<std::pair<int, int>> cands;
+    if (M <= 32)
+        for (int ks : {1, 2, 4, 8})
+            cands.push_back({WQ_VARIANT_GEMV, ks});
+    for (int s : {1, 2, 4, 8, 16, 32})
+        if (s <= max_gemm_split(K))
+            cands.push_back({WQ_VARIANT_GEMM, s});
+
+    // Flush buffer larger than L2, so every timed call streams its weights
+    // from HBM (the weights of a decode step are not L2-resident).
+    int l2 = 0;
+    int tdev = 0;
+    cudaGetDevice(&tdev);
+    cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, tdev);
+    const size_t flush_bytes = std::max<size_t>((size_t)l2 * 2, 64u << 20);
+    void *flush = nullptr;
+    if (cudaMalloc(&flush, flush_bytes) != cudaSuccess)
+        return WQ_ERR_CUDA;
+    cudaEvent_t e0, e1;
+    cudaEventCreate(&e0);
+    cudaEventCreate(&e1);
+    Choice best{-1, 0, 0.f};
+    int result = WQ_OK;
+    for (auto [v, s] : cands) {
+        int rc = WQ_OK;
+        for (int i = 0; i < warmup && rc == WQ_OK; ++i)
+            rc = linear_impl(x, M, K, Wq, scales, zeros, group, N, y, v, s, nullptr, 0, stream);
+        if (rc != WQ_OK)
+            continue; // e.g. no workspace large enough for this split
+        std::vector<float> t;
+        for (int i = 0; i < iters && rc == WQ_OK; ++i) {
+            cudaMemsetAsync(flush, i & 0xff, flush_bytes, stream);
+            cudaEventRecord(e0, stream);
+            rc = linear_impl(x, M, K, Wq, scales, zeros, group, N, y, v, s, nullptr, 0, stream);
+            cudaEventRecord(e1, stream);
+            if (cudaEventSynchronize(e1) != cudaSuccess) {
+                rc = WQ_ERR_CUDA;
+                break;
+            }
+            float ms = 0.f;
+            cudaEventElapsedTime(&ms, e0, e1);
+            t.push_back(ms * 1000.f);
+        }
+        if (rc != WQ_OK) {
+            if (rc == WQ_ERR_CUDA)
+                result = rc;
+            continue;
+        }
+        std::sort(t.begin(), t.end());
+        const float med = t[t.size() / 2];
+        // ">=": on an exact tie the later (larger) split wins, as in the page's loop
+        if (best.variant < 0 || best.us >= med)
+            best = {v, s, med};
+    }
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    cudaFree(flush);
+    if (result != WQ_OK)
+        return result;
+    if (best.variant < 0)
+        return WQ_ERR_VARIANT;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_table[Key{device_key(d), M, K, N, bits, group}] = best;
+    return WQ_OK;
+}
+
+int wq_get_choice(int M, int K, int N, int bits, int group, int *variant, int *split)
+{
+    if (!variant || !split)
+        return WQ_ERR_NULL;
+    DeviceInfo d;
+    int st = current_device_info(&d);
+    if (st != WQ_OK)
+        return st;
+    Choice c;
+    lookup_choice(d, M, K, N, bits, group, &c);
+    *variant = c.variant;
+    *split = c.split;
+    return WQ_OK;
+}
+
+int wq_set_choice(int M, int K, int N, int bits, int group, int variant, int split)
+{
+    DeviceInfo d;
+    int st = current_device_info(&d);
+    if (st != WQ_OK)
+        return st;
+    if (!choice_valid(variant, split, M, K))
+        return WQ_ERR_VARIANT;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_table[Key{device_key(d), M, K, N, bits, group}] = Choice{variant, split, 0.f};
+    return WQ_OK;
+}
+
+int wq_clear_tuning(void)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_table.clear();
+    return WQ_OK;
+}
+
+int wq_save_tuning(const char *path)
+{
+    if (!path)
+        return WQ_ERR_NULL;
+    FILE *f = fopen(path, "w");
+    if (!f)
+        return WQ_ERR_TUNING;
+    std::lock_guard<std::mutex> lk(g_mu);
+    fprintf(f, "# wq tuning v1: device|sms M K N bits group variant split median_us\n");
+    for (auto &kv : g_table) {
+        const auto &k = kv.first;
+        fprintf(f, "%s %d %d %d %d %d %d %d %.3f\n", std::get<0>(k).c_str(), std::get<1>(k), std::get<2>(k),
+                std::get<3>(k), std::get<4>(k), std::get<5>(k), kv.second.variant, kv.second.split, kv.second.us);
+    }
+    const bool bad = ferror(f) != 0;
+    fclose(f);
+    return bad ? WQ_ERR_TUNING : WQ_OK;
+}
+
+// Host-only parser (no CUDA calls), so it can be tested without a GPU.
+int wq_load_tuning(const char *path)
+{
+    if (!path)
+        return WQ_ERR_NULL;
+    FILE *f = fopen(path, "r");
+    if (!f)
+        return WQ_ERR_TUNING;
+    std::map<Key, Choice> loaded;
+    char line[1024];
+    bool bad = false;
+    while (fgets(line, sizeof line, f)) {
+        const size_t len = strlen(line);
+        if (len == 0 || line[0] == '#' || line[0] == '\n')
+            continue;
+        if (line[len - 1] != '\n' && !feof(f)) {
+            bad = true;
+            break;
+        }
+        // device key is everything up to the first '|' plus the SM count token
+        char *bar = strchr(line, '|');
+        if (!bar) {
+            bad = true;
+            break;
+        }
+        char *rest = strchr(bar, ' ');
+        if (!rest) {
+            bad = true;
+            break;
+        }
+        std::string dkey(line, rest - line);
+        int M, K, N, bits, group, variant, split;
+        float us;
+        char tail;
+        const int n = sscanf(rest, " %d %d %d %d %d %d %d %f %c", &M, &K, &N, &bits, &group, &variant, &split, &us,
+                             &tail);
+        if (n != 8 || check_weight_shape(bits, K, N, group) != WQ_OK || M < 1 || M > 128 ||
+            !choice_valid(variant, split, M, K)) {
+            bad = true;
+            break;
+        }
+        loaded[Key{dkey, M, K, N, bits, group}] = Choice{variant, split, us};
+    }
+    fclose(f);
+    if (bad)
+        return WQ_ERR_TUNING;
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (auto &kv : loaded)
+        g_table[kv.first] = kv.second;
+    return WQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Debug views
+// ---------------------------------------------------------------------------
+int wq_unpack_debug(const void *Wq, const void *zeros, int bits, int K, int N, int group, int8_t *q_out,
+                    int8_t *z_out, cudaStream_t stream)
+{
+    if (!Wq || !q_out || (bits == 4 && (!zeros || !z_out)))
+        return WQ_ERR_NULL;
+    const int st = check_weight_shape(bits, K, N, group);
+    if (st != WQ_OK)
+        return st;
+    return cuda_status(launch_unpack_debug(Wq, zeros, Shape{bits, K, N, group}, q_out, z_out, stream));
+}
+
+int wq_dequant_debug(const void *Wq, const void *scales, const void *zeros, int bits, int K, int N, int group,
+                     float *w_out, cudaStream_t stream)
+{
+    if (!Wq || !scales || !w_out || (bits == 4 && !zeros))
+        return WQ_ERR_NULL;
+    const int st = check_weight_shape(bits, K, N, group);
+    if (st != WQ_OK)
+        return st;
+    return cuda_status(launch_dequant_debug(Wq, scales, zeros, Shape{bits, K, N, group}, w_out, stream));
+}
+
+int wq_device_error(cudaStream_t stream)
+{
+    int code = 0;
+    if (read_device_error(&code, stream) != cudaSuccess)
+        return WQ_ERR_CUDA;
+    return code == 0 ? WQ_OK : WQ_ERR_TIMEOUT;
+}
+
+} // extern "C"

@@ -1,0 +1,438 @@
+// wq_gemm.cu -- small-M (8..128 tokens) split-K GEMM on tcgen05 tensor cores.
+//
+// y^T = dequant(W) . x^T: the weight rows are the MMA's M side (128 rows per
+// CTA), the tokens its N side (NT = 16/32/64/128), so decode-sized batches
+// still fill a 128-row tensor-core tile.  One CTA owns a 128-row panel and a
+// K range (split-K over 128-k blocks; the split-factor grid and its
+// trade-off are those of the split_k auto-tune in Mit han lab Llm awq Kernel
+// Selection Thresholds, The Insight).
+//
+// Warp roles (192 threads):
+//   warp 0     TMA producer: per 128-k block, the x tile (2-D tensor map,
+//              128-byte swizzle) and the packed weight block (+ INT4 scales
+//              and zeros) as 1-D bulk copies into a STAGES-deep ring.
+//   warp 1     allocates tensor memory; one thread issues tcgen05.mma with
+//              the dequantized weights as the A operand *from tensor memory*
+//              and x as the B operand from shared memory; fp32 accumulators
+//              stay in tensor memory.
+//   warps 2-5  dequantize the block (INT4: bf16(s*(q - z)); INT8: exact q,
+//              scale applied in the epilogue) and write it to tensor memory
+//              with tcgen05.st 16x256b -- the packed tile is already that
+//              store's register layout -- then run the epilogue.
+// Epilogue: split == 1 stores bf16 y.  split > 1 stores fp32 partials; the
+// last CTA of a panel to arrive (atomic ticket, no waiting) sums all partials
+// in split order 0..S-1, so each (variant, split) is run-to-run deterministic,
+// and resets the ticket to zero.
+//
+// Every mbarrier wait is bounded (2 s); a wait that gives up records
+// kErrTimeout in the device error word and the CTA winds down.
+#include <cstdint>
+#include <cstdio>
+
+#include <cudaTypedefs.h>
+
+#include "wq_device.cuh"
+#include "wq_internal.h"
+
+namespace wq {
+
+static __device__ int g_gemm_error = 0;
+
+struct GemmParams {
+    int M, K, N, KB, S;
+    const uint8_t *wq;
+    const uint16_t *scales;
+    const uint8_t *zeros;
+    uint16_t *y;
+    float *part;   // [S][M][N] fp32 partials (S > 1)
+    uint32_t *cnt; // [panels] tickets (S > 1)
+};
+
+template <int BITS>
+struct GemmBits {
+    static constexpr int kWBytes = BITS == 4 ? 8192 : 16384; // packed block per stage
+    static constexpr int kSZBytes = BITS == 4 ? 512 : 0;     // scales (256) + zeros (64), padded
+    static constexpr int kSZTx = BITS == 4 ? 320 : 0;
+    static constexpr int kTilesPerRb = BITS == 4 ? 2 : 4;
+};
+
+template <int NT>
+struct GemmTile {
+    static constexpr int kStages = NT == 128 ? 4 : 3;
+    static constexpr int kTmemCols = NT == 128 ? 512 : 256;
+    static constexpr int kA0 = NT < 64 ? 64 : NT; // first tensor-memory column of the A ring
+    static constexpr int kMinBlocks = NT == 128 ? 1 : 2;
+    static_assert(kA0 + 64 * kStages <= kTmemCols, "tensor memory budget");
+};
+
+template <int BITS, int NT>
+constexpr size_t gemm_smem_bytes()
+{
+    return 1024 + (size_t)GemmTile<NT>::kStages * (NT * 256 + GemmBits<BITS>::kWBytes + GemmBits<BITS>::kSZBytes) +
+           (4 * GemmTile<NT>::kStages + 1) * 8 + 16;
+}
+
+// Dequantize one INT4 tile (16 rows x 64 k) into the 16 registers of a
+// tcgen05.st 16x256b.x4 store: bf16(s * (q - z)), natural k order.
+__device__ __forceinline__ void int4_tile_regs(const uint4 &w, uint32_t zlo, uint32_t zhi, uint32_t slo,
+                                               uint32_t shi, uint32_t (&r)[16])
+{
+    auto d = [](uint32_t word, int i, uint32_t zz, uint32_t ss) {
+        return bf16x2_mul(bf16x2_sub(nib_pair_bf16(word >> (4 * i)), zz), ss);
+    };
+    r[0] = d(w.x, 0, zlo, slo);
+    r[1] = d(w.x, 1, zlo, slo);
+    r[2] = d(w.y, 0, zhi, shi);
+    r[3] = d(w.y, 1, zhi, shi);
+    r[4] = d(w.x, 2, zlo, slo);
+    r[5] = d(w.x, 3, zlo, slo);
+    r[6] = d(w.y, 2, zhi, shi);
+    r[7] = d(w.y, 3, zhi, shi);
+    r[8] = d(w.z, 0, zlo, slo);
+    r[9] = d(w.z, 1, zlo, slo);
+    r[10] = d(w.w, 0, zhi, shi);
+    r[11] = d(w.w, 1, zhi, shi);
+    r[12] = d(w.z, 2, zlo, slo);
+    r[13] = d(w.z, 3, zlo, slo);
+    r[14] = d(w.w, 2, zhi, shi);
+    r[15] = d(w.w, 3, zhi, shi);
+}
+
+// One INT8 tile (16 rows x 32 k) -> 8 registers of a 16x256b.x2 store: exact q.
+__device__ __forceinline__ void int8_tile_regs(const uint4 &w, uint32_t (&r)[8])
+{
+    const uint32_t ux = w.x ^ 0x80808080u, uy = w.y ^ 0x80808080u;
+    const uint32_t uz = w.z ^ 0x80808080u, uw = w.w ^ 0x80808080u;
+    r[0] = s8pair_bf16(ux, 0);
+    r[1] = s8pair_bf16(ux, 1);
+    r[2] = s8pair_bf16(uy, 0);
+    r[3] = s8pair_bf16(uy, 1);
+    r[4] = s8pair_bf16(uz, 0);
+    r[5] = s8pair_bf16(uz, 1);
+    r[6] = s8pair_bf16(uw, 0);
+    r[7] = s8pair_bf16(uw, 1);
+}
+
+template <int BITS, int NT>
+__global__ void __launch_bounds__(192, GemmTile<NT>::kMinBlocks)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmx, const GemmParams p)
+{
+    constexpr int STAGES = GemmTile<NT>::kStages;
+    constexpr int TCOLS = GemmTile<NT>::kTmemCols;
+    constexpr int A0 = GemmTile<NT>::kA0;
+    constexpr int XB = NT * 256;
+    constexpr int WB = GemmBits<BITS>::kWBytes;
+    constexpr int SZB = GemmBits<BITS>::kSZBytes;
+    constexpr int TPR = GemmBits<BITS>::kTilesPerRb;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sX = smem;
+    uint8_t *sW = sX + STAGES * XB;
+    uint8_t *sSZ = sW + STAGES * WB;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sSZ + STAGES * SZB);
+    uint64_t *full = bars, *ldempty = bars + STAGES, *afull = bars + 2 * STAGES, *aempty = bars + 3 * STAGES;
+    uint64_t *accfull = bars + 4 * STAGES;
+    uint32_t *s_misc = reinterpret_cast<uint32_t *>(bars + 4 * STAGES + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int panel = blockIdx.x, split = blockIdx.y;
+    const int kb0 = (int)((long long)p.KB * split / p.S);
+    const int kb1 = (int)((long long)p.KB * (split + 1) / p.S);
+    const int nk = kb1 - kb0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&ldempty[s], 1 + 4);
+            mbar_init(&afull[s], 4);
+            mbar_init(&aempty[s], 1);
+        }
+        mbar_init(accfull, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&s_misc[0], TCOLS);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0)
+        prefetch_tensormap(&tmx);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_misc[0];
+    bool ok = true;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
+            for (int i = 0; i < nk; ++i) {
+                const int st = i % STAGES, use = i / STAGES;
+                if (use > 0 && !mbar_wait(&ldempty[st], (use - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const int kb = kb0 + i;
+                const size_t blk = (size_t)panel * p.KB + kb;
+                mbar_arrive_expect_tx(&full[st], XB + WB + GemmBits<BITS>::kSZTx);
+                tma_load_2d(sX + st * XB, &tmx, kb * kBlockK, 0, &full[st], pol_x);
+                tma_load_2d(sX + st * XB + NT * 128, &tmx, kb * kBlockK + 64, 0, &full[st], pol_x);
+                bulk_g2s(sW + st * WB, p.wq + blk * WB, WB, &full[st], pol_w);
+                if constexpr (BITS == 4) {
+                    bulk_g2s(sSZ + st * SZB, p.scales + blk * kPanelRows, 256, &full[st], pol_w);
+                    bulk_g2s(sSZ + st * SZB + 256, p.zeros + blk * 64, 64, &full[st], pol_w);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16(NT);
+            for (int i = 0; i < nk; ++i) {
+                const int st = i % STAGES, use = i / STAGES;
+                if (!mbar_wait(&afull[st], use & 1) || !mbar_wait(&full[st], use & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t xs = smem_u32(sX + st * XB);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t bdesc = smem_desc_sw128(xs + (kk >> 2) * (NT * 128) + (kk & 3) * 32);
+                    umma_ts(tmem, tmem + A0 + st * 64 + kk * 8, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&aempty[st]);
+                umma_commit(&ldempty[st]);
+            }
+            umma_commit(accfull);
+        }
+    } else {
+        // ---------------- dequant warps ----------------
+        const int quad = warp & 3; // tensor-memory lane quadrant this warp may access
+        const int g = lane >> 2;
+        for (int i = 0; i < nk; ++i) {
+            const int st = i % STAGES, use = i / STAGES;
+            if (!mbar_wait(&full[st], use & 1)) {
+                ok = false;
+                break;
+            }
+            uint4 w[2][TPR];
+            uint32_t zz[2][2], ss[2][2];
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int j = 2 * quad + jj;
+#pragma unroll
+                for (int tt = 0; tt < TPR; ++tt)
+                    w[jj][tt] = *reinterpret_cast<const uint4 *>(sW + st * WB + j * (TPR * kTileBytes) +
+                                                                 tt * kTileBytes + lane * 16);
+                if constexpr (BITS == 4) {
+                    const uint16_t *s16 = reinterpret_cast<const uint16_t *>(sSZ + st * SZB);
+                    const uint8_t *z8 = sSZ + st * SZB + 256;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int row = 16 * j + g + 8 * h;
+                        const uint32_t z = (z8[row >> 1] >> (4 * (row & 1))) & 0xFu;
+                        const uint32_t s = s16[row];
+                        zz[jj][h] = 0x43004300u | z | (z << 16);
+                        ss[jj][h] = s | (s << 16);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&ldempty[st]);
+            if (use > 0 && !mbar_wait(&aempty[st], (use - 1) & 1)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const uint32_t ta = tmem + ((uint32_t)(32 * quad + 16 * jj) << 16) + A0 + st * 64;
+#pragma unroll
+                for (int tt = 0; tt < TPR; ++tt) {
+                    if constexpr (BITS == 4) {
+                        uint32_t r[16];
+                        int4_tile_regs(w[jj][tt], zz[jj][0], zz[jj][1], ss[jj][0], ss[jj][1], r);
+                        tmem_st_16x256b_x4(ta + tt * 32, r);
+                    } else {
+                        uint32_t r[8];
+                        int8_tile_regs(w[jj][tt], r);
+                        tmem_st_16x256b_x2(ta + tt * 16, r);
+                    }
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&afull[st]);
+        }
+
+        // ---------------- epilogue ----------------
+        if (!mbar_wait(accfull, 0))
+            ok = false;
+        tc_fence_after();
+        const int row = 32 * quad + lane;
+        const int n = panel * kPanelRows + row;
+        const bool nvalid = n < p.N;
+        float scale = 1.f;
+        if constexpr (BITS == 8)
+            scale = nvalid ? bf16_bits_to_float(p.scales[n]) : 0.f;
+        const uint32_t tacc = tmem + ((uint32_t)(32 * quad) << 16);
+        if (p.S == 1) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < NT; c0 += 16) {
+                float v[16];
+                tmem_ld_32x32b_x16(tacc + c0, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int m = c0 + e;
+                    if (m < p.M && nvalid)
+                        p.y[(size_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v[e] * scale));
+                }
+            }
+        } else {
+#pragma unroll 1
+            for (int c0 = 0; c0 < NT; c0 += 16) {
+                float v[16];
+                tmem_ld_32x32b_x16(tacc + c0, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int m = c0 + e;
+                    if (m < p.M && nvalid)
+                        p.part[((size_t)split * p.M + m) * p.N + n] = v[e];
+                }
+            }
+            __threadfence();
+            named_barrier_sync(1, 128);
+            if (warp == 2 && lane == 0)
+                s_misc[1] = atomicAdd(&p.cnt[panel], 1u);
+            named_barrier_sync(1, 128);
+            if (s_misc[1] == (uint32_t)(p.S - 1)) {
+                __threadfence();
+                if (nvalid) {
+                    for (int m = 0; m < p.M; ++m) {
+                        float sum = 0.f;
+                        for (int s = 0; s < p.S; ++s)
+                            sum += __ldcg(&p.part[((size_t)s * p.M + m) * p.N + n]);
+                        p.y[(size_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(sum * scale));
+                    }
+                }
+                if (warp == 2 && lane == 0)
+                    atomicExch(&p.cnt[panel], 0u);
+            }
+        }
+    }
+
+    if (!ok)
+        atomicExch(&g_gemm_error, kErrTimeout);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TCOLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+template <int NT>
+static bool make_x_map(CUtensorMap *map, const uint16_t *x, int M, int K)
+{
+    auto fn = get_encode_fn();
+    if (!fn)
+        return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)NT};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(x), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int BITS, int NT>
+static cudaError_t launch_gemm_t(const LinearArgs &a, int S, void *ws, cudaStream_t st)
+{
+    constexpr size_t smem = gemm_smem_bytes<BITS, NT>();
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BITS, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess)
+            return e;
+        attr_set = true;
+    }
+    CUtensorMap map;
+    if (!make_x_map<NT>(&map, a.x, a.M, a.K))
+        return cudaErrorInvalidValue;
+    const Shape sh{a.bits, a.K, a.N, a.group};
+    GemmParams p;
+    p.M = a.M;
+    p.K = a.K;
+    p.N = a.N;
+    p.KB = sh.kblocks();
+    p.S = S;
+    p.wq = (const uint8_t *)a.wq;
+    p.scales = (const uint16_t *)a.scales;
+    p.zeros = (const uint8_t *)a.zeros;
+    p.y = a.y;
+    p.cnt = (uint32_t *)ws;
+    p.part = ws ? (float *)((uint8_t *)ws + ws_counter_bytes(a.N)) : nullptr;
+    dim3 grid(sh.panels(), S);
+    gemm_kernel<BITS, NT><<<grid, 192, smem, st>>>(map, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const LinearArgs &a, int split, void *ws, int sm_count, cudaStream_t st)
+{
+    (void)sm_count;
+    const int nt = a.M <= 16 ? 16 : a.M <= 32 ? 32 : a.M <= 64 ? 64 : 128;
+    if (a.bits == 4) {
+        switch (nt) {
+        case 16: return launch_gemm_t<4, 16>(a, split, ws, st);
+        case 32: return launch_gemm_t<4, 32>(a, split, ws, st);
+        case 64: return launch_gemm_t<4, 64>(a, split, ws, st);
+        default: return launch_gemm_t<4, 128>(a, split, ws, st);
+        }
+    }
+    switch (nt) {
+    case 16: return launch_gemm_t<8, 16>(a, split, ws, st);
+    case 32: return launch_gemm_t<8, 32>(a, split, ws, st);
+    case 64: return launch_gemm_t<8, 64>(a, split, ws, st);
+    default: return launch_gemm_t<8, 128>(a, split, ws, st);
+    }
+}
+
+cudaError_t read_device_error(int *code, cudaStream_t st)
+{
+    int host = 0, zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&host, g_gemm_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess)
+        return e;
+    e = cudaMemcpyToSymbolAsync(g_gemm_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess)
+        return e;
+    e = cudaStreamSynchronize(st);
+    *code = host;
+    return e;
+}
+
+} // namespace wq

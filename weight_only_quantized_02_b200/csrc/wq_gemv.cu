@@ -1,0 +1,302 @@
+// wq_gemv.cu -- decode-regime GEMV (M <= 32) for W8A16 and W4A16.
+//
+// Register-level dequantization with 128-bit weight loads and no shared
+// memory on the weight path (the "BitBLAS-style GEMV" row of the tileInfer
+// README, Features table).  Each warp streams the 512-byte tiles of one
+// 16-row block over a K slice; every lane's 16 bytes are already an
+// m16n8k16 A fragment (see wq_layout.h), so the unpacked integers go straight
+// into mma.sync with the activations as the 8-token B operand and fp32
+// accumulators.  For W4A16 the MMA sees exact (q - z) integers and the bf16
+// group scale is applied in fp32 after each group of 128 k, so the weights
+// are never rounded.  For W8A16 the per-channel scale is applied once in the
+// epilogue.  K slices of one row block are summed across warps through
+// shared memory in a fixed order (deterministic).
+#include <cstdint>
+
+#include "wq_device.cuh"
+#include "wq_internal.h"
+
+namespace wq {
+
+struct GemvParams {
+    const uint16_t *x;
+    int M, K, N;
+    const uint8_t *wq;
+    const uint16_t *scales;
+    const uint8_t *zeros;
+    uint16_t *y;
+    Shape sh;
+    int ks; // K slices per 16-row block (1, 2, 4, 8); the 8 warps of a CTA
+            // cover 8/ks row blocks
+};
+
+constexpr int kGemvWarps = 8;
+
+template <int MT>
+__device__ __forceinline__ void load_x_frag(const GemvParams &p, int g, int k, uint2 (&xf)[MT])
+{
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int m = 8 * mt + g;
+        xf[mt] = (m < p.M) ? ldg_keep(p.x + (size_t)m * p.K + k) : make_uint2(0u, 0u);
+    }
+}
+
+// One INT8 tile (16 rows x 32 k): two MMAs per 8-token tile.
+template <int MT>
+__device__ __forceinline__ void int8_tile(const GemvParams &p, const uint4 &w, int kt_base, int g, int t,
+                                          float (&acc)[MT][4])
+{
+    const uint32_t ux = w.x ^ 0x80808080u, uy = w.y ^ 0x80808080u;
+    const uint32_t uz = w.z ^ 0x80808080u, uw = w.w ^ 0x80808080u;
+    const uint32_t a0 = s8pair_bf16(ux, 0), a1 = s8pair_bf16(uy, 0);
+    const uint32_t a2 = s8pair_bf16(ux, 1), a3 = s8pair_bf16(uy, 1);
+    const uint32_t b0 = s8pair_bf16(uz, 0), b1 = s8pair_bf16(uw, 0);
+    const uint32_t b2 = s8pair_bf16(uz, 1), b3 = s8pair_bf16(uw, 1);
+    uint2 xa[MT], xb[MT];
+    load_x_frag<MT>(p, g, kt_base + 4 * t, xa);
+    load_x_frag<MT>(p, g, kt_base + 16 + 4 * t, xb);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        mma_bf16_16816(acc[mt], a0, a1, a2, a3, xa[mt].x, xa[mt].y);
+        mma_bf16_16816(acc[mt], b0, b1, b2, b3, xb[mt].x, xb[mt].y);
+    }
+}
+
+// One INT4 tile (16 rows x 64 k): four MMAs per 8-token tile on exact
+// (q - z) values.  zlo / zhi are bf16x2 {128+z, 128+z} of rows g and g+8.
+template <int MT>
+__device__ __forceinline__ void int4_tile(const GemvParams &p, const uint4 &w, int kt_base, int g, int t,
+                                          uint32_t zlo, uint32_t zhi, float (&cg)[MT][4])
+{
+    uint32_t xr[4], yr[4], zr[4], wr[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        xr[i] = bf16x2_sub(nib_pair_bf16(w.x >> (4 * i)), zlo);
+        yr[i] = bf16x2_sub(nib_pair_bf16(w.y >> (4 * i)), zhi);
+        zr[i] = bf16x2_sub(nib_pair_bf16(w.z >> (4 * i)), zlo);
+        wr[i] = bf16x2_sub(nib_pair_bf16(w.w >> (4 * i)), zhi);
+    }
+    uint2 xa[MT], xb[MT], xc[MT], xd[MT];
+    load_x_frag<MT>(p, g, kt_base + 4 * t, xa);
+    load_x_frag<MT>(p, g, kt_base + 16 + 4 * t, xb);
+    load_x_frag<MT>(p, g, kt_base + 32 + 4 * t, xc);
+    load_x_frag<MT>(p, g, kt_base + 48 + 4 * t, xd);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        mma_bf16_16816(cg[mt], xr[0], yr[0], xr[1], yr[1], xa[mt].x, xa[mt].y);
+        mma_bf16_16816(cg[mt], xr[2], yr[2], xr[3], yr[3], xb[mt].x, xb[mt].y);
+        mma_bf16_16816(cg[mt], zr[0], wr[0], zr[1], wr[1], xc[mt].x, xc[mt].y);
+        mma_bf16_16816(cg[mt], zr[2], wr[2], zr[3], wr[3], xd[mt].x, xd[mt].y);
+    }
+}
+
+template <int MT>
+__device__ __forceinline__ void gemv_int8_slice(const GemvParams &p, int rb, int kt0, int kt1, int lane,
+                                                float (&acc)[MT][4])
+{
+    constexpr int U = 4;
+    const int g = lane >> 2, t = lane & 3;
+    const uint8_t *base = p.wq + 16 * lane;
+    uint4 cur[U], nxt[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+        cur[u] = (kt0 + u < kt1) ? ldg_stream(base + p.sh.tile_offset(rb, kt0 + u)) : make_uint4(0, 0, 0, 0);
+    for (int kt = kt0; kt < kt1; kt += U) {
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            nxt[u] = (kt + U + u < kt1) ? ldg_stream(base + p.sh.tile_offset(rb, kt + U + u))
+                                        : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (kt + u < kt1)
+                int8_tile<MT>(p, cur[u], 32 * (kt + u), g, t, acc);
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            cur[u] = nxt[u];
+    }
+}
+
+template <int MT>
+__device__ __forceinline__ void gemv_int4_slice(const GemvParams &p, int rb, int g0, int g1, int lane,
+                                                float (&acc)[MT][4])
+{
+    constexpr int UG = 2; // groups per prefetch batch (2 tiles each)
+    const int g = lane >> 2, t = lane & 3;
+    const int KB = p.sh.kblocks();
+    const int pnl = rb >> 3, rowp = 16 * (rb & 7) + g; // row inside the panel
+    const uint8_t *base = p.wq + 16 * lane;
+    uint4 cw[UG][2], nw[UG][2];
+    uint16_t cs[UG][2], ns[UG][2];
+    uint8_t cz[UG][2], nz[UG][2];
+    auto load = [&](int gi, uint4 (&w)[2], uint16_t (&s)[2], uint8_t (&z)[2]) {
+        if (gi < g1) {
+            const size_t blk = (size_t)pnl * KB + gi;
+            w[0] = ldg_stream(base + p.sh.tile_offset(rb, 2 * gi));
+            w[1] = ldg_stream(base + p.sh.tile_offset(rb, 2 * gi + 1));
+            s[0] = __ldg(p.scales + blk * kPanelRows + rowp);
+            s[1] = __ldg(p.scales + blk * kPanelRows + rowp + 8);
+            z[0] = __ldg(p.zeros + blk * 64 + rowp / 2);
+            z[1] = __ldg(p.zeros + blk * 64 + (rowp + 8) / 2);
+        } else {
+            w[0] = w[1] = make_uint4(0, 0, 0, 0);
+            s[0] = s[1] = 0;
+            z[0] = z[1] = 0;
+        }
+    };
+#pragma unroll
+    for (int u = 0; u < UG; ++u)
+        load(g0 + u, cw[u], cs[u], cz[u]);
+    const int zsh = 4 * (rowp & 1);
+    for (int gi = g0; gi < g1; gi += UG) {
+#pragma unroll
+        for (int u = 0; u < UG; ++u)
+            load(gi + UG + u, nw[u], ns[u], nz[u]);
+#pragma unroll
+        for (int u = 0; u < UG; ++u) {
+            if (gi + u < g1) {
+                const uint32_t zl = (cz[u][0] >> zsh) & 0xFu, zh = (cz[u][1] >> zsh) & 0xFu;
+                const uint32_t zlo = 0x43004300u | zl | (zl << 16);
+                const uint32_t zhi = 0x43004300u | zh | (zh << 16);
+                float cg[MT][4];
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+                    cg[mt][0] = cg[mt][1] = cg[mt][2] = cg[mt][3] = 0.f;
+                const int kt_base = 128 * (gi + u);
+                int4_tile<MT>(p, cw[u][0], kt_base, g, t, zlo, zhi, cg);
+                int4_tile<MT>(p, cw[u][1], kt_base + 64, g, t, zlo, zhi, cg);
+                const float slo = bf16_bits_to_float(cs[u][0]), shi = bf16_bits_to_float(cs[u][1]);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    acc[mt][0] = fmaf(slo, cg[mt][0], acc[mt][0]);
+                    acc[mt][1] = fmaf(slo, cg[mt][1], acc[mt][1]);
+                    acc[mt][2] = fmaf(shi, cg[mt][2], acc[mt][2]);
+                    acc[mt][3] = fmaf(shi, cg[mt][3], acc[mt][3]);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < UG; ++u) {
+            cw[u][0] = nw[u][0];
+            cw[u][1] = nw[u][1];
+            cs[u][0] = ns[u][0];
+            cs[u][1] = ns[u][1];
+            cz[u][0] = nz[u][0];
+            cz[u][1] = nz[u][1];
+        }
+    }
+}
+
+template <int BITS, int MT>
+__global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvParams p)
+{
+    __shared__ float red[kGemvWarps][MT * 4][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int ks = p.ks, rbs_per_cta = kGemvWarps / ks;
+    const int nrb = p.N >> 4;
+    const int units = (nrb + rbs_per_cta - 1) / rbs_per_cta;
+    const int ks_i = warp % ks;
+
+    for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
+        const int rb = unit * rbs_per_cta + warp / ks;
+        float acc[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+            acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+        if (rb < nrb) {
+            if constexpr (BITS == 8) {
+                const int T = p.K / 32;
+                gemv_int8_slice<MT>(p, rb, (int)((long long)T * ks_i / ks), (int)((long long)T * (ks_i + 1) / ks),
+                                    lane, acc);
+            } else {
+                const int G = p.K / 128;
+                gemv_int4_slice<MT>(p, rb, (int)((long long)G * ks_i / ks), (int)((long long)G * (ks_i + 1) / ks),
+                                    lane, acc);
+            }
+        }
+        if (ks > 1) {
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    red[warp][mt * 4 + i][lane] = acc[mt][i];
+            __syncthreads();
+            if (ks_i == 0) {
+                for (int s = 1; s < ks; ++s)
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            acc[mt][i] += red[warp + s][mt * 4 + i][lane];
+            }
+            __syncthreads();
+        }
+        if (ks_i == 0 && rb < nrb) {
+            const int n_lo = 16 * rb + g, n_hi = n_lo + 8;
+            float s_lo = 1.f, s_hi = 1.f;
+            if constexpr (BITS == 8) {
+                s_lo = bf16_bits_to_float(__ldg(p.scales + n_lo));
+                s_hi = bf16_bits_to_float(__ldg(p.scales + n_hi));
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const int m0 = 8 * mt + 2 * t, m1 = m0 + 1;
+                if (m0 < p.M) {
+                    p.y[(size_t)m0 * p.N + n_lo] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[mt][0] * s_lo));
+                    p.y[(size_t)m0 * p.N + n_hi] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[mt][2] * s_hi));
+                }
+                if (m1 < p.M) {
+                    p.y[(size_t)m1 * p.N + n_lo] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[mt][1] * s_lo));
+                    p.y[(size_t)m1 * p.N + n_hi] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[mt][3] * s_hi));
+                }
+            }
+        }
+    }
+}
+
+template <int BITS, int MT>
+static cudaError_t launch_gemv_t(const GemvParams &p, int sm_count, cudaStream_t st)
+{
+    static int occ = -1; // CTAs per SM, from the hardware occupancy query (cached)
+    if (occ < 0) {
+        int o = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, gemv_kernel<BITS, MT>, kGemvWarps * 32, 0);
+        if (e != cudaSuccess)
+            return e;
+        occ = o > 0 ? o : 1;
+    }
+    const int rbs_per_cta = kGemvWarps / p.ks;
+    const int units = ((p.N >> 4) + rbs_per_cta - 1) / rbs_per_cta;
+    int grid = occ * sm_count;
+    if (grid > units)
+        grid = units;
+    gemv_kernel<BITS, MT><<<grid, kGemvWarps * 32, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemv(const LinearArgs &a, int ks, int sm_count, cudaStream_t st)
+{
+    GemvParams p;
+    p.x = a.x;
+    p.M = a.M;
+    p.K = a.K;
+    p.N = a.N;
+    p.wq = (const uint8_t *)a.wq;
+    p.scales = (const uint16_t *)a.scales;
+    p.zeros = (const uint8_t *)a.zeros;
+    p.y = a.y;
+    p.sh = Shape{a.bits, a.K, a.N, a.group};
+    p.ks = ks;
+    const int mt = (a.M + 7) / 8;
+    if (a.bits == 8) {
+        if (mt == 1) return launch_gemv_t<8, 1>(p, sm_count, st);
+        if (mt == 2) return launch_gemv_t<8, 2>(p, sm_count, st);
+        return launch_gemv_t<8, 4>(p, sm_count, st);
+    }
+    if (mt == 1) return launch_gemv_t<4, 1>(p, sm_count, st);
+    if (mt == 2) return launch_gemv_t<4, 2>(p, sm_count, st);
+    return launch_gemv_t<4, 4>(p, sm_count, st);
+}
+
+} // namespace wq

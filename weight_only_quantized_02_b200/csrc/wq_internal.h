@@ -1,0 +1,48 @@
+// wq_internal.h -- declarations shared by the C ABI and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime_api.h>
+
+#include "wq_layout.h"
+
+namespace wq {
+
+struct LinearArgs {
+    const uint16_t *x;
+    int M, K, N;
+    const void *wq, *scales, *zeros;
+    int bits, group;
+    uint16_t *y;
+};
+
+// split-K workspace: [ticket counters, 256-byte padded][fp32 partials S*M*N]
+inline size_t ws_counter_bytes(int N) { return (((size_t)((N + 127) / 128) * 4) + 255) / 256 * 256; }
+inline size_t ws_bytes(int M, int N, int S)
+{
+    return ws_counter_bytes(N) + (S > 1 ? (size_t)S * M * N * sizeof(float) : 0);
+}
+
+cudaError_t launch_quantize_int8(const float *W, int K, int N, int8_t *q, uint16_t *s, cudaStream_t st);
+cudaError_t launch_quantize_int4(const float *W, int K, int N, uint32_t *q, uint16_t *s, uint32_t *z,
+                                 cudaStream_t st);
+cudaError_t launch_pack_int8(const int8_t *q, const uint16_t *s, int K, int N, void *wq, void *s_out,
+                             cudaStream_t st);
+cudaError_t launch_pack_int4(const uint32_t *q, const uint16_t *s, const uint32_t *z, int K, int N, void *wq,
+                             void *s_out, void *z_out, cudaStream_t st);
+cudaError_t launch_unpack_debug(const void *wq, const void *zeros, const Shape &sh, int8_t *q_out,
+                                int8_t *z_out, cudaStream_t st);
+cudaError_t launch_dequant_debug(const void *wq, const void *scales, const void *zeros, const Shape &sh,
+                                 float *w_out, cudaStream_t st);
+
+// GEMV: ks = K slices per 16-row block (1, 2, 4, 8); M <= 32.
+cudaError_t launch_gemv(const LinearArgs &a, int ks, int sm_count, cudaStream_t st);
+
+// GEMM: split = K splits (1..32); ws holds counters + partials when split > 1.
+cudaError_t launch_gemm(const LinearArgs &a, int split, void *ws, int sm_count, cudaStream_t st);
+
+// Reads and clears the device error word of the current device.
+cudaError_t read_device_error(int *code, cudaStream_t st);
+
+} // namespace wq

@@ -1,0 +1,94 @@
+// wq_layout.h -- the packed weight layout shared by the packers, the GEMV
+// and the GEMM.  Host and device.
+//
+// Weights of shape [N][K] are cut into 128-row panels p and 128-k blocks kb.
+// A (panel, k-block) block is contiguous: 8 row-blocks j of 16 rows, each
+// holding `tiles_per_block` tiles of 512 bytes (INT4: 2 tiles of 64 k;
+// INT8: 4 tiles of 32 k).  Inside a tile, lane l = 4g + t (g = l/4, t = l%4)
+// owns the 16 bytes at offset 16 l:
+//
+//   INT8 tile (k base kt):  .x = q[g][kt+4t .. +4]      .y = q[g+8][kt+4t .. +4]
+//                           .z = q[g][kt+16+4t .. +4]   .w = q[g+8][kt+16+4t .. +4]
+//   INT4 tile (k base kt):  .x = row g,   runs a = kt+4t, b = kt+16+4t
+//                           .y = row g+8, runs a, b
+//                           .z = row g,   runs c = kt+32+4t, d = kt+48+4t
+//                           .w = row g+8, runs c, d
+//   an INT4 word holding runs (a, b) stores nibble positions
+//   [a0, a2, b0, b2, a1, a3, b1, b3], so (word >> 4i) & 0x000F000F yields the
+//   natural pairs (a0,a1), (a2,a3), (b0,b1), (b2,b3) for i = 0..3.
+//
+// This is the m16n8k16 mma.sync A fragment of a 16-row block (rows g, g+8,
+// k-slots 2t, 2t+1, 2t+8, 2t+9 taken from a run of four consecutive k), and
+// also the register layout of a tcgen05.st 16x256b store of the same rows
+// into tensor memory in natural k order.  One packed buffer therefore feeds
+// both kernel families, and a warp's 128-bit load of a tile is one
+// contiguous 512-byte segment.
+//
+// Scales: INT8 bf16 [P*128] (s[n], zero past N).  INT4 bf16 [P][K/128][128].
+// Zeros (INT4): [P][K/128][128 nibbles = 64 bytes], row i at nibble i
+// (low nibble first).  A 64-byte trailer follows the packed weights.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#ifdef __CUDACC__
+#define WQ_HD __host__ __device__ __forceinline__
+#else
+#define WQ_HD inline
+#endif
+
+namespace wq {
+
+constexpr int kPanelRows = 128;
+constexpr int kBlockK = 128;
+constexpr int kTileBytes = 512;
+constexpr int kTrailerBytes = 64;
+constexpr uint32_t kMagic = 0x32425157u; // "WQB2"
+constexpr uint32_t kLayoutVersion = 1;
+
+struct Shape {
+    int bits;  // 4 or 8
+    int K, N;
+    int group; // 128 (INT4) or 0 (INT8)
+    WQ_HD int panels() const { return (N + kPanelRows - 1) / kPanelRows; }
+    WQ_HD int kblocks() const { return (K + kBlockK - 1) / kBlockK; }
+    WQ_HD int tile_k() const { return bits == 4 ? 64 : 32; }
+    WQ_HD int tiles_per_block() const { return kBlockK / tile_k(); }
+    WQ_HD int rb_bytes() const { return tiles_per_block() * kTileBytes; }        // one 16-row block, 128 k
+    WQ_HD int block_bytes() const { return 8 * rb_bytes(); }                       // one panel, 128 k
+    WQ_HD size_t weight_bytes() const { return (size_t)panels() * kblocks() * block_bytes(); }
+    WQ_HD size_t wq_bytes() const { return weight_bytes() + kTrailerBytes; }
+    WQ_HD size_t scale_bytes() const
+    {
+        return bits == 8 ? (size_t)panels() * kPanelRows * 2
+                         : (size_t)panels() * kblocks() * kPanelRows * 2;
+    }
+    WQ_HD size_t zero_bytes() const { return bits == 8 ? 0 : (size_t)panels() * kblocks() * 64; }
+    // byte offset of tile (row-block rb = 16-row index, k tile index kt)
+    WQ_HD size_t tile_offset(int rb, int kt) const
+    {
+        const int p = rb >> 3, j = rb & 7;
+        const int tpb = tiles_per_block();
+        const int kb = kt / tpb, t = kt % tpb;
+        return ((size_t)(p * kblocks() + kb) * 8 + j) * rb_bytes() + (size_t)t * kTileBytes;
+    }
+    WQ_HD size_t block_offset(int p, int kb) const { return (size_t)(p * kblocks() + kb) * block_bytes(); }
+};
+
+struct Trailer {
+    uint32_t magic, version, bits, K, N, group, layout_bytes_lo, layout_bytes_hi;
+    uint32_t reserved[8];
+};
+static_assert(sizeof(Trailer) == kTrailerBytes, "trailer is 64 bytes");
+
+// Position of element k (0..7 relative to the word's 8-k group) inside an
+// INT4 word: runs a = k 0..3, b = k 4..7 -> nibble positions.
+WQ_HD int int4_nibble_pos(int e) // e in 0..7: a0..a3 = 0..3, b0..b3 = 4..7
+{
+    // positions [a0, a2, b0, b2, a1, a3, b1, b3]
+    constexpr int pos[8] = {0, 4, 1, 5, 2, 6, 3, 7};
+    return pos[e];
+}
+
+} // namespace wq

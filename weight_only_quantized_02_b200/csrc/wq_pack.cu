@@ -1,0 +1,384 @@
+// wq_pack.cu -- quantizers, packers and debug views of the packed layout.
+//
+// Quantizers turn fp32 source weights into the canonical W8A16 / W4A16
+// tensors (the shapes of the decode workloads).  Every decision is taken in
+// binary64 with IEEE round-to-nearest-even division, as in the CPU oracle.
+// Packers rewrite canonical tensors into the layout of wq_layout.h.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "wq_device.cuh"
+#include "wq_internal.h"
+
+namespace wq {
+
+// ---------------------------------------------------------------------------
+// binary64 -> bf16 rounding (device), from the IEEE-754 definition: find the
+// quantum of |v|'s binade (8 significant bits; fixed 2^-133 below the
+// smallest normal), round the exact count of quanta, scale back.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ double pow2_exact(int e) // 2^e, -1022 <= e <= 1023
+{
+    return __longlong_as_double((long long)(1023 + e) << 52);
+}
+
+__device__ uint16_t f64_to_bf16(double v, bool toward_pos_inf)
+{
+    if (v == 0.0)
+        return signbit(v) ? 0x8000 : 0x0000;
+    const bool neg = signbit(v);
+    const double a = fabs(v);
+    const int e = (int)((__double_as_longlong(a) >> 52) & 0x7FF) - 1023;
+    const int qe = (e >= -126) ? e - 7 : -133;
+    const double count = a * pow2_exact(-qe); // exact
+    double r;
+    if (toward_pos_inf)
+        r = neg ? floor(count) : ceil(count);
+    else
+        r = rint(count); // ties to even
+    const double res = r * pow2_exact(qe);
+    if (res >= 0x1p128)
+        return (toward_pos_inf && neg) ? 0xFF7F : (neg ? 0xFF80 : 0x7F80);
+    const uint32_t fb = __float_as_uint((float)res); // exact
+    return (uint16_t)((fb >> 16) | (neg ? 0x8000u : 0u));
+}
+
+// ---------------------------------------------------------------------------
+// INT8 symmetric per-channel quantizer: one block per output row.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quant_int8_kernel(const float *__restrict__ W, int K,
+                                                         int8_t *__restrict__ q,
+                                                         uint16_t *__restrict__ s)
+{
+    const int n = blockIdx.x;
+    const float *row = W + (size_t)n * K;
+    float amax = 0.f;
+    for (int k = threadIdx.x; k < K; k += blockDim.x)
+        amax = fmaxf(amax, fabsf(row[k]));
+    for (int o = 16; o; o >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    __shared__ float red[8];
+    __shared__ double s_d;
+    if ((threadIdx.x & 31) == 0)
+        red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = 0.f;
+        for (int i = 0; i < (int)(blockDim.x >> 5); ++i)
+            m = fmaxf(m, red[i]);
+        const uint16_t sb = f64_to_bf16((double)m / 127.0, false);
+        s[n] = sb;
+        s_d = (double)bf16_bits_to_float(sb);
+    }
+    __syncthreads();
+    const double sd = s_d;
+    for (int k = threadIdx.x; k < K; k += blockDim.x) {
+        double v = 0.0;
+        if (sd != 0.0) {
+            v = rint((double)row[k] / sd);
+            v = fmin(fmax(v, -127.0), 127.0);
+        }
+        q[(size_t)n * K + k] = (int8_t)v;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// INT4 asymmetric group quantizer: a half-warp per (row, group of 128), each
+// lane owning 8 consecutive k (one canonical word).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quant_int4_kernel(const float *__restrict__ W, int K, int N,
+                                                         uint32_t *__restrict__ q,
+                                                         uint16_t *__restrict__ s,
+                                                         uint32_t *__restrict__ z)
+{
+    const int KG = K / 128, ZW = (KG + 7) / 8;
+    const long long unit = (long long)blockIdx.x * 16 + (threadIdx.x >> 4);
+    const int l16 = threadIdx.x & 15;
+    const bool active = unit < (long long)N * KG;
+    const int n = active ? (int)(unit / KG) : 0;
+    const int g = active ? (int)(unit % KG) : 0;
+    float v[8];
+    const float *src = W + (size_t)n * K + (size_t)g * 128 + 8 * l16;
+    float mn = 0.f, mx = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        v[e] = active ? src[e] : 0.f;
+        mn = fminf(mn, v[e]);
+        mx = fmaxf(mx, v[e]);
+    }
+#pragma unroll
+    for (int o = 8; o; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o, 16));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o, 16));
+    }
+    if (!active)
+        return;
+    const double lo = (double)mn, hi = (double)mx; // lo <= 0 <= hi
+    uint16_t sb = 0;
+    double sd = 0.0;
+    uint32_t zq = 0;
+    if (hi - lo > 0.0) {
+        sb = f64_to_bf16((hi - lo) / 15.0, true);
+        sd = (double)bf16_bits_to_float(sb);
+        zq = (uint32_t)fmin(fmax(rint(-lo / sd), 0.0), 15.0);
+    }
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        uint32_t qe = 0;
+        if (sd != 0.0)
+            qe = (uint32_t)fmin(fmax(rint((double)v[e] / sd) + (double)zq, 0.0), 15.0);
+        word |= qe << (4 * e);
+    }
+    q[(size_t)n * (K / 8) + (size_t)g * 16 + l16] = word;
+    if (l16 == 0) {
+        s[(size_t)n * KG + g] = sb;
+        if (zq)
+            atomicOr(&z[(size_t)n * ZW + g / 8], zq << (4 * (g % 8)));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Packers
+// ---------------------------------------------------------------------------
+__global__ void pack_int8_kernel(const int8_t *__restrict__ q, int K, int N, uint4 *__restrict__ out,
+                                 size_t n_vec, Shape sh)
+{
+    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= n_vec)
+        return;
+    const int vec_per_block = sh.block_bytes() / 16, vec_per_rb = sh.rb_bytes() / 16;
+    const size_t b = idx / vec_per_block;
+    const int u = (int)(idx % vec_per_block);
+    const int p = (int)(b / sh.kblocks()), kb = (int)(b % sh.kblocks());
+    const int j = u / vec_per_rb, rem = u % vec_per_rb;
+    const int t = rem / 32, l = rem % 32, g = l >> 2, tt = l & 3;
+    const int n0 = p * kPanelRows + 16 * j;
+    const int kt = kb * kBlockK + 32 * t;
+    auto run = [&](int row, int k) -> uint32_t {
+        if (row >= N || k >= K)
+            return 0u;
+        return *reinterpret_cast<const uint32_t *>(q + (size_t)row * K + k);
+    };
+    uint4 v;
+    v.x = run(n0 + g, kt + 4 * tt);
+    v.y = run(n0 + g + 8, kt + 4 * tt);
+    v.z = run(n0 + g, kt + 16 + 4 * tt);
+    v.w = run(n0 + g + 8, kt + 16 + 4 * tt);
+    out[idx] = v;
+}
+
+__device__ __forceinline__ uint32_t canon_nibble(const uint32_t *q, int K, int row, int k)
+{
+    return (q[(size_t)row * (K / 8) + k / 8] >> (4 * (k % 8))) & 0xFu;
+}
+
+__global__ void pack_int4_kernel(const uint32_t *__restrict__ q, int K, int N, uint4 *__restrict__ out,
+                                 size_t n_vec, Shape sh)
+{
+    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= n_vec)
+        return;
+    const int vec_per_block = sh.block_bytes() / 16, vec_per_rb = sh.rb_bytes() / 16;
+    const size_t b = idx / vec_per_block;
+    const int u = (int)(idx % vec_per_block);
+    const int p = (int)(b / sh.kblocks()), kb = (int)(b % sh.kblocks());
+    const int j = u / vec_per_rb, rem = u % vec_per_rb;
+    const int t = rem / 32, l = rem % 32, g = l >> 2, tt = l & 3;
+    const int n0 = p * kPanelRows + 16 * j;
+    const int kt = kb * kBlockK + 64 * t;
+    auto word = [&](int row, int ka, int kbb) -> uint32_t {
+        if (row >= N)
+            return 0u;
+        uint32_t w = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int k = (e < 4) ? ka + e : kbb + (e - 4);
+            w |= canon_nibble(q, K, row, k) << (4 * int4_nibble_pos(e));
+        }
+        return w;
+    };
+    uint4 v;
+    v.x = word(n0 + g, kt + 4 * tt, kt + 16 + 4 * tt);
+    v.y = word(n0 + g + 8, kt + 4 * tt, kt + 16 + 4 * tt);
+    v.z = word(n0 + g, kt + 32 + 4 * tt, kt + 48 + 4 * tt);
+    v.w = word(n0 + g + 8, kt + 32 + 4 * tt, kt + 48 + 4 * tt);
+    out[idx] = v;
+}
+
+__global__ void pack_scales_int8_kernel(const uint16_t *__restrict__ s, int N, uint16_t *__restrict__ out,
+                                        int total)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < total)
+        out[i] = i < N ? s[i] : 0;
+}
+
+__global__ void pack_sz_int4_kernel(const uint16_t *__restrict__ s, const uint32_t *__restrict__ z, int K,
+                                    int N, uint16_t *__restrict__ s_out, uint8_t *__restrict__ z_out,
+                                    Shape sh)
+{
+    const int KG = K / 128, ZW = (KG + 7) / 8;
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long total = (long long)sh.panels() * KG * kPanelRows;
+    if (idx >= total)
+        return;
+    const int i = (int)(idx % kPanelRows);
+    const long long pg = idx / kPanelRows;
+    const int g = (int)(pg % KG), p = (int)(pg / KG);
+    const int row = p * kPanelRows + i;
+    s_out[idx] = row < N ? s[(size_t)row * KG + g] : 0;
+    if ((i & 1) == 0) {
+        uint32_t z0 = 0, z1 = 0;
+        if (row < N)
+            z0 = (z[(size_t)row * ZW + g / 8] >> (4 * (g % 8))) & 0xFu;
+        if (row + 1 < N)
+            z1 = (z[(size_t)(row + 1) * ZW + g / 8] >> (4 * (g % 8))) & 0xFu;
+        z_out[pg * 64 + i / 2] = (uint8_t)(z0 | (z1 << 4));
+    }
+}
+
+__global__ void write_trailer_kernel(uint8_t *wq, Shape sh)
+{
+    Trailer t{};
+    t.magic = kMagic;
+    t.version = kLayoutVersion;
+    t.bits = (uint32_t)sh.bits;
+    t.K = (uint32_t)sh.K;
+    t.N = (uint32_t)sh.N;
+    t.group = (uint32_t)sh.group;
+    const size_t wb = sh.weight_bytes();
+    t.layout_bytes_lo = (uint32_t)(wb & 0xffffffffu);
+    t.layout_bytes_hi = (uint32_t)(wb >> 32);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(wq + wb);
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(&t);
+    for (int i = 0; i < 16; ++i)
+        dst[i] = src[i];
+}
+
+// ---------------------------------------------------------------------------
+// Debug views: element (n, k) of the packed layout.
+// ---------------------------------------------------------------------------
+__device__ int packed_q(const uint8_t *wq, const Shape &sh, int n, int k)
+{
+    const int rb = n >> 4, r = n & 15, g = r & 7, hi = r >> 3;
+    const int tk = sh.tile_k();
+    const int kt = k / tk, kk = k % tk;
+    const uint8_t *tile = wq + sh.tile_offset(rb, kt);
+    if (sh.bits == 8) {
+        const int run = kk / 16, t = (kk % 16) / 4, e = kk % 4;
+        const int comp = run * 2 + hi;
+        return (int)(int8_t)tile[16 * (4 * g + t) + 4 * comp + e];
+    }
+    const int half = kk / 32, hk = kk % 32, run = hk / 16, t = (hk % 16) / 4;
+    const int e = run * 4 + hk % 4;
+    const int comp = half * 2 + hi;
+    const uint32_t w = *reinterpret_cast<const uint32_t *>(tile + 16 * (4 * g + t) + 4 * comp);
+    return (int)((w >> (4 * int4_nibble_pos(e))) & 0xFu);
+}
+
+__device__ int packed_z(const uint8_t *zeros, const Shape &sh, int n, int g)
+{
+    const int p = n / kPanelRows, i = n % kPanelRows;
+    const uint8_t b = zeros[((size_t)p * sh.kblocks() + g) * 64 + i / 2];
+    return (i & 1) ? (b >> 4) : (b & 0xF);
+}
+
+__global__ void unpack_debug_kernel(const uint8_t *wq, const uint8_t *zeros, Shape sh, int8_t *q_out,
+                                    int8_t *z_out)
+{
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long total = (long long)sh.N * sh.K;
+    if (idx >= total)
+        return;
+    const int n = (int)(idx / sh.K), k = (int)(idx % sh.K);
+    q_out[idx] = (int8_t)packed_q(wq, sh, n, k);
+    if (sh.bits == 4 && z_out && (k % 128) == 0)
+        z_out[(size_t)n * (sh.K / 128) + k / 128] = (int8_t)packed_z(zeros, sh, n, k / 128);
+}
+
+__global__ void dequant_debug_kernel(const uint8_t *wq, const uint16_t *scales, const uint8_t *zeros,
+                                     Shape sh, float *w_out)
+{
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long total = (long long)sh.N * sh.K;
+    if (idx >= total)
+        return;
+    const int n = (int)(idx / sh.K), k = (int)(idx % sh.K);
+    const int q = packed_q(wq, sh, n, k);
+    if (sh.bits == 8) {
+        w_out[idx] = bf16_bits_to_float(scales[n]) * (float)q;
+    } else {
+        const int p = n / kPanelRows, i = n % kPanelRows, g = k / 128;
+        const float s = bf16_bits_to_float(scales[((size_t)p * sh.kblocks() + g) * kPanelRows + i]);
+        w_out[idx] = s * (float)(q - packed_z(zeros, sh, n, g));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------
+static inline unsigned nblk(long long total, int threads) { return (unsigned)((total + threads - 1) / threads); }
+
+cudaError_t launch_quantize_int8(const float *W, int K, int N, int8_t *q, uint16_t *s, cudaStream_t st)
+{
+    quant_int8_kernel<<<N, 256, 0, st>>>(W, K, q, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_int4(const float *W, int K, int N, uint32_t *q, uint16_t *s, uint32_t *z,
+                                 cudaStream_t st)
+{
+    const int KG = K / 128, ZW = (KG + 7) / 8;
+    cudaError_t e = cudaMemsetAsync(z, 0, (size_t)N * ZW * sizeof(uint32_t), st);
+    if (e != cudaSuccess)
+        return e;
+    const long long units = (long long)N * KG;
+    quant_int4_kernel<<<nblk(units, 16), 256, 0, st>>>(W, K, N, q, s, z);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_int8(const int8_t *q, const uint16_t *s, int K, int N, void *wq, void *s_out,
+                             cudaStream_t st)
+{
+    const Shape sh{8, K, N, 0};
+    const size_t n_vec = sh.weight_bytes() / 16;
+    pack_int8_kernel<<<nblk((long long)n_vec, 256), 256, 0, st>>>(q, K, N, (uint4 *)wq, n_vec, sh);
+    const int total = sh.panels() * kPanelRows;
+    pack_scales_int8_kernel<<<nblk(total, 256), 256, 0, st>>>(s, N, (uint16_t *)s_out, total);
+    write_trailer_kernel<<<1, 1, 0, st>>>((uint8_t *)wq, sh);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_int4(const uint32_t *q, const uint16_t *s, const uint32_t *z, int K, int N,
+                             void *wq, void *s_out, void *z_out, cudaStream_t st)
+{
+    const Shape sh{4, K, N, 128};
+    const size_t n_vec = sh.weight_bytes() / 16;
+    pack_int4_kernel<<<nblk((long long)n_vec, 256), 256, 0, st>>>(q, K, N, (uint4 *)wq, n_vec, sh);
+    const long long total = (long long)sh.panels() * (K / 128) * kPanelRows;
+    pack_sz_int4_kernel<<<nblk(total, 256), 256, 0, st>>>(s, z, K, N, (uint16_t *)s_out, (uint8_t *)z_out, sh);
+    write_trailer_kernel<<<1, 1, 0, st>>>((uint8_t *)wq, sh);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_debug(const void *wq, const void *zeros, const Shape &sh, int8_t *q_out,
+                                int8_t *z_out, cudaStream_t st)
+{
+    const long long total = (long long)sh.N * sh.K;
+    unpack_debug_kernel<<<nblk(total, 256), 256, 0, st>>>((const uint8_t *)wq, (const uint8_t *)zeros, sh,
+                                                         q_out, z_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_debug(const void *wq, const void *scales, const void *zeros, const Shape &sh,
+                                 float *w_out, cudaStream_t st)
+{
+    const long long total = (long long)sh.N * sh.K;
+    dequant_debug_kernel<<<nblk(total, 256), 256, 0, st>>>((const uint8_t *)wq, (const uint16_t *)scales,
+                                                          (const uint8_t *)zeros, sh, w_out);
+    return cudaGetLastError();
+}
+
+} // namespace wq

@@ -1,0 +1,582 @@
+#!/usr/bin/env python
+"""Benchmark of the weight-only quantized linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME|all]
+
+Metric: effective weight GB/s -- algorithmic bytes (packed weight codes +
+scales + zeros + activations in + outputs out, each counted once) per second
+-- with the fraction of the HBM roofline, and TFLOP/s (2*M*K*N per call).
+
+Default workload: the W8A16 decode GEMV, K = 5120, N = 17408, M in {1, 2, 4}.
+One step = one wq_linear call per M on every one of R packed-weight copies,
+R chosen so the copies span more than 5x the L2 size.  Every call therefore
+streams its weights from HBM (rotation instead of an L2 flush).  Each call
+is captured once in its own CUDA graph and replayed; CUDA events recorded on
+the launching stream between the graph launches bracket every kernel, so
+per-kernel durations come from the timed region itself.
+
+With --gpus N > 1 (launched by torchrun) every rank runs the same workload
+on its own GPU: the layer needs no exchange step, so this is weak scaling
+over replicas.  Time is the maximum over ranks, and the value is the total
+over all ranks divided by it.
+
+--impl reference times the CPU oracle (the plain fp64 implementation) on
+the host cores over a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import wq_inputs as gen  # noqa: E402
+
+DEFAULT_WORKLOAD = "w8_decode_5120x17408"
+L2_ROTATION_FACTOR = 5
+
+
+# ---------------------------------------------------------------------------
+# workload arithmetic (bytes, flops)
+# ---------------------------------------------------------------------------
+
+def weight_bytes(bits, K, N, group):
+    if bits == 8:
+        return N * K + 2 * N
+    g = K // group
+    return N * K // 2 + 2 * N * g + N * g // 2
+
+
+def call_bytes(bits, K, N, group, M):
+    return weight_bytes(bits, K, N, group) + 2 * M * K + 2 * M * N
+
+
+def call_flops(K, N, M):
+    return 2 * M * K * N
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def init_dist(world, backend):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def reduce_over_ranks(value: float, op: str, device=None) -> float:
+    """max/sum of a per-rank scalar over all ranks (identity with one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate(per_rank_bytes: float, per_rank_seconds: float, device=None):
+    """Whole-job throughput: bytes of all ranks over the slowest rank's time."""
+    total = reduce_over_ranks(per_rank_bytes, "sum", device)
+    tmax = reduce_over_ranks(per_rank_seconds, "max", device)
+    return total, tmax, (total / tmax if tmax > 0 else 0.0)
+
+
+# ---------------------------------------------------------------------------
+# measurement helpers
+# ---------------------------------------------------------------------------
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms in the background while work runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, smax, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                clk, mx = float(parts[1]), float(parts[2])
+                pw = float(parts[3])
+            except ValueError:
+                continue
+            smax = mx
+            if pw > 200:  # under load
+                sm.append(clk)
+                power.append(pw)
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples_under_load": len(sm), "samples": len(self.lines),
+                "power_w_median": statistics.median(power) if power else None}
+
+
+def profile_traffic(kernel_file: str, summary_name: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken
+    on the current kernel source (sha256 recorded in the summary)."""
+    path = os.path.join(ROOT, "profiles", summary_name)
+    src = os.path.join(ROOT, "weight_only_quantized_02_b200", "csrc", kernel_file)
+    try:
+        text = open(path).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip().lstrip("- ").strip("`")] = v.strip().strip("`")
+    if vals.get("source_sha256") != sha:
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def build_weights(name, device, copies):
+    import torch
+
+    import weight_only_quantized_02_b200 as wq
+    cfg = gen.WORKLOADS[name]
+    K, N, bits = cfg["K"], cfg["N"], cfg["bits"]
+    if cfg.get("direct"):
+        q, s = gen.direct_int8(K, N)
+        pw0 = wq.wq_pack_int8(torch.from_numpy(q).to(device), torch.from_numpy(s.view(np.int16)).to(device))
+    else:
+        W = torch.from_numpy(gen.W_f32(0, N, K)).to(device)
+        if bits == 8:
+            q, s = wq.wq_quantize_int8(W)
+            pw0 = wq.wq_pack_int8(q, s)
+        else:
+            q, s, z = wq.wq_quantize_int4(W)
+            pw0 = wq.wq_pack_int4(q, s, z)
+        del W, q, s
+    pws = [pw0]
+    for _ in range(copies - 1):
+        pws.append(wq.PackedWeight(pw0.wq.clone(), pw0.scales.clone(),
+                                   None if pw0.zeros is None else pw0.zeros.clone(), pw0.bits, pw0.K, pw0.N,
+                                   pw0.group))
+    torch.cuda.synchronize(device)
+    torch.cuda.empty_cache()
+    return cfg, pws
+
+
+def kernel_name(variant, bits):
+    return ("gemv" if variant == 0 else "gemm") + f"_w{bits}"
+
+
+def bench_ours(args, device, rank, world):
+    import torch
+
+    import weight_only_quantized_02_b200 as wq
+    name = args.workload
+    cfg0 = gen.WORKLOADS[name]
+    K, N, bits, group = cfg0["K"], cfg0["N"], cfg0["bits"], cfg0["group"]
+    Ms = list(cfg0["Ms"])
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    wbytes = weight_bytes(bits, K, N, group)
+    copies = max(2, math.ceil(L2_ROTATION_FACTOR * l2 / wbytes))
+    cfg, pws = build_weights(name, device, copies)
+    ws = torch.zeros(wq.wq_workspace_bytes(max(Ms), N, 32), dtype=torch.uint8, device=device)
+    wq.wq_set_workspace(ws)
+    xs = {M: torch.from_numpy(gen.x_bf16(M, K).view(np.int16)).view(torch.bfloat16).to(device) for M in Ms}
+    ys = {M: torch.empty((M, N), dtype=torch.bfloat16, device=device) for M in Ms}
+    choices = {M: wq.wq_get_choice(M, K, N, bits, group) for M in Ms}
+
+    # tuning (the dispatcher's measured choice), untimed
+    if args.tune:
+        for M in Ms:
+            choices[M] = wq.wq_tune(xs[M], pws[0], ys[M], warmup=2, iters=7)
+
+    calls = [(M, c) for c in range(copies) for M in Ms]  # one step
+    stream = torch.cuda.Stream(device)
+    P = max(1, min(args.steps, 64))  # event sets: per-launch times of the last P steps
+
+    # warm the launch path before capture (attributes, tensor maps)
+    with torch.cuda.stream(stream):
+        for M, c in calls:
+            wq.wq_linear(xs[M], pws[c], y=ys[M], stream=stream)
+    torch.cuda.synchronize(device)
+
+    # one CUDA graph per call; events are recorded on the stream between
+    # graph launches so each kernel's device duration is measurable
+    graphs = []
+    for M, c in calls:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            wq.wq_linear(xs[M], pws[c], y=ys[M], stream=stream)
+        graphs.append(g)
+    torch.cuda.synchronize(device)
+    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(calls))] for _ in range(P)]
+
+    def run_step(evs):
+        for i, g in enumerate(graphs):
+            if evs is not None:
+                evs[2 * i].record(stream)
+            g.replay()
+            if evs is not None:
+                evs[2 * i + 1].record(stream)
+
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    sampler = ClockSampler(vis.split(",")[device.index] if vis else device.index)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        # device warm-up before measuring (as the page's timing protocol does)
+        t0 = time.time()
+        i = 0
+        while time.time() - t0 < args.soak:
+            run_step(None)
+            i += 1
+            if i % 20 == 0:
+                torch.cuda.synchronize(device)
+        for w in range(args.warmup):
+            run_step(evsets[w % P])
+    torch.cuda.synchronize(device)
+
+    barrier(device)
+    torch.cuda.synchronize(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for s in range(args.steps):
+            run_step(evsets[s % P])
+        end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clocks = sampler.stop()
+    elapsed_s = start.elapsed_time(end) / 1000.0
+
+    # per-launch durations from the timed region (its last P steps)
+    per_call_us = {M: [] for M in Ms}
+    for evs in evsets[:min(P, args.steps)]:
+        for i, (M, c) in enumerate(calls):
+            per_call_us[M].append(evs[2 * i].elapsed_time(evs[2 * i + 1]) * 1000.0)
+
+    step_bytes = sum(call_bytes(bits, K, N, group, M) for M, _ in calls)
+    step_flops = sum(call_flops(K, N, M) for M, _ in calls)
+    total_bytes, tmax, value_bps = aggregate(step_bytes * args.steps, elapsed_s, device)
+    peaks = read_peaks()
+
+    per_shape = []
+    for M in Ms:
+        us = statistics.mean(per_call_us[M])
+        b = call_bytes(bits, K, N, group, M)
+        f = call_flops(K, N, M)
+        per_shape.append({
+            "M": M, "K": K, "N": N, "variant": kernel_name(choices[M][0], bits), "split": choices[M][1],
+            "us_per_call": round(us, 3), "gbs": round(b / us / 1e3, 1),
+            "hbm_frac_of_measured": round(b / us / 1e3 / peaks["hbm_gbs"], 4),
+            "hbm_frac_of_8tbs": round(b / us / 1e3 / 8000.0, 4),
+            "tflops": round(f / us / 1e6, 3),
+            "roofline_frac": round(max(b / (peaks["hbm_gbs"] * 1e3), f / (peaks["bf16_tflops"] * 1e6)) / us, 4),
+        })
+
+    # dominant kernel: the shape with the largest share of device time
+    share = {M: statistics.mean(per_call_us[M]) for M in Ms}
+    Mdom = max(Ms, key=lambda m: share[m])
+    dom = next(p for p in per_shape if p["M"] == Mdom)
+    vdom = choices[Mdom][0]
+    kfile = "wq_gemv.cu" if vdom == 0 else "wq_gemm.cu"
+    summary = f"{dom['variant']}_{name}_M{Mdom}.md"
+    traffic = profile_traffic(kfile, summary)
+    bound = "hbm"
+    achieved = call_bytes(bits, K, N, group, Mdom) / (share[Mdom] * 1e-6) / 1e9
+    roofline = {"bound": bound, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "kernel": f"{dom['variant']} M={Mdom} split={dom['split']}",
+                "algorithmic_bytes_per_launch": call_bytes(bits, K, N, group, Mdom),
+                "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)",
+                "frac_of_8tbs": round(achieved / 8000.0, 4)}
+
+    e2e = bench_e2e(args, device, xs, pws, Ms, calls, bits, K, N, group, stream)
+    wq.wq_set_workspace(None)
+    return {
+        "value": value_bps / 1e9, "ms_per_step": tmax / args.steps * 1e3, "per_shape": per_shape,
+        "roofline": roofline, "clocks": clocks, "e2e": e2e, "copies": copies,
+        "gpu_launches": args.steps * len(calls), "tflops": step_flops * args.steps * world / tmax / 1e12,
+        "choices": {str(M): list(choices[M]) for M in Ms}, "l2_bytes": l2,
+    }
+
+
+def bench_e2e(args, device, xs, pws, Ms, calls, bits, K, N, group, stream):
+    """Same metric through the public call with host buffers: every step
+    copies its activations in from pinned host memory and its outputs back."""
+    import torch
+
+    import weight_only_quantized_02_b200 as wq
+    hx = {M: xs[M].cpu().pin_memory() for M in Ms}
+    hy = {M: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M in Ms}
+    dx = {M: torch.empty_like(xs[M]) for M in Ms}
+    dy = {M: torch.empty((M, N), dtype=torch.bfloat16, device=device) for M in Ms}
+    steps = max(1, min(args.steps, args.e2e_steps))
+
+    def step():
+        with torch.cuda.stream(stream):
+            for M, c in calls:
+                dx[M].copy_(hx[M], non_blocking=True)
+                wq.wq_linear(dx[M], pws[c], y=dy[M], stream=stream)
+                hy[M].copy_(dy[M], non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 5))):
+        step()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    t = a.elapsed_time(b) / 1000.0
+    step_bytes = sum(call_bytes(bits, K, N, group, M) for M, _ in calls)
+    total, tmax, v = aggregate(step_bytes * steps, t, device)
+    return {"value": round(v / 1e9, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": sum(2 * M * K for M, _ in calls),
+            "d2h_bytes_per_step": sum(2 * M * N for M, _ in calls), "steps": steps,
+            "note": "eager launches through wq_linear, pinned host buffers"}
+
+
+def cpu_baseline(name, budget_s=15.0, rows_cap=None):
+    """The CPU oracle as it stands, on the host cores, over a bounded sample
+    of the workload: every M of one step, on a contiguous block of output
+    channels sized to about `budget_s` seconds of work."""
+    import oracle
+    cfg = gen.WORKLOADS[name]
+    K, N, bits, group = cfg["K"], cfg["N"], cfg["bits"], cfg["group"]
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_threads(threads)
+    xs = {M: gen.x_bf16(M, K) for M in cfg["Ms"]}
+
+    def codes(n0, n1):
+        if cfg.get("direct"):
+            q, s = gen.direct_int8(K, N)
+            return q[n0:n1], s[n0:n1]
+        W = gen.W_f32(n0, n1, K)
+        return oracle.quant_int8(W) if bits == 8 else oracle.quant_int4(W)
+
+    def run(c):
+        for M in cfg["Ms"]:
+            if bits == 8:
+                oracle.linear_int8(xs[M], c[0], c[1])
+            else:
+                oracle.linear_int4(xs[M], c[0], c[1], c[2])
+
+    probe = min(N, 512)
+    c = codes(0, probe)
+    t0 = time.perf_counter()
+    run(c)
+    tp = time.perf_counter() - t0
+    rows = int(min(N, max(probe, probe * budget_s / max(tp, 1e-6))))
+    if rows_cap:
+        rows = min(rows, rows_cap)
+    rows = max(16, rows // 16 * 16)
+    c = codes(0, rows)
+    t0 = time.perf_counter()
+    run(c)
+    t = time.perf_counter() - t0
+    frac = rows / N
+    b = sum(call_bytes(bits, K, N, group, M) for M in cfg["Ms"]) * frac
+    return {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "seconds": round(t, 3),
+            "sample": f"{rows} of {N} output channels, all M in {list(cfg['Ms'])}, one weight copy; "
+                      f"bytes scaled by {rows}/{N}"}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------
+
+def bench_reference(args, rank, world):
+    if rank != 0:
+        return None
+    name = args.workload
+    import oracle
+    cfg = gen.WORKLOADS[name]
+    K, N, bits, group = cfg["K"], cfg["N"], cfg["bits"], cfg["group"]
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_threads(threads)
+    # size each step so the whole run stays within about 90 s of CPU time
+    budget = 90.0 / max(1, args.steps + args.warmup)
+    base = cpu_baseline(name, budget_s=budget)
+    rows = int(base["sample"].split()[0])
+    xs = {M: gen.x_bf16(M, K) for M in cfg["Ms"]}
+    if cfg.get("direct"):
+        q, s = gen.direct_int8(K, N)
+        c = (q[:rows], s[:rows])
+    else:
+        W = gen.W_f32(0, rows, K)
+        c = oracle.quant_int8(W) if bits == 8 else oracle.quant_int4(W)
+
+    def step():
+        for M in cfg["Ms"]:
+            if bits == 8:
+                oracle.linear_int8(xs[M], c[0], c[1])
+            else:
+                oracle.linear_int4(xs[M], c[0], c[1], c[2])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    t = time.perf_counter() - t0
+    b = sum(call_bytes(bits, K, N, group, M) for M in cfg["Ms"]) * rows / N * args.steps
+    value = b / t / 1e9
+    sample = f"{rows} of {N} output channels per step, all M in {list(cfg['Ms'])}"
+    return {
+        "metric": "effective weight GB/s (W8A16/W4A16 linear, algorithmic bytes)", "impl": "reference",
+        "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": name, "K": K, "N": N, "bits": bits, "group": group, "Ms": list(cfg["Ms"]),
+                   "parallelism": "cpu oracle, rank 0 only"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed device warm-up")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--tune", action="store_true", help="run wq_tune per M before timing")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank, local_rank, world = dist_env()
+    if args.impl == "reference":
+        line = bench_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    init_dist(world, "nccl")
+    names = list(gen.WORKLOADS) if args.workload == "all" else [args.workload]
+    for name in names:
+        args.workload = name
+        r = bench_ours(args, device, rank, world)
+        if rank != 0:
+            continue
+        cfg = gen.WORKLOADS[name]
+        line = {
+            "metric": "effective weight GB/s (W8A16/W4A16 linear, algorithmic bytes)",
+            "value": round(r["value"], 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02^2) weights quantized on device)",
+            "config": {"workload": name, "K": cfg["K"], "N": cfg["N"], "bits": cfg["bits"],
+                       "group": cfg["group"], "Ms": list(cfg["Ms"]), "weight_copies": r["copies"],
+                       "l2": f"weights rotated over {r['copies']} copies (> {L2_ROTATION_FACTOR}x L2 of "
+                             f"{r['l2_bytes'] // 2**20} MiB); no flush",
+                       "parallelism": "replicas" if world > 1 else "single GPU", "timing": "CUDA graphs, "
+                       "CUDA events on the launching stream, max over ranks"},
+            "tflops": round(r["tflops"], 2), "per_shape": r["per_shape"], "roofline": r["roofline"],
+            "clocks": r["clocks"], "e2e": r["e2e"], "gpu_launches": r["gpu_launches"],
+            "dispatch": r["choices"],
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(name)
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

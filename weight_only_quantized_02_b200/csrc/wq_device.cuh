@@ -82,6 +82,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
     }
 }
 
+// Warp-uniform form for warps that go on to execute .sync.aligned
+// instructions: every lane polls, the warp agrees on the outcome.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity)) != 0;
+}
+
 // ---------------------------------------------------------------------------
 // Bulk (TMA engine) copies, global -> shared, completing on an mbarrier.
 // No multicast anywhere in this library.

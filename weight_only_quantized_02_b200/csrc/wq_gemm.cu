@@ -14,11 +14,16 @@
 //   warp 1     allocates tensor memory; one thread issues tcgen05.mma with
 //              the dequantized weights as the A operand *from tensor memory*
 //              and x as the B operand from shared memory; fp32 accumulators
-//              stay in tensor memory.
-//   warps 2-5  dequantize the block (INT4: bf16(s*(q - z)); INT8: exact q,
-//              scale applied in the epilogue) and write it to tensor memory
-//              with tcgen05.st 16x256b -- the packed tile is already that
-//              store's register layout -- then run the epilogue.
+//              in tensor memory.
+//   warps 2-5  dequantize the block to exact integers in bf16 (INT4: q - z,
+//              INT8: q) and write it to tensor memory with tcgen05.st
+//              16x256b -- the packed tile is already that store's register
+//              layout.  The weights are never rounded: INT8's per-channel
+//              scale is applied in the epilogue; INT4 accumulates each
+//              128-k group into one of two tensor-memory buffers and these
+//              warps fold s[row][g] * D_g into fp32 register totals one group
+//              behind the MMA (the same arithmetic as the GEMV).  Then they
+//              run the epilogue.
 // Epilogue: split == 1 stores bf16 y.  split > 1 stores fp32 partials; the
 // last CTA of a panel to arrive (atomic ticket, no waiting) sums all partials
 // in split order 0..S-1, so each (variant, split) is run-to-run deterministic,
@@ -56,46 +61,53 @@ struct GemmBits {
     static constexpr int kTilesPerRb = BITS == 4 ? 2 : 4;
 };
 
-template <int NT>
+// Tensor-memory plan per (bits, token tile).  INT4 keeps two group
+// accumulators (double-buffered, NT columns each) so the MMA of group g+1
+// overlaps the fp32 rescale of group g; INT8 keeps one accumulator for the
+// whole K range.  The A ring (64 columns = 128 k of bf16 per stage) follows.
+template <int BITS, int NT>
 struct GemmTile {
-    static constexpr int kStages = NT == 128 ? 4 : 3;
+    static constexpr int kAccBufs = BITS == 4 ? 2 : 1;
     static constexpr int kTmemCols = NT == 128 ? 512 : 256;
-    static constexpr int kA0 = NT < 64 ? 64 : NT; // first tensor-memory column of the A ring
-    static constexpr int kMinBlocks = NT == 128 ? 1 : 2;
+    static constexpr int kA0 = (kAccBufs * NT + 63) / 64 * 64 < 64 ? 64 : (kAccBufs * NT + 63) / 64 * 64;
+    static constexpr int kTmemStages = (kTmemCols - kA0) / 64;
+    static constexpr int kSmemStageBytes = NT * 256 + GemmBits<BITS>::kWBytes + GemmBits<BITS>::kSZBytes;
+    static constexpr int kSmemStages = (200 * 1024) / kSmemStageBytes;
+    static constexpr int kStagesRaw = kTmemStages < kSmemStages ? kTmemStages : kSmemStages;
+    static constexpr int kStages = kStagesRaw > 4 ? 4 : kStagesRaw;
+    static constexpr int kMinBlocks = kTmemCols == 512 ? 1 : 2;
+    static_assert(kStages >= 2, "pipeline needs two stages");
     static_assert(kA0 + 64 * kStages <= kTmemCols, "tensor memory budget");
 };
 
 template <int BITS, int NT>
 constexpr size_t gemm_smem_bytes()
 {
-    return 1024 + (size_t)GemmTile<NT>::kStages * (NT * 256 + GemmBits<BITS>::kWBytes + GemmBits<BITS>::kSZBytes) +
-           (4 * GemmTile<NT>::kStages + 1) * 8 + 16;
+    return 1024 + (size_t)GemmTile<BITS, NT>::kStages * GemmTile<BITS, NT>::kSmemStageBytes +
+           (4 * GemmTile<BITS, NT>::kStages + 5) * 8 + 16;
 }
 
-// Dequantize one INT4 tile (16 rows x 64 k) into the 16 registers of a
-// tcgen05.st 16x256b.x4 store: bf16(s * (q - z)), natural k order.
-__device__ __forceinline__ void int4_tile_regs(const uint4 &w, uint32_t zlo, uint32_t zhi, uint32_t slo,
-                                               uint32_t shi, uint32_t (&r)[16])
+// One INT4 tile (16 rows x 64 k) -> the 16 registers of a tcgen05.st
+// 16x256b.x4 store: the exact integers (q - z) as bf16, natural k order.
+__device__ __forceinline__ void int4_tile_regs(const uint4 &w, uint32_t zlo, uint32_t zhi, uint32_t (&r)[16])
 {
-    auto d = [](uint32_t word, int i, uint32_t zz, uint32_t ss) {
-        return bf16x2_mul(bf16x2_sub(nib_pair_bf16(word >> (4 * i)), zz), ss);
-    };
-    r[0] = d(w.x, 0, zlo, slo);
-    r[1] = d(w.x, 1, zlo, slo);
-    r[2] = d(w.y, 0, zhi, shi);
-    r[3] = d(w.y, 1, zhi, shi);
-    r[4] = d(w.x, 2, zlo, slo);
-    r[5] = d(w.x, 3, zlo, slo);
-    r[6] = d(w.y, 2, zhi, shi);
-    r[7] = d(w.y, 3, zhi, shi);
-    r[8] = d(w.z, 0, zlo, slo);
-    r[9] = d(w.z, 1, zlo, slo);
-    r[10] = d(w.w, 0, zhi, shi);
-    r[11] = d(w.w, 1, zhi, shi);
-    r[12] = d(w.z, 2, zlo, slo);
-    r[13] = d(w.z, 3, zlo, slo);
-    r[14] = d(w.w, 2, zhi, shi);
-    r[15] = d(w.w, 3, zhi, shi);
+    auto d = [](uint32_t word, int i, uint32_t zz) { return bf16x2_sub(nib_pair_bf16(word >> (4 * i)), zz); };
+    r[0] = d(w.x, 0, zlo);
+    r[1] = d(w.x, 1, zlo);
+    r[2] = d(w.y, 0, zhi);
+    r[3] = d(w.y, 1, zhi);
+    r[4] = d(w.x, 2, zlo);
+    r[5] = d(w.x, 3, zlo);
+    r[6] = d(w.y, 2, zhi);
+    r[7] = d(w.y, 3, zhi);
+    r[8] = d(w.z, 0, zlo);
+    r[9] = d(w.z, 1, zlo);
+    r[10] = d(w.w, 0, zhi);
+    r[11] = d(w.w, 1, zhi);
+    r[12] = d(w.z, 2, zlo);
+    r[13] = d(w.z, 3, zlo);
+    r[14] = d(w.w, 2, zhi);
+    r[15] = d(w.w, 3, zhi);
 }
 
 // One INT8 tile (16 rows x 32 k) -> 8 registers of a 16x256b.x2 store: exact q.
@@ -113,13 +125,57 @@ __device__ __forceinline__ void int8_tile_regs(const uint4 &w, uint32_t (&r)[8])
     r[7] = s8pair_bf16(uw, 1);
 }
 
+// Stores one output row's NT values (token m = column) as y, or as split-K
+// partials followed by the last-arriver reduction.  Runs on the 128
+// dequant/epilogue threads (named barrier 1).
+template <int NT>
+__device__ __forceinline__ void gemm_store(const GemmParams &p, int panel, int split, int n, bool nvalid,
+                                           float scale, int warp, int lane, uint32_t *s_ticket,
+                                           const float (&v)[NT])
+{
+    if (p.S == 1) {
+        if (nvalid) {
+#pragma unroll
+            for (int m = 0; m < NT; ++m)
+                if (m < p.M)
+                    p.y[(size_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v[m] * scale));
+        }
+        return;
+    }
+    if (nvalid) {
+#pragma unroll
+        for (int m = 0; m < NT; ++m)
+            if (m < p.M)
+                p.part[((size_t)split * p.M + m) * p.N + n] = v[m];
+    }
+    __threadfence();
+    named_barrier_sync(1, 128);
+    if (warp == 2 && lane == 0)
+        *s_ticket = atomicAdd(&p.cnt[panel], 1u);
+    named_barrier_sync(1, 128);
+    if (*s_ticket == (uint32_t)(p.S - 1)) {
+        __threadfence();
+        if (nvalid) {
+            for (int m = 0; m < p.M; ++m) {
+                float sum = 0.f;
+                for (int s = 0; s < p.S; ++s)
+                    sum += __ldcg(&p.part[((size_t)s * p.M + m) * p.N + n]);
+                p.y[(size_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(sum * scale));
+            }
+        }
+        if (warp == 2 && lane == 0)
+            atomicExch(&p.cnt[panel], 0u);
+    }
+}
+
 template <int BITS, int NT>
-__global__ void __launch_bounds__(192, GemmTile<NT>::kMinBlocks)
+__global__ void __launch_bounds__(192, GemmTile<BITS, NT>::kMinBlocks)
     gemm_kernel(const __grid_constant__ CUtensorMap tmx, const GemmParams p)
 {
-    constexpr int STAGES = GemmTile<NT>::kStages;
-    constexpr int TCOLS = GemmTile<NT>::kTmemCols;
-    constexpr int A0 = GemmTile<NT>::kA0;
+    using T = GemmTile<BITS, NT>;
+    constexpr int STAGES = T::kStages;
+    constexpr int TCOLS = T::kTmemCols;
+    constexpr int A0 = T::kA0;
     constexpr int XB = NT * 256;
     constexpr int WB = GemmBits<BITS>::kWBytes;
     constexpr int SZB = GemmBits<BITS>::kSZBytes;
@@ -132,8 +188,9 @@ __global__ void __launch_bounds__(192, GemmTile<NT>::kMinBlocks)
     uint8_t *sSZ = sW + STAGES * WB;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sSZ + STAGES * SZB);
     uint64_t *full = bars, *ldempty = bars + STAGES, *afull = bars + 2 * STAGES, *aempty = bars + 3 * STAGES;
-    uint64_t *accfull = bars + 4 * STAGES;
-    uint32_t *s_misc = reinterpret_cast<uint32_t *>(bars + 4 * STAGES + 1);
+    uint64_t *accfull = bars + 4 * STAGES;      // [2]
+    uint64_t *accempty = bars + 4 * STAGES + 2; // [2]
+    uint32_t *s_misc = reinterpret_cast<uint32_t *>(bars + 4 * STAGES + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int panel = blockIdx.x, split = blockIdx.y;
@@ -148,7 +205,10 @@ __global__ void __launch_bounds__(192, GemmTile<NT>::kMinBlocks)
             mbar_init(&afull[s], 4);
             mbar_init(&aempty[s], 1);
         }
-        mbar_init(accfull, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accfull[b], 1);
+            mbar_init(&accempty[b], 4);
+        }
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -193,30 +253,75 @@ __global__ void __launch_bounds__(192, GemmTile<NT>::kMinBlocks)
                     ok = false;
                     break;
                 }
+                uint32_t dcol = 0;
+                if constexpr (BITS == 4) {
+                    const int b = i & 1;
+                    if (i >= 2 && !mbar_wait(&accempty[b], ((i >> 1) - 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    dcol = b * NT;
+                }
                 tc_fence_after();
                 const uint32_t xs = smem_u32(sX + st * XB);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t bdesc = smem_desc_sw128(xs + (kk >> 2) * (NT * 128) + (kk & 3) * 32);
-                    umma_ts(tmem, tmem + A0 + st * 64 + kk * 8, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                    const uint32_t acc = BITS == 4 ? (kk > 0 ? 1u : 0u) : ((i > 0 || kk > 0) ? 1u : 0u);
+                    umma_ts(tmem + dcol, tmem + A0 + st * 64 + kk * 8, bdesc, idesc, acc);
                 }
                 umma_commit(&aempty[st]);
                 umma_commit(&ldempty[st]);
+                if constexpr (BITS == 4)
+                    umma_commit(&accfull[i & 1]);
             }
-            umma_commit(accfull);
+            if constexpr (BITS == 8)
+                umma_commit(&accfull[0]);
         }
     } else {
-        // ---------------- dequant warps ----------------
+        // ---------------- dequant / rescale / epilogue warps ----------------
         const int quad = warp & 3; // tensor-memory lane quadrant this warp may access
         const int g = lane >> 2;
-        for (int i = 0; i < nk; ++i) {
+        const int row = 32 * quad + lane; // this thread's output row in the panel
+        const uint32_t tlane = (uint32_t)(32 * quad) << 16;
+        float acc[NT]; // INT4: fp32 totals of this row, one per token
+#pragma unroll
+        for (int c = 0; c < NT; ++c)
+            acc[c] = 0.f;
+        float s_prev = 0.f;
+
+        // fold group j's accumulator into the fp32 totals: acc += s_row * D_j
+        auto rescale = [&](int j, float s) {
+            const int b = j & 1;
+            if (!mbar_wait_warp(&accfull[b], (j >> 1) & 1)) {
+                ok = false;
+                return;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < NT; c0 += 16) {
+                float v[16];
+                tmem_ld_32x32b_x16(tmem + tlane + b * NT + c0, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    acc[c0 + e] = fmaf(s, v[e], acc[c0 + e]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&accempty[b]);
+        };
+
+        for (int i = 0; i < nk && ok; ++i) {
             const int st = i % STAGES, use = i / STAGES;
-            if (!mbar_wait(&full[st], use & 1)) {
+            if (!mbar_wait_warp(&full[st], use & 1)) {
                 ok = false;
                 break;
             }
             uint4 w[2][TPR];
-            uint32_t zz[2][2], ss[2][2];
+            uint32_t zz[2][2];
+            float s_mine = 0.f;
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
                 const int j = 2 * quad + jj;
@@ -225,22 +330,21 @@ __global__ void __launch_bounds__(192, GemmTile<NT>::kMinBlocks)
                     w[jj][tt] = *reinterpret_cast<const uint4 *>(sW + st * WB + j * (TPR * kTileBytes) +
                                                                  tt * kTileBytes + lane * 16);
                 if constexpr (BITS == 4) {
-                    const uint16_t *s16 = reinterpret_cast<const uint16_t *>(sSZ + st * SZB);
                     const uint8_t *z8 = sSZ + st * SZB + 256;
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const int row = 16 * j + g + 8 * h;
-                        const uint32_t z = (z8[row >> 1] >> (4 * (row & 1))) & 0xFu;
-                        const uint32_t s = s16[row];
+                        const int r = 16 * j + g + 8 * h;
+                        const uint32_t z = (z8[r >> 1] >> (4 * (r & 1))) & 0xFu;
                         zz[jj][h] = 0x43004300u | z | (z << 16);
-                        ss[jj][h] = s | (s << 16);
                     }
                 }
             }
+            if constexpr (BITS == 4)
+                s_mine = bf16_bits_to_float(reinterpret_cast<const uint16_t *>(sSZ + st * SZB)[row]);
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&ldempty[st]);
-            if (use > 0 && !mbar_wait(&aempty[st], (use - 1) & 1)) {
+            if (use > 0 && !mbar_wait_warp(&aempty[st], (use - 1) & 1)) {
                 ok = false;
                 break;
             }
@@ -252,7 +356,7 @@ __global__ void __launch_bounds__(192, GemmTile<NT>::kMinBlocks)
                 for (int tt = 0; tt < TPR; ++tt) {
                     if constexpr (BITS == 4) {
                         uint32_t r[16];
-                        int4_tile_regs(w[jj][tt], zz[jj][0], zz[jj][1], ss[jj][0], ss[jj][1], r);
+                        int4_tile_regs(w[jj][tt], zz[jj][0], zz[jj][1], r);
                         tmem_st_16x256b_x4(ta + tt * 32, r);
                     } else {
                         uint32_t r[8];
@@ -266,63 +370,39 @@ __global__ void __launch_bounds__(192, GemmTile<NT>::kMinBlocks)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&afull[st]);
+            if constexpr (BITS == 4) {
+                if (i >= 1)
+                    rescale(i - 1, s_prev);
+                s_prev = s_mine;
+            }
+        }
+        if constexpr (BITS == 4) {
+            if (ok && nk >= 1)
+                rescale(nk - 1, s_prev);
         }
 
         // ---------------- epilogue ----------------
-        if (!mbar_wait(accfull, 0))
-            ok = false;
-        tc_fence_after();
-        const int row = 32 * quad + lane;
         const int n = panel * kPanelRows + row;
         const bool nvalid = n < p.N;
-        float scale = 1.f;
-        if constexpr (BITS == 8)
-            scale = nvalid ? bf16_bits_to_float(p.scales[n]) : 0.f;
-        const uint32_t tacc = tmem + ((uint32_t)(32 * quad) << 16);
-        if (p.S == 1) {
-#pragma unroll 1
-            for (int c0 = 0; c0 < NT; c0 += 16) {
-                float v[16];
-                tmem_ld_32x32b_x16(tacc + c0, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int m = c0 + e;
-                    if (m < p.M && nvalid)
-                        p.y[(size_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v[e] * scale));
-                }
-            }
+        if constexpr (BITS == 4) {
+            gemm_store<NT>(p, panel, split, n, nvalid, 1.f, warp, lane, &s_misc[1], acc);
         } else {
-#pragma unroll 1
+            if (!mbar_wait_warp(&accfull[0], 0))
+                ok = false;
+            tc_fence_after();
+            const float scale = nvalid ? bf16_bits_to_float(p.scales[n]) : 0.f;
+            // stage this row's NT accumulators through registers 16 columns at a time
+            float v[NT];
+#pragma unroll
             for (int c0 = 0; c0 < NT; c0 += 16) {
-                float v[16];
-                tmem_ld_32x32b_x16(tacc + c0, v);
+                float t[16];
+                tmem_ld_32x32b_x16(tmem + tlane + c0, t);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int m = c0 + e;
-                    if (m < p.M && nvalid)
-                        p.part[((size_t)split * p.M + m) * p.N + n] = v[e];
-                }
+                for (int e = 0; e < 16; ++e)
+                    v[c0 + e] = t[e];
             }
-            __threadfence();
-            named_barrier_sync(1, 128);
-            if (warp == 2 && lane == 0)
-                s_misc[1] = atomicAdd(&p.cnt[panel], 1u);
-            named_barrier_sync(1, 128);
-            if (s_misc[1] == (uint32_t)(p.S - 1)) {
-                __threadfence();
-                if (nvalid) {
-                    for (int m = 0; m < p.M; ++m) {
-                        float sum = 0.f;
-                        for (int s = 0; s < p.S; ++s)
-                            sum += __ldcg(&p.part[((size_t)s * p.M + m) * p.N + n]);
-                        p.y[(size_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(sum * scale));
-                    }
-                }
-                if (warp == 2 && lane == 0)
-                    atomicExch(&p.cnt[panel], 0u);
-            }
+            gemm_store<NT>(p, panel, split, n, nvalid, scale, warp, lane, &s_misc[1], v);
         }
     }
 
@@ -372,6 +452,7 @@ template <int BITS, int NT>
 static cudaError_t launch_gemm_t(const LinearArgs &a, int S, void *ws, cudaStream_t st)
 {
     constexpr size_t smem = gemm_smem_bytes<BITS, NT>();
+    static_assert(smem <= 227 * 1024, "shared memory per CTA");
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BITS, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -74,8 +74,9 @@ typedef enum {
 
 /* Kernel variants (wq_linear_forced, wq_get_choice). */
 #define WQ_VARIANT_AUTO (-1)
-#define WQ_VARIANT_GEMV 0 /* mma.sync register-dequant GEMV, M <= 32 */
-#define WQ_VARIANT_GEMM 1 /* tcgen05 split-K GEMM, M <= 128 */
+#define WQ_VARIANT_GEMV 0    /* stream-K GEMV, M <= 32: TMA-fed ring, mma.sync; needs the workspace */
+#define WQ_VARIANT_GEMM 1    /* tcgen05 split-K GEMM, M <= 128 */
+#define WQ_VARIANT_GEMV_RB 2 /* row-block GEMV, M <= 32, direct 128-bit loads; no workspace */
 
 /* Static description of a status code. Host. Never NULL. */
 const char *wq_strerror(int status);
@@ -153,15 +154,18 @@ int wq_check_packed(const void *Wq, int bits, int K, int N, int group, cudaStrea
  *   y       device, bf16 [M][N], row-major, 16-byte aligned. Every element
  *           is written: bf16_rne of the fp32-accumulated sum.
  * The kernel and split factor come from the dispatcher (tuned table, else
- * the default rule). A split factor > 1 uses the workspace registered with
- * wq_set_workspace for the current device. Calls that share that workspace
- * must not overlap on the GPU (keep them on one stream). */
+ * the default rule). The stream-K GEMV and a GEMM split > 1 use the
+ * workspace registered with wq_set_workspace for the current device; with
+ * no workspace, decode-sized M falls back to the row-block GEMV. Calls that
+ * share a workspace must not overlap on the GPU (keep them on one stream). */
 int wq_linear(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
               const void *zeros, int group, int N, uint16_t *y, cudaStream_t stream);
 
 /* wq_linear with an explicit kernel variant (WQ_VARIANT_*) and split factor.
  * variant = WQ_VARIANT_AUTO, or split = 0, leaves that choice to the dispatcher.
- * GEMV: split = K-slices per 16-row block, one of 1, 2, 4, 8.
+ * GEMV: split = CTAs per SM, 1..4, capped by occupancy (the K range of
+ *       every CTA is set by the stream-K partition).
+ * GEMV_RB: split = K-slices per 16-row block, one of 1, 2, 4, 8.
  * GEMM: split = K-splits, 1 <= split <= min(32, ceil(K/128)).
  * Returns WQ_ERR_VARIANT if the pair does not fit the shape. */
 int wq_linear_forced(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
@@ -174,9 +178,10 @@ int wq_linear_ex(const uint16_t *x, int M, int K, const void *Wq, const void *sc
                  const void *zeros, int group, int N, uint16_t *y, int variant, int split,
                  void *ws, size_t ws_bytes, cudaStream_t stream);
 
-/* Bytes of split-K workspace for M tokens, N channels and up to max_split
- * splits: the fp32 partial sums [split][M][N] and one ticket counter per
- * 128-channel panel. Host. */
+/* Bytes of workspace for M tokens, N channels and GEMM splits up to
+ * max_split. It holds one ticket counter per 128-channel panel and the
+ * larger of the GEMM's fp32 partials [split][M][N] and the stream-K GEMV's
+ * per-CTA panel partials (M <= 32). Host. */
 size_t wq_workspace_bytes(int M, int N, int max_split);
 
 /* Registers a caller-owned device workspace for the current device, used by

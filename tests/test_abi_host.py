@@ -65,9 +65,12 @@ def test_packed_bytes_rejects(bits, K, N, group, status):
 
 
 def test_workspace_bytes():
-    # 40 panel tickets padded to 256 bytes + fp32 partials
+    # 40 panel tickets padded to 256 bytes + the larger of the GEMM's fp32
+    # partials and the stream-K GEMV's per-CTA panel partials
     assert wq.wq_workspace_bytes(128, 5120, 32) == 256 + 32 * 128 * 5120 * 4
-    assert wq.wq_workspace_bytes(16, 5120, 1) == 256
+    assert wq.wq_workspace_bytes(64, 5120, 1) == 256
+    assert wq.wq_workspace_bytes(16, 5120, 1) == 256 + 512 * 2 * 128 * 16 * 4
+    assert wq.wq_workspace_bytes(1, 17408, 1) == 768 + 512 * 2 * 128 * 8 * 4  # 136 tickets -> 768 bytes
     assert wq.wq_workspace_bytes(0, 5120, 4) == 0
 
 
@@ -82,7 +85,8 @@ def test_tuning_file_parse_errors(tmp_path):
     good.write_text("# comment\nNVIDIA B200|148 1 5120 17408 8 0 0 4 12.500\n")
     assert wq.wq_load_tuning(str(good)) == 0
     for bad_line in [
-        "NVIDIA B200|148 1 5120 17408 8 0 0 3 12.5\n",      # GEMV split must be 1/2/4/8
+        "NVIDIA B200|148 1 5120 17408 8 0 2 3 12.5\n",      # row-block GEMV split must be 1/2/4/8
+        "NVIDIA B200|148 1 5120 17408 8 0 0 5 12.5\n",      # stream-K GEMV: 1..4 CTAs per SM
         "NVIDIA B200|148 200 5120 17408 8 0 1 4 12.5\n",    # M > 128
         "NVIDIA B200|148 1 5120 17408 8 64 0 4 12.5\n",     # bad group
         "NVIDIA B200 1 5120 17408 8 0 0 4 12.5\n",          # no device key separator

@@ -22,7 +22,7 @@ from wqtest_helpers import (assert_parity, bf16_dev, dev, oracle_linear, pack_ca
 
 pytestmark = pytest.mark.gpu
 
-GEMV, GEMM = wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM
+GEMV, GEMM, GEMV_RB = wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB
 SHAPES = {8: (1120, 400), 4: (1152, 400)}  # (K, N): 3 full panels + a 16-row tail
 M_ALL = [1, 7, 8, 9, 16, 17, 32, 33, 64, 65, 100, 128]
 
@@ -48,7 +48,8 @@ def _cases(M, K):
     kb = (K + 127) // 128
     out = []
     if M <= 32:
-        out += [(GEMV, ks) for ks in (1, 2, 4, 8)]
+        out += [(GEMV, c) for c in (1, 2, 3)]
+        out += [(GEMV_RB, ks) for ks in (1, 2, 4, 8)]
     out += [(GEMM, s) for s in (1, 2, 4, 8, 16, 32) if s <= kb]
     return out
 
@@ -225,20 +226,25 @@ def test_argument_errors(weight, ws):
     bits, K, N, pw, canon = weight
     x = bf16_dev(gen.x_bf16(4, K))
     y = torch.empty((4, N), dtype=torch.bfloat16, device=dev())
-    assert wq.wq_linear_status(x, pw, y, GEMV, 3) == -11          # split not 1/2/4/8
+    assert wq.wq_linear_status(x, pw, y, GEMV_RB, 3) == -11       # split not 1/2/4/8
+    assert wq.wq_linear_status(x, pw, y, GEMV, 5) == -11          # CTAs per SM 1..4
     assert wq.wq_linear_status(x, pw, y, GEMM, 33) == -11         # split above 32
     assert wq.wq_linear_status(x, pw, y, 7, 1) == -11             # unknown variant
     xb = bf16_dev(gen.x_bf16(40, K))
     yb = torch.empty((40, N), dtype=torch.bfloat16, device=dev())
     assert wq.wq_linear_status(xb, pw, yb, GEMV, 1) == -11        # GEMV takes M <= 32
+    assert wq.wq_linear_status(xb, pw, yb, GEMV_RB, 1) == -11
     # misaligned output pointer
     raw = torch.empty(4 * N + 8, dtype=torch.bfloat16, device=dev())
-    assert wq.wq_linear_status(x, pw, raw[1:1 + 4 * N].view(4, N), GEMV, 1) == -3
+    assert wq.wq_linear_status(x, pw, raw[1:1 + 4 * N].view(4, N), GEMV_RB, 1) == -3
     # split > 1 without a workspace
     wq.wq_set_workspace(None)
     try:
         assert wq.wq_linear_status(x, pw, y, GEMM, 4) == -6
+        assert wq.wq_linear_status(x, pw, y, GEMV, 1) == -6
         assert wq.wq_linear_status(x, pw, y, GEMM, 1) == 0
+        assert wq.wq_linear_status(x, pw, y, GEMV_RB, 2) == 0
+        assert wq.wq_linear_status(x, pw, y) == 0  # dispatcher falls back to the row-block GEMV
     finally:
         wq.wq_set_workspace(ws)
     small = torch.zeros(512, dtype=torch.uint8, device=dev())
@@ -267,7 +273,7 @@ def test_explicit_workspace_on_two_streams(weight):
 
 def test_cuda_graph_replay(weight, ws):
     bits, K, N, pw, canon = weight
-    for M, variant, split in [(1, GEMV, 4), (16, GEMM, 4), (128, GEMM, 2)]:
+    for M, variant, split in [(1, GEMV, 2), (1, GEMV_RB, 4), (16, GEMM, 4), (128, GEMM, 2)]:
         x = gen.x_bf16(M, K)
         xd = bf16_dev(x)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
@@ -301,6 +307,6 @@ def test_tuner_and_table_roundtrip(weight, ws, tmp_path):
     wq.wq_clear_tuning()
     assert wq.wq_load_tuning(path) == 0
     assert wq.wq_get_choice(M, K, N, bits, 0 if bits == 8 else 128) == (v, s)
-    wq.wq_set_choice(M, K, N, bits, 0 if bits == 8 else 128, GEMV, 8)
-    assert wq.wq_get_choice(M, K, N, bits, 0 if bits == 8 else 128) == (GEMV, 8)
+    wq.wq_set_choice(M, K, N, bits, 0 if bits == 8 else 128, GEMV_RB, 8)
+    assert wq.wq_get_choice(M, K, N, bits, 0 if bits == 8 else 128) == (GEMV_RB, 8)
     wq.wq_clear_tuning()

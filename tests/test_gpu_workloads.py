@@ -19,7 +19,7 @@ from wqtest_helpers import assert_parity, bf16_dev, bits_u16, bits_u32, dev, wor
 
 pytestmark = pytest.mark.gpu
 
-GEMV, GEMM = wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM
+GEMV, GEMM, GEMV_RB = wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB
 
 
 def _build(name):
@@ -73,7 +73,8 @@ def _ref(cfg, x, codes):
 def _variants(M, K):
     out = []
     if M <= 32:
-        out += [(GEMV, ks) for ks in (1, 2, 4, 8)]
+        out += [(GEMV, c) for c in (1, 2, 3)]
+        out += [(GEMV_RB, ks) for ks in (1, 2, 4, 8)]
     out += [(GEMM, s) for s in (1, 2, 4, 8, 16, 32) if s <= (K + 127) // 128]
     return out
 

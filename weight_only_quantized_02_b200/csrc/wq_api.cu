@@ -111,27 +111,36 @@ int max_gemm_split(int K) { return std::min(32, (K + kBlockK - 1) / kBlockK); }
 bool choice_valid(int variant, int split, int M, int K)
 {
     if (variant == WQ_VARIANT_GEMV)
+        return M <= 32 && split >= 1 && split <= 4;
+    if (variant == WQ_VARIANT_GEMV_RB)
         return M <= 32 && (split == 1 || split == 2 || split == 4 || split == 8);
     if (variant == WQ_VARIANT_GEMM)
         return M <= 128 && split >= 1 && split <= max_gemm_split(K);
     return false;
 }
 
+// Row-block GEMV K-slices: keep about 32 warps per SM busy.
+int default_rb_slices(int K, int N, int sm_count)
+{
+    const long long rbs = N / 16;
+    int ks = 1;
+    while (ks < 8 && rbs * ks < (long long)sm_count * 32)
+        ks *= 2;
+    while (ks > 1 && K / 128 < ks)
+        ks /= 2;
+    return ks;
+}
+
 // The pages' untuned rule: fewer than 8 tokens -> GEMV, otherwise the GEMM
 // with split_k = 8 (Mit han lab Llm awq Kernel Selection Thresholds, The
-// Insight).  The GEMV's K-slice count keeps about 32 warps per SM busy.
-Choice default_choice(int M, int K, int N, int sm_count)
+// Insight).  The stream-K GEMV needs the split-K workspace; without one the
+// row-block GEMV is used.
+Choice default_choice(int M, int K, int N, int sm_count, bool have_ws = true)
 {
     if (M < 8) {
-        const long long rbs = N / 16;
-        int ks = 1;
-        while (ks < 8 && rbs * ks < (long long)sm_count * 32)
-            ks *= 2;
-        if (K / 128 < ks)
-            ks = std::max(1, K / 128);
-        while (ks > 1 && (ks & (ks - 1)))
-            --ks;
-        return {WQ_VARIANT_GEMV, ks, 0.f};
+        if (have_ws)
+            return {WQ_VARIANT_GEMV, 2, 0.f};
+        return {WQ_VARIANT_GEMV_RB, default_rb_slices(K, N, sm_count), 0.f};
     }
     return {WQ_VARIANT_GEMM, std::min(8, max_gemm_split(K)), 0.f};
 }
@@ -173,46 +182,54 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
     if (d.major != 10)
         return WQ_ERR_ARCH;
 
+    // the workspace this call would use (explicit, else the registered one)
+    void *w = ws;
+    size_t have = ws_bytes_given;
+    if (!w) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_ws.find(dev);
+        if (it != g_ws.end()) {
+            w = it->second.first;
+            have = it->second.second;
+        }
+    }
+    if (w && !aligned16(w))
+        return WQ_ERR_ALIGN;
+    const bool sk_ws_ok = w && have >= ws_bytes_gemv_sk(M, N);
+
     Choice c;
     lookup_choice(d, M, K, N, bits, group, &c);
     if (variant != WQ_VARIANT_AUTO) {
         c.variant = variant;
         if (split <= 0)
-            c.split = default_choice(variant == WQ_VARIANT_GEMV ? 1 : 8, K, N, d.sm_count).split;
+            c.split = variant == WQ_VARIANT_GEMV      ? 2
+                      : variant == WQ_VARIANT_GEMV_RB ? default_rb_slices(K, N, d.sm_count)
+                                                      : std::min(8, max_gemm_split(K));
     }
     if (split > 0)
         c.split = split;
-    if (variant == WQ_VARIANT_AUTO && !choice_valid(c.variant, c.split, M, K))
-        c = default_choice(M, K, N, d.sm_count);
+    if (variant == WQ_VARIANT_AUTO) {
+        if (!choice_valid(c.variant, c.split, M, K))
+            c = default_choice(M, K, N, d.sm_count, sk_ws_ok);
+        if (c.variant == WQ_VARIANT_GEMV && !sk_ws_ok)
+            c = {WQ_VARIANT_GEMV_RB, default_rb_slices(K, N, d.sm_count), 0.f};
+    }
     if (!choice_valid(c.variant, c.split, M, K))
         return WQ_ERR_VARIANT;
 
     LinearArgs a{x, M, K, N, Wq, scales, zeros, bits, group, y};
-    if (c.variant == WQ_VARIANT_GEMV)
+    if (c.variant == WQ_VARIANT_GEMV_RB)
         return cuda_status(launch_gemv(a, c.split, d.sm_count, stream));
-
-    void *w = nullptr;
-    if (c.split > 1) {
-        size_t have = 0;
-        if (ws) {
-            w = ws;
-            have = ws_bytes_given;
-        } else {
-            int dev = 0;
-            cudaGetDevice(&dev);
-            std::lock_guard<std::mutex> lk(g_mu);
-            auto it = g_ws.find(dev);
-            if (it != g_ws.end()) {
-                w = it->second.first;
-                have = it->second.second;
-            }
-        }
-        if (!w || have < ws_bytes(M, N, c.split))
+    if (c.variant == WQ_VARIANT_GEMV) {
+        if (!sk_ws_ok)
             return WQ_ERR_WORKSPACE;
-        if (!aligned16(w))
-            return WQ_ERR_ALIGN;
+        return cuda_status(launch_gemv_sk(a, c.split, w, d.sm_count, stream));
     }
-    return cuda_status(launch_gemm(a, c.split, w, d.sm_count, stream));
+    if (c.split > 1 && (!w || have < ws_bytes(M, N, c.split)))
+        return WQ_ERR_WORKSPACE;
+    return cuda_status(launch_gemm(a, c.split, c.split > 1 ? w : nullptr, d.sm_count, stream));
 }
 
 } // namespace
@@ -348,7 +365,10 @@ size_t wq_workspace_bytes(int M, int N, int max_split)
 {
     if (M < 1 || N < 1 || max_split < 1)
         return 0;
-    return ws_bytes(M, N, max_split);
+    size_t b = ws_bytes(M, N, max_split);
+    if (M <= 32)
+        b = std::max(b, ws_bytes_gemv_sk(M, N));
+    return b;
 }
 
 int wq_set_workspace(void *ws, size_t bytes)
@@ -386,9 +406,12 @@ int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
     if (warmup < 0 || iters < 1)
         return WQ_ERR_SHAPE;
     std::vector<std::pair<int, int>> cands;
-    if (M <= 32)
+    if (M <= 32) {
+        for (int c : {1, 2, 3})
+            cands.push_back({WQ_VARIANT_GEMV, c});
         for (int ks : {1, 2, 4, 8})
-            cands.push_back({WQ_VARIANT_GEMV, ks});
+            cands.push_back({WQ_VARIANT_GEMV_RB, ks});
+    }
     for (int s : {1, 2, 4, 8, 16, 32})
         if (s <= max_gemm_split(K))
             cands.push_back({WQ_VARIANT_GEMM, s});
@@ -584,10 +607,10 @@ int wq_dequant_debug(const void *Wq, const void *scales, const void *zeros, int 
 
 int wq_device_error(cudaStream_t stream)
 {
-    int code = 0;
-    if (read_device_error(&code, stream) != cudaSuccess)
+    int a = 0, b = 0;
+    if (read_device_error(&a, stream) != cudaSuccess || read_gemv_sk_error(&b, stream) != cudaSuccess)
         return WQ_ERR_CUDA;
-    return code == 0 ? WQ_OK : WQ_ERR_TIMEOUT;
+    return (a == 0 && b == 0) ? WQ_OK : WQ_ERR_TIMEOUT;
 }
 
 } // extern "C"

@@ -1,0 +1,410 @@
+// wq_gemv_sk.cu -- stream-K GEMV for decode-sized M (<= 32), W8A16 / W4A16.
+//
+// The packed weights are one contiguous stream of (128-row panel, 128-k
+// block) units.  Each persistent CTA takes an equal contiguous share of that
+// stream (units [U*c/G, U*(c+1)/G)), so every SM moves the same number of
+// bytes whatever N and K are; a producer warp pulls the share through a
+// STAGES-deep ring of 1-D bulk copies (the TMA engine, no multicast), which
+// keeps tens of KB in flight per SM without registers.  Eight consumer warps
+// own the eight 16-row blocks of a panel: each reads its 512-byte tiles from
+// shared memory -- already m16n8k16 A fragments (wq_layout.h) -- unpacks them
+// in registers and runs mma.sync with the activations as the B operand
+// ("register-level dequantize GEMV with 128-bit loads", tileInfer README,
+// Features table; the 128-bit loads are here the 16-byte shared-memory reads
+// of each lane).  INT4 groups are scaled in fp32 after their 8 MMAs and
+// INT8 rows once at the end, so weights are never rounded.
+//
+// A panel whose k-blocks are split between two or more CTAs is finished by
+// the last contributor to arrive (atomic ticket per panel, never waited on):
+// it sums the fp32 partials of all contributors in CTA order, so the result
+// is deterministic, and it resets the ticket to zero.  Partials live in the
+// split-K workspace: [G CTAs][2 slots (first/last panel of the range)]
+// [128 rows][8*MT tokens].
+#include <cstdint>
+
+#include "wq_device.cuh"
+#include "wq_internal.h"
+
+namespace wq {
+
+static __device__ int g_gemv_sk_error = 0;
+
+struct GemvSkParams {
+    const uint16_t *x;
+    int M, K, N;
+    const uint8_t *wq;
+    const uint16_t *scales;
+    const uint8_t *zeros;
+    uint16_t *y;
+    int KB, U; // k-blocks per panel, units = panels * KB
+    float *part;
+    uint32_t *cnt;
+};
+
+template <int BITS>
+struct SkCfg {
+    static constexpr int kTPB = BITS == 4 ? 2 : 4;   // tiles per 16-row block per unit
+    static constexpr int kRBB = kTPB * kTileBytes;   // bytes of one 16-row block per unit
+    static constexpr int kPBB = 8 * kRBB;            // packed bytes per unit
+    static constexpr int kSZB = BITS == 4 ? 512 : 0; // scales 256 + zeros 64, padded
+    static constexpr int kSZTx = BITS == 4 ? 320 : 0;
+    static constexpr int kStageBytes = kPBB + kSZB;
+    static constexpr int kStages = BITS == 4 ? 8 : 6;
+};
+
+constexpr int kSkConsumers = 8;
+constexpr int kSkThreads = 32 * (1 + kSkConsumers);
+
+template <int MT>
+__device__ __forceinline__ void x_frags(const uint16_t *const (&xr)[MT], int k, uint2 (&xf)[MT])
+{
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+        xf[mt] = xr[mt] ? ldg_keep(xr[mt] + k) : make_uint2(0u, 0u);
+}
+
+// bytes 0..3 of w (int8) -> two bf16x2: {q0, q1}, {q2, q3}; exact.
+__device__ __forceinline__ void s8quad_bf16(uint32_t w, uint32_t &lo, uint32_t &hi)
+{
+    const uint32_t u = w ^ 0x80808080u;
+    const uint32_t f0 = __byte_perm(u, 0x4B000000u, 0x7540u), f1 = __byte_perm(u, 0x4B000000u, 0x7541u);
+    const uint32_t f2 = __byte_perm(u, 0x4B000000u, 0x7542u), f3 = __byte_perm(u, 0x4B000000u, 0x7543u);
+    const uint64_t c = 0x4B0000804B000080ull; // {2^23 + 128, 2^23 + 128}
+    uint64_t d01, d23;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d01) : "l"(((uint64_t)f1 << 32) | f0), "l"(c));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d23) : "l"(((uint64_t)f3 << 32) | f2), "l"(c));
+    // |q| <= 128 has at most 8 significant bits: the fp32 value's upper half is its bf16
+    lo = __byte_perm((uint32_t)d01, (uint32_t)(d01 >> 32), 0x7632u);
+    hi = __byte_perm((uint32_t)d23, (uint32_t)(d23 >> 32), 0x7632u);
+}
+
+template <int MT>
+__device__ __forceinline__ void sk_int8_tile(const uint4 &w, const uint16_t *const (&xr)[MT], int kt, float (&acc)[MT][4])
+{
+    uint32_t a0, a2, a1, a3, b0, b2, b1, b3;
+    s8quad_bf16(w.x, a0, a2); // row g,   k 4t..4t+3
+    s8quad_bf16(w.y, a1, a3); // row g+8
+    s8quad_bf16(w.z, b0, b2); // row g,   k 16+4t..
+    s8quad_bf16(w.w, b1, b3); // row g+8
+    uint2 xa[MT], xb[MT];
+    x_frags<MT>(xr, kt, xa);
+    x_frags<MT>(xr, kt + 16, xb);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        mma_bf16_16816(acc[mt], a0, a1, a2, a3, xa[mt].x, xa[mt].y);
+        mma_bf16_16816(acc[mt], b0, b1, b2, b3, xb[mt].x, xb[mt].y);
+    }
+}
+
+template <int MT>
+__device__ __forceinline__ void sk_int4_tile(const uint4 &w, const uint16_t *const (&xr)[MT], int kt, uint32_t zlo,
+                                             uint32_t zhi, float (&cg)[MT][4])
+{
+    uint32_t xr_[4], yr[4], zr[4], wr[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        xr_[i] = bf16x2_sub(nib_pair_bf16(w.x >> (4 * i)), zlo);
+        yr[i] = bf16x2_sub(nib_pair_bf16(w.y >> (4 * i)), zhi);
+        zr[i] = bf16x2_sub(nib_pair_bf16(w.z >> (4 * i)), zlo);
+        wr[i] = bf16x2_sub(nib_pair_bf16(w.w >> (4 * i)), zhi);
+    }
+    uint2 xa[MT], xb[MT], xc[MT], xd[MT];
+    x_frags<MT>(xr, kt, xa);
+    x_frags<MT>(xr, kt + 16, xb);
+    x_frags<MT>(xr, kt + 32, xc);
+    x_frags<MT>(xr, kt + 48, xd);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        mma_bf16_16816(cg[mt], xr_[0], yr[0], xr_[1], yr[1], xa[mt].x, xa[mt].y);
+        mma_bf16_16816(cg[mt], xr_[2], yr[2], xr_[3], yr[3], xb[mt].x, xb[mt].y);
+        mma_bf16_16816(cg[mt], zr[0], wr[0], zr[1], wr[1], xc[mt].x, xc[mt].y);
+        mma_bf16_16816(cg[mt], zr[2], wr[2], zr[3], wr[3], xd[mt].x, xd[mt].y);
+    }
+}
+
+__device__ __forceinline__ int sk_start(long long U, int G, int c) { return (int)(U * c / G); }
+
+// CTA that owns unit u (ranges [start(c), start(c+1)); empty ranges skipped)
+__device__ __forceinline__ int sk_owner(long long U, int G, int u)
+{
+    int c = (int)(((long long)u * G) / U);
+    if (c >= G)
+        c = G - 1;
+    while (c + 1 < G && sk_start(U, G, c + 1) <= u)
+        ++c;
+    while (c > 0 && sk_start(U, G, c) > u)
+        --c;
+    return c;
+}
+
+template <int BITS, int MT>
+__global__ void __launch_bounds__(kSkThreads) gemv_sk_kernel(const GemvSkParams p)
+{
+    using C = SkCfg<BITS>;
+    constexpr int STAGES = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint64_t *full = reinterpret_cast<uint64_t *>(ring + STAGES * C::kStageBytes);
+    uint64_t *empty = full + STAGES;
+    uint32_t *s_ticket = reinterpret_cast<uint32_t *>(empty + STAGES);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = gridDim.x, c = blockIdx.x;
+    const long long U = p.U;
+    const int u0 = sk_start(U, G, c), u1 = sk_start(U, G, c + 1);
+    const int n = u1 - u0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kSkConsumers);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    bool ok = true;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            for (int i = 0; i < n; ++i) {
+                const int st = i % STAGES, use = i / STAGES;
+                if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const size_t u = (size_t)(u0 + i);
+                uint8_t *dst = ring + st * C::kStageBytes;
+                mbar_arrive_expect_tx(&full[st], C::kPBB + C::kSZTx);
+                bulk_g2s(dst, p.wq + u * C::kPBB, C::kPBB, &full[st], pol);
+                if constexpr (BITS == 4) {
+                    bulk_g2s(dst + C::kPBB, p.scales + u * kPanelRows, 256, &full[st], pol);
+                    bulk_g2s(dst + C::kPBB + 256, p.zeros + u * 64, 64, &full[st], pol);
+                }
+            }
+        }
+    } else {
+        const int j = warp - 1; // 16-row block of the panel
+        const int g = lane >> 2, t = lane & 3;
+        const int KB = p.KB;
+        float acc[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+            acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+        const uint16_t *xr[MT];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int m = 8 * mt + g;
+            xr[mt] = m < p.M ? p.x + (size_t)m * p.K + 4 * t : nullptr;
+        }
+
+        // write this warp's rows of panel pnl: to y if this CTA covered the
+        // whole panel, else as a partial + ticket (last arriver reduces).
+        auto flush = [&](int pnl) {
+            const int lo = max(u0, pnl * KB), hi = min(u1, (pnl + 1) * KB);
+            const int n_lo = pnl * kPanelRows + 16 * j + g, n_hi = n_lo + 8;
+            float s_lo = 1.f, s_hi = 1.f;
+            if constexpr (BITS == 8) {
+                s_lo = n_lo < p.N ? bf16_bits_to_float(p.scales[n_lo]) : 0.f;
+                s_hi = n_hi < p.N ? bf16_bits_to_float(p.scales[n_hi]) : 0.f;
+            }
+            auto store_y = [&](const float (&v)[MT][4]) {
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    const int m0 = 8 * mt + 2 * t;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        if (m0 + e < p.M) {
+                            if (n_lo < p.N)
+                                p.y[(size_t)(m0 + e) * p.N + n_lo] =
+                                    __bfloat16_as_ushort(__float2bfloat16_rn(v[mt][e] * s_lo));
+                            if (n_hi < p.N)
+                                p.y[(size_t)(m0 + e) * p.N + n_hi] =
+                                    __bfloat16_as_ushort(__float2bfloat16_rn(v[mt][2 + e] * s_hi));
+                        }
+                    }
+                }
+            };
+            if (lo == pnl * KB && hi == (pnl + 1) * KB) {
+                store_y(acc);
+                return;
+            }
+            constexpr int TOK = 8 * MT;
+            const int slot = (pnl == u0 / KB) ? 0 : 1;
+            float *mine = p.part + ((size_t)(c * 2 + slot) * kPanelRows) * TOK;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const int m0 = 8 * mt + 2 * t;
+                *reinterpret_cast<float2 *>(mine + (size_t)(16 * j + g) * TOK + m0) = make_float2(acc[mt][0], acc[mt][1]);
+                *reinterpret_cast<float2 *>(mine + (size_t)(16 * j + g + 8) * TOK + m0) =
+                    make_float2(acc[mt][2], acc[mt][3]);
+            }
+            __threadfence();
+            named_barrier_sync(1, 32 * kSkConsumers);
+            if (warp == 1 && lane == 0)
+                *s_ticket = atomicAdd(&p.cnt[pnl], 1u);
+            named_barrier_sync(1, 32 * kSkConsumers);
+            const int cf = sk_owner(U, G, pnl * KB), cl = sk_owner(U, G, (pnl + 1) * KB - 1);
+            const uint32_t ticket = *s_ticket;
+            named_barrier_sync(1, 32 * kSkConsumers); // ticket slot may be reused by the next flush
+            if (ticket == (uint32_t)(cl - cf)) {
+                __threadfence();
+                float tot[MT][4];
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+                    tot[mt][0] = tot[mt][1] = tot[mt][2] = tot[mt][3] = 0.f;
+                for (int cc = cf; cc <= cl; ++cc) {
+                    const int sl = (pnl == sk_start(U, G, cc) / KB) ? 0 : 1;
+                    const float *src = p.part + ((size_t)(cc * 2 + sl) * kPanelRows) * TOK;
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const int m0 = 8 * mt + 2 * t;
+                        const float2 a = __ldcg(reinterpret_cast<const float2 *>(src + (size_t)(16 * j + g) * TOK + m0));
+                        const float2 b =
+                            __ldcg(reinterpret_cast<const float2 *>(src + (size_t)(16 * j + g + 8) * TOK + m0));
+                        tot[mt][0] += a.x;
+                        tot[mt][1] += a.y;
+                        tot[mt][2] += b.x;
+                        tot[mt][3] += b.y;
+                    }
+                }
+                store_y(tot);
+                if (warp == 1 && lane == 0)
+                    atomicExch(&p.cnt[pnl], 0u);
+            }
+        };
+
+        int cur = n > 0 ? u0 / KB : -1;
+        for (int i = 0; i < n; ++i) {
+            const int u = u0 + i, pnl = u / KB, kb = u - pnl * KB;
+            if (pnl != cur) {
+                flush(cur);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+                    acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+                cur = pnl;
+            }
+            const int st = i % STAGES, use = i / STAGES;
+            if (ok && !mbar_wait(&full[st], use & 1))
+                ok = false;
+            const uint8_t *stage = ring + st * C::kStageBytes;
+            uint4 w[C::kTPB];
+#pragma unroll
+            for (int tt = 0; tt < C::kTPB; ++tt)
+                w[tt] = *reinterpret_cast<const uint4 *>(stage + j * C::kRBB + tt * kTileBytes + lane * 16);
+            uint32_t zlo = 0, zhi = 0;
+            float slo = 0.f, shi = 0.f;
+            if constexpr (BITS == 4) {
+                const uint16_t *s16 = reinterpret_cast<const uint16_t *>(stage + C::kPBB);
+                const uint8_t *z8 = stage + C::kPBB + 256;
+                const int r = 16 * j + g;
+                const uint32_t zl = (z8[r >> 1] >> (4 * (r & 1))) & 0xFu;
+                const uint32_t zh = (z8[(r + 8) >> 1] >> (4 * (r & 1))) & 0xFu;
+                zlo = 0x43004300u | zl | (zl << 16);
+                zhi = 0x43004300u | zh | (zh << 16);
+                slo = bf16_bits_to_float(s16[r]);
+                shi = bf16_bits_to_float(s16[r + 8]);
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&empty[st]);
+            if (!ok)
+                continue;
+            const int kbase = kb * kBlockK;
+            if constexpr (BITS == 8) {
+#pragma unroll
+                for (int tt = 0; tt < 4; ++tt)
+                    if (kbase + 32 * tt < p.K)
+                        sk_int8_tile<MT>(w[tt], xr, kbase + 32 * tt, acc);
+            } else {
+                float cg[MT][4];
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+                    cg[mt][0] = cg[mt][1] = cg[mt][2] = cg[mt][3] = 0.f;
+                sk_int4_tile<MT>(w[0], xr, kbase, zlo, zhi, cg);
+                sk_int4_tile<MT>(w[1], xr, kbase + 64, zlo, zhi, cg);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    acc[mt][0] = fmaf(slo, cg[mt][0], acc[mt][0]);
+                    acc[mt][1] = fmaf(slo, cg[mt][1], acc[mt][1]);
+                    acc[mt][2] = fmaf(shi, cg[mt][2], acc[mt][2]);
+                    acc[mt][3] = fmaf(shi, cg[mt][3], acc[mt][3]);
+                }
+            }
+        }
+        if (cur >= 0)
+            flush(cur);
+    }
+    if (!ok)
+        atomicExch(&g_gemv_sk_error, kErrTimeout);
+}
+
+template <int BITS, int MT>
+static cudaError_t launch_sk_t(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st)
+{
+    using C = SkCfg<BITS>;
+    constexpr size_t smem = 128 + (size_t)C::kStages * C::kStageBytes + 2 * C::kStages * 8 + 16;
+    static int occ = -1;
+    if (occ < 0) {
+        cudaError_t e = cudaFuncSetAttribute(gemv_sk_kernel<BITS, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess)
+            return e;
+        int o = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, gemv_sk_kernel<BITS, MT>, kSkThreads, smem);
+        if (e != cudaSuccess)
+            return e;
+        occ = o > 0 ? o : 1;
+    }
+    const int per_sm = (ctas_per_sm > 0 && ctas_per_sm < occ) ? ctas_per_sm : occ;
+    const Shape sh{a.bits, a.K, a.N, a.group};
+    GemvSkParams p;
+    p.x = a.x;
+    p.M = a.M;
+    p.K = a.K;
+    p.N = a.N;
+    p.wq = (const uint8_t *)a.wq;
+    p.scales = (const uint16_t *)a.scales;
+    p.zeros = (const uint8_t *)a.zeros;
+    p.y = a.y;
+    p.KB = sh.kblocks();
+    p.U = sh.panels() * sh.kblocks();
+    p.cnt = (uint32_t *)ws;
+    p.part = (float *)((uint8_t *)ws + ws_counter_bytes(a.N));
+    int G = per_sm * sm_count;
+    if (G > kSkMaxCtas)
+        G = kSkMaxCtas;
+    if (G > p.U)
+        G = p.U;
+    gemv_sk_kernel<BITS, MT><<<G, kSkThreads, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemv_sk(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st)
+{
+    const int mt = (a.M + 7) / 8;
+    if (a.bits == 8) {
+        if (mt == 1) return launch_sk_t<8, 1>(a, ctas_per_sm, ws, sm_count, st);
+        if (mt == 2) return launch_sk_t<8, 2>(a, ctas_per_sm, ws, sm_count, st);
+        return launch_sk_t<8, 4>(a, ctas_per_sm, ws, sm_count, st);
+    }
+    if (mt == 1) return launch_sk_t<4, 1>(a, ctas_per_sm, ws, sm_count, st);
+    if (mt == 2) return launch_sk_t<4, 2>(a, ctas_per_sm, ws, sm_count, st);
+    return launch_sk_t<4, 4>(a, ctas_per_sm, ws, sm_count, st);
+}
+
+cudaError_t read_gemv_sk_error(int *code, cudaStream_t st)
+{
+    int host = 0, zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&host, g_gemv_sk_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess)
+        return e;
+    e = cudaMemcpyToSymbolAsync(g_gemv_sk_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess)
+        return e;
+    e = cudaStreamSynchronize(st);
+    *code = host;
+    return e;
+}
+
+} // namespace wq

@@ -17,11 +17,19 @@ struct LinearArgs {
     uint16_t *y;
 };
 
-// split-K workspace: [ticket counters, 256-byte padded][fp32 partials S*M*N]
+// Split-K workspace: [ticket counters, 256-byte padded][fp32 partials].
+// GEMM with S splits: partials [S][M][N].  Stream-K GEMV: partials
+// [CTAs <= kSkMaxCtas][2][128 rows][8 * ceil(M/8) tokens].
+constexpr int kSkMaxCtas = 512;
 inline size_t ws_counter_bytes(int N) { return (((size_t)((N + 127) / 128) * 4) + 255) / 256 * 256; }
 inline size_t ws_bytes(int M, int N, int S)
 {
     return ws_counter_bytes(N) + (S > 1 ? (size_t)S * M * N * sizeof(float) : 0);
+}
+inline size_t ws_bytes_gemv_sk(int M, int N)
+{
+    const int tok = 8 * ((M + 7) / 8);
+    return ws_counter_bytes(N) + (size_t)kSkMaxCtas * 2 * 128 * tok * sizeof(float);
 }
 
 cudaError_t launch_quantize_int8(const float *W, int K, int N, int8_t *q, uint16_t *s, cudaStream_t st);
@@ -38,6 +46,10 @@ cudaError_t launch_dequant_debug(const void *wq, const void *scales, const void 
 
 // GEMV: ks = K slices per 16-row block (1, 2, 4, 8); M <= 32.
 cudaError_t launch_gemv(const LinearArgs &a, int ks, int sm_count, cudaStream_t st);
+
+// Stream-K GEMV: ctas_per_sm = 0 (occupancy) or 1/2; ws >= ws_bytes_gemv_sk.
+cudaError_t launch_gemv_sk(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st);
+cudaError_t read_gemv_sk_error(int *code, cudaStream_t st);
 
 // GEMM: split = K splits (1..32); ws holds counters + partials when split > 1.
 cudaError_t launch_gemm(const LinearArgs &a, int split, void *ws, int sm_count, cudaStream_t st);

@@ -243,8 +243,11 @@ def build_weights(name, device, copies):
     return cfg, pws
 
 
+KERNELS = {0: ("gemv_sk", "wq_gemv_sk.cu"), 1: ("gemm", "wq_gemm.cu"), 2: ("gemv_rb", "wq_gemv.cu")}
+
+
 def kernel_name(variant, bits):
-    return ("gemv" if variant == 0 else "gemm") + f"_w{bits}"
+    return KERNELS[variant][0] + f"_w{bits}"
 
 
 def bench_ours(args, device, rank, world):
@@ -358,7 +361,7 @@ def bench_ours(args, device, rank, world):
     Mdom = max(Ms, key=lambda m: share[m])
     dom = next(p for p in per_shape if p["M"] == Mdom)
     vdom = choices[Mdom][0]
-    kfile = "wq_gemv.cu" if vdom == 0 else "wq_gemm.cu"
+    kfile = KERNELS[vdom][1]
     summary = f"{dom['variant']}_{name}_M{Mdom}.md"
     traffic = profile_traffic(kfile, summary)
     bound = "hbm"

@@ -277,9 +277,24 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Barrier over a subset of the CTA's warps.  The non-aligned form, after a
+// __syncwarp, so that a branch taken by one lane just before it (the ticket
+// atomic) cannot leave the warp diverged at an aligned barrier.
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads)
 {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+    __syncwarp();
+    asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Ticket for "last CTA to arrive finishes the reduction": a release fence
+// (covering the partials this CTA's threads stored before the barrier) and
+// an acquire fence after the atomic.
+__device__ __forceinline__ uint32_t ticket_take(uint32_t *counter)
+{
+    __threadfence();
+    const uint32_t t = atomicAdd(counter, 1u);
+    __threadfence();
+    return t;
 }
 
 // ---------------------------------------------------------------------------

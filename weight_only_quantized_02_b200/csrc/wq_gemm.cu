@@ -151,7 +151,7 @@ __device__ __forceinline__ void gemm_store(const GemmParams &p, int panel, int s
     __threadfence();
     named_barrier_sync(1, 128);
     if (warp == 2 && lane == 0)
-        *s_ticket = atomicAdd(&p.cnt[panel], 1u);
+        *s_ticket = ticket_take(&p.cnt[panel]);
     named_barrier_sync(1, 128);
     if (*s_ticket == (uint32_t)(p.S - 1)) {
         __threadfence();

@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(kSkThreads) gemv_sk_kernel(const GemvSkParams 
             __threadfence();
             named_barrier_sync(1, 32 * kSkConsumers);
             if (warp == 1 && lane == 0)
-                *s_ticket = atomicAdd(&p.cnt[pnl], 1u);
+                *s_ticket = ticket_take(&p.cnt[pnl]);
             named_barrier_sync(1, 32 * kSkConsumers);
             const int cf = sk_owner(U, G, pnl * KB), cl = sk_owner(U, G, (pnl + 1) * KB - 1);
             const uint32_t ticket = *s_ticket;

@@ -41,26 +41,34 @@ struct GemvSkParams {
     uint32_t *cnt;
 };
 
-template <int BITS>
+// Ring stage: packed weights of the unit, INT4 scales/zeros, and the unit's
+// activation slice x[0..M)[128 k] (one 256-byte bulk copy per token row,
+// rows 288 bytes apart so the eight rows a warp reads hit distinct banks).
+template <int BITS, int MT>
 struct SkCfg {
     static constexpr int kTPB = BITS == 4 ? 2 : 4;   // tiles per 16-row block per unit
     static constexpr int kRBB = kTPB * kTileBytes;   // bytes of one 16-row block per unit
     static constexpr int kPBB = 8 * kRBB;            // packed bytes per unit
     static constexpr int kSZB = BITS == 4 ? 512 : 0; // scales 256 + zeros 64, padded
     static constexpr int kSZTx = BITS == 4 ? 320 : 0;
-    static constexpr int kStageBytes = kPBB + kSZB;
-    static constexpr int kStages = BITS == 4 ? 8 : 6;
+    static constexpr int kXRow = 288;                // smem stride of one token row (256 B + pad)
+    static constexpr int kXB = 8 * MT * kXRow;
+    static constexpr int kStageBytes = kPBB + kSZB + kXB;
+    static constexpr int kStages = (110 * 1024) / kStageBytes > 8 ? 8 : (110 * 1024) / kStageBytes;
 };
 
 constexpr int kSkConsumers = 8;
 constexpr int kSkThreads = 32 * (1 + kSkConsumers);
 
-template <int MT>
-__device__ __forceinline__ void x_frags(const uint16_t *const (&xr)[MT], int k, uint2 (&xf)[MT])
+// B fragments of mma.m16n8k16 from the staged activation slice: lane
+// (g, t) takes x[8*mt + g][k .. k+4) (k relative to the unit's 128-k block);
+// xs already points at row g, column 4t of the stage's x area.
+template <int MT, int XROW>
+__device__ __forceinline__ void x_frags(const uint8_t *xs, int k, uint2 (&xf)[MT])
 {
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
-        xf[mt] = xr[mt] ? ldg_keep(xr[mt] + k) : make_uint2(0u, 0u);
+        xf[mt] = *reinterpret_cast<const uint2 *>(xs + mt * 8 * XROW + 2 * k);
 }
 
 // bytes 0..3 of w (int8) -> two bf16x2: {q0, q1}, {q2, q3}; exact.
@@ -78,8 +86,8 @@ __device__ __forceinline__ void s8quad_bf16(uint32_t w, uint32_t &lo, uint32_t &
     hi = __byte_perm((uint32_t)d23, (uint32_t)(d23 >> 32), 0x7632u);
 }
 
-template <int MT>
-__device__ __forceinline__ void sk_int8_tile(const uint4 &w, const uint16_t *const (&xr)[MT], int kt, float (&acc)[MT][4])
+template <int MT, int XROW>
+__device__ __forceinline__ void sk_int8_tile(const uint4 &w, const uint8_t *xs, int kt, float (&acc)[MT][4])
 {
     uint32_t a0, a2, a1, a3, b0, b2, b1, b3;
     s8quad_bf16(w.x, a0, a2); // row g,   k 4t..4t+3
@@ -87,8 +95,8 @@ __device__ __forceinline__ void sk_int8_tile(const uint4 &w, const uint16_t *con
     s8quad_bf16(w.z, b0, b2); // row g,   k 16+4t..
     s8quad_bf16(w.w, b1, b3); // row g+8
     uint2 xa[MT], xb[MT];
-    x_frags<MT>(xr, kt, xa);
-    x_frags<MT>(xr, kt + 16, xb);
+    x_frags<MT, XROW>(xs, kt, xa);
+    x_frags<MT, XROW>(xs, kt + 16, xb);
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
         mma_bf16_16816(acc[mt], a0, a1, a2, a3, xa[mt].x, xa[mt].y);
@@ -96,9 +104,9 @@ __device__ __forceinline__ void sk_int8_tile(const uint4 &w, const uint16_t *con
     }
 }
 
-template <int MT>
-__device__ __forceinline__ void sk_int4_tile(const uint4 &w, const uint16_t *const (&xr)[MT], int kt, uint32_t zlo,
-                                             uint32_t zhi, float (&cg)[MT][4])
+template <int MT, int XROW>
+__device__ __forceinline__ void sk_int4_tile(const uint4 &w, const uint8_t *xs, int kt, uint32_t zlo, uint32_t zhi,
+                                             float (&cg)[MT][4])
 {
     uint32_t xr_[4], yr[4], zr[4], wr[4];
 #pragma unroll
@@ -109,10 +117,10 @@ __device__ __forceinline__ void sk_int4_tile(const uint4 &w, const uint16_t *con
         wr[i] = bf16x2_sub(nib_pair_bf16(w.w >> (4 * i)), zhi);
     }
     uint2 xa[MT], xb[MT], xc[MT], xd[MT];
-    x_frags<MT>(xr, kt, xa);
-    x_frags<MT>(xr, kt + 16, xb);
-    x_frags<MT>(xr, kt + 32, xc);
-    x_frags<MT>(xr, kt + 48, xd);
+    x_frags<MT, XROW>(xs, kt, xa);
+    x_frags<MT, XROW>(xs, kt + 16, xb);
+    x_frags<MT, XROW>(xs, kt + 32, xc);
+    x_frags<MT, XROW>(xs, kt + 48, xd);
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
         mma_bf16_16816(cg[mt], xr_[0], yr[0], xr_[1], yr[1], xa[mt].x, xa[mt].y);
@@ -140,7 +148,7 @@ __device__ __forceinline__ int sk_owner(long long U, int G, int u)
 template <int BITS, int MT>
 __global__ void __launch_bounds__(kSkThreads) gemv_sk_kernel(const GemvSkParams p)
 {
-    using C = SkCfg<BITS>;
+    using C = SkCfg<BITS, MT>;
     constexpr int STAGES = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -161,12 +169,23 @@ __global__ void __launch_bounds__(kSkThreads) gemv_sk_kernel(const GemvSkParams 
         }
         fence_mbar_init();
     }
+    // token rows M..8*MT of every stage's x area stay zero (the B operand's padding)
+    {
+        const int pad_rows = 8 * MT - p.M;
+        const int words = pad_rows * (C::kXRow / 4);
+        for (int s = 0; s < STAGES; ++s) {
+            uint32_t *xz = reinterpret_cast<uint32_t *>(ring + s * C::kStageBytes + C::kPBB + C::kSZB + p.M * C::kXRow);
+            for (int i = threadIdx.x; i < words; i += blockDim.x)
+                xz[i] = 0u;
+        }
+    }
+    fence_proxy_async_smem();
     __syncthreads();
     bool ok = true;
 
     if (warp == 0) {
         if (lane == 0) {
-            const uint64_t pol = policy_evict_first();
+            const uint64_t pol = policy_evict_first(), pol_x = policy_evict_last();
             for (int i = 0; i < n; ++i) {
                 const int st = i % STAGES, use = i / STAGES;
                 if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1)) {
@@ -174,13 +193,19 @@ __global__ void __launch_bounds__(kSkThreads) gemv_sk_kernel(const GemvSkParams 
                     break;
                 }
                 const size_t u = (size_t)(u0 + i);
+                const int kb = (int)(u % p.KB);
+                // activation bytes of this k-block (the last block of a ragged K is short)
+                const int xbytes = min(2 * kBlockK, 2 * (p.K - kb * kBlockK));
                 uint8_t *dst = ring + st * C::kStageBytes;
-                mbar_arrive_expect_tx(&full[st], C::kPBB + C::kSZTx);
+                mbar_arrive_expect_tx(&full[st], C::kPBB + C::kSZTx + p.M * xbytes);
                 bulk_g2s(dst, p.wq + u * C::kPBB, C::kPBB, &full[st], pol);
                 if constexpr (BITS == 4) {
                     bulk_g2s(dst + C::kPBB, p.scales + u * kPanelRows, 256, &full[st], pol);
                     bulk_g2s(dst + C::kPBB + 256, p.zeros + u * 64, 64, &full[st], pol);
                 }
+                for (int m = 0; m < p.M; ++m)
+                    bulk_g2s(dst + C::kPBB + C::kSZB + m * C::kXRow, p.x + (size_t)m * p.K + (size_t)kb * kBlockK,
+                             xbytes, &full[st], pol_x);
             }
         }
     } else {
@@ -191,12 +216,7 @@ __global__ void __launch_bounds__(kSkThreads) gemv_sk_kernel(const GemvSkParams 
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
             acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-        const uint16_t *xr[MT];
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            const int m = 8 * mt + g;
-            xr[mt] = m < p.M ? p.x + (size_t)m * p.K + 4 * t : nullptr;
-        }
+        const int xoff = C::kPBB + C::kSZB + g * C::kXRow + 8 * t; // row g, column 4t
 
         // write this warp's rows of panel pnl: to y if this CTA covered the
         // whole panel, else as a partial + ticket (last arriver reduces).
@@ -288,49 +308,47 @@ __global__ void __launch_bounds__(kSkThreads) gemv_sk_kernel(const GemvSkParams 
             if (ok && !mbar_wait(&full[st], use & 1))
                 ok = false;
             const uint8_t *stage = ring + st * C::kStageBytes;
-            uint4 w[C::kTPB];
+            if (ok) {
+                uint4 w[C::kTPB];
 #pragma unroll
-            for (int tt = 0; tt < C::kTPB; ++tt)
-                w[tt] = *reinterpret_cast<const uint4 *>(stage + j * C::kRBB + tt * kTileBytes + lane * 16);
-            uint32_t zlo = 0, zhi = 0;
-            float slo = 0.f, shi = 0.f;
-            if constexpr (BITS == 4) {
-                const uint16_t *s16 = reinterpret_cast<const uint16_t *>(stage + C::kPBB);
-                const uint8_t *z8 = stage + C::kPBB + 256;
-                const int r = 16 * j + g;
-                const uint32_t zl = (z8[r >> 1] >> (4 * (r & 1))) & 0xFu;
-                const uint32_t zh = (z8[(r + 8) >> 1] >> (4 * (r & 1))) & 0xFu;
-                zlo = 0x43004300u | zl | (zl << 16);
-                zhi = 0x43004300u | zh | (zh << 16);
-                slo = bf16_bits_to_float(s16[r]);
-                shi = bf16_bits_to_float(s16[r + 8]);
+                for (int tt = 0; tt < C::kTPB; ++tt)
+                    w[tt] = *reinterpret_cast<const uint4 *>(stage + j * C::kRBB + tt * kTileBytes + lane * 16);
+                const uint8_t *xs = stage + xoff;
+                if constexpr (BITS == 8) {
+                    const int kbase = kb * kBlockK;
+#pragma unroll
+                    for (int tt = 0; tt < 4; ++tt)
+                        if (kbase + 32 * tt < p.K)
+                            sk_int8_tile<MT, C::kXRow>(w[tt], xs, 32 * tt, acc);
+                } else {
+                    const uint16_t *s16 = reinterpret_cast<const uint16_t *>(stage + C::kPBB);
+                    const uint8_t *z8 = stage + C::kPBB + 256;
+                    const int r = 16 * j + g;
+                    const uint32_t zl = (z8[r >> 1] >> (4 * (r & 1))) & 0xFu;
+                    const uint32_t zh = (z8[(r + 8) >> 1] >> (4 * (r & 1))) & 0xFu;
+                    const uint32_t zlo = 0x43004300u | zl | (zl << 16);
+                    const uint32_t zhi = 0x43004300u | zh | (zh << 16);
+                    const float slo = bf16_bits_to_float(s16[r]);
+                    const float shi = bf16_bits_to_float(s16[r + 8]);
+                    float cg[MT][4];
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+                        cg[mt][0] = cg[mt][1] = cg[mt][2] = cg[mt][3] = 0.f;
+                    sk_int4_tile<MT, C::kXRow>(w[0], xs, 0, zlo, zhi, cg);
+                    sk_int4_tile<MT, C::kXRow>(w[1], xs, 64, zlo, zhi, cg);
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        acc[mt][0] = fmaf(slo, cg[mt][0], acc[mt][0]);
+                        acc[mt][1] = fmaf(slo, cg[mt][1], acc[mt][1]);
+                        acc[mt][2] = fmaf(shi, cg[mt][2], acc[mt][2]);
+                        acc[mt][3] = fmaf(shi, cg[mt][3], acc[mt][3]);
+                    }
+                }
             }
+            // every read of this stage (weights, scales, activations) is done
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&empty[st]);
-            if (!ok)
-                continue;
-            const int kbase = kb * kBlockK;
-            if constexpr (BITS == 8) {
-#pragma unroll
-                for (int tt = 0; tt < 4; ++tt)
-                    if (kbase + 32 * tt < p.K)
-                        sk_int8_tile<MT>(w[tt], xr, kbase + 32 * tt, acc);
-            } else {
-                float cg[MT][4];
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
-                    cg[mt][0] = cg[mt][1] = cg[mt][2] = cg[mt][3] = 0.f;
-                sk_int4_tile<MT>(w[0], xr, kbase, zlo, zhi, cg);
-                sk_int4_tile<MT>(w[1], xr, kbase + 64, zlo, zhi, cg);
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    acc[mt][0] = fmaf(slo, cg[mt][0], acc[mt][0]);
-                    acc[mt][1] = fmaf(slo, cg[mt][1], acc[mt][1]);
-                    acc[mt][2] = fmaf(shi, cg[mt][2], acc[mt][2]);
-                    acc[mt][3] = fmaf(shi, cg[mt][3], acc[mt][3]);
-                }
-            }
         }
         if (cur >= 0)
             flush(cur);
@@ -342,7 +360,7 @@ __global__ void __launch_bounds__(kSkThreads) gemv_sk_kernel(const GemvSkParams 
 template <int BITS, int MT>
 static cudaError_t launch_sk_t(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st)
 {
-    using C = SkCfg<BITS>;
+    using C = SkCfg<BITS, MT>;
     constexpr size_t smem = 128 + (size_t)C::kStages * C::kStageBytes + 2 * C::kStages * 8 + 16;
     static int occ = -1;
     if (occ < 0) {

@@ -133,6 +133,16 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch (the kernel is launched with the
+// programmatic-stream-serialization attribute).  wait: block until the
+// preceding kernel in the stream has completed and its writes are visible;
+// a no-op without such a predecessor.  launch_dependents: allow the next
+// kernel to begin launching once every CTA of this grid has signalled.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // Global loads
 // ---------------------------------------------------------------------------
 // Streaming 128-bit load: read once, keep out of L1.

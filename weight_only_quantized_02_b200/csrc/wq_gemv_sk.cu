@@ -54,7 +54,9 @@ struct SkCfg {
     static constexpr int kXRow = 288;                // smem stride of one token row (256 B + pad)
     static constexpr int kXB = 8 * MT * kXRow;
     static constexpr int kStageBytes = kPBB + kSZB + kXB;
-    static constexpr int kStages = (110 * 1024) / kStageBytes > 8 ? 8 : (110 * 1024) / kStageBytes;
+    // about 72 KB of ring per CTA, so three CTAs (27 warps) fit on an SM
+    static constexpr int kStagesRaw = (72 * 1024) / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 8 ? 8 : (kStagesRaw < 2 ? 2 : kStagesRaw);
 };
 
 constexpr int kSkConsumers = 8;
@@ -146,7 +148,7 @@ __device__ __forceinline__ int sk_owner(long long U, int G, int u)
 }
 
 template <int BITS, int MT>
-__global__ void __launch_bounds__(kSkThreads) gemv_sk_kernel(const GemvSkParams p)
+__global__ void __launch_bounds__(kSkThreads, MT == 4 ? 2 : 3) gemv_sk_kernel(const GemvSkParams p)
 {
     using C = SkCfg<BITS, MT>;
     constexpr int STAGES = C::kStages;
@@ -186,29 +188,47 @@ __global__ void __launch_bounds__(kSkThreads) gemv_sk_kernel(const GemvSkParams 
     if (warp == 0) {
         if (lane == 0) {
             const uint64_t pol = policy_evict_first(), pol_x = policy_evict_last();
-            for (int i = 0; i < n; ++i) {
-                const int st = i % STAGES, use = i / STAGES;
-                if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
+            auto xbytes_of = [&](int kb) { return min(2 * kBlockK, 2 * (p.K - kb * kBlockK)); };
+            auto issue_weights = [&](int i, int st) {
                 const size_t u = (size_t)(u0 + i);
-                const int kb = (int)(u % p.KB);
-                // activation bytes of this k-block (the last block of a ragged K is short)
-                const int xbytes = min(2 * kBlockK, 2 * (p.K - kb * kBlockK));
                 uint8_t *dst = ring + st * C::kStageBytes;
-                mbar_arrive_expect_tx(&full[st], C::kPBB + C::kSZTx + p.M * xbytes);
+                mbar_arrive_expect_tx(&full[st], C::kPBB + C::kSZTx + p.M * xbytes_of((int)(u % p.KB)));
                 bulk_g2s(dst, p.wq + u * C::kPBB, C::kPBB, &full[st], pol);
                 if constexpr (BITS == 4) {
                     bulk_g2s(dst + C::kPBB, p.scales + u * kPanelRows, 256, &full[st], pol);
                     bulk_g2s(dst + C::kPBB + 256, p.zeros + u * 64, 64, &full[st], pol);
                 }
+            };
+            auto issue_x = [&](int i, int st) {
+                const int kb = (u0 + i) % p.KB;
+                uint8_t *dst = ring + st * C::kStageBytes + C::kPBB + C::kSZB;
                 for (int m = 0; m < p.M; ++m)
-                    bulk_g2s(dst + C::kPBB + C::kSZB + m * C::kXRow, p.x + (size_t)m * p.K + (size_t)kb * kBlockK,
-                             xbytes, &full[st], pol_x);
+                    bulk_g2s(dst + m * C::kXRow, p.x + (size_t)m * p.K + (size_t)kb * kBlockK, xbytes_of(kb),
+                             &full[st], pol_x);
+            };
+            // weights do not depend on the preceding kernel: start streaming them
+            // before waiting for it; activations only after
+            const int pre = n < STAGES ? n : STAGES;
+            for (int i = 0; i < pre; ++i)
+                issue_weights(i, i);
+            pdl_wait();
+            for (int i = 0; i < pre; ++i)
+                issue_x(i, i);
+            for (int i = pre; i < n; ++i) {
+                const int st = i % STAGES, use = i / STAGES;
+                if (!mbar_wait(&empty[st], (use - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                issue_weights(i, st);
+                issue_x(i, st);
             }
+        } else {
+            pdl_wait();
         }
+        pdl_launch_dependents();
     } else {
+        pdl_wait(); // the workspace and y may still be in use by the preceding kernel
         const int j = warp - 1; // 16-row block of the panel
         const int g = lane >> 2, t = lane & 3;
         const int KB = p.KB;
@@ -315,11 +335,17 @@ __global__ void __launch_bounds__(kSkThreads) gemv_sk_kernel(const GemvSkParams 
                     w[tt] = *reinterpret_cast<const uint4 *>(stage + j * C::kRBB + tt * kTileBytes + lane * 16);
                 const uint8_t *xs = stage + xoff;
                 if constexpr (BITS == 8) {
-                    const int kbase = kb * kBlockK;
+                    const int kleft = p.K - kb * kBlockK;
+                    if (kleft >= kBlockK) {
 #pragma unroll
-                    for (int tt = 0; tt < 4; ++tt)
-                        if (kbase + 32 * tt < p.K)
+                        for (int tt = 0; tt < 4; ++tt)
                             sk_int8_tile<MT, C::kXRow>(w[tt], xs, 32 * tt, acc);
+                    } else { // ragged last block of K
+#pragma unroll
+                        for (int tt = 0; tt < 4; ++tt)
+                            if (32 * tt < kleft)
+                                sk_int8_tile<MT, C::kXRow>(w[tt], xs, 32 * tt, acc);
+                    }
                 } else {
                     const uint16_t *s16 = reinterpret_cast<const uint16_t *>(stage + C::kPBB);
                     const uint8_t *z8 = stage + C::kPBB + 256;
@@ -350,6 +376,7 @@ __global__ void __launch_bounds__(kSkThreads) gemv_sk_kernel(const GemvSkParams 
             if (lane == 0)
                 mbar_arrive(&empty[st]);
         }
+        pdl_launch_dependents();
         if (cur >= 0)
             flush(cur);
     }
@@ -394,8 +421,17 @@ static cudaError_t launch_sk_t(const LinearArgs &a, int ctas_per_sm, void *ws, i
         G = kSkMaxCtas;
     if (G > p.U)
         G = p.U;
-    gemv_sk_kernel<BITS, MT><<<G, kSkThreads, smem, st>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(kSkThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemv_sk_kernel<BITS, MT>, p);
 }
 
 cudaError_t launch_gemv_sk(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st)

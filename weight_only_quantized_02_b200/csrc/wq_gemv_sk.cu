@@ -14,12 +14,12 @@
 // of each lane).  INT4 groups are scaled in fp32 after their 8 MMAs and
 // INT8 rows once at the end, so weights are never rounded.
 //
-// A panel whose k-blocks are split between two or more CTAs is finished by
-// the last contributor to arrive (atomic ticket per panel, never waited on):
-// it sums the fp32 partials of all contributors in CTA order, so the result
-// is deterministic, and it resets the ticket to zero.  Partials live in the
-// split-K workspace: [G CTAs][2 slots (first/last panel of the range)]
-// [128 rows][8*MT tokens].
+// A panel whose k-blocks are split between two or more CTAs is finished,
+// 16 rows at a time, by the last warp to arrive for those rows (atomic
+// ticket per (panel, 16-row block), never waited on): it sums the fp32
+// partials of all contributors in CTA order, so the result is deterministic,
+// and resets the ticket to zero.  Partials live in the workspace:
+// [G CTAs][2 slots (first/last panel of the range)][128 rows][8*MT tokens].
 #include <cstdint>
 
 #include "wq_device.cuh"
@@ -279,39 +279,56 @@ __global__ void __launch_bounds__(kSkThreads, MT == 4 ? 2 : 3) gemv_sk_kernel(co
                 *reinterpret_cast<float2 *>(mine + (size_t)(16 * j + g + 8) * TOK + m0) =
                     make_float2(acc[mt][2], acc[mt][3]);
             }
+            // Each warp takes its own ticket for its 16 rows of the panel, so the
+            // fix-up never stalls the CTA's other warps.
             __threadfence();
-            named_barrier_sync(1, 32 * kSkConsumers);
-            if (warp == 1 && lane == 0)
-                *s_ticket = ticket_take(&p.cnt[pnl]);
-            named_barrier_sync(1, 32 * kSkConsumers);
+            __syncwarp();
+            uint32_t ticket = 0;
+            if (lane == 0)
+                ticket = ticket_take(&p.cnt[pnl * 8 + j]);
+            ticket = __shfl_sync(0xffffffffu, ticket, 0);
             const int cf = sk_owner(U, G, pnl * KB), cl = sk_owner(U, G, (pnl + 1) * KB - 1);
-            const uint32_t ticket = *s_ticket;
-            named_barrier_sync(1, 32 * kSkConsumers); // ticket slot may be reused by the next flush
-            if (ticket == (uint32_t)(cl - cf)) {
-                __threadfence();
-                float tot[MT][4];
+            if (ticket != (uint32_t)(cl - cf))
+                return;
+            __threadfence();
+            float tot[MT][4];
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
-                    tot[mt][0] = tot[mt][1] = tot[mt][2] = tot[mt][3] = 0.f;
-                for (int cc = cf; cc <= cl; ++cc) {
-                    const int sl = (pnl == sk_start(U, G, cc) / KB) ? 0 : 1;
-                    const float *src = p.part + ((size_t)(cc * 2 + sl) * kPanelRows) * TOK;
+            for (int mt = 0; mt < MT; ++mt)
+                tot[mt][0] = tot[mt][1] = tot[mt][2] = tot[mt][3] = 0.f;
+            // contributors in CTA order, QC at a time with their loads in flight together
+            constexpr int QC = MT == 1 ? 4 : (MT == 2 ? 2 : 1);
+            for (int c0 = cf; c0 <= cl; c0 += QC) {
+                float2 a[QC][MT], b[QC][MT];
 #pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        const int m0 = 8 * mt + 2 * t;
-                        const float2 a = __ldcg(reinterpret_cast<const float2 *>(src + (size_t)(16 * j + g) * TOK + m0));
-                        const float2 b =
-                            __ldcg(reinterpret_cast<const float2 *>(src + (size_t)(16 * j + g + 8) * TOK + m0));
-                        tot[mt][0] += a.x;
-                        tot[mt][1] += a.y;
-                        tot[mt][2] += b.x;
-                        tot[mt][3] += b.y;
+                for (int q = 0; q < QC; ++q) {
+                    const int cc = c0 + q;
+                    if (cc <= cl) {
+                        const int sl = (pnl == sk_start(U, G, cc) / KB) ? 0 : 1;
+                        const float *src = p.part + ((size_t)(cc * 2 + sl) * kPanelRows) * TOK;
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            const int m0 = 8 * mt + 2 * t;
+                            a[q][mt] = __ldcg(reinterpret_cast<const float2 *>(src + (size_t)(16 * j + g) * TOK + m0));
+                            b[q][mt] = __ldcg(reinterpret_cast<const float2 *>(src + (size_t)(16 * j + g + 8) * TOK + m0));
+                        }
                     }
                 }
-                store_y(tot);
-                if (warp == 1 && lane == 0)
-                    atomicExch(&p.cnt[pnl], 0u);
+#pragma unroll
+                for (int q = 0; q < QC; ++q) {
+                    if (c0 + q <= cl) {
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            tot[mt][0] += a[q][mt].x;
+                            tot[mt][1] += a[q][mt].y;
+                            tot[mt][2] += b[q][mt].x;
+                            tot[mt][3] += b[q][mt].y;
+                        }
+                    }
+                }
             }
+            store_y(tot);
+            if (lane == 0)
+                atomicExch(&p.cnt[pnl * 8 + j], 0u);
         };
 
         int cur = n > 0 ? u0 / KB : -1;

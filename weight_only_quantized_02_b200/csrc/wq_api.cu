@@ -139,7 +139,7 @@ Choice default_choice(int M, int K, int N, int sm_count, bool have_ws = true)
 {
     if (M < 8) {
         if (have_ws)
-            return {WQ_VARIANT_GEMV, 2, 0.f};
+            return {WQ_VARIANT_GEMV, 3, 0.f};
         return {WQ_VARIANT_GEMV_RB, default_rb_slices(K, N, sm_count), 0.f};
     }
     return {WQ_VARIANT_GEMM, std::min(8, max_gemm_split(K)), 0.f};
@@ -204,7 +204,7 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
     if (variant != WQ_VARIANT_AUTO) {
         c.variant = variant;
         if (split <= 0)
-            c.split = variant == WQ_VARIANT_GEMV      ? 2
+            c.split = variant == WQ_VARIANT_GEMV      ? 3
                       : variant == WQ_VARIANT_GEMV_RB ? default_rb_slices(K, N, d.sm_count)
                                                       : std::min(8, max_gemm_split(K));
     }

@@ -155,9 +155,11 @@ int wq_check_packed(const void *Wq, int bits, int K, int N, int group, cudaStrea
  *           is written: bf16_rne of the fp32-accumulated sum.
  * The kernel and split factor come from the dispatcher (tuned table, else
  * the default rule). The stream-K GEMV and a GEMM split > 1 use the
- * workspace registered with wq_set_workspace for the current device; with
- * no workspace, decode-sized M falls back to the row-block GEMV. Calls that
- * share a workspace must not overlap on the GPU (keep them on one stream). */
+ * workspace registered with wq_set_workspace for the current device. With
+ * no workspace (or too small a one), decode-sized M falls back to the
+ * row-block GEMV and the GEMM runs unsplit, so wq_linear never fails for
+ * lack of workspace. Calls that share a workspace must not overlap on the
+ * GPU (keep them on one stream). */
 int wq_linear(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
               const void *zeros, int group, int N, uint16_t *y, cudaStream_t stream);
 

@@ -245,6 +245,9 @@ def test_argument_errors(weight, ws):
         assert wq.wq_linear_status(x, pw, y, GEMM, 1) == 0
         assert wq.wq_linear_status(x, pw, y, GEMV_RB, 2) == 0
         assert wq.wq_linear_status(x, pw, y) == 0  # dispatcher falls back to the row-block GEMV
+        xm = bf16_dev(gen.x_bf16(40, K))
+        ym = torch.empty((40, N), dtype=torch.bfloat16, device=dev())
+        assert wq.wq_linear_status(xm, pw, ym) == 0  # ... and to the unsplit GEMM
     finally:
         wq.wq_set_workspace(ws)
     small = torch.zeros(512, dtype=torch.uint8, device=dev())

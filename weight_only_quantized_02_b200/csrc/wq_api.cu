@@ -215,6 +215,10 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
             c = default_choice(M, K, N, d.sm_count, sk_ws_ok);
         if (c.variant == WQ_VARIANT_GEMV && !sk_ws_ok)
             c = {WQ_VARIANT_GEMV_RB, default_rb_slices(K, N, d.sm_count), 0.f};
+        // an automatic choice never fails for lack of workspace: split-K GEMM
+        // without a large enough workspace runs unsplit
+        if (c.variant == WQ_VARIANT_GEMM && c.split > 1 && (!w || have < ws_bytes(M, N, c.split)))
+            c.split = 1;
     }
     if (!choice_valid(c.variant, c.split, M, K))
         return WQ_ERR_VARIANT;

@@ -180,6 +180,24 @@ int wq_linear_ex(const uint16_t *x, int M, int K, const void *Wq, const void *sc
                  const void *zeros, int group, int N, uint16_t *y, int variant, int split,
                  void *ws, size_t ws_bytes, cudaStream_t stream);
 
+/* wq_linear for callers that cannot allocate device memory when they run
+ * the layer: code inside a captured CUDA graph or an allocator's critical
+ * section, runtimes whose device memory is pre-partitioned, and plugin hosts
+ * that hand over only input and output buffers. The pages have no
+ * counterpart; this entry exists for those callers.
+ * It runs the stream-K GEMV. Its tickets and partial sums sit in a fixed
+ * array of about 4 MiB inside the library's device image. Every GPU that
+ * loads the library holds that array until the process exits. No call here
+ * allocates or frees memory.
+ *   Limits: 1 <= M <= 8 and N <= 262144. Larger shapes return WQ_ERR_SHAPE
+ *   before anything is enqueued. Other arguments are as for wq_linear.
+ *   The first call on a device looks up the array's device address (with
+ *   that device current). Make that first call before any stream capture.
+ *   Every call shares the array and enqueues a small memset of its tickets,
+ *   so calls that overlap on the GPU race: keep them on one stream. */
+int wq_linear_noalloc(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
+                      const void *zeros, int group, int N, uint16_t *y, cudaStream_t stream);
+
 /* Bytes of workspace for M tokens, N channels and GEMM splits up to
  * max_split. It holds one ticket counter per 128-channel panel and the
  * larger of the GEMM's fp32 partials [split][M][N] and the stream-K GEMV's

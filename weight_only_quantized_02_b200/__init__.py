@@ -60,6 +60,7 @@ def _load():
         "wq_linear": (I, [P, I, I, P, P, P, I, I, P, P]),
         "wq_linear_forced": (I, [P, I, I, P, P, P, I, I, P, I, I, P]),
         "wq_linear_ex": (I, [P, I, I, P, P, P, I, I, P, I, I, P, SZ, P]),
+        "wq_linear_noalloc": (I, [P, I, I, P, P, P, I, I, P, P]),
         "wq_workspace_bytes": (SZ, [I, I, I]),
         "wq_set_workspace": (I, [P, SZ]),
         "wq_tune": (I, [P, I, I, P, P, P, I, I, P, I, I, P]),
@@ -235,6 +236,16 @@ def wq_linear_ex(x: torch.Tensor, pw: PackedWeight, variant: int, split: int, ws
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(lib.wq_linear_ex(_p(x), M, K, _p(pw.wq), _p(pw.scales), _p(pw.zeros), pw.group, pw.N, _p(y),
                             variant, split, _p(ws), nbytes, _s(stream)), "wq_linear_ex")
+    return y
+
+
+def wq_linear_noalloc(x: torch.Tensor, pw: PackedWeight, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """wq_linear without any device allocation by the library (M <= 8).  Its
+    scratch is a fixed array inside the library; see include/wq.h."""
+    M, K = x.shape
+    y = _y_for(x, pw.N, y)
+    _check(lib.wq_linear_noalloc(_p(x), M, K, _p(pw.wq), _p(pw.scales), _p(pw.zeros), pw.group, pw.N, _p(y),
+                                 _s(stream)), "wq_linear_noalloc")
     return y
 
 

@@ -365,6 +365,30 @@ int wq_linear_ex(const uint16_t *x, int M, int K, const void *Wq, const void *sc
     return linear_impl(x, M, K, Wq, scales, zeros, group, N, y, variant, split, ws, ws_bytes_given, stream);
 }
 
+int wq_linear_noalloc(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros,
+                      int group, int N, uint16_t *y, cudaStream_t stream)
+{
+    int bits = 0;
+    int st = bits_of_group(group, &bits);
+    if (st != WQ_OK)
+        return st;
+    if (!x || !Wq || !scales || !y || (bits == 4 && !zeros))
+        return WQ_ERR_NULL;
+    if ((st = check_weight_shape(bits, K, N, group)) != WQ_OK)
+        return st;
+    if (M < 1 || M > noalloc_max_m() || N > noalloc_max_n())
+        return WQ_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(Wq) || !aligned16(scales) || (zeros && !aligned16(zeros)))
+        return WQ_ERR_ALIGN;
+    DeviceInfo d;
+    if ((st = current_device_info(&d)) != WQ_OK)
+        return st;
+    if (d.major != 10)
+        return WQ_ERR_ARCH;
+    LinearArgs a{x, M, K, N, Wq, scales, zeros, bits, group, y};
+    return cuda_status(launch_gemv_sk_noalloc(a, d.sm_count, stream));
+}
+
 size_t wq_workspace_bytes(int M, int N, int max_split)
 {
     if (M < 1 || N < 1 || max_split < 1)

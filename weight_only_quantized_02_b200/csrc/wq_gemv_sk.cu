@@ -21,6 +21,7 @@
 // and resets the ticket to zero.  Partials live in the workspace:
 // [G CTAs][2 slots (first/last panel of the range)][128 rows][8*MT tokens].
 #include <cstdint>
+#include <mutex>
 
 #include "wq_device.cuh"
 #include "wq_internal.h"
@@ -44,7 +45,7 @@ struct GemvSkParams {
 // Ring stage: packed weights of the unit, INT4 scales/zeros, and the unit's
 // activation slice x[0..M)[128 k] (one 256-byte bulk copy per token row,
 // rows 288 bytes apart so the eight rows a warp reads hit distinct banks).
-template <int BITS, int MT>
+template <int BITS, int MT, int OCC>
 struct SkCfg {
     static constexpr int kTPB = BITS == 4 ? 2 : 4;   // tiles per 16-row block per unit
     static constexpr int kRBB = kTPB * kTileBytes;   // bytes of one 16-row block per unit
@@ -54,8 +55,9 @@ struct SkCfg {
     static constexpr int kXRow = 288;                // smem stride of one token row (256 B + pad)
     static constexpr int kXB = 8 * MT * kXRow;
     static constexpr int kStageBytes = kPBB + kSZB + kXB;
-    // about 72 KB of ring per CTA, so three CTAs (27 warps) fit on an SM
-    static constexpr int kStagesRaw = (72 * 1024) / kStageBytes;
+    // ring sized so OCC CTAs fit in an SM's 228 KB of shared memory
+    static constexpr int kBudget = (220 * 1024) / OCC - 1024;
+    static constexpr int kStagesRaw = kBudget / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : (kStagesRaw < 2 ? 2 : kStagesRaw);
 };
 
@@ -147,10 +149,11 @@ __device__ __forceinline__ int sk_owner(long long U, int G, int u)
     return c;
 }
 
-template <int BITS, int MT>
-__global__ void __launch_bounds__(kSkThreads, MT == 4 ? 2 : 3) gemv_sk_kernel(const GemvSkParams p)
+// OCC = CTAs per SM the instance is built for (register bound and ring depth).
+template <int BITS, int MT, int OCC>
+__global__ void __launch_bounds__(kSkThreads, OCC) gemv_sk_kernel(const GemvSkParams p)
 {
-    using C = SkCfg<BITS, MT>;
+    using C = SkCfg<BITS, MT, OCC>;
     constexpr int STAGES = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -401,24 +404,24 @@ __global__ void __launch_bounds__(kSkThreads, MT == 4 ? 2 : 3) gemv_sk_kernel(co
         atomicExch(&g_gemv_sk_error, kErrTimeout);
 }
 
-template <int BITS, int MT>
-static cudaError_t launch_sk_t(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st)
+template <int BITS, int MT, int OCC>
+static cudaError_t launch_sk_t(const LinearArgs &a, void *ws, int sm_count, cudaStream_t st)
 {
-    using C = SkCfg<BITS, MT>;
+    using C = SkCfg<BITS, MT, OCC>;
     constexpr size_t smem = 128 + (size_t)C::kStages * C::kStageBytes + 2 * C::kStages * 8 + 16;
     static int occ = -1;
     if (occ < 0) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_sk_kernel<BITS, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(gemv_sk_kernel<BITS, MT, OCC>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess)
             return e;
         int o = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, gemv_sk_kernel<BITS, MT>, kSkThreads, smem);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, gemv_sk_kernel<BITS, MT, OCC>, kSkThreads, smem);
         if (e != cudaSuccess)
             return e;
         occ = o > 0 ? o : 1;
     }
-    const int per_sm = (ctas_per_sm > 0 && ctas_per_sm < occ) ? ctas_per_sm : occ;
+    const int per_sm = OCC < occ ? OCC : occ; // every CTA resident at once
     const Shape sh{a.bits, a.K, a.N, a.group};
     GemvSkParams p;
     p.x = a.x;
@@ -448,20 +451,31 @@ static cudaError_t launch_sk_t(const LinearArgs &a, int ctas_per_sm, void *ws, i
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemv_sk_kernel<BITS, MT>, p);
+    return cudaLaunchKernelEx(&cfg, gemv_sk_kernel<BITS, MT, OCC>, p);
+}
+
+template <int BITS, int MT>
+static cudaError_t launch_sk_occ(const LinearArgs &a, int occ, void *ws, int sm_count, cudaStream_t st)
+{
+    switch (occ) {
+    case 1: return launch_sk_t<BITS, MT, 1>(a, ws, sm_count, st);
+    case 2: return launch_sk_t<BITS, MT, 2>(a, ws, sm_count, st);
+    case 4: return launch_sk_t<BITS, MT, 4>(a, ws, sm_count, st);
+    default: return launch_sk_t<BITS, MT, 3>(a, ws, sm_count, st);
+    }
 }
 
 cudaError_t launch_gemv_sk(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st)
 {
     const int mt = (a.M + 7) / 8;
     if (a.bits == 8) {
-        if (mt == 1) return launch_sk_t<8, 1>(a, ctas_per_sm, ws, sm_count, st);
-        if (mt == 2) return launch_sk_t<8, 2>(a, ctas_per_sm, ws, sm_count, st);
-        return launch_sk_t<8, 4>(a, ctas_per_sm, ws, sm_count, st);
+        if (mt == 1) return launch_sk_occ<8, 1>(a, ctas_per_sm, ws, sm_count, st);
+        if (mt == 2) return launch_sk_occ<8, 2>(a, ctas_per_sm, ws, sm_count, st);
+        return launch_sk_occ<8, 4>(a, ctas_per_sm, ws, sm_count, st);
     }
-    if (mt == 1) return launch_sk_t<4, 1>(a, ctas_per_sm, ws, sm_count, st);
-    if (mt == 2) return launch_sk_t<4, 2>(a, ctas_per_sm, ws, sm_count, st);
-    return launch_sk_t<4, 4>(a, ctas_per_sm, ws, sm_count, st);
+    if (mt == 1) return launch_sk_occ<4, 1>(a, ctas_per_sm, ws, sm_count, st);
+    if (mt == 2) return launch_sk_occ<4, 2>(a, ctas_per_sm, ws, sm_count, st);
+    return launch_sk_occ<4, 4>(a, ctas_per_sm, ws, sm_count, st);
 }
 
 cudaError_t read_gemv_sk_error(int *code, cudaStream_t st)
@@ -476,6 +490,119 @@ cudaError_t read_gemv_sk_error(int *code, cudaStream_t st)
     e = cudaStreamSynchronize(st);
     *code = host;
     return e;
+}
+
+// ===========================================================================
+// Allocation-free entry: the stream-K GEMV with its tickets and partial sums
+// in a fixed array that lives in the library's own device memory.
+//
+// For callers that cannot call cudaMalloc when they run the layer: code
+// inside a CUDA-graph-captured region or a custom allocator's critical
+// section, embedded runtimes whose device memory is fully pre-partitioned, or
+// plugin hosts that hand out only input and output buffers.  The array is
+// part of the loaded module, so every GPU that loads the library holds it
+// (about 4 MiB) until the process exits.
+//
+// Limits: M <= kNoAllocMaxM tokens and N <= kNoAllocMaxN output channels;
+// larger calls are rejected before anything is enqueued.  Every call shares
+// the array, so calls that overlap on the GPU (different streams, or
+// different host threads without ordering) race; keep them on one stream.
+// ===========================================================================
+namespace {
+constexpr int kNoAllocMaxM = 8;
+constexpr int kNoAllocMaxN = 262144;
+constexpr size_t kNoAllocTicketBytes = (size_t)(kNoAllocMaxN / kPanelRows) * 8 * sizeof(uint32_t); // 64 KiB
+constexpr size_t kNoAllocPartBytes = (size_t)kSkMaxCtas * 2 * kPanelRows * 8 * sizeof(float);       // 4 MiB
+constexpr int kNoAllocMaxDevices = 64;
+} // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocTicketBytes + kNoAllocPartBytes];
+
+// Device address of g_noalloc_scratch per device.  In host code the array's
+// name is only a host-side stand-in for the device symbol, so the address
+// is looked up once per device (with that device current) on the first call.
+static void *g_noalloc_addr[kNoAllocMaxDevices] = {};
+static std::mutex g_noalloc_mu;
+
+template <int BITS, int OCC>
+static cudaError_t launch_sk_noalloc_t(const LinearArgs &a, uint32_t *cnt, float *part, int sm_count,
+                                       cudaStream_t st)
+{
+    using C = SkCfg<BITS, 1, OCC>;
+    constexpr size_t smem = 128 + (size_t)C::kStages * C::kStageBytes + 2 * C::kStages * 8 + 16;
+    static int occ = -1;
+    if (occ < 0) {
+        cudaError_t e = cudaFuncSetAttribute(gemv_sk_kernel<BITS, 1, OCC>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+        int o = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, gemv_sk_kernel<BITS, 1, OCC>, kSkThreads, smem);
+        if (e != cudaSuccess)
+            return e;
+        occ = o > 0 ? o : 1;
+    }
+    const int per_sm = OCC < occ ? OCC : occ;
+    const Shape sh{a.bits, a.K, a.N, a.group};
+    GemvSkParams p;
+    p.x = a.x;
+    p.M = a.M;
+    p.K = a.K;
+    p.N = a.N;
+    p.wq = (const uint8_t *)a.wq;
+    p.scales = (const uint16_t *)a.scales;
+    p.zeros = (const uint8_t *)a.zeros;
+    p.y = a.y;
+    p.KB = sh.kblocks();
+    p.U = sh.panels() * sh.kblocks();
+    p.cnt = cnt;
+    p.part = part;
+    int G = per_sm * sm_count;
+    if (G > kSkMaxCtas)
+        G = kSkMaxCtas;
+    if (G > p.U)
+        G = p.U;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(kSkThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    return cudaLaunchKernelEx(&cfg, gemv_sk_kernel<BITS, 1, OCC>, p);
+}
+
+int noalloc_max_m() { return kNoAllocMaxM; }
+int noalloc_max_n() { return kNoAllocMaxN; }
+
+cudaError_t launch_gemv_sk_noalloc(const LinearArgs &a, int sm_count, cudaStream_t st)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kNoAllocMaxDevices)
+        return cudaErrorInvalidDevice;
+    void *base = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (!g_noalloc_addr[dev]) {
+            void *ptr = nullptr;
+            e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+            if (e != cudaSuccess)
+                return e;
+            g_noalloc_addr[dev] = ptr;
+        }
+        base = g_noalloc_addr[dev];
+    }
+    uint32_t *cnt = static_cast<uint32_t *>(base);
+    float *part = reinterpret_cast<float *>(static_cast<unsigned char *>(base) + kNoAllocTicketBytes);
+    // the tickets this call uses must start at zero (the array keeps the last
+    // call's contents); the partial sums are always written before they are read
+    const size_t ticket_bytes = (size_t)((a.N + kPanelRows - 1) / kPanelRows) * 8 * sizeof(uint32_t);
+    e = cudaMemsetAsync(cnt, 0, ticket_bytes, st);
+    if (e != cudaSuccess)
+        return e;
+    return a.bits == 8 ? launch_sk_noalloc_t<8, 3>(a, cnt, part, sm_count, st)
+                       : launch_sk_noalloc_t<4, 3>(a, cnt, part, sm_count, st);
 }
 
 } // namespace wq

@@ -52,6 +52,12 @@ cudaError_t launch_gemv(const LinearArgs &a, int ks, int sm_count, cudaStream_t 
 cudaError_t launch_gemv_sk(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st);
 cudaError_t read_gemv_sk_error(int *code, cudaStream_t st);
 
+// Allocation-free stream-K GEMV (scratch in a fixed device array of the
+// library); M <= noalloc_max_m(), N <= noalloc_max_n().
+cudaError_t launch_gemv_sk_noalloc(const LinearArgs &a, int sm_count, cudaStream_t st);
+int noalloc_max_m();
+int noalloc_max_n();
+
 // GEMM: split = K splits (1..32); ws holds counters + partials when split > 1.
 cudaError_t launch_gemm(const LinearArgs &a, int split, void *ws, int sm_count, cudaStream_t st);
 

@@ -188,9 +188,10 @@ class ClockSampler:
                 "power_w_median": statistics.median(power) if power else None}
 
 
-def profile_traffic(kernel_file: str, summary_name: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken
-    on the current kernel source (sha256 recorded in the summary)."""
+def profile_traffic(kernel_file: str, summary_name: str, M: int):
+    """DRAM bytes per launch (read + write) of this kernel at this M, from the
+    committed ncu summary -- only if it was captured on the current kernel
+    source (its sha256 is recorded in the summary)."""
     path = os.path.join(ROOT, "profiles", summary_name)
     src = os.path.join(ROOT, "weight_only_quantized_02_b200", "csrc", kernel_file)
     try:
@@ -198,17 +199,16 @@ def profile_traffic(kernel_file: str, summary_name: str):
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
     except OSError:
         return None
-    vals = {}
+    if f"source_sha256: {sha}" not in text:
+        return None
     for line in text.splitlines():
-        if ":" in line:
-            k, v = line.split(":", 1)
-            vals[k.strip().lstrip("- ").strip("`")] = v.strip().strip("`")
-    if vals.get("source_sha256") != sha:
-        return None
-    try:
-        return float(vals["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+        line = line.strip().lstrip("- ")
+        if line.startswith(f"traffic_bytes_per_launch M={M}:"):
+            try:
+                return float(line.split(":", 1)[1])
+            except ValueError:
+                return None
+    return None
 
 
 # ---------------------------------------------------------------------------
@@ -243,7 +243,8 @@ def build_weights(name, device, copies):
     return cfg, pws
 
 
-KERNELS = {0: ("gemv_sk", "wq_gemv_sk.cu"), 1: ("gemm", "wq_gemm.cu"), 2: ("gemv_rb", "wq_gemv.cu")}
+KERNELS = {0: ("gemv_sk", "wq_gemv_sk.cu"), 1: ("gemm", "wq_gemm.cu"), 2: ("gemv_rb", "wq_gemv.cu"),
+           3: ("gemm_sk", "wq_gemm_sk.cu")}
 
 
 def kernel_name(variant, bits):
@@ -268,10 +269,17 @@ def bench_ours(args, device, rank, world):
     ys = {M: torch.empty((M, N), dtype=torch.bfloat16, device=device) for M in Ms}
     choices = {M: wq.wq_get_choice(M, K, N, bits, group) for M in Ms}
 
-    # tuning (the dispatcher's measured choice), untimed
-    if args.tune:
+    # the dispatcher's measured choice (the load-time tuning of the split_k
+    # auto-tune in Mit han lab Llm awq Kernel Selection Thresholds), untimed
+    if args.tuning_file and os.path.exists(args.tuning_file):
+        if wq.wq_load_tuning(args.tuning_file) != 0:
+            raise RuntimeError("unreadable tuning file " + args.tuning_file)
+        choices = {M: wq.wq_get_choice(M, K, N, bits, group) for M in Ms}
+    elif args.tune:
         for M in Ms:
             choices[M] = wq.wq_tune(xs[M], pws[0], ys[M], warmup=2, iters=7)
+        if args.tuning_file:
+            wq.wq_save_tuning(args.tuning_file)
 
     calls = [(M, c) for c in range(copies) for M in Ms]  # one step
     stream = torch.cuda.Stream(device)
@@ -362,13 +370,14 @@ def bench_ours(args, device, rank, world):
     dom = next(p for p in per_shape if p["M"] == Mdom)
     vdom = choices[Mdom][0]
     kfile = KERNELS[vdom][1]
-    summary = f"{dom['variant']}_{name}_M{Mdom}.md"
-    traffic = profile_traffic(kfile, summary)
+    summary = f"{dom['variant']}_{name}.md"
+    traffic = profile_traffic(kfile, summary, Mdom)
     bound = "hbm"
     achieved = call_bytes(bits, K, N, group, Mdom) / (share[Mdom] * 1e-6) / 1e9
     roofline = {"bound": bound, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "kernel": f"{dom['variant']} M={Mdom} split={dom['split']}",
+                "traffic_source": f"profiles/{summary}" if traffic is not None else None,
                 "algorithmic_bytes_per_launch": call_bytes(bits, K, N, group, Mdom),
                 "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)",
                 "frac_of_8tbs": round(achieved / 8000.0, 4)}
@@ -533,7 +542,10 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed device warm-up")
     ap.add_argument("--e2e-steps", type=int, default=200)
-    ap.add_argument("--tune", action="store_true", help="run wq_tune per M before timing")
+    ap.add_argument("--no-tune", dest="tune", action="store_false",
+                    help="time the dispatcher's untuned default instead of its tuned choice")
+    ap.add_argument("--tuning-file", default=None,
+                    help="load this dispatcher table instead of tuning (saved there after tuning if absent)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -77,6 +77,7 @@ typedef enum {
 #define WQ_VARIANT_GEMV 0    /* stream-K GEMV, M <= 32: TMA-fed ring, mma.sync; needs the workspace */
 #define WQ_VARIANT_GEMM 1    /* tcgen05 split-K GEMM, M <= 128 */
 #define WQ_VARIANT_GEMV_RB 2 /* row-block GEMV, M <= 32, direct 128-bit loads; no workspace */
+#define WQ_VARIANT_GEMM_SK 3 /* stream-K tcgen05 GEMM, M <= 128, persistent; needs the workspace */
 
 /* Static description of a status code. Host. Never NULL. */
 const char *wq_strerror(int status);
@@ -168,6 +169,7 @@ int wq_linear(const uint16_t *x, int M, int K, const void *Wq, const void *scale
  * GEMV: split = CTAs per SM, 1..4, capped by occupancy (the K range of
  *       every CTA is set by the stream-K partition).
  * GEMV_RB: split = K-slices per 16-row block, one of 1, 2, 4, 8.
+ * GEMM_SK: split = CTAs per SM, 1 or 2, capped by the tile's resources.
  * GEMM: split = K-splits, 1 <= split <= min(32, ceil(K/128)).
  * Returns WQ_ERR_VARIANT if the pair does not fit the shape. */
 int wq_linear_forced(const uint16_t *x, int M, int K, const void *Wq, const void *scales,

@@ -65,12 +65,13 @@ def test_packed_bytes_rejects(bits, K, N, group, status):
 
 
 def test_workspace_bytes():
-    # 8 tickets per 128-row panel, padded to 256 bytes, + the larger of the
-    # GEMM's fp32 partials and the stream-K GEMV's per-CTA panel partials
+    # 8 tickets per 128-row panel, padded to 256 bytes, + the largest of the
+    # split-K GEMM's fp32 partials [S][M][N] and the stream-K kernels'
+    # per-CTA panel partials [512 CTAs][2][128 rows][token tile]
     assert wq.wq_workspace_bytes(128, 5120, 32) == 1280 + 32 * 128 * 5120 * 4
-    assert wq.wq_workspace_bytes(64, 5120, 1) == 1280
+    assert wq.wq_workspace_bytes(64, 5120, 1) == 1280 + 512 * 2 * 128 * 64 * 4
     assert wq.wq_workspace_bytes(16, 5120, 1) == 1280 + 512 * 2 * 128 * 16 * 4
-    assert wq.wq_workspace_bytes(1, 17408, 1) == 4352 + 512 * 2 * 128 * 8 * 4  # 136 panels -> 4352 bytes
+    assert wq.wq_workspace_bytes(1, 17408, 1) == 4352 + 512 * 2 * 128 * 16 * 4  # 136 panels -> 4352 bytes
     assert wq.wq_workspace_bytes(0, 5120, 4) == 0
 
 

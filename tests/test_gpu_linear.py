@@ -22,7 +22,8 @@ from wqtest_helpers import (assert_parity, bf16_dev, dev, oracle_linear, pack_ca
 
 pytestmark = pytest.mark.gpu
 
-GEMV, GEMM, GEMV_RB = wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB
+GEMV, GEMM, GEMV_RB, GEMM_SK = (wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB,
+                                wq.WQ_VARIANT_GEMM_SK)
 SHAPES = {8: (1120, 400), 4: (1152, 400)}  # (K, N): 3 full panels + a 16-row tail
 M_ALL = [1, 7, 8, 9, 16, 17, 32, 33, 64, 65, 100, 128]
 
@@ -51,6 +52,7 @@ def _cases(M, K):
         out += [(GEMV, c) for c in (1, 2, 3)]
         out += [(GEMV_RB, ks) for ks in (1, 2, 4, 8)]
     out += [(GEMM, s) for s in (1, 2, 4, 8, 16, 32) if s <= kb]
+    out += [(GEMM_SK, c) for c in (1, 2)]
     return out
 
 

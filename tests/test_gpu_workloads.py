@@ -19,7 +19,8 @@ from wqtest_helpers import assert_parity, bf16_dev, bits_u16, bits_u32, dev, wor
 
 pytestmark = pytest.mark.gpu
 
-GEMV, GEMM, GEMV_RB = wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB
+GEMV, GEMM, GEMV_RB, GEMM_SK = (wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB,
+                                wq.WQ_VARIANT_GEMM_SK)
 
 
 def _build(name):
@@ -76,6 +77,7 @@ def _variants(M, K):
         out += [(GEMV, c) for c in (1, 2, 3)]
         out += [(GEMV_RB, ks) for ks in (1, 2, 4, 8)]
     out += [(GEMM, s) for s in (1, 2, 4, 8, 16, 32) if s <= (K + 127) // 128]
+    out += [(GEMM_SK, c) for c in (1, 2)]
     return out
 
 

@@ -27,6 +27,7 @@ WQ_VARIANT_AUTO = -1
 WQ_VARIANT_GEMV = 0     # stream-K GEMV (needs the workspace), M <= 32
 WQ_VARIANT_GEMM = 1     # tcgen05 split-K GEMM, M <= 128
 WQ_VARIANT_GEMV_RB = 2  # row-block GEMV, no workspace, M <= 32
+WQ_VARIANT_GEMM_SK = 3  # stream-K tcgen05 GEMM (needs the workspace), M <= 128
 
 STATUS = {
     0: "WQ_OK", -1: "WQ_ERR_NULL", -2: "WQ_ERR_SHAPE", -3: "WQ_ERR_ALIGN", -4: "WQ_ERR_GROUP",

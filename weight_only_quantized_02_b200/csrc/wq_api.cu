@@ -116,6 +116,8 @@ bool choice_valid(int variant, int split, int M, int K)
         return M <= 32 && (split == 1 || split == 2 || split == 4 || split == 8);
     if (variant == WQ_VARIANT_GEMM)
         return M <= 128 && split >= 1 && split <= max_gemm_split(K);
+    if (variant == WQ_VARIANT_GEMM_SK)
+        return M <= 128 && (split == 1 || split == 2);
     return false;
 }
 
@@ -206,6 +208,7 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
         if (split <= 0)
             c.split = variant == WQ_VARIANT_GEMV      ? 3
                       : variant == WQ_VARIANT_GEMV_RB ? default_rb_slices(K, N, d.sm_count)
+                      : variant == WQ_VARIANT_GEMM_SK ? 2
                                                       : std::min(8, max_gemm_split(K));
     }
     if (split > 0)
@@ -219,6 +222,8 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
         // without a large enough workspace runs unsplit
         if (c.variant == WQ_VARIANT_GEMM && c.split > 1 && (!w || have < ws_bytes(M, N, c.split)))
             c.split = 1;
+        if (c.variant == WQ_VARIANT_GEMM_SK && (!w || have < ws_bytes_gemm_sk(M, N)))
+            c = {WQ_VARIANT_GEMM, 1, 0.f};
     }
     if (!choice_valid(c.variant, c.split, M, K))
         return WQ_ERR_VARIANT;
@@ -230,6 +235,11 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
         if (!sk_ws_ok)
             return WQ_ERR_WORKSPACE;
         return cuda_status(launch_gemv_sk(a, c.split, w, d.sm_count, stream));
+    }
+    if (c.variant == WQ_VARIANT_GEMM_SK) {
+        if (!w || have < ws_bytes_gemm_sk(M, N))
+            return WQ_ERR_WORKSPACE;
+        return cuda_status(launch_gemm_sk(a, c.split, w, d.sm_count, stream));
     }
     if (c.split > 1 && (!w || have < ws_bytes(M, N, c.split)))
         return WQ_ERR_WORKSPACE;
@@ -393,7 +403,7 @@ size_t wq_workspace_bytes(int M, int N, int max_split)
 {
     if (M < 1 || N < 1 || max_split < 1)
         return 0;
-    size_t b = ws_bytes(M, N, max_split);
+    size_t b = std::max(ws_bytes(M, N, max_split), ws_bytes_gemm_sk(M, N));
     if (M <= 32)
         b = std::max(b, ws_bytes_gemv_sk(M, N));
     return b;
@@ -443,6 +453,8 @@ int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
     for (int s : {1, 2, 4, 8, 16, 32})
         if (s <= max_gemm_split(K))
             cands.push_back({WQ_VARIANT_GEMM, s});
+    for (int c : {1, 2})
+        cands.push_back({WQ_VARIANT_GEMM_SK, c});
 
     // Flush buffer larger than L2, so every timed call streams its weights
     // from HBM (the weights of a decode step are not L2-resident).
@@ -635,10 +647,11 @@ int wq_dequant_debug(const void *Wq, const void *scales, const void *zeros, int 
 
 int wq_device_error(cudaStream_t stream)
 {
-    int a = 0, b = 0;
-    if (read_device_error(&a, stream) != cudaSuccess || read_gemv_sk_error(&b, stream) != cudaSuccess)
+    int a = 0, b = 0, c = 0;
+    if (read_device_error(&a, stream) != cudaSuccess || read_gemv_sk_error(&b, stream) != cudaSuccess ||
+        read_gemm_sk_error(&c, stream) != cudaSuccess)
         return WQ_ERR_CUDA;
-    return (a == 0 && b == 0) ? WQ_OK : WQ_ERR_TIMEOUT;
+    return (a == 0 && b == 0 && c == 0) ? WQ_OK : WQ_ERR_TIMEOUT;
 }
 
 } // extern "C"

@@ -282,6 +282,19 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, float (&v)[16
         v[i] = __uint_as_float(r[i]);
 }
 
+// 32 TMEM lanes x 8 columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, float (&v)[8])
+{
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -305,6 +318,25 @@ __device__ __forceinline__ uint32_t ticket_take(uint32_t *counter)
     const uint32_t t = atomicAdd(counter, 1u);
     __threadfence();
     return t;
+}
+
+// ---------------------------------------------------------------------------
+// Stream-K partition: U units cut into G contiguous ranges [start(c),
+// start(c+1)); a panel of consecutive units may span several ranges.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int sk_start(long long U, int G, int c) { return (int)(U * c / G); }
+
+// CTA that owns unit u (ranges [start(c), start(c+1)); empty ranges skipped)
+__device__ __forceinline__ int sk_owner(long long U, int G, int u)
+{
+    int c = (int)(((long long)u * G) / U);
+    if (c >= G)
+        c = G - 1;
+    while (c + 1 < G && sk_start(U, G, c + 1) <= u)
+        ++c;
+    while (c > 0 && sk_start(U, G, c) > u)
+        --c;
+    return c;
 }
 
 // ---------------------------------------------------------------------------

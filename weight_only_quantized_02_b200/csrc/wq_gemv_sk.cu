@@ -134,21 +134,6 @@ __device__ __forceinline__ void sk_int4_tile(const uint4 &w, const uint8_t *xs, 
     }
 }
 
-__device__ __forceinline__ int sk_start(long long U, int G, int c) { return (int)(U * c / G); }
-
-// CTA that owns unit u (ranges [start(c), start(c+1)); empty ranges skipped)
-__device__ __forceinline__ int sk_owner(long long U, int G, int u)
-{
-    int c = (int)(((long long)u * G) / U);
-    if (c >= G)
-        c = G - 1;
-    while (c + 1 < G && sk_start(U, G, c + 1) <= u)
-        ++c;
-    while (c > 0 && sk_start(U, G, c) > u)
-        --c;
-    return c;
-}
-
 // OCC = CTAs per SM the instance is built for (register bound and ring depth).
 template <int BITS, int MT, int OCC>
 __global__ void __launch_bounds__(kSkThreads, OCC) gemv_sk_kernel(const GemvSkParams p)
@@ -159,7 +144,6 @@ __global__ void __launch_bounds__(kSkThreads, OCC) gemv_sk_kernel(const GemvSkPa
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     uint64_t *full = reinterpret_cast<uint64_t *>(ring + STAGES * C::kStageBytes);
     uint64_t *empty = full + STAGES;
-    uint32_t *s_ticket = reinterpret_cast<uint32_t *>(empty + STAGES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, c = blockIdx.x;

@@ -27,6 +27,11 @@ inline size_t ws_bytes(int M, int N, int S)
 {
     return ws_counter_bytes(N) + (S > 1 ? (size_t)S * M * N * sizeof(float) : 0);
 }
+inline int gemm_token_tile(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
+inline size_t ws_bytes_gemm_sk(int M, int N)
+{
+    return ws_counter_bytes(N) + (size_t)kSkMaxCtas * 2 * 128 * gemm_token_tile(M) * sizeof(float);
+}
 inline size_t ws_bytes_gemv_sk(int M, int N)
 {
     const int tok = 8 * ((M + 7) / 8);
@@ -60,6 +65,10 @@ int noalloc_max_n();
 
 // GEMM: split = K splits (1..32); ws holds counters + partials when split > 1.
 cudaError_t launch_gemm(const LinearArgs &a, int split, void *ws, int sm_count, cudaStream_t st);
+
+// Stream-K GEMM: ctas_per_sm = 0 (default) or 1/2; ws >= ws_bytes_gemm_sk.
+cudaError_t launch_gemm_sk(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st);
+cudaError_t read_gemm_sk_error(int *code, cudaStream_t st);
 
 // Reads and clears the device error word of the current device.
 cudaError_t read_device_error(int *code, cudaStream_t st);

@@ -244,7 +244,7 @@ def build_weights(name, device, copies):
 
 
 KERNELS = {0: ("gemv_sk", "wq_gemv_sk.cu"), 1: ("gemm", "wq_gemm.cu"), 2: ("gemv_rb", "wq_gemv.cu"),
-           3: ("gemm_sk", "wq_gemm_sk.cu")}
+           3: ("gemm_sk", "wq_gemm_sk.cu"), 4: ("gemm_i8", "wq_gemm_i8.cu")}
 
 
 def kernel_name(variant, bits):
@@ -263,7 +263,7 @@ def bench_ours(args, device, rank, world):
     wbytes = weight_bytes(bits, K, N, group)
     copies = max(2, math.ceil(L2_ROTATION_FACTOR * l2 / wbytes))
     cfg, pws = build_weights(name, device, copies)
-    ws = torch.zeros(wq.wq_workspace_bytes(max(Ms), N, 32), dtype=torch.uint8, device=device)
+    ws = torch.zeros(wq.wq_workspace_bytes(max(Ms), K, N, 32), dtype=torch.uint8, device=device)
     wq.wq_set_workspace(ws)
     xs = {M: torch.from_numpy(gen.x_bf16(M, K).view(np.int16)).view(torch.bfloat16).to(device) for M in Ms}
     ys = {M: torch.empty((M, N), dtype=torch.bfloat16, device=device) for M in Ms}

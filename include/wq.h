@@ -16,16 +16,23 @@
  *          layout, scales, zero points and group size. This is the review of
  *          Figure 4 in "Toward a Cleaner Quantization Stack in SGLang".)
  *
- * Two kernel families sit behind one call:
+ * Three kernel families sit behind one call:
  *   - a GEMV for decode-sized M, with register-level dequantization and
  *     128-bit weight loads ("BitBLAS-style GEMV", tileInfer README, Features
  *     table). Its fp32 dot products run on mma.sync tensor-core fragments.
  *   - a small-M GEMM (tcgen05 tensor cores, accumulators in tensor memory)
  *     with split-K and a fixed-order fp32 reduction ("split_k" auto-tuning,
  *     Mit han lab Llm awq Kernel Selection Thresholds, The Insight).
+ *   - for W8A16, M <= 64: the integer tensor cores (tcgen05 kind::i8) on the
+ *     raw INT8 codes. The per-channel scale factors out of the k sum, x is
+ *     written per token row as an integer X = round(x * 2^e) with |X| < 2^22
+ *     (three base-256 digits), the sums over k are exact int32, and
+ *     y = s * 2^-e * sum is formed in binary64 before the bf16 rounding.
  * A per-(M,K,N,bits,group) dispatcher picks the kernel and split factor. It
- * starts from the pages' rule (fewer than 8 tokens -> GEMV, else GEMM with
- * split 8; same page) and is overridden by measured timings (wq_tune).
+ * starts from an untuned rule (W8A16 within the integer path's limits -> the
+ * integer path; otherwise the pages' rule: fewer than 8 tokens -> GEMV, else
+ * GEMM with split 8; same page) and is overridden by measured timings
+ * (wq_tune).
  *
  * Conventions for every entry point:
  *   - The return value is a wq_status: 0 on success, negative on error.
@@ -78,6 +85,8 @@ typedef enum {
 #define WQ_VARIANT_GEMM 1    /* tcgen05 split-K GEMM, M <= 128 */
 #define WQ_VARIANT_GEMV_RB 2 /* row-block GEMV, M <= 32, direct 128-bit loads; no workspace */
 #define WQ_VARIANT_GEMM_SK 3 /* stream-K tcgen05 GEMM, M <= 128, persistent; needs the workspace */
+#define WQ_VARIANT_I8MMA 4   /* W8A16 only: stream-K tcgen05 kind::i8 on the raw codes, M <= 64,
+                                K <= 65536; needs the workspace */
 
 /* Static description of a status code. Host. Never NULL. */
 const char *wq_strerror(int status);
@@ -155,11 +164,11 @@ int wq_check_packed(const void *Wq, int bits, int K, int N, int group, cudaStrea
  *   y       device, bf16 [M][N], row-major, 16-byte aligned. Every element
  *           is written: bf16_rne of the fp32-accumulated sum.
  * The kernel and split factor come from the dispatcher (tuned table, else
- * the default rule). The stream-K GEMV and a GEMM split > 1 use the
- * workspace registered with wq_set_workspace for the current device. With
- * no workspace (or too small a one), decode-sized M falls back to the
- * row-block GEMV and the GEMM runs unsplit, so wq_linear never fails for
- * lack of workspace. Calls that share a workspace must not overlap on the
+ * the default rule). The stream-K kernels, the integer path and a GEMM
+ * split > 1 use the workspace registered with wq_set_workspace for the
+ * current device. With no workspace (or too small a one), decode-sized M
+ * falls back to the row-block GEMV and the GEMM runs unsplit, so wq_linear
+ * never fails for lack of workspace. Calls that share a workspace must not overlap on the
  * GPU (keep them on one stream). */
 int wq_linear(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
               const void *zeros, int group, int N, uint16_t *y, cudaStream_t stream);
@@ -171,6 +180,7 @@ int wq_linear(const uint16_t *x, int M, int K, const void *Wq, const void *scale
  * GEMV_RB: split = K-slices per 16-row block, one of 1, 2, 4, 8.
  * GEMM_SK: split = CTAs per SM, 1 or 2, capped by the tile's resources.
  * GEMM: split = K-splits, 1 <= split <= min(32, ceil(K/128)).
+ * I8MMA: split = 1 (one persistent CTA per SM).
  * Returns WQ_ERR_VARIANT if the pair does not fit the shape. */
 int wq_linear_forced(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
                      const void *zeros, int group, int N, uint16_t *y, int variant, int split,
@@ -200,11 +210,14 @@ int wq_linear_ex(const uint16_t *x, int M, int K, const void *Wq, const void *sc
 int wq_linear_noalloc(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
                       const void *zeros, int group, int N, uint16_t *y, cudaStream_t stream);
 
-/* Bytes of workspace for M tokens, N channels and GEMM splits up to
- * max_split. It holds one ticket counter per 128-channel panel and the
- * larger of the GEMM's fp32 partials [split][M][N] and the stream-K GEMV's
- * per-CTA panel partials (M <= 32). Host. */
-size_t wq_workspace_bytes(int M, int N, int max_split);
+/* Bytes of workspace for M tokens, a K x N weight and GEMM splits up to
+ * max_split: enough for every variant of that shape. It holds eight ticket
+ * counters per 128-channel panel and the largest of the GEMM's fp32
+ * partials [split][M][N], the stream-K kernels' per-CTA panel partials, and
+ * the integer path's activation digits (ceil(K/128) x 128 x up to 192
+ * bytes) with its int32 per-CTA partials. Returns 0 for M, K, N or
+ * max_split < 1. Host. */
+size_t wq_workspace_bytes(int M, int K, int N, int max_split);
 
 /* Registers a caller-owned device workspace for the current device, used by
  * wq_linear. Zeroes its counters with a synchronous cudaMemset. The kernels

@@ -66,13 +66,17 @@ def test_packed_bytes_rejects(bits, K, N, group, status):
 
 def test_workspace_bytes():
     # 8 tickets per 128-row panel, padded to 256 bytes, + the largest of the
-    # split-K GEMM's fp32 partials [S][M][N] and the stream-K kernels'
-    # per-CTA panel partials [512 CTAs][2][128 rows][token tile]
-    assert wq.wq_workspace_bytes(128, 5120, 32) == 1280 + 32 * 128 * 5120 * 4
-    assert wq.wq_workspace_bytes(64, 5120, 1) == 1280 + 512 * 2 * 128 * 64 * 4
-    assert wq.wq_workspace_bytes(16, 5120, 1) == 1280 + 512 * 2 * 128 * 16 * 4
-    assert wq.wq_workspace_bytes(1, 17408, 1) == 4352 + 512 * 2 * 128 * 16 * 4  # 136 panels -> 4352 bytes
-    assert wq.wq_workspace_bytes(0, 5120, 4) == 0
+    # split-K GEMM's fp32 partials [S][M][N], the stream-K kernels' per-CTA
+    # panel partials [512 CTAs][2][128 rows][token tile] and the integer
+    # path's digits + int32 partials (smaller than the stream-K GEMM's here)
+    assert wq.wq_workspace_bytes(128, 5120, 5120, 32) == 1280 + 32 * 128 * 5120 * 4
+    assert wq.wq_workspace_bytes(64, 5120, 5120, 1) == 1280 + 512 * 2 * 128 * 64 * 4
+    assert wq.wq_workspace_bytes(16, 5120, 5120, 1) == 1280 + 512 * 2 * 128 * 16 * 4
+    assert wq.wq_workspace_bytes(1, 5120, 17408, 1) == 4352 + 512 * 2 * 128 * 16 * 4  # 136 panels -> 4352 bytes
+    # integer path, M = 1 (16 digit rows): 256 + 40 k-blocks x 16 x 128 + 160 x 2 x 16 x 128 x 4
+    assert 256 + 40 * 16 * 128 + 160 * 2 * 16 * 128 * 4 < 512 * 2 * 128 * 16 * 4
+    assert wq.wq_workspace_bytes(0, 5120, 5120, 4) == 0
+    assert wq.wq_workspace_bytes(1, 0, 5120, 4) == 0
 
 
 def test_null_pointer_checks_need_no_device():
@@ -83,7 +87,8 @@ def test_null_pointer_checks_need_no_device():
 
 def test_tuning_file_parse_errors(tmp_path):
     good = tmp_path / "good.txt"
-    good.write_text("# comment\nNVIDIA B200|148 1 5120 17408 8 0 0 4 12.500\n")
+    good.write_text("# comment\nNVIDIA B200|148 1 5120 17408 8 0 0 4 12.500\n"
+                    "NVIDIA B200|148 4 5120 17408 8 0 4 1 9.000\n")
     assert wq.wq_load_tuning(str(good)) == 0
     for bad_line in [
         "NVIDIA B200|148 1 5120 17408 8 0 2 3 12.5\n",      # row-block GEMV split must be 1/2/4/8
@@ -94,6 +99,9 @@ def test_tuning_file_parse_errors(tmp_path):
         "NVIDIA B200|148 1 5120 17408 8 0 0\n",             # truncated
         "NVIDIA B200|148 1 5120 17408 8 0 0 4 12.5 extra\n",
         "NVIDIA B200|148 64 17408 5120 4 128 1 64 1.0\n",   # split above 32
+        "NVIDIA B200|148 4 5120 17408 4 128 4 1 9.0\n",     # integer path: INT8 only
+        "NVIDIA B200|148 65 5120 17408 8 0 4 1 9.0\n",      # integer path: M <= 64
+        "NVIDIA B200|148 4 5120 17408 8 0 4 2 9.0\n",       # integer path: split 1 only
     ]:
         p = tmp_path / "bad.txt"
         p.write_text(bad_line)

@@ -17,20 +17,20 @@ import torch
 import oracle
 import wq_inputs as gen
 import weight_only_quantized_02_b200 as wq
-from wqtest_helpers import (assert_parity, bf16_dev, dev, oracle_linear, pack_canonical_int4, pack_canonical_int8,
-                            quantize_and_pack, to_dev, workspace, y_host)
+from wqtest_helpers import (assert_parity, bf16_dev, dev, i8_fixed_point, oracle_linear, pack_canonical_int4,
+                            pack_canonical_int8, quantize_and_pack, to_dev, workspace, y_host)
 
 pytestmark = pytest.mark.gpu
 
-GEMV, GEMM, GEMV_RB, GEMM_SK = (wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB,
-                                wq.WQ_VARIANT_GEMM_SK)
+GEMV, GEMM, GEMV_RB, GEMM_SK, I8 = (wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB,
+                                    wq.WQ_VARIANT_GEMM_SK, wq.WQ_VARIANT_I8MMA)
 SHAPES = {8: (1120, 400), 4: (1152, 400)}  # (K, N): 3 full panels + a 16-row tail
 M_ALL = [1, 7, 8, 9, 16, 17, 32, 33, 64, 65, 100, 128]
 
 
 @pytest.fixture(scope="module")
 def ws():
-    t = workspace(128, 1024, 32)
+    t = workspace(128, 1152, 1024, 32)
     wq.wq_set_workspace(t)
     yield t
     wq.wq_set_workspace(None)
@@ -45,7 +45,7 @@ def weight(request):
     return bits, K, N, pw, canon
 
 
-def _cases(M, K):
+def _cases(M, K, bits):
     kb = (K + 127) // 128
     out = []
     if M <= 32:
@@ -53,6 +53,8 @@ def _cases(M, K):
         out += [(GEMV_RB, ks) for ks in (1, 2, 4, 8)]
     out += [(GEMM, s) for s in (1, 2, 4, 8, 16, 32) if s <= kb]
     out += [(GEMM_SK, c) for c in (1, 2)]
+    if bits == 8 and M <= 64:
+        out += [(I8, 1)]
     return out
 
 
@@ -62,7 +64,7 @@ def test_linear_parity_all_variants(weight, ws, M):
     x = gen.x_bf16(M, K)
     y_ref = oracle_linear(x, canon, bits)
     xd = bf16_dev(x)
-    for variant, split in _cases(M, K):
+    for variant, split in _cases(M, K, bits):
         y = wq.wq_linear_forced(xd, pw, variant, split)
         assert_parity(y_host(y), y_ref, f"bits={bits} M={M} variant={variant} split={split}")
     # the dispatcher's own choice
@@ -72,7 +74,7 @@ def test_linear_parity_all_variants(weight, ws, M):
 def test_deterministic_and_splits_agree(weight, ws):
     bits, K, N, pw, canon = weight
     x = bf16_dev(gen.x_bf16(24, K))
-    for variant, split in _cases(24, K):
+    for variant, split in _cases(24, K, bits):
         a = wq.wq_linear_forced(x, pw, variant, split)
         b = wq.wq_linear_forced(x, pw, variant, split)
         assert torch.equal(a.view(torch.int16), b.view(torch.int16)), (variant, split)
@@ -94,8 +96,17 @@ def test_repeated_dispatch_resets_tickets(weight, ws):
 # closed-form special cases, bit for bit
 # ---------------------------------------------------------------------------
 
-def _all_cases(M, K):
-    return _cases(M, K)
+def _all_cases(M, K, bits):
+    return _cases(M, K, bits)
+
+
+def _i8_want_one_hot(x_bits, q, s):
+    """y of an INT8 weight with one nonzero per row, on the integer path's
+    fixed-point activations: bf16_rne(s[n] * q[n][c] * xq[m][c]), exact in
+    binary64 (8 + 8 + 22 significant bits)."""
+    xq = i8_fixed_point(x_bits)
+    y = xq @ (q.astype(np.float64).T * oracle.bf16_to_f64(s)[None, :])
+    return oracle.bf16_to_f64(oracle.bf16_rne_of(y))
 
 
 @pytest.mark.parametrize("bits", [8, 4])
@@ -110,7 +121,7 @@ def test_one_hot_activations_pick_weights_exactly(bits, ws):
     for m, k in enumerate(ks):
         x[m, k] = 0x3F80  # 1.0
     want = oracle.bf16_to_f64(oracle.bf16_rne_of(oracle_linear(x, canon, bits)))
-    for variant, split in _all_cases(M, K):
+    for variant, split in _all_cases(M, K, bits):  # the integer path included: 1.0 and 0 are exact
         y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
         assert np.array_equal(y, want), (variant, split)
 
@@ -125,9 +136,14 @@ def test_one_hot_int8_weights_exact(ws):
     pw = pack_canonical_int8(q, s)
     x = gen.x_bf16(M, K)
     want = oracle.bf16_to_f64(oracle.bf16_rne_of(oracle.linear_int8(x, q, s)))
-    for variant, split in _all_cases(M, K):
+    for variant, split in _all_cases(M, K, 8):
         y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
-        assert np.array_equal(y, want), (variant, split)
+        if variant == I8:
+            # exact on its fixed-point activations, and within the layer's tolerance of the oracle
+            assert np.array_equal(y, _i8_want_one_hot(x, q, s)), (variant, split)
+            assert_parity(y, oracle.linear_int8(x, q, s), "one-hot int8 weights, integer path")
+        else:
+            assert np.array_equal(y, want), (variant, split)
 
 
 def test_one_hot_int4_weights_exact(ws):
@@ -150,7 +166,7 @@ def test_one_hot_int4_weights_exact(ws):
     pw = pack_canonical_int4(q, s, z)
     x = gen.x_bf16(M, K)
     want = oracle.bf16_to_f64(oracle.bf16_rne_of(oracle.linear_int4(x, q, s, z)))
-    for variant, split in _all_cases(M, K):
+    for variant, split in _all_cases(M, K, 4):
         y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
         assert np.array_equal(y, want), (variant, split)
 
@@ -173,9 +189,10 @@ def test_identity_weights_reproduce_x(bits, ws):
             z[:, gi // 8] |= np.uint32(8) << np.uint32(4 * (gi % 8))
         pw = pack_canonical_int4(q, np.full((N, K // 128), 0x3F80, np.uint16), z)
     want = oracle.bf16_to_f64(x)
-    for variant, split in _all_cases(M, K):
+    want_i8 = oracle.bf16_to_f64(oracle.bf16_rne_of(i8_fixed_point(x)))
+    for variant, split in _all_cases(M, K, bits):
         y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
-        assert np.array_equal(y, want), (variant, split)
+        assert np.array_equal(y, want_i8 if variant == I8 else want), (variant, split)
 
 
 @pytest.mark.parametrize("bits", [8, 4])
@@ -189,7 +206,7 @@ def test_zero_scales_give_zero(bits, ws):
         z = g.integers(0, 2**32, size=(N, oracle.zero_words_per_row(K)), dtype=np.uint64).astype(np.uint32)
         pw = pack_canonical_int4(q, np.zeros((N, K // 128), np.uint16), z)
     x = bf16_dev(gen.x_bf16(17, K))
-    for variant, split in _all_cases(17, K):
+    for variant, split in _all_cases(17, K, bits):
         y = y_host(wq.wq_linear_forced(x, pw, variant, split))
         assert np.all(y == 0), (variant, split)
 
@@ -200,7 +217,7 @@ def test_power_of_two_scaling_is_exact(weight, ws):
     xd = bf16_dev(x)
     x2 = bf16_dev((x.astype(np.uint32) + (1 << 7)).astype(np.uint16))  # 2x exactly (no zeros in x)
     assert np.all((x & 0x7F80) != 0)
-    for variant, split in _cases(9, K):
+    for variant, split in _cases(9, K, bits):
         a = y_host(wq.wq_linear_forced(xd, pw, variant, split))
         b = y_host(wq.wq_linear_forced(x2, pw, variant, split))
         assert np.array_equal(2 * a, b), (variant, split)
@@ -217,7 +234,7 @@ def test_output_canaries_untouched(weight, ws):
         pad = 4096
         buf = torch.full((M * N + 2 * pad,), -1234, dtype=torch.int16, device=dev())
         y = buf[pad:pad + M * N].view(torch.bfloat16).view(M, N)
-        for variant, split in _cases(M, K):
+        for variant, split in _cases(M, K, bits):
             wq.wq_linear_forced(bf16_dev(x), pw, variant, split, y=y)
             torch.cuda.synchronize()
             assert int((buf[:pad] != -1234).sum()) == 0 and int((buf[-pad:] != -1234).sum()) == 0, (variant, split)
@@ -232,6 +249,12 @@ def test_argument_errors(weight, ws):
     assert wq.wq_linear_status(x, pw, y, GEMV, 5) == -11          # CTAs per SM 1..4
     assert wq.wq_linear_status(x, pw, y, GEMM, 33) == -11         # split above 32
     assert wq.wq_linear_status(x, pw, y, 7, 1) == -11             # unknown variant
+    assert wq.wq_linear_status(x, pw, y, I8, 2) == -11            # one CTA per SM only
+    if bits == 4:
+        assert wq.wq_linear_status(x, pw, y, I8, 1) == -11        # integer path: INT8 only
+    xc = bf16_dev(gen.x_bf16(65, K))
+    yc = torch.empty((65, N), dtype=torch.bfloat16, device=dev())
+    assert wq.wq_linear_status(xc, pw, yc, I8, 1) == -11          # integer path takes M <= 64
     xb = bf16_dev(gen.x_bf16(40, K))
     yb = torch.empty((40, N), dtype=torch.bfloat16, device=dev())
     assert wq.wq_linear_status(xb, pw, yb, GEMV, 1) == -11        # GEMV takes M <= 32
@@ -244,6 +267,8 @@ def test_argument_errors(weight, ws):
     try:
         assert wq.wq_linear_status(x, pw, y, GEMM, 4) == -6
         assert wq.wq_linear_status(x, pw, y, GEMV, 1) == -6
+        if bits == 8:
+            assert wq.wq_linear_status(x, pw, y, I8, 1) == -6
         assert wq.wq_linear_status(x, pw, y, GEMM, 1) == 0
         assert wq.wq_linear_status(x, pw, y, GEMV_RB, 2) == 0
         assert wq.wq_linear_status(x, pw, y) == 0  # dispatcher falls back to the row-block GEMV
@@ -264,7 +289,7 @@ def test_explicit_workspace_on_two_streams(weight):
     x = gen.x_bf16(48, K)
     xd = bf16_dev(x)
     s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
-    w1, w2 = workspace(48, N, 8), workspace(48, N, 8)
+    w1, w2 = workspace(48, K, N, 8), workspace(48, K, N, 8)
     torch.cuda.synchronize()
     with torch.cuda.stream(s1):
         y1 = wq.wq_linear_ex(xd, pw, GEMM, 8, w1, stream=s1)
@@ -278,7 +303,10 @@ def test_explicit_workspace_on_two_streams(weight):
 
 def test_cuda_graph_replay(weight, ws):
     bits, K, N, pw, canon = weight
-    for M, variant, split in [(1, GEMV, 2), (1, GEMV_RB, 4), (16, GEMM, 4), (128, GEMM, 2)]:
+    runs = [(1, GEMV, 2), (1, GEMV_RB, 4), (16, GEMM, 4), (128, GEMM, 2)]
+    if bits == 8:
+        runs += [(1, I8, 1), (16, I8, 1)]
+    for M, variant, split in runs:
         x = gen.x_bf16(M, K)
         xd = bf16_dev(x)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
@@ -305,7 +333,7 @@ def test_tuner_and_table_roundtrip(weight, ws, tmp_path):
     x = gen.x_bf16(M, K)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
     v, s = wq.wq_tune(bf16_dev(x), pw, y, warmup=1, iters=3)
-    assert (v, s) in _cases(M, K)
+    assert (v, s) in _cases(M, K, bits)
     assert_parity(y_host(wq.wq_linear(bf16_dev(x), pw)), oracle_linear(x, canon, bits), "tuned")
     path = str(tmp_path / "table.txt")
     wq.wq_save_tuning(path)

@@ -19,8 +19,8 @@ from wqtest_helpers import assert_parity, bf16_dev, bits_u16, bits_u32, dev, wor
 
 pytestmark = pytest.mark.gpu
 
-GEMV, GEMM, GEMV_RB, GEMM_SK = (wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB,
-                                wq.WQ_VARIANT_GEMM_SK)
+GEMV, GEMM, GEMV_RB, GEMM_SK, I8 = (wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB,
+                                    wq.WQ_VARIANT_GEMM_SK, wq.WQ_VARIANT_I8MMA)
 
 
 def _build(name):
@@ -71,13 +71,15 @@ def _ref(cfg, x, codes):
     return oracle.linear_int4(x, codes[0], codes[1], codes[2])
 
 
-def _variants(M, K):
+def _variants(M, K, bits):
     out = []
     if M <= 32:
         out += [(GEMV, c) for c in (1, 2, 3)]
         out += [(GEMV_RB, ks) for ks in (1, 2, 4, 8)]
     out += [(GEMM, s) for s in (1, 2, 4, 8, 16, 32) if s <= (K + 127) // 128]
     out += [(GEMM_SK, c) for c in (1, 2)]
+    if bits == 8 and M <= 64:
+        out += [(I8, 1)]
     return out
 
 
@@ -89,7 +91,7 @@ def test_workload_full_size(name):
     rows = gen.sample_rows(N, 96)
     codes = _oracle_rows(cfg, src, rows)
     Mmax = max(cfg["Ms"])
-    ws = workspace(Mmax, N, 32)
+    ws = workspace(Mmax, K, N, 32)
     wq.wq_set_workspace(ws)
     idx = torch.from_numpy(rows).to(dev())
     try:
@@ -98,7 +100,7 @@ def test_workload_full_size(name):
             y_ref = _ref(cfg, x, codes)
             xd = bf16_dev(x)
             y = torch.empty((M, N), dtype=torch.bfloat16, device=dev())
-            for variant, split in _variants(M, K):
+            for variant, split in _variants(M, K, cfg["bits"]):
                 wq.wq_linear_forced(xd, pw, variant, split, y=y)
                 assert_parity(y_host(y.index_select(1, idx)), y_ref, f"{name} M={M} {variant}/{split}")
             y.zero_()

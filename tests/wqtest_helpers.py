@@ -85,6 +85,25 @@ def oracle_linear(x_bits: np.ndarray, canon, bits: int, rows=None) -> np.ndarray
     return oracle.linear_int4(x_bits, canon[0], canon[1], canon[2], 128, rows=rows)
 
 
-def workspace(M: int, N: int, max_split: int = 32) -> torch.Tensor:
-    nbytes = wq.wq_workspace_bytes(M, N, max_split)
+def workspace(M: int, K: int, N: int, max_split: int = 32) -> torch.Tensor:
+    nbytes = wq.wq_workspace_bytes(M, K, N, max_split)
     return torch.zeros(nbytes, dtype=torch.uint8, device=dev())
+
+
+def i8_fixed_point(x_bits: np.ndarray) -> np.ndarray:
+    """The activations as the integer tensor-core path represents them, from
+    the library's stated contract (include/wq.h): per token row, e = 21 - E
+    with E the binary exponent of the row's largest magnitude (2^E <= max|x|
+    < 2^(E+1); subnormal rows use E = -126), and x -> round(x * 2^e) * 2^-e,
+    ties to even.  Every element within 2^14 of the row's largest is
+    unchanged.  Returns binary64 values."""
+    x = oracle.bf16_to_f64(x_bits)
+    out = np.zeros_like(x)
+    for m in range(x.shape[0]):
+        amax = np.max(np.abs(x[m])) if x.shape[1] else 0.0
+        if amax == 0.0:
+            continue
+        E = max(int(np.frexp(amax)[1]) - 1, -126)  # amax = f * 2^(E+1), f in [0.5, 1)
+        e = 21 - E
+        out[m] = np.rint(np.ldexp(x[m], e)) * np.ldexp(1.0, -e)  # exact: |X| < 2^22
+    return out

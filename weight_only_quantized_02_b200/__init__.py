@@ -28,6 +28,7 @@ WQ_VARIANT_GEMV = 0     # stream-K GEMV (needs the workspace), M <= 32
 WQ_VARIANT_GEMM = 1     # tcgen05 split-K GEMM, M <= 128
 WQ_VARIANT_GEMV_RB = 2  # row-block GEMV, no workspace, M <= 32
 WQ_VARIANT_GEMM_SK = 3  # stream-K tcgen05 GEMM (needs the workspace), M <= 128
+WQ_VARIANT_I8MMA = 4    # W8A16: tcgen05 kind::i8 on the raw codes (needs the workspace), M <= 64
 
 STATUS = {
     0: "WQ_OK", -1: "WQ_ERR_NULL", -2: "WQ_ERR_SHAPE", -3: "WQ_ERR_ALIGN", -4: "WQ_ERR_GROUP",
@@ -62,7 +63,7 @@ def _load():
         "wq_linear_forced": (I, [P, I, I, P, P, P, I, I, P, I, I, P]),
         "wq_linear_ex": (I, [P, I, I, P, P, P, I, I, P, I, I, P, SZ, P]),
         "wq_linear_noalloc": (I, [P, I, I, P, P, P, I, I, P, P]),
-        "wq_workspace_bytes": (SZ, [I, I, I]),
+        "wq_workspace_bytes": (SZ, [I, I, I, I]),
         "wq_set_workspace": (I, [P, SZ]),
         "wq_tune": (I, [P, I, I, P, P, P, I, I, P, I, I, P]),
         "wq_get_choice": (I, [I, I, I, I, I, P, P]),
@@ -132,8 +133,8 @@ def wq_packed_bytes(bits: int, K: int, N: int, group: int):
     return a.value, b.value, c.value
 
 
-def wq_workspace_bytes(M: int, N: int, max_split: int) -> int:
-    return int(lib.wq_workspace_bytes(M, N, max_split))
+def wq_workspace_bytes(M: int, K: int, N: int, max_split: int) -> int:
+    return int(lib.wq_workspace_bytes(M, K, N, max_split))
 
 
 # ---------------------------------------------------------------------------

@@ -1,6 +1,6 @@
 """Build the CUDA library libwq.so in-tree for sm_100a (B200).
 
-    python -m weight_only_quantized_02_b200.build [--force] [--verbose]
+    python weight_only_quantized_02_b200/build.py [--force] [--verbose]
 
 Each .cu file under csrc/ is compiled with nvcc for
 ``-gencode arch=compute_100a,code=sm_100a`` and linked into one shared
@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libwq.so")
 
-SOURCES = ["wq_api.cu", "wq_pack.cu", "wq_gemv.cu", "wq_gemv_sk.cu", "wq_gemm.cu", "wq_gemm_sk.cu"]
+SOURCES = ["wq_api.cu", "wq_pack.cu", "wq_gemv.cu", "wq_gemv_sk.cu", "wq_gemm.cu", "wq_gemm_sk.cu", "wq_gemm_i8.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -35,6 +35,7 @@ def nvcc() -> str:
 def _deps():
     files = [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
     files.append(os.path.join(INCLUDE, "wq.h"))
+    files.append(os.path.abspath(__file__))  # the source list and flags
     return files
 
 

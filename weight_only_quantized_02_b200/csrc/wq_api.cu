@@ -108,8 +108,12 @@ int check_weight_shape(int bits, int K, int N, int group)
 
 int max_gemm_split(int K) { return std::min(32, (K + kBlockK - 1) / kBlockK); }
 
-bool choice_valid(int variant, int split, int M, int K)
+bool i8_fits(int bits, int M, int K) { return bits == 8 && M <= kI8MaxM && K <= kI8MaxK; }
+
+bool choice_valid(int variant, int split, int M, int K, int bits)
 {
+    if (variant == WQ_VARIANT_I8MMA)
+        return i8_fits(bits, M, K) && split == 1;
     if (variant == WQ_VARIANT_GEMV)
         return M <= 32 && split >= 1 && split <= 4;
     if (variant == WQ_VARIANT_GEMV_RB)
@@ -133,12 +137,15 @@ int default_rb_slices(int K, int N, int sm_count)
     return ks;
 }
 
-// The pages' untuned rule: fewer than 8 tokens -> GEMV, otherwise the GEMM
-// with split_k = 8 (Mit han lab Llm awq Kernel Selection Thresholds, The
-// Insight).  The stream-K GEMV needs the split-K workspace; without one the
-// row-block GEMV is used.
-Choice default_choice(int M, int K, int N, int sm_count, bool have_ws = true)
+// Untuned rule.  INT8 runs on the integer tensor cores whenever the shape
+// and the workspace allow it.  Otherwise the pages' rule: fewer than 8
+// tokens -> GEMV, else the GEMM with split_k = 8 (Mit han lab Llm awq Kernel
+// Selection Thresholds, The Insight).  The stream-K GEMV needs the split-K
+// workspace; without one the row-block GEMV is used.
+Choice default_choice(int M, int K, int N, int bits, int sm_count, bool have_ws = true, bool have_i8_ws = true)
 {
+    if (i8_fits(bits, M, K) && have_i8_ws)
+        return {WQ_VARIANT_I8MMA, 1, 0.f};
     if (M < 8) {
         if (have_ws)
             return {WQ_VARIANT_GEMV, 3, 0.f};
@@ -157,7 +164,7 @@ int lookup_choice(const DeviceInfo &d, int M, int K, int N, int bits, int group,
             return WQ_OK;
         }
     }
-    *c = default_choice(M, K, N, d.sm_count);
+    *c = default_choice(M, K, N, bits, d.sm_count);
     return WQ_OK;
 }
 
@@ -200,6 +207,7 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
     if (w && !aligned16(w))
         return WQ_ERR_ALIGN;
     const bool sk_ws_ok = w && have >= ws_bytes_gemv_sk(M, N);
+    const bool i8_ws_ok = w && i8_fits(bits, M, K) && have >= ws_bytes_gemm_i8(M, K, N);
 
     Choice c;
     lookup_choice(d, M, K, N, bits, group, &c);
@@ -209,13 +217,14 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
             c.split = variant == WQ_VARIANT_GEMV      ? 3
                       : variant == WQ_VARIANT_GEMV_RB ? default_rb_slices(K, N, d.sm_count)
                       : variant == WQ_VARIANT_GEMM_SK ? 2
+                      : variant == WQ_VARIANT_I8MMA   ? 1
                                                       : std::min(8, max_gemm_split(K));
     }
     if (split > 0)
         c.split = split;
     if (variant == WQ_VARIANT_AUTO) {
-        if (!choice_valid(c.variant, c.split, M, K))
-            c = default_choice(M, K, N, d.sm_count, sk_ws_ok);
+        if (!choice_valid(c.variant, c.split, M, K, bits) || (c.variant == WQ_VARIANT_I8MMA && !i8_ws_ok))
+            c = default_choice(M, K, N, bits, d.sm_count, sk_ws_ok, i8_ws_ok);
         if (c.variant == WQ_VARIANT_GEMV && !sk_ws_ok)
             c = {WQ_VARIANT_GEMV_RB, default_rb_slices(K, N, d.sm_count), 0.f};
         // an automatic choice never fails for lack of workspace: split-K GEMM
@@ -225,10 +234,15 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
         if (c.variant == WQ_VARIANT_GEMM_SK && (!w || have < ws_bytes_gemm_sk(M, N)))
             c = {WQ_VARIANT_GEMM, 1, 0.f};
     }
-    if (!choice_valid(c.variant, c.split, M, K))
+    if (!choice_valid(c.variant, c.split, M, K, bits))
         return WQ_ERR_VARIANT;
 
     LinearArgs a{x, M, K, N, Wq, scales, zeros, bits, group, y};
+    if (c.variant == WQ_VARIANT_I8MMA) {
+        if (!i8_ws_ok)
+            return WQ_ERR_WORKSPACE;
+        return cuda_status(launch_gemm_i8(a, w, d.sm_count, stream));
+    }
     if (c.variant == WQ_VARIANT_GEMV_RB)
         return cuda_status(launch_gemv(a, c.split, d.sm_count, stream));
     if (c.variant == WQ_VARIANT_GEMV) {
@@ -272,7 +286,7 @@ const char *wq_strerror(int status)
     }
 }
 
-int wq_version(void) { return 100; }
+int wq_version(void) { return 200; }
 
 int wq_packed_bytes(int bits, int K, int N, int group, size_t *wq_bytes, size_t *scale_bytes, size_t *zero_bytes)
 {
@@ -399,13 +413,15 @@ int wq_linear_noalloc(const uint16_t *x, int M, int K, const void *Wq, const voi
     return cuda_status(launch_gemv_sk_noalloc(a, d.sm_count, stream));
 }
 
-size_t wq_workspace_bytes(int M, int N, int max_split)
+size_t wq_workspace_bytes(int M, int K, int N, int max_split)
 {
-    if (M < 1 || N < 1 || max_split < 1)
+    if (M < 1 || K < 1 || N < 1 || max_split < 1)
         return 0;
     size_t b = std::max(ws_bytes(M, N, max_split), ws_bytes_gemm_sk(M, N));
     if (M <= 32)
         b = std::max(b, ws_bytes_gemv_sk(M, N));
+    if (M <= kI8MaxM && K <= kI8MaxK)
+        b = std::max(b, ws_bytes_gemm_i8(M, K, N));
     return b;
 }
 
@@ -455,6 +471,8 @@ int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
             cands.push_back({WQ_VARIANT_GEMM, s});
     for (int c : {1, 2})
         cands.push_back({WQ_VARIANT_GEMM_SK, c});
+    if (i8_fits(bits, M, K))
+        cands.push_back({WQ_VARIANT_I8MMA, 1});
 
     // Flush buffer larger than L2, so every timed call streams its weights
     // from HBM (the weights of a decode step are not L2-resident).
@@ -535,7 +553,7 @@ int wq_set_choice(int M, int K, int N, int bits, int group, int variant, int spl
     int st = current_device_info(&d);
     if (st != WQ_OK)
         return st;
-    if (!choice_valid(variant, split, M, K))
+    if (!choice_valid(variant, split, M, K, bits))
         return WQ_ERR_VARIANT;
     std::lock_guard<std::mutex> lk(g_mu);
     g_table[Key{device_key(d), M, K, N, bits, group}] = Choice{variant, split, 0.f};
@@ -605,7 +623,7 @@ int wq_load_tuning(const char *path)
         const int n = sscanf(rest, " %d %d %d %d %d %d %d %f %c", &M, &K, &N, &bits, &group, &variant, &split, &us,
                              &tail);
         if (n != 8 || check_weight_shape(bits, K, N, group) != WQ_OK || M < 1 || M > 128 ||
-            !choice_valid(variant, split, M, K)) {
+            !choice_valid(variant, split, M, K, bits)) {
             bad = true;
             break;
         }
@@ -647,11 +665,11 @@ int wq_dequant_debug(const void *Wq, const void *scales, const void *zeros, int 
 
 int wq_device_error(cudaStream_t stream)
 {
-    int a = 0, b = 0, c = 0;
+    int a = 0, b = 0, c = 0, e = 0;
     if (read_device_error(&a, stream) != cudaSuccess || read_gemv_sk_error(&b, stream) != cudaSuccess ||
-        read_gemm_sk_error(&c, stream) != cudaSuccess)
+        read_gemm_sk_error(&c, stream) != cudaSuccess || read_gemm_i8_error(&e, stream) != cudaSuccess)
         return WQ_ERR_CUDA;
-    return (a == 0 && b == 0 && c == 0) ? WQ_OK : WQ_ERR_TIMEOUT;
+    return (a == 0 && b == 0 && c == 0 && e == 0) ? WQ_OK : WQ_ERR_TIMEOUT;
 }
 
 } // extern "C"

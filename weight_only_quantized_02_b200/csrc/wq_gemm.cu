@@ -16,9 +16,10 @@
 //              and x as the B operand from shared memory; fp32 accumulators
 //              in tensor memory.
 //   warps 2-5  dequantize the block to exact integers in bf16 (INT4: q - z,
-//              INT8: q) and write it to tensor memory with tcgen05.st
-//              16x256b -- the packed tile is already that store's register
-//              layout.  The weights are never rounded: INT8's per-channel
+//              INT8: q) and write it to tensor memory: INT4 with tcgen05.st
+//              16x256b (the packed tile is that store's register layout),
+//              INT8 one row per thread with 32x32b (the swizzled block gives
+//              each thread its row's chunks without bank conflicts).  The weights are never rounded: INT8's per-channel
 //              scale is applied in the epilogue; INT4 accumulates each
 //              128-k group into one of two tensor-memory buffers and these
 //              warps fold s[row][g] * D_g into fp32 register totals one group
@@ -282,16 +283,20 @@ __global__ void __launch_bounds__(192, GemmTile<BITS, NT>::kMinBlocks)
                 ok = false;
                 break;
             }
-            uint4 w[2][TPR];
+            uint4 w[2][TPR]; // INT4: tiles of row blocks 2*quad + jj; INT8: chunk 4*jj + tt of this thread's row
             uint32_t zz[2][2];
             float s_mine = 0.f;
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
                 const int j = 2 * quad + jj;
 #pragma unroll
-                for (int tt = 0; tt < TPR; ++tt)
-                    w[jj][tt] = *reinterpret_cast<const uint4 *>(sW + st * WB + j * (TPR * kTileBytes) +
-                                                                 tt * kTileBytes + lane * 16);
+                for (int tt = 0; tt < TPR; ++tt) {
+                    if constexpr (BITS == 8)
+                        w[jj][tt] = *reinterpret_cast<const uint4 *>(sW + st * WB + int8_chunk_in_block(row, 4 * jj + tt));
+                    else
+                        w[jj][tt] = *reinterpret_cast<const uint4 *>(sW + st * WB + j * (TPR * kTileBytes) +
+                                                                     tt * kTileBytes + lane * 16);
+                }
                 if constexpr (BITS == 4) {
                     const uint8_t *z8 = sSZ + st * SZB + 256;
 #pragma unroll
@@ -312,20 +317,25 @@ __global__ void __launch_bounds__(192, GemmTile<BITS, NT>::kMinBlocks)
                 break;
             }
             tc_fence_after();
+            if constexpr (BITS == 4) {
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const uint32_t ta = tmem + ((uint32_t)(32 * quad + 16 * jj) << 16) + A0 + st * 64;
+                for (int jj = 0; jj < 2; ++jj) {
+                    const uint32_t ta = tmem + ((uint32_t)(32 * quad + 16 * jj) << 16) + A0 + st * 64;
 #pragma unroll
-                for (int tt = 0; tt < TPR; ++tt) {
-                    if constexpr (BITS == 4) {
+                    for (int tt = 0; tt < TPR; ++tt) {
                         uint32_t r[16];
                         int4_tile_regs(w[jj][tt], zz[jj][0], zz[jj][1], r);
                         tmem_st_16x256b_x4(ta + tt * 32, r);
-                    } else {
-                        uint32_t r[8];
-                        int8_tile_regs(w[jj][tt], r);
-                        tmem_st_16x256b_x2(ta + tt * 16, r);
                     }
+                }
+            } else {
+                // this thread's row, chunks 0..7 -> columns 8c .. 8c+7 of the stage
+                const uint32_t ta = tmem + tlane + A0 + st * 64;
+#pragma unroll
+                for (int cp = 0; cp < 4; ++cp) {
+                    uint32_t r[16];
+                    int8_chunks_regs(w[cp >> 1][2 * (cp & 1)], w[cp >> 1][2 * (cp & 1) + 1], r);
+                    tmem_st_32x32b_x16(ta + 16 * cp, r);
                 }
             }
             tmem_wait_st();

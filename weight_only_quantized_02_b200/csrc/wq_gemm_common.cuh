@@ -1,6 +1,7 @@
 // wq_gemm_common.cuh -- helpers shared by the tcgen05 GEMM kernels:
-// dequantization of a packed 16-row tile straight into the register layout
-// of a tcgen05.st 16x256b store (natural k order, exact integers as bf16).
+// dequantization of packed weights straight into the register layout of a
+// tensor-memory store (natural k order, exact integers as bf16): a 16-row
+// INT4 tile for tcgen05.st 16x256b, one row's INT8 chunks for 32x32b.
 #pragma once
 
 #include <cudaTypedefs.h>
@@ -32,19 +33,18 @@ __device__ __forceinline__ void int4_tile_regs(const uint4 &w, uint32_t zlo, uin
     r[15] = d(w.w, 3, zhi);
 }
 
-// One INT8 tile (16 rows x 32 k) -> 8 registers of a 16x256b.x2 store: exact q.
-__device__ __forceinline__ void int8_tile_regs(const uint4 &w, uint32_t (&r)[8])
+// Two INT8 chunks of one row (k = 16c .. 16c+31, natural order) -> the 16
+// registers of one thread's tcgen05.st 32x32b.x16 store: bf16 pairs of the
+// exact codes, column j = k pair (2j, 2j+1).
+__device__ __forceinline__ void int8_chunks_regs(const uint4 &w0, const uint4 &w1, uint32_t (&r)[16])
 {
-    const uint32_t ux = w.x ^ 0x80808080u, uy = w.y ^ 0x80808080u;
-    const uint32_t uz = w.z ^ 0x80808080u, uw = w.w ^ 0x80808080u;
-    r[0] = s8pair_bf16(ux, 0);
-    r[1] = s8pair_bf16(ux, 1);
-    r[2] = s8pair_bf16(uy, 0);
-    r[3] = s8pair_bf16(uy, 1);
-    r[4] = s8pair_bf16(uz, 0);
-    r[5] = s8pair_bf16(uz, 1);
-    r[6] = s8pair_bf16(uw, 0);
-    r[7] = s8pair_bf16(uw, 1);
+    const uint32_t v[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t u = v[i] ^ 0x80808080u;
+        r[2 * i] = s8pair_bf16(u, 0);
+        r[2 * i + 1] = s8pair_bf16(u, 1);
+    }
 }
 
 inline PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn()

@@ -14,9 +14,11 @@
 //              prefetched before the programmatic-launch wait, x after.
 //   warp 1     allocates tensor memory; one thread issues tcgen05.mma with
 //              the dequantized tile as the A operand from tensor memory.
-//   warps 2-9  two dequant warps per tensor-memory lane quadrant, one per
-//              16-row block: exact integers (INT4 q - z, INT8 q) as bf16 into
-//              tensor memory with tcgen05.st 16x256b.  One unit behind the
+//   warps 2-9  two dequant warps per tensor-memory lane quadrant: exact
+//              integers (INT4 q - z, INT8 q) as bf16 into tensor memory.
+//              INT4: one 16-row block per warp, tcgen05.st 16x256b; INT8:
+//              one row per thread, half of the block's k each, 32x32b.
+//              One unit behind the
 //              MMA they retire finished work: INT4 folds s[row][g] * D_g of
 //              every group into fp32 register totals (two group accumulators
 //              in tensor memory, double-buffered); INT8 reads a panel's
@@ -240,7 +242,7 @@ __global__ void __launch_bounds__(kGskThreads) __maxnreg__((GskCfg<BITS, NT>::kM
         pdl_wait(); // y and the workspace may still be in use by the preceding kernel
         const int dw = warp - 2;          // 0..7
         const int q = warp & 3, h = dw >> 2;
-        const int j = 2 * q + h;          // 16-row block this warp dequantizes
+        const int j = 2 * q + h;          // INT4: 16-row block this warp dequantizes
         const int g = lane >> 2;
         const int r = 32 * q + lane;      // output row (in the panel) this thread retires
         const uint32_t tq = (uint32_t)(32 * q) << 16;
@@ -380,11 +382,15 @@ __global__ void __launch_bounds__(kGskThreads) __maxnreg__((GskCfg<BITS, NT>::kM
                 ok = false;
                 break;
             }
-            uint4 w[TPR];
+            uint4 w[TPR]; // INT4: tiles of row block j; INT8: chunks 4h .. 4h+3 of row r
 #pragma unroll
-            for (int tt = 0; tt < TPR; ++tt)
-                w[tt] = *reinterpret_cast<const uint4 *>(sW + st * WB + j * (TPR * kTileBytes) + tt * kTileBytes +
-                                                         lane * 16);
+            for (int tt = 0; tt < TPR; ++tt) {
+                if constexpr (BITS == 8)
+                    w[tt] = *reinterpret_cast<const uint4 *>(sW + st * WB + int8_chunk_in_block(r, 4 * h + tt));
+                else
+                    w[tt] = *reinterpret_cast<const uint4 *>(sW + st * WB + j * (TPR * kTileBytes) +
+                                                             tt * kTileBytes + lane * 16);
+            }
             uint32_t zlo = 0, zhi = 0;
             float s_mine = 0.f;
             if constexpr (BITS == 4) {
@@ -404,17 +410,22 @@ __global__ void __launch_bounds__(kGskThreads) __maxnreg__((GskCfg<BITS, NT>::kM
                 break;
             }
             tc_fence_after();
-            const uint32_t ta = tmem + ((uint32_t)(32 * q + 16 * h) << 16) + A0 + st * 64;
+            if constexpr (BITS == 4) {
+                const uint32_t ta = tmem + ((uint32_t)(32 * q + 16 * h) << 16) + A0 + st * 64;
 #pragma unroll
-            for (int tt = 0; tt < TPR; ++tt) {
-                if constexpr (BITS == 4) {
+                for (int tt = 0; tt < TPR; ++tt) {
                     uint32_t rr[16];
                     int4_tile_regs(w[tt], zlo, zhi, rr);
                     tmem_st_16x256b_x4(ta + tt * 32, rr);
-                } else {
-                    uint32_t rr[8];
-                    int8_tile_regs(w[tt], rr);
-                    tmem_st_16x256b_x2(ta + tt * 16, rr);
+                }
+            } else {
+                // row r, chunks 4h .. 4h+3 -> columns 32h .. 32h+31 of the stage
+                const uint32_t ta = tmem + tq + A0 + st * 64 + 32 * h;
+#pragma unroll
+                for (int cp = 0; cp < 2; ++cp) {
+                    uint32_t rr[16];
+                    int8_chunks_regs(w[2 * cp], w[2 * cp + 1], rr);
+                    tmem_st_32x32b_x16(ta + 16 * cp, rr);
                 }
             }
             tmem_wait_st();

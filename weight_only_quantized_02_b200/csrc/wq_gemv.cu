@@ -2,13 +2,12 @@
 //
 // Register-level dequantization with 128-bit weight loads and no shared
 // memory on the weight path (the "BitBLAS-style GEMV" row of the tileInfer
-// README, Features table).  Each warp streams the 512-byte tiles of one
-// 16-row block over a K slice; every lane's 16 bytes are already an
-// m16n8k16 A fragment (see wq_layout.h), so the unpacked integers go straight
-// into mma.sync with the activations as the 8-token B operand and fp32
-// accumulators.  For W4A16 the MMA sees exact (q - z) integers and the bf16
-// group scale is applied in fp32 after each group of 128 k, so the weights
-// are never rounded.  For W8A16 the per-channel scale is applied once in the
+// README, Features table).  Each warp streams one 16-row block over a K
+// slice; every lane's 16-byte loads unpack straight into m16n8k16 A
+// fragments (see wq_layout.h), which go into mma.sync with the activations
+// as the 8-token B operand and fp32 accumulators.  For W4A16 the MMA sees
+// exact (q - z) integers and the bf16 group scale is applied in fp32 after
+// each group of 128 k, so the weights are never rounded.  For W8A16 the per-channel scale is applied once in the
 // epilogue.  K slices of one row block are summed across warps through
 // shared memory in a fixed order (deterministic).
 #include <cstdint>
@@ -42,24 +41,26 @@ __device__ __forceinline__ void load_x_frag(const GemvParams &p, int g, int k, u
     }
 }
 
-// One INT8 tile (16 rows x 32 k): two MMAs per 8-token tile.
+// One INT8 chunk pair: this lane's 16 consecutive k (kc .. kc+15) of rows g
+// (wa) and g+8 (wb).  Step i = 0..3 is an m16n8k16 MMA whose k-slots 2t,
+// 2t+1, 2t+8, 2t+9 take k = kc+4i .. kc+4i+3; the activations of the same k
+// are xv[mt] (kc .. kc+7) and xw[mt] (kc+8 .. kc+15) of token row 8*mt + g.
 template <int MT>
-__device__ __forceinline__ void int8_tile(const GemvParams &p, const uint4 &w, int kt_base, int g, int t,
-                                          float (&acc)[MT][4])
+__device__ __forceinline__ void int8_chunk(const uint4 &wa, const uint4 &wb, const uint4 (&xv)[MT],
+                                           const uint4 (&xw)[MT], float (&acc)[MT][4])
 {
-    const uint32_t ux = w.x ^ 0x80808080u, uy = w.y ^ 0x80808080u;
-    const uint32_t uz = w.z ^ 0x80808080u, uw = w.w ^ 0x80808080u;
-    const uint32_t a0 = s8pair_bf16(ux, 0), a1 = s8pair_bf16(uy, 0);
-    const uint32_t a2 = s8pair_bf16(ux, 1), a3 = s8pair_bf16(uy, 1);
-    const uint32_t b0 = s8pair_bf16(uz, 0), b1 = s8pair_bf16(uw, 0);
-    const uint32_t b2 = s8pair_bf16(uz, 1), b3 = s8pair_bf16(uw, 1);
-    uint2 xa[MT], xb[MT];
-    load_x_frag<MT>(p, g, kt_base + 4 * t, xa);
-    load_x_frag<MT>(p, g, kt_base + 16 + 4 * t, xb);
+    const uint32_t ra[4] = {wa.x, wa.y, wa.z, wa.w}, rb[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-        mma_bf16_16816(acc[mt], a0, a1, a2, a3, xa[mt].x, xa[mt].y);
-        mma_bf16_16816(acc[mt], b0, b1, b2, b3, xb[mt].x, xb[mt].y);
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t ua = ra[i] ^ 0x80808080u, ub = rb[i] ^ 0x80808080u;
+        const uint32_t a0 = s8pair_bf16(ua, 0), a2 = s8pair_bf16(ua, 1);
+        const uint32_t a1 = s8pair_bf16(ub, 0), a3 = s8pair_bf16(ub, 1);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const uint4 &xx = i < 2 ? xv[mt] : xw[mt];
+            const uint32_t b0 = (i & 1) ? xx.z : xx.x, b1 = (i & 1) ? xx.w : xx.y;
+            mma_bf16_16816(acc[mt], a0, a1, a2, a3, b0, b1);
+        }
     }
 }
 
@@ -91,29 +92,54 @@ __device__ __forceinline__ void int4_tile(const GemvParams &p, const uint4 &w, i
     }
 }
 
+// INT8: the K range of this slice is a run of 64-k half-blocks [h0, h1);
+// in half-block hb lane (g, t) takes chunk c = 4*(hb%2) + t of rows g and g+8.
 template <int MT>
-__device__ __forceinline__ void gemv_int8_slice(const GemvParams &p, int rb, int kt0, int kt1, int lane,
+__device__ __forceinline__ void gemv_int8_slice(const GemvParams &p, int rb, int h0, int h1, int lane,
                                                 float (&acc)[MT][4])
 {
-    constexpr int U = 4;
+    constexpr int U = 2;
     const int g = lane >> 2, t = lane & 3;
-    const uint8_t *base = p.wq + 16 * lane;
-    uint4 cur[U], nxt[U];
+    const int pnl = rb >> 3, r = 16 * (rb & 7) + g; // row of the panel (and r + 8)
+    const uint8_t *panel = p.wq + p.sh.block_offset(pnl, 0);
+    auto load_w = [&](int hb, uint4 &wa, uint4 &wb) {
+        if (hb < h1) {
+            const uint8_t *src = panel + (size_t)(hb >> 1) * 16384 + int8_chunk_in_block(r, 4 * (hb & 1) + t);
+            wa = ldg_stream(src);
+            wb = ldg_stream(src + 1024);
+        } else {
+            wa = wb = make_uint4(0, 0, 0, 0);
+        }
+    };
+    uint4 ca[U], cb[U], na[U], nb[U];
 #pragma unroll
     for (int u = 0; u < U; ++u)
-        cur[u] = (kt0 + u < kt1) ? ldg_stream(base + p.sh.tile_offset(rb, kt0 + u)) : make_uint4(0, 0, 0, 0);
-    for (int kt = kt0; kt < kt1; kt += U) {
+        load_w(h0 + u, ca[u], cb[u]);
+    for (int hb = h0; hb < h1; hb += U) {
 #pragma unroll
         for (int u = 0; u < U; ++u)
-            nxt[u] = (kt + U + u < kt1) ? ldg_stream(base + p.sh.tile_offset(rb, kt + U + u))
-                                        : make_uint4(0, 0, 0, 0);
+            load_w(hb + U + u, na[u], nb[u]);
 #pragma unroll
-        for (int u = 0; u < U; ++u)
-            if (kt + u < kt1)
-                int8_tile<MT>(p, cur[u], 32 * (kt + u), g, t, acc);
+        for (int u = 0; u < U; ++u) {
+            const int kc = 64 * (hb + u) + 16 * t;
+            if (hb + u < h1) {
+                uint4 xv[MT], xw[MT];
 #pragma unroll
-        for (int u = 0; u < U; ++u)
-            cur[u] = nxt[u];
+                for (int mt = 0; mt < MT; ++mt) {
+                    const int m = 8 * mt + g;
+                    const bool ok = m < p.M && kc < p.K; // k past K: zero weights, keep x finite
+                    const uint16_t *xr = p.x + (size_t)m * p.K + kc;
+                    xv[mt] = ok ? ldg_keep4(xr) : make_uint4(0, 0, 0, 0);
+                    xw[mt] = ok ? ldg_keep4(xr + 8) : make_uint4(0, 0, 0, 0);
+                }
+                int8_chunk<MT>(ca[u], cb[u], xv, xw, acc);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            ca[u] = na[u];
+            cb[u] = nb[u];
+        }
     }
 }
 
@@ -206,7 +232,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvParams 
             acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
         if (rb < nrb) {
             if constexpr (BITS == 8) {
-                const int T = p.K / 32;
+                const int T = (p.K + 63) / 64;
                 gemv_int8_slice<MT>(p, rb, (int)((long long)T * ks_i / ks), (int)((long long)T * (ks_i + 1) / ks),
                                     lane, acc);
             } else {

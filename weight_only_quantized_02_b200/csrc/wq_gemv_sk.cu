@@ -43,8 +43,11 @@ struct GemvSkParams {
 };
 
 // Ring stage: packed weights of the unit, INT4 scales/zeros, and the unit's
-// activation slice x[0..M)[128 k] (one 256-byte bulk copy per token row,
-// rows 288 bytes apart so the eight rows a warp reads hit distinct banks).
+// activation slice x[0..M)[128 k] (one 256-byte bulk copy per token row).
+// The row stride makes a warp's activation reads conflict-free: INT4 lanes
+// read 8 bytes at row g, column 4t (288 = 72 words: rows 8 banks apart);
+// INT8 lanes read 16 bytes at row g, column 16t (272 = 68 words: the two
+// rows of a quarter-warp 4 banks apart).
 template <int BITS, int MT, int OCC>
 struct SkCfg {
     static constexpr int kTPB = BITS == 4 ? 2 : 4;   // tiles per 16-row block per unit
@@ -52,7 +55,7 @@ struct SkCfg {
     static constexpr int kPBB = 8 * kRBB;            // packed bytes per unit
     static constexpr int kSZB = BITS == 4 ? 512 : 0; // scales 256 + zeros 64, padded
     static constexpr int kSZTx = BITS == 4 ? 320 : 0;
-    static constexpr int kXRow = 288;                // smem stride of one token row (256 B + pad)
+    static constexpr int kXRow = BITS == 8 ? 272 : 288; // smem stride of one token row (256 B + pad)
     static constexpr int kXB = 8 * MT * kXRow;
     static constexpr int kStageBytes = kPBB + kSZB + kXB;
     // ring sized so OCC CTAs fit in an SM's 228 KB of shared memory
@@ -90,21 +93,26 @@ __device__ __forceinline__ void s8quad_bf16(uint32_t w, uint32_t &lo, uint32_t &
     hi = __byte_perm((uint32_t)d23, (uint32_t)(d23 >> 32), 0x7632u);
 }
 
-template <int MT, int XROW>
-__device__ __forceinline__ void sk_int8_tile(const uint4 &w, const uint8_t *xs, int kt, float (&acc)[MT][4])
+// One INT8 chunk pair of the stage: lane (g, t) holds k = kc .. kc+15 of
+// rows g (wa) and g+8 (wb); step i = 0..3 is an m16n8k16 MMA whose k-slots
+// 2t, 2t+1, 2t+8, 2t+9 take k = kc+4i .. kc+4i+3.  xv / xw: the same k of
+// token row 8*mt + g (kc .. kc+7 and kc+8 .. kc+15).
+template <int MT>
+__device__ __forceinline__ void sk_int8_chunk(const uint4 &wa, const uint4 &wb, const uint4 (&xv)[MT],
+                                              const uint4 (&xw)[MT], float (&acc)[MT][4])
 {
-    uint32_t a0, a2, a1, a3, b0, b2, b1, b3;
-    s8quad_bf16(w.x, a0, a2); // row g,   k 4t..4t+3
-    s8quad_bf16(w.y, a1, a3); // row g+8
-    s8quad_bf16(w.z, b0, b2); // row g,   k 16+4t..
-    s8quad_bf16(w.w, b1, b3); // row g+8
-    uint2 xa[MT], xb[MT];
-    x_frags<MT, XROW>(xs, kt, xa);
-    x_frags<MT, XROW>(xs, kt + 16, xb);
+    const uint32_t ra[4] = {wa.x, wa.y, wa.z, wa.w}, rb[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-        mma_bf16_16816(acc[mt], a0, a1, a2, a3, xa[mt].x, xa[mt].y);
-        mma_bf16_16816(acc[mt], b0, b1, b2, b3, xb[mt].x, xb[mt].y);
+    for (int i = 0; i < 4; ++i) {
+        uint32_t a0, a2, a1, a3;
+        s8quad_bf16(ra[i], a0, a2);
+        s8quad_bf16(rb[i], a1, a3);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const uint4 &xx = i < 2 ? xv[mt] : xw[mt];
+            const uint32_t b0 = (i & 1) ? xx.z : xx.x, b1 = (i & 1) ? xx.w : xx.y;
+            mma_bf16_16816(acc[mt], a0, a1, a2, a3, b0, b1);
+        }
     }
 }
 
@@ -223,7 +231,8 @@ __global__ void __launch_bounds__(kSkThreads, OCC) gemv_sk_kernel(const GemvSkPa
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
             acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-        const int xoff = C::kPBB + C::kSZB + g * C::kXRow + 8 * t; // row g, column 4t
+        // activations of this lane: row g, column 4t (INT4) or 16t (INT8)
+        const int xoff = C::kPBB + C::kSZB + g * C::kXRow + (BITS == 8 ? 32 : 8) * t;
 
         // write this warp's rows of panel pnl: to y if this CTA covered the
         // whole panel, else as a partial + ticket (last arriver reduces).
@@ -333,24 +342,31 @@ __global__ void __launch_bounds__(kSkThreads, OCC) gemv_sk_kernel(const GemvSkPa
                 ok = false;
             const uint8_t *stage = ring + st * C::kStageBytes;
             if (ok) {
-                uint4 w[C::kTPB];
-#pragma unroll
-                for (int tt = 0; tt < C::kTPB; ++tt)
-                    w[tt] = *reinterpret_cast<const uint4 *>(stage + j * C::kRBB + tt * kTileBytes + lane * 16);
                 const uint8_t *xs = stage + xoff;
                 if constexpr (BITS == 8) {
+                    // rows 16j + g and 16j + 8 + g: 8-row groups 2j and 2j + 1, row g of each
+                    const uint8_t *wr = stage + (2 * j) * 1024 + g * 128;
                     const int kleft = p.K - kb * kBlockK;
-                    if (kleft >= kBlockK) {
 #pragma unroll
-                        for (int tt = 0; tt < 4; ++tt)
-                            sk_int8_tile<MT, C::kXRow>(w[tt], xs, 32 * tt, acc);
-                    } else { // ragged last block of K
+                    for (int h = 0; h < 2; ++h) {
+                        const int cc = t + 4 * h;
+                        const uint4 wa = *reinterpret_cast<const uint4 *>(wr + ((cc ^ g) << 4));
+                        const uint4 wb = *reinterpret_cast<const uint4 *>(wr + 1024 + ((cc ^ g) << 4));
+                        const bool kin = 16 * cc < kleft; // chunks past K: zero weights, activations not staged
+                        uint4 xv[MT], xw[MT];
 #pragma unroll
-                        for (int tt = 0; tt < 4; ++tt)
-                            if (32 * tt < kleft)
-                                sk_int8_tile<MT, C::kXRow>(w[tt], xs, 32 * tt, acc);
+                        for (int mt = 0; mt < MT; ++mt) {
+                            const uint8_t *xp = xs + mt * 8 * C::kXRow + 128 * h;
+                            xv[mt] = kin ? *reinterpret_cast<const uint4 *>(xp) : make_uint4(0, 0, 0, 0);
+                            xw[mt] = kin ? *reinterpret_cast<const uint4 *>(xp + 16) : make_uint4(0, 0, 0, 0);
+                        }
+                        sk_int8_chunk<MT>(wa, wb, xv, xw, acc);
                     }
                 } else {
+                    uint4 w[C::kTPB];
+#pragma unroll
+                    for (int tt = 0; tt < C::kTPB; ++tt)
+                        w[tt] = *reinterpret_cast<const uint4 *>(stage + j * C::kRBB + tt * kTileBytes + lane * 16);
                     const uint16_t *s16 = reinterpret_cast<const uint16_t *>(stage + C::kPBB);
                     const uint8_t *z8 = stage + C::kPBB + 256;
                     const int r = 16 * j + g;

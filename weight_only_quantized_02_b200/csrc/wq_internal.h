@@ -38,6 +38,15 @@ inline size_t ws_bytes_gemv_sk(int M, int N)
     return ws_counter_bytes(N) + (size_t)kSkMaxCtas * 2 * 128 * tok * sizeof(float);
 }
 
+// Integer tensor-core GEMM (INT8 only): M <= kI8MaxM, K <= kI8MaxK, at most
+// kI8MaxCtas persistent CTAs.  Workspace: [tickets][exponents 256 B]
+// [digit blocks KB x NR x 128][int32 partials kI8MaxCtas x 2 x NR x 128].
+constexpr int kI8MaxM = 64;
+constexpr int kI8MaxK = 65536;
+constexpr int kI8MaxCtas = 160;
+int i8_digit_rows(int M);
+size_t ws_bytes_gemm_i8(int M, int K, int N);
+
 cudaError_t launch_quantize_int8(const float *W, int K, int N, int8_t *q, uint16_t *s, cudaStream_t st);
 cudaError_t launch_quantize_int4(const float *W, int K, int N, uint32_t *q, uint16_t *s, uint32_t *z,
                                  cudaStream_t st);
@@ -69,6 +78,10 @@ cudaError_t launch_gemm(const LinearArgs &a, int split, void *ws, int sm_count, 
 // Stream-K GEMM: ctas_per_sm = 0 (default) or 1/2; ws >= ws_bytes_gemm_sk.
 cudaError_t launch_gemm_sk(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st);
 cudaError_t read_gemm_sk_error(int *code, cudaStream_t st);
+
+// Integer tensor-core GEMM: ws >= ws_bytes_gemm_i8 (always needed).
+cudaError_t launch_gemm_i8(const LinearArgs &a, void *ws, int sm_count, cudaStream_t st);
+cudaError_t read_gemm_i8_error(int *code, cudaStream_t st);
 
 // Reads and clears the device error word of the current device.
 cudaError_t read_device_error(int *code, cudaStream_t st);

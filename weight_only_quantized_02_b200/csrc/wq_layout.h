@@ -2,13 +2,25 @@
 // and the GEMM.  Host and device.
 //
 // Weights of shape [N][K] are cut into 128-row panels p and 128-k blocks kb.
-// A (panel, k-block) block is contiguous: 8 row-blocks j of 16 rows, each
-// holding `tiles_per_block` tiles of 512 bytes (INT4: 2 tiles of 64 k;
-// INT8: 4 tiles of 32 k).  Inside a tile, lane l = 4g + t (g = l/4, t = l%4)
-// owns the 16 bytes at offset 16 l:
+// A (panel, k-block) block is contiguous (16 KB INT8, 8 KB INT4), blocks in
+// panel-major order, so a panel's whole K range is one contiguous run.
 //
-//   INT8 tile (k base kt):  .x = q[g][kt+4t .. +4]      .y = q[g+8][kt+4t .. +4]
-//                           .z = q[g][kt+16+4t .. +4]   .w = q[g+8][kt+16+4t .. +4]
+// INT8 block: the tcgen05 K-major canonical layout with 128-byte swizzle.
+// Row r (0..127) of the block sits at (r/8)*1024 + (r%8)*128; its 16-byte
+// chunk c (k = 16c .. 16c+15, natural order) sits at chunk slot c ^ (r%8) of
+// that 128-byte row.  A 1-D bulk copy of the block into 1024-byte aligned
+// shared memory is therefore directly the A operand of a tcgen05.mma
+// kind::i8 (8-row groups 1024 B apart, K advanced 32 B per instruction).
+// The same bytes serve the register paths: one thread per row reads its
+// 16-byte chunks without bank conflicts (eight consecutive rows hit the
+// eight chunk slots), and an mma.sync lane (g, t) reads chunk c of rows g
+// and g+8, whose four 32-bit words feed four m16n8k16 steps (k-slots 2t,
+// 2t+1, 2t+8, 2t+9 taken from a run of four consecutive k).
+//
+// INT4 block: 8 row-blocks j of 16 rows, each holding 2 tiles of 512 bytes
+// (64 k each).  Inside a tile, lane l = 4g + t (g = l/4, t = l%4) owns the
+// 16 bytes at offset 16 l:
+//
 //   INT4 tile (k base kt):  .x = row g,   runs a = kt+4t, b = kt+16+4t
 //                           .y = row g+8, runs a, b
 //                           .z = row g,   runs c = kt+32+4t, d = kt+48+4t
@@ -20,10 +32,10 @@
 // This is the m16n8k16 mma.sync A fragment of a 16-row block (rows g, g+8,
 // k-slots 2t, 2t+1, 2t+8, 2t+9 taken from a run of four consecutive k), and
 // also the register layout of a tcgen05.st 16x256b store of the same rows
-// into tensor memory in natural k order.  One packed buffer therefore feeds
-// both kernel families, and a warp's 128-bit load of a tile is one
-// contiguous 512-byte segment.
+// into tensor memory in natural k order; a warp's 128-bit load of a tile is
+// one contiguous 512-byte segment.
 //
+// Rows past N and k past K are zero in both formats.
 // Scales: INT8 bf16 [P*128] (s[n], zero past N).  INT4 bf16 [P][K/128][128].
 // Zeros (INT4): [P][K/128][128 nibbles = 64 bytes], row i at nibble i
 // (low nibble first).  A 64-byte trailer follows the packed weights.
@@ -45,7 +57,7 @@ constexpr int kBlockK = 128;
 constexpr int kTileBytes = 512;
 constexpr int kTrailerBytes = 64;
 constexpr uint32_t kMagic = 0x32425157u; // "WQB2"
-constexpr uint32_t kLayoutVersion = 1;
+constexpr uint32_t kLayoutVersion = 2;
 
 struct Shape {
     int bits;  // 4 or 8
@@ -65,7 +77,7 @@ struct Shape {
                          : (size_t)panels() * kblocks() * kPanelRows * 2;
     }
     WQ_HD size_t zero_bytes() const { return bits == 8 ? 0 : (size_t)panels() * kblocks() * 64; }
-    // byte offset of tile (row-block rb = 16-row index, k tile index kt)
+    // INT4: byte offset of tile (row-block rb = 16-row index, k tile index kt)
     WQ_HD size_t tile_offset(int rb, int kt) const
     {
         const int p = rb >> 3, j = rb & 7;
@@ -75,6 +87,16 @@ struct Shape {
     }
     WQ_HD size_t block_offset(int p, int kb) const { return (size_t)(p * kblocks() + kb) * block_bytes(); }
 };
+
+// INT8: byte offset of element (r, kk) inside its block (r = row in the
+// panel 0..127, kk = k in the block 0..127).
+WQ_HD int int8_in_block(int r, int kk)
+{
+    return (r >> 3) * 1024 + (r & 7) * 128 + ((((kk >> 4) ^ (r & 7)) & 7) << 4) + (kk & 15);
+}
+
+// INT8: byte offset of the 16-byte chunk c of row r inside its block.
+WQ_HD int int8_chunk_in_block(int r, int c) { return (r >> 3) * 1024 + (r & 7) * 128 + (((c ^ (r & 7)) & 7) << 4); }
 
 struct Trailer {
     uint32_t magic, version, bits, K, N, group, layout_bytes_lo, layout_bytes_hi;

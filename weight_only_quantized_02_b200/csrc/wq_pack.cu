@@ -148,25 +148,20 @@ __global__ void pack_int8_kernel(const int8_t *__restrict__ q, int K, int N, uin
     const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= n_vec)
         return;
-    const int vec_per_block = sh.block_bytes() / 16, vec_per_rb = sh.rb_bytes() / 16;
-    const size_t b = idx / vec_per_block;
-    const int u = (int)(idx % vec_per_block);
+    // 16-byte vector u of block b: row r = u / 8 of the panel, chunk slot u % 8
+    // holds chunk c = slot ^ (r % 8), i.e. k = 16c .. 16c+15 of the block
+    const size_t b = idx / 1024;
+    const int u = (int)(idx % 1024);
     const int p = (int)(b / sh.kblocks()), kb = (int)(b % sh.kblocks());
-    const int j = u / vec_per_rb, rem = u % vec_per_rb;
-    const int t = rem / 32, l = rem % 32, g = l >> 2, tt = l & 3;
-    const int n0 = p * kPanelRows + 16 * j;
-    const int kt = kb * kBlockK + 32 * t;
-    auto run = [&](int row, int k) -> uint32_t {
+    const int r = u >> 3, c = (u & 7) ^ (r & 7);
+    const int row = p * kPanelRows + r;
+    const int k0 = kb * kBlockK + 16 * c;
+    auto run = [&](int k) -> uint32_t {
         if (row >= N || k >= K)
             return 0u;
         return *reinterpret_cast<const uint32_t *>(q + (size_t)row * K + k);
     };
-    uint4 v;
-    v.x = run(n0 + g, kt + 4 * tt);
-    v.y = run(n0 + g + 8, kt + 4 * tt);
-    v.z = run(n0 + g, kt + 16 + 4 * tt);
-    v.w = run(n0 + g + 8, kt + 16 + 4 * tt);
-    out[idx] = v;
+    out[idx] = make_uint4(run(k0), run(k0 + 4), run(k0 + 8), run(k0 + 12));
 }
 
 __device__ __forceinline__ uint32_t canon_nibble(const uint32_t *q, int K, int row, int k)
@@ -262,15 +257,14 @@ __global__ void write_trailer_kernel(uint8_t *wq, Shape sh)
 // ---------------------------------------------------------------------------
 __device__ int packed_q(const uint8_t *wq, const Shape &sh, int n, int k)
 {
+    if (sh.bits == 8) {
+        const int p = n / kPanelRows, kb = k / kBlockK;
+        return (int)(int8_t)wq[sh.block_offset(p, kb) + int8_in_block(n % kPanelRows, k % kBlockK)];
+    }
     const int rb = n >> 4, r = n & 15, g = r & 7, hi = r >> 3;
     const int tk = sh.tile_k();
     const int kt = k / tk, kk = k % tk;
     const uint8_t *tile = wq + sh.tile_offset(rb, kt);
-    if (sh.bits == 8) {
-        const int run = kk / 16, t = (kk % 16) / 4, e = kk % 4;
-        const int comp = run * 2 + hi;
-        return (int)(int8_t)tile[16 * (4 * g + t) + 4 * comp + e];
-    }
     const int half = kk / 32, hk = kk % 32, run = hk / 16, t = (hk % 16) / 4;
     const int e = run * 4 + hk % 4;
     const int comp = half * 2 + hi;

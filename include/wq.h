@@ -25,8 +25,10 @@
  *     Mit han lab Llm awq Kernel Selection Thresholds, The Insight).
  *   - for W8A16, M <= 64: the integer tensor cores (tcgen05 kind::i8) on the
  *     raw INT8 codes. The per-channel scale factors out of the k sum, x is
- *     written per token row as an integer X = round(x * 2^e) with |X| < 2^22
- *     (three base-256 digits), the sums over k are exact int32, and
+ *     written per token row as an integer X = round(x * 2^e), ties to even,
+ *     with e = min(21 - E, 127) for 2^E <= max|x| < 2^(E+1), so |X| < 2^22
+ *     (three base-256 digits) and every element within 2^14 of the row's
+ *     largest is exact. The sums over k are exact int32, and
  *     y = s * 2^-e * sum is formed in binary64 before the bf16 rounding.
  * A per-(M,K,N,bits,group) dispatcher picks the kernel and split factor. It
  * starts from an untuned rule (W8A16 within the integer path's limits -> the
@@ -214,8 +216,7 @@ int wq_linear_noalloc(const uint16_t *x, int M, int K, const void *Wq, const voi
  * max_split: enough for every variant of that shape. It holds eight ticket
  * counters per 128-channel panel and the largest of the GEMM's fp32
  * partials [split][M][N], the stream-K kernels' per-CTA panel partials, and
- * the integer path's activation digits (ceil(K/128) x 128 x up to 192
- * bytes) with its int32 per-CTA partials. Returns 0 for M, K, N or
+ * the integer path's int32 per-CTA partials. Returns 0 for M, K, N or
  * max_split < 1. Host. */
 size_t wq_workspace_bytes(int M, int K, int N, int max_split);
 

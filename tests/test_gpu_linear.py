@@ -81,15 +81,19 @@ def test_deterministic_and_splits_agree(weight, ws):
 
 
 def test_repeated_dispatch_resets_tickets(weight, ws):
-    """Many split-K calls in a row reuse the workspace tickets; each must
-    leave them at zero for the next (different split, different M)."""
+    """Many split-K and stream-K calls in a row reuse the workspace counters;
+    each must leave them at zero for the next (different variant, split, M)."""
     bits, K, N, pw, canon = weight
-    for M, split in [(16, 2), (16, 8), (40, 4), (128, 9), (16, 2)]:
+    runs = [(GEMM, 16, 2), (GEMM, 16, 8), (GEMM_SK, 40, 2), (GEMV, 5, 3), (GEMM, 40, 4), (GEMM, 128, 9)]
+    if bits == 8:
+        runs += [(I8, 5, 1), (I8, 40, 1), (GEMV, 3, 2), (I8, 1, 1)]
+    runs += [(GEMM, 16, 2)]
+    for variant, M, split in runs:
         x = gen.x_bf16(M, K)
-        y = wq.wq_linear_forced(bf16_dev(x), pw, GEMM, split)
-        assert_parity(y_host(y), oracle_linear(x, canon, bits), f"M={M} split={split}")
-    ticket = ws[: 32 * ((N + 127) // 128)].view(torch.int32)
-    assert int(ticket.abs().sum()) == 0
+        y = wq.wq_linear_forced(bf16_dev(x), pw, variant, split)
+        assert_parity(y_host(y), oracle_linear(x, canon, bits), f"variant={variant} M={M} split={split}")
+    counters = ws[: 4 * (8 * ((N + 127) // 128) + 2)].view(torch.int32)  # tickets + the integer path's grid counters
+    assert int(counters.abs().sum()) == 0
 
 
 # ---------------------------------------------------------------------------

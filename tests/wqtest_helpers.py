@@ -94,9 +94,9 @@ def i8_fixed_point(x_bits: np.ndarray) -> np.ndarray:
     """The activations as the integer tensor-core path represents them, from
     the library's stated contract (include/wq.h): per token row, e = 21 - E
     with E the binary exponent of the row's largest magnitude (2^E <= max|x|
-    < 2^(E+1); subnormal rows use E = -126), and x -> round(x * 2^e) * 2^-e,
-    ties to even.  Every element within 2^14 of the row's largest is
-    unchanged.  Returns binary64 values."""
+    < 2^(E+1); subnormal rows use E = -126), at most 127, and
+    x -> round(x * 2^e) * 2^-e, ties to even.  Every element within 2^14 of
+    the row's largest is unchanged.  Returns binary64 values."""
     x = oracle.bf16_to_f64(x_bits)
     out = np.zeros_like(x)
     for m in range(x.shape[0]):
@@ -104,6 +104,6 @@ def i8_fixed_point(x_bits: np.ndarray) -> np.ndarray:
         if amax == 0.0:
             continue
         E = max(int(np.frexp(amax)[1]) - 1, -126)  # amax = f * 2^(E+1), f in [0.5, 1)
-        e = 21 - E
+        e = min(21 - E, 127)
         out[m] = np.rint(np.ldexp(x[m], e)) * np.ldexp(1.0, -e)  # exact: |X| < 2^22
     return out

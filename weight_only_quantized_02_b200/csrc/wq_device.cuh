@@ -339,6 +339,17 @@ __device__ __forceinline__ uint32_t ticket_take(uint32_t *counter)
     return t;
 }
 
+// Ticket with one acquire-release atomic at GPU scope: the release orders the
+// partials the warp stored before a __syncwarp (cumulativity through the
+// warp barrier), the acquire lets the last arriver read every other
+// contributor's partials after a __syncwarp.  Called by one lane.
+__device__ __forceinline__ uint32_t ticket_take_acq_rel(uint32_t *counter)
+{
+    uint32_t t;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(counter) : "memory");
+    return t;
+}
+
 // ---------------------------------------------------------------------------
 // Stream-K partition: U units cut into G contiguous ranges [start(c),
 // start(c+1)); a panel of consecutive units may span several ranges.

@@ -1,43 +1,52 @@
 // wq_gemm_i8.cu -- W8A16 on the integer tensor cores: tcgen05.mma kind::i8
-// straight on the packed INT8 codes, no dequantization instructions at all.
+// straight on the packed INT8 codes, no weight dequantization at all.
 //
 // The per-channel scale of W8A16 factors out of the k sum ("Per-channel
 // W8A16 quantization", tileInfer README, Features table):
 //     y[m][n] = s[n] * sum_k q[n][k] * x[m][k]
-// so the sum over k can run on integers.  A small pre-pass turns every
-// token row of x into integers X = round(x * 2^e_m), with e_m chosen from
-// the row's largest magnitude so that |X| < 2^22 (every element within 2^14
-// of the row's largest is exact; smaller ones are rounded to nearest, ties
-// to even, at 2^-e_m), and writes X as three signed base-256 digits
+// so the sum over k can run on integers.  Every token row of x becomes
+// integers X = round(x * 2^e_m), e_m chosen from the row's largest
+// magnitude so that |X| < 2^22 (every element within 2^14 of the row's
+// largest is exact; smaller ones are rounded to nearest, ties to even, at
+// 2^-e_m), and X is written as three signed base-256 digits
 //     X = d0 + 256 d1 + 65536 d2,   d0, d1 in [-128, 127], |d2| <= 64.
 // The tensor cores multiply the weight codes (the A operand, 128 output
-// channels) by the digit rows (the B operand, column 3m + i = digit i of
-// token m) with int32 accumulators in tensor memory:
-//     D[n][3m + i] = sum_k q[n][k] d_i[m][k]        exact, K <= 65536
+// channels) by the digit rows (the B operand, row 3m + i = digit i of token
+// m) with int32 accumulators in tensor memory:
+//     D[n][3m + i] = sum_k q[n][k] d_i[m][k]        exact for K <= 65536
 // and the epilogue recombines y = s[n] 2^-e_m (D0 + 256 D1 + 65536 D2) in
 // binary64 before the bf16 rounding.
 //
-// Why: on B200 the bf16-dequantizing kernels spend tens of instructions per
-// 16 bytes of weights, which caps them well below HBM bandwidth at decode
-// sizes.  Here the packed block is already the tensor cores' canonical
-// K-major 128-byte-swizzled layout (wq_layout.h), so a 1-D bulk copy lands it
-// where the MMA reads it and the SM's threads only issue copies and MMAs.
+// Why: the bf16-dequantizing kernels spend tens of instructions per 16
+// bytes of weights, which caps them below HBM bandwidth at decode sizes.
+// Here the packed block is already the tensor cores' canonical K-major
+// 128-byte-swizzled layout (wq_layout.h): a 1-D bulk copy lands it where the
+// MMA reads it, and the SM's threads never touch the weights.
 //
 // Work split: stream-K.  The (panel, k-block) units form one stream; CTA c of
 // G (one per SM) takes units [U*c/G, U*(c+1)/G).  Warp roles (192 threads):
-//   warp 0     producer: per unit one 16 KB bulk copy of the weight block
-//              and one of the digit block into a STAGES-deep ring; weights
-//              are prefetched before the programmatic-launch wait.
+//   warp 0     producer: per unit one 16 KB bulk copy of the weight block and
+//              one of the unit's digit block (L2-resident) into a ring; the
+//              first stages' weights are issued before the programmatic-launch
+//              wait (weights never depend on the preceding kernel), digit
+//              blocks only once the grid has written them.
 //   warp 1     allocates tensor memory; one thread issues four
 //              tcgen05.mma kind::i8 (K = 32 each) per unit into one of two
-//              accumulator buffers (a panel segment per buffer).
-//   warps 2-5  epilogue, one thread per output channel: read the segment's
-//              accumulator, then either write y (the CTA covered the whole
-//              panel) or store int32 partials and take a ticket; the last
-//              arriver for a panel's rows sums every contributor's partial
-//              (integer sums: exact in any order) and writes y.
-// Every mbarrier wait is bounded (2 s); on a timeout the device error word
-// is set and the CTA winds down.
+//              accumulator buffers (one panel segment per buffer).
+//   warps 2-5  first the activations: every CTA computes the row maxima
+//              (e_m) and writes 1/G of the digit blocks to the workspace,
+//              then counts itself on a grid counter (release); the producer
+//              waits for all G (acquire, bounded).  Then the epilogue, one
+//              thread per output channel: write y when the CTA covered the
+//              whole panel, else store int32 partials and take a ticket; the
+//              last arriver for a panel's rows sums every contributor's
+//              partial (integer sums: exact in any order) and writes y.
+// All G CTAs are resident at once (one per SM, G <= SMs), so the grid
+// counter wait always ends; the last CTA to exit resets it.  For small M the
+// ring fits two CTAs per SM, so the next call's CTAs can stream their first
+// weights while this call's last CTAs finish.
+// Every wait is bounded (2 s); on a timeout the device error word is set and
+// the CTA winds down.
 #include <cstdint>
 
 #include <cuda_bf16.h>
@@ -49,134 +58,46 @@ namespace wq {
 
 static __device__ int g_i8_error = 0;
 
-// ---------------------------------------------------------------------------
-// Pre-pass: activations -> exponent e_m and base-256 digit blocks.
-// xd: [KB][NR rows][128 bytes], each k-block in the same canonical swizzled
-// layout as an INT8 weight block; row 3m + i = digit i of token m; rows
-// 3M .. NR-1 and k past K are zero.  xe[m] = e_m.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ int bf16_to_scaled_int(uint32_t b, int e)
-{
-    const uint32_t ex = (b >> 7) & 0xFFu;
-    const int mant = (int)(ex ? (0x80u | (b & 0x7Fu)) : (b & 0x7Fu));
-    const int sh = (int)(ex ? ex : 1u) - 134 + e; // x = mant * 2^(ex' - 134)
-    int X;
-    if (sh >= 0) {
-        X = mant << sh; // sh <= 14 for every element of the row
-    } else if (sh < -15) {
-        X = 0; // below half a unit
-    } else {
-        const int rs = -sh;
-        const int q = mant >> rs, rem = mant - (q << rs), half = 1 << (rs - 1);
-        X = q + ((rem > half || (rem == half && (q & 1))) ? 1 : 0);
-    }
-    return (b & 0x8000u) ? -X : X;
-}
-
-__global__ void __launch_bounds__(256) xdigits_kernel(const uint16_t *__restrict__ x, int M, int K, int KB, int NR,
-                                                      uint8_t *__restrict__ xd, int *__restrict__ xe)
-{
-    pdl_launch_dependents(); // the GEMM may start streaming weights now
-    pdl_wait();              // x may come from the preceding kernel
-    const int m = blockIdx.x;
-    const size_t kb_bytes = (size_t)NR * 128;
-    if (m == M) { // padding rows 3M .. NR-1 of every k-block
-        const int rows = NR - 3 * M;
-        const int vec = rows * 8; // 16-byte vectors per k-block
-        for (int i = threadIdx.x; i < KB * vec; i += blockDim.x) {
-            const int kb = i / vec, v = i % vec;
-            const int j = 3 * M + v / 8, slot = v % 8;
-            *reinterpret_cast<uint4 *>(xd + kb * kb_bytes + (j >> 3) * 1024 + (j & 7) * 128 + slot * 16) =
-                make_uint4(0, 0, 0, 0);
-        }
-        return;
-    }
-    __shared__ uint32_t s_max[8];
-    const uint16_t *row = x + (size_t)m * K;
-    uint32_t amax = 0;
-    for (int k = 8 * threadIdx.x; k < K; k += 8 * blockDim.x) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(row + k);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            amax = max(amax, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1)
-        amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if ((threadIdx.x & 31) == 0)
-        s_max[threadIdx.x >> 5] = amax;
-    __syncthreads();
-    amax = s_max[0];
-    for (int i = 1; i < (int)(blockDim.x >> 5); ++i)
-        amax = max(amax, s_max[i]);
-    // |x| < 2^(E+1) with E the largest element's exponent: e = 21 - E gives |X| < 2^22
-    const int ebits = (int)(amax >> 7);
-    const int e = amax == 0 ? 0 : 21 - ((ebits ? ebits : 1) - 127);
-    if (threadIdx.x == 0)
-        xe[m] = e;
-    const int chunks = KB * 8;
-    for (int ci = threadIdx.x; ci < chunks; ci += blockDim.x) {
-        const int kb = ci >> 3, c = ci & 7, k0 = 16 * ci;
-        uint32_t d[3][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}};
-        if (k0 < K) {
-            const uint4 v0 = *reinterpret_cast<const uint4 *>(row + k0);
-            const uint4 v1 = *reinterpret_cast<const uint4 *>(row + k0 + 8);
-            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint32_t b = (w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
-                const int X = bf16_to_scaled_int(b, e);
-                const int d0 = ((X + 128) & 255) - 128;
-                const int X1 = (X - d0) >> 8;
-                const int d1 = ((X1 + 128) & 255) - 128;
-                const int d2 = (X1 - d1) >> 8;
-                d[0][i >> 2] |= (uint32_t)(d0 & 255) << (8 * (i & 3));
-                d[1][i >> 2] |= (uint32_t)(d1 & 255) << (8 * (i & 3));
-                d[2][i >> 2] |= (uint32_t)(d2 & 255) << (8 * (i & 3));
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 3; ++i) {
-            const int j = 3 * m + i;
-            *reinterpret_cast<uint4 *>(xd + kb * kb_bytes + (j >> 3) * 1024 + (j & 7) * 128 + ((c ^ (j & 7)) << 4)) =
-                make_uint4(d[i][0], d[i][1], d[i][2], d[i][3]);
-        }
-    }
-}
-
-// ---------------------------------------------------------------------------
-// The GEMM.
-// ---------------------------------------------------------------------------
 struct I8Params {
+    const uint16_t *x;
     int M, K, N, KB, U;
     const uint8_t *wq;
     const uint16_t *scales;
     uint16_t *y;
-    const uint8_t *xd;
-    const int *xe;
+    uint8_t *xd;    // [KB][NR][128] digit blocks
     int32_t *part;  // [G][2 slots][NR][128 rows] int32
     uint32_t *cnt;  // [panels][4] tickets
+    uint32_t *grid; // [2]: digit blocks written, CTAs exited
 };
 
-// Per digit-row count NR (the MMA's N): ring depth and tensor-memory columns.
+// Per digit-row count NR (the MMA's N): ring depth, tensor-memory columns and
+// CTAs per SM.  Up to NR = 48 (M <= 16) the ring stays near 100 KB so two
+// CTAs fit on an SM.
 template <int NR>
 struct I8Cfg {
-    static constexpr int kAB = 16384;          // weight block
-    static constexpr int kBB = NR * 128;       // digit block
+    static constexpr int kAB = 16384;    // weight block
+    static constexpr int kBB = NR * 128; // digit block
     static constexpr int kStageBytes = kAB + kBB;
-    static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
+    static constexpr int kOcc = NR <= 48 ? 2 : 1;
+    static constexpr int kBudget = kOcc == 2 ? 100 * 1024 : 200 * 1024;
+    static constexpr int kStagesRaw = kBudget / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
     static constexpr int kTmemCols = 2 * NR <= 32 ? 32 : 2 * NR <= 64 ? 64 : 2 * NR <= 128 ? 128 : 2 * NR <= 256 ? 256 : 512;
-    static constexpr int kColGroup = NR < 48 ? NR : 48; // epilogue columns per pass (16 tokens)
+    // epilogue columns per pass: whole tokens (3 columns each), a multiple of 8
+    static constexpr int kColGroup = NR < 48 ? NR : 48;
     static_assert(NR % 16 == 0 && NR <= 256, "MMA N: multiple of 16, at most 256");
-    static_assert(kStages >= 3, "ring depth");
+    static_assert(kStages >= 4, "ring depth");
 };
+
+constexpr int kI8Threads = 192;
 
 template <int NR>
 constexpr size_t i8_smem_bytes()
 {
-    return 1024 + (size_t)I8Cfg<NR>::kStages * I8Cfg<NR>::kStageBytes + (2 * I8Cfg<NR>::kStages + 4) * 8 + 16;
+    // ring + barriers (full, empty per stage; accfull, accempty x 2) +
+    // tensor-memory slot + row maxima / exponents
+    return 1024 + (size_t)I8Cfg<NR>::kStages * I8Cfg<NR>::kStageBytes + (2 * I8Cfg<NR>::kStages + 4) * 8 + 16 +
+           2 * kI8MaxM * 4;
 }
 
 // Instruction descriptor, kind::i8: signed 8-bit A and B, int32 D, both
@@ -210,8 +131,64 @@ __device__ __forceinline__ uint16_t i8_output(int32_t d0, int32_t d1, int32_t d2
     return __bfloat16_as_ushort(__double2bfloat16(v));
 }
 
+// Exponent e_m of a token row from the largest magnitude's bf16 bits:
+// |x| < 2^(E+1), e = 21 - E gives |X| < 2^22.  Rows whose largest magnitude
+// is below 2^-106 use e = 127 (the largest power of two a binary32 holds).
+__device__ __forceinline__ int row_exponent(uint32_t amax_bits)
+{
+    if (amax_bits == 0)
+        return 0;
+    const int eb = (int)(amax_bits >> 7);
+    const int e = 21 - ((eb ? eb : 1) - 127);
+    return e > 127 ? 127 : e;
+}
+
+// 16 consecutive activations (bf16 bits in w[8]) -> the digit planes of one
+// 16-byte chunk: p[i][j] = bytes 4j..4j+3 of digit plane i.  With the fused
+// multiply-add F = x * 2^e + 1.5 * 2^23 rounded once (to nearest, ties to
+// even), the binary32 bits of F are 0x4B400000 + X for |X| < 2^22, and
+// X + 0x808080 holds the three biased digits d_i + 128 in its low three
+// bytes (the balanced base-256 expansion is unique, so no byte carries).
+__device__ __forceinline__ void digit_planes(const uint32_t (&w)[8], float s, uint32_t (&p)[3][4])
+{
+    uint32_t Y[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
+        Y[2 * i] = __float_as_uint(fmaf(lo, s, 12582912.0f)) - 0x4ABF7F80u;     // X + 0x808080
+        Y[2 * i + 1] = __float_as_uint(fmaf(hi, s, 12582912.0f)) - 0x4ABF7F80u;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t a01 = __byte_perm(Y[4 * j], Y[4 * j + 1], 0x5140u);     // d0 d0 d1 d1
+        const uint32_t a23 = __byte_perm(Y[4 * j + 2], Y[4 * j + 3], 0x5140u);
+        const uint32_t b01 = __byte_perm(Y[4 * j], Y[4 * j + 1], 0x0062u);     // d2 d2 . .
+        const uint32_t b23 = __byte_perm(Y[4 * j + 2], Y[4 * j + 3], 0x0062u);
+        p[0][j] = __byte_perm(a01, a23, 0x5410u) ^ 0x80808080u; // biased -> two's complement
+        p[1][j] = __byte_perm(a01, a23, 0x7632u) ^ 0x80808080u;
+        p[2][j] = __byte_perm(b01, b23, 0x5410u) ^ 0x80808080u;
+    }
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(uint32_t *p, uint32_t v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 template <int NR>
-__global__ void __launch_bounds__(192, 1) gemm_i8_kernel(const I8Params p)
+__global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(const I8Params p)
 {
     using C = I8Cfg<NR>;
     constexpr int STAGES = C::kStages;
@@ -225,11 +202,13 @@ __global__ void __launch_bounds__(192, 1) gemm_i8_kernel(const I8Params p)
     uint64_t *accfull = empty + STAGES; // [2]
     uint64_t *accempty = accfull + 2;   // [2]
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(accempty + 2);
+    uint32_t *s_amax = s_tmem + 4;                        // [kI8MaxM] row maxima (bf16 magnitude bits)
+    int *s_e = reinterpret_cast<int *>(s_amax + kI8MaxM); // [kI8MaxM] exponents e_m
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, c = blockIdx.x;
     const long long U = p.U;
-    const int KB = p.KB;
+    const int KB = p.KB, M = p.M;
     const int u0 = sk_start(U, G, c), u1 = sk_start(U, G, c + 1);
     const int n = u1 - u0;
 
@@ -244,6 +223,8 @@ __global__ void __launch_bounds__(192, 1) gemm_i8_kernel(const I8Params p)
         }
         fence_mbar_init();
     }
+    if (threadIdx.x < kI8MaxM)
+        s_amax[threadIdx.x] = 0u;
     if (warp == 1) {
         tmem_alloc(s_tmem, TCOLS);
         tmem_relinquish();
@@ -258,22 +239,30 @@ __global__ void __launch_bounds__(192, 1) gemm_i8_kernel(const I8Params p)
         if (lane == 0) {
             const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
             auto issue_w = [&](int i, int st) {
-                uint8_t *dst = ring + st * C::kStageBytes;
                 mbar_arrive_expect_tx(&full[st], C::kStageBytes);
-                bulk_g2s(dst, p.wq + (size_t)(u0 + i) * C::kAB, C::kAB, &full[st], pol_w);
+                bulk_g2s(ring + st * C::kStageBytes, p.wq + (size_t)(u0 + i) * C::kAB, C::kAB, &full[st], pol_w);
             };
             auto issue_x = [&](int i, int st) {
                 const int kb = (u0 + i) % KB;
                 bulk_g2s(ring + st * C::kStageBytes + C::kAB, p.xd + (size_t)kb * C::kBB, C::kBB, &full[st], pol_x);
             };
-            // weights do not depend on the preceding kernels: stream them before waiting
             const int pre = n < STAGES ? n : STAGES;
-            for (int i = 0; i < pre; ++i)
+            for (int i = 0; i < pre; ++i) // weights never depend on the preceding kernel
                 issue_w(i, i);
+            // the preceding call (same workspace) has finished and reset the grid
+            // counters; then wait until every CTA's share of the digit blocks is written
             pdl_wait();
-            for (int i = 0; i < pre; ++i)
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_gpu(&p.grid[0]) < (uint32_t)G) {
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    ok = false;
+                    break;
+                }
+            }
+            fence_proxy_async_global(); // the digit blocks are read by the bulk-copy (async) proxy
+            for (int i = 0; i < pre && ok; ++i)
                 issue_x(i, i);
-            for (int i = pre; i < n; ++i) {
+            for (int i = pre; i < n && ok; ++i) {
                 const int st = i % STAGES, use = i / STAGES;
                 if (!mbar_wait(&empty[st], (use - 1) & 1)) {
                     ok = false;
@@ -282,12 +271,11 @@ __global__ void __launch_bounds__(192, 1) gemm_i8_kernel(const I8Params p)
                 issue_w(i, st);
                 issue_x(i, st);
             }
-        } else {
-            pdl_wait();
         }
+        __syncwarp();
+        pdl_wait();
         pdl_launch_dependents();
     } else if (warp == 1) {
-        pdl_wait();
         if (lane == 0) {
             constexpr uint32_t idesc = umma_idesc_s8(NR);
             int seg = -1;
@@ -319,19 +307,134 @@ __global__ void __launch_bounds__(192, 1) gemm_i8_kernel(const I8Params p)
             }
         }
         __syncwarp();
+        pdl_wait();
         pdl_launch_dependents();
     } else {
-        // ---------------- epilogue: one thread per output channel ----------------
-        pdl_wait(); // xe, y and the workspace may still be in use by the preceding kernels
+        pdl_wait(); // x, y and the workspace may come from / be in use by the preceding kernel
+        const int et = threadIdx.x - 64; // 0..127
         const int quad = warp & 3;
+        const int K = p.K;
+        // ---------------- activations: row maxima, then 1/G of the digit blocks ----------------
+        {
+            // items (token slot m, k-block, 16-k chunk); slots M .. ceil(NR/3)-1 write the zero padding rows
+            constexpr int MS = (NR + 2) / 3;
+            const long long items = (long long)MS * KB * 8;
+            const long long i0 = items * c / G, i1 = items * (c + 1) / G;
+            auto item_x = [&](long long it, uint4 &a, uint4 &b) {
+                const int m = (int)(it / (KB * 8)), rem = (int)(it % (KB * 8));
+                const int k0 = (rem >> 3) * kBlockK + 16 * (rem & 7);
+                if (m < M && k0 < K) {
+                    a = ldg_keep4(p.x + (size_t)m * K + k0);
+                    b = ldg_keep4(p.x + (size_t)m * K + k0 + 8);
+                } else { // k past K or a padding slot: zero activations (zero weights there too)
+                    a = b = make_uint4(0, 0, 0, 0);
+                }
+            };
+            // this thread's first item is loaded together with the row maxima (one round trip)
+            uint4 fa = make_uint4(0, 0, 0, 0), fb = fa;
+            if (i0 + et < i1)
+                item_x(i0 + et, fa, fb);
+            const int vpr = K / 8; // 16-byte vectors per token row
+            const long long total = (long long)M * vpr;
+            int cur_m = -1;
+            uint32_t cur = 0;
+            constexpr int BATCH = 8;
+            for (long long v0 = et; v0 < total; v0 += BATCH * 128) {
+                uint4 q[BATCH];
+#pragma unroll
+                for (int b = 0; b < BATCH; ++b) {
+                    const long long v = v0 + (long long)b * 128;
+                    q[b] = v < total ? ldg_keep4(p.x + v * 8) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int b = 0; b < BATCH; ++b) {
+                    const long long v = v0 + (long long)b * 128;
+                    if (v >= total)
+                        break;
+                    const int m = (int)(v / vpr);
+                    if (m != cur_m) {
+                        if (cur_m >= 0)
+                            atomicMax(&s_amax[cur_m], cur);
+                        cur_m = m;
+                        cur = 0;
+                    }
+                    const uint32_t wv[4] = {q[b].x, q[b].y, q[b].z, q[b].w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        cur = max(cur, max(wv[h] & 0x7FFFu, (wv[h] >> 16) & 0x7FFFu));
+                }
+            }
+            if (cur_m >= 0)
+                atomicMax(&s_amax[cur_m], cur);
+            named_barrier_sync(1, 128);
+            if (et < M)
+                s_e[et] = row_exponent(s_amax[et]);
+            named_barrier_sync(1, 128);
+            for (long long it = i0 + et; it < i1; it += 128) {
+                const int m = (int)(it / (KB * 8)), rem = (int)(it % (KB * 8));
+                const int kb = rem >> 3, cc = rem & 7;
+                uint4 a = fa, b = fb;
+                if (it != i0 + et)
+                    item_x(it, a, b);
+                uint32_t pl[3][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}};
+                if (m < M) {
+                    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                    digit_planes(w, __uint_as_float((uint32_t)(127 + s_e[m]) << 23), pl); // 2^e, -106 <= e <= 127
+                }
+                uint8_t *blk = p.xd + (size_t)kb * C::kBB;
+#pragma unroll
+                for (int d = 0; d < 3; ++d) {
+                    const int jr = 3 * m + d;
+                    if (jr < NR)
+                        *reinterpret_cast<uint4 *>(blk + (jr >> 3) * 1024 + (jr & 7) * 128 + ((cc ^ (jr & 7)) << 4)) =
+                            make_uint4(pl[d][0], pl[d][1], pl[d][2], pl[d][3]);
+                }
+            }
+            fence_proxy_async_global();
+            named_barrier_sync(1, 128);
+            if (et == 0)
+                red_release_gpu_add(&p.grid[0], 1u); // cumulative over the 128 threads' stores
+        }
+        // ---------------- epilogue: one thread per output channel ----------------
         const int row = 32 * quad + lane;
         const uint32_t tq = (uint32_t)(32 * quad) << 16;
-        const int M = p.M;
         int seg = 0;
         for (int pnl = n > 0 ? u0 / KB : 0; n > 0 && pnl <= (u1 - 1) / KB && ok; ++pnl, ++seg) {
             const int lo = max(u0, pnl * KB), hi = min(u1, (pnl + 1) * KB);
             const bool whole = (lo == pnl * KB && hi == (pnl + 1) * KB);
             const int b = seg & 1;
+            const int cf = sk_owner(U, G, pnl * KB), cl = sk_owner(U, G, (pnl + 1) * KB - 1);
+            // A split panel whose other contributors have all taken their tickets
+            // (typically the last segment of the range: its partner did its part
+            // first): this warp is the last arriver.  It reads their partials now,
+            // while its own MMAs are still running, and takes no ticket.
+            bool early_last = false;
+            int32_t pre[CG];
+#pragma unroll
+            for (int j = 0; j < CG; ++j)
+                pre[j] = 0;
+            if (!whole && 3 * M <= CG) {
+                uint32_t seen = 0;
+                if (lane == 0)
+                    seen = ld_acquire_gpu(&p.cnt[pnl * 4 + quad]);
+                early_last = __shfl_sync(0xffffffffu, seen, 0) == (uint32_t)(cl - cf);
+                if (early_last) {
+                    __syncwarp(); // lane 0's acquire orders every lane's reads below
+                    for (int cc = cf; cc <= cl; ++cc) {
+                        if (cc == c)
+                            continue;
+                        const int sl = (pnl == sk_start(U, G, cc) / KB) ? 0 : 1;
+                        const int32_t *src = p.part + (size_t)(cc * 2 + sl) * NR * 128 + row;
+                        int32_t v[CG];
+#pragma unroll
+                        for (int j = 0; j < CG; ++j)
+                            v[j] = (j < 3 * M) ? __ldcg(src + (size_t)j * 128) : 0;
+#pragma unroll
+                        for (int j = 0; j < CG; ++j)
+                            pre[j] += v[j];
+                    }
+                }
+            }
             if (!mbar_wait_warp(&accfull[b], (seg >> 1) & 1)) {
                 ok = false;
                 break;
@@ -345,11 +448,11 @@ __global__ void __launch_bounds__(192, 1) gemm_i8_kernel(const I8Params p)
             for (int c0 = 0; c0 < NR; c0 += CG) {
                 int32_t v[CG];
 #pragma unroll
-                for (int cc = 0; cc < CG; cc += 16) {
-                    float f[16];
-                    tmem_ld_32x32b_x16(tmem + tq + (uint32_t)(b * NR + c0 + cc), f);
+                for (int cc = 0; cc < CG; cc += 8) {
+                    float f[8];
+                    tmem_ld_32x32b_x8(tmem + tq + (uint32_t)(b * NR + c0 + cc), f);
 #pragma unroll
-                    for (int e2 = 0; e2 < 16; ++e2)
+                    for (int e2 = 0; e2 < 8; ++e2)
                         v[cc + e2] = __float_as_int(f[e2]);
                 }
                 tmem_wait_ld();
@@ -359,14 +462,19 @@ __global__ void __launch_bounds__(192, 1) gemm_i8_kernel(const I8Params p)
                     if (lane == 0)
                         mbar_arrive(&accempty[b]);
                 }
-                if (whole) {
+                if (whole || early_last) {
+                    if (early_last) { // one pass: 3M <= CG
+#pragma unroll
+                        for (int j = 0; j < CG; ++j)
+                            v[j] += pre[j];
+                    }
                     if (nrow < p.N) {
 #pragma unroll
                         for (int t = 0; t < CG / 3; ++t) {
                             const int m = c0 / 3 + t;
                             if (m < M)
                                 p.y[(size_t)m * p.N + nrow] =
-                                    i8_output(v[3 * t], v[3 * t + 1], v[3 * t + 2], s_n * pow2_of(-__ldg(p.xe + m)));
+                                    i8_output(v[3 * t], v[3 * t + 1], v[3 * t + 2], s_n * pow2_of(-s_e[m]));
                         }
                     }
                 } else {
@@ -378,18 +486,22 @@ __global__ void __launch_bounds__(192, 1) gemm_i8_kernel(const I8Params p)
             }
             if (whole)
                 continue;
+            if (early_last) { // every other contributor is done: reset the ticket for the next call
+                if (lane == 0)
+                    atomicExch(&p.cnt[pnl * 4 + quad], 0u);
+                continue;
+            }
             // Split panel: every contributor's warp takes a ticket for its 32
-            // rows; the last one sums all partials (exact integers) and writes y.
-            __threadfence();
+            // rows (one acquire-release atomic after a warp barrier); the last
+            // one sums all partials (exact integers) and writes y.
             __syncwarp();
             uint32_t ticket = 0;
             if (lane == 0)
-                ticket = ticket_take(&p.cnt[pnl * 4 + quad]);
+                ticket = ticket_take_acq_rel(&p.cnt[pnl * 4 + quad]);
             ticket = __shfl_sync(0xffffffffu, ticket, 0);
-            const int cf = sk_owner(U, G, pnl * KB), cl = sk_owner(U, G, (pnl + 1) * KB - 1);
             if (ticket != (uint32_t)(cl - cf))
                 continue;
-            __threadfence();
+            __syncwarp(); // lane 0's acquire orders every lane's reads below
             for (int c0 = 0; c0 < 3 * M; c0 += CG) {
                 int32_t tot[CG];
 #pragma unroll
@@ -412,7 +524,7 @@ __global__ void __launch_bounds__(192, 1) gemm_i8_kernel(const I8Params p)
                         const int m = c0 / 3 + t;
                         if (m < M)
                             p.y[(size_t)m * p.N + nrow] =
-                                i8_output(tot[3 * t], tot[3 * t + 1], tot[3 * t + 2], s_n * pow2_of(-__ldg(p.xe + m)));
+                                i8_output(tot[3 * t], tot[3 * t + 1], tot[3 * t + 2], s_n * pow2_of(-s_e[m]));
                     }
                 }
             }
@@ -430,6 +542,11 @@ __global__ void __launch_bounds__(192, 1) gemm_i8_kernel(const I8Params p)
         tc_fence_after();
         tmem_dealloc(tmem, TCOLS);
     }
+    // the last CTA out resets the grid counters for the next call
+    if (threadIdx.x == 0 && atomicAdd(&p.grid[1], 1u) == (uint32_t)(G - 1)) {
+        atomicExch(&p.grid[0], 0u);
+        atomicExch(&p.grid[1], 0u);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -439,11 +556,11 @@ int i8_digit_rows(int M) { return M <= 5 ? 16 : M <= 10 ? 32 : M <= 16 ? 48 : M 
 
 size_t ws_bytes_gemm_i8(int M, int K, int N)
 {
-    if (M < 1 || M > kI8MaxM)
+    if (M < 1 || M > kI8MaxM || K < 1)
         return 0;
     const int NR = i8_digit_rows(M);
     const size_t KB = (size_t)(K + kBlockK - 1) / kBlockK;
-    return ws_counter_bytes(N) + 256 + KB * NR * 128 + (size_t)kI8MaxCtas * 2 * NR * 128 * sizeof(int32_t);
+    return ws_counter_bytes(N) + KB * NR * 128 + (size_t)kI8MaxCtas * 2 * NR * 128 * sizeof(int32_t);
 }
 
 template <int NR>
@@ -451,6 +568,7 @@ static cudaError_t launch_i8_t(const LinearArgs &a, void *ws, int sm_count, cuda
 {
     constexpr size_t smem = i8_smem_bytes<NR>();
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
+    static_assert(I8Cfg<NR>::kOcc == 1 || 2 * (smem + 1024) <= 228 * 1024, "two CTAs per SM");
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(gemm_i8_kernel<NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -460,13 +578,23 @@ static cudaError_t launch_i8_t(const LinearArgs &a, void *ws, int sm_count, cuda
         attr_set = true;
     }
     const Shape sh{8, a.K, a.N, 0};
-    const int KB = sh.kblocks();
-    uint8_t *base = (uint8_t *)ws + ws_counter_bytes(a.N);
-    int *xe = (int *)base;
-    uint8_t *xd = base + 256;
-    int32_t *part = (int32_t *)(xd + (size_t)KB * NR * 128);
-
-    // the pre-pass: one block per token row plus one for the padding rows
+    I8Params p;
+    p.x = a.x;
+    p.M = a.M;
+    p.K = a.K;
+    p.N = a.N;
+    p.KB = sh.kblocks();
+    p.U = sh.panels() * p.KB;
+    p.wq = (const uint8_t *)a.wq;
+    p.scales = (const uint16_t *)a.scales;
+    p.y = a.y;
+    p.cnt = (uint32_t *)ws;
+    p.grid = p.cnt + ws_grid_counter(a.N);
+    p.xd = (uint8_t *)ws + ws_counter_bytes(a.N);
+    p.part = (int32_t *)(p.xd + (size_t)p.KB * NR * 128);
+    int G = sm_count < kI8MaxCtas ? sm_count : kI8MaxCtas;
+    if (G > p.U)
+        G = p.U;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -474,31 +602,8 @@ static cudaError_t launch_i8_t(const LinearArgs &a, void *ws, int sm_count, cuda
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cfg.stream = st;
-    cfg.gridDim = dim3(a.M + 1);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, xdigits_kernel, a.x, a.M, a.K, KB, NR, xd, xe);
-    if (e != cudaSuccess)
-        return e;
-
-    I8Params p;
-    p.M = a.M;
-    p.K = a.K;
-    p.N = a.N;
-    p.KB = KB;
-    p.U = sh.panels() * KB;
-    p.wq = (const uint8_t *)a.wq;
-    p.scales = (const uint16_t *)a.scales;
-    p.y = a.y;
-    p.xd = xd;
-    p.xe = xe;
-    p.part = part;
-    p.cnt = (uint32_t *)ws;
-    int G = sm_count < kI8MaxCtas ? sm_count : kI8MaxCtas;
-    if (G > p.U)
-        G = p.U;
     cfg.gridDim = dim3(G);
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(kI8Threads);
     cfg.dynamicSmemBytes = smem;
     return cudaLaunchKernelEx(&cfg, gemm_i8_kernel<NR>, p);
 }

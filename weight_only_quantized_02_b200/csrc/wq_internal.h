@@ -17,12 +17,16 @@ struct LinearArgs {
     uint16_t *y;
 };
 
-// Split-K workspace: [ticket counters, 256-byte padded][fp32 partials].
-// Tickets: 8 per 128-row panel (one per 16-row block; the GEMM uses the
-// first panel-count entries).  GEMM with S splits: partials [S][M][N].
-// Stream-K GEMV: partials [CTAs <= kSkMaxCtas][2][128 rows][8 * ceil(M/8) tokens].
+// Split-K workspace: [counters, 256-byte padded][partials].
+// Counters: 8 tickets per 128-row panel (one per 16-row block; the GEMM uses
+// the first panel-count entries), then two grid counters of the integer
+// path (ws_grid_counter).  Every kernel leaves the counters it used at zero.
+// GEMM with S splits: partials [S][M][N].  Stream-K GEMV: partials
+// [CTAs <= kSkMaxCtas][2][128 rows][8 * ceil(M/8) tokens].
 constexpr int kSkMaxCtas = 512;
-inline size_t ws_counter_bytes(int N) { return (((size_t)((N + 127) / 128) * 8 * 4) + 255) / 256 * 256; }
+inline size_t ws_counter_words(int N) { return (size_t)((N + 127) / 128) * 8 + 2; }
+inline size_t ws_counter_bytes(int N) { return (ws_counter_words(N) * 4 + 255) / 256 * 256; }
+inline size_t ws_grid_counter(int N) { return (size_t)((N + 127) / 128) * 8; } // word index of the first
 inline size_t ws_bytes(int M, int N, int S)
 {
     return ws_counter_bytes(N) + (S > 1 ? (size_t)S * M * N * sizeof(float) : 0);

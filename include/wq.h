@@ -23,8 +23,8 @@
  *   - a small-M GEMM (tcgen05 tensor cores, accumulators in tensor memory)
  *     with split-K and a fixed-order fp32 reduction ("split_k" auto-tuning,
  *     Mit han lab Llm awq Kernel Selection Thresholds, The Insight).
- *   - for W8A16, M <= 64: the integer tensor cores (tcgen05 kind::i8) on the
- *     raw INT8 codes. The per-channel scale factors out of the k sum, x is
+ *   - on the integer tensor cores (tcgen05 kind::i8): W8A16 (M <= 64) on the
+ *     raw INT8 codes, W4A16 (M <= 32) on the exact integers q - z. The per-channel scale factors out of the k sum, x is
  *     written per token row as an integer X = round(x * 2^e), ties to even,
  *     with e = min(21 - E, 127) for 2^E <= max|x| < 2^(E+1), so |X| < 2^22
  *     (three base-256 digits) and every element within 2^14 of the row's
@@ -34,7 +34,7 @@
  * starts from an untuned rule (W8A16 within the integer path's limits -> the
  * integer path; otherwise the pages' rule: fewer than 8 tokens -> GEMV, else
  * GEMM with split 8; same page) and is overridden by measured timings
- * (wq_tune).
+ * (wq_tune), whose candidates include the integer path for W4A16 too.
  *
  * Conventions for every entry point:
  *   - The return value is a wq_status: 0 on success, negative on error.
@@ -87,8 +87,8 @@ typedef enum {
 #define WQ_VARIANT_GEMM 1    /* tcgen05 split-K GEMM, M <= 128 */
 #define WQ_VARIANT_GEMV_RB 2 /* row-block GEMV, M <= 32, direct 128-bit loads; no workspace */
 #define WQ_VARIANT_GEMM_SK 3 /* stream-K tcgen05 GEMM, M <= 128, persistent; needs the workspace */
-#define WQ_VARIANT_I8MMA 4   /* W8A16 only: stream-K tcgen05 kind::i8 on the raw codes, M <= 64,
-                                K <= 65536; needs the workspace */
+#define WQ_VARIANT_I8MMA 4   /* stream-K tcgen05 kind::i8: W8A16 (M <= 64) on the raw codes,
+                                W4A16 (M <= 32) on q - z; K <= 65536; needs the workspace */
 
 /* Static description of a status code. Host. Never NULL. */
 const char *wq_strerror(int status);

@@ -99,8 +99,8 @@ def test_tuning_file_parse_errors(tmp_path):
         "NVIDIA B200|148 1 5120 17408 8 0 0\n",             # truncated
         "NVIDIA B200|148 1 5120 17408 8 0 0 4 12.5 extra\n",
         "NVIDIA B200|148 64 17408 5120 4 128 1 64 1.0\n",   # split above 32
-        "NVIDIA B200|148 4 5120 17408 4 128 4 1 9.0\n",     # integer path: INT8 only
         "NVIDIA B200|148 65 5120 17408 8 0 4 1 9.0\n",      # integer path: M <= 64
+        "NVIDIA B200|148 33 5120 17408 4 128 4 1 9.0\n",    # integer path, W4A16: M <= 32
         "NVIDIA B200|148 4 5120 17408 8 0 4 2 9.0\n",       # integer path: split 1 only
     ]:
         p = tmp_path / "bad.txt"

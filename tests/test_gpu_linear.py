@@ -53,7 +53,7 @@ def _cases(M, K, bits):
         out += [(GEMV_RB, ks) for ks in (1, 2, 4, 8)]
     out += [(GEMM, s) for s in (1, 2, 4, 8, 16, 32) if s <= kb]
     out += [(GEMM_SK, c) for c in (1, 2)]
-    if bits == 8 and M <= 64:
+    if M <= (64 if bits == 8 else 32):  # integer tensor-core path: W8A16 M <= 64, W4A16 M <= 32
         out += [(I8, 1)]
     return out
 
@@ -84,9 +84,8 @@ def test_repeated_dispatch_resets_tickets(weight, ws):
     """Many split-K and stream-K calls in a row reuse the workspace counters;
     each must leave them at zero for the next (different variant, split, M)."""
     bits, K, N, pw, canon = weight
-    runs = [(GEMM, 16, 2), (GEMM, 16, 8), (GEMM_SK, 40, 2), (GEMV, 5, 3), (GEMM, 40, 4), (GEMM, 128, 9)]
-    if bits == 8:
-        runs += [(I8, 5, 1), (I8, 40, 1), (GEMV, 3, 2), (I8, 1, 1)]
+    runs = [(GEMM, 16, 2), (GEMM, 16, 8), (GEMM_SK, 40, 2), (GEMV, 5, 3), (GEMM, 40, 4), (GEMM, 128, 9),
+            (I8, 5, 1), (I8, 40 if bits == 8 else 30, 1), (GEMV, 3, 2), (I8, 1, 1)]
     runs += [(GEMM, 16, 2)]
     for variant, M, split in runs:
         x = gen.x_bf16(M, K)
@@ -170,9 +169,20 @@ def test_one_hot_int4_weights_exact(ws):
     pw = pack_canonical_int4(q, s, z)
     x = gen.x_bf16(M, K)
     want = oracle.bf16_to_f64(oracle.bf16_rne_of(oracle.linear_int4(x, q, s, z)))
+    # integer path: per group s * fp32((q - z) X) with X the fixed-point activations
+    xq, e = i8_fixed_point(x, with_exponents=True)
+    X = np.ldexp(xq, e[:, None])                                   # exact integers
+    d = (qn[np.arange(N), cols] - zn[np.arange(N), cols // G]).astype(np.float64)
+    prod = np.float32(X[:, cols] * d[None, :]).astype(np.float64)  # one binary32 rounding
+    sc = oracle.bf16_to_f64(s[np.arange(N), cols // G])
+    want_i8 = oracle.bf16_to_f64(oracle.bf16_rne_of(np.ldexp(prod * sc[None, :], -e[:, None])))
     for variant, split in _all_cases(M, K, 4):
         y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
-        assert np.array_equal(y, want), (variant, split)
+        if variant == I8:
+            assert np.array_equal(y, want_i8), (variant, split)
+            assert_parity(y, oracle.linear_int4(x, q, s, z), "one-hot int4 weights, integer path")
+        else:
+            assert np.array_equal(y, want), (variant, split)
 
 
 @pytest.mark.parametrize("bits", [8, 4])
@@ -254,11 +264,12 @@ def test_argument_errors(weight, ws):
     assert wq.wq_linear_status(x, pw, y, GEMM, 33) == -11         # split above 32
     assert wq.wq_linear_status(x, pw, y, 7, 1) == -11             # unknown variant
     assert wq.wq_linear_status(x, pw, y, I8, 2) == -11            # one CTA per SM only
-    if bits == 4:
-        assert wq.wq_linear_status(x, pw, y, I8, 1) == -11        # integer path: INT8 only
     xc = bf16_dev(gen.x_bf16(65, K))
     yc = torch.empty((65, N), dtype=torch.bfloat16, device=dev())
-    assert wq.wq_linear_status(xc, pw, yc, I8, 1) == -11          # integer path takes M <= 64
+    assert wq.wq_linear_status(xc, pw, yc, I8, 1) == -11          # integer path takes M <= 64 (W4A16: 32)
+    xd33 = bf16_dev(gen.x_bf16(33, K))
+    yd33 = torch.empty((33, N), dtype=torch.bfloat16, device=dev())
+    assert wq.wq_linear_status(xd33, pw, yd33, I8, 1) == (0 if bits == 8 else -11)
     xb = bf16_dev(gen.x_bf16(40, K))
     yb = torch.empty((40, N), dtype=torch.bfloat16, device=dev())
     assert wq.wq_linear_status(xb, pw, yb, GEMV, 1) == -11        # GEMV takes M <= 32
@@ -271,8 +282,7 @@ def test_argument_errors(weight, ws):
     try:
         assert wq.wq_linear_status(x, pw, y, GEMM, 4) == -6
         assert wq.wq_linear_status(x, pw, y, GEMV, 1) == -6
-        if bits == 8:
-            assert wq.wq_linear_status(x, pw, y, I8, 1) == -6
+        assert wq.wq_linear_status(x, pw, y, I8, 1) == -6
         assert wq.wq_linear_status(x, pw, y, GEMM, 1) == 0
         assert wq.wq_linear_status(x, pw, y, GEMV_RB, 2) == 0
         assert wq.wq_linear_status(x, pw, y) == 0  # dispatcher falls back to the row-block GEMV
@@ -307,9 +317,7 @@ def test_explicit_workspace_on_two_streams(weight):
 
 def test_cuda_graph_replay(weight, ws):
     bits, K, N, pw, canon = weight
-    runs = [(1, GEMV, 2), (1, GEMV_RB, 4), (16, GEMM, 4), (128, GEMM, 2)]
-    if bits == 8:
-        runs += [(1, I8, 1), (16, I8, 1)]
+    runs = [(1, GEMV, 2), (1, GEMV_RB, 4), (16, GEMM, 4), (128, GEMM, 2), (1, I8, 1), (16, I8, 1)]
     for M, variant, split in runs:
         x = gen.x_bf16(M, K)
         xd = bf16_dev(x)

@@ -78,7 +78,7 @@ def _variants(M, K, bits):
         out += [(GEMV_RB, ks) for ks in (1, 2, 4, 8)]
     out += [(GEMM, s) for s in (1, 2, 4, 8, 16, 32) if s <= (K + 127) // 128]
     out += [(GEMM_SK, c) for c in (1, 2)]
-    if bits == 8 and M <= 64:
+    if M <= (64 if bits == 8 else 32):  # integer tensor-core path: W8A16 M <= 64, W4A16 M <= 32
         out += [(I8, 1)]
     return out
 

@@ -90,20 +90,23 @@ def workspace(M: int, K: int, N: int, max_split: int = 32) -> torch.Tensor:
     return torch.zeros(nbytes, dtype=torch.uint8, device=dev())
 
 
-def i8_fixed_point(x_bits: np.ndarray) -> np.ndarray:
+def i8_fixed_point(x_bits: np.ndarray, with_exponents: bool = False):
     """The activations as the integer tensor-core path represents them, from
     the library's stated contract (include/wq.h): per token row, e = 21 - E
     with E the binary exponent of the row's largest magnitude (2^E <= max|x|
     < 2^(E+1); subnormal rows use E = -126), at most 127, and
     x -> round(x * 2^e) * 2^-e, ties to even.  Every element within 2^14 of
-    the row's largest is unchanged.  Returns binary64 values."""
+    the row's largest is unchanged.  Returns binary64 values (and the
+    exponents e per row when asked)."""
     x = oracle.bf16_to_f64(x_bits)
     out = np.zeros_like(x)
+    es = np.zeros(x.shape[0], np.int64)
     for m in range(x.shape[0]):
         amax = np.max(np.abs(x[m])) if x.shape[1] else 0.0
         if amax == 0.0:
             continue
         E = max(int(np.frexp(amax)[1]) - 1, -126)  # amax = f * 2^(E+1), f in [0.5, 1)
         e = min(21 - E, 127)
+        es[m] = e
         out[m] = np.rint(np.ldexp(x[m], e)) * np.ldexp(1.0, -e)  # exact: |X| < 2^22
-    return out
+    return (out, es) if with_exponents else out

@@ -108,7 +108,14 @@ int check_weight_shape(int bits, int K, int N, int group)
 
 int max_gemm_split(int K) { return std::min(32, (K + kBlockK - 1) / kBlockK); }
 
-bool i8_fits(int bits, int M, int K) { return bits == 8 && M <= kI8MaxM && K <= kI8MaxK; }
+bool i8_fits(int bits, int M, int K)
+{
+    return ((bits == 8 && M <= kI8MaxM) || (bits == 4 && M <= kI4MaxM)) && K <= kI8MaxK;
+}
+size_t ws_bytes_imma(int bits, int M, int K, int N)
+{
+    return bits == 8 ? ws_bytes_gemm_i8(M, K, N) : ws_bytes_gemm_i4(M, K, N);
+}
 
 bool choice_valid(int variant, int split, int M, int K, int bits)
 {
@@ -137,14 +144,14 @@ int default_rb_slices(int K, int N, int sm_count)
     return ks;
 }
 
-// Untuned rule.  INT8 runs on the integer tensor cores whenever the shape
-// and the workspace allow it.  Otherwise the pages' rule: fewer than 8
+// Untuned rule.  W8A16 runs on the integer tensor cores whenever the shape
+// and the workspace allow it (W4A16 there is a tuning candidate only).  Otherwise the pages' rule: fewer than 8
 // tokens -> GEMV, else the GEMM with split_k = 8 (Mit han lab Llm awq Kernel
 // Selection Thresholds, The Insight).  The stream-K GEMV needs the split-K
 // workspace; without one the row-block GEMV is used.
 Choice default_choice(int M, int K, int N, int bits, int sm_count, bool have_ws = true, bool have_i8_ws = true)
 {
-    if (i8_fits(bits, M, K) && have_i8_ws)
+    if (bits == 8 && i8_fits(bits, M, K) && have_i8_ws)
         return {WQ_VARIANT_I8MMA, 1, 0.f};
     if (M < 8) {
         if (have_ws)
@@ -207,7 +214,7 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
     if (w && !aligned16(w))
         return WQ_ERR_ALIGN;
     const bool sk_ws_ok = w && have >= ws_bytes_gemv_sk(M, N);
-    const bool i8_ws_ok = w && i8_fits(bits, M, K) && have >= ws_bytes_gemm_i8(M, K, N);
+    const bool i8_ws_ok = w && i8_fits(bits, M, K) && have >= ws_bytes_imma(bits, M, K, N);
 
     Choice c;
     lookup_choice(d, M, K, N, bits, group, &c);
@@ -241,7 +248,8 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
     if (c.variant == WQ_VARIANT_I8MMA) {
         if (!i8_ws_ok)
             return WQ_ERR_WORKSPACE;
-        return cuda_status(launch_gemm_i8(a, w, d.sm_count, stream));
+        return cuda_status(bits == 8 ? launch_gemm_i8(a, w, d.sm_count, stream)
+                                     : launch_gemm_i4(a, w, d.sm_count, stream));
     }
     if (c.variant == WQ_VARIANT_GEMV_RB)
         return cuda_status(launch_gemv(a, c.split, d.sm_count, stream));
@@ -421,7 +429,7 @@ size_t wq_workspace_bytes(int M, int K, int N, int max_split)
     if (M <= 32)
         b = std::max(b, ws_bytes_gemv_sk(M, N));
     if (M <= kI8MaxM && K <= kI8MaxK)
-        b = std::max(b, ws_bytes_gemm_i8(M, K, N));
+        b = std::max(b, std::max(ws_bytes_gemm_i8(M, K, N), ws_bytes_gemm_i4(M, K, N)));
     return b;
 }
 
@@ -665,11 +673,12 @@ int wq_dequant_debug(const void *Wq, const void *scales, const void *zeros, int 
 
 int wq_device_error(cudaStream_t stream)
 {
-    int a = 0, b = 0, c = 0, e = 0;
+    int a = 0, b = 0, c = 0, e = 0, f = 0;
     if (read_device_error(&a, stream) != cudaSuccess || read_gemv_sk_error(&b, stream) != cudaSuccess ||
-        read_gemm_sk_error(&c, stream) != cudaSuccess || read_gemm_i8_error(&e, stream) != cudaSuccess)
+        read_gemm_sk_error(&c, stream) != cudaSuccess || read_gemm_i8_error(&e, stream) != cudaSuccess ||
+        read_gemm_i4_error(&f, stream) != cudaSuccess)
         return WQ_ERR_CUDA;
-    return (a == 0 && b == 0 && c == 0 && e == 0) ? WQ_OK : WQ_ERR_TIMEOUT;
+    return (a == 0 && b == 0 && c == 0 && e == 0 && f == 0) ? WQ_OK : WQ_ERR_TIMEOUT;
 }
 
 } // extern "C"

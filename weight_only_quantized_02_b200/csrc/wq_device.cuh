@@ -69,15 +69,31 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
 // failure in its device error word and winds down without further waits.
 constexpr uint64_t kWaitLimitNs = 2000000000ull; // 2 s
 
+// One try_wait that may suspend the thread in hardware until the phase
+// completes or about `ns` nanoseconds pass, so a waiting thread takes no
+// issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t parity, uint32_t ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
 {
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity))
+    for (;;) {
+        if (mbar_try_wait_suspend(bar, parity, 1000000u)) // suspended for up to 1 ms per try
             return true;
-        if ((it & 255u) == 255u && globaltimer_ns() - t0 > kWaitLimitNs)
+        if (globaltimer_ns() - t0 > kWaitLimitNs)
             return false;
     }
 }

@@ -52,6 +52,7 @@
 #include <cuda_bf16.h>
 
 #include "wq_device.cuh"
+#include "wq_imma.cuh"
 #include "wq_internal.h"
 
 namespace wq {
@@ -98,93 +99,6 @@ constexpr size_t i8_smem_bytes()
     // tensor-memory slot + row maxima / exponents
     return 1024 + (size_t)I8Cfg<NR>::kStages * I8Cfg<NR>::kStageBytes + (2 * I8Cfg<NR>::kStages + 4) * 8 + 16 +
            2 * kI8MaxM * 4;
-}
-
-// Instruction descriptor, kind::i8: signed 8-bit A and B, int32 D, both
-// K-major, M = 128 (weight rows), N = n (digit rows).
-__host__ __device__ constexpr uint32_t umma_idesc_s8(int n)
-{
-    return (2u << 4)                          // D format s32
-           | (1u << 7)                        // A format signed 8-bit
-           | (1u << 10)                       // B format signed 8-bit
-           | ((uint32_t)(n >> 3) << 17)       // N >> 3
-           | ((uint32_t)(128 >> 4) << 24);    // M >> 4
-}
-
-// D(tmem) (+)= A(smem descriptor) * B(smem descriptor); kind::i8.
-__device__ __forceinline__ void umma_ss_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                           uint32_t accumulate)
-{
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "setp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-                 : "memory");
-}
-
-// 2^e as a binary64, built from its exponent field (|e| < 1000 here).
-__device__ __forceinline__ double pow2_of(int e) { return __longlong_as_double((long long)(1023 + e) << 52); }
-
-__device__ __forceinline__ uint16_t i8_output(int32_t d0, int32_t d1, int32_t d2, double scale_pow2)
-{
-    const double v = ((double)d2 * 65536.0 + (double)d1 * 256.0 + (double)d0) * scale_pow2;
-    return __bfloat16_as_ushort(__double2bfloat16(v));
-}
-
-// Exponent e_m of a token row from the largest magnitude's bf16 bits:
-// |x| < 2^(E+1), e = 21 - E gives |X| < 2^22.  Rows whose largest magnitude
-// is below 2^-106 use e = 127 (the largest power of two a binary32 holds).
-__device__ __forceinline__ int row_exponent(uint32_t amax_bits)
-{
-    if (amax_bits == 0)
-        return 0;
-    const int eb = (int)(amax_bits >> 7);
-    const int e = 21 - ((eb ? eb : 1) - 127);
-    return e > 127 ? 127 : e;
-}
-
-// 16 consecutive activations (bf16 bits in w[8]) -> the digit planes of one
-// 16-byte chunk: p[i][j] = bytes 4j..4j+3 of digit plane i.  With the fused
-// multiply-add F = x * 2^e + 1.5 * 2^23 rounded once (to nearest, ties to
-// even), the binary32 bits of F are 0x4B400000 + X for |X| < 2^22, and
-// X + 0x808080 holds the three biased digits d_i + 128 in its low three
-// bytes (the balanced base-256 expansion is unique, so no byte carries).
-__device__ __forceinline__ void digit_planes(const uint32_t (&w)[8], float s, uint32_t (&p)[3][4])
-{
-    uint32_t Y[16];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
-        Y[2 * i] = __float_as_uint(fmaf(lo, s, 12582912.0f)) - 0x4ABF7F80u;     // X + 0x808080
-        Y[2 * i + 1] = __float_as_uint(fmaf(hi, s, 12582912.0f)) - 0x4ABF7F80u;
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint32_t a01 = __byte_perm(Y[4 * j], Y[4 * j + 1], 0x5140u);     // d0 d0 d1 d1
-        const uint32_t a23 = __byte_perm(Y[4 * j + 2], Y[4 * j + 3], 0x5140u);
-        const uint32_t b01 = __byte_perm(Y[4 * j], Y[4 * j + 1], 0x0062u);     // d2 d2 . .
-        const uint32_t b23 = __byte_perm(Y[4 * j + 2], Y[4 * j + 3], 0x0062u);
-        p[0][j] = __byte_perm(a01, a23, 0x5410u) ^ 0x80808080u; // biased -> two's complement
-        p[1][j] = __byte_perm(a01, a23, 0x7632u) ^ 0x80808080u;
-        p[2][j] = __byte_perm(b01, b23, 0x5410u) ^ 0x80808080u;
-    }
-}
-
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void red_release_gpu_add(uint32_t *p, uint32_t v)
-{
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_global()
-{
-    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 template <int NR>
@@ -315,86 +229,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
         const int quad = warp & 3;
         const int K = p.K;
         // ---------------- activations: row maxima, then 1/G of the digit blocks ----------------
-        {
-            // items (token slot m, k-block, 16-k chunk); slots M .. ceil(NR/3)-1 write the zero padding rows
-            constexpr int MS = (NR + 2) / 3;
-            const long long items = (long long)MS * KB * 8;
-            const long long i0 = items * c / G, i1 = items * (c + 1) / G;
-            auto item_x = [&](long long it, uint4 &a, uint4 &b) {
-                const int m = (int)(it / (KB * 8)), rem = (int)(it % (KB * 8));
-                const int k0 = (rem >> 3) * kBlockK + 16 * (rem & 7);
-                if (m < M && k0 < K) {
-                    a = ldg_keep4(p.x + (size_t)m * K + k0);
-                    b = ldg_keep4(p.x + (size_t)m * K + k0 + 8);
-                } else { // k past K or a padding slot: zero activations (zero weights there too)
-                    a = b = make_uint4(0, 0, 0, 0);
-                }
-            };
-            // this thread's first item is loaded together with the row maxima (one round trip)
-            uint4 fa = make_uint4(0, 0, 0, 0), fb = fa;
-            if (i0 + et < i1)
-                item_x(i0 + et, fa, fb);
-            const int vpr = K / 8; // 16-byte vectors per token row
-            const long long total = (long long)M * vpr;
-            int cur_m = -1;
-            uint32_t cur = 0;
-            constexpr int BATCH = 8;
-            for (long long v0 = et; v0 < total; v0 += BATCH * 128) {
-                uint4 q[BATCH];
-#pragma unroll
-                for (int b = 0; b < BATCH; ++b) {
-                    const long long v = v0 + (long long)b * 128;
-                    q[b] = v < total ? ldg_keep4(p.x + v * 8) : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int b = 0; b < BATCH; ++b) {
-                    const long long v = v0 + (long long)b * 128;
-                    if (v >= total)
-                        break;
-                    const int m = (int)(v / vpr);
-                    if (m != cur_m) {
-                        if (cur_m >= 0)
-                            atomicMax(&s_amax[cur_m], cur);
-                        cur_m = m;
-                        cur = 0;
-                    }
-                    const uint32_t wv[4] = {q[b].x, q[b].y, q[b].z, q[b].w};
-#pragma unroll
-                    for (int h = 0; h < 4; ++h)
-                        cur = max(cur, max(wv[h] & 0x7FFFu, (wv[h] >> 16) & 0x7FFFu));
-                }
-            }
-            if (cur_m >= 0)
-                atomicMax(&s_amax[cur_m], cur);
-            named_barrier_sync(1, 128);
-            if (et < M)
-                s_e[et] = row_exponent(s_amax[et]);
-            named_barrier_sync(1, 128);
-            for (long long it = i0 + et; it < i1; it += 128) {
-                const int m = (int)(it / (KB * 8)), rem = (int)(it % (KB * 8));
-                const int kb = rem >> 3, cc = rem & 7;
-                uint4 a = fa, b = fb;
-                if (it != i0 + et)
-                    item_x(it, a, b);
-                uint32_t pl[3][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}};
-                if (m < M) {
-                    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-                    digit_planes(w, __uint_as_float((uint32_t)(127 + s_e[m]) << 23), pl); // 2^e, -106 <= e <= 127
-                }
-                uint8_t *blk = p.xd + (size_t)kb * C::kBB;
-#pragma unroll
-                for (int d = 0; d < 3; ++d) {
-                    const int jr = 3 * m + d;
-                    if (jr < NR)
-                        *reinterpret_cast<uint4 *>(blk + (jr >> 3) * 1024 + (jr & 7) * 128 + ((cc ^ (jr & 7)) << 4)) =
-                            make_uint4(pl[d][0], pl[d][1], pl[d][2], pl[d][3]);
-                }
-            }
-            fence_proxy_async_global();
-            named_barrier_sync(1, 128);
-            if (et == 0)
-                red_release_gpu_add(&p.grid[0], 1u); // cumulative over the 128 threads' stores
-        }
+        imma_digit_phase<NR>(p.x, M, K, KB, c, G, et, p.xd, s_amax, s_e, p.grid);
         // ---------------- epilogue: one thread per output channel ----------------
         const int row = 32 * quad + lane;
         const uint32_t tq = (uint32_t)(32 * quad) << 16;

@@ -42,10 +42,12 @@ inline size_t ws_bytes_gemv_sk(int M, int N)
     return ws_counter_bytes(N) + (size_t)kSkMaxCtas * 2 * 128 * tok * sizeof(float);
 }
 
-// Integer tensor-core GEMM (INT8 only): M <= kI8MaxM, K <= kI8MaxK, at most
-// kI8MaxCtas persistent CTAs.  Workspace: [tickets][exponents 256 B]
-// [digit blocks KB x NR x 128][int32 partials kI8MaxCtas x 2 x NR x 128].
+// Integer tensor-core GEMMs (W8A16 and W4A16): M <= kI8MaxM, K <= kI8MaxK, at
+// most kI8MaxCtas persistent CTAs.  Workspace: [counters][digit blocks
+// KB x NR x 128][partials: INT8 int32 kI8MaxCtas x 2 x NR x 128, INT4 fp32
+// kI8MaxCtas x 2 x NR/3 x 128].
 constexpr int kI8MaxM = 64;
+constexpr int kI4MaxM = 32; // W4A16 on the integer path
 constexpr int kI8MaxK = 65536;
 constexpr int kI8MaxCtas = 160;
 int i8_digit_rows(int M);
@@ -83,9 +85,12 @@ cudaError_t launch_gemm(const LinearArgs &a, int split, void *ws, int sm_count, 
 cudaError_t launch_gemm_sk(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st);
 cudaError_t read_gemm_sk_error(int *code, cudaStream_t st);
 
-// Integer tensor-core GEMM: ws >= ws_bytes_gemm_i8 (always needed).
+// Integer tensor-core GEMM: ws >= ws_bytes_gemm_i8 / ws_bytes_gemm_i4 (always needed).
 cudaError_t launch_gemm_i8(const LinearArgs &a, void *ws, int sm_count, cudaStream_t st);
 cudaError_t read_gemm_i8_error(int *code, cudaStream_t st);
+size_t ws_bytes_gemm_i4(int M, int K, int N);
+cudaError_t launch_gemm_i4(const LinearArgs &a, void *ws, int sm_count, cudaStream_t st);
+cudaError_t read_gemm_i4_error(int *code, cudaStream_t st);
 
 // Reads and clears the device error word of the current device.
 cudaError_t read_device_error(int *code, cudaStream_t st);

@@ -188,12 +188,12 @@ class ClockSampler:
                 "power_w_median": statistics.median(power) if power else None}
 
 
-def profile_traffic(kernel_file: str, summary_name: str, M: int):
+def profile_traffic(src_file: str, summary_name: str, M: int):
     """DRAM bytes per launch (read + write) of this kernel at this M, from the
     committed ncu summary -- only if it was captured on the current kernel
     source (its sha256 is recorded in the summary)."""
     path = os.path.join(ROOT, "profiles", summary_name)
-    src = os.path.join(ROOT, "weight_only_quantized_02_b200", "csrc", kernel_file)
+    src = os.path.join(ROOT, "weight_only_quantized_02_b200", "csrc", src_file)
     try:
         text = open(path).read()
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
@@ -244,11 +244,18 @@ def build_weights(name, device, copies):
 
 
 KERNELS = {0: ("gemv_sk", "wq_gemv_sk.cu"), 1: ("gemm", "wq_gemm.cu"), 2: ("gemv_rb", "wq_gemv.cu"),
-           3: ("gemm_sk", "wq_gemm_sk.cu"), 4: ("gemm_i8", "wq_gemm_i8.cu")}
+           3: ("gemm_sk", "wq_gemm_sk.cu"), 4: ("gemm_i8", "wq_gemm_i8.cu"), 5: ("gemv_i8", "wq_gemv_i8.cu")}
 
 
 def kernel_name(variant, bits):
     return KERNELS[variant][0] + f"_w{bits}"
+
+
+def kernel_file(variant, bits):
+    """Source file of a variant's kernel (the integer path has one per format)."""
+    if variant == 4 and bits == 4:
+        return "wq_gemm_i4.cu"
+    return KERNELS[variant][1]
 
 
 def bench_ours(args, device, rank, world):
@@ -369,7 +376,7 @@ def bench_ours(args, device, rank, world):
     Mdom = max(Ms, key=lambda m: share[m])
     dom = next(p for p in per_shape if p["M"] == Mdom)
     vdom = choices[Mdom][0]
-    kfile = KERNELS[vdom][1]
+    kfile = kernel_file(vdom, bits)
     summary = f"{dom['variant']}_{name}.md"
     traffic = profile_traffic(kfile, summary, Mdom)
     bound = "hbm"

@@ -16,7 +16,7 @@
  *          layout, scales, zero points and group size. This is the review of
  *          Figure 4 in "Toward a Cleaner Quantization Stack in SGLang".)
  *
- * Three kernel families sit behind one call:
+ * Four kernel families sit behind one call:
  *   - a GEMV for decode-sized M, with register-level dequantization and
  *     128-bit weight loads ("BitBLAS-style GEMV", tileInfer README, Features
  *     table). Its fp32 dot products run on mma.sync tensor-core fragments.
@@ -30,6 +30,10 @@
  *     (three base-256 digits) and every element within 2^14 of the row's
  *     largest is exact. The sums over k are exact int32, and
  *     y = s * 2^-e * sum is formed in binary64 before the bf16 rounding.
+ *   - the integer GEMV (M <= 8): the same integer sums on mma.sync
+ *     m16n8k32 s8 fragments taken straight from the packed codes; for
+ *     W4A16 the zero point enters through the activations' digit sum per
+ *     group and the group scale is applied in fp32 per group.
  * A per-(M,K,N,bits,group) dispatcher picks the kernel and split factor. It
  * starts from an untuned rule (W8A16 within the integer path's limits -> the
  * integer path; otherwise the pages' rule: fewer than 8 tokens -> GEMV, else
@@ -89,6 +93,10 @@ typedef enum {
 #define WQ_VARIANT_GEMM_SK 3 /* stream-K tcgen05 GEMM, M <= 128, persistent; needs the workspace */
 #define WQ_VARIANT_I8MMA 4   /* stream-K tcgen05 kind::i8: W8A16 (M <= 64) on the raw codes,
                                 W4A16 (M <= 32) on q - z; K <= 65536; needs the workspace */
+#define WQ_VARIANT_GEMV_I8 5 /* warp-level stream-K GEMV on mma.sync m16n8k32 s8 (the packed codes
+                                as they are, activations as exact digits in shared memory), M <= 8,
+                                3 * M * K bytes <= ~200 KB; split = CTAs per SM (1..3); needs the
+                                workspace */
 
 /* Static description of a status code. Host. Never NULL. */
 const char *wq_strerror(int status);
@@ -183,6 +191,7 @@ int wq_linear(const uint16_t *x, int M, int K, const void *Wq, const void *scale
  * GEMM_SK: split = CTAs per SM, 1 or 2, capped by the tile's resources.
  * GEMM: split = K-splits, 1 <= split <= min(32, ceil(K/128)).
  * I8MMA: split = 1 (one persistent CTA per SM).
+ * GEMV_I8: split = CTAs per SM, 1..3, capped by occupancy.
  * Returns WQ_ERR_VARIANT if the pair does not fit the shape. */
 int wq_linear_forced(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
                      const void *zeros, int group, int N, uint16_t *y, int variant, int split,
@@ -215,8 +224,9 @@ int wq_linear_noalloc(const uint16_t *x, int M, int K, const void *Wq, const voi
 /* Bytes of workspace for M tokens, a K x N weight and GEMM splits up to
  * max_split: enough for every variant of that shape. It holds eight ticket
  * counters per 128-channel panel and the largest of the GEMM's fp32
- * partials [split][M][N], the stream-K kernels' per-CTA panel partials, and
- * the integer path's int32 per-CTA partials. Returns 0 for M, K, N or
+ * partials [split][M][N], the stream-K kernels' per-CTA panel partials,
+ * the integer path's int32 per-CTA partials, and the integer GEMV's
+ * per-warp partials. Returns 0 for M, K, N or
  * max_split < 1. Host. */
 size_t wq_workspace_bytes(int M, int K, int N, int max_split);
 

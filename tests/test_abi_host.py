@@ -72,6 +72,8 @@ def test_workspace_bytes():
     assert wq.wq_workspace_bytes(128, 5120, 5120, 32) == 1536 + 32 * 128 * 5120 * 4
     assert wq.wq_workspace_bytes(64, 5120, 5120, 1) == 1536 + 512 * 2 * 128 * 64 * 4
     assert wq.wq_workspace_bytes(16, 5120, 5120, 1) == 1536 + 512 * 2 * 128 * 16 * 4
+    # M = 8: the integer GEMV's per-warp partials 448 CTAs x 8 warps x 2 x 16 rows x 24 x 4 bytes
+    assert wq.wq_workspace_bytes(8, 5120, 5120, 1) == 1536 + 448 * 8 * 2 * 16 * 24 * 4
     assert wq.wq_workspace_bytes(1, 5120, 17408, 1) == 4608 + 512 * 2 * 128 * 16 * 4  # 136 panels -> 1090 words -> 4608 bytes
     # integer path, M = 1 (16 digit rows): int32 partials 160 CTAs x 2 x 16 x 128
     assert 160 * 2 * 16 * 128 * 4 < 512 * 2 * 128 * 16 * 4
@@ -88,7 +90,8 @@ def test_null_pointer_checks_need_no_device():
 def test_tuning_file_parse_errors(tmp_path):
     good = tmp_path / "good.txt"
     good.write_text("# comment\nNVIDIA B200|148 1 5120 17408 8 0 0 4 12.500\n"
-                    "NVIDIA B200|148 4 5120 17408 8 0 4 1 9.000\n")
+                    "NVIDIA B200|148 4 5120 17408 8 0 4 1 9.000\n"
+                    "NVIDIA B200|148 2 5120 25600 4 128 5 2 20.000\n")
     assert wq.wq_load_tuning(str(good)) == 0
     for bad_line in [
         "NVIDIA B200|148 1 5120 17408 8 0 2 3 12.5\n",      # row-block GEMV split must be 1/2/4/8
@@ -102,6 +105,9 @@ def test_tuning_file_parse_errors(tmp_path):
         "NVIDIA B200|148 65 5120 17408 8 0 4 1 9.0\n",      # integer path: M <= 64
         "NVIDIA B200|148 33 5120 17408 4 128 4 1 9.0\n",    # integer path, W4A16: M <= 32
         "NVIDIA B200|148 4 5120 17408 8 0 4 2 9.0\n",       # integer path: split 1 only
+        "NVIDIA B200|148 9 5120 17408 8 0 5 1 9.0\n",       # integer GEMV: M <= 8
+        "NVIDIA B200|148 8 65536 17408 8 0 5 1 9.0\n",      # integer GEMV: digit rows over 200 KB
+        "NVIDIA B200|148 4 5120 17408 4 128 5 4 9.0\n",     # integer GEMV: 1..3 CTAs per SM
     ]:
         p = tmp_path / "bad.txt"
         p.write_text(bad_line)

@@ -22,8 +22,9 @@ from wqtest_helpers import (assert_parity, bf16_dev, dev, i8_fixed_point, oracle
 
 pytestmark = pytest.mark.gpu
 
-GEMV, GEMM, GEMV_RB, GEMM_SK, I8 = (wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB,
-                                    wq.WQ_VARIANT_GEMM_SK, wq.WQ_VARIANT_I8MMA)
+GEMV, GEMM, GEMV_RB, GEMM_SK, I8, GI = (wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB,
+                                        wq.WQ_VARIANT_GEMM_SK, wq.WQ_VARIANT_I8MMA, wq.WQ_VARIANT_GEMV_I8)
+INTEGER = (I8, GI)  # the integer paths: fixed-point activations
 SHAPES = {8: (1120, 400), 4: (1152, 400)}  # (K, N): 3 full panels + a 16-row tail
 M_ALL = [1, 7, 8, 9, 16, 17, 32, 33, 64, 65, 100, 128]
 
@@ -55,6 +56,8 @@ def _cases(M, K, bits):
     out += [(GEMM_SK, c) for c in (1, 2)]
     if M <= (64 if bits == 8 else 32):  # integer tensor-core path: W8A16 M <= 64, W4A16 M <= 32
         out += [(I8, 1)]
+    if M <= 8:  # integer GEMV
+        out += [(GI, c) for c in (1, 2, 3)]
     return out
 
 
@@ -85,7 +88,8 @@ def test_repeated_dispatch_resets_tickets(weight, ws):
     each must leave them at zero for the next (different variant, split, M)."""
     bits, K, N, pw, canon = weight
     runs = [(GEMM, 16, 2), (GEMM, 16, 8), (GEMM_SK, 40, 2), (GEMV, 5, 3), (GEMM, 40, 4), (GEMM, 128, 9),
-            (I8, 5, 1), (I8, 40 if bits == 8 else 30, 1), (GEMV, 3, 2), (I8, 1, 1)]
+            (I8, 5, 1), (I8, 40 if bits == 8 else 30, 1), (GEMV, 3, 2), (I8, 1, 1), (GI, 1, 2), (GI, 8, 1),
+            (GEMM_SK, 7, 1), (GI, 4, 3), (I8, 3, 1), (GI, 6, 2)]
     runs += [(GEMM, 16, 2)]
     for variant, M, split in runs:
         x = gen.x_bf16(M, K)
@@ -141,7 +145,7 @@ def test_one_hot_int8_weights_exact(ws):
     want = oracle.bf16_to_f64(oracle.bf16_rne_of(oracle.linear_int8(x, q, s)))
     for variant, split in _all_cases(M, K, 8):
         y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
-        if variant == I8:
+        if variant in INTEGER:
             # exact on its fixed-point activations, and within the layer's tolerance of the oracle
             assert np.array_equal(y, _i8_want_one_hot(x, q, s)), (variant, split)
             assert_parity(y, oracle.linear_int8(x, q, s), "one-hot int8 weights, integer path")
@@ -176,11 +180,19 @@ def test_one_hot_int4_weights_exact(ws):
     prod = np.float32(X[:, cols] * d[None, :]).astype(np.float64)  # one binary32 rounding
     sc = oracle.bf16_to_f64(s[np.arange(N), cols // G])
     want_i8 = oracle.bf16_to_f64(oracle.bf16_rne_of(np.ldexp(prod * sc[None, :], -e[:, None])))
+    # integer GEMV: per digit plane s * fp32((q - z) d_i), exact here, recombined in binary64; a row
+    # block split between warps passes through one binary32 partial before the bf16 rounding
+    exact = np.ldexp(X[:, cols] * d[None, :] * sc[None, :], -e[:, None])
+    want_gi = oracle.bf16_to_f64(oracle.bf16_rne_of(exact))
+    want_gi32 = oracle.bf16_to_f64(oracle.bf16_rne_of(np.float32(exact).astype(np.float64)))
     for variant, split in _all_cases(M, K, 4):
         y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
         if variant == I8:
             assert np.array_equal(y, want_i8), (variant, split)
             assert_parity(y, oracle.linear_int4(x, q, s, z), "one-hot int4 weights, integer path")
+        elif variant == GI:
+            assert np.all((y == want_gi) | (y == want_gi32)), (variant, split)
+            assert_parity(y, oracle.linear_int4(x, q, s, z), "one-hot int4 weights, integer GEMV")
         else:
             assert np.array_equal(y, want), (variant, split)
 
@@ -206,7 +218,7 @@ def test_identity_weights_reproduce_x(bits, ws):
     want_i8 = oracle.bf16_to_f64(oracle.bf16_rne_of(i8_fixed_point(x)))
     for variant, split in _all_cases(M, K, bits):
         y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
-        assert np.array_equal(y, want_i8 if variant == I8 else want), (variant, split)
+        assert np.array_equal(y, want_i8 if variant in INTEGER else want), (variant, split)
 
 
 @pytest.mark.parametrize("bits", [8, 4])
@@ -264,12 +276,17 @@ def test_argument_errors(weight, ws):
     assert wq.wq_linear_status(x, pw, y, GEMM, 33) == -11         # split above 32
     assert wq.wq_linear_status(x, pw, y, 7, 1) == -11             # unknown variant
     assert wq.wq_linear_status(x, pw, y, I8, 2) == -11            # one CTA per SM only
+    assert wq.wq_linear_status(x, pw, y, GI, 4) == -11            # integer GEMV: 1..3 CTAs per SM
+    assert wq.wq_linear_status(x, pw, y, GI, 0) == 0              # 0: the default
     xc = bf16_dev(gen.x_bf16(65, K))
     yc = torch.empty((65, N), dtype=torch.bfloat16, device=dev())
     assert wq.wq_linear_status(xc, pw, yc, I8, 1) == -11          # integer path takes M <= 64 (W4A16: 32)
     xd33 = bf16_dev(gen.x_bf16(33, K))
     yd33 = torch.empty((33, N), dtype=torch.bfloat16, device=dev())
     assert wq.wq_linear_status(xd33, pw, yd33, I8, 1) == (0 if bits == 8 else -11)
+    x9 = bf16_dev(gen.x_bf16(9, K))
+    y9 = torch.empty((9, N), dtype=torch.bfloat16, device=dev())
+    assert wq.wq_linear_status(x9, pw, y9, GI, 1) == -11          # integer GEMV takes M <= 8
     xb = bf16_dev(gen.x_bf16(40, K))
     yb = torch.empty((40, N), dtype=torch.bfloat16, device=dev())
     assert wq.wq_linear_status(xb, pw, yb, GEMV, 1) == -11        # GEMV takes M <= 32
@@ -283,6 +300,7 @@ def test_argument_errors(weight, ws):
         assert wq.wq_linear_status(x, pw, y, GEMM, 4) == -6
         assert wq.wq_linear_status(x, pw, y, GEMV, 1) == -6
         assert wq.wq_linear_status(x, pw, y, I8, 1) == -6
+        assert wq.wq_linear_status(x, pw, y, GI, 2) == -6
         assert wq.wq_linear_status(x, pw, y, GEMM, 1) == 0
         assert wq.wq_linear_status(x, pw, y, GEMV_RB, 2) == 0
         assert wq.wq_linear_status(x, pw, y) == 0  # dispatcher falls back to the row-block GEMV
@@ -317,7 +335,8 @@ def test_explicit_workspace_on_two_streams(weight):
 
 def test_cuda_graph_replay(weight, ws):
     bits, K, N, pw, canon = weight
-    runs = [(1, GEMV, 2), (1, GEMV_RB, 4), (16, GEMM, 4), (128, GEMM, 2), (1, I8, 1), (16, I8, 1)]
+    runs = [(1, GEMV, 2), (1, GEMV_RB, 4), (16, GEMM, 4), (128, GEMM, 2), (1, I8, 1), (16, I8, 1), (1, GI, 2),
+            (7, GI, 1)]
     for M, variant, split in runs:
         x = gen.x_bf16(M, K)
         xd = bf16_dev(x)

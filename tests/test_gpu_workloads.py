@@ -19,8 +19,8 @@ from wqtest_helpers import assert_parity, bf16_dev, bits_u16, bits_u32, dev, wor
 
 pytestmark = pytest.mark.gpu
 
-GEMV, GEMM, GEMV_RB, GEMM_SK, I8 = (wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB,
-                                    wq.WQ_VARIANT_GEMM_SK, wq.WQ_VARIANT_I8MMA)
+GEMV, GEMM, GEMV_RB, GEMM_SK, I8, GI = (wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB,
+                                        wq.WQ_VARIANT_GEMM_SK, wq.WQ_VARIANT_I8MMA, wq.WQ_VARIANT_GEMV_I8)
 
 
 def _build(name):
@@ -80,6 +80,8 @@ def _variants(M, K, bits):
     out += [(GEMM_SK, c) for c in (1, 2)]
     if M <= (64 if bits == 8 else 32):  # integer tensor-core path: W8A16 M <= 64, W4A16 M <= 32
         out += [(I8, 1)]
+    if M <= 8:  # integer GEMV
+        out += [(GI, c) for c in (1, 2)]
     return out
 
 

@@ -121,6 +121,8 @@ bool choice_valid(int variant, int split, int M, int K, int bits)
 {
     if (variant == WQ_VARIANT_I8MMA)
         return i8_fits(bits, M, K) && split == 1;
+    if (variant == WQ_VARIANT_GEMV_I8)
+        return gi_fits(bits, M, K) && split >= 1 && split <= 3;
     if (variant == WQ_VARIANT_GEMV)
         return M <= 32 && split >= 1 && split <= 4;
     if (variant == WQ_VARIANT_GEMV_RB)
@@ -215,6 +217,7 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
         return WQ_ERR_ALIGN;
     const bool sk_ws_ok = w && have >= ws_bytes_gemv_sk(M, N);
     const bool i8_ws_ok = w && i8_fits(bits, M, K) && have >= ws_bytes_imma(bits, M, K, N);
+    const bool gi_ws_ok = w && gi_fits(bits, M, K) && have >= ws_bytes_gemv_i8(M, K, N);
 
     Choice c;
     lookup_choice(d, M, K, N, bits, group, &c);
@@ -225,12 +228,14 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
                       : variant == WQ_VARIANT_GEMV_RB ? default_rb_slices(K, N, d.sm_count)
                       : variant == WQ_VARIANT_GEMM_SK ? 2
                       : variant == WQ_VARIANT_I8MMA   ? 1
+                      : variant == WQ_VARIANT_GEMV_I8 ? 2
                                                       : std::min(8, max_gemm_split(K));
     }
     if (split > 0)
         c.split = split;
     if (variant == WQ_VARIANT_AUTO) {
-        if (!choice_valid(c.variant, c.split, M, K, bits) || (c.variant == WQ_VARIANT_I8MMA && !i8_ws_ok))
+        if (!choice_valid(c.variant, c.split, M, K, bits) || (c.variant == WQ_VARIANT_I8MMA && !i8_ws_ok) ||
+            (c.variant == WQ_VARIANT_GEMV_I8 && !gi_ws_ok))
             c = default_choice(M, K, N, bits, d.sm_count, sk_ws_ok, i8_ws_ok);
         if (c.variant == WQ_VARIANT_GEMV && !sk_ws_ok)
             c = {WQ_VARIANT_GEMV_RB, default_rb_slices(K, N, d.sm_count), 0.f};
@@ -245,6 +250,11 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
         return WQ_ERR_VARIANT;
 
     LinearArgs a{x, M, K, N, Wq, scales, zeros, bits, group, y};
+    if (c.variant == WQ_VARIANT_GEMV_I8) {
+        if (!gi_ws_ok)
+            return WQ_ERR_WORKSPACE;
+        return cuda_status(launch_gemv_i8(a, c.split, w, d.sm_count, stream));
+    }
     if (c.variant == WQ_VARIANT_I8MMA) {
         if (!i8_ws_ok)
             return WQ_ERR_WORKSPACE;
@@ -430,6 +440,8 @@ size_t wq_workspace_bytes(int M, int K, int N, int max_split)
         b = std::max(b, ws_bytes_gemv_sk(M, N));
     if (M <= kI8MaxM && K <= kI8MaxK)
         b = std::max(b, std::max(ws_bytes_gemm_i8(M, K, N), ws_bytes_gemm_i4(M, K, N)));
+    if (M <= kGiMaxM && K <= kI8MaxK)
+        b = std::max(b, ws_bytes_gemv_i8(M, K, N));
     return b;
 }
 
@@ -481,6 +493,9 @@ int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
         cands.push_back({WQ_VARIANT_GEMM_SK, c});
     if (i8_fits(bits, M, K))
         cands.push_back({WQ_VARIANT_I8MMA, 1});
+    if (gi_fits(bits, M, K))
+        for (int c : {1, 2})
+            cands.push_back({WQ_VARIANT_GEMV_I8, c});
 
     // Flush buffer larger than L2, so every timed call streams its weights
     // from HBM (the weights of a decode step are not L2-resident).

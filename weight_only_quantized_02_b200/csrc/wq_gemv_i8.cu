@@ -1,0 +1,537 @@
+// wq_gemv_i8.cu -- decode-regime GEMV (M <= 8) on the integer mma.sync
+// path: mma.sync m16n8k32 s8 x s8 -> s32 straight on the packed weight
+// codes, the activations as exact base-256 digits.
+//
+// The sum over k of the weight-only linear layer is an integer sum once the
+// activations are integers ("Per-channel W8A16 quantization" and
+// "Group-wise W4A16 quantization", tileInfer README, Features table):
+//     W8A16:  y[m][n] = s[n] 2^-e_m sum_k q[n][k] X[m][k]
+//     W4A16:  y[m][n] = 2^-e_m sum_g s[g][n] (sum_{k in g} q[n][k] X[m][k] - z[g][n] sum_{k in g} X[m][k])
+// with X = round(x 2^e_m) = d0 + 256 d1 + 65536 d2 (the activations'
+// fixed-point form of the integer tensor-core kernels, wq_imma.cuh).  The
+// A operand of every MMA is the packed weights exactly as they sit in HBM:
+// INT8 codes need no instruction at all, INT4 codes one mask (and one shift)
+// per 4 nibbles; the zero point becomes one integer multiply-add per output
+// and group with the digit sum of the group.  The bf16-dequantizing GEMV
+// spends several instructions per weight and is issue-bound below HBM
+// bandwidth at decode sizes; this one issues a fraction of that.
+//
+// Activations: every CTA first turns all of x into digit rows in its own
+// shared memory (row maxima, then the digits; M*K values, a few tens per
+// thread at decode sizes), so no CTA waits for another and the B fragments
+// come from shared memory.  The digit rows' byte order inside a 128-k block
+// matches the weights' k order (INT8: natural; INT4: the nibble order of
+// the packed mma tiles, see gi_digits), so a lane's B fragment is one
+// contiguous load.
+//
+// Work split: warp-level stream-K.  The items (16-row block, 128-k block),
+// row-block-major, are cut into G*8 equal contiguous ranges, one per warp;
+// each warp streams its range through a D-deep ring of register prefetches
+// (the first D issued before the programmatic-launch wait: weights never
+// depend on the preceding kernel).  A row block whose k range is split
+// between warps is finished by the last contributor to take the block's
+// ticket (acquire-release, never waited on): it sums the partials in warp
+// order and writes y (INT8 partials are exact integers).
+#include <cstdint>
+
+#include <cuda_bf16.h>
+
+#include "wq_device.cuh"
+#include "wq_imma.cuh"
+#include "wq_internal.h"
+
+namespace wq {
+
+constexpr int kGiWarps = 8;
+constexpr int kGiThreads = 32 * kGiWarps;
+
+struct GiParams {
+    const uint16_t *x;
+    int M, K, N, KB;
+    int I;          // items = (N / 16) * KB
+    const uint8_t *wq;
+    const uint16_t *scales;
+    const uint8_t *zeros;
+    uint16_t *y;
+    uint32_t *part; // [G * 8 warps][2 slots][16 rows][NR] partials
+    uint32_t *cnt;  // one ticket per 16-row block
+};
+
+// Prefetch depth (items in flight per warp) by weight format.
+template <int BITS>
+struct GiCfg {
+    static constexpr int D = BITS == 8 ? 4 : 6;
+};
+
+__device__ __forceinline__ void imma_16832(int32_t (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 "
+                 "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Shared-memory digit rows: row 3m + i (digit i of token m) of S bytes,
+// S = 128 * KB + 64 (INT8) or K + 16 (INT4): the stride puts the two rows a
+// quarter-warp reads in different banks.  INT4 adds the digit sums of every
+// row and 128-k block.
+template <int BITS>
+__host__ __device__ constexpr int gi_row_stride(int K)
+{
+    return BITS == 8 ? (K + 127) / 128 * 128 + 64 : K + 16;
+}
+
+// The activations of the whole layer as digit rows in shared memory (all
+// 256 threads): the row maxima (e_m), then every 16-k chunk of every token
+// row, thread ch = chunk % 8 of each group of eight converting k = 16 c ..
+// 16 c + 15 (zero past K).  Each CTA converts all of x (M*K values, a few
+// tens per thread at decode sizes) and no CTA waits for another.  Digit row
+// 3m + i of block kb holds its 128 bytes in the order the B fragments read:
+//   INT8: natural, byte kk holds k = kk (a lane's 16-byte weight chunk and
+//         its 16 digit bytes cover the same k).
+//   INT4: byte 32 t + 8 st + 2 a + s holds k = 32 st + 16 s + 4 t + a: the
+//         packed mma tile gives lane t of 32-k step st the nibbles of
+//         k = 4t + a (low nibbles) and 16 + 4t + a (high nibbles) interleaved,
+//         so a lane's 32 bytes of a block are its four steps' B fragments.
+template <int BITS, int NR>
+__device__ __forceinline__ void gi_digits(const GiParams &p, uint8_t *sd, int32_t *s_dsum, uint32_t *s_amax,
+                                          int *s_e)
+{
+    const int et = threadIdx.x, ch = et & 7;
+    const int M = p.M, K = p.K, KB = p.KB;
+    const int S = gi_row_stride<BITS>(K);
+    imma_row_maxima<kGiThreads, 2>(p.x, M, K, et, s_amax); // few registers: the weight prefetch is live
+    __syncthreads();
+    if (et < M)
+        s_e[et] = row_exponent(s_amax[et]);
+    __syncthreads();
+    const int cpr = KB * 8; // 16-k chunks per token row
+    const int items = M * cpr;
+    for (int base = 0; base < items; base += kGiThreads) { // uniform trip count: shuffles below
+        const int it = base + et;
+        const bool act = it < items;
+        const int m = act ? it / cpr : 0, c = act ? it % cpr : 0; // chunk c: k = 16c .. 16c + 15
+        uint4 a = make_uint4(0, 0, 0, 0), b = a;
+        if (act && 16 * c < K) {
+            const uint16_t *src = p.x + (size_t)m * K + 16 * c;
+            a = ldg_keep4(src);
+            b = ldg_keep4(src + 8);
+        }
+        uint32_t pl[3][4];
+#pragma unroll
+        for (int i = 0; i < 3; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                pl[i][j] = 0u;
+        if (act) {
+            const float sc = __uint_as_float((uint32_t)(127 + s_e[m]) << 23); // 2^e
+            const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            digit_planes(w, sc, pl);
+        }
+        if constexpr (BITS == 8) {
+            if (act) {
+#pragma unroll
+                for (int i = 0; i < 3; ++i)
+                    *reinterpret_cast<uint4 *>(sd + (3 * m + i) * S + 16 * c) =
+                        make_uint4(pl[i][0], pl[i][1], pl[i][2], pl[i][3]);
+            }
+        } else {
+            const int kb = c >> 3, s = ch & 1, st = ch >> 1;
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {
+                uint32_t o[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    o[j] = __shfl_xor_sync(0xffffffffu, pl[i][j], 1);
+                // lo: the chunk of step st with s = 0, hi: with s = 1
+                uint32_t lo[4], hi[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    lo[j] = s ? o[j] : pl[i][j];
+                    hi[j] = s ? pl[i][j] : o[j];
+                }
+                int sum = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    sum = __dp4a((int)pl[i][j], 0x01010101, sum);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+                if (act) {
+                    uint8_t *row = sd + (3 * m + i) * S + kb * 128 + 8 * st;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) { // this thread writes lanes t = 2s, 2s + 1
+                        const int t = 2 * s + h;
+                        const uint32_t x0 = s ? lo[2 + h] : lo[h], x1 = s ? hi[2 + h] : hi[h];
+                        *reinterpret_cast<uint2 *>(row + 32 * t) =
+                            make_uint2(__byte_perm(x0, x1, 0x5140u), __byte_perm(x0, x1, 0x7362u));
+                    }
+                    if (ch == 0)
+                        s_dsum[kb * NR + 3 * m + i] = sum;
+                }
+            }
+        }
+    }
+    __syncthreads();
+}
+
+// End of a warp's segment of row block rb: the accumulators are in red
+// ([16 rows][NR]; INT8 int32 digit sums D_i, INT4 fp32 group-scaled sums
+// A_i).  Writes y, or the warp's partial and its ticket; the last arriver
+// sums all partials in warp order and writes y.
+template <int BITS, int NR>
+__device__ __forceinline__ void gi_flush(const GiParams &p, int rb, bool whole, int slot, int w, int Wt,
+                                      uint32_t *red, const int *s_e, int lane)
+{
+    const int M = p.M, N = p.N, KB = p.KB;
+    const int n0 = 16 * rb;
+    __syncwarp();
+    if constexpr (BITS == 8) {
+        if (whole) {
+            for (int q = lane; q < 16 * M; q += 32) {
+                const int r = q & 15, m = q >> 4;
+                const int32_t *d = reinterpret_cast<const int32_t *>(red) + r * NR + 3 * m;
+                const double sc = (double)bf16_bits_to_float(p.scales[n0 + r]) * pow2_of(-s_e[m]);
+                p.y[(size_t)m * N + n0 + r] = i8_output(d[0], d[1], d[2], sc);
+            }
+            __syncwarp();
+            return;
+        }
+        uint32_t *mine = p.part + ((size_t)w * 2 + slot) * 16 * NR;
+        for (int i = lane; i < 16 * NR; i += 32)
+            mine[i] = red[i];
+    } else {
+        uint32_t *mine = p.part + ((size_t)w * 2 + slot) * 16 * NR;
+        for (int q = lane; q < 16 * M; q += 32) {
+            const int r = q & 15, m = q >> 4;
+            const float *a = reinterpret_cast<const float *>(red) + r * NR + 3 * m;
+            const double v = ((double)a[2] * 65536.0 + (double)a[1] * 256.0 + (double)a[0]) * pow2_of(-s_e[m]);
+            if (whole)
+                p.y[(size_t)m * N + n0 + r] = __bfloat16_as_ushort(__double2bfloat16(v));
+            else
+                mine[r * NR + m] = __float_as_uint((float)v);
+        }
+        if (whole) {
+            __syncwarp();
+            return;
+        }
+    }
+    __syncwarp();
+    uint32_t ticket = 0;
+    if (lane == 0)
+        ticket = ticket_take_acq_rel(&p.cnt[rb]);
+    ticket = __shfl_sync(0xffffffffu, ticket, 0);
+    const int wf = sk_owner(p.I, Wt, rb * KB), wl = sk_owner(p.I, Wt, rb * KB + KB - 1);
+    if (ticket == (uint32_t)(wl - wf)) {
+        __syncwarp(); // lane 0's acquire orders every lane's reads below
+        for (int q = lane; q < 16 * M; q += 32) {
+            const int r = q & 15, m = q >> 4;
+            if constexpr (BITS == 8) {
+                int32_t t0 = 0, t1 = 0, t2 = 0;
+                for (int ww = wf; ww <= wl; ++ww) {
+                    const int sl = (sk_start(p.I, Wt, ww) / KB == rb) ? 0 : 1;
+                    const int32_t *src =
+                        reinterpret_cast<const int32_t *>(p.part) + ((size_t)ww * 2 + sl) * 16 * NR + r * NR + 3 * m;
+                    t0 += __ldcg(src);
+                    t1 += __ldcg(src + 1);
+                    t2 += __ldcg(src + 2);
+                }
+                const double sc = (double)bf16_bits_to_float(p.scales[n0 + r]) * pow2_of(-s_e[m]);
+                p.y[(size_t)m * N + n0 + r] = i8_output(t0, t1, t2, sc);
+            } else {
+                float tot = 0.f;
+                for (int ww = wf; ww <= wl; ++ww) {
+                    const int sl = (sk_start(p.I, Wt, ww) / KB == rb) ? 0 : 1;
+                    tot += __ldcg(reinterpret_cast<const float *>(p.part) + ((size_t)ww * 2 + sl) * 16 * NR + r * NR + m);
+                }
+                p.y[(size_t)m * N + n0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(tot));
+            }
+        }
+        if (lane == 0)
+            atomicExch(&p.cnt[rb], 0u); // ready for the next call
+    }
+    __syncwarp();
+}
+
+template <int BITS, int NT>
+__global__ void __launch_bounds__(kGiThreads) gemv_i8_kernel(const GiParams p)
+{
+    constexpr int NR = 8 * NT;
+    constexpr int D = GiCfg<BITS>::D;
+    constexpr int WV = BITS == 8 ? 4 : 2; // 16-byte weight loads per lane and item
+    extern __shared__ __align__(16) uint8_t sd[]; // digit rows [3M][S], then (INT4) digit sums [KB][NR]
+    __shared__ uint32_t s_amax[kGiMaxM];
+    __shared__ int s_e[kGiMaxM];
+    __shared__ uint32_t s_red[kGiWarps][16 * NR];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int G = gridDim.x, c = blockIdx.x;
+    const int Wt = G * kGiWarps, w = c * kGiWarps + warp;
+    const int KB = p.KB, M = p.M;
+    const int S = gi_row_stride<BITS>(p.K);
+    int32_t *s_dsum = reinterpret_cast<int32_t *>(sd + 3 * M * S);
+    const int i0 = sk_start(p.I, Wt, w), i1 = sk_start(p.I, Wt, w + 1);
+    const int n = i1 - i0;
+
+    // ---------------- weights of the first D items (before the launch wait) ----------------
+    uint4 wb[D][WV];
+    uint32_t sz[D][2]; // INT4: bf16 scales of rows g, g+8 | their zero-point bytes
+    auto load_item = [&](int rb, int kb, uint4 (&v)[WV], uint32_t (&e)[2]) {
+        const int blk = (rb >> 3) * KB + kb, j = rb & 7;
+        if constexpr (BITS == 8) {
+            const uint8_t *b = p.wq + ((size_t)blk << 14) + (j << 11) + (g << 7);
+            v[0] = ldg_stream(b + ((t ^ g) << 4));              // row g,     chunk t
+            v[1] = ldg_stream(b + 1024 + ((t ^ g) << 4));       // row g + 8, chunk t
+            v[2] = ldg_stream(b + (((t + 4) ^ g) << 4));        // row g,     chunk t + 4
+            v[3] = ldg_stream(b + 1024 + (((t + 4) ^ g) << 4)); // row g + 8, chunk t + 4
+        } else {
+            const uint8_t *b = p.wq + (((size_t)blk * 8 + j) << 10) + 16 * lane;
+            v[0] = ldg_stream(b);
+            v[1] = ldg_stream(b + 512);
+            const uint16_t *sp = p.scales + (size_t)blk * kPanelRows + 16 * j + g;
+            e[0] = (uint32_t)__ldg(sp) | ((uint32_t)__ldg(sp + 8) << 16);
+            const uint8_t *zp = p.zeros + (size_t)blk * 64 + 8 * j + (g >> 1);
+            e[1] = (uint32_t)__ldg(zp) | ((uint32_t)__ldg(zp + 4) << 8);
+        }
+    };
+    int lrb = n > 0 ? i0 / KB : 0, lkb = n > 0 ? i0 % KB : 0; // next item to load
+    const int rb_first = lrb;
+#pragma unroll
+    for (int s = 0; s < D; ++s) {
+        if (s < n) {
+            load_item(lrb, lkb, wb[s], sz[s]);
+            if (++lkb == KB) {
+                lkb = 0;
+                ++lrb;
+            }
+        }
+    }
+
+    // ---------------- activations: this CTA's digit rows ----------------
+    if (threadIdx.x < kGiMaxM)
+        s_amax[threadIdx.x] = 0u;
+    __syncthreads();
+    pdl_wait(); // x, y and the workspace may come from / be in use by the preceding kernel
+    gi_digits<BITS, NR>(p, sd, s_dsum, s_amax, s_e);
+
+    // ---------------- stream the warp's items ----------------
+    int32_t acc_i[NT][4];
+    float acc_f[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            acc_i[nt][r] = 0;
+            acc_f[nt][r] = 0.f;
+        }
+    int crb = rb_first, ckb = n > 0 ? i0 % KB : 0, seg_kb0 = ckb;
+    const int zsh = 4 * (g & 1);
+    uint32_t *red = s_red[warp];
+    for (int j0 = 0; j0 < n; j0 += D) {
+#pragma unroll
+        for (int s = 0; s < D; ++s) {
+            const int jj = j0 + s;
+            if (jj < n) {
+                const uint8_t *xb = sd + ckb * 128;
+                if constexpr (BITS == 8) {
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const int row = 8 * nt + g;
+                        uint4 d0 = make_uint4(0, 0, 0, 0), d1 = d0;
+                        if (row < 3 * M) {
+                            d0 = *reinterpret_cast<const uint4 *>(xb + row * S + 16 * t);
+                            d1 = *reinterpret_cast<const uint4 *>(xb + row * S + 16 * (t + 4));
+                        }
+                        const uint4 *v = wb[s];
+                        imma_16832(acc_i[nt], v[0].x, v[1].x, v[0].y, v[1].y, d0.x, d0.y);
+                        imma_16832(acc_i[nt], v[0].z, v[1].z, v[0].w, v[1].w, d0.z, d0.w);
+                        imma_16832(acc_i[nt], v[2].x, v[3].x, v[2].y, v[3].y, d1.x, d1.y);
+                        imma_16832(acc_i[nt], v[2].z, v[3].z, v[2].w, v[3].w, d1.z, d1.w);
+                    }
+                } else {
+                    constexpr uint32_t lo4 = 0x0F0F0F0Fu;
+                    uint32_t a[2][8]; // per tile: lo/hi of words x, y, z, w
+#pragma unroll
+                    for (int tau = 0; tau < 2; ++tau) {
+                        const uint4 &v = wb[s][tau];
+                        a[tau][0] = v.x & lo4;
+                        a[tau][1] = (v.x >> 4) & lo4;
+                        a[tau][2] = v.y & lo4;
+                        a[tau][3] = (v.y >> 4) & lo4;
+                        a[tau][4] = v.z & lo4;
+                        a[tau][5] = (v.z >> 4) & lo4;
+                        a[tau][6] = v.w & lo4;
+                        a[tau][7] = (v.w >> 4) & lo4;
+                    }
+                    const float s_lo = __uint_as_float(sz[s][0] << 16), s_hi = __uint_as_float(sz[s][0] & 0xFFFF0000u);
+                    const int z_lo = (int)((sz[s][1] >> zsh) & 0xFu), z_hi = (int)((sz[s][1] >> (8 + zsh)) & 0xFu);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const int row = 8 * nt + g;
+                        uint4 d0 = make_uint4(0, 0, 0, 0), d1 = d0;
+                        if (row < 3 * M) {
+                            d0 = *reinterpret_cast<const uint4 *>(xb + row * S + 32 * t);
+                            d1 = *reinterpret_cast<const uint4 *>(xb + row * S + 32 * t + 16);
+                        }
+                        int32_t ci[4] = {0, 0, 0, 0};
+                        imma_16832(ci, a[0][0], a[0][2], a[0][1], a[0][3], d0.x, d0.y);
+                        imma_16832(ci, a[0][4], a[0][6], a[0][5], a[0][7], d0.z, d0.w);
+                        imma_16832(ci, a[1][0], a[1][2], a[1][1], a[1][3], d1.x, d1.y);
+                        imma_16832(ci, a[1][4], a[1][6], a[1][5], a[1][7], d1.z, d1.w);
+                        const int col = 8 * nt + 2 * t;
+                        int2 ds = make_int2(0, 0);
+                        if (col < 3 * M)
+                            ds = *reinterpret_cast<const int2 *>(s_dsum + ckb * NR + col);
+                        acc_f[nt][0] = fmaf(s_lo, (float)(ci[0] - z_lo * ds.x), acc_f[nt][0]);
+                        acc_f[nt][1] = fmaf(s_lo, (float)(ci[1] - z_lo * ds.y), acc_f[nt][1]);
+                        acc_f[nt][2] = fmaf(s_hi, (float)(ci[2] - z_hi * ds.x), acc_f[nt][2]);
+                        acc_f[nt][3] = fmaf(s_hi, (float)(ci[3] - z_hi * ds.y), acc_f[nt][3]);
+                    }
+                }
+                // refill this slot with item jj + D
+                if (jj + D < n) {
+                    load_item(lrb, lkb, wb[s], sz[s]);
+                    if (++lkb == KB) {
+                        lkb = 0;
+                        ++lrb;
+                    }
+                }
+                // end of a segment: the row block's last k-block or the warp's last item
+                if (ckb == KB - 1 || jj == n - 1) {
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const int col = 8 * nt + 2 * t;
+                        if constexpr (BITS == 8) {
+                            red[g * NR + col] = (uint32_t)acc_i[nt][0];
+                            red[g * NR + col + 1] = (uint32_t)acc_i[nt][1];
+                            red[(g + 8) * NR + col] = (uint32_t)acc_i[nt][2];
+                            red[(g + 8) * NR + col + 1] = (uint32_t)acc_i[nt][3];
+                        } else {
+                            red[g * NR + col] = __float_as_uint(acc_f[nt][0]);
+                            red[g * NR + col + 1] = __float_as_uint(acc_f[nt][1]);
+                            red[(g + 8) * NR + col] = __float_as_uint(acc_f[nt][2]);
+                            red[(g + 8) * NR + col + 1] = __float_as_uint(acc_f[nt][3]);
+                        }
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            acc_i[nt][r] = 0;
+                            acc_f[nt][r] = 0.f;
+                        }
+                    }
+                    const bool whole = seg_kb0 == 0 && ckb == KB - 1;
+                    gi_flush<BITS, NR>(p, crb, whole, crb == rb_first ? 0 : 1, w, Wt, red, s_e, lane);
+                    seg_kb0 = 0;
+                }
+                if (++ckb == KB) {
+                    ckb = 0;
+                    ++crb;
+                }
+            }
+        }
+    }
+    pdl_launch_dependents();
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+int gi_ntiles(int M) { return M <= 2 ? 1 : M <= 5 ? 2 : 3; }
+
+size_t gi_smem_bytes(int bits, int M, int K)
+{
+    const size_t KB = (size_t)(K + kBlockK - 1) / kBlockK;
+    const size_t rows = (size_t)3 * M * (bits == 8 ? gi_row_stride<8>(K) : gi_row_stride<4>(K));
+    return rows + (bits == 4 ? KB * 8 * gi_ntiles(M) * sizeof(int32_t) : 0);
+}
+
+bool gi_fits(int bits, int M, int K)
+{
+    return M >= 1 && M <= kGiMaxM && K >= 1 && K <= kI8MaxK && gi_smem_bytes(bits, M, K) <= kGiMaxSmem;
+}
+
+size_t ws_bytes_gemv_i8(int M, int K, int N)
+{
+    if (M < 1 || M > kGiMaxM || K < 1 || K > kI8MaxK)
+        return 0;
+    const size_t NR = 8 * gi_ntiles(M);
+    return ws_counter_bytes(N) + (size_t)kGiMaxCtas * kGiWarps * 2 * 16 * NR * 4;
+}
+
+template <int BITS, int NT>
+static cudaError_t launch_gi_t(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st)
+{
+    constexpr int NR = 8 * NT;
+    const int smem = (int)gi_smem_bytes(BITS, a.M, a.K);
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(gemv_i8_kernel<BITS, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kGiMaxSmem);
+        if (e != cudaSuccess)
+            return e;
+        attr_set = true;
+    }
+    static int occ_smem = -1, occ = 1; // occupancy of the last shared-memory size asked for
+    if (occ_smem != smem) {
+        int o = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, gemv_i8_kernel<BITS, NT>, kGiThreads, smem);
+        if (e != cudaSuccess)
+            return e;
+        occ = o > 0 ? o : 1;
+        occ_smem = smem;
+    }
+    const int per_sm = ctas_per_sm > 0 && ctas_per_sm < occ ? ctas_per_sm : occ;
+    const Shape sh{a.bits, a.K, a.N, a.group};
+    GiParams p;
+    p.x = a.x;
+    p.M = a.M;
+    p.K = a.K;
+    p.N = a.N;
+    p.KB = sh.kblocks();
+    p.I = (a.N / 16) * p.KB;
+    p.wq = (const uint8_t *)a.wq;
+    p.scales = (const uint16_t *)a.scales;
+    p.zeros = (const uint8_t *)a.zeros;
+    p.y = a.y;
+    p.cnt = (uint32_t *)ws;
+    p.part = (uint32_t *)((uint8_t *)ws + ws_counter_bytes(a.N));
+    int G = per_sm * sm_count;
+    if (G > kGiMaxCtas)
+        G = kGiMaxCtas;
+    const int want = (p.I + 4 * kGiWarps - 1) / (4 * kGiWarps); // at least ~4 items per warp
+    if (G > want)
+        G = want;
+    if (G < 1)
+        G = 1;
+    (void)NR;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.stream = st;
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(kGiThreads);
+    cfg.dynamicSmemBytes = smem;
+    return cudaLaunchKernelEx(&cfg, gemv_i8_kernel<BITS, NT>, p);
+}
+
+cudaError_t launch_gemv_i8(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st)
+{
+    const int nt = gi_ntiles(a.M);
+    if (a.bits == 8) {
+        switch (nt) {
+        case 1: return launch_gi_t<8, 1>(a, ctas_per_sm, ws, sm_count, st);
+        case 2: return launch_gi_t<8, 2>(a, ctas_per_sm, ws, sm_count, st);
+        default: return launch_gi_t<8, 3>(a, ctas_per_sm, ws, sm_count, st);
+        }
+    }
+    switch (nt) {
+    case 1: return launch_gi_t<4, 1>(a, ctas_per_sm, ws, sm_count, st);
+    case 2: return launch_gi_t<4, 2>(a, ctas_per_sm, ws, sm_count, st);
+    default: return launch_gi_t<4, 3>(a, ctas_per_sm, ws, sm_count, st);
+    }
+}
+
+} // namespace wq

@@ -121,6 +121,47 @@ __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar)
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Row maxima of x (bf16 magnitude bits, the order of magnitudes) by NTH
+// threads et = 0 .. NTH-1, BATCH 16-byte loads in flight per thread; each
+// thread's running maximum per row is folded into s_amax[m] (zeroed by the
+// caller) with a shared-memory atomicMax.  The caller synchronizes before reading s_amax.
+template <int NTH, int BATCH = 8>
+__device__ __forceinline__ void imma_row_maxima(const uint16_t *__restrict__ x, int M, int K, int et,
+                                                uint32_t *s_amax)
+{
+    const int vpr = K / 8; // 16-byte vectors per token row
+    const long long total = (long long)M * vpr;
+    int cur_m = -1;
+    uint32_t cur = 0;
+    for (long long v0 = et; v0 < total; v0 += BATCH * NTH) {
+        uint4 q[BATCH];
+#pragma unroll
+        for (int b = 0; b < BATCH; ++b) {
+            const long long v = v0 + (long long)b * NTH;
+            q[b] = v < total ? ldg_keep4(x + v * 8) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int b = 0; b < BATCH; ++b) {
+            const long long v = v0 + (long long)b * NTH;
+            if (v >= total)
+                break;
+            const int m = (int)(v / vpr);
+            if (m != cur_m) {
+                if (cur_m >= 0)
+                    atomicMax(&s_amax[cur_m], cur);
+                cur_m = m;
+                cur = 0;
+            }
+            const uint32_t wv[4] = {q[b].x, q[b].y, q[b].z, q[b].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+                cur = max(cur, max(wv[h] & 0x7FFFu, (wv[h] >> 16) & 0x7FFFu));
+        }
+    }
+    if (cur_m >= 0)
+        atomicMax(&s_amax[cur_m], cur);
+}
+
 // The digit phase, run by 128 threads (et = 0..127) of CTA c of G after the
 // programmatic-launch wait: the row maxima of x (every CTA computes all of
 // them, into s_amax / s_e), then CTA c's 1/G share of the digit blocks
@@ -160,38 +201,7 @@ __device__ __forceinline__ void imma_digit_phase(const uint16_t *__restrict__ x,
         first[j] = make_uint4(0, 0, 0, 0);
     if (i0 + et < i1)
         item_x(i0 + et, first);
-    const int vpr = K / 8; // 16-byte vectors per token row
-    const long long total = (long long)M * vpr;
-    int cur_m = -1;
-    uint32_t cur = 0;
-    constexpr int BATCH = 8;
-    for (long long v0 = et; v0 < total; v0 += BATCH * 128) {
-        uint4 q[BATCH];
-#pragma unroll
-        for (int b = 0; b < BATCH; ++b) {
-            const long long v = v0 + (long long)b * 128;
-            q[b] = v < total ? ldg_keep4(x + v * 8) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int b = 0; b < BATCH; ++b) {
-            const long long v = v0 + (long long)b * 128;
-            if (v >= total)
-                break;
-            const int m = (int)(v / vpr);
-            if (m != cur_m) {
-                if (cur_m >= 0)
-                    atomicMax(&s_amax[cur_m], cur);
-                cur_m = m;
-                cur = 0;
-            }
-            const uint32_t wv[4] = {q[b].x, q[b].y, q[b].z, q[b].w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h)
-                cur = max(cur, max(wv[h] & 0x7FFFu, (wv[h] >> 16) & 0x7FFFu));
-        }
-    }
-    if (cur_m >= 0)
-        atomicMax(&s_amax[cur_m], cur);
+    imma_row_maxima<128>(x, M, K, et, s_amax);
     named_barrier_sync(1, 128);
     if (et < M)
         s_e[et] = row_exponent(s_amax[et]);

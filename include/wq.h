@@ -95,8 +95,8 @@ typedef enum {
                                 W4A16 (M <= 32) on q - z; K <= 65536; needs the workspace */
 #define WQ_VARIANT_GEMV_I8 5 /* warp-level stream-K GEMV on mma.sync m16n8k32 s8 (the packed codes
                                 as they are, activations as exact digits in shared memory), M <= 8,
-                                3 * M * K bytes <= ~200 KB; split = CTAs per SM (1..3); needs the
-                                workspace */
+                                3 * M * K bytes <= ~200 KB; split 1 = one 16-warp CTA per SM, 2 = two
+                                8-warp CTAs per SM; needs the workspace */
 
 /* Static description of a status code. Host. Never NULL. */
 const char *wq_strerror(int status);
@@ -191,7 +191,7 @@ int wq_linear(const uint16_t *x, int M, int K, const void *Wq, const void *scale
  * GEMM_SK: split = CTAs per SM, 1 or 2, capped by the tile's resources.
  * GEMM: split = K-splits, 1 <= split <= min(32, ceil(K/128)).
  * I8MMA: split = 1 (one persistent CTA per SM).
- * GEMV_I8: split = CTAs per SM, 1..3, capped by occupancy.
+ * GEMV_I8: split = 1 (one 16-warp CTA per SM) or 2 (two 8-warp CTAs per SM).
  * Returns WQ_ERR_VARIANT if the pair does not fit the shape. */
 int wq_linear_forced(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
                      const void *zeros, int group, int N, uint16_t *y, int variant, int split,

@@ -107,7 +107,7 @@ def test_tuning_file_parse_errors(tmp_path):
         "NVIDIA B200|148 4 5120 17408 8 0 4 2 9.0\n",       # integer path: split 1 only
         "NVIDIA B200|148 9 5120 17408 8 0 5 1 9.0\n",       # integer GEMV: M <= 8
         "NVIDIA B200|148 8 65536 17408 8 0 5 1 9.0\n",      # integer GEMV: digit rows over 200 KB
-        "NVIDIA B200|148 4 5120 17408 4 128 5 4 9.0\n",     # integer GEMV: 1..3 CTAs per SM
+        "NVIDIA B200|148 4 5120 17408 4 128 5 3 9.0\n",     # integer GEMV: split 1 or 2
     ]:
         p = tmp_path / "bad.txt"
         p.write_text(bad_line)

@@ -57,7 +57,7 @@ def _cases(M, K, bits):
     if M <= (64 if bits == 8 else 32):  # integer tensor-core path: W8A16 M <= 64, W4A16 M <= 32
         out += [(I8, 1)]
     if M <= 8:  # integer GEMV
-        out += [(GI, c) for c in (1, 2, 3)]
+        out += [(GI, c) for c in (1, 2)]
     return out
 
 
@@ -89,7 +89,7 @@ def test_repeated_dispatch_resets_tickets(weight, ws):
     bits, K, N, pw, canon = weight
     runs = [(GEMM, 16, 2), (GEMM, 16, 8), (GEMM_SK, 40, 2), (GEMV, 5, 3), (GEMM, 40, 4), (GEMM, 128, 9),
             (I8, 5, 1), (I8, 40 if bits == 8 else 30, 1), (GEMV, 3, 2), (I8, 1, 1), (GI, 1, 2), (GI, 8, 1),
-            (GEMM_SK, 7, 1), (GI, 4, 3), (I8, 3, 1), (GI, 6, 2)]
+            (GEMM_SK, 7, 1), (GI, 4, 1), (I8, 3, 1), (GI, 6, 2)]
     runs += [(GEMM, 16, 2)]
     for variant, M, split in runs:
         x = gen.x_bf16(M, K)
@@ -276,7 +276,7 @@ def test_argument_errors(weight, ws):
     assert wq.wq_linear_status(x, pw, y, GEMM, 33) == -11         # split above 32
     assert wq.wq_linear_status(x, pw, y, 7, 1) == -11             # unknown variant
     assert wq.wq_linear_status(x, pw, y, I8, 2) == -11            # one CTA per SM only
-    assert wq.wq_linear_status(x, pw, y, GI, 4) == -11            # integer GEMV: 1..3 CTAs per SM
+    assert wq.wq_linear_status(x, pw, y, GI, 3) == -11            # integer GEMV: split 1 or 2
     assert wq.wq_linear_status(x, pw, y, GI, 0) == 0              # 0: the default
     xc = bf16_dev(gen.x_bf16(65, K))
     yc = torch.empty((65, N), dtype=torch.bfloat16, device=dev())

@@ -122,7 +122,7 @@ bool choice_valid(int variant, int split, int M, int K, int bits)
     if (variant == WQ_VARIANT_I8MMA)
         return i8_fits(bits, M, K) && split == 1;
     if (variant == WQ_VARIANT_GEMV_I8)
-        return gi_fits(bits, M, K) && split >= 1 && split <= 3;
+        return gi_fits(bits, M, K) && (split == 1 || split == 2);
     if (variant == WQ_VARIANT_GEMV)
         return M <= 32 && split >= 1 && split <= 4;
     if (variant == WQ_VARIANT_GEMV_RB)
@@ -228,7 +228,7 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
                       : variant == WQ_VARIANT_GEMV_RB ? default_rb_slices(K, N, d.sm_count)
                       : variant == WQ_VARIANT_GEMM_SK ? 2
                       : variant == WQ_VARIANT_I8MMA   ? 1
-                      : variant == WQ_VARIANT_GEMV_I8 ? 2
+                      : variant == WQ_VARIANT_GEMV_I8 ? 1
                                                       : std::min(8, max_gemm_split(K));
     }
     if (split > 0)

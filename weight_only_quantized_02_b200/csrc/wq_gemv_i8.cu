@@ -42,18 +42,19 @@
 
 namespace wq {
 
-constexpr int kGiWarps = 8;
-constexpr int kGiThreads = 32 * kGiWarps;
+// Warps of the stream-K partition (every launch shape): at most kGiMaxCtas * 8.
+constexpr int kGiMaxWarps = kGiMaxCtas * 8;
 
 struct GiParams {
     const uint16_t *x;
     int M, K, N, KB;
-    int I;          // items = (N / 16) * KB
+    int CPR;        // chunks (D consecutive k-blocks, the last one ragged) per 16-row block
+    int I;          // chunks = (N / 16) * CPR
     const uint8_t *wq;
     const uint16_t *scales;
     const uint8_t *zeros;
     uint16_t *y;
-    uint32_t *part; // [G * 8 warps][2 slots][16 rows][NR] partials
+    uint32_t *part; // [kGiMaxWarps][2 slots][16 rows][NR] partials
     uint32_t *cnt;  // one ticket per 16-row block
 };
 
@@ -83,7 +84,7 @@ __host__ __device__ constexpr int gi_row_stride(int K)
 }
 
 // The activations of the whole layer as digit rows in shared memory (all
-// 256 threads): the row maxima (e_m), then every 16-k chunk of every token
+// NTH threads of the CTA): the row maxima (e_m), then every 16-k chunk of every token
 // row, thread ch = chunk % 8 of each group of eight converting k = 16 c ..
 // 16 c + 15 (zero past K).  Each CTA converts all of x (M*K values, a few
 // tens per thread at decode sizes) and no CTA waits for another.  Digit row
@@ -94,21 +95,21 @@ __host__ __device__ constexpr int gi_row_stride(int K)
 //         packed mma tile gives lane t of 32-k step st the nibbles of
 //         k = 4t + a (low nibbles) and 16 + 4t + a (high nibbles) interleaved,
 //         so a lane's 32 bytes of a block are its four steps' B fragments.
-template <int BITS, int NR>
+template <int BITS, int NR, int NTH>
 __device__ __forceinline__ void gi_digits(const GiParams &p, uint8_t *sd, int32_t *s_dsum, uint32_t *s_amax,
                                           int *s_e)
 {
     const int et = threadIdx.x, ch = et & 7;
     const int M = p.M, K = p.K, KB = p.KB;
     const int S = gi_row_stride<BITS>(K);
-    imma_row_maxima<kGiThreads, 2>(p.x, M, K, et, s_amax); // few registers: the weight prefetch is live
+    imma_row_maxima<NTH, 2>(p.x, M, K, et, s_amax); // few registers: the weight prefetch is live
     __syncthreads();
     if (et < M)
         s_e[et] = row_exponent(s_amax[et]);
     __syncthreads();
     const int cpr = KB * 8; // 16-k chunks per token row
     const int items = M * cpr;
-    for (int base = 0; base < items; base += kGiThreads) { // uniform trip count: shuffles below
+    for (int base = 0; base < items; base += NTH) { // uniform trip count: shuffles below
         const int it = base + et;
         const bool act = it < items;
         const int m = act ? it / cpr : 0, c = act ? it % cpr : 0; // chunk c: k = 16c .. 16c + 15
@@ -184,7 +185,7 @@ template <int BITS, int NR>
 __device__ __forceinline__ void gi_flush(const GiParams &p, int rb, bool whole, int slot, int w, int Wt,
                                       uint32_t *red, const int *s_e, int lane)
 {
-    const int M = p.M, N = p.N, KB = p.KB;
+    const int M = p.M, N = p.N;
     const int n0 = 16 * rb;
     __syncwarp();
     if constexpr (BITS == 8) {
@@ -222,7 +223,8 @@ __device__ __forceinline__ void gi_flush(const GiParams &p, int rb, bool whole, 
     if (lane == 0)
         ticket = ticket_take_acq_rel(&p.cnt[rb]);
     ticket = __shfl_sync(0xffffffffu, ticket, 0);
-    const int wf = sk_owner(p.I, Wt, rb * KB), wl = sk_owner(p.I, Wt, rb * KB + KB - 1);
+    const int CPR = p.CPR;
+    const int wf = sk_owner(p.I, Wt, rb * CPR), wl = sk_owner(p.I, Wt, rb * CPR + CPR - 1);
     if (ticket == (uint32_t)(wl - wf)) {
         __syncwarp(); // lane 0's acquire orders every lane's reads below
         for (int q = lane; q < 16 * M; q += 32) {
@@ -230,7 +232,7 @@ __device__ __forceinline__ void gi_flush(const GiParams &p, int rb, bool whole, 
             if constexpr (BITS == 8) {
                 int32_t t0 = 0, t1 = 0, t2 = 0;
                 for (int ww = wf; ww <= wl; ++ww) {
-                    const int sl = (sk_start(p.I, Wt, ww) / KB == rb) ? 0 : 1;
+                    const int sl = (sk_start(p.I, Wt, ww) / CPR == rb) ? 0 : 1;
                     const int32_t *src =
                         reinterpret_cast<const int32_t *>(p.part) + ((size_t)ww * 2 + sl) * 16 * NR + r * NR + 3 * m;
                     t0 += __ldcg(src);
@@ -242,7 +244,7 @@ __device__ __forceinline__ void gi_flush(const GiParams &p, int rb, bool whole, 
             } else {
                 float tot = 0.f;
                 for (int ww = wf; ww <= wl; ++ww) {
-                    const int sl = (sk_start(p.I, Wt, ww) / KB == rb) ? 0 : 1;
+                    const int sl = (sk_start(p.I, Wt, ww) / CPR == rb) ? 0 : 1;
                     tot += __ldcg(reinterpret_cast<const float *>(p.part) + ((size_t)ww * 2 + sl) * 16 * NR + r * NR + m);
                 }
                 p.y[(size_t)m * N + n0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(tot));
@@ -254,8 +256,10 @@ __device__ __forceinline__ void gi_flush(const GiParams &p, int rb, bool whole, 
     __syncwarp();
 }
 
-template <int BITS, int NT>
-__global__ void __launch_bounds__(kGiThreads) gemv_i8_kernel(const GiParams p)
+// WARPS = 16: one CTA per SM (the digit rows made once per SM); WARPS = 8:
+// two per SM.  Either way 128 registers per thread and 16 warps per SM.
+template <int BITS, int NT, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const GiParams p)
 {
     constexpr int NR = 8 * NT;
     constexpr int D = GiCfg<BITS>::D;
@@ -263,49 +267,78 @@ __global__ void __launch_bounds__(kGiThreads) gemv_i8_kernel(const GiParams p)
     extern __shared__ __align__(16) uint8_t sd[]; // digit rows [3M][S], then (INT4) digit sums [KB][NR]
     __shared__ uint32_t s_amax[kGiMaxM];
     __shared__ int s_e[kGiMaxM];
-    __shared__ uint32_t s_red[kGiWarps][16 * NR];
+    __shared__ uint32_t s_red[WARPS][16 * NR];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int G = gridDim.x, c = blockIdx.x;
-    const int Wt = G * kGiWarps, w = c * kGiWarps + warp;
+    const int Wt = G * WARPS, w = c * WARPS + warp;
     const int KB = p.KB, M = p.M;
     const int S = gi_row_stride<BITS>(p.K);
     int32_t *s_dsum = reinterpret_cast<int32_t *>(sd + 3 * M * S);
     const int i0 = sk_start(p.I, Wt, w), i1 = sk_start(p.I, Wt, w + 1);
     const int n = i1 - i0;
 
-    // ---------------- weights of the first D items (before the launch wait) ----------------
+    // ---------------- weights of the first chunk (before the launch wait) ----------------
+    // The warp's work is chunks [i0, i1): chunk (rb, q) = k-blocks D q ..
+    // D q + D - 1 (those below KB) of 16-row block rb.  Ring slot s holds
+    // k-block D q + s of a chunk: consuming a slot is followed by loading
+    // the same slot of the next chunk, so D k-blocks stay in flight.
+    // Loader state: the next chunk to load is (lrb, lq); lw points at its
+    // first k-block (INT8: the 16-row block's 2 KB; INT4: this lane's 16
+    // bytes of the first tile), ls / lz at its INT4 scales and zero points.
+    // Consecutive k-blocks of one 16-row block are 16 KB (INT8) / 8 KB
+    // (INT4) apart.
+    constexpr int kWStep = BITS == 8 ? 16384 : 8192;
+    const int CPR = p.CPR;
     uint4 wb[D][WV];
     uint32_t sz[D][2]; // INT4: bf16 scales of rows g, g+8 | their zero-point bytes
-    auto load_item = [&](int rb, int kb, uint4 (&v)[WV], uint32_t (&e)[2]) {
-        const int blk = (rb >> 3) * KB + kb, j = rb & 7;
+    const int oa = (g << 7) + ((t ^ g) << 4), ob = (g << 7) + (((t + 4) ^ g) << 4); // INT8 chunks t, t+4
+    int lrb = n > 0 ? i0 / CPR : 0, lq = n > 0 ? i0 % CPR : 0;
+    const uint8_t *lw = nullptr;
+    const uint16_t *ls = nullptr;
+    const uint8_t *lz = nullptr;
+    auto seek = [&]() { // pointers of chunk (lrb, lq)
+        const size_t blk = (size_t)(lrb >> 3) * KB + D * lq;
+        const int j = lrb & 7;
         if constexpr (BITS == 8) {
-            const uint8_t *b = p.wq + ((size_t)blk << 14) + (j << 11) + (g << 7);
-            v[0] = ldg_stream(b + ((t ^ g) << 4));              // row g,     chunk t
-            v[1] = ldg_stream(b + 1024 + ((t ^ g) << 4));       // row g + 8, chunk t
-            v[2] = ldg_stream(b + (((t + 4) ^ g) << 4));        // row g,     chunk t + 4
-            v[3] = ldg_stream(b + 1024 + (((t + 4) ^ g) << 4)); // row g + 8, chunk t + 4
+            lw = p.wq + (blk << 14) + (j << 11);
         } else {
-            const uint8_t *b = p.wq + (((size_t)blk * 8 + j) << 10) + 16 * lane;
+            lw = p.wq + ((blk * 8 + j) << 10) + 16 * lane;
+            ls = p.scales + blk * kPanelRows + 16 * j + g;
+            lz = p.zeros + blk * 64 + 8 * j + (g >> 1);
+        }
+    };
+    auto load_slot = [&](int s, uint4 (&v)[WV], uint32_t (&e)[2]) {
+        const uint8_t *b = lw + s * kWStep;
+        if constexpr (BITS == 8) {
+            v[0] = ldg_stream(b + oa);        // row g,     chunk t
+            v[1] = ldg_stream(b + 1024 + oa); // row g + 8, chunk t
+            v[2] = ldg_stream(b + ob);        // row g,     chunk t + 4
+            v[3] = ldg_stream(b + 1024 + ob); // row g + 8, chunk t + 4
+        } else {
             v[0] = ldg_stream(b);
             v[1] = ldg_stream(b + 512);
-            const uint16_t *sp = p.scales + (size_t)blk * kPanelRows + 16 * j + g;
+            const uint16_t *sp = ls + s * kPanelRows;
+            const uint8_t *zp = lz + s * 64;
             e[0] = (uint32_t)__ldg(sp) | ((uint32_t)__ldg(sp + 8) << 16);
-            const uint8_t *zp = p.zeros + (size_t)blk * 64 + 8 * j + (g >> 1);
             e[1] = (uint32_t)__ldg(zp) | ((uint32_t)__ldg(zp + 4) << 8);
         }
     };
-    int lrb = n > 0 ? i0 / KB : 0, lkb = n > 0 ? i0 % KB : 0; // next item to load
-    const int rb_first = lrb;
-#pragma unroll
-    for (int s = 0; s < D; ++s) {
-        if (s < n) {
-            load_item(lrb, lkb, wb[s], sz[s]);
-            if (++lkb == KB) {
-                lkb = 0;
-                ++lrb;
-            }
+    auto next_chunk = [&]() {
+        if (++lq == CPR) {
+            lq = 0;
+            ++lrb;
         }
+        seek();
+    };
+    seek();
+    const int rb_first = lrb;
+    if (n > 0) {
+#pragma unroll
+        for (int s = 0; s < D; ++s)
+            if (D * lq + s < KB)
+                load_slot(s, wb[s], sz[s]);
+        next_chunk();
     }
 
     // ---------------- activations: this CTA's digit rows ----------------
@@ -313,9 +346,9 @@ __global__ void __launch_bounds__(kGiThreads) gemv_i8_kernel(const GiParams p)
         s_amax[threadIdx.x] = 0u;
     __syncthreads();
     pdl_wait(); // x, y and the workspace may come from / be in use by the preceding kernel
-    gi_digits<BITS, NR>(p, sd, s_dsum, s_amax, s_e);
+    gi_digits<BITS, NR, WARPS * 32>(p, sd, s_dsum, s_amax, s_e);
 
-    // ---------------- stream the warp's items ----------------
+    // ---------------- stream the warp's chunks ----------------
     int32_t acc_i[NT][4];
     float acc_f[NT][4];
 #pragma unroll
@@ -325,109 +358,124 @@ __global__ void __launch_bounds__(kGiThreads) gemv_i8_kernel(const GiParams p)
             acc_i[nt][r] = 0;
             acc_f[nt][r] = 0.f;
         }
-    int crb = rb_first, ckb = n > 0 ? i0 % KB : 0, seg_kb0 = ckb;
+    // this lane's digit rows: INT8 bytes 16t and 16(t+4) of a block, INT4 bytes 32t .. 32t+31
+    const uint8_t *xrow[NT];
+    bool xon[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        xon[nt] = 8 * nt + g < 3 * M;
+        xrow[nt] = sd + (xon[nt] ? (8 * nt + g) * S : 0) + (BITS == 8 ? 16 * t : 32 * t);
+    }
     const int zsh = 4 * (g & 1);
     uint32_t *red = s_red[warp];
-    for (int j0 = 0; j0 < n; j0 += D) {
+
+    // k-block xo (byte offset 128 * kb in a digit row) of ring slot s
+    auto consume = [&](int s, int xo) {
+        if constexpr (BITS == 8) {
 #pragma unroll
-        for (int s = 0; s < D; ++s) {
-            const int jj = j0 + s;
-            if (jj < n) {
-                const uint8_t *xb = sd + ckb * 128;
+            for (int nt = 0; nt < NT; ++nt) {
+                uint4 d0 = make_uint4(0, 0, 0, 0), d1 = d0;
+                if (xon[nt]) {
+                    d0 = *reinterpret_cast<const uint4 *>(xrow[nt] + xo);
+                    d1 = *reinterpret_cast<const uint4 *>(xrow[nt] + xo + 64);
+                }
+                const uint4 *v = wb[s];
+                imma_16832(acc_i[nt], v[0].x, v[1].x, v[0].y, v[1].y, d0.x, d0.y);
+                imma_16832(acc_i[nt], v[0].z, v[1].z, v[0].w, v[1].w, d0.z, d0.w);
+                imma_16832(acc_i[nt], v[2].x, v[3].x, v[2].y, v[3].y, d1.x, d1.y);
+                imma_16832(acc_i[nt], v[2].z, v[3].z, v[2].w, v[3].w, d1.z, d1.w);
+            }
+        } else {
+            constexpr uint32_t lo4 = 0x0F0F0F0Fu;
+            uint32_t a[2][8]; // per tile: lo/hi of words x, y, z, w
+#pragma unroll
+            for (int tau = 0; tau < 2; ++tau) {
+                const uint4 &v = wb[s][tau];
+                a[tau][0] = v.x & lo4;
+                a[tau][1] = (v.x >> 4) & lo4;
+                a[tau][2] = v.y & lo4;
+                a[tau][3] = (v.y >> 4) & lo4;
+                a[tau][4] = v.z & lo4;
+                a[tau][5] = (v.z >> 4) & lo4;
+                a[tau][6] = v.w & lo4;
+                a[tau][7] = (v.w >> 4) & lo4;
+            }
+            const float s_lo = __uint_as_float(sz[s][0] << 16), s_hi = __uint_as_float(sz[s][0] & 0xFFFF0000u);
+            const int z_lo = (int)((sz[s][1] >> zsh) & 0xFu), z_hi = (int)((sz[s][1] >> (8 + zsh)) & 0xFu);
+            const int32_t *dsum = s_dsum + (xo >> 7) * NR + 2 * t;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                uint4 d0 = make_uint4(0, 0, 0, 0), d1 = d0;
+                if (xon[nt]) {
+                    d0 = *reinterpret_cast<const uint4 *>(xrow[nt] + xo);
+                    d1 = *reinterpret_cast<const uint4 *>(xrow[nt] + xo + 16);
+                }
+                int32_t ci[4] = {0, 0, 0, 0};
+                imma_16832(ci, a[0][0], a[0][2], a[0][1], a[0][3], d0.x, d0.y);
+                imma_16832(ci, a[0][4], a[0][6], a[0][5], a[0][7], d0.z, d0.w);
+                imma_16832(ci, a[1][0], a[1][2], a[1][1], a[1][3], d1.x, d1.y);
+                imma_16832(ci, a[1][4], a[1][6], a[1][5], a[1][7], d1.z, d1.w);
+                int2 ds = make_int2(0, 0);
+                if (8 * nt + 2 * t < 3 * M)
+                    ds = *reinterpret_cast<const int2 *>(dsum + 8 * nt);
+                acc_f[nt][0] = fmaf(s_lo, (float)(ci[0] - z_lo * ds.x), acc_f[nt][0]);
+                acc_f[nt][1] = fmaf(s_lo, (float)(ci[1] - z_lo * ds.y), acc_f[nt][1]);
+                acc_f[nt][2] = fmaf(s_hi, (float)(ci[2] - z_hi * ds.x), acc_f[nt][2]);
+                acc_f[nt][3] = fmaf(s_hi, (float)(ci[3] - z_hi * ds.y), acc_f[nt][3]);
+            }
+        }
+    };
+
+    int crb = rb_first, cq = n > 0 ? i0 % CPR : 0;
+    bool seg_whole = cq == 0; // the current segment started at the row block's first chunk
+    for (int ch = 0; ch < n; ++ch) {
+        const int kb0 = D * cq, xo = kb0 * 128;
+        const bool more = ch + 1 < n; // the loader points at chunk ch + 1
+        if (kb0 + D <= KB && more && D * lq + D <= KB) {
+#pragma unroll
+            for (int s = 0; s < D; ++s) { // common case: one straight block
+                consume(s, xo + 128 * s);
+                load_slot(s, wb[s], sz[s]);
+            }
+        } else {
+#pragma unroll
+            for (int s = 0; s < D; ++s) {
+                if (kb0 + s < KB)
+                    consume(s, xo + 128 * s);
+                if (more && D * lq + s < KB)
+                    load_slot(s, wb[s], sz[s]);
+            }
+        }
+        if (more)
+            next_chunk();
+        if (cq == CPR - 1 || !more) { // end of a segment: the row block's last chunk or the warp's last
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int col = 8 * nt + 2 * t;
                 if constexpr (BITS == 8) {
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const int row = 8 * nt + g;
-                        uint4 d0 = make_uint4(0, 0, 0, 0), d1 = d0;
-                        if (row < 3 * M) {
-                            d0 = *reinterpret_cast<const uint4 *>(xb + row * S + 16 * t);
-                            d1 = *reinterpret_cast<const uint4 *>(xb + row * S + 16 * (t + 4));
-                        }
-                        const uint4 *v = wb[s];
-                        imma_16832(acc_i[nt], v[0].x, v[1].x, v[0].y, v[1].y, d0.x, d0.y);
-                        imma_16832(acc_i[nt], v[0].z, v[1].z, v[0].w, v[1].w, d0.z, d0.w);
-                        imma_16832(acc_i[nt], v[2].x, v[3].x, v[2].y, v[3].y, d1.x, d1.y);
-                        imma_16832(acc_i[nt], v[2].z, v[3].z, v[2].w, v[3].w, d1.z, d1.w);
-                    }
+                    red[g * NR + col] = (uint32_t)acc_i[nt][0];
+                    red[g * NR + col + 1] = (uint32_t)acc_i[nt][1];
+                    red[(g + 8) * NR + col] = (uint32_t)acc_i[nt][2];
+                    red[(g + 8) * NR + col + 1] = (uint32_t)acc_i[nt][3];
                 } else {
-                    constexpr uint32_t lo4 = 0x0F0F0F0Fu;
-                    uint32_t a[2][8]; // per tile: lo/hi of words x, y, z, w
-#pragma unroll
-                    for (int tau = 0; tau < 2; ++tau) {
-                        const uint4 &v = wb[s][tau];
-                        a[tau][0] = v.x & lo4;
-                        a[tau][1] = (v.x >> 4) & lo4;
-                        a[tau][2] = v.y & lo4;
-                        a[tau][3] = (v.y >> 4) & lo4;
-                        a[tau][4] = v.z & lo4;
-                        a[tau][5] = (v.z >> 4) & lo4;
-                        a[tau][6] = v.w & lo4;
-                        a[tau][7] = (v.w >> 4) & lo4;
-                    }
-                    const float s_lo = __uint_as_float(sz[s][0] << 16), s_hi = __uint_as_float(sz[s][0] & 0xFFFF0000u);
-                    const int z_lo = (int)((sz[s][1] >> zsh) & 0xFu), z_hi = (int)((sz[s][1] >> (8 + zsh)) & 0xFu);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const int row = 8 * nt + g;
-                        uint4 d0 = make_uint4(0, 0, 0, 0), d1 = d0;
-                        if (row < 3 * M) {
-                            d0 = *reinterpret_cast<const uint4 *>(xb + row * S + 32 * t);
-                            d1 = *reinterpret_cast<const uint4 *>(xb + row * S + 32 * t + 16);
-                        }
-                        int32_t ci[4] = {0, 0, 0, 0};
-                        imma_16832(ci, a[0][0], a[0][2], a[0][1], a[0][3], d0.x, d0.y);
-                        imma_16832(ci, a[0][4], a[0][6], a[0][5], a[0][7], d0.z, d0.w);
-                        imma_16832(ci, a[1][0], a[1][2], a[1][1], a[1][3], d1.x, d1.y);
-                        imma_16832(ci, a[1][4], a[1][6], a[1][5], a[1][7], d1.z, d1.w);
-                        const int col = 8 * nt + 2 * t;
-                        int2 ds = make_int2(0, 0);
-                        if (col < 3 * M)
-                            ds = *reinterpret_cast<const int2 *>(s_dsum + ckb * NR + col);
-                        acc_f[nt][0] = fmaf(s_lo, (float)(ci[0] - z_lo * ds.x), acc_f[nt][0]);
-                        acc_f[nt][1] = fmaf(s_lo, (float)(ci[1] - z_lo * ds.y), acc_f[nt][1]);
-                        acc_f[nt][2] = fmaf(s_hi, (float)(ci[2] - z_hi * ds.x), acc_f[nt][2]);
-                        acc_f[nt][3] = fmaf(s_hi, (float)(ci[3] - z_hi * ds.y), acc_f[nt][3]);
-                    }
+                    red[g * NR + col] = __float_as_uint(acc_f[nt][0]);
+                    red[g * NR + col + 1] = __float_as_uint(acc_f[nt][1]);
+                    red[(g + 8) * NR + col] = __float_as_uint(acc_f[nt][2]);
+                    red[(g + 8) * NR + col + 1] = __float_as_uint(acc_f[nt][3]);
                 }
-                // refill this slot with item jj + D
-                if (jj + D < n) {
-                    load_item(lrb, lkb, wb[s], sz[s]);
-                    if (++lkb == KB) {
-                        lkb = 0;
-                        ++lrb;
-                    }
-                }
-                // end of a segment: the row block's last k-block or the warp's last item
-                if (ckb == KB - 1 || jj == n - 1) {
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const int col = 8 * nt + 2 * t;
-                        if constexpr (BITS == 8) {
-                            red[g * NR + col] = (uint32_t)acc_i[nt][0];
-                            red[g * NR + col + 1] = (uint32_t)acc_i[nt][1];
-                            red[(g + 8) * NR + col] = (uint32_t)acc_i[nt][2];
-                            red[(g + 8) * NR + col + 1] = (uint32_t)acc_i[nt][3];
-                        } else {
-                            red[g * NR + col] = __float_as_uint(acc_f[nt][0]);
-                            red[g * NR + col + 1] = __float_as_uint(acc_f[nt][1]);
-                            red[(g + 8) * NR + col] = __float_as_uint(acc_f[nt][2]);
-                            red[(g + 8) * NR + col + 1] = __float_as_uint(acc_f[nt][3]);
-                        }
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            acc_i[nt][r] = 0;
-                            acc_f[nt][r] = 0.f;
-                        }
-                    }
-                    const bool whole = seg_kb0 == 0 && ckb == KB - 1;
-                    gi_flush<BITS, NR>(p, crb, whole, crb == rb_first ? 0 : 1, w, Wt, red, s_e, lane);
-                    seg_kb0 = 0;
-                }
-                if (++ckb == KB) {
-                    ckb = 0;
-                    ++crb;
+                for (int r = 0; r < 4; ++r) {
+                    acc_i[nt][r] = 0;
+                    acc_f[nt][r] = 0.f;
                 }
             }
+            const bool whole = seg_whole && cq == CPR - 1;
+            gi_flush<BITS, NR>(p, crb, whole, crb == rb_first ? 0 : 1, w, Wt, red, s_e, lane);
+            ++crb;
+            cq = 0;
+            seg_whole = true;
+        } else {
+            ++cq;
         }
     }
     pdl_launch_dependents();
@@ -455,18 +503,17 @@ size_t ws_bytes_gemv_i8(int M, int K, int N)
     if (M < 1 || M > kGiMaxM || K < 1 || K > kI8MaxK)
         return 0;
     const size_t NR = 8 * gi_ntiles(M);
-    return ws_counter_bytes(N) + (size_t)kGiMaxCtas * kGiWarps * 2 * 16 * NR * 4;
+    return ws_counter_bytes(N) + (size_t)kGiMaxWarps * 2 * 16 * NR * 4;
 }
 
-template <int BITS, int NT>
-static cudaError_t launch_gi_t(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st)
+template <int BITS, int NT, int WARPS>
+static cudaError_t launch_gi_t(const LinearArgs &a, void *ws, int sm_count, cudaStream_t st)
 {
-    constexpr int NR = 8 * NT;
     const int smem = (int)gi_smem_bytes(BITS, a.M, a.K);
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_i8_kernel<BITS, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kGiMaxSmem);
+        cudaError_t e = cudaFuncSetAttribute(gemv_i8_kernel<BITS, NT, WARPS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kGiMaxSmem);
         if (e != cudaSuccess)
             return e;
         attr_set = true;
@@ -474,13 +521,14 @@ static cudaError_t launch_gi_t(const LinearArgs &a, int ctas_per_sm, void *ws, i
     static int occ_smem = -1, occ = 1; // occupancy of the last shared-memory size asked for
     if (occ_smem != smem) {
         int o = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, gemv_i8_kernel<BITS, NT>, kGiThreads, smem);
+        cudaError_t e =
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, gemv_i8_kernel<BITS, NT, WARPS>, WARPS * 32, smem);
         if (e != cudaSuccess)
             return e;
         occ = o > 0 ? o : 1;
         occ_smem = smem;
     }
-    const int per_sm = ctas_per_sm > 0 && ctas_per_sm < occ ? ctas_per_sm : occ;
+    const int per_sm = occ < 16 / WARPS ? occ : 16 / WARPS;
     const Shape sh{a.bits, a.K, a.N, a.group};
     GiParams p;
     p.x = a.x;
@@ -488,7 +536,8 @@ static cudaError_t launch_gi_t(const LinearArgs &a, int ctas_per_sm, void *ws, i
     p.K = a.K;
     p.N = a.N;
     p.KB = sh.kblocks();
-    p.I = (a.N / 16) * p.KB;
+    p.CPR = (p.KB + GiCfg<BITS>::D - 1) / GiCfg<BITS>::D;
+    p.I = (a.N / 16) * p.CPR;
     p.wq = (const uint8_t *)a.wq;
     p.scales = (const uint16_t *)a.scales;
     p.zeros = (const uint8_t *)a.zeros;
@@ -496,14 +545,13 @@ static cudaError_t launch_gi_t(const LinearArgs &a, int ctas_per_sm, void *ws, i
     p.cnt = (uint32_t *)ws;
     p.part = (uint32_t *)((uint8_t *)ws + ws_counter_bytes(a.N));
     int G = per_sm * sm_count;
-    if (G > kGiMaxCtas)
-        G = kGiMaxCtas;
-    const int want = (p.I + 4 * kGiWarps - 1) / (4 * kGiWarps); // at least ~4 items per warp
+    if (G * WARPS > kGiMaxWarps)
+        G = kGiMaxWarps / WARPS;
+    const int want = (p.I + 2 * WARPS - 1) / (2 * WARPS); // at least ~2 chunks per warp
     if (G > want)
         G = want;
     if (G < 1)
         G = 1;
-    (void)NR;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -512,25 +560,31 @@ static cudaError_t launch_gi_t(const LinearArgs &a, int ctas_per_sm, void *ws, i
     cfg.numAttrs = 1;
     cfg.stream = st;
     cfg.gridDim = dim3(G);
-    cfg.blockDim = dim3(kGiThreads);
+    cfg.blockDim = dim3(WARPS * 32);
     cfg.dynamicSmemBytes = smem;
-    return cudaLaunchKernelEx(&cfg, gemv_i8_kernel<BITS, NT>, p);
+    return cudaLaunchKernelEx(&cfg, gemv_i8_kernel<BITS, NT, WARPS>, p);
 }
 
-cudaError_t launch_gemv_i8(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st)
+template <int BITS, int NT>
+static cudaError_t launch_gi_w(const LinearArgs &a, int split, void *ws, int sm_count, cudaStream_t st)
+{
+    return split == 2 ? launch_gi_t<BITS, NT, 8>(a, ws, sm_count, st) : launch_gi_t<BITS, NT, 16>(a, ws, sm_count, st);
+}
+
+cudaError_t launch_gemv_i8(const LinearArgs &a, int split, void *ws, int sm_count, cudaStream_t st)
 {
     const int nt = gi_ntiles(a.M);
     if (a.bits == 8) {
         switch (nt) {
-        case 1: return launch_gi_t<8, 1>(a, ctas_per_sm, ws, sm_count, st);
-        case 2: return launch_gi_t<8, 2>(a, ctas_per_sm, ws, sm_count, st);
-        default: return launch_gi_t<8, 3>(a, ctas_per_sm, ws, sm_count, st);
+        case 1: return launch_gi_w<8, 1>(a, split, ws, sm_count, st);
+        case 2: return launch_gi_w<8, 2>(a, split, ws, sm_count, st);
+        default: return launch_gi_w<8, 3>(a, split, ws, sm_count, st);
         }
     }
     switch (nt) {
-    case 1: return launch_gi_t<4, 1>(a, ctas_per_sm, ws, sm_count, st);
-    case 2: return launch_gi_t<4, 2>(a, ctas_per_sm, ws, sm_count, st);
-    default: return launch_gi_t<4, 3>(a, ctas_per_sm, ws, sm_count, st);
+    case 1: return launch_gi_w<4, 1>(a, split, ws, sm_count, st);
+    case 2: return launch_gi_w<4, 2>(a, split, ws, sm_count, st);
+    default: return launch_gi_w<4, 3>(a, split, ws, sm_count, st);
     }
 }
 

@@ -94,9 +94,9 @@ cudaError_t read_gemm_i4_error(int *code, cudaStream_t st);
 
 // Integer GEMV (mma.sync m16n8k32 on the packed codes): M <= kGiMaxM,
 // K <= kI8MaxK, the CTA's digit rows (gi_smem_bytes) at most kGiMaxSmem of
-// shared memory; at most kGiMaxCtas CTAs of 8 warps.  Workspace:
-// [counters][partials kGiMaxCtas x 8 x 2 x 16 x NR x 4 bytes],
-// NR = 8 * gi_ntiles(M).
+// shared memory; split 1 = one 16-warp CTA per SM, 2 = two 8-warp CTAs;
+// at most kGiMaxCtas * 8 warps.  Workspace: [counters][partials
+// kGiMaxCtas x 8 x 2 x 16 x NR x 4 bytes], NR = 8 * gi_ntiles(M).
 constexpr int kGiMaxM = 8;
 constexpr int kGiMaxCtas = 448;
 constexpr int kGiMaxSmem = 200 * 1024;
@@ -104,7 +104,7 @@ int gi_ntiles(int M);
 size_t gi_smem_bytes(int bits, int M, int K);
 bool gi_fits(int bits, int M, int K);
 size_t ws_bytes_gemv_i8(int M, int K, int N);
-cudaError_t launch_gemv_i8(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st);
+cudaError_t launch_gemv_i8(const LinearArgs &a, int split, void *ws, int sm_count, cudaStream_t st);
 
 // Reads and clears the device error word of the current device.
 cudaError_t read_device_error(int *code, cudaStream_t st);

@@ -11,10 +11,11 @@ scales + zeros + activations in + outputs out, each counted once) per second
 Default workload: the W8A16 decode GEMV, K = 5120, N = 17408, M in {1, 2, 4}.
 One step = one wq_linear call per M on every one of R packed-weight copies,
 R chosen so the copies span more than 5x the L2 size.  Every call therefore
-streams its weights from HBM (rotation instead of an L2 flush).  Each call
-is captured once in its own CUDA graph and replayed; CUDA events recorded on
-the launching stream between the graph launches bracket every kernel, so
-per-kernel durations come from the timed region itself.
+streams its weights from HBM (rotation instead of an L2 flush).  The calls
+of one M are captured once as a CUDA graph, back to back (as the layers of a
+decode step run); a step replays the graphs of every M with CUDA events
+recorded between them on the launching stream, so each M's average launch
+duration comes from the timed region itself.
 
 With --gpus N > 1 (launched by torchrun) every rank runs the same workload
 on its own GPU: the layer needs no exchange step, so this is weak scaling
@@ -215,6 +216,18 @@ def profile_traffic(src_file: str, summary_name: str, M: int):
 # our arm
 # ---------------------------------------------------------------------------
 
+def tuned_shapes(path):
+    """(M, K, N, bits, group) of every entry of a dispatcher table file."""
+    out = set()
+    for line in open(path):
+        if line.startswith("#") or "|" not in line:
+            continue
+        f = line.split("|", 1)[1].split()
+        if len(f) >= 6:
+            out.add(tuple(int(v) for v in f[1:6]))
+    return out
+
+
 def build_weights(name, device, copies):
     import torch
 
@@ -277,18 +290,22 @@ def bench_ours(args, device, rank, world):
     choices = {M: wq.wq_get_choice(M, K, N, bits, group) for M in Ms}
 
     # the dispatcher's measured choice (the load-time tuning of the split_k
-    # auto-tune in Mit han lab Llm awq Kernel Selection Thresholds), untimed
+    # auto-tune in Mit han lab Llm awq Kernel Selection Thresholds), untimed;
+    # shapes the tuning file already holds are loaded, the others tuned
+    have = set()
     if args.tuning_file and os.path.exists(args.tuning_file):
         if wq.wq_load_tuning(args.tuning_file) != 0:
             raise RuntimeError("unreadable tuning file " + args.tuning_file)
+        have = tuned_shapes(args.tuning_file)
         choices = {M: wq.wq_get_choice(M, K, N, bits, group) for M in Ms}
-    elif args.tune:
+    if args.tune and any((M, K, N, bits, group) not in have for M in Ms):
         for M in Ms:
-            choices[M] = wq.wq_tune(xs[M], pws[0], ys[M], warmup=2, iters=7)
+            if (M, K, N, bits, group) not in have:
+                choices[M] = wq.wq_tune(xs[M], pws[0], ys[M], warmup=2, iters=7)
         if args.tuning_file:
             wq.wq_save_tuning(args.tuning_file)
 
-    calls = [(M, c) for c in range(copies) for M in Ms]  # one step
+    calls = [(M, c) for M in Ms for c in range(copies)]  # one step
     stream = torch.cuda.Stream(device)
     P = max(1, min(args.steps, 64))  # event sets: per-launch times of the last P steps
 
@@ -298,24 +315,28 @@ def bench_ours(args, device, rank, world):
             wq.wq_linear(xs[M], pws[c], y=ys[M], stream=stream)
     torch.cuda.synchronize(device)
 
-    # one CUDA graph per call; events are recorded on the stream between
-    # graph launches so each kernel's device duration is measurable
+    # one CUDA graph per M: its calls on every weight copy back to back (as
+    # the layers of a decode step run, the next launch may start while the
+    # previous one drains); events recorded on the stream between the graphs
+    # give each M's average launch duration inside the timed region
     graphs = []
-    for M, c in calls:
+    for M in Ms:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            wq.wq_linear(xs[M], pws[c], y=ys[M], stream=stream)
+            for c in range(copies):
+                wq.wq_linear(xs[M], pws[c], y=ys[M], stream=stream)
         graphs.append(g)
     torch.cuda.synchronize(device)
-    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(calls))] for _ in range(P)]
+    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(len(Ms) + 1)] for _ in range(P)]
 
-    def run_step(evs):
+    def run_step(s):
+        evs = evsets[s % P] if s is not None else None
+        if evs is not None:
+            evs[0].record(stream)
         for i, g in enumerate(graphs):
-            if evs is not None:
-                evs[2 * i].record(stream)
             g.replay()
             if evs is not None:
-                evs[2 * i + 1].record(stream)
+                evs[i + 1].record(stream)
 
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     sampler = ClockSampler(vis.split(",")[device.index] if vis else device.index)
@@ -330,7 +351,7 @@ def bench_ours(args, device, rank, world):
             if i % 20 == 0:
                 torch.cuda.synchronize(device)
         for w in range(args.warmup):
-            run_step(evsets[w % P])
+            run_step(w)
     torch.cuda.synchronize(device)
 
     barrier(device)
@@ -339,18 +360,19 @@ def bench_ours(args, device, rank, world):
     with torch.cuda.stream(stream):
         start.record(stream)
         for s in range(args.steps):
-            run_step(evsets[s % P])
+            run_step(s)
         end.record(stream)
     torch.cuda.synchronize(device)
     barrier(device)
     clocks = sampler.stop()
     elapsed_s = start.elapsed_time(end) / 1000.0
 
-    # per-launch durations from the timed region (its last P steps)
+    # per-launch durations from the timed region (its last P steps): each M's
+    # graph time over its launches
     per_call_us = {M: [] for M in Ms}
     for evs in evsets[:min(P, args.steps)]:
-        for i, (M, c) in enumerate(calls):
-            per_call_us[M].append(evs[2 * i].elapsed_time(evs[2 * i + 1]) * 1000.0)
+        for i, M in enumerate(Ms):
+            per_call_us[M].append(evs[i].elapsed_time(evs[i + 1]) * 1000.0 / copies)
 
     step_bytes = sum(call_bytes(bits, K, N, group, M) for M, _ in calls)
     step_flops = sum(call_flops(K, N, M) for M, _ in calls)
@@ -586,8 +608,8 @@ def main():
                        "group": cfg["group"], "Ms": list(cfg["Ms"]), "weight_copies": r["copies"],
                        "l2": f"weights rotated over {r['copies']} copies (> {L2_ROTATION_FACTOR}x L2 of "
                              f"{r['l2_bytes'] // 2**20} MiB); no flush",
-                       "parallelism": "replicas" if world > 1 else "single GPU", "timing": "CUDA graphs, "
-                       "CUDA events on the launching stream, max over ranks"},
+                       "parallelism": "replicas" if world > 1 else "single GPU", "timing": "one CUDA graph "
+                       "per M (its calls back to back), CUDA events between the graphs, max over ranks"},
             "tflops": round(r["tflops"], 2), "per_shape": r["per_shape"], "roofline": r["roofline"],
             "clocks": r["clocks"], "e2e": r["e2e"], "gpu_launches": r["gpu_launches"],
             "dispatch": r["choices"],

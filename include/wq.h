@@ -46,7 +46,8 @@
  *   - "device" pointers are CUDA device pointers on the current device.
  *     "host" pointers are ordinary host memory.
  *   - The caller owns every buffer. No call allocates device memory, except
- *     wq_tune. wq_tune allocates and frees only its timing events.
+ *     wq_tune, which allocates and frees its timing events and a scrub
+ *     buffer of twice the L2 size.
  *   - Work is enqueued on `stream` (0 = legacy default stream). Calls return
  *     after the enqueue, with no implicit synchronization, unless the entry
  *     says "synchronizes".
@@ -242,7 +243,8 @@ int wq_set_workspace(void *ws, size_t bytes);
 
 /* Times every valid (variant, split) for the shape on the caller's own
  * buffers with CUDA events: `warmup` untimed and `iters` timed calls each.
- * It keeps the fastest by median time. On an exact tie the later, larger
+ * Before each timed call it reads a buffer of twice the L2 size, so the
+ * call streams its weights from HBM. It keeps the fastest by median time. On an exact tie the later, larger
  * split wins, as in the split_k auto-tune loop of Mit han lab Llm awq Kernel
  * Selection Thresholds, The Insight. Overwrites y. Synchronizes `stream`.
  * Needs a registered workspace that fits split 32 to try every split. */

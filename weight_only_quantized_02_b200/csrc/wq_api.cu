@@ -179,6 +179,20 @@ int lookup_choice(const DeviceInfo &d, int M, int K, int N, int bits, int group,
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
 
+// Reads a buffer larger than L2 (L2-allocating loads, no L1), so the timed
+// call that follows finds none of its weights in L2 and no dirty lines to
+// write back.  The store is never taken (it keeps the loads).
+__global__ void l2_scrub_kernel(const uint4 *__restrict__ buf, size_t n, uint32_t *sink)
+{
+    uint32_t acc = 0;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const uint4 v = __ldcg(buf + i);
+        acc ^= v.x ^ v.y ^ v.z ^ v.w;
+    }
+    if (acc == 0x9E3779B9u && threadIdx.x == 0x3ff)
+        *sink = acc;
+}
+
 int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros, int group,
                 int N, uint16_t *y, int variant, int split, void *ws, size_t ws_bytes_given, cudaStream_t stream)
 {
@@ -497,16 +511,28 @@ int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
         for (int c : {1, 2})
             cands.push_back({WQ_VARIANT_GEMV_I8, c});
 
-    // Flush buffer larger than L2, so every timed call streams its weights
-    // from HBM (the weights of a decode step are not L2-resident).
+    // Scrub buffer twice the L2 size, read before every timed call, so each
+    // call streams its weights from HBM (the weights of a decode step are not
+    // L2-resident) and finds only clean lines in L2.  Reading it also keeps
+    // the GPU busy while the host enqueues the call.  (A memset flush would
+    // leave L2 full of dirty lines whose write-back the timed call would pay.)
     int l2 = 0;
     int tdev = 0;
     cudaGetDevice(&tdev);
     cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, tdev);
-    const size_t flush_bytes = std::max<size_t>((size_t)l2 * 2, 64u << 20);
+    const size_t flush_bytes = std::max<size_t>((size_t)l2 * 2, 64u << 20) / 16 * 16;
     void *flush = nullptr;
     if (cudaMalloc(&flush, flush_bytes) != cudaSuccess)
         return WQ_ERR_CUDA;
+    auto scrub = [&]() {
+        l2_scrub_kernel<<<4 * d.sm_count, 512, 0, stream>>>(reinterpret_cast<const uint4 *>(flush), flush_bytes / 16,
+                                                            reinterpret_cast<uint32_t *>(flush));
+    };
+    if (cudaMemsetAsync(flush, 0x5a, flush_bytes, stream) != cudaSuccess) {
+        cudaFree(flush);
+        return WQ_ERR_CUDA;
+    }
+    scrub(); // writes the memset's dirty lines back once
     cudaEvent_t e0, e1;
     cudaEventCreate(&e0);
     cudaEventCreate(&e1);
@@ -520,7 +546,7 @@ int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
             continue; // e.g. no workspace large enough for this split
         std::vector<float> t;
         for (int i = 0; i < iters && rc == WQ_OK; ++i) {
-            cudaMemsetAsync(flush, i & 0xff, flush_bytes, stream);
+            scrub();
             cudaEventRecord(e0, stream);
             rc = linear_impl(x, M, K, Wq, scales, zeros, group, N, y, v, s, nullptr, 0, stream);
             cudaEventRecord(e1, stream);

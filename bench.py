@@ -278,7 +278,7 @@ def bench_ours(args, device, rank, world):
     name = args.workload
     cfg0 = gen.WORKLOADS[name]
     K, N, bits, group = cfg0["K"], cfg0["N"], cfg0["bits"], cfg0["group"]
-    Ms = list(cfg0["Ms"])
+    Ms = list(args.ms) if args.ms else list(cfg0["Ms"])
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     wbytes = weight_bytes(bits, K, N, group)
     copies = max(2, math.ceil(L2_ROTATION_FACTOR * l2 / wbytes))
@@ -298,7 +298,12 @@ def bench_ours(args, device, rank, world):
             raise RuntimeError("unreadable tuning file " + args.tuning_file)
         have = tuned_shapes(args.tuning_file)
         choices = {M: wq.wq_get_choice(M, K, N, bits, group) for M in Ms}
-    if args.tune and any((M, K, N, bits, group) not in have for M in Ms):
+    if args.choice is not None:
+        # one fixed (variant, split) for every M: a single kernel to profile
+        for M in Ms:
+            wq.wq_set_choice(M, K, N, bits, group, args.choice[0], args.choice[1])
+        choices = {M: wq.wq_get_choice(M, K, N, bits, group) for M in Ms}
+    elif args.tune and any((M, K, N, bits, group) not in have for M in Ms):
         for M in Ms:
             if (M, K, N, bits, group) not in have:
                 choices[M] = wq.wq_tune(xs[M], pws[0], ys[M], warmup=2, iters=7)
@@ -417,7 +422,7 @@ def bench_ours(args, device, rank, world):
         "value": value_bps / 1e9, "ms_per_step": tmax / args.steps * 1e3, "per_shape": per_shape,
         "roofline": roofline, "clocks": clocks, "e2e": e2e, "copies": copies,
         "gpu_launches": args.steps * len(calls), "tflops": step_flops * args.steps * world / tmax / 1e12,
-        "choices": {str(M): list(choices[M]) for M in Ms}, "l2_bytes": l2,
+        "choices": {str(M): list(choices[M]) for M in Ms}, "l2_bytes": l2, "Ms": Ms,
     }
 
 
@@ -576,6 +581,10 @@ def main():
     ap.add_argument("--tuning-file", default=None,
                     help="load this dispatcher table instead of tuning (saved there after tuning if absent)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ms", type=lambda v: [int(t) for t in v.split(",")], default=None,
+                    help="comma-separated subset of the workload's M values")
+    ap.add_argument("--choice", type=lambda v: tuple(int(t) for t in v.split(":")), default=None,
+                    help="VARIANT:SPLIT used for every M instead of tuning (e.g. to profile one kernel)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -605,7 +614,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02^2) weights quantized on device)",
             "config": {"workload": name, "K": cfg["K"], "N": cfg["N"], "bits": cfg["bits"],
-                       "group": cfg["group"], "Ms": list(cfg["Ms"]), "weight_copies": r["copies"],
+                       "group": cfg["group"], "Ms": r["Ms"], "weight_copies": r["copies"],
                        "l2": f"weights rotated over {r['copies']} copies (> {L2_ROTATION_FACTOR}x L2 of "
                              f"{r['l2_bytes'] // 2**20} MiB); no flush",
                        "parallelism": "replicas" if world > 1 else "single GPU", "timing": "one CUDA graph "

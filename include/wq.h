@@ -46,8 +46,9 @@
  *   - "device" pointers are CUDA device pointers on the current device.
  *     "host" pointers are ordinary host memory.
  *   - The caller owns every buffer. No call allocates device memory, except
- *     wq_tune, which allocates and frees its timing events and a scrub
- *     buffer of twice the L2 size.
+ *     wq_tune, which allocates and frees its timing events and rotation
+ *     copies of the packed weights (about three L2 sizes, at least two
+ *     copies).
  *   - Work is enqueued on `stream` (0 = legacy default stream). Calls return
  *     after the enqueue, with no implicit synchronization, unless the entry
  *     says "synchronizes".
@@ -241,10 +242,12 @@ int wq_set_workspace(void *ws, size_t bytes);
  * bits, group) and guarded by a mutex.
  * ------------------------------------------------------------------- */
 
-/* Times every valid (variant, split) for the shape on the caller's own
- * buffers with CUDA events: `warmup` untimed and `iters` timed calls each.
- * Before each timed call it reads a buffer of twice the L2 size, so the
- * call streams its weights from HBM. It keeps the fastest by median time. On an exact tie the later, larger
+/* Times every valid (variant, split) for the shape with CUDA events, as
+ * decode runs it: R copies of the packed weights (R >= 2, spanning about
+ * three L2 sizes, so no call finds its weights in L2) are called back to
+ * back in rotation with the caller's x and y; `warmup` untimed and `iters`
+ * timed rotations per candidate, per-call time = rotation time / R. It
+ * keeps the fastest by the mean of the middle half of its sorted times. On an exact tie the later, larger
  * split wins, as in the split_k auto-tune loop of Mit han lab Llm awq Kernel
  * Selection Thresholds, The Insight. Overwrites y. Synchronizes `stream`.
  * Needs a registered workspace that fits split 32 to try every split. */

@@ -179,20 +179,6 @@ int lookup_choice(const DeviceInfo &d, int M, int K, int N, int bits, int group,
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
 
-// Reads a buffer larger than L2 (L2-allocating loads, no L1), so the timed
-// call that follows finds none of its weights in L2 and no dirty lines to
-// write back.  The store is never taken (it keeps the loads).
-__global__ void l2_scrub_kernel(const uint4 *__restrict__ buf, size_t n, uint32_t *sink)
-{
-    uint32_t acc = 0;
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
-        const uint4 v = __ldcg(buf + i);
-        acc ^= v.x ^ v.y ^ v.z ^ v.w;
-    }
-    if (acc == 0x9E3779B9u && threadIdx.x == 0x3ff)
-        *sink = acc;
-}
-
 int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros, int group,
                 int N, uint16_t *y, int variant, int split, void *ws, size_t ws_bytes_given, cudaStream_t stream)
 {
@@ -511,28 +497,47 @@ int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
         for (int c : {1, 2})
             cands.push_back({WQ_VARIANT_GEMV_I8, c});
 
-    // Scrub buffer twice the L2 size, read before every timed call, so each
-    // call streams its weights from HBM (the weights of a decode step are not
-    // L2-resident) and finds only clean lines in L2.  Reading it also keeps
-    // the GPU busy while the host enqueues the call.  (A memset flush would
-    // leave L2 full of dirty lines whose write-back the timed call would pay.)
+    // Decode runs its layers back to back, each streaming its own weights
+    // from HBM while the next one is launched behind it.  The tuner times
+    // the same thing: R copies of the packed weights spanning at least three
+    // L2 sizes, called back to back in rotation, one event pair around each
+    // full rotation (per call = rotation time / R), so no call finds its
+    // weights in L2 and launch overlap counts as it does in a decode step.
+    // Copy contents do not affect timing; they are the caller's weights.
     int l2 = 0;
     int tdev = 0;
     cudaGetDevice(&tdev);
     cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, tdev);
-    const size_t flush_bytes = std::max<size_t>((size_t)l2 * 2, 64u << 20) / 16 * 16;
-    void *flush = nullptr;
-    if (cudaMalloc(&flush, flush_bytes) != cudaSuccess)
+    size_t wb = 0, sb = 0, zb = 0;
+    if ((st = wq_packed_bytes(bits, K, N, group, &wb, &sb, &zb)) != WQ_OK)
+        return st;
+    const size_t wb_al = (wb + 255) / 256 * 256, sb_al = (sb + 255) / 256 * 256, zb_al = (zb + 255) / 256 * 256;
+    const size_t copy_bytes = wb_al + sb_al + zb_al;
+    const int R = (int)std::max<size_t>(2, std::min<size_t>(64, (3 * (size_t)l2 + copy_bytes - 1) / copy_bytes));
+    uint8_t *rot = nullptr;
+    if (cudaMalloc(&rot, copy_bytes * R) != cudaSuccess)
         return WQ_ERR_CUDA;
-    auto scrub = [&]() {
-        l2_scrub_kernel<<<4 * d.sm_count, 512, 0, stream>>>(reinterpret_cast<const uint4 *>(flush), flush_bytes / 16,
-                                                            reinterpret_cast<uint32_t *>(flush));
-    };
-    if (cudaMemsetAsync(flush, 0x5a, flush_bytes, stream) != cudaSuccess) {
-        cudaFree(flush);
-        return WQ_ERR_CUDA;
+    std::vector<const void *> rw(R), rs(R), rz(R);
+    for (int c = 0; c < R; ++c) {
+        uint8_t *base = rot + copy_bytes * c;
+        rw[c] = base;
+        rs[c] = base + wb_al;
+        rz[c] = zb ? base + wb_al + sb_al : nullptr;
+        bool okc = cudaMemcpyAsync(base, Wq, wb, cudaMemcpyDeviceToDevice, stream) == cudaSuccess &&
+                   cudaMemcpyAsync(base + wb_al, scales, sb, cudaMemcpyDeviceToDevice, stream) == cudaSuccess &&
+                   (!zb || cudaMemcpyAsync(base + wb_al + sb_al, zeros, zb, cudaMemcpyDeviceToDevice, stream) ==
+                               cudaSuccess);
+        if (!okc) {
+            cudaFree(rot);
+            return WQ_ERR_CUDA;
+        }
     }
-    scrub(); // writes the memset's dirty lines back once
+    auto rotation = [&](int v, int s) {
+        int rc = WQ_OK;
+        for (int c = 0; c < R && rc == WQ_OK; ++c)
+            rc = linear_impl(x, M, K, rw[c], rs[c], rz[c], group, N, y, v, s, nullptr, 0, stream);
+        return rc;
+    };
     cudaEvent_t e0, e1;
     cudaEventCreate(&e0);
     cudaEventCreate(&e1);
@@ -540,15 +545,14 @@ int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
     int result = WQ_OK;
     for (auto [v, s] : cands) {
         int rc = WQ_OK;
-        for (int i = 0; i < warmup && rc == WQ_OK; ++i)
-            rc = linear_impl(x, M, K, Wq, scales, zeros, group, N, y, v, s, nullptr, 0, stream);
+        for (int i = 0; i < std::max(1, warmup) && rc == WQ_OK; ++i)
+            rc = rotation(v, s);
         if (rc != WQ_OK)
             continue; // e.g. no workspace large enough for this split
         std::vector<float> t;
         for (int i = 0; i < iters && rc == WQ_OK; ++i) {
-            scrub();
             cudaEventRecord(e0, stream);
-            rc = linear_impl(x, M, K, Wq, scales, zeros, group, N, y, v, s, nullptr, 0, stream);
+            rc = rotation(v, s);
             cudaEventRecord(e1, stream);
             if (cudaEventSynchronize(e1) != cudaSuccess) {
                 rc = WQ_ERR_CUDA;
@@ -556,22 +560,33 @@ int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
             }
             float ms = 0.f;
             cudaEventElapsedTime(&ms, e0, e1);
-            t.push_back(ms * 1000.f);
+            t.push_back(ms * 1000.f / R);
         }
         if (rc != WQ_OK) {
             if (rc == WQ_ERR_CUDA)
                 result = rc;
             continue;
         }
+        // The event clock ticks in about 1 us steps, as coarse as the
+        // differences between candidates: take the mean of the middle half
+        // of the sorted times (the median's robustness, finer resolution).
         std::sort(t.begin(), t.end());
-        const float med = t[t.size() / 2];
+        const size_t lo = t.size() / 4, hi = t.size() - t.size() / 4;
+        float med = 0.f;
+        for (size_t i = lo; i < hi; ++i)
+            med += t[i];
+        med /= (float)(hi - lo);
+        if (const char *lg = getenv("WQ_TUNE_LOG"); lg && *lg && *lg != '0')
+            fprintf(stderr, "wq_tune M=%d K=%d N=%d bits=%d group=%d variant=%d split=%d us=%.3f\n", M, K, N,
+                    bits, group, v, s, med);
         // ">=": on an exact tie the later (larger) split wins, as in the page's loop
         if (best.variant < 0 || best.us >= med)
             best = {v, s, med};
     }
     cudaEventDestroy(e0);
     cudaEventDestroy(e1);
-    cudaFree(flush);
+    cudaStreamSynchronize(stream);
+    cudaFree(rot);
     if (result != WQ_OK)
         return result;
     if (best.variant < 0)
@@ -624,7 +639,7 @@ int wq_save_tuning(const char *path)
     if (!f)
         return WQ_ERR_TUNING;
     std::lock_guard<std::mutex> lk(g_mu);
-    fprintf(f, "# wq tuning v1: device|sms M K N bits group variant split median_us\n");
+    fprintf(f, "# wq tuning v1: device|sms M K N bits group variant split us_per_call\n");
     for (auto &kv : g_table) {
         const auto &k = kv.first;
         fprintf(f, "%s %d %d %d %d %d %d %d %.3f\n", std::get<0>(k).c_str(), std::get<1>(k), std::get<2>(k),

@@ -257,7 +257,8 @@ def build_weights(name, device, copies):
 
 
 KERNELS = {0: ("gemv_sk", "wq_gemv_sk.cu"), 1: ("gemm", "wq_gemm.cu"), 2: ("gemv_rb", "wq_gemv.cu"),
-           3: ("gemm_sk", "wq_gemm_sk.cu"), 4: ("gemm_i8", "wq_gemm_i8.cu"), 5: ("gemv_i8", "wq_gemv_i8.cu")}
+           3: ("gemm_sk", "wq_gemm_sk.cu"), 4: ("gemm_i8", "wq_gemm_i8.cu"), 5: ("gemv_i8", "wq_gemv_i8.cu"),
+           6: ("gemm_w4", "wq_gemm_w4.cu")}
 
 
 def kernel_name(variant, bits):

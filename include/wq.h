@@ -99,6 +99,9 @@ typedef enum {
                                 as they are, activations as exact digits in shared memory), M <= 8,
                                 3 * M * K bytes <= ~200 KB; split 1 = one 16-warp CTA per SM, 2 = two
                                 8-warp CTAs per SM; needs the workspace */
+#define WQ_VARIANT_GEMM_W4 6 /* W4A16 only, M <= 128: stream-K tcgen05 GEMM with one 512-thread CTA
+                                per SM, every role (weight and x loads, dequantization, MMA, group
+                                rescale) on its own warps with its own ring; needs the workspace */
 
 /* Static description of a status code. Host. Never NULL. */
 const char *wq_strerror(int status);
@@ -194,6 +197,7 @@ int wq_linear(const uint16_t *x, int M, int K, const void *Wq, const void *scale
  * GEMM: split = K-splits, 1 <= split <= min(32, ceil(K/128)).
  * I8MMA: split = 1 (one persistent CTA per SM).
  * GEMV_I8: split = 1 (one 16-warp CTA per SM) or 2 (two 8-warp CTAs per SM).
+ * GEMM_W4: split = 1.
  * Returns WQ_ERR_VARIANT if the pair does not fit the shape. */
 int wq_linear_forced(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
                      const void *zeros, int group, int N, uint16_t *y, int variant, int split,

@@ -24,6 +24,7 @@ pytestmark = pytest.mark.gpu
 
 GEMV, GEMM, GEMV_RB, GEMM_SK, I8, GI = (wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB,
                                         wq.WQ_VARIANT_GEMM_SK, wq.WQ_VARIANT_I8MMA, wq.WQ_VARIANT_GEMV_I8)
+GW4 = wq.WQ_VARIANT_GEMM_W4
 INTEGER = (I8, GI)  # the integer paths: fixed-point activations
 SHAPES = {8: (1120, 400), 4: (1152, 400)}  # (K, N): 3 full panels + a 16-row tail
 M_ALL = [1, 7, 8, 9, 16, 17, 32, 33, 64, 65, 100, 128]
@@ -58,6 +59,8 @@ def _cases(M, K, bits):
         out += [(I8, 1)]
     if M <= 8:  # integer GEMV
         out += [(GI, c) for c in (1, 2)]
+    if bits == 4:  # role-split W4A16 GEMM
+        out += [(GW4, 1)]
     return out
 
 
@@ -278,6 +281,8 @@ def test_argument_errors(weight, ws):
     assert wq.wq_linear_status(x, pw, y, I8, 2) == -11            # one CTA per SM only
     assert wq.wq_linear_status(x, pw, y, GI, 3) == -11            # integer GEMV: split 1 or 2
     assert wq.wq_linear_status(x, pw, y, GI, 0) == 0              # 0: the default
+    assert wq.wq_linear_status(x, pw, y, GW4, 2) == -11           # role-split W4A16 GEMM: split 1 only
+    assert wq.wq_linear_status(x, pw, y, GW4, 1) == (-11 if bits == 8 else 0)  # W4A16 only
     xc = bf16_dev(gen.x_bf16(65, K))
     yc = torch.empty((65, N), dtype=torch.bfloat16, device=dev())
     assert wq.wq_linear_status(xc, pw, yc, I8, 1) == -11          # integer path takes M <= 64 (W4A16: 32)

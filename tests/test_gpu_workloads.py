@@ -21,6 +21,7 @@ pytestmark = pytest.mark.gpu
 
 GEMV, GEMM, GEMV_RB, GEMM_SK, I8, GI = (wq.WQ_VARIANT_GEMV, wq.WQ_VARIANT_GEMM, wq.WQ_VARIANT_GEMV_RB,
                                         wq.WQ_VARIANT_GEMM_SK, wq.WQ_VARIANT_I8MMA, wq.WQ_VARIANT_GEMV_I8)
+GW4 = wq.WQ_VARIANT_GEMM_W4
 
 
 def _build(name):
@@ -82,6 +83,8 @@ def _variants(M, K, bits):
         out += [(I8, 1)]
     if M <= 8:  # integer GEMV
         out += [(GI, c) for c in (1, 2)]
+    if bits == 4:  # role-split W4A16 GEMM
+        out += [(GW4, 1)]
     return out
 
 

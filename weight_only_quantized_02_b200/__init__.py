@@ -30,6 +30,7 @@ WQ_VARIANT_GEMV_RB = 2  # row-block GEMV, no workspace, M <= 32
 WQ_VARIANT_GEMM_SK = 3  # stream-K tcgen05 GEMM (needs the workspace), M <= 128
 WQ_VARIANT_I8MMA = 4    # tcgen05 kind::i8 (needs the workspace): W8A16 M <= 64, W4A16 M <= 32
 WQ_VARIANT_GEMV_I8 = 5  # integer GEMV, mma.sync m16n8k32 s8 on the packed codes (needs the workspace), M <= 8
+WQ_VARIANT_GEMM_W4 = 6  # W4A16 stream-K tcgen05 GEMM, one role-split CTA per SM (needs the workspace), M <= 128
 
 STATUS = {
     0: "WQ_OK", -1: "WQ_ERR_NULL", -2: "WQ_ERR_SHAPE", -3: "WQ_ERR_ALIGN", -4: "WQ_ERR_GROUP",

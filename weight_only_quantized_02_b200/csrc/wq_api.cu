@@ -131,6 +131,8 @@ bool choice_valid(int variant, int split, int M, int K, int bits)
         return M <= 128 && split >= 1 && split <= max_gemm_split(K);
     if (variant == WQ_VARIANT_GEMM_SK)
         return M <= 128 && (split == 1 || split == 2);
+    if (variant == WQ_VARIANT_GEMM_W4)
+        return bits == 4 && M <= 128 && split == 1;
     return false;
 }
 
@@ -229,6 +231,7 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
                       : variant == WQ_VARIANT_GEMM_SK ? 2
                       : variant == WQ_VARIANT_I8MMA   ? 1
                       : variant == WQ_VARIANT_GEMV_I8 ? 1
+                      : variant == WQ_VARIANT_GEMM_W4 ? 1
                                                       : std::min(8, max_gemm_split(K));
     }
     if (split > 0)
@@ -272,6 +275,11 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
         if (!w || have < ws_bytes_gemm_sk(M, N))
             return WQ_ERR_WORKSPACE;
         return cuda_status(launch_gemm_sk(a, c.split, w, d.sm_count, stream));
+    }
+    if (c.variant == WQ_VARIANT_GEMM_W4) {
+        if (!w || have < ws_bytes_gemm_sk(M, N))
+            return WQ_ERR_WORKSPACE;
+        return cuda_status(launch_gemm_w4(a, w, d.sm_count, stream));
     }
     if (c.split > 1 && (!w || have < ws_bytes(M, N, c.split)))
         return WQ_ERR_WORKSPACE;
@@ -493,6 +501,8 @@ int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
         cands.push_back({WQ_VARIANT_GEMM_SK, c});
     if (i8_fits(bits, M, K))
         cands.push_back({WQ_VARIANT_I8MMA, 1});
+    if (bits == 4)
+        cands.push_back({WQ_VARIANT_GEMM_W4, 1});
     if (gi_fits(bits, M, K))
         for (int c : {1, 2})
             cands.push_back({WQ_VARIANT_GEMV_I8, c});
@@ -729,12 +739,12 @@ int wq_dequant_debug(const void *Wq, const void *scales, const void *zeros, int 
 
 int wq_device_error(cudaStream_t stream)
 {
-    int a = 0, b = 0, c = 0, e = 0, f = 0;
+    int a = 0, b = 0, c = 0, e = 0, f = 0, h = 0;
     if (read_device_error(&a, stream) != cudaSuccess || read_gemv_sk_error(&b, stream) != cudaSuccess ||
         read_gemm_sk_error(&c, stream) != cudaSuccess || read_gemm_i8_error(&e, stream) != cudaSuccess ||
-        read_gemm_i4_error(&f, stream) != cudaSuccess)
+        read_gemm_i4_error(&f, stream) != cudaSuccess || read_gemm_w4_error(&h, stream) != cudaSuccess)
         return WQ_ERR_CUDA;
-    return (a == 0 && b == 0 && c == 0 && e == 0 && f == 0) ? WQ_OK : WQ_ERR_TIMEOUT;
+    return (a == 0 && b == 0 && c == 0 && e == 0 && f == 0 && h == 0) ? WQ_OK : WQ_ERR_TIMEOUT;
 }
 
 } // extern "C"

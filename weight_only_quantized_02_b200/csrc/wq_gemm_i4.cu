@@ -291,14 +291,9 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
                 sring[(i % C::kSQ) * 128 + r0] = sc[r0];
                 sring[(i % C::kSQ) * 128 + r1] = sc[r1];
             }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&pempty[st]); // the packed stage is free for the next load
-            if (i >= SA && !mbar_wait_warp(&aempty[sa], ((i / SA) - 1) & 1)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
+            // Expand before releasing the stage: the producer refills a
+            // released stage at once, and a load still in flight could
+            // otherwise return the next block's bytes.
             const uint32_t z40 = z0 * 0x01010101u, z41 = z1 * 0x01010101u;
             // tcgen05.st 16x256b.x4: column group 2 tt + half holds runs (a, b)
             // (half 0) or (c, d) (half 1) of tile tt: lane g / g+8, columns
@@ -312,6 +307,14 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
                 expand_word(w.z, z40, r[8 * tt + 4], r[8 * tt + 5]); // row g,   runs c, d
                 expand_word(w.w, z41, r[8 * tt + 6], r[8 * tt + 7]); // row g+8, runs c, d
             }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&pempty[st]); // the packed stage is free for the next load
+            if (i >= SA && !mbar_wait_warp(&aempty[sa], ((i / SA) - 1) & 1)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
             tmem_st_16x256b_x4(tmem + tl + (uint32_t)(C::kA0 + 32 * sa), r);
             tmem_wait_st();
             tc_fence_before();

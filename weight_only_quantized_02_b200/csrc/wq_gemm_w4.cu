@@ -1,0 +1,491 @@
+// wq_gemm_w4.cu -- W4A16 (group 128, scale and zero point per group) small-M
+// GEMM on tcgen05: persistent stream-K, one CTA per SM, every role on its
+// own warps with its own ring, so no role waits for another role's round
+// trip on every unit.
+//
+//     y[m][n] = sum_g s[n][g] * D_g[n][m],
+//     D_g[n][m] = sum_{k in g} (q[n][k] - z[n][g]) * x[m][k]
+//
+// (the WnA16 grouping of "Toward a Cleaner Quantization Stack in SGLang",
+// Figure 4).  The tensor cores take the exact integers q - z as bf16, so the
+// only rounding is the fp32 accumulation; the group scale is applied in fp32
+// to each group's accumulator.  Weights are the MMA's M side (128 rows of a
+// panel) and tokens its N side (NT = 16 .. 128), so every M <= 128 uses the
+// same instruction shape.
+//
+// Units are (128-row panel, 128-k block) pairs, one group each, laid out
+// contiguously in HBM by the packer (wq_layout.h); each CTA takes an equal
+// contiguous range of them (the stream-K partitioning that the Marlin
+// register and launch scheduling benchmark names as the alternative to a
+// fixed split-K).
+//
+// Warp roles (512 threads):
+//   warp 0     weight producer: per unit the 8 KB packed block and its 64
+//              bytes of zero points into a deep ring (kWS stages), and the
+//              group's 256 bytes of scales into a separate scale ring.  A
+//              weight stage is released as soon as the dequant warps have
+//              read it, so the ring turns over at the memory latency.
+//              Weights never depend on the preceding kernel: no launch wait.
+//   warp 1     allocates all 512 tensor-memory columns; one thread issues
+//              eight tcgen05.mma kind::f16 (K = 16 each) per unit, A (the
+//              dequantized tile) from tensor memory, B (x) from shared
+//              memory, D into one of kACC per-unit group accumulators.
+//   warp 2     x producer: the unit's x tile (NT tokens x 128 k, 2-D tensor
+//              map, 128-byte swizzle, rows past M read as zero) into its own
+//              ring (kXS stages), released by the MMA's commit.
+//   warps 4..  retire warps, one per tensor-memory lane quadrant and column
+//              slice: per unit, s[n][g] * D_g into fp32 register totals;
+//              at the end of a panel, y (or a partial and a ticket; the last
+//              contributor sums every partial in CTA order: deterministic).
+//   rest       dequant warps: packed tiles -> exact bf16 integers q - z in
+//              tensor memory (tcgen05.st 16x256b, the register layout the
+//              packed tile already has), into one of kAS A stages.
+// Every mbarrier wait is bounded (2 s); on a timeout the device error word
+// is set and every role winds down.
+#include <cstdint>
+
+#include <cuda_bf16.h>
+
+#include "wq_device.cuh"
+#include "wq_gemm_common.cuh"
+#include "wq_internal.h"
+
+namespace wq {
+
+static __device__ int g_gemm_w4_error = 0;
+
+struct GemmW4Params {
+    int M, K, N, KB, U;
+    const uint8_t *wq;
+    const uint16_t *scales;
+    const uint8_t *zeros;
+    uint16_t *y;
+    float *part;   // [CTAs][2 slots][128 rows][NT]
+    uint32_t *cnt; // [panels][8] tickets
+};
+
+constexpr int kW4Threads = 512;
+constexpr int kW4Warps = kW4Threads / 32;
+
+template <int NT>
+struct W4Cfg {
+    static constexpr int kXB = NT * 256;                 // x tile: NT rows x 128 k bf16
+    static constexpr int kWSB = 8192 + 64;               // packed block + zero points
+    static constexpr int kSS = 32;                       // scale stages (256 B each)
+    static constexpr int kXS = NT == 16 ? 8 : NT == 32 ? 6 : NT == 64 ? 4 : 3;
+    static constexpr int kWS = NT <= 32 ? 16 : NT == 64 ? 14 : 12;
+    static constexpr int kACC = NT <= 32 ? 128 / NT : 256 / NT; // group accumulators
+    static constexpr int kA0 = kACC * NT;                // first A column
+    static constexpr int kAS = (512 - kA0) / 64;         // A stages, 64 columns each
+    static constexpr int kRW = NT == 128 ? 8 : 4;        // retire warps
+    static constexpr int kCW = NT * 4 / kRW;             // token columns per retire warp
+    static constexpr int kDW = kW4Warps - 4 - kRW;       // dequant warps
+    static constexpr int kBPW = 8 / kDW;                 // 16-row blocks per dequant warp
+    static_assert(kA0 + 64 * kAS == 512, "tensor memory plan");
+    static_assert(kAS >= 2 && kACC >= 2, "double buffering");
+    static_assert(kDW == 4 || kDW == 8, "dequant warps cover the four lane quadrants evenly");
+    static_assert(kCW % 16 == 0, "retire loads 16 columns at a time");
+};
+
+template <int NT>
+constexpr size_t gemm_w4_smem_bytes()
+{
+    using C = W4Cfg<NT>;
+    return 1024 + (size_t)C::kXS * C::kXB + (size_t)C::kWS * C::kWSB + (size_t)C::kSS * 256 +
+           (size_t)(2 * C::kWS + 2 * C::kXS + 2 * C::kSS + 2 * C::kAS + 2 * C::kACC) * 8 + 16;
+}
+
+// The last contributor to a split panel: sums the fp32 partials of CTAs
+// cf .. cl for its row r and tokens t0 .. t0 + CW - 1 in CTA order and
+// writes y.  Kept out of line: it runs once per split panel, and inlined its
+// registers would add to those of the retire loop's totals.
+template <int NT, int CW>
+__device__ __noinline__ void w4_fixup(const GemmW4Params &p, long long U, int G, int pnl, int cf, int cl, int r,
+                                      int t0)
+{
+    const int KB = p.KB;
+    const int nrow = pnl * kPanelRows + r;
+    for (int j0 = 0; j0 < CW; j0 += 16) {
+        float acc[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            acc[j] = 0.f;
+        for (int cc = cf; cc <= cl; ++cc) {
+            const int sl = (pnl == sk_start(U, G, cc) / KB) ? 0 : 1;
+            const float *src = p.part + ((size_t)(cc * 2 + sl) * kPanelRows + r) * NT + t0 + j0;
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + j));
+                acc[j] += v.x;
+                acc[j + 1] += v.y;
+                acc[j + 2] += v.z;
+                acc[j + 3] += v.w;
+            }
+        }
+        if (nrow < p.N) {
+            const int jn = min(16, p.M - t0 - j0);
+            uint16_t *yp = p.y + (size_t)(t0 + j0) * p.N + nrow;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (j < jn)
+                    *yp = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
+                yp += p.N;
+            }
+        }
+    }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_constant__ CUtensorMap tmx,
+                                                                const GemmW4Params p)
+{
+    using C = W4Cfg<NT>;
+    constexpr int XS = C::kXS, WS = C::kWS, SS = C::kSS, AS = C::kAS, ACC = C::kACC;
+    constexpr int XB = C::kXB, WSB = C::kWSB, A0 = C::kA0;
+    constexpr int RW = C::kRW, CW = C::kCW, DW = C::kDW, BPW = C::kBPW;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sX = smem;              // XS x tiles, 1024-byte aligned (swizzled operand)
+    uint8_t *sW = sX + XS * XB;      // WS packed blocks + zero points
+    uint8_t *sS = sW + WS * WSB;     // SS group scales
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sS + SS * 256);
+    uint64_t *wfull = bars, *wempty = wfull + WS;
+    uint64_t *xfull = wempty + WS, *xempty = xfull + XS;
+    uint64_t *sfull = xempty + XS, *sempty = sfull + SS;
+    uint64_t *afull = sempty + SS, *aempty = afull + AS;
+    uint64_t *accfull = aempty + AS, *accempty = accfull + ACC;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(accempty + ACC);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = gridDim.x, cta = blockIdx.x;
+    const long long U = p.U;
+    const int KB = p.KB;
+    const int u0 = sk_start(U, G, cta), u1 = sk_start(U, G, cta + 1);
+    const int n = u1 - u0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < WS; ++s) {
+            mbar_init(&wfull[s], 1);
+            mbar_init(&wempty[s], DW);
+        }
+        for (int s = 0; s < XS; ++s) {
+            mbar_init(&xfull[s], 1);
+            mbar_init(&xempty[s], 1);
+        }
+        for (int s = 0; s < SS; ++s) {
+            mbar_init(&sfull[s], 1);
+            mbar_init(&sempty[s], RW);
+        }
+        for (int s = 0; s < AS; ++s) {
+            mbar_init(&afull[s], DW);
+            mbar_init(&aempty[s], 1);
+        }
+        for (int s = 0; s < ACC; ++s) {
+            mbar_init(&accfull[s], 1);
+            mbar_init(&accempty[s], RW);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(s_tmem, 512);
+        tmem_relinquish();
+    }
+    if (warp == 2 && lane == 0)
+        prefetch_tensormap(&tmx);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // The next kernel on the stream may launch now; whatever it shares with
+    // this grid (its x, y, the workspace) waits behind its own launch wait.
+    pdl_launch_dependents();
+    const uint32_t tmem = *s_tmem;
+    bool ok = true;
+
+    auto panel_of = [&](int i) { return (u0 + i) / KB; };
+    auto last_of_panel = [&](int i) { return i == n - 1 || panel_of(i + 1) != panel_of(i); };
+
+    if (warp == 0) {
+        // ---------------- weight + scale producer ----------------
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            for (int i = 0; i < n; ++i) {
+                const size_t u = (size_t)(u0 + i);
+                const int ws = i % WS, ss = i % SS;
+                if (i >= WS && !mbar_wait(&wempty[ws], ((i / WS) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&wfull[ws], 8192 + 64);
+                bulk_g2s(sW + ws * WSB, p.wq + u * 8192, 8192, &wfull[ws], pol);
+                bulk_g2s(sW + ws * WSB + 8192, p.zeros + u * 64, 64, &wfull[ws], pol);
+                if (i >= SS && !mbar_wait(&sempty[ss], ((i / SS) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&sfull[ss], 256);
+                bulk_g2s(sS + ss * 256, p.scales + u * kPanelRows, 256, &sfull[ss], pol);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16(NT);
+            for (int i = 0; i < n; ++i) {
+                const int as = i % AS, xs = i % XS, ac = i % ACC;
+                if (!mbar_wait(&afull[as], (i / AS) & 1) || !mbar_wait(&xfull[xs], (i / XS) & 1) ||
+                    (i >= ACC && !mbar_wait(&accempty[ac], ((i / ACC) - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t xaddr = smem_u32(sX + xs * XB);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t bdesc = smem_desc_sw128(xaddr + (kk >> 2) * (NT * 128) + (kk & 3) * 32);
+                    umma_ts(tmem + ac * NT, tmem + A0 + as * 64 + kk * 8, bdesc, idesc, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&aempty[as]);
+                umma_commit(&xempty[xs]);
+                umma_commit(&accfull[ac]);
+            }
+        }
+    } else if (warp == 2) {
+        // ---------------- x producer ----------------
+        if (lane == 0) {
+            pdl_wait(); // x may be written by the preceding kernel
+            const uint64_t pol = policy_evict_last();
+            for (int i = 0; i < n; ++i) {
+                const int xs = i % XS, kb = (u0 + i) % KB;
+                if (i >= XS && !mbar_wait(&xempty[xs], ((i / XS) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&xfull[xs], XB);
+                tma_load_2d(sX + xs * XB, &tmx, kb * kBlockK, 0, &xfull[xs], pol);
+                tma_load_2d(sX + xs * XB + NT * 128, &tmx, kb * kBlockK + 64, 0, &xfull[xs], pol);
+            }
+        }
+    } else if (warp >= 4 && warp < 4 + RW) {
+        // ---------------- retire warps ----------------
+        pdl_wait(); // y and the workspace may still be in use by the preceding kernel
+        const int q = warp & 3, c = (warp - 4) >> 2; // lane quadrant, column slice
+        const int dw = q + 4 * c;                    // ticket owner index within a panel
+        const int r = 32 * q + lane;                 // output row (in the panel) of this thread
+        const uint32_t tq = (uint32_t)(32 * q) << 16;
+        float tot[CW];
+#pragma unroll
+        for (int j = 0; j < CW; ++j)
+            tot[j] = 0.f;
+
+        // This thread's CW totals of panel pnl: to y when this CTA covered
+        // the whole panel, else as a partial + per-warp ticket.
+        auto flush = [&](int pnl) {
+            const int lo = max(u0, pnl * KB), hi = min(u1, (pnl + 1) * KB);
+            const int nrow = pnl * kPanelRows + r;
+            const int t0 = c * CW; // first token of this slice
+            if (lo == pnl * KB && hi == (pnl + 1) * KB) {
+                if (nrow < p.N) {
+                    const int jn = min(CW, p.M - t0); // tokens of this slice that exist
+                    uint16_t *yp = p.y + (size_t)t0 * p.N + nrow;
+#pragma unroll
+                    for (int j = 0; j < CW; ++j) {
+                        if (j < jn)
+                            *yp = __bfloat16_as_ushort(__float2bfloat16_rn(tot[j]));
+                        yp += p.N;
+                    }
+                }
+                return;
+            }
+            const int slot = (pnl == u0 / KB) ? 0 : 1;
+            float *mine = p.part + ((size_t)(cta * 2 + slot) * kPanelRows + r) * NT + t0;
+#pragma unroll
+            for (int j = 0; j < CW; j += 4)
+                *reinterpret_cast<float4 *>(mine + j) = make_float4(tot[j], tot[j + 1], tot[j + 2], tot[j + 3]);
+            __threadfence(); // every lane's partial is visible before lane 0's ticket
+            __syncwarp();
+            uint32_t ticket = 0;
+            if (lane == 0)
+                ticket = ticket_take_acq_rel(&p.cnt[pnl * 8 + dw]);
+            ticket = __shfl_sync(0xffffffffu, ticket, 0);
+            const int cf = sk_owner(U, G, pnl * KB), cl = sk_owner(U, G, (pnl + 1) * KB - 1);
+            if (ticket != (uint32_t)(cl - cf))
+                return;
+            __syncwarp(); // lane 0's acquire orders every lane's reads below
+            w4_fixup<NT, CW>(p, U, G, pnl, cf, cl, r, t0);
+            if (lane == 0)
+                atomicExch(&p.cnt[pnl * 8 + dw], 0u); // ready for the next call
+        };
+
+        for (int i = 0; i < n; ++i) {
+            const int ac = i % ACC, ss = i % SS;
+            if (!mbar_wait_warp(&accfull[ac], (i / ACC) & 1) || !mbar_wait_warp(&sfull[ss], (i / SS) & 1)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float s = bf16_bits_to_float(reinterpret_cast<const uint16_t *>(sS + ss * 256)[r]);
+            const uint32_t ta = tmem + tq + ac * NT + c * CW;
+#pragma unroll
+            for (int j0 = 0; j0 < CW; j0 += 16) { // 16 columns per load keeps the totals in registers
+                float v[16];
+                tmem_ld_32x32b_x16(ta + j0, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    tot[j0 + j] = fmaf(s, v[j], tot[j0 + j]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&accempty[ac]);
+                mbar_arrive(&sempty[ss]);
+            }
+            if (last_of_panel(i)) {
+                flush(panel_of(i));
+#pragma unroll
+                for (int j = 0; j < CW; ++j)
+                    tot[j] = 0.f;
+            }
+        }
+    } else if (warp >= 4 + RW) {
+        // ---------------- dequant warps ----------------
+        const int d = warp - 4 - RW;  // 0 .. DW-1
+        const int q = warp & 3;       // lane quadrant
+        const int g = lane >> 2;
+        int jb[BPW];                  // this warp's 16-row blocks (rows 32q .. 32q+31)
+#pragma unroll
+        for (int b = 0; b < BPW; ++b)
+            jb[b] = BPW == 1 ? 2 * q + (d >> 2) : 2 * q + b;
+        for (int i = 0; i < n; ++i) {
+            const int ws = i % WS, as = i % AS;
+            if (!mbar_wait_warp(&wfull[ws], (i / WS) & 1)) {
+                ok = false;
+                break;
+            }
+            // Dequantize straight from the stage and release it only after
+            // every loaded value has been consumed: the producer refills a
+            // released stage at once, and a load still in flight could
+            // otherwise return the next block's bytes.
+            const uint8_t *blk = sW + ws * WSB;
+            uint32_t rr[BPW][2][16];
+#pragma unroll
+            for (int b = 0; b < BPW; ++b) {
+                const uint4 w0 = *reinterpret_cast<const uint4 *>(blk + jb[b] * 1024 + lane * 16);
+                const uint4 w1 = *reinterpret_cast<const uint4 *>(blk + jb[b] * 1024 + 512 + lane * 16);
+                const int r0 = 16 * jb[b] + g, r1 = r0 + 8;
+                const uint32_t z0 = (blk[8192 + (r0 >> 1)] >> (4 * (r0 & 1))) & 0xFu;
+                const uint32_t z1 = (blk[8192 + (r1 >> 1)] >> (4 * (r1 & 1))) & 0xFu;
+                const uint32_t zlo = 0x43004300u | z0 | (z0 << 16); // bf16x2 {128 + z, 128 + z}
+                const uint32_t zhi = 0x43004300u | z1 | (z1 << 16);
+                int4_tile_regs(w0, zlo, zhi, rr[b][0]);
+                int4_tile_regs(w1, zlo, zhi, rr[b][1]);
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&wempty[ws]);
+            if (i >= AS && !mbar_wait_warp(&aempty[as], ((i / AS) - 1) & 1)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int b = 0; b < BPW; ++b) {
+                const uint32_t ta = tmem + ((uint32_t)(32 * q + 16 * (jb[b] & 1)) << 16) + A0 + as * 64;
+                tmem_st_16x256b_x4(ta, rr[b][0]);
+                tmem_st_16x256b_x4(ta + 32, rr[b][1]);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&afull[as]);
+        }
+    }
+
+    if (!ok)
+        atomicExch(&g_gemm_w4_error, kErrTimeout);
+    tc_fence_before();
+    // Lane 0 of warps 0-2 ran its role alone: reconverge every warp first, so
+    // the CTA barrier below (aligned: whole warps) waits for every role to
+    // finish before tensor memory is released.
+    __syncwarp();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int NT>
+static cudaError_t launch_gemm_w4_t(const LinearArgs &a, void *ws, int sm_count, cudaStream_t st)
+{
+    constexpr size_t smem = gemm_w4_smem_bytes<NT>();
+    static_assert(smem <= 227 * 1024, "shared memory per CTA");
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e =
+            cudaFuncSetAttribute(gemm_w4_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+        attr_set = true;
+    }
+    CUtensorMap map;
+    if (!make_x_map<NT>(&map, a.x, a.M, a.K))
+        return cudaErrorInvalidValue;
+    const Shape sh{a.bits, a.K, a.N, a.group};
+    GemmW4Params p;
+    p.M = a.M;
+    p.K = a.K;
+    p.N = a.N;
+    p.KB = sh.kblocks();
+    p.U = sh.panels() * sh.kblocks();
+    p.wq = (const uint8_t *)a.wq;
+    p.scales = (const uint16_t *)a.scales;
+    p.zeros = (const uint8_t *)a.zeros;
+    p.y = a.y;
+    p.cnt = (uint32_t *)ws;
+    p.part = (float *)((uint8_t *)ws + ws_counter_bytes(a.N));
+    int G = sm_count;
+    if (G > kSkMaxCtas)
+        G = kSkMaxCtas;
+    if (G > p.U)
+        G = p.U;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(kW4Threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_w4_kernel<NT>, map, p);
+}
+
+cudaError_t launch_gemm_w4(const LinearArgs &a, void *ws, int sm_count, cudaStream_t st)
+{
+    switch (gemm_token_tile(a.M)) {
+    case 16: return launch_gemm_w4_t<16>(a, ws, sm_count, st);
+    case 32: return launch_gemm_w4_t<32>(a, ws, sm_count, st);
+    case 64: return launch_gemm_w4_t<64>(a, ws, sm_count, st);
+    default: return launch_gemm_w4_t<128>(a, ws, sm_count, st);
+    }
+}
+
+cudaError_t read_gemm_w4_error(int *code, cudaStream_t st)
+{
+    int host = 0, zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&host, g_gemm_w4_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess)
+        return e;
+    e = cudaMemcpyToSymbolAsync(g_gemm_w4_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess)
+        return e;
+    e = cudaStreamSynchronize(st);
+    *code = host;
+    return e;
+}
+
+} // namespace wq

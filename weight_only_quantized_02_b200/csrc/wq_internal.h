@@ -85,6 +85,11 @@ cudaError_t launch_gemm(const LinearArgs &a, int split, void *ws, int sm_count, 
 cudaError_t launch_gemm_sk(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st);
 cudaError_t read_gemm_sk_error(int *code, cudaStream_t st);
 
+// W4A16 stream-K GEMM (the GEMM_SK variant for 4-bit weights): one
+// 512-thread CTA per SM; ws >= ws_bytes_gemm_sk.
+cudaError_t launch_gemm_w4(const LinearArgs &a, void *ws, int sm_count, cudaStream_t st);
+cudaError_t read_gemm_w4_error(int *code, cudaStream_t st);
+
 // Integer tensor-core GEMM: ws >= ws_bytes_gemm_i8 / ws_bytes_gemm_i4 (always needed).
 cudaError_t launch_gemm_i8(const LinearArgs &a, void *ws, int sm_count, cudaStream_t st);
 cudaError_t read_gemm_i8_error(int *code, cudaStream_t st);

@@ -296,16 +296,30 @@ __global__ void __launch_bounds__(kGskThreads) __maxnreg__((GskCfg<BITS, NT>::kM
 #pragma unroll
                 for (int c = 0; c < CH; ++c)
                     tot[c] = 0.f;
-                for (int cc = cf; cc <= cl; ++cc) {
-                    const int sl = (pnl == sk_start(U, G, cc) / KB) ? 0 : 1;
-                    const float *src = p.part + ((size_t)(cc * 2 + sl) * kPanelRows + r) * NT + h * HALF + c0;
+                // two contributors' partials in flight at once, summed in CTA order
+                for (int cc0 = cf; cc0 <= cl; cc0 += 2) {
+                    float4 t4[2][CH / 4];
 #pragma unroll
-                    for (int c = 0; c < CH; c += 4) {
-                        const float4 t4 = __ldcg(reinterpret_cast<const float4 *>(src + c));
-                        tot[c] += t4.x;
-                        tot[c + 1] += t4.y;
-                        tot[c + 2] += t4.z;
-                        tot[c + 3] += t4.w;
+                    for (int u = 0; u < 2; ++u) {
+                        const int cc = cc0 + u;
+                        const int sl = (cc <= cl && pnl == sk_start(U, G, cc) / KB) ? 0 : 1;
+                        const float *src = p.part + ((size_t)(cc * 2 + sl) * kPanelRows + r) * NT + h * HALF + c0;
+#pragma unroll
+                        for (int c = 0; c < CH; c += 4)
+                            t4[u][c / 4] = cc <= cl ? __ldcg(reinterpret_cast<const float4 *>(src + c))
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        if (cc0 + u > cl)
+                            break;
+#pragma unroll
+                        for (int c = 0; c < CH; c += 4) {
+                            tot[c] += t4[u][c / 4].x;
+                            tot[c + 1] += t4[u][c / 4].y;
+                            tot[c + 2] += t4[u][c / 4].z;
+                            tot[c + 3] += t4[u][c / 4].w;
+                        }
                     }
                 }
                 if (nrow < p.N) {

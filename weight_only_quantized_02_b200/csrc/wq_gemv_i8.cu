@@ -227,25 +227,51 @@ __device__ __forceinline__ void gi_flush(const GiParams &p, int rb, bool whole, 
     const int wf = sk_owner(p.I, Wt, rb * CPR), wl = sk_owner(p.I, Wt, rb * CPR + CPR - 1);
     if (ticket == (uint32_t)(wl - wf)) {
         __syncwarp(); // lane 0's acquire orders every lane's reads below
+        // the partials of up to four contributors are loaded together (one
+        // round trip to L2 instead of one per contributor), then summed in
+        // warp order
+        auto src_of = [&](int ww) {
+            const int sl = (sk_start(p.I, Wt, ww) / CPR == rb) ? 0 : 1;
+            return p.part + ((size_t)ww * 2 + sl) * 16 * NR;
+        };
         for (int q = lane; q < 16 * M; q += 32) {
             const int r = q & 15, m = q >> 4;
             if constexpr (BITS == 8) {
                 int32_t t0 = 0, t1 = 0, t2 = 0;
-                for (int ww = wf; ww <= wl; ++ww) {
-                    const int sl = (sk_start(p.I, Wt, ww) / CPR == rb) ? 0 : 1;
-                    const int32_t *src =
-                        reinterpret_cast<const int32_t *>(p.part) + ((size_t)ww * 2 + sl) * 16 * NR + r * NR + 3 * m;
-                    t0 += __ldcg(src);
-                    t1 += __ldcg(src + 1);
-                    t2 += __ldcg(src + 2);
+                for (int w0 = wf; w0 <= wl; w0 += 4) {
+                    int32_t v[4][3];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        v[u][0] = v[u][1] = v[u][2] = 0;
+                        if (w0 + u <= wl) {
+                            const int32_t *src = reinterpret_cast<const int32_t *>(src_of(w0 + u)) + r * NR + 3 * m;
+                            v[u][0] = __ldcg(src);
+                            v[u][1] = __ldcg(src + 1);
+                            v[u][2] = __ldcg(src + 2);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        t0 += v[u][0];
+                        t1 += v[u][1];
+                        t2 += v[u][2];
+                    }
                 }
                 const double sc = (double)bf16_bits_to_float(p.scales[n0 + r]) * pow2_of(-s_e[m]);
                 p.y[(size_t)m * N + n0 + r] = i8_output(t0, t1, t2, sc);
             } else {
                 float tot = 0.f;
-                for (int ww = wf; ww <= wl; ++ww) {
-                    const int sl = (sk_start(p.I, Wt, ww) / CPR == rb) ? 0 : 1;
-                    tot += __ldcg(reinterpret_cast<const float *>(p.part) + ((size_t)ww * 2 + sl) * 16 * NR + r * NR + m);
+                for (int w0 = wf; w0 <= wl; w0 += 4) {
+                    float v[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        v[u] = w0 + u <= wl
+                                   ? __ldcg(reinterpret_cast<const float *>(src_of(w0 + u)) + r * NR + m)
+                                   : 0.f;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (w0 + u <= wl)
+                            tot += v[u];
                 }
                 p.y[(size_t)m * N + n0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(tot));
             }

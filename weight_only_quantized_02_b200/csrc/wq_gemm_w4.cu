@@ -20,16 +20,13 @@
 // fixed split-K).
 //
 // Warp roles (512 threads):
-//   warp 0     weight producer: per unit the 8 KB packed block and its 64
-//              bytes of zero points into a deep ring (kWS stages), and the
-//              group's 256 bytes of scales into a separate scale ring.  A
-//              weight stage is released as soon as the dequant warps have
-//              read it, so the ring turns over at the memory latency.
-//              Weights never depend on the preceding kernel: no launch wait.
-//   warp 1     allocates all 512 tensor-memory columns; one thread issues
-//              eight tcgen05.mma kind::f16 (K = 16 each) per unit, A (the
-//              dequantized tile) from tensor memory, B (x) from shared
-//              memory, D into one of kACC per-unit group accumulators.
+//   warp 0     scale producer: per unit the group's 256 bytes of scales into
+//              a scale ring (bulk copies).
+//   warps 1, 3 warp 1 allocates all 512 tensor-memory columns; one thread of
+//              each issues eight tcgen05.mma kind::f16 (K = 16 each) per
+//              unit, even units and odd units: A (the dequantized tile)
+//              from tensor memory, B (x) from shared memory, D into one of
+//              kACC per-unit group accumulators.
 //   warp 2     x producer: the unit's x tile (NT tokens x 128 k, 2-D tensor
 //              map, 128-byte swizzle, rows past M read as zero) into its own
 //              ring (kXS stages), released by the MMA's commit.
@@ -37,9 +34,14 @@
 //              slice: per unit, s[n][g] * D_g into fp32 register totals;
 //              at the end of a panel, y (or a partial and a ticket; the last
 //              contributor sums every partial in CTA order: deterministic).
-//   rest       dequant warps: packed tiles -> exact bf16 integers q - z in
-//              tensor memory (tcgen05.st 16x256b, the register layout the
-//              packed tile already has), into one of kAS A stages.
+//   rest       dequant warps: each fetches its own 16-row blocks of every
+//              unit (and their zero points) with 16-byte cp.async into a
+//              private shared-memory ring kDepth units deep (the load path,
+//              many requests per SM in flight: one thread's bulk copies
+//              stream too slowly for the layer), then writes the exact bf16
+//              integers q - z into tensor memory (tcgen05.st 16x256b, the
+//              register layout the packed tile already has), into one of kAS
+//              A stages.  Weights never depend on the preceding kernel.
 // Every mbarrier wait is bounded (2 s); on a timeout the device error word
 // is set and every role winds down.
 #include <cstdint>
@@ -70,29 +72,41 @@ constexpr int kW4Warps = kW4Threads / 32;
 template <int NT>
 struct W4Cfg {
     static constexpr int kXB = NT * 256;                 // x tile: NT rows x 128 k bf16
-    static constexpr int kWSB = 8192 + 64;               // packed block + zero points
     static constexpr int kSS = 32;                       // scale stages (256 B each)
     static constexpr int kXS = NT == 16 ? 8 : NT == 32 ? 6 : NT == 64 ? 4 : 3;
-    static constexpr int kWS = NT <= 32 ? 16 : NT == 64 ? 14 : 12;
+    static constexpr int kDepth = NT <= 32 ? 16 : NT == 64 ? 14 : 12; // units in each dequant warp's ring
     static constexpr int kACC = NT <= 32 ? 128 / NT : 256 / NT; // group accumulators
     static constexpr int kA0 = kACC * NT;                // first A column
     static constexpr int kAS = (512 - kA0) / 64;         // A stages, 64 columns each
-    static constexpr int kRW = NT == 128 ? 8 : 4;        // retire warps
+    static constexpr int kRW = NT >= 64 ? 8 : 4;         // retire warps
     static constexpr int kCW = NT * 4 / kRW;             // token columns per retire warp
     static constexpr int kDW = kW4Warps - 4 - kRW;       // dequant warps
     static constexpr int kBPW = 8 / kDW;                 // 16-row blocks per dequant warp
+    static constexpr int kSlot = kBPW * 1024 + 16;       // a unit's blocks + its 16-byte zero-point segment
     static_assert(kA0 + 64 * kAS == 512, "tensor memory plan");
     static_assert(kAS >= 2 && kACC >= 2, "double buffering");
     static_assert(kDW == 4 || kDW == 8, "dequant warps cover the four lane quadrants evenly");
     static_assert(kCW % 16 == 0, "retire loads 16 columns at a time");
 };
 
+// 16-byte asynchronous global -> shared copy (L2 only) and its groups.
+__device__ __forceinline__ void cp_async_cg16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 template <int NT>
 constexpr size_t gemm_w4_smem_bytes()
 {
     using C = W4Cfg<NT>;
-    return 1024 + (size_t)C::kXS * C::kXB + (size_t)C::kWS * C::kWSB + (size_t)C::kSS * 256 +
-           (size_t)(2 * C::kWS + 2 * C::kXS + 2 * C::kSS + 2 * C::kAS + 2 * C::kACC) * 8 + 16;
+    return 1024 + (size_t)C::kXS * C::kXB + (size_t)C::kSS * 256 + (size_t)C::kDW * C::kDepth * C::kSlot +
+           (size_t)(2 * C::kXS + 2 * C::kSS + 2 * C::kAS + 2 * C::kACC) * 8 + 16;
 }
 
 // The last contributor to a split panel: sums the fp32 partials of CTAs
@@ -140,18 +154,17 @@ __global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_con
                                                                 const GemmW4Params p)
 {
     using C = W4Cfg<NT>;
-    constexpr int XS = C::kXS, WS = C::kWS, SS = C::kSS, AS = C::kAS, ACC = C::kACC;
-    constexpr int XB = C::kXB, WSB = C::kWSB, A0 = C::kA0;
+    constexpr int XS = C::kXS, SS = C::kSS, AS = C::kAS, ACC = C::kACC, DEPTH = C::kDepth, SLOT = C::kSlot;
+    constexpr int XB = C::kXB, A0 = C::kA0;
     constexpr int RW = C::kRW, CW = C::kCW, DW = C::kDW, BPW = C::kBPW;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sX = smem;              // XS x tiles, 1024-byte aligned (swizzled operand)
-    uint8_t *sW = sX + XS * XB;      // WS packed blocks + zero points
-    uint8_t *sS = sW + WS * WSB;     // SS group scales
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sS + SS * 256);
-    uint64_t *wfull = bars, *wempty = wfull + WS;
-    uint64_t *xfull = wempty + WS, *xempty = xfull + XS;
+    uint8_t *sS = sX + XS * XB;      // SS group scales
+    uint8_t *sQ = sS + SS * 256;     // DW private rings of DEPTH slots
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sQ + (size_t)DW * DEPTH * SLOT);
+    uint64_t *xfull = bars, *xempty = xfull + XS;
     uint64_t *sfull = xempty + XS, *sempty = sfull + SS;
     uint64_t *afull = sempty + SS, *aempty = afull + AS;
     uint64_t *accfull = aempty + AS, *accempty = accfull + ACC;
@@ -165,10 +178,6 @@ __global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_con
     const int n = u1 - u0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < WS; ++s) {
-            mbar_init(&wfull[s], 1);
-            mbar_init(&wempty[s], DW);
-        }
         for (int s = 0; s < XS; ++s) {
             mbar_init(&xfull[s], 1);
             mbar_init(&xempty[s], 1);
@@ -206,19 +215,12 @@ __global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_con
     auto last_of_panel = [&](int i) { return i == n - 1 || panel_of(i + 1) != panel_of(i); };
 
     if (warp == 0) {
-        // ---------------- weight + scale producer ----------------
+        // ---------------- scale producer ----------------
         if (lane == 0) {
             const uint64_t pol = policy_evict_first();
             for (int i = 0; i < n; ++i) {
                 const size_t u = (size_t)(u0 + i);
-                const int ws = i % WS, ss = i % SS;
-                if (i >= WS && !mbar_wait(&wempty[ws], ((i / WS) - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                mbar_arrive_expect_tx(&wfull[ws], 8192 + 64);
-                bulk_g2s(sW + ws * WSB, p.wq + u * 8192, 8192, &wfull[ws], pol);
-                bulk_g2s(sW + ws * WSB + 8192, p.zeros + u * 64, 64, &wfull[ws], pol);
+                const int ss = i % SS;
                 if (i >= SS && !mbar_wait(&sempty[ss], ((i / SS) - 1) & 1)) {
                     ok = false;
                     break;
@@ -227,11 +229,16 @@ __global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_con
                 bulk_g2s(sS + ss * 256, p.scales + u * kPanelRows, 256, &sfull[ss], pol);
             }
         }
-    } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
+    } else if (warp == 1 || warp == 3) {
+        // ---------------- MMA issuers ----------------
+        // Two issuing threads, warp 1 for even units and warp 3 for odd ones:
+        // one thread's waits, descriptor arithmetic and commits cost more
+        // per unit than the eight small MMAs do on the tensor core.  Every
+        // unit has its own A stage and accumulator, so the two streams of
+        // MMAs are independent.
         if (lane == 0) {
             constexpr uint32_t idesc = umma_idesc_bf16(NT);
-            for (int i = 0; i < n; ++i) {
+            for (int i = warp == 1 ? 0 : 1; i < n; i += 2) {
                 const int as = i % AS, xs = i % XS, ac = i % ACC;
                 if (!mbar_wait(&afull[as], (i / AS) & 1) || !mbar_wait(&xfull[xs], (i / XS) & 1) ||
                     (i >= ACC && !mbar_wait(&accempty[ac], ((i / ACC) - 1) & 1))) {
@@ -239,12 +246,14 @@ __global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_con
                     break;
                 }
                 tc_fence_after();
-                const uint32_t xaddr = smem_u32(sX + xs * XB);
+                // the descriptor's start-address field is addr >> 4: step along
+                // K inside the swizzled tile by adding the byte offset >> 4
+                const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sX + xs * XB));
+                const uint32_t d_t = tmem + ac * NT, a_t = tmem + A0 + as * 64;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t bdesc = smem_desc_sw128(xaddr + (kk >> 2) * (NT * 128) + (kk & 3) * 32);
-                    umma_ts(tmem + ac * NT, tmem + A0 + as * 64 + kk * 8, bdesc, idesc, kk > 0 ? 1u : 0u);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(d_t, a_t + kk * 8, bdesc0 + (uint64_t)((((kk >> 2) * (NT * 128)) + (kk & 3) * 32) >> 4),
+                            idesc, kk > 0 ? 1u : 0u);
                 umma_commit(&aempty[as]);
                 umma_commit(&xempty[xs]);
                 umma_commit(&accfull[ac]);
@@ -327,13 +336,19 @@ __global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_con
             const float s = bf16_bits_to_float(reinterpret_cast<const uint16_t *>(sS + ss * 256)[r]);
             const uint32_t ta = tmem + tq + ac * NT + c * CW;
 #pragma unroll
-            for (int j0 = 0; j0 < CW; j0 += 16) { // 16 columns per load keeps the totals in registers
-                float v[16];
-                tmem_ld_32x32b_x16(ta + j0, v);
+            for (int j0 = 0; j0 < CW; j0 += 32) { // up to 32 columns per wait
+                float v[2][16];
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    if (j0 + 16 * h < CW)
+                        tmem_ld_32x32b_x16(ta + j0 + 16 * h, v[h]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    tot[j0 + j] = fmaf(s, v[j], tot[j0 + j]);
+                for (int h = 0; h < 2; ++h)
+                    if (j0 + 16 * h < CW)
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            tot[j0 + 16 * h + j] = fmaf(s, v[h][j], tot[j0 + 16 * h + j]);
             }
             tc_fence_before();
             __syncwarp();
@@ -357,33 +372,47 @@ __global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_con
 #pragma unroll
         for (int b = 0; b < BPW; ++b)
             jb[b] = BPW == 1 ? 2 * q + (d >> 2) : 2 * q + b;
-        for (int i = 0; i < n; ++i) {
-            const int ws = i % WS, as = i % AS;
-            if (!mbar_wait_warp(&wfull[ws], (i / WS) & 1)) {
-                ok = false;
-                break;
+        uint8_t *ring = sQ + (size_t)d * DEPTH * SLOT;
+        const int zseg = 16 * (jb[0] >> 1); // the 16-byte segment of a unit's zero points holding these rows
+        auto issue = [&](int i) {           // this warp's part of unit i into slot i % DEPTH
+            const uint8_t *src = p.wq + (size_t)(u0 + i) * 8192;
+            const uint32_t dst = smem_u32(ring + (i % DEPTH) * SLOT);
+#pragma unroll
+            for (int b = 0; b < BPW; ++b) {
+                cp_async_cg16(dst + b * 1024 + lane * 16, src + jb[b] * 1024 + lane * 16);
+                cp_async_cg16(dst + b * 1024 + 512 + lane * 16, src + jb[b] * 1024 + 512 + lane * 16);
             }
-            // Dequantize straight from the stage and release it only after
-            // every loaded value has been consumed: the producer refills a
-            // released stage at once, and a load still in flight could
-            // otherwise return the next block's bytes.
-            const uint8_t *blk = sW + ws * WSB;
+            if (lane == 0)
+                cp_async_cg16(dst + BPW * 1024, p.zeros + (size_t)(u0 + i) * 64 + zseg);
+        };
+#pragma unroll 1
+        for (int i = 0; i < DEPTH - 1; ++i) { // one commit group per unit, DEPTH - 1 ahead
+            if (i < n)
+                issue(i);
+            cp_async_commit();
+        }
+        for (int i = 0; i < n; ++i) {
+            const int as = i % AS;
+            __syncwarp(); // every lane has read the slot refilled next (the zero points are shared)
+            if (i + DEPTH - 1 < n)
+                issue(i + DEPTH - 1);
+            cp_async_commit();
+            cp_async_wait_group<DEPTH - 1>(); // unit i has landed (this lane's copies)
+            __syncwarp();                     // ... and lane 0's zero points
+            const uint8_t *blk = ring + (i % DEPTH) * SLOT;
             uint32_t rr[BPW][2][16];
 #pragma unroll
             for (int b = 0; b < BPW; ++b) {
-                const uint4 w0 = *reinterpret_cast<const uint4 *>(blk + jb[b] * 1024 + lane * 16);
-                const uint4 w1 = *reinterpret_cast<const uint4 *>(blk + jb[b] * 1024 + 512 + lane * 16);
-                const int r0 = 16 * jb[b] + g, r1 = r0 + 8;
-                const uint32_t z0 = (blk[8192 + (r0 >> 1)] >> (4 * (r0 & 1))) & 0xFu;
-                const uint32_t z1 = (blk[8192 + (r1 >> 1)] >> (4 * (r1 & 1))) & 0xFu;
+                const uint4 w0 = *reinterpret_cast<const uint4 *>(blk + b * 1024 + lane * 16);
+                const uint4 w1 = *reinterpret_cast<const uint4 *>(blk + b * 1024 + 512 + lane * 16);
+                const int zo = BPW * 1024 + 8 * (jb[b] & 1) + (g >> 1); // rows 16 jb + g and 16 jb + g + 8
+                const uint32_t z0 = (blk[zo] >> (4 * (g & 1))) & 0xFu;
+                const uint32_t z1 = (blk[zo + 4] >> (4 * (g & 1))) & 0xFu;
                 const uint32_t zlo = 0x43004300u | z0 | (z0 << 16); // bf16x2 {128 + z, 128 + z}
                 const uint32_t zhi = 0x43004300u | z1 | (z1 << 16);
                 int4_tile_regs(w0, zlo, zhi, rr[b][0]);
                 int4_tile_regs(w1, zlo, zhi, rr[b][1]);
             }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&wempty[ws]);
             if (i >= AS && !mbar_wait_warp(&aempty[as], ((i / AS) - 1) & 1)) {
                 ok = false;
                 break;
@@ -401,6 +430,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_con
             if (lane == 0)
                 mbar_arrive(&afull[as]);
         }
+        cp_async_wait_group<0>(); // no copy outlives the CTA (a timeout leaves the loop early)
     }
 
     if (!ok)

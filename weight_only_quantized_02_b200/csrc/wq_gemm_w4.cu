@@ -111,30 +111,48 @@ constexpr size_t gemm_w4_smem_bytes()
 
 // The last contributor to a split panel: sums the fp32 partials of CTAs
 // cf .. cl for its row r and tokens t0 .. t0 + CW - 1 in CTA order and
-// writes y.  Kept out of line: it runs once per split panel, and inlined its
-// registers would add to those of the retire loop's totals.
+// writes y.  The partials of up to five contributors are loaded together
+// (one round trip to L2 per 16 columns, not one per contributor: this runs
+// at the very end of the call, on the critical path).  Called after the
+// retire loop, whose register totals are dead by then.
 template <int NT, int CW>
-__device__ __noinline__ void w4_fixup(const GemmW4Params &p, long long U, int G, int pnl, int cf, int cl, int r,
+__device__ __forceinline__ void w4_fixup(const GemmW4Params &p, long long U, int G, int pnl, int cf, int cl, int r,
                                       int t0)
 {
     const int KB = p.KB;
     const int nrow = pnl * kPanelRows + r;
+    // contributors whose partials are in flight together (a panel usually has <= 5; fewer at NT = 128,
+    // where the retire warps already hold 64 totals and more would spill)
+    constexpr int CG = NT == 128 ? 2 : 5;
     for (int j0 = 0; j0 < CW; j0 += 16) {
         float acc[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             acc[j] = 0.f;
-        for (int cc = cf; cc <= cl; ++cc) {
-            const int sl = (pnl == sk_start(U, G, cc) / KB) ? 0 : 1;
-            const float *src = p.part + ((size_t)(cc * 2 + sl) * kPanelRows + r) * NT + t0 + j0;
+        for (int c0 = cf; c0 <= cl; c0 += CG) {
+            float4 v[CG][4];
 #pragma unroll
-            for (int j = 0; j < 16; j += 4) {
-                const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + j));
-                acc[j] += v.x;
-                acc[j + 1] += v.y;
-                acc[j + 2] += v.z;
-                acc[j + 3] += v.w;
+            for (int u = 0; u < CG; ++u) {
+                const int cc = c0 + u;
+                if (cc <= cl) {
+                    const int sl = (pnl == sk_start(U, G, cc) / KB) ? 0 : 1;
+                    const float4 *src =
+                        reinterpret_cast<const float4 *>(p.part + ((size_t)(cc * 2 + sl) * kPanelRows + r) * NT + t0 + j0);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        v[u][j] = __ldcg(src + j);
+                }
             }
+#pragma unroll
+            for (int u = 0; u < CG; ++u) // in CTA order
+                if (c0 + u <= cl)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        acc[4 * j] += v[u][j].x;
+                        acc[4 * j + 1] += v[u][j].y;
+                        acc[4 * j + 2] += v[u][j].z;
+                        acc[4 * j + 3] += v[u][j].w;
+                    }
         }
         if (nrow < p.N) {
             const int jn = min(16, p.M - t0 - j0);
@@ -286,6 +304,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_con
 #pragma unroll
         for (int j = 0; j < CW; ++j)
             tot[j] = 0.f;
+        int fix_pnl[2], fix_cf[2], fix_cl[2], nfix = 0; // split panels this warp finishes (a range touches <= 2 panels)
 
         // This thread's CW totals of panel pnl: to y when this CTA covered
         // the whole panel, else as a partial + per-warp ticket.
@@ -320,10 +339,11 @@ __global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_con
             const int cf = sk_owner(U, G, pnl * KB), cl = sk_owner(U, G, (pnl + 1) * KB - 1);
             if (ticket != (uint32_t)(cl - cf))
                 return;
-            __syncwarp(); // lane 0's acquire orders every lane's reads below
-            w4_fixup<NT, CW>(p, U, G, pnl, cf, cl, r, t0);
-            if (lane == 0)
-                atomicExch(&p.cnt[pnl * 8 + dw], 0u); // ready for the next call
+            // the last contributor: sum the partials once the loop is done
+            fix_pnl[nfix] = pnl;
+            fix_cf[nfix] = cf;
+            fix_cl[nfix] = cl;
+            ++nfix;
         };
 
         for (int i = 0; i < n; ++i) {
@@ -362,6 +382,12 @@ __global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_con
                 for (int j = 0; j < CW; ++j)
                     tot[j] = 0.f;
             }
+        }
+        __syncwarp(); // lane 0's acquire (the tickets) orders every lane's reads below
+        for (int f = 0; f < nfix && ok; ++f) {
+            w4_fixup<NT, CW>(p, U, G, fix_pnl[f], fix_cf[f], fix_cl[f], r, c * CW);
+            if (lane == 0)
+                atomicExch(&p.cnt[fix_pnl[f] * 8 + dw], 0u); // ready for the next call
         }
     } else if (warp >= 4 + RW) {
         // ---------------- dequant warps ----------------

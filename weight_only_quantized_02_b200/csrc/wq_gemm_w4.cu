@@ -73,8 +73,8 @@ template <int NT>
 struct W4Cfg {
     static constexpr int kXB = NT * 256;                 // x tile: NT rows x 128 k bf16
     static constexpr int kSS = 32;                       // scale stages (256 B each)
-    static constexpr int kXS = NT == 16 ? 8 : NT == 32 ? 6 : NT == 64 ? 4 : 3;
-    static constexpr int kDepth = NT <= 32 ? 16 : NT == 64 ? 14 : 12; // units in each dequant warp's ring
+    static constexpr int kXS = NT == 16 ? 8 : NT == 32 ? 6 : 4;
+    static constexpr int kDepth = NT <= 32 ? 16 : NT == 64 ? 14 : 10; // units in each dequant warp's ring
     static constexpr int kACC = NT <= 32 ? 128 / NT : 256 / NT; // group accumulators
     static constexpr int kA0 = kACC * NT;                // first A column
     static constexpr int kAS = (512 - kA0) / 64;         // A stages, 64 columns each
@@ -87,6 +87,10 @@ struct W4Cfg {
     static_assert(kAS >= 2 && kACC >= 2, "double buffering");
     static_assert(kDW == 4 || kDW == 8, "dequant warps cover the four lane quadrants evenly");
     static_assert(kCW % 16 == 0, "retire loads 16 columns at a time");
+    // The two MMA issuers take alternate units, so a stage of every ring they
+    // wait on must come back to the same issuer: with an odd ring an issuer
+    // could test a barrier two phases ahead, where the parity wait passes.
+    static_assert(kXS % 2 == 0 && kAS % 2 == 0 && kACC % 2 == 0, "rings the MMA issuers wait on are even");
 };
 
 // 16-byte asynchronous global -> shared copy (L2 only) and its groups.

@@ -291,6 +291,17 @@ int wq_dequant_debug(const void *Wq, const void *scales, const void *zeros, int 
  * `stream`. */
 int wq_device_error(cudaStream_t stream);
 
+/* Failure detection under test. Enqueues one small kernel whose thread
+ * waits, through the same bounded wait every kernel uses (an mbarrier
+ * try_wait loop against %globaltimer), on an mbarrier that nothing
+ * completes, with the limit shortened to limit_us microseconds (1 ..
+ * 2000000; the kernels use 2 s). The wait gives up, the kernel records
+ * WQ_ERR_TIMEOUT in the device error word and returns: no trap, no fault,
+ * the context stays usable. A following wq_device_error returns
+ * WQ_ERR_TIMEOUT (and clears it). Returns WQ_ERR_SHAPE for a limit out of
+ * range, WQ_ERR_CUDA if the launch fails. */
+int wq_wait_selftest(int limit_us, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -10,6 +10,8 @@ power-of-two scaling) are compared bit for bit.
 """
 import os
 
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -379,3 +381,20 @@ def test_tuner_and_table_roundtrip(weight, ws, tmp_path):
     wq.wq_set_choice(M, K, N, bits, 0 if bits == 8 else 128, GEMV_RB, 8)
     assert wq.wq_get_choice(M, K, N, bits, 0 if bits == 8 else 128) == (GEMV_RB, 8)
     wq.wq_clear_tuning()
+
+
+@pytest.mark.gpu
+def test_bounded_wait_runs_out_and_reports():
+    """Failure detection: a bounded wait on an mbarrier that nothing completes
+    gives up, the kernel records a timeout and returns; the host reads it as
+    WQ_ERR_TIMEOUT, the error word is cleared, and the context stays usable."""
+    assert wq.wq_device_error() == 0
+    t0 = time.perf_counter()
+    wq.wq_wait_selftest(50000)  # 50 ms
+    assert wq.wq_device_error() == -9  # WQ_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    assert wq.wq_device_error() == 0  # read and cleared
+    # the context still runs work
+    z = torch.ones(1024, device=dev())
+    assert float(z.sum()) == 1024.0
+    assert wq.lib.wq_wait_selftest(0, None) == -2  # limit out of range

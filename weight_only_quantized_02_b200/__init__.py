@@ -76,6 +76,7 @@ def _load():
         "wq_unpack_debug": (I, [P, P, I, I, I, I, P, P, P]),
         "wq_dequant_debug": (I, [P, P, P, I, I, I, I, P, P]),
         "wq_device_error": (I, [P]),
+        "wq_wait_selftest": (I, [I, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -321,3 +322,10 @@ def wq_dequant_debug(pw: PackedWeight, stream=None) -> torch.Tensor:
 
 def wq_device_error(stream=None) -> int:
     return int(lib.wq_device_error(_s(stream)))
+
+
+def wq_wait_selftest(limit_us: int = 50000, stream=None) -> None:
+    """Enqueues a kernel whose bounded wait runs out after limit_us (nothing
+    completes its mbarrier); it records WQ_ERR_TIMEOUT in the device error
+    word, which wq_device_error then reports."""
+    _check(lib.wq_wait_selftest(int(limit_us), _s(stream)), "wq_wait_selftest")

@@ -737,6 +737,17 @@ int wq_dequant_debug(const void *Wq, const void *scales, const void *zeros, int 
     return cuda_status(launch_dequant_debug(Wq, scales, zeros, Shape{bits, K, N, group}, w_out, stream));
 }
 
+int wq_wait_selftest(int limit_us, cudaStream_t stream)
+{
+    if (limit_us < 1 || limit_us > 2000000)
+        return WQ_ERR_SHAPE;
+    DeviceInfo d;
+    int st = current_device_info(&d);
+    if (st != WQ_OK)
+        return st;
+    return cuda_status(launch_wait_selftest((uint64_t)limit_us * 1000u, stream));
+}
+
 int wq_device_error(cudaStream_t stream)
 {
     int a = 0, b = 0, c = 0, e = 0, f = 0, h = 0;

@@ -85,7 +85,7 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t pa
     return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -93,9 +93,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
     for (;;) {
         if (mbar_try_wait_suspend(bar, parity, 1000000u)) // suspended for up to 1 ms per try
             return true;
-        if (globaltimer_ns() - t0 > kWaitLimitNs)
+        if (globaltimer_ns() - t0 > limit_ns)
             return false;
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+{
+    return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
 // Warp-uniform form for warps that go on to execute .sync.aligned

@@ -446,6 +446,28 @@ cudaError_t launch_gemm(const LinearArgs &a, int split, void *ws, int sm_count, 
     }
 }
 
+// One thread waits, through the kernels' bounded wait, on an mbarrier that
+// nothing arrives on: the wait gives up after limit_ns, the timeout is
+// recorded in the device error word exactly as a kernel records it, and the
+// kernel returns.  Failure detection under test, without a fault or a hang.
+__global__ void wait_selftest_kernel(uint64_t limit_ns)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait_for(&bar, 0, limit_ns))
+        atomicExch(&g_gemm_error, kErrTimeout);
+}
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t st)
+{
+    wait_selftest_kernel<<<1, 32, 0, st>>>(limit_ns);
+    return cudaGetLastError();
+}
+
 cudaError_t read_device_error(int *code, cudaStream_t st)
 {
     int host = 0, zero = 0;

@@ -114,4 +114,7 @@ cudaError_t launch_gemv_i8(const LinearArgs &a, int split, void *ws, int sm_coun
 // Reads and clears the device error word of the current device.
 cudaError_t read_device_error(int *code, cudaStream_t st);
 
+// A bounded wait that runs out (limit_ns) and records the timeout.
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t st);
+
 } // namespace wq

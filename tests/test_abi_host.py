@@ -108,12 +108,24 @@ def test_tuning_file_parse_errors(tmp_path):
         "NVIDIA B200|148 9 5120 17408 8 0 5 1 9.0\n",       # integer GEMV: M <= 8
         "NVIDIA B200|148 8 65536 17408 8 0 5 1 9.0\n",      # integer GEMV: digit rows over 200 KB
         "NVIDIA B200|148 4 5120 17408 4 128 5 3 9.0\n",     # integer GEMV: split 1 or 2
+        "NVIDIA B200|148 16 17408 5120 8 0 6 1 9.0\n",      # role-split GEMM: W4A16 only
+        "NVIDIA B200|148 16 17408 5120 4 128 6 2 9.0\n",    # role-split GEMM: split 1 only
     ]:
         p = tmp_path / "bad.txt"
         p.write_text(bad_line)
         assert wq.wq_load_tuning(str(p)) == -8, bad_line
     assert wq.wq_load_tuning(str(tmp_path / "missing.txt")) == -8
     assert wq.lib.wq_load_tuning(None) == -1
+
+
+def test_shipped_tuning_table_loads():
+    """The measured B200 table that ships with the package parses and holds
+    only valid (variant, split) choices."""
+    path = os.path.join(os.path.dirname(wq.__file__), "tuning_b200.txt")
+    assert wq.wq_load_tuning(path) == 0
+    entries = [l for l in open(path) if "|" in l and not l.startswith("#")]
+    assert len(entries) >= 14
+    wq.wq_clear_tuning()
 
 
 def test_no_oracle_in_product():

@@ -35,10 +35,12 @@
  *     W4A16 the zero point enters through the activations' digit sum per
  *     group and the group scale is applied in fp32 per group.
  * A per-(M,K,N,bits,group) dispatcher picks the kernel and split factor. It
- * starts from an untuned rule (W8A16 within the integer path's limits -> the
- * integer path; otherwise the pages' rule: fewer than 8 tokens -> GEMV, else
- * GEMM with split 8; same page) and is overridden by measured timings
- * (wq_tune), whose candidates include the integer path for W4A16 too.
+ * starts from an untuned rule (the page's threshold: fewer than 8 tokens ->
+ * a GEMV, else a GEMM; within each, the kernel measured fastest on B200 where
+ * the workspace allows it: the integer GEMV; the integer tensor-core GEMM for
+ * W8A16 up to 64 tokens, the role-split GEMM for W4A16; else the stream-K or
+ * row-block GEMV and the split-8 GEMM) and is overridden by measured timings
+ * (wq_tune).
  *
  * Conventions for every entry point:
  *   - The return value is a wq_status: 0 on success, negative on error.

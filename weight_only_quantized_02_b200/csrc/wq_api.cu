@@ -148,20 +148,27 @@ int default_rb_slices(int K, int N, int sm_count)
     return ks;
 }
 
-// Untuned rule.  W8A16 runs on the integer tensor cores whenever the shape
-// and the workspace allow it (W4A16 there is a tuning candidate only).  Otherwise the pages' rule: fewer than 8
-// tokens -> GEMV, else the GEMM with split_k = 8 (Mit han lab Llm awq Kernel
-// Selection Thresholds, The Insight).  The stream-K GEMV needs the split-K
-// workspace; without one the row-block GEMV is used.
-Choice default_choice(int M, int K, int N, int bits, int sm_count, bool have_ws = true, bool have_i8_ws = true)
+// Untuned rule: the pages' threshold, fewer than 8 tokens -> a GEMV, else a
+// GEMM (Mit han lab Llm awq Kernel Selection Thresholds, The Insight), and
+// within each the kernel that measured fastest on B200 across the five
+// workloads, workspace permitting: the integer GEMV; the integer
+// tensor-core GEMM for W8A16 (M <= 64); the role-split GEMM for W4A16.
+// Without a workspace: the row-block GEMV, else the pages' split_k = 8 GEMM
+// (run unsplit when no workspace holds its partials).
+Choice default_choice(int M, int K, int N, int bits, int sm_count, bool have_ws = true, bool have_i8_ws = true,
+                      bool have_gi_ws = true, bool have_w4_ws = true)
 {
-    if (bits == 8 && i8_fits(bits, M, K) && have_i8_ws)
-        return {WQ_VARIANT_I8MMA, 1, 0.f};
     if (M < 8) {
+        if (gi_fits(bits, M, K) && have_gi_ws)
+            return {WQ_VARIANT_GEMV_I8, 1, 0.f};
         if (have_ws)
             return {WQ_VARIANT_GEMV, 3, 0.f};
         return {WQ_VARIANT_GEMV_RB, default_rb_slices(K, N, sm_count), 0.f};
     }
+    if (bits == 8 && i8_fits(bits, M, K) && have_i8_ws)
+        return {WQ_VARIANT_I8MMA, 1, 0.f};
+    if (bits == 4 && have_w4_ws)
+        return {WQ_VARIANT_GEMM_W4, 1, 0.f};
     return {WQ_VARIANT_GEMM, std::min(8, max_gemm_split(K)), 0.f};
 }
 
@@ -237,9 +244,10 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
     if (split > 0)
         c.split = split;
     if (variant == WQ_VARIANT_AUTO) {
+        const bool w4_ws_ok = w && have >= ws_bytes_gemm_sk(M, N);
         if (!choice_valid(c.variant, c.split, M, K, bits) || (c.variant == WQ_VARIANT_I8MMA && !i8_ws_ok) ||
-            (c.variant == WQ_VARIANT_GEMV_I8 && !gi_ws_ok))
-            c = default_choice(M, K, N, bits, d.sm_count, sk_ws_ok, i8_ws_ok);
+            (c.variant == WQ_VARIANT_GEMV_I8 && !gi_ws_ok) || (c.variant == WQ_VARIANT_GEMM_W4 && !w4_ws_ok))
+            c = default_choice(M, K, N, bits, d.sm_count, sk_ws_ok, i8_ws_ok, gi_ws_ok, w4_ws_ok);
         if (c.variant == WQ_VARIANT_GEMV && !sk_ws_ok)
             c = {WQ_VARIANT_GEMV_RB, default_rb_slices(K, N, d.sm_count), 0.f};
         // an automatic choice never fails for lack of workspace: split-K GEMM

@@ -24,14 +24,18 @@
 // the packed mma tiles, see gi_digits), so a lane's B fragment is one
 // contiguous load.
 //
-// Work split: warp-level stream-K.  The items (16-row block, 128-k block),
-// row-block-major, are cut into G*8 equal contiguous ranges, one per warp;
-// each warp streams its range through a D-deep ring of register prefetches
-// (the first D issued before the programmatic-launch wait: weights never
-// depend on the preceding kernel).  A row block whose k range is split
-// between warps is finished by the last contributor to take the block's
-// ticket (acquire-release, never waited on): it sums the partials in warp
-// order and writes y (INT8 partials are exact integers).
+// Work split: each CTA owns LB = (N/16) / G whole 16-row blocks, split in
+// equal contiguous runs of chunks (D k-blocks of one row block) between
+// most of its warps; the remaining row blocks' chunks are cut stream-K
+// style between the CTAs, and each CTA's share between its first few warps
+// (see gi_cta).  Each warp streams its run through a D-deep ring of
+// register prefetches (the first D issued before the programmatic-launch
+// wait: weights never depend on the preceding kernel).  A CTA's own row
+// block split between its warps is summed from shared memory once all of
+// them are done: no round trip to L2 at the end of the stream.  A shared
+// row block is finished by the last contributor to take its ticket
+// (acquire-release, never waited on), which sums the partials in
+// contributor order and writes y (INT8 partials are exact integers).
 #include <cstdint>
 
 #include <cuda_bf16.h>
@@ -49,7 +53,9 @@ struct GiParams {
     const uint16_t *x;
     int M, K, N, KB;
     int CPR;        // chunks (D consecutive k-blocks, the last one ragged) per 16-row block
-    int I;          // chunks = (N / 16) * CPR
+    int LB;         // 16-row blocks each CTA owns whole: CTA c has c LB .. c LB + LB - 1
+    int RB0;        // G LB: row blocks RB0 .. N/16 - 1 are shared between CTAs
+    int RL;         // chunks of the shared row blocks, (N/16 - RB0) CPR
     const uint8_t *wq;
     const uint16_t *scales;
     const uint8_t *zeros;
@@ -177,109 +183,217 @@ __device__ __forceinline__ void gi_digits(const GiParams &p, uint8_t *sd, int32_
     __syncthreads();
 }
 
-// End of a warp's segment of row block rb: the accumulators are in red
-// ([16 rows][NR]; INT8 int32 digit sums D_i, INT4 fp32 group-scaled sums
-// A_i).  Writes y, or the warp's partial and its ticket; the last arriver
-// sums all partials in warp order and writes y.
-template <int BITS, int NR>
-__device__ __forceinline__ void gi_flush(const GiParams &p, int rb, bool whole, int slot, int w, int Wt,
-                                      uint32_t *red, const int *s_e, int lane)
+// Stream-K cuts in 32-bit arithmetic (every U * c and u * G here stays far
+// below 2^32; the launch checks the bound): range c of G over U units
+// starts at U c / G; gi_owner is the range holding unit u.
+__device__ __forceinline__ int gi_start(int U, int G, int c) { return (int)((unsigned)U * (unsigned)c / (unsigned)G); }
+
+__device__ __forceinline__ int gi_owner(int U, int G, int u)
 {
-    const int M = p.M, N = p.N;
-    const int n0 = 16 * rb;
-    __syncwarp();
-    if constexpr (BITS == 8) {
-        if (whole) {
-            for (int q = lane; q < 16 * M; q += 32) {
-                const int r = q & 15, m = q >> 4;
-                const int32_t *d = reinterpret_cast<const int32_t *>(red) + r * NR + 3 * m;
-                const double sc = (double)bf16_bits_to_float(p.scales[n0 + r]) * pow2_of(-s_e[m]);
-                p.y[(size_t)m * N + n0 + r] = i8_output(d[0], d[1], d[2], sc);
-            }
-            __syncwarp();
-            return;
+    int c = (int)((unsigned)u * (unsigned)G / (unsigned)U);
+    c = c < G - 1 ? c : G - 1;
+    while (c + 1 < G && gi_start(U, G, c + 1) <= u)
+        ++c;
+    while (c > 0 && gi_start(U, G, c) > u)
+        --c;
+    return c;
+}
+
+// CTA c's work: its stream-K share [lo, lo + L) of the RL chunks of the
+// shared row blocks, taken by its first ws warps, and its LB own row blocks
+// (own = LB CPR chunks), split between the other WARPS - ws warps.  A shared
+// warp gets about 0.8 of an even share: its tickets and fix-ups (round trips
+// to L2) take the rest of its time.  With no own row blocks every warp is a
+// shared warp.
+struct GiCta {
+    int lo, L, ws;
+};
+
+__device__ __forceinline__ GiCta gi_cta(const GiParams &p, int G, int c, int warps)
+{
+    GiCta t;
+    t.lo = gi_start(p.RL, G, c);
+    t.L = gi_start(p.RL, G, c + 1) - t.lo;
+    const int own = p.LB * p.CPR;
+    if (t.L == 0) {
+        t.ws = 0;
+    } else if (own == 0) {
+        t.ws = warps;
+    } else {
+        const int ws = (5 * t.L * warps + 4 * (t.L + own) - 1) / (4 * (t.L + own)); // ceil(1.25 L warps / total)
+        t.ws = ws < 1 ? 1 : ws > warps / 2 ? warps / 2 : ws;
+    }
+    return t;
+}
+
+// One segment's output, its accumulators in red ([16 rows][NR]; INT8 int32
+// digit sums D_i, INT4 fp32 group-scaled sums A_i): y of the 16 x M outputs.
+template <int BITS, int NR>
+__device__ __forceinline__ void gi_write_y(const GiParams &p, int rb, const uint32_t *red, const int *s_e, int lane)
+{
+    const int M = p.M, N = p.N, n0 = 16 * rb;
+    for (int q = lane; q < 16 * M; q += 32) {
+        const int r = q & 15, m = q >> 4;
+        if constexpr (BITS == 8) {
+            const int32_t *d = reinterpret_cast<const int32_t *>(red) + r * NR + 3 * m;
+            const double sc = (double)bf16_bits_to_float(p.scales[n0 + r]) * pow2_of(-s_e[m]);
+            p.y[(size_t)m * N + n0 + r] = i8_output(d[0], d[1], d[2], sc);
+        } else {
+            const float *a = reinterpret_cast<const float *>(red) + r * NR + 3 * m;
+            const double v = ((double)a[2] * 65536.0 + (double)a[1] * 256.0 + (double)a[0]) * pow2_of(-s_e[m]);
+            p.y[(size_t)m * N + n0 + r] = __bfloat16_as_ushort(__double2bfloat16(v));
         }
-        uint32_t *mine = p.part + ((size_t)w * 2 + slot) * 16 * NR;
+    }
+}
+
+// A partial segment of shared row block rb ended: the warp's partial into
+// its slot, then its ticket (acquire-release), returned.
+template <int BITS, int NR>
+__device__ __forceinline__ uint32_t gi_shared_partial(const GiParams &p, int rb, int slot, int w, const uint32_t *red,
+                                                      const int *s_e, int lane)
+{
+    const int M = p.M;
+    __syncwarp();
+    uint32_t *mine = p.part + ((size_t)w * 2 + slot) * 16 * NR;
+    if constexpr (BITS == 8) {
         for (int i = lane; i < 16 * NR; i += 32)
             mine[i] = red[i];
     } else {
-        uint32_t *mine = p.part + ((size_t)w * 2 + slot) * 16 * NR;
         for (int q = lane; q < 16 * M; q += 32) {
             const int r = q & 15, m = q >> 4;
             const float *a = reinterpret_cast<const float *>(red) + r * NR + 3 * m;
             const double v = ((double)a[2] * 65536.0 + (double)a[1] * 256.0 + (double)a[0]) * pow2_of(-s_e[m]);
-            if (whole)
-                p.y[(size_t)m * N + n0 + r] = __bfloat16_as_ushort(__double2bfloat16(v));
-            else
-                mine[r * NR + m] = __float_as_uint((float)v);
-        }
-        if (whole) {
-            __syncwarp();
-            return;
+            mine[r * NR + m] = __float_as_uint((float)v);
         }
     }
     __syncwarp();
     uint32_t ticket = 0;
     if (lane == 0)
         ticket = ticket_take_acq_rel(&p.cnt[rb]);
-    ticket = __shfl_sync(0xffffffffu, ticket, 0);
-    const int CPR = p.CPR;
-    const int wf = sk_owner(p.I, Wt, rb * CPR), wl = sk_owner(p.I, Wt, rb * CPR + CPR - 1);
-    if (ticket == (uint32_t)(wl - wf)) {
-        __syncwarp(); // lane 0's acquire orders every lane's reads below
-        // the partials of up to four contributors are loaded together (one
-        // round trip to L2 instead of one per contributor), then summed in
-        // warp order
-        auto src_of = [&](int ww) {
-            const int sl = (sk_start(p.I, Wt, ww) / CPR == rb) ? 0 : 1;
-            return p.part + ((size_t)ww * 2 + sl) * 16 * NR;
-        };
-        for (int q = lane; q < 16 * M; q += 32) {
-            const int r = q & 15, m = q >> 4;
-            if constexpr (BITS == 8) {
-                int32_t t0 = 0, t1 = 0, t2 = 0;
-                for (int w0 = wf; w0 <= wl; w0 += 4) {
-                    int32_t v[4][3];
+    return __shfl_sync(0xffffffffu, ticket, 0);
+}
+
+// After the warp's last chunk, for each shared row block it took a ticket
+// of: the contributors are listed (one lane per chunk of the row block
+// marks where a contributor's run starts: the row block's first chunk, a
+// CTA's share or a warp's run), and the last contributor sums their
+// partials in order (up to four loaded per round trip to L2) and writes y.
+// Its ticket's acquire (taken earlier in program order) orders the reads.
+// list: this warp's scratch of at least CPR words (partial offsets).
+template <int BITS, int NT, int WARPS>
+__device__ __forceinline__ void gi_shared_fixup(const GiParams &p, int rb, uint32_t ticket, int G, const int *s_e,
+                                                uint32_t *list, int lane)
+{
+    constexpr int NR = 8 * NT;
+    const int M = p.M, N = p.N, n0 = 16 * rb, CPR = p.CPR;
+    const int u0 = (rb - p.RB0) * CPR;
+    int nc = 0;
+    for (int base = 0; base < CPR; base += 32) {
+        const int i = base + lane;
+        bool start = false;
+        uint32_t off = 0;
+        if (i < CPR) {
+            const int u = u0 + i, cc = gi_owner(p.RL, G, u);
+            const GiCta t = gi_cta(p, G, cc, WARPS);
+            const int o = u - t.lo, wi = gi_owner(t.L, t.ws, o), s0 = gi_start(t.L, t.ws, wi);
+            start = i == 0 || o == s0;
+            const int sl = p.RB0 + (t.lo + s0) / CPR == rb ? 0 : 1; // rb is the warp's first row block?
+            off = ((uint32_t)(cc * WARPS + wi) * 2 + sl) * 16 * NR;
+        }
+        const uint32_t mask = __ballot_sync(0xffffffffu, start);
+        if (start)
+            list[nc + __popc(mask & ((1u << lane) - 1u))] = off;
+        nc += __popc(mask);
+    }
+    __syncwarp();
+    if (ticket != (uint32_t)(nc - 1))
+        return;
+    for (int q = lane; q < 16 * M; q += 32) {
+        const int r = q & 15, m = q >> 4;
+        if constexpr (BITS == 8) {
+            int32_t t0 = 0, t1 = 0, t2 = 0;
+            for (int k0 = 0; k0 < nc; k0 += 4) {
+                int32_t v[4][3];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        v[u][0] = v[u][1] = v[u][2] = 0;
-                        if (w0 + u <= wl) {
-                            const int32_t *src = reinterpret_cast<const int32_t *>(src_of(w0 + u)) + r * NR + 3 * m;
-                            v[u][0] = __ldcg(src);
-                            v[u][1] = __ldcg(src + 1);
-                            v[u][2] = __ldcg(src + 2);
-                        }
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        t0 += v[u][0];
-                        t1 += v[u][1];
-                        t2 += v[u][2];
+                for (int u = 0; u < 4; ++u) {
+                    v[u][0] = v[u][1] = v[u][2] = 0;
+                    if (k0 + u < nc) {
+                        const int32_t *src = reinterpret_cast<const int32_t *>(p.part + list[k0 + u]) + r * NR + 3 * m;
+                        v[u][0] = __ldcg(src);
+                        v[u][1] = __ldcg(src + 1);
+                        v[u][2] = __ldcg(src + 2);
                     }
                 }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    t0 += v[u][0];
+                    t1 += v[u][1];
+                    t2 += v[u][2];
+                }
+            }
+            const double sc = (double)bf16_bits_to_float(p.scales[n0 + r]) * pow2_of(-s_e[m]);
+            p.y[(size_t)m * N + n0 + r] = i8_output(t0, t1, t2, sc);
+        } else {
+            float tot = 0.f;
+            for (int k0 = 0; k0 < nc; k0 += 4) {
+                float v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    v[u] = k0 + u < nc ? __ldcg(reinterpret_cast<const float *>(p.part + list[k0 + u]) + r * NR + m)
+                                       : 0.f;
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (k0 + u < nc)
+                        tot += v[u];
+            }
+            p.y[(size_t)m * N + n0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(tot));
+        }
+    }
+    __syncwarp();
+    if (lane == 0)
+        atomicExch(&p.cnt[rb], 0u); // ready for the next call
+}
+
+// After every warp of the CTA has streamed its share: the CTA's own row
+// blocks that were split between its warps, summed from the stash in warp
+// order (INT8: exact integers; INT4: each contributor's value in binary64,
+// summed in binary64) and written to y.
+template <int BITS, int NT, int WARPS>
+__device__ __forceinline__ void gi_local_out(const GiParams &p, const GiCta &ct, int c, const uint32_t *stash,
+                                             const int *s_e, int warp, int lane)
+{
+    constexpr int NR = 8 * NT;
+    const int M = p.M, N = p.N, CPR = p.CPR;
+    const int own = p.LB * CPR, wo = WARPS - ct.ws; // own chunks and the warps that take them
+    for (int j = warp; j < p.LB; j += WARPS) {
+        const int wf = ct.ws + gi_owner(own, wo, j * CPR), wl = ct.ws + gi_owner(own, wo, j * CPR + CPR - 1);
+        if (wf == wl)
+            continue; // one warp had it whole and wrote y
+        const int n0 = 16 * (c * p.LB + j);
+        for (int q = lane; q < 16 * M; q += 32) {
+            const int r = q & 15, m = q >> 4;
+            int32_t t0 = 0, t1 = 0, t2 = 0;
+            double v = 0.0;
+            for (int wi = wf; wi <= wl; ++wi) {
+                const int sl = gi_start(own, wo, wi - ct.ws) / CPR == j ? 0 : 1; // j is the warp's first row block?
+                const uint32_t *a = stash + ((size_t)wi * 2 + sl) * 16 * NR + r * NR + 3 * m;
+                if constexpr (BITS == 8) {
+                    t0 += (int32_t)a[0];
+                    t1 += (int32_t)a[1];
+                    t2 += (int32_t)a[2];
+                } else {
+                    v += (double)__uint_as_float(a[2]) * 65536.0 + (double)__uint_as_float(a[1]) * 256.0 +
+                         (double)__uint_as_float(a[0]);
+                }
+            }
+            if constexpr (BITS == 8) {
                 const double sc = (double)bf16_bits_to_float(p.scales[n0 + r]) * pow2_of(-s_e[m]);
                 p.y[(size_t)m * N + n0 + r] = i8_output(t0, t1, t2, sc);
             } else {
-                float tot = 0.f;
-                for (int w0 = wf; w0 <= wl; w0 += 4) {
-                    float v[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        v[u] = w0 + u <= wl
-                                   ? __ldcg(reinterpret_cast<const float *>(src_of(w0 + u)) + r * NR + m)
-                                   : 0.f;
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        if (w0 + u <= wl)
-                            tot += v[u];
-                }
-                p.y[(size_t)m * N + n0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(tot));
+                p.y[(size_t)m * N + n0 + r] = __bfloat16_as_ushort(__double2bfloat16(v * pow2_of(-s_e[m])));
             }
         }
-        if (lane == 0)
-            atomicExch(&p.cnt[rb], 0u); // ready for the next call
     }
-    __syncwarp();
 }
 
 // WARPS = 16: one CTA per SM (the digit rows made once per SM); WARPS = 8:
@@ -290,23 +404,39 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
     constexpr int NR = 8 * NT;
     constexpr int D = GiCfg<BITS>::D;
     constexpr int WV = BITS == 8 ? 4 : 2; // 16-byte weight loads per lane and item
-    extern __shared__ __align__(16) uint8_t sd[]; // digit rows [3M][S], then (INT4) digit sums [KB][NR]
+    // dynamic: digit rows [3M][S], (INT4) digit sums [KB][NR], then the
+    // stash [WARPS][2][16 rows][NR] of partial sums of the CTA's own row blocks
+    extern __shared__ __align__(16) uint8_t sd[];
     __shared__ uint32_t s_amax[kGiMaxM];
     __shared__ int s_e[kGiMaxM];
-    __shared__ uint32_t s_red[WARPS][16 * NR];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int G = gridDim.x, c = blockIdx.x;
-    const int Wt = G * WARPS, w = c * WARPS + warp;
+    const int w = c * WARPS + warp;
     const int KB = p.KB, M = p.M;
     const int S = gi_row_stride<BITS>(p.K);
     int32_t *s_dsum = reinterpret_cast<int32_t *>(sd + 3 * M * S);
-    const int i0 = sk_start(p.I, Wt, w), i1 = sk_start(p.I, Wt, w + 1);
-    const int n = i1 - i0;
+    uint32_t *stash = reinterpret_cast<uint32_t *>(sd + 3 * M * S + (BITS == 4 ? KB * NR * 4 : 0));
+    uint32_t *st0 = stash + (size_t)warp * 2 * 16 * NR, *st1 = st0 + 16 * NR;
+    const GiCta ct = gi_cta(p, G, c, WARPS);
+    const bool shared_warp = warp < ct.ws;
+    // the warp's run of chunks: n chunks from chunk q0 of row block rb0
+    int rb0, q0, n;
+    if (shared_warp) {
+        const int o0 = gi_start(ct.L, ct.ws, warp);
+        n = gi_start(ct.L, ct.ws, warp + 1) - o0;
+        rb0 = p.RB0 + (ct.lo + o0) / p.CPR;
+        q0 = (ct.lo + o0) % p.CPR;
+    } else {
+        const int own = p.LB * p.CPR, o0 = gi_start(own, WARPS - ct.ws, warp - ct.ws);
+        n = gi_start(own, WARPS - ct.ws, warp - ct.ws + 1) - o0;
+        rb0 = c * p.LB + o0 / p.CPR;
+        q0 = o0 % p.CPR;
+    }
 
     // ---------------- weights of the first chunk (before the launch wait) ----------------
-    // The warp's work is chunks [i0, i1): chunk (rb, q) = k-blocks D q ..
-    // D q + D - 1 (those below KB) of 16-row block rb.  Ring slot s holds
+    // The warp's work is n consecutive chunks from (rb0, q0): chunk (rb, q) =
+    // k-blocks D q .. D q + D - 1 (those below KB) of 16-row block rb.  Ring slot s holds
     // k-block D q + s of a chunk: consuming a slot is followed by loading
     // the same slot of the next chunk, so D k-blocks stay in flight.
     // Loader state: the next chunk to load is (lrb, lq); lw points at its
@@ -319,7 +449,7 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
     uint4 wb[D][WV];
     uint32_t sz[D][2]; // INT4: bf16 scales of rows g, g+8 | their zero-point bytes
     const int oa = (g << 7) + ((t ^ g) << 4), ob = (g << 7) + (((t + 4) ^ g) << 4); // INT8 chunks t, t+4
-    int lrb = n > 0 ? i0 / CPR : 0, lq = n > 0 ? i0 % CPR : 0;
+    int lrb = rb0, lq = q0;
     const uint8_t *lw = nullptr;
     const uint16_t *ls = nullptr;
     const uint8_t *lz = nullptr;
@@ -393,7 +523,6 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
         xrow[nt] = sd + (xon[nt] ? (8 * nt + g) * S : 0) + (BITS == 8 ? 16 * t : 32 * t);
     }
     const int zsh = 4 * (g & 1);
-    uint32_t *red = s_red[warp];
 
     // k-block xo (byte offset 128 * kb in a digit row) of ring slot s
     auto consume = [&](int s, int xo) {
@@ -452,7 +581,9 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
         }
     };
 
-    int crb = rb_first, cq = n > 0 ? i0 % CPR : 0;
+    int crb = rb0, cq = q0; // the chunk being consumed
+    int npend = 0, pend_rb0 = 0, pend_rb1 = 0; // shared row blocks with a ticket taken
+    uint32_t pend_t0 = 0, pend_t1 = 0;
     bool seg_whole = cq == 0; // the current segment started at the row block's first chunk
     for (int ch = 0; ch < n; ++ch) {
         const int kb0 = D * cq, xo = kb0 * 128;
@@ -475,6 +606,11 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
         if (more)
             next_chunk();
         if (cq == CPR - 1 || !more) { // end of a segment: the row block's last chunk or the warp's last
+            const bool whole = seg_whole && cq == CPR - 1;
+            // an own row block's partial stays in the stash (slot 0: the
+            // warp's first row block, 1: its last); everything else passes
+            // through slot 1, free until the warp's last segment
+            uint32_t *red = (!shared_warp && !whole && crb == rb_first) ? st0 : st1;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const int col = 8 * nt + 2 * t;
@@ -495,8 +631,21 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
                     acc_f[nt][r] = 0.f;
                 }
             }
-            const bool whole = seg_whole && cq == CPR - 1;
-            gi_flush<BITS, NR>(p, crb, whole, crb == rb_first ? 0 : 1, w, Wt, red, s_e, lane);
+            if (shared_warp && !whole) { // at most two: the first and the last row block of the run
+                const uint32_t tk = gi_shared_partial<BITS, NR>(p, crb, crb == rb_first ? 0 : 1, w, red, s_e, lane);
+                if (npend == 0) {
+                    pend_rb0 = crb;
+                    pend_t0 = tk;
+                } else {
+                    pend_rb1 = crb;
+                    pend_t1 = tk;
+                }
+                ++npend;
+            } else if (whole) {
+                __syncwarp();
+                gi_write_y<BITS, NR>(p, crb, red, s_e, lane);
+                __syncwarp(); // red is rewritten by the next segment
+            }
             ++crb;
             cq = 0;
             seg_whole = true;
@@ -504,6 +653,12 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
             ++cq;
         }
     }
+    if (npend > 0)
+        gi_shared_fixup<BITS, NT, WARPS>(p, pend_rb0, pend_t0, G, s_e, st0, lane);
+    if (npend > 1)
+        gi_shared_fixup<BITS, NT, WARPS>(p, pend_rb1, pend_t1, G, s_e, st0, lane);
+    __syncthreads(); // every warp's stash is complete
+    gi_local_out<BITS, NT, WARPS>(p, ct, c, stash, s_e, warp, lane);
     pdl_launch_dependents();
 }
 
@@ -512,12 +667,17 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
 // ---------------------------------------------------------------------------
 int gi_ntiles(int M) { return M <= 2 ? 1 : M <= 5 ? 2 : 3; }
 
-size_t gi_smem_bytes(int bits, int M, int K)
+// Dynamic shared memory of a CTA of `warps` warps: digit rows, INT4 digit
+// sums, the stash of partial sums (2 x 16 x NR words per warp).
+static size_t gi_smem_bytes_w(int bits, int M, int K, int warps)
 {
     const size_t KB = (size_t)(K + kBlockK - 1) / kBlockK;
+    const size_t NR = (size_t)8 * gi_ntiles(M);
     const size_t rows = (size_t)3 * M * (bits == 8 ? gi_row_stride<8>(K) : gi_row_stride<4>(K));
-    return rows + (bits == 4 ? KB * 8 * gi_ntiles(M) * sizeof(int32_t) : 0);
+    return rows + (bits == 4 ? KB * NR * sizeof(int32_t) : 0) + (size_t)warps * 2 * 16 * NR * sizeof(uint32_t);
 }
+
+size_t gi_smem_bytes(int bits, int M, int K) { return gi_smem_bytes_w(bits, M, K, 16); }
 
 bool gi_fits(int bits, int M, int K)
 {
@@ -535,7 +695,7 @@ size_t ws_bytes_gemv_i8(int M, int K, int N)
 template <int BITS, int NT, int WARPS>
 static cudaError_t launch_gi_t(const LinearArgs &a, void *ws, int sm_count, cudaStream_t st)
 {
-    const int smem = (int)gi_smem_bytes(BITS, a.M, a.K);
+    const int smem = (int)gi_smem_bytes_w(BITS, a.M, a.K, WARPS);
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(gemv_i8_kernel<BITS, NT, WARPS>,
@@ -563,7 +723,7 @@ static cudaError_t launch_gi_t(const LinearArgs &a, void *ws, int sm_count, cuda
     p.N = a.N;
     p.KB = sh.kblocks();
     p.CPR = (p.KB + GiCfg<BITS>::D - 1) / GiCfg<BITS>::D;
-    p.I = (a.N / 16) * p.CPR;
+    const int NRB = a.N / 16, I = NRB * p.CPR;
     p.wq = (const uint8_t *)a.wq;
     p.scales = (const uint16_t *)a.scales;
     p.zeros = (const uint8_t *)a.zeros;
@@ -573,11 +733,16 @@ static cudaError_t launch_gi_t(const LinearArgs &a, void *ws, int sm_count, cuda
     int G = per_sm * sm_count;
     if (G * WARPS > kGiMaxWarps)
         G = kGiMaxWarps / WARPS;
-    const int want = (p.I + 2 * WARPS - 1) / (2 * WARPS); // at least ~2 chunks per warp
+    const int want = (I + 2 * WARPS - 1) / (2 * WARPS); // at least ~2 chunks per warp
     if (G > want)
         G = want;
     if (G < 1)
         G = 1;
+    p.LB = NRB / G;
+    p.RB0 = G * p.LB;
+    p.RL = (NRB - p.RB0) * p.CPR;
+    if ((long long)I * WARPS >= (1LL << 31) || (long long)p.RL * G >= (1LL << 31))
+        return cudaErrorInvalidValue; // the kernel's 32-bit stream-K cuts
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

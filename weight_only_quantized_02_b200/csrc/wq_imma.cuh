@@ -130,22 +130,22 @@ __device__ __forceinline__ void imma_row_maxima(const uint16_t *__restrict__ x, 
                                                 uint32_t *s_amax)
 {
     const int vpr = K / 8; // 16-byte vectors per token row
-    const long long total = (long long)M * vpr;
+    const int total = M * vpr; // M <= 128, K <= 65536: 32-bit index arithmetic
     int cur_m = -1;
     uint32_t cur = 0;
-    for (long long v0 = et; v0 < total; v0 += BATCH * NTH) {
+    for (int v0 = et; v0 < total; v0 += BATCH * NTH) {
         uint4 q[BATCH];
 #pragma unroll
         for (int b = 0; b < BATCH; ++b) {
-            const long long v = v0 + (long long)b * NTH;
-            q[b] = v < total ? ldg_keep4(x + v * 8) : make_uint4(0, 0, 0, 0);
+            const int v = v0 + b * NTH;
+            q[b] = v < total ? ldg_keep4(x + (size_t)v * 8) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int b = 0; b < BATCH; ++b) {
-            const long long v = v0 + (long long)b * NTH;
+            const int v = v0 + b * NTH;
             if (v >= total)
                 break;
-            const int m = (int)(v / vpr);
+            const int m = v / vpr;
             if (m != cur_m) {
                 if (cur_m >= 0)
                     atomicMax(&s_amax[cur_m], cur);
@@ -185,10 +185,11 @@ __device__ __forceinline__ void imma_digit_phase(const uint16_t *__restrict__ x,
     constexpr int NV = W / 8;            // 16-byte activation vectors per item
     // items (token slot m, k-block, W-k step); slots M .. ceil(NR/3)-1 write the zero padding rows
     constexpr int MS = (NR + 2) / 3;
-    const long long items = (long long)MS * KB * IPB;
-    const long long i0 = items * c / G, i1 = items * (c + 1) / G;
-    auto item_x = [&](long long it, uint4 (&v)[NV]) {
-        const int m = (int)(it / (KB * IPB)), rem = (int)(it % (KB * IPB));
+    const int items = MS * KB * IPB; // items * G stays below 2^32: 32-bit index arithmetic
+    const int i0 = (int)((unsigned)items * (unsigned)c / (unsigned)G),
+              i1 = (int)((unsigned)items * (unsigned)(c + 1) / (unsigned)G);
+    auto item_x = [&](int it, uint4 (&v)[NV]) {
+        const int m = it / (KB * IPB), rem = it % (KB * IPB);
         const int k0 = (rem / IPB) * kBlockK + W * (rem % IPB);
 #pragma unroll
         for (int j = 0; j < NV; ++j) // k past K or a padding slot: zero activations (zero weights there too)
@@ -206,8 +207,8 @@ __device__ __forceinline__ void imma_digit_phase(const uint16_t *__restrict__ x,
     if (et < M)
         s_e[et] = row_exponent(s_amax[et]);
     named_barrier_sync(1, 128);
-    for (long long it = i0 + et; it < i1; it += 128) {
-        const int m = (int)(it / (KB * IPB)), rem = (int)(it % (KB * IPB));
+    for (int it = i0 + et; it < i1; it += 128) {
+        const int m = it / (KB * IPB), rem = it % (KB * IPB);
         const int kb = rem / IPB, st = rem % IPB;
         uint4 v[NV];
 #pragma unroll

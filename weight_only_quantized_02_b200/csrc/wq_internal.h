@@ -98,13 +98,14 @@ cudaError_t launch_gemm_i4(const LinearArgs &a, void *ws, int sm_count, cudaStre
 cudaError_t read_gemm_i4_error(int *code, cudaStream_t st);
 
 // Integer GEMV (mma.sync m16n8k32 on the packed codes): M <= kGiMaxM,
-// K <= kI8MaxK, the CTA's digit rows (gi_smem_bytes) at most kGiMaxSmem of
-// shared memory; split 1 = one 16-warp CTA per SM, 2 = two 8-warp CTAs;
+// K <= kI8MaxK, the 16-warp CTA's dynamic shared memory (digit rows, INT4
+// digit sums, stash of partial sums: gi_smem_bytes) at most kGiMaxSmem;
+// split 1 = one 16-warp CTA per SM, 2 = two 8-warp CTAs;
 // at most kGiMaxCtas * 8 warps.  Workspace: [counters][partials
 // kGiMaxCtas x 8 x 2 x 16 x NR x 4 bytes], NR = 8 * gi_ntiles(M).
 constexpr int kGiMaxM = 8;
 constexpr int kGiMaxCtas = 448;
-constexpr int kGiMaxSmem = 200 * 1024;
+constexpr int kGiMaxSmem = 226 * 1024;
 int gi_ntiles(int M);
 size_t gi_smem_bytes(int bits, int M, int K);
 bool gi_fits(int bits, int M, int K);

@@ -375,20 +375,12 @@ __device__ __forceinline__ uint32_t ticket_take_acq_rel(uint32_t *counter)
 // Stream-K partition: U units cut into G contiguous ranges [start(c),
 // start(c+1)); a panel of consecutive units may span several ranges.
 // ---------------------------------------------------------------------------
-// U * G below 2^32 (every decode shape) takes the 32-bit division: a 64-bit
-// one is a long dependent chain, and the fix-ups call these in loops.
-__device__ __forceinline__ int sk_start(long long U, int G, int c)
-{
-    if ((unsigned long long)U * (unsigned)G < (1ull << 32))
-        return (int)((unsigned)U * (unsigned)c / (unsigned)G);
-    return (int)(U * c / G);
-}
+__device__ __forceinline__ int sk_start(long long U, int G, int c) { return (int)(U * c / G); }
 
 // CTA that owns unit u (ranges [start(c), start(c+1)); empty ranges skipped)
 __device__ __forceinline__ int sk_owner(long long U, int G, int u)
 {
-    int c = (unsigned long long)U * (unsigned)G < (1ull << 32) ? (int)((unsigned)u * (unsigned)G / (unsigned)U)
-                                                                 : (int)(((long long)u * G) / U);
+    int c = (int)(((long long)u * G) / U);
     if (c >= G)
         c = G - 1;
     while (c + 1 < G && sk_start(U, G, c + 1) <= u)

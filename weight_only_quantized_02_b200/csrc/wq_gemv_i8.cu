@@ -108,23 +108,54 @@ __device__ __forceinline__ void gi_digits(const GiParams &p, uint8_t *sd, int32_
     const int et = threadIdx.x, ch = et & 7;
     const int M = p.M, K = p.K, KB = p.KB;
     const int S = gi_row_stride<BITS>(K);
-    imma_row_maxima<NTH, 2>(p.x, M, K, et, s_amax); // few registers: the weight prefetch is live
-    __syncthreads();
-    if (et < M)
-        s_e[et] = row_exponent(s_amax[et]);
-    __syncthreads();
     const int cpr = KB * 8; // 16-k chunks per token row
     const int items = M * cpr;
-    for (int base = 0; base < items; base += NTH) { // uniform trip count: shuffles below
-        const int it = base + et;
-        const bool act = it < items;
-        const int m = act ? it / cpr : 0, c = act ? it % cpr : 0; // chunk c: k = 16c .. 16c + 15
-        uint4 a = make_uint4(0, 0, 0, 0), b = a;
-        if (act && 16 * c < K) {
+    // The thread's first HOLD chunks are loaded once, together (one round
+    // trip to L2), and kept in registers from the row maxima to the digits;
+    // chunks beyond HOLD * NTH (M > 4 at K = 5120 with 512 threads) are
+    // loaded in both passes.
+    constexpr int HOLD = NR == 8 ? 2 : 3;
+    auto load_chunk = [&](int it, uint4 &a, uint4 &b) {
+        a = make_uint4(0, 0, 0, 0);
+        b = a;
+        const int m = it / cpr, c = it % cpr; // chunk c: k = 16c .. 16c + 15
+        if (it < items && 16 * c < K) {
             const uint16_t *src = p.x + (size_t)m * K + 16 * c;
             a = ldg_keep4(src);
             b = ldg_keep4(src + 8);
         }
+    };
+    auto chunk_max = [&](int it, const uint4 &a, const uint4 &b) {
+        if (it >= items)
+            return;
+        const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t mx = 0;
+#pragma unroll
+        for (int h = 0; h < 8; ++h)
+            mx = max(mx, max(wv[h] & 0x7FFFu, (wv[h] >> 16) & 0x7FFFu));
+        atomicMax(&s_amax[it / cpr], mx);
+    };
+    uint4 ha[HOLD], hb[HOLD];
+#pragma unroll
+    for (int h = 0; h < HOLD; ++h)
+        load_chunk(h * NTH + et, ha[h], hb[h]);
+#pragma unroll
+    for (int h = 0; h < HOLD; ++h)
+        chunk_max(h * NTH + et, ha[h], hb[h]);
+    for (int it = HOLD * NTH + et; it < items; it += NTH) {
+        uint4 a, b;
+        load_chunk(it, a, b);
+        chunk_max(it, a, b);
+    }
+    __syncthreads();
+    if (et < M)
+        s_e[et] = row_exponent(s_amax[et]);
+    __syncthreads();
+    // chunk it (bf16 in a, b) -> its digit rows; all threads of a warp call
+    // it together (the INT4 byte order is made with shuffles)
+    auto convert = [&](int it, const uint4 &a, const uint4 &b) {
+        const bool act = it < items;
+        const int m = act ? it / cpr : 0, c = act ? it % cpr : 0;
         uint32_t pl[3][4];
 #pragma unroll
         for (int i = 0; i < 3; ++i)
@@ -179,6 +210,15 @@ __device__ __forceinline__ void gi_digits(const GiParams &p, uint8_t *sd, int32_
                 }
             }
         }
+    };
+#pragma unroll
+    for (int h = 0; h < HOLD; ++h)
+        if (h * NTH < items) // uniform
+            convert(h * NTH + et, ha[h], hb[h]);
+    for (int base = HOLD * NTH; base < items; base += NTH) { // uniform trip count: shuffles
+        uint4 a, b;
+        load_chunk(base + et, a, b);
+        convert(base + et, a, b);
     }
     __syncthreads();
 }

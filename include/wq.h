@@ -97,10 +97,12 @@ typedef enum {
 #define WQ_VARIANT_GEMM_SK 3 /* stream-K tcgen05 GEMM, M <= 128, persistent; needs the workspace */
 #define WQ_VARIANT_I8MMA 4   /* stream-K tcgen05 kind::i8: W8A16 (M <= 64) on the raw codes,
                                 W4A16 (M <= 32) on q - z; K <= 65536; needs the workspace */
-#define WQ_VARIANT_GEMV_I8 5 /* warp-level stream-K GEMV on mma.sync m16n8k32 s8 (the packed codes
-                                as they are, activations as exact digits in shared memory), M <= 8,
-                                3 * M * K bytes <= ~200 KB; split 1 = one 16-warp CTA per SM, 2 = two
-                                8-warp CTAs per SM; needs the workspace */
+#define WQ_VARIANT_GEMV_I8 5 /* GEMV on mma.sync m16n8k32 s8 (the packed codes as they are,
+                                activations as exact digits in shared memory): each CTA owns whole
+                                16-row blocks, the rest are cut stream-K style across CTAs; M <= 8,
+                                3 * M * K bytes of digits plus 16-48 KB of partial sums <= 226 KB;
+                                split 1 = one 16-warp CTA per SM, 2 = two 8-warp CTAs per SM; needs
+                                the workspace */
 #define WQ_VARIANT_GEMM_W4 6 /* W4A16 only, M <= 128: stream-K tcgen05 GEMM with one 512-thread CTA
                                 per SM, every role (weight and x loads, dequantization, MMA, group
                                 rescale) on its own warps with its own ring; needs the workspace */

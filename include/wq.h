@@ -306,6 +306,29 @@ int wq_device_error(cudaStream_t stream);
  * range, WQ_ERR_CUDA if the launch fails. */
 int wq_wait_selftest(int limit_us, cudaStream_t stream);
 
+/* Debug views of the integer GEMV's (WQ_VARIANT_GEMV_I8) work split, for a
+ * grid of G CTAs (1..448) of `warps` warps (16: split 1, 8: split 2), bits 4
+ * or 8, 1 <= K <= 65536, N a positive multiple of 16. The pages have no
+ * counterpart; the tests check the split with them. Host only, no GPU.
+ * Row blocks are 16 output channels; a chunk is the D consecutive 128-k
+ * blocks of one row block that a warp takes together (D = 4 for INT8, 6
+ * for INT4; a row block's last chunk may be shorter).
+ *   wq_gemv_i8_plan: meta[4] = {chunks per row block CPR, row blocks each
+ *   CTA owns LB (CTA c owns c LB .. c LB + LB - 1), first shared row block
+ *   RB0 = G LB, chunks of the shared row blocks RL}; runs[G][warps][4] =
+ *   {first row block, its first chunk, number of chunks, 1 if the warp takes
+ *   shared chunks}: a warp's chunks are consecutive, row-block-major.
+ *   wq_gemv_i8_contributors: for shared row block rb (RB0 <= rb < N/16),
+ *   the warps (global index c * warps + w) whose chunks meet it, in the
+ *   order their partials are summed, and each one's partial slot (0 if rb
+ *   is the warp's first row block, else 1); warp_ids and slots hold at
+ *   least CPR entries, *count receives the number.
+ * Both return WQ_ERR_SHAPE for arguments out of range (or a split beyond
+ * 32-bit index arithmetic), WQ_ERR_NULL for a null pointer. */
+int wq_gemv_i8_plan(int bits, int K, int N, int G, int warps, int *meta, int *runs);
+int wq_gemv_i8_contributors(int bits, int K, int N, int G, int warps, int rb, int *warp_ids, int *slots,
+                            int *count);
+
 #ifdef __cplusplus
 }
 #endif

@@ -77,6 +77,8 @@ def _load():
         "wq_dequant_debug": (I, [P, P, P, I, I, I, I, P, P]),
         "wq_device_error": (I, [P]),
         "wq_wait_selftest": (I, [I, P]),
+        "wq_gemv_i8_plan": (I, [I, I, I, I, I, P, P]),
+        "wq_gemv_i8_contributors": (I, [I, I, I, I, I, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -329,3 +331,25 @@ def wq_wait_selftest(limit_us: int = 50000, stream=None) -> None:
     completes its mbarrier); it records WQ_ERR_TIMEOUT in the device error
     word, which wq_device_error then reports."""
     _check(lib.wq_wait_selftest(int(limit_us), _s(stream)), "wq_wait_selftest")
+
+
+def wq_gemv_i8_plan(bits: int, K: int, N: int, G: int, warps: int = 16):
+    """The integer GEMV's work split for G CTAs of `warps` warps (host only):
+    (meta {CPR, LB, RB0, RL}, runs [G][warps][4] = first row block, its
+    first chunk, chunks, shared-warp flag)."""
+    meta = (ctypes.c_int * 4)()
+    runs = (ctypes.c_int * (G * warps * 4))()
+    _check(lib.wq_gemv_i8_plan(bits, K, N, G, warps, meta, runs), "wq_gemv_i8_plan")
+    return dict(CPR=meta[0], LB=meta[1], RB0=meta[2], RL=meta[3]), \
+        [[tuple(runs[(c * warps + w) * 4:(c * warps + w) * 4 + 4]) for w in range(warps)] for c in range(G)]
+
+
+def wq_gemv_i8_contributors(bits: int, K: int, N: int, G: int, warps: int, rb: int, cpr: int):
+    """Contributors of shared row block rb, in summation order: a list of
+    (global warp index, partial slot)."""
+    ids = (ctypes.c_int * max(cpr, 1))()
+    slots = (ctypes.c_int * max(cpr, 1))()
+    n = ctypes.c_int(0)
+    _check(lib.wq_gemv_i8_contributors(bits, K, N, G, warps, rb, ids, slots, ctypes.byref(n)),
+           "wq_gemv_i8_contributors")
+    return [(ids[i], slots[i]) for i in range(n.value)]

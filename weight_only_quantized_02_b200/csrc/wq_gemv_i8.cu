@@ -40,6 +40,7 @@
 
 #include <cuda_bf16.h>
 
+#include "wq.h"
 #include "wq_device.cuh"
 #include "wq_imma.cuh"
 #include "wq_internal.h"
@@ -226,9 +227,12 @@ __device__ __forceinline__ void gi_digits(const GiParams &p, uint8_t *sd, int32_
 // Stream-K cuts in 32-bit arithmetic (every U * c and u * G here stays far
 // below 2^32; the launch checks the bound): range c of G over U units
 // starts at U c / G; gi_owner is the range holding unit u.
-__device__ __forceinline__ int gi_start(int U, int G, int c) { return (int)((unsigned)U * (unsigned)c / (unsigned)G); }
+__host__ __device__ __forceinline__ int gi_start(int U, int G, int c)
+{
+    return (int)((unsigned)U * (unsigned)c / (unsigned)G);
+}
 
-__device__ __forceinline__ int gi_owner(int U, int G, int u)
+__host__ __device__ __forceinline__ int gi_owner(int U, int G, int u)
 {
     int c = (int)((unsigned)u * (unsigned)G / (unsigned)U);
     c = c < G - 1 ? c : G - 1;
@@ -249,7 +253,7 @@ struct GiCta {
     int lo, L, ws;
 };
 
-__device__ __forceinline__ GiCta gi_cta(const GiParams &p, int G, int c, int warps)
+__host__ __device__ __forceinline__ GiCta gi_cta(const GiParams &p, int G, int c, int warps)
 {
     GiCta t;
     t.lo = gi_start(p.RL, G, c);
@@ -264,6 +268,40 @@ __device__ __forceinline__ GiCta gi_cta(const GiParams &p, int G, int c, int war
         t.ws = ws < 1 ? 1 : ws > warps / 2 ? warps / 2 : ws;
     }
     return t;
+}
+
+// Warp `warp` of CTA c: n chunks from chunk q0 of row block rb0 (shared
+// warps: its cut of the CTA's shared chunks; the others: its cut of the
+// CTA's own row blocks).
+__host__ __device__ __forceinline__ void gi_warp_run(const GiParams &p, const GiCta &ct, int c, int warp, int warps,
+                                                     int &rb0, int &q0, int &n)
+{
+    if (warp < ct.ws) {
+        const int o0 = gi_start(ct.L, ct.ws, warp);
+        n = gi_start(ct.L, ct.ws, warp + 1) - o0;
+        rb0 = p.RB0 + (ct.lo + o0) / p.CPR;
+        q0 = (ct.lo + o0) % p.CPR;
+    } else {
+        const int own = p.LB * p.CPR, o0 = gi_start(own, warps - ct.ws, warp - ct.ws);
+        n = gi_start(own, warps - ct.ws, warp - ct.ws + 1) - o0;
+        rb0 = c * p.LB + o0 / p.CPR;
+        q0 = o0 % p.CPR;
+    }
+}
+
+// Chunk i of shared row block rb: whether a contributor's run starts there
+// (the row block's first chunk, or the start of a CTA's share or of a
+// warp's cut), that warp (global index) and its partial slot (0 if rb is
+// its first row block).
+__host__ __device__ __forceinline__ bool gi_contrib_at(const GiParams &p, int G, int warps, int rb, int i, int &gw,
+                                                       int &slot)
+{
+    const int u = (rb - p.RB0) * p.CPR + i, cc = gi_owner(p.RL, G, u);
+    const GiCta t = gi_cta(p, G, cc, warps);
+    const int o = u - t.lo, wi = gi_owner(t.L, t.ws, o), s0 = gi_start(t.L, t.ws, wi);
+    gw = cc * warps + wi;
+    slot = p.RB0 + (t.lo + s0) / p.CPR == rb ? 0 : 1;
+    return i == 0 || o == s0;
 }
 
 // One segment's output, its accumulators in red ([16 rows][NR]; INT8 int32
@@ -326,19 +364,15 @@ __device__ __forceinline__ void gi_shared_fixup(const GiParams &p, int rb, uint3
 {
     constexpr int NR = 8 * NT;
     const int M = p.M, N = p.N, n0 = 16 * rb, CPR = p.CPR;
-    const int u0 = (rb - p.RB0) * CPR;
     int nc = 0;
     for (int base = 0; base < CPR; base += 32) {
         const int i = base + lane;
         bool start = false;
         uint32_t off = 0;
         if (i < CPR) {
-            const int u = u0 + i, cc = gi_owner(p.RL, G, u);
-            const GiCta t = gi_cta(p, G, cc, WARPS);
-            const int o = u - t.lo, wi = gi_owner(t.L, t.ws, o), s0 = gi_start(t.L, t.ws, wi);
-            start = i == 0 || o == s0;
-            const int sl = p.RB0 + (t.lo + s0) / CPR == rb ? 0 : 1; // rb is the warp's first row block?
-            off = ((uint32_t)(cc * WARPS + wi) * 2 + sl) * 16 * NR;
+            int gw, sl;
+            start = gi_contrib_at(p, G, WARPS, rb, i, gw, sl);
+            off = ((uint32_t)gw * 2 + sl) * 16 * NR;
         }
         const uint32_t mask = __ballot_sync(0xffffffffu, start);
         if (start)
@@ -460,19 +494,8 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
     uint32_t *st0 = stash + (size_t)warp * 2 * 16 * NR, *st1 = st0 + 16 * NR;
     const GiCta ct = gi_cta(p, G, c, WARPS);
     const bool shared_warp = warp < ct.ws;
-    // the warp's run of chunks: n chunks from chunk q0 of row block rb0
-    int rb0, q0, n;
-    if (shared_warp) {
-        const int o0 = gi_start(ct.L, ct.ws, warp);
-        n = gi_start(ct.L, ct.ws, warp + 1) - o0;
-        rb0 = p.RB0 + (ct.lo + o0) / p.CPR;
-        q0 = (ct.lo + o0) % p.CPR;
-    } else {
-        const int own = p.LB * p.CPR, o0 = gi_start(own, WARPS - ct.ws, warp - ct.ws);
-        n = gi_start(own, WARPS - ct.ws, warp - ct.ws + 1) - o0;
-        rb0 = c * p.LB + o0 / p.CPR;
-        q0 = o0 % p.CPR;
-    }
+    int rb0, q0, n; // the warp's run: n chunks from chunk q0 of row block rb0
+    gi_warp_run(p, ct, c, warp, WARPS, rb0, q0, n);
 
     // ---------------- weights of the first chunk (before the launch wait) ----------------
     // The warp's work is n consecutive chunks from (rb0, q0): chunk (rb, q) =
@@ -732,6 +755,21 @@ size_t ws_bytes_gemv_i8(int M, int K, int N)
     return ws_counter_bytes(N) + (size_t)kGiMaxWarps * 2 * 16 * NR * 4;
 }
 
+// The work split of a grid of G CTAs of `warps` warps: chunks per row block,
+// own row blocks per CTA, the first shared row block, shared chunks.  False
+// when the cuts would leave 32-bit arithmetic.
+static bool gi_plan(GiParams &p, int bits, int K, int N, int G, int warps)
+{
+    const int D = bits == 8 ? GiCfg<8>::D : GiCfg<4>::D;
+    const int NRB = N / 16;
+    p.KB = (K + kBlockK - 1) / kBlockK;
+    p.CPR = (p.KB + D - 1) / D;
+    p.LB = NRB / G;
+    p.RB0 = G * p.LB;
+    p.RL = (NRB - p.RB0) * p.CPR;
+    return (long long)NRB * p.CPR * warps < (1LL << 31) && (long long)p.RL * G < (1LL << 31);
+}
+
 template <int BITS, int NT, int WARPS>
 static cudaError_t launch_gi_t(const LinearArgs &a, void *ws, int sm_count, cudaStream_t st)
 {
@@ -763,7 +801,7 @@ static cudaError_t launch_gi_t(const LinearArgs &a, void *ws, int sm_count, cuda
     p.N = a.N;
     p.KB = sh.kblocks();
     p.CPR = (p.KB + GiCfg<BITS>::D - 1) / GiCfg<BITS>::D;
-    const int NRB = a.N / 16, I = NRB * p.CPR;
+    const int I = (a.N / 16) * p.CPR;
     p.wq = (const uint8_t *)a.wq;
     p.scales = (const uint16_t *)a.scales;
     p.zeros = (const uint8_t *)a.zeros;
@@ -778,11 +816,8 @@ static cudaError_t launch_gi_t(const LinearArgs &a, void *ws, int sm_count, cuda
         G = want;
     if (G < 1)
         G = 1;
-    p.LB = NRB / G;
-    p.RB0 = G * p.LB;
-    p.RL = (NRB - p.RB0) * p.CPR;
-    if ((long long)I * WARPS >= (1LL << 31) || (long long)p.RL * G >= (1LL << 31))
-        return cudaErrorInvalidValue; // the kernel's 32-bit stream-K cuts
+    if (!gi_plan(p, BITS, a.K, a.N, G, WARPS))
+        return cudaErrorInvalidValue; // beyond the kernel's 32-bit stream-K cuts
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -820,3 +855,63 @@ cudaError_t launch_gemv_i8(const LinearArgs &a, int split, void *ws, int sm_coun
 }
 
 } // namespace wq
+
+// ---------------------------------------------------------------------------
+// Debug views of the integer GEMV's work split (host only; no GPU)
+// ---------------------------------------------------------------------------
+static int gi_debug_args(int bits, int K, int N, int G, int warps)
+{
+    if ((bits != 4 && bits != 8) || K < 1 || K > wq::kI8MaxK || N < 16 || N % 16 != 0 || G < 1 ||
+        G > wq::kGiMaxCtas || (warps != 8 && warps != 16))
+        return WQ_ERR_SHAPE;
+    return WQ_OK;
+}
+
+extern "C" int wq_gemv_i8_plan(int bits, int K, int N, int G, int warps, int *meta, int *runs)
+{
+    if (meta == nullptr || runs == nullptr)
+        return WQ_ERR_NULL;
+    const int st = gi_debug_args(bits, K, N, G, warps);
+    if (st != WQ_OK)
+        return st;
+    wq::GiParams p{};
+    if (!wq::gi_plan(p, bits, K, N, G, warps))
+        return WQ_ERR_SHAPE;
+    meta[0] = p.CPR;
+    meta[1] = p.LB;
+    meta[2] = p.RB0;
+    meta[3] = p.RL;
+    for (int c = 0; c < G; ++c) {
+        const wq::GiCta ct = wq::gi_cta(p, G, c, warps);
+        for (int w = 0; w < warps; ++w) {
+            int *r = runs + ((size_t)c * warps + w) * 4;
+            wq::gi_warp_run(p, ct, c, w, warps, r[0], r[1], r[2]);
+            r[3] = w < ct.ws ? 1 : 0;
+        }
+    }
+    return WQ_OK;
+}
+
+extern "C" int wq_gemv_i8_contributors(int bits, int K, int N, int G, int warps, int rb, int *warp_ids, int *slots,
+                                       int *count)
+{
+    if (warp_ids == nullptr || slots == nullptr || count == nullptr)
+        return WQ_ERR_NULL;
+    const int st = gi_debug_args(bits, K, N, G, warps);
+    if (st != WQ_OK)
+        return st;
+    wq::GiParams p{};
+    if (!wq::gi_plan(p, bits, K, N, G, warps) || rb < p.RB0 || rb >= N / 16)
+        return WQ_ERR_SHAPE;
+    int n = 0;
+    for (int i = 0; i < p.CPR; ++i) {
+        int gw, sl;
+        if (wq::gi_contrib_at(p, G, warps, rb, i, gw, sl)) {
+            warp_ids[n] = gw;
+            slots[n] = sl;
+            ++n;
+        }
+    }
+    *count = n;
+    return WQ_OK;
+}

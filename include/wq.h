@@ -273,7 +273,12 @@ int wq_set_choice(int M, int K, int N, int bits, int group, int variant, int spl
 int wq_clear_tuning(void);
 
 /* Text file, one entry per line. Host. WQ_ERR_TUNING on a malformed line;
- * in that case the table is left unchanged. */
+ * in that case the table is left unchanged.
+ * The environment variable WQ_TUNING_FILE names a table that is loaded the
+ * same way when the library is loaded. If it cannot be read or parsed,
+ * every automatic choice (wq_linear; wq_linear_forced and wq_linear_ex
+ * with WQ_VARIANT_AUTO; wq_get_choice) returns WQ_ERR_TUNING; forced
+ * variants still run. */
 int wq_save_tuning(const char *path);
 int wq_load_tuning(const char *path);
 

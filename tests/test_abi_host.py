@@ -7,6 +7,7 @@ behave as documented.
 import ctypes
 import os
 import subprocess
+import sys
 
 import pytest
 
@@ -136,3 +137,36 @@ def test_no_oracle_in_product():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 text = open(os.path.join(root, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text and "liboracle" not in text, f
+
+
+def _run_with_env(code, env_extra):
+    env = dict(os.environ)
+    env.update(env_extra)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, cwd=root, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    return out.stdout
+
+
+def test_tuning_file_from_environment_is_loaded(tmp_path):
+    shipped = os.path.join(os.path.dirname(wq.__file__), "tuning_b200.txt")
+    saved = tmp_path / "saved.txt"
+    _run_with_env(f"import weight_only_quantized_02_b200 as wq; assert wq.lib.wq_save_tuning({str(saved)!r}.encode()) == 0",
+                  {"WQ_TUNING_FILE": shipped})
+
+    def entries(path):
+        return sorted(" ".join(l.split()[:9]) for l in open(path) if l.strip() and not l.startswith("#"))
+
+    assert entries(saved) == entries(shipped)
+
+
+def test_unreadable_tuning_file_from_environment_fails_automatic_choices(tmp_path):
+    code = ("import ctypes, weight_only_quantized_02_b200 as wq\n"
+            "v, s = ctypes.c_int(0), ctypes.c_int(0)\n"
+            "print(wq.lib.wq_get_choice(1, 5120, 17408, 8, 0, ctypes.byref(v), ctypes.byref(s)))\n")
+    out = _run_with_env(code, {"WQ_TUNING_FILE": str(tmp_path / "missing.txt")})
+    assert int(out.strip().splitlines()[-1]) == -8  # WQ_ERR_TUNING
+    bad = tmp_path / "bad.txt"
+    bad.write_text("this is not a table\n")
+    out = _run_with_env(code, {"WQ_TUNING_FILE": str(bad)})
+    assert int(out.strip().splitlines()[-1]) == -8

@@ -55,6 +55,10 @@ int current_device_info(DeviceInfo *out)
     return WQ_OK;
 }
 
+// Status of the table named by the environment variable WQ_TUNING_FILE,
+// loaded when the library is loaded (WQ_OK when the variable is unset).
+int g_env_tuning = WQ_OK;
+
 std::string device_key(const DeviceInfo &d)
 {
     std::string n = d.name;
@@ -228,6 +232,8 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
     const bool i8_ws_ok = w && i8_fits(bits, M, K) && have >= ws_bytes_imma(bits, M, K, N);
     const bool gi_ws_ok = w && gi_fits(bits, M, K) && have >= ws_bytes_gemv_i8(M, K, N);
 
+    if (variant == WQ_VARIANT_AUTO && g_env_tuning != WQ_OK)
+        return g_env_tuning; // the table named by WQ_TUNING_FILE did not load
     Choice c;
     lookup_choice(d, M, K, N, bits, group, &c);
     if (variant != WQ_VARIANT_AUTO) {
@@ -618,6 +624,8 @@ int wq_get_choice(int M, int K, int N, int bits, int group, int *variant, int *s
 {
     if (!variant || !split)
         return WQ_ERR_NULL;
+    if (g_env_tuning != WQ_OK)
+        return g_env_tuning;
     DeviceInfo d;
     int st = current_device_info(&d);
     if (st != WQ_OK)
@@ -767,3 +775,18 @@ int wq_device_error(cudaStream_t stream)
 }
 
 } // extern "C"
+
+// WQ_TUNING_FILE: a dispatcher table (the wq_save_tuning format) loaded when
+// the library is loaded, so a deployment can ship measured choices without
+// code.  A file that cannot be read or parsed makes every automatic choice
+// (wq_linear, wq_get_choice) return WQ_ERR_TUNING; forced variants still run.
+namespace {
+struct EnvTuningLoader {
+    EnvTuningLoader()
+    {
+        const char *path = getenv("WQ_TUNING_FILE");
+        if (path && *path)
+            g_env_tuning = wq_load_tuning(path);
+    }
+} g_env_tuning_loader;
+} // namespace

@@ -18,7 +18,7 @@
  *
  * Four kernel families sit behind one call:
  *   - a GEMV for decode-sized M, with register-level dequantization and
- *     128-bit weight loads ("BitBLAS-style GEMV", tileInfer README, Features
+ *     128-bit weight loads (the GEMV row of the tileInfer README, Features
  *     table). Its fp32 dot products run on mma.sync tensor-core fragments.
  *   - a small-M GEMM (tcgen05 tensor cores, accumulators in tensor memory)
  *     with split-K and a fixed-order fp32 reduction ("split_k" auto-tuning,

@@ -9,6 +9,7 @@ torch's own runtime).  Objects go to ``_build/`` next to this file.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import os
 import shutil
 import subprocess
@@ -53,17 +54,22 @@ def build(force: bool = False, verbose: bool = False) -> str:
     ]
     if verbose:
         common += ["-Xptxas", "-v"]
-    objs = []
-    for src in SOURCES:
-        obj = os.path.join(BUILD, src.replace(".cu", ".o"))
-        cmd = [cc] + common + ["-c", os.path.join(CSRC, src), "-o", obj]
-        r = subprocess.run(cmd, capture_output=True, text=True)
+    objs = [os.path.join(BUILD, src.replace(".cu", ".o")) for src in SOURCES]
+
+    def compile_one(i):
+        cmd = [cc] + common + ["-c", os.path.join(CSRC, SOURCES[i]), "-o", objs[i]]
+        return subprocess.run(cmd, capture_output=True, text=True)
+
+    # the translation units are independent: compile them side by side
+    jobs = max(1, min(len(SOURCES), os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(jobs) as ex:
+        results = list(ex.map(compile_one, range(len(SOURCES))))
+    for src, r in zip(SOURCES, results):
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
             raise RuntimeError("nvcc failed on " + src)
         if verbose:
             sys.stderr.write(r.stdout + r.stderr)
-        objs.append(obj)
     tmp = LIB + ".tmp"
     cmd = [cc] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs + ["-lpthread", "-ldl", "-lrt"]
     r = subprocess.run(cmd, capture_output=True, text=True)

@@ -302,6 +302,53 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
 
 } // namespace
 
+namespace wq {
+
+namespace {
+struct SetupKey {
+    int dev;
+    const void *func;
+    bool operator<(const SetupKey &o) const { return dev != o.dev ? dev < o.dev : func < o.func; }
+};
+struct SetupState {
+    size_t optin = 0;
+    std::map<std::pair<int, size_t>, int> occ; // (threads, smem) -> CTAs per SM
+};
+std::mutex g_setup_mu;
+std::map<SetupKey, SetupState> g_setup;
+} // namespace
+
+cudaError_t kernel_setup(const void *func, size_t smem_optin, int threads, size_t smem, int *occ)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    std::lock_guard<std::mutex> lk(g_setup_mu);
+    SetupState &s = g_setup[SetupKey{dev, func}];
+    if (smem_optin > s.optin) {
+        e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_optin);
+        if (e != cudaSuccess)
+            return e;
+        s.optin = smem_optin;
+    }
+    if (occ) {
+        const auto k = std::make_pair(threads, smem);
+        auto it = s.occ.find(k);
+        if (it == s.occ.end()) {
+            int o = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, func, threads, smem);
+            if (e != cudaSuccess)
+                return e;
+            it = s.occ.emplace(k, o > 0 ? o : 1).first;
+        }
+        *occ = it->second;
+    }
+    return cudaSuccess;
+}
+
+} // namespace wq
+
 // ===========================================================================
 // C ABI
 // ===========================================================================
@@ -603,7 +650,8 @@ int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
         if (const char *lg = getenv("WQ_TUNE_LOG"); lg && *lg && *lg != '0')
             fprintf(stderr, "wq_tune M=%d K=%d N=%d bits=%d group=%d variant=%d split=%d us=%.3f\n", M, K, N,
                     bits, group, v, s, med);
-        // ">=": on an exact tie the later (larger) split wins, as in the page's loop
+        // ">=": on an exact tie the later (larger) split wins (Mit han lab Llm awq
+        // Kernel Selection Thresholds, The Insight: the split_k auto-tune)
         if (best.variant < 0 || best.us >= med)
             best = {v, s, med};
     }

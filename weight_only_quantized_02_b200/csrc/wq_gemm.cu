@@ -397,13 +397,10 @@ static cudaError_t launch_gemm_t(const LinearArgs &a, int S, void *ws, cudaStrea
 {
     constexpr size_t smem = gemm_smem_bytes<BITS, NT>();
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BITS, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+    {
+        const cudaError_t e = kernel_setup((const void *)gemm_kernel<BITS, NT>, smem, 0, 0, nullptr);
         if (e != cudaSuccess)
             return e;
-        attr_set = true;
     }
     CUtensorMap map;
     if (!make_x_map<NT>(&map, a.x, a.M, a.K))

@@ -468,13 +468,10 @@ static cudaError_t launch_i4_t(const LinearArgs &a, void *ws, int sm_count, cuda
 {
     constexpr size_t smem = i4_smem_bytes<NR>();
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_i4_kernel<NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+    {
+        const cudaError_t e = kernel_setup((const void *)gemm_i4_kernel<NR>, smem, 0, 0, nullptr);
         if (e != cudaSuccess)
             return e;
-        attr_set = true;
     }
     const Shape sh{4, a.K, a.N, 128};
     I4Params p;

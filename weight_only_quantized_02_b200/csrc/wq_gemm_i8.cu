@@ -404,13 +404,10 @@ static cudaError_t launch_i8_t(const LinearArgs &a, void *ws, int sm_count, cuda
     constexpr size_t smem = i8_smem_bytes<NR>();
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
     static_assert(I8Cfg<NR>::kOcc == 1 || 2 * (smem + 1024) <= 228 * 1024, "two CTAs per SM");
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_i8_kernel<NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+    {
+        const cudaError_t e = kernel_setup((const void *)gemm_i8_kernel<NR>, smem, 0, 0, nullptr);
         if (e != cudaSuccess)
             return e;
-        attr_set = true;
     }
     const Shape sh{8, a.K, a.N, 0};
     I8Params p;

@@ -471,13 +471,10 @@ static cudaError_t launch_gemm_sk_t(const LinearArgs &a, int ctas_per_sm, void *
     using C = GskCfg<BITS, NT>;
     constexpr size_t smem = gemm_sk_smem_bytes<BITS, NT>();
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_sk_kernel<BITS, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+    {
+        const cudaError_t e = kernel_setup((const void *)gemm_sk_kernel<BITS, NT>, smem, 0, 0, nullptr);
         if (e != cudaSuccess)
             return e;
-        attr_set = true;
     }
     CUtensorMap map;
     if (!make_x_map<NT>(&map, a.x, a.M, a.K))

@@ -482,13 +482,10 @@ static cudaError_t launch_gemm_w4_t(const LinearArgs &a, void *ws, int sm_count,
 {
     constexpr size_t smem = gemm_w4_smem_bytes<NT>();
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e =
-            cudaFuncSetAttribute(gemm_w4_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    {
+        const cudaError_t e = kernel_setup((const void *)gemm_w4_kernel<NT>, smem, 0, 0, nullptr);
         if (e != cudaSuccess)
             return e;
-        attr_set = true;
     }
     CUtensorMap map;
     if (!make_x_map<NT>(&map, a.x, a.M, a.K))

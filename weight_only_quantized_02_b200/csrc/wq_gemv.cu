@@ -284,13 +284,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvParams 
 template <int BITS, int MT>
 static cudaError_t launch_gemv_t(const GemvParams &p, int sm_count, cudaStream_t st)
 {
-    static int occ = -1; // CTAs per SM, from the hardware occupancy query (cached)
-    if (occ < 0) {
-        int o = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, gemv_kernel<BITS, MT>, kGemvWarps * 32, 0);
+    int occ = 1; // CTAs per SM, from the hardware occupancy query (cached per device)
+    {
+        const cudaError_t e = kernel_setup((const void *)gemv_kernel<BITS, MT>, 0, kGemvWarps * 32, 0, &occ);
         if (e != cudaSuccess)
             return e;
-        occ = o > 0 ? o : 1;
     }
     const int rbs_per_cta = kGemvWarps / p.ks;
     const int units = ((p.N >> 4) + rbs_per_cta - 1) / rbs_per_cta;

@@ -774,23 +774,12 @@ template <int BITS, int NT, int WARPS>
 static cudaError_t launch_gi_t(const LinearArgs &a, void *ws, int sm_count, cudaStream_t st)
 {
     const int smem = (int)gi_smem_bytes_w(BITS, a.M, a.K, WARPS);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_i8_kernel<BITS, NT, WARPS>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kGiMaxSmem);
+    int occ = 1;
+    {
+        const cudaError_t e =
+            kernel_setup((const void *)gemv_i8_kernel<BITS, NT, WARPS>, kGiMaxSmem, WARPS * 32, smem, &occ);
         if (e != cudaSuccess)
             return e;
-        attr_set = true;
-    }
-    static int occ_smem = -1, occ = 1; // occupancy of the last shared-memory size asked for
-    if (occ_smem != smem) {
-        int o = 0;
-        cudaError_t e =
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, gemv_i8_kernel<BITS, NT, WARPS>, WARPS * 32, smem);
-        if (e != cudaSuccess)
-            return e;
-        occ = o > 0 ? o : 1;
-        occ_smem = smem;
     }
     const int per_sm = occ < 16 / WARPS ? occ : 16 / WARPS;
     const Shape sh{a.bits, a.K, a.N, a.group};

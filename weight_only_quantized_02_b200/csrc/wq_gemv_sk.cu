@@ -8,10 +8,10 @@
 // keeps tens of KB in flight per SM without registers.  Eight consumer warps
 // own the eight 16-row blocks of a panel: each reads its 512-byte tiles from
 // shared memory -- already m16n8k16 A fragments (wq_layout.h) -- unpacks them
-// in registers and runs mma.sync with the activations as the B operand
-// ("register-level dequantize GEMV with 128-bit loads", tileInfer README,
-// Features table; the 128-bit loads are here the 16-byte shared-memory reads
-// of each lane).  INT4 groups are scaled in fp32 after their 8 MMAs and
+// in registers and runs mma.sync with the activations as the B operand (the
+// GEMV row of the tileInfer README, Features table: dequantization in
+// registers and 16-byte loads, here each lane's 16-byte shared-memory
+// reads).  INT4 groups are scaled in fp32 after their 8 MMAs and
 // INT8 rows once at the end, so weights are never rounded.
 //
 // A panel whose k-blocks are split between two or more CTAs is finished,
@@ -409,17 +409,11 @@ static cudaError_t launch_sk_t(const LinearArgs &a, void *ws, int sm_count, cuda
 {
     using C = SkCfg<BITS, MT, OCC>;
     constexpr size_t smem = 128 + (size_t)C::kStages * C::kStageBytes + 2 * C::kStages * 8 + 16;
-    static int occ = -1;
-    if (occ < 0) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_sk_kernel<BITS, MT, OCC>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int occ = 1;
+    {
+        const cudaError_t e = kernel_setup((const void *)gemv_sk_kernel<BITS, MT, OCC>, smem, kSkThreads, smem, &occ);
         if (e != cudaSuccess)
             return e;
-        int o = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, gemv_sk_kernel<BITS, MT, OCC>, kSkThreads, smem);
-        if (e != cudaSuccess)
-            return e;
-        occ = o > 0 ? o : 1;
     }
     const int per_sm = OCC < occ ? OCC : occ; // every CTA resident at once
     const Shape sh{a.bits, a.K, a.N, a.group};
@@ -530,17 +524,11 @@ static cudaError_t launch_sk_noalloc_t(const LinearArgs &a, uint32_t *cnt, float
 {
     using C = SkCfg<BITS, 1, OCC>;
     constexpr size_t smem = 128 + (size_t)C::kStages * C::kStageBytes + 2 * C::kStages * 8 + 16;
-    static int occ = -1;
-    if (occ < 0) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_sk_kernel<BITS, 1, OCC>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int occ = 1;
+    {
+        const cudaError_t e = kernel_setup((const void *)gemv_sk_kernel<BITS, 1, OCC>, smem, kSkThreads, smem, &occ);
         if (e != cudaSuccess)
             return e;
-        int o = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, gemv_sk_kernel<BITS, 1, OCC>, kSkThreads, smem);
-        if (e != cudaSuccess)
-            return e;
-        occ = o > 0 ? o : 1;
     }
     const int per_sm = OCC < occ ? OCC : occ;
     const Shape sh{a.bits, a.K, a.N, a.group};

@@ -112,6 +112,15 @@ bool gi_fits(int bits, int M, int K);
 size_t ws_bytes_gemv_i8(int M, int K, int N);
 cudaError_t launch_gemv_i8(const LinearArgs &a, int split, void *ws, int sm_count, cudaStream_t st);
 
+// Launch preparation of one kernel on the current device: raises its
+// dynamic shared-memory limit to smem_optin bytes (0: leave it) the first
+// time it is launched on that device, and returns in *occ (if not NULL) its
+// resident CTAs per SM for `threads` threads and `smem` bytes of dynamic
+// shared memory (at least 1).  Both are cached per (device, kernel), under a
+// mutex: a kernel attribute belongs to one device's context, so a launch on a
+// second device repeats the set-up there.
+cudaError_t kernel_setup(const void *func, size_t smem_optin, int threads, size_t smem, int *occ);
+
 // Reads and clears the device error word of the current device.
 cudaError_t read_device_error(int *code, cudaStream_t st);
 

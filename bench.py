@@ -45,8 +45,21 @@ sys.path.insert(0, ROOT)
 
 import wq_inputs as gen  # noqa: E402
 
-DEFAULT_WORKLOAD = "w8_decode_5120x17408"
+DEFAULT_WORKLOAD = "all"
 L2_ROTATION_FACTOR = 5
+# With several workloads in one step, the copies of a small weight are capped:
+# the other workloads stream gigabytes between two steps, so every copy is
+# read from HBM once per step all the same.
+MAX_COPIES = 64
+
+
+def workload_names(spec):
+    """'all' (every workload, in the order of wq_inputs.WORKLOADS) or one name."""
+    if spec == "all":
+        return list(gen.WORKLOADS)
+    if spec not in gen.WORKLOADS:
+        raise SystemExit(f"unknown workload {spec!r}; choose 'all' or one of {list(gen.WORKLOADS)}")
+    return [spec]
 
 
 # ---------------------------------------------------------------------------
@@ -273,22 +286,32 @@ def kernel_file(variant, bits):
 
 
 def bench_ours(args, device, rank, world):
+    """Every (workload, M) of the run in one timed region: a step replays,
+    for each workload and each M, one CUDA graph of that M's calls on every
+    weight copy, with CUDA events between the graphs."""
     import torch
 
     import weight_only_quantized_02_b200 as wq
-    name = args.workload
-    cfg0 = gen.WORKLOADS[name]
-    K, N, bits, group = cfg0["K"], cfg0["N"], cfg0["bits"], cfg0["group"]
-    Ms = list(args.ms) if args.ms else list(cfg0["Ms"])
+    names = workload_names(args.workload)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    wbytes = weight_bytes(bits, K, N, group)
-    copies = max(2, math.ceil(L2_ROTATION_FACTOR * l2 / wbytes))
-    cfg, pws = build_weights(name, device, copies)
-    ws = torch.zeros(wq.wq_workspace_bytes(max(Ms), K, N, 32), dtype=torch.uint8, device=device)
+    works = []  # one dict per workload
+    for name in names:
+        cfg0 = gen.WORKLOADS[name]
+        K, N, bits, group = cfg0["K"], cfg0["N"], cfg0["bits"], cfg0["group"]
+        Ms = list(args.ms) if args.ms else list(cfg0["Ms"])
+        wbytes = weight_bytes(bits, K, N, group)
+        copies = max(2, math.ceil(L2_ROTATION_FACTOR * l2 / wbytes))
+        if len(names) > 1:
+            copies = min(copies, MAX_COPIES)
+        cfg, pws = build_weights(name, device, copies)
+        works.append(dict(name=name, K=K, N=N, bits=bits, group=group, Ms=Ms, copies=copies, pws=pws))
+    ws_need = max(wq.wq_workspace_bytes(max(w["Ms"]), w["K"], w["N"], 32) for w in works)
+    ws = torch.zeros(ws_need, dtype=torch.uint8, device=device)
     wq.wq_set_workspace(ws)
-    xs = {M: torch.from_numpy(gen.x_bf16(M, K).view(np.int16)).view(torch.bfloat16).to(device) for M in Ms}
-    ys = {M: torch.empty((M, N), dtype=torch.bfloat16, device=device) for M in Ms}
-    choices = {M: wq.wq_get_choice(M, K, N, bits, group) for M in Ms}
+    for w in works:
+        w["xs"] = {M: torch.from_numpy(gen.x_bf16(M, w["K"]).view(np.int16)).view(torch.bfloat16).to(device)
+                   for M in w["Ms"]}
+        w["ys"] = {M: torch.empty((M, w["N"]), dtype=torch.bfloat16, device=device) for M in w["Ms"]}
 
     # the dispatcher's measured choice (the load-time tuning of the split_k
     # auto-tune in Mit han lab Llm awq Kernel Selection Thresholds), untimed;
@@ -298,42 +321,48 @@ def bench_ours(args, device, rank, world):
         if wq.wq_load_tuning(args.tuning_file) != 0:
             raise RuntimeError("unreadable tuning file " + args.tuning_file)
         have = tuned_shapes(args.tuning_file)
-        choices = {M: wq.wq_get_choice(M, K, N, bits, group) for M in Ms}
-    if args.choice is not None:
-        # one fixed (variant, split) for every M: a single kernel to profile
-        for M in Ms:
-            wq.wq_set_choice(M, K, N, bits, group, args.choice[0], args.choice[1])
-        choices = {M: wq.wq_get_choice(M, K, N, bits, group) for M in Ms}
-    elif args.tune and any((M, K, N, bits, group) not in have for M in Ms):
-        for M in Ms:
-            if (M, K, N, bits, group) not in have:
-                choices[M] = wq.wq_tune(xs[M], pws[0], ys[M], warmup=2, iters=7)
-        if args.tuning_file:
-            wq.wq_save_tuning(args.tuning_file)
+    tuned_any = False
+    for w in works:
+        K, N, bits, group = w["K"], w["N"], w["bits"], w["group"]
+        for M in w["Ms"]:
+            key = (M, K, N, bits, group)
+            if args.choice is not None:
+                # one fixed (variant, split): a single kernel to profile
+                wq.wq_set_choice(M, K, N, bits, group, args.choice[0], args.choice[1])
+            elif args.tune and key not in have:
+                wq.wq_tune(w["xs"][M], w["pws"][0], w["ys"][M], warmup=2, iters=7)
+                tuned_any = True
+        w["choices"] = {M: wq.wq_get_choice(M, K, N, bits, group) for M in w["Ms"]}
+    if tuned_any and args.tuning_file:
+        wq.wq_save_tuning(args.tuning_file)
 
-    calls = [(M, c) for M in Ms for c in range(copies)]  # one step
     stream = torch.cuda.Stream(device)
     P = max(1, min(args.steps, 64))  # event sets: per-launch times of the last P steps
 
     # warm the launch path before capture (attributes, tensor maps)
     with torch.cuda.stream(stream):
-        for M, c in calls:
-            wq.wq_linear(xs[M], pws[c], y=ys[M], stream=stream)
+        for w in works:
+            for M in w["Ms"]:
+                for c in range(w["copies"]):
+                    wq.wq_linear(w["xs"][M], w["pws"][c], y=w["ys"][M], stream=stream)
     torch.cuda.synchronize(device)
 
-    # one CUDA graph per M: its calls on every weight copy back to back (as
-    # the layers of a decode step run, the next launch may start while the
-    # previous one drains); events recorded on the stream between the graphs
-    # give each M's average launch duration inside the timed region
-    graphs = []
-    for M in Ms:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for c in range(copies):
-                wq.wq_linear(xs[M], pws[c], y=ys[M], stream=stream)
-        graphs.append(g)
+    # one CUDA graph per (workload, M): its calls on every weight copy back to
+    # back (as the layers of a decode step run, the next launch may start
+    # while the previous one drains); events recorded on the stream between
+    # the graphs give each one's average launch duration inside the timed
+    # region
+    graphs, points = [], []
+    for w in works:
+        for M in w["Ms"]:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for c in range(w["copies"]):
+                    wq.wq_linear(w["xs"][M], w["pws"][c], y=w["ys"][M], stream=stream)
+            graphs.append(g)
+            points.append((w, M))
     torch.cuda.synchronize(device)
-    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(len(Ms) + 1)] for _ in range(P)]
+    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)] for _ in range(P)]
 
     def run_step(s):
         evs = evsets[s % P] if s is not None else None
@@ -354,10 +383,10 @@ def bench_ours(args, device, rank, world):
         while time.time() - t0 < args.soak:
             run_step(None)
             i += 1
-            if i % 20 == 0:
+            if i % 4 == 0:
                 torch.cuda.synchronize(device)
-        for w in range(args.warmup):
-            run_step(w)
+        for s in range(args.warmup):
+            run_step(s)
     torch.cuda.synchronize(device)
 
     barrier(device)
@@ -373,43 +402,50 @@ def bench_ours(args, device, rank, world):
     clocks = sampler.stop()
     elapsed_s = start.elapsed_time(end) / 1000.0
 
-    # per-launch durations from the timed region (its last P steps): each M's
-    # graph time over its launches
-    per_call_us = {M: [] for M in Ms}
+    # per-launch durations from the timed region (its last P steps): each
+    # graph's time over its launches
+    per_call_us = [[] for _ in points]
     for evs in evsets[:min(P, args.steps)]:
-        for i, M in enumerate(Ms):
-            per_call_us[M].append(evs[i].elapsed_time(evs[i + 1]) * 1000.0 / copies)
+        for i, (w, M) in enumerate(points):
+            per_call_us[i].append(evs[i].elapsed_time(evs[i + 1]) * 1000.0 / w["copies"])
 
-    step_bytes = sum(call_bytes(bits, K, N, group, M) for M, _ in calls)
-    step_flops = sum(call_flops(K, N, M) for M, _ in calls)
+    def pbytes(w, M):
+        return call_bytes(w["bits"], w["K"], w["N"], w["group"], M)
+
+    step_bytes = sum(pbytes(w, M) * w["copies"] for w, M in points)
+    step_flops = sum(call_flops(w["K"], w["N"], M) * w["copies"] for w, M in points)
     total_bytes, tmax, value_bps = aggregate(step_bytes * args.steps, elapsed_s, device)
     peaks = read_peaks()
 
     per_shape = []
-    for M in Ms:
-        us = statistics.mean(per_call_us[M])
-        b = call_bytes(bits, K, N, group, M)
-        f = call_flops(K, N, M)
+    for i, (w, M) in enumerate(points):
+        us = statistics.mean(per_call_us[i])
+        b, f = pbytes(w, M), call_flops(w["K"], w["N"], M)
+        v, sp = w["choices"][M]
+        t_roof = max(b / (peaks["hbm_gbs"] * 1e3), f / (peaks["bf16_tflops"] * 1e6))
         per_shape.append({
-            "M": M, "K": K, "N": N, "variant": kernel_name(choices[M][0], bits), "split": choices[M][1],
+            "workload": w["name"], "M": M, "K": w["K"], "N": w["N"], "bits": w["bits"], "group": w["group"],
+            "variant": kernel_name(v, w["bits"]), "split": sp, "calls_per_step": w["copies"],
             "us_per_call": round(us, 3), "gbs": round(b / us / 1e3, 1),
             "hbm_frac_of_measured": round(b / us / 1e3 / peaks["hbm_gbs"], 4),
             "hbm_frac_of_8tbs": round(b / us / 1e3 / 8000.0, 4),
             "tflops": round(f / us / 1e6, 3),
-            "roofline_frac": round(max(b / (peaks["hbm_gbs"] * 1e3), f / (peaks["bf16_tflops"] * 1e6)) / us, 4),
+            "bound": "tensor" if f / (peaks["bf16_tflops"] * 1e6) > b / (peaks["hbm_gbs"] * 1e3) else "hbm",
+            "roofline_us": round(t_roof, 3), "roofline_frac": round(t_roof / us, 4),
         })
 
-    # dominant kernel: the shape with the largest share of device time
-    share = {M: statistics.mean(per_call_us[M]) for M in Ms}
-    Mdom = max(Ms, key=lambda m: share[m])
-    dom = next(p for p in per_shape if p["M"] == Mdom)
-    vdom = choices[Mdom][0]
-    kfile = kernel_file(vdom, bits)
-    summary = f"{dom['variant']}_{name}.md"
+    # dominant kernel: the (workload, M) with the largest share of device time
+    shares = [statistics.mean(per_call_us[i]) * w["copies"] for i, (w, M) in enumerate(points)]
+    idom = max(range(len(points)), key=lambda i: shares[i])
+    wdom, Mdom = points[idom]
+    dom = per_shape[idom]
+    vdom = wdom["choices"][Mdom][0]
+    kfile = kernel_file(vdom, wdom["bits"])
+    summary = f"{dom['variant']}_{wdom['name']}.md"
     traffic = profile_traffic(kfile, summary, Mdom)
-    # the dominant call's bound: HBM unless its flops take longer than its bytes
-    b_dom, f_dom, us_dom = call_bytes(bits, K, N, group, Mdom), call_flops(K, N, Mdom), share[Mdom]
-    if f_dom / (peaks["bf16_tflops"] * 1e12) > b_dom / (peaks["hbm_gbs"] * 1e9):
+    b_dom, f_dom = pbytes(wdom, Mdom), call_flops(wdom["K"], wdom["N"], Mdom)
+    us_dom = statistics.mean(per_call_us[idom])
+    if dom["bound"] == "tensor":
         achieved = f_dom / (us_dom * 1e-6) / 1e12
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
                     "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": traffic,
@@ -421,48 +457,51 @@ def bench_ours(args, device, rank, world):
                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                     "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)",
                     "frac_of_8tbs": round(achieved / 8000.0, 4)}
-    roofline.update({"kernel": f"{dom['variant']} M={Mdom} split={dom['split']}",
+    roofline.update({"kernel": f"{dom['variant']} {wdom['name']} M={Mdom} split={dom['split']}",
+                     "share_of_step": round(shares[idom] / sum(shares), 4),
                      "traffic_source": f"profiles/{summary}" if traffic is not None else None,
                      "algorithmic_bytes_per_launch": b_dom})
 
-    e2e = bench_e2e(args, device, xs, pws, Ms, calls, bits, K, N, group, stream)
+    e2e = bench_e2e(args, device, works, stream)
     wq.wq_set_workspace(None)
     return {
         "value": value_bps / 1e9, "ms_per_step": tmax / args.steps * 1e3, "per_shape": per_shape,
-        "roofline": roofline, "clocks": clocks, "e2e": e2e, "copies": copies,
-        "gpu_launches": args.steps * len(calls), "tflops": step_flops * args.steps * world / tmax / 1e12,
-        "choices": {str(M): list(choices[M]) for M in Ms}, "l2_bytes": l2, "Ms": Ms,
+        "roofline": roofline, "clocks": clocks, "e2e": e2e, "works": works,
+        "gpu_launches": args.steps * sum(w["copies"] for w, _ in points),
+        "tflops": step_flops * args.steps * world / tmax / 1e12, "l2_bytes": l2,
     }
 
 
-def bench_e2e(args, device, xs, pws, Ms, calls, bits, K, N, group, stream):
+def bench_e2e(args, device, works, stream):
     """Same metric through the public call with host buffers.  Every step
-    copies its inputs (the activations of each M) in from pinned host memory,
-    runs its calls, and copies every call's output back to pinned host
-    memory: each output on a side stream as soon as its call is done, so the
-    copies overlap the following calls, as a decode runtime overlaps them.
-    The step is captured once as a CUDA graph (fork and join included);
-    every replay performs every copy."""
+    copies its inputs (the activations of every workload and M) in from
+    pinned host memory, runs its calls, and copies every call's output back
+    to pinned host memory: each output on a side stream as soon as its call
+    is done, so the copies overlap the following calls, as a decode runtime
+    overlaps them.  The step is captured once as a CUDA graph (fork and join
+    included); every replay performs every copy."""
     import torch
 
     import weight_only_quantized_02_b200 as wq
-    hx = {M: xs[M].cpu().pin_memory() for M in Ms}
-    hy = {(M, c): torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M, c in calls}
-    dx = {M: torch.empty_like(xs[M]) for M in Ms}
-    dy = {(M, c): torch.empty((M, N), dtype=torch.bfloat16, device=device) for M, c in calls}
+    calls = [(wi, M, c) for wi, w in enumerate(works) for M in w["Ms"] for c in range(w["copies"])]
+    hx = {(wi, M): works[wi]["xs"][M].cpu().pin_memory() for wi, w in enumerate(works) for M in w["Ms"]}
+    dx = {k: torch.empty_like(works[k[0]]["xs"][k[1]]) for k in hx}
+    hy = {k: torch.empty((k[1], works[k[0]]["N"]), dtype=torch.bfloat16).pin_memory() for k in calls}
+    dy = {k: torch.empty((k[1], works[k[0]]["N"]), dtype=torch.bfloat16, device=device) for k in calls}
     side = torch.cuda.Stream(device)
     steps = max(1, min(args.steps, args.e2e_steps))
 
     def step():
-        for M in Ms:
-            dx[M].copy_(hx[M], non_blocking=True)
-        for M, c in calls:
-            wq.wq_linear(dx[M], pws[c], y=dy[(M, c)], stream=stream)
+        for k in hx:
+            dx[k].copy_(hx[k], non_blocking=True)
+        for k in calls:
+            wi, M, c = k
+            wq.wq_linear(dx[(wi, M)], works[wi]["pws"][c], y=dy[k], stream=stream)
             done = torch.cuda.Event()
             done.record(stream)
             side.wait_event(done)
             with torch.cuda.stream(side):
-                hy[(M, c)].copy_(dy[(M, c)], non_blocking=True)
+                hy[k].copy_(dy[k], non_blocking=True)
         stream.wait_stream(side)
 
     with torch.cuda.stream(stream):
@@ -487,68 +526,95 @@ def bench_e2e(args, device, xs, pws, Ms, calls, bits, K, N, group, stream):
     barrier(device)
     t = a.elapsed_time(b) / 1000.0
     # the outputs that came back match the device results of the last replay
-    for M, c in calls[:1]:
-        if not torch.equal(hy[(M, c)].view(torch.int16), dy[(M, c)].cpu().view(torch.int16)):
+    for k in (calls[0], calls[-1]):
+        if not torch.equal(hy[k].view(torch.int16), dy[k].cpu().view(torch.int16)):
             raise RuntimeError("end-to-end outputs differ from the device results")
-    step_bytes = sum(call_bytes(bits, K, N, group, M) for M, _ in calls)
+    step_bytes = sum(call_bytes(works[wi]["bits"], works[wi]["K"], works[wi]["N"], works[wi]["group"], M)
+                     for wi, M, _ in calls)
     total, tmax, v = aggregate(step_bytes * steps, t, device)
     return {"value": round(v / 1e9, 1), "unit": "GB/s",
-            "h2d_bytes_per_step": sum(2 * M * K for M in Ms),
-            "d2h_bytes_per_step": sum(2 * M * N for M, _ in calls), "steps": steps,
+            "h2d_bytes_per_step": sum(2 * k[1] * works[k[0]]["K"] for k in hx),
+            "d2h_bytes_per_step": sum(2 * M * works[wi]["N"] for wi, M, _ in calls), "steps": steps,
             "note": "wq_linear with pinned host buffers: the step's activations copied in, every call's output "
                     "copied out on a side stream overlapping the next calls; the step replayed as one CUDA graph"}
 
 
-def cpu_baseline(name, budget_s=15.0, rows_cap=None):
+class OracleSample:
+    """The CPU oracle as it stands on a bounded sample of one workload: every
+    M of one step on the first `rows` output channels."""
+
+    def __init__(self, name, rows=None):
+        import oracle
+        self.oracle = oracle
+        cfg = gen.WORKLOADS[name]
+        self.name = name
+        self.K, self.N, self.bits, self.group = cfg["K"], cfg["N"], cfg["bits"], cfg["group"]
+        self.Ms = list(cfg["Ms"])
+        self.direct = cfg.get("direct", False)
+        self.xs = {M: gen.x_bf16(M, self.K) for M in self.Ms}
+        self.set_rows(rows or min(self.N, 256))
+
+    def set_rows(self, rows):
+        rows = max(16, min(self.N, int(rows)) // 16 * 16)
+        self.rows = rows
+        if self.direct:
+            q, s = gen.direct_int8(self.K, self.N)
+            self.c = (q[:rows], s[:rows])
+        else:
+            W = gen.W_f32(0, rows, self.K)
+            self.c = self.oracle.quant_int8(W) if self.bits == 8 else self.oracle.quant_int4(W)
+
+    def run(self):
+        for M in self.Ms:
+            if self.bits == 8:
+                self.oracle.linear_int8(self.xs[M], self.c[0], self.c[1])
+            else:
+                self.oracle.linear_int4(self.xs[M], self.c[0], self.c[1], self.c[2])
+
+    def bytes(self):
+        """Algorithmic bytes of one pass, scaled to the sampled channels."""
+        return sum(call_bytes(self.bits, self.K, self.N, self.group, M) for M in self.Ms) * self.rows / self.N
+
+    def describe(self):
+        return f"{self.name}: {self.rows} of {self.N} output channels, M in {self.Ms}"
+
+
+def sized_samples(names, budget_s):
+    """One OracleSample per workload, each sized to about budget_s / len(names)
+    seconds of oracle work per pass (at most the whole layer)."""
+    each = budget_s / max(1, len(names))
+    out = []
+    for name in names:
+        smp = OracleSample(name)
+        t0 = time.perf_counter()
+        smp.run()
+        tp = time.perf_counter() - t0
+        smp.set_rows(smp.rows * each / max(tp, 1e-6))
+        out.append(smp)
+    return out
+
+
+def cpu_baseline(names, budget_s=16.0):
     """The CPU oracle as it stands, on the host cores, over a bounded sample
-    of the workload: every M of one step, on a contiguous block of output
-    channels sized to about `budget_s` seconds of work."""
+    of the run's workloads: every M of each workload on a contiguous block of
+    output channels sized to about budget_s seconds of work in all, passed
+    over again until about budget_s / 2 seconds have gone."""
     import oracle
-    cfg = gen.WORKLOADS[name]
-    K, N, bits, group = cfg["K"], cfg["N"], cfg["bits"], cfg["group"]
     threads = len(os.sched_getaffinity(0))
     oracle.set_threads(threads)
-    xs = {M: gen.x_bf16(M, K) for M in cfg["Ms"]}
-
-    def codes(n0, n1):
-        if cfg.get("direct"):
-            q, s = gen.direct_int8(K, N)
-            return q[n0:n1], s[n0:n1]
-        W = gen.W_f32(n0, n1, K)
-        return oracle.quant_int8(W) if bits == 8 else oracle.quant_int4(W)
-
-    def run(c):
-        for M in cfg["Ms"]:
-            if bits == 8:
-                oracle.linear_int8(xs[M], c[0], c[1])
-            else:
-                oracle.linear_int4(xs[M], c[0], c[1], c[2])
-
-    probe = min(N, 512)
-    c = codes(0, probe)
-    t0 = time.perf_counter()
-    run(c)
-    tp = time.perf_counter() - t0
-    rows = int(min(N, max(probe, probe * budget_s / max(tp, 1e-6))))
-    if rows_cap:
-        rows = min(rows, rows_cap)
-    rows = max(16, rows // 16 * 16)
-    c = codes(0, rows)
-    # the whole sample again until about budget_s / 2 seconds have passed
-    # (at least once): a layer the oracle finishes in milliseconds is timed
-    # over many passes
+    smps = sized_samples(names, budget_s)
     reps, t = 0, 0.0
     t0 = time.perf_counter()
     while reps == 0 or (t < budget_s / 2 and reps < 10000):
-        run(c)
+        for smp in smps:
+            smp.run()
         reps += 1
         t = time.perf_counter() - t0
-    frac = rows / N
-    b = sum(call_bytes(bits, K, N, group, M) for M in cfg["Ms"]) * frac * reps
+    b = sum(smp.bytes() for smp in smps) * reps
     return {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
             "seconds": round(t, 3),
-            "sample": f"{rows} of {N} output channels, all M in {list(cfg['Ms'])}, one weight copy, "
-                      f"{reps} pass(es); bytes scaled by {rows}/{N}"}
+            "sample": "; ".join(smp.describe() for smp in smps) + f"; one weight copy, {reps} pass(es); "
+                      "bytes scaled to the sampled channels"}
 
 
 # ---------------------------------------------------------------------------
@@ -558,30 +624,16 @@ def cpu_baseline(name, budget_s=15.0, rows_cap=None):
 def bench_reference(args, rank, world):
     if rank != 0:
         return None
-    name = args.workload
     import oracle
-    cfg = gen.WORKLOADS[name]
-    K, N, bits, group = cfg["K"], cfg["N"], cfg["bits"], cfg["group"]
+    names = workload_names(args.workload)
     threads = len(os.sched_getaffinity(0))
     oracle.set_threads(threads)
     # size each step so the whole run stays within about 90 s of CPU time
-    budget = 90.0 / max(1, args.steps + args.warmup)
-    base = cpu_baseline(name, budget_s=budget)
-    rows = int(base["sample"].split()[0])
-    xs = {M: gen.x_bf16(M, K) for M in cfg["Ms"]}
-    if cfg.get("direct"):
-        q, s = gen.direct_int8(K, N)
-        c = (q[:rows], s[:rows])
-    else:
-        W = gen.W_f32(0, rows, K)
-        c = oracle.quant_int8(W) if bits == 8 else oracle.quant_int4(W)
+    smps = sized_samples(names, 90.0 / max(1, args.steps + args.warmup))
 
     def step():
-        for M in cfg["Ms"]:
-            if bits == 8:
-                oracle.linear_int8(xs[M], c[0], c[1])
-            else:
-                oracle.linear_int4(xs[M], c[0], c[1], c[2])
+        for smp in smps:
+            smp.run()
 
     for _ in range(args.warmup):
         step()
@@ -589,20 +641,32 @@ def bench_reference(args, rank, world):
     for _ in range(args.steps):
         step()
     t = time.perf_counter() - t0
-    b = sum(call_bytes(bits, K, N, group, M) for M in cfg["Ms"]) * rows / N * args.steps
-    value = b / t / 1e9
-    sample = f"{rows} of {N} output channels per step, all M in {list(cfg['Ms'])}"
+    value = sum(smp.bytes() for smp in smps) * args.steps / t / 1e9
+    sample = "; ".join(smp.describe() for smp in smps) + " per step"
     return {
-        "metric": "effective weight GB/s (W8A16/W4A16 linear, algorithmic bytes)", "impl": "reference",
+        "metric": METRIC, "impl": "reference",
         "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": name, "K": K, "N": N, "bits": bits, "group": group, "Ms": list(cfg["Ms"]),
-                   "parallelism": "cpu oracle, rank 0 only"},
+        "config": dict(run_config(names), parallelism="cpu oracle, rank 0 only"),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+
+
+METRIC = "effective weight GB/s (W8A16/W4A16 linear, algorithmic bytes)"
+
+
+def run_config(names):
+    """The run's workloads, named by what they are."""
+    ws = []
+    for name in names:
+        c = gen.WORKLOADS[name]
+        ws.append({"name": name, "bits": c["bits"], "group": c["group"], "K": c["K"], "N": c["N"],
+                   "Ms": list(c["Ms"])})
+    label = ("all five workloads: " if len(names) == len(gen.WORKLOADS) else "") + ", ".join(names)
+    return {"workload": label, "workloads": ws}
 
 
 # ---------------------------------------------------------------------------
@@ -640,31 +704,32 @@ def main():
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     init_dist(world, "nccl")
-    names = list(gen.WORKLOADS) if args.workload == "all" else [args.workload]
-    for name in names:
-        args.workload = name
-        r = bench_ours(args, device, rank, world)
-        if rank != 0:
-            continue
-        cfg = gen.WORKLOADS[name]
+    names = workload_names(args.workload)
+    r = bench_ours(args, device, rank, world)
+    if rank == 0:
+        conf = run_config(names)
+        conf.update({
+            "weight_copies": {w["name"]: w["copies"] for w in r["works"]},
+            "l2": f"inputs larger than L2: each workload's weights rotated over copies spanning > "
+                  f"{L2_ROTATION_FACTOR}x the {r['l2_bytes'] // 2**20} MiB L2 (at most {MAX_COPIES} copies of a "
+                  f"small weight when other workloads stream between steps); no flush",
+            "parallelism": "replicas" if world > 1 else "single GPU",
+            "timing": "one CUDA graph per (workload, M) of its calls back to back, CUDA events between the "
+                      "graphs, max over ranks"})
         line = {
-            "metric": "effective weight GB/s (W8A16/W4A16 linear, algorithmic bytes)",
+            "metric": METRIC,
             "value": round(r["value"], 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0,1) activations, N(0,0.02^2) weights quantized on device)",
-            "config": {"workload": name, "K": cfg["K"], "N": cfg["N"], "bits": cfg["bits"],
-                       "group": cfg["group"], "Ms": r["Ms"], "weight_copies": r["copies"],
-                       "l2": f"weights rotated over {r['copies']} copies (> {L2_ROTATION_FACTOR}x L2 of "
-                             f"{r['l2_bytes'] // 2**20} MiB); no flush",
-                       "parallelism": "replicas" if world > 1 else "single GPU", "timing": "one CUDA graph "
-                       "per M (its calls back to back), CUDA events between the graphs, max over ranks"},
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02^2) weights quantized on device; the direct "
+                    "W8A16 case draws its codes and scales)",
+            "config": conf,
             "tflops": round(r["tflops"], 2), "per_shape": r["per_shape"], "roofline": r["roofline"],
             "clocks": r["clocks"], "e2e": r["e2e"], "gpu_launches": r["gpu_launches"],
-            "dispatch": r["choices"],
+            "dispatch": {f"{w['name']} M={M}": list(w["choices"][M]) for w in r["works"] for M in w["Ms"]},
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(name)
+            line["cpu_baseline"] = cpu_baseline(names)
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():

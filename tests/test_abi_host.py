@@ -66,16 +66,18 @@ def test_packed_bytes_rejects(bits, K, N, group, status):
 
 
 def test_workspace_bytes():
-    # 8 tickets per 128-row panel + 2 grid counters, padded to 256 bytes, + the largest of the
-    # split-K GEMM's fp32 partials [S][M][N], the stream-K kernels' per-CTA
+    # counters: 8 tickets per 128-row panel + 2 grid counters + 64 two-word
+    # residual sums of the integer path's exactness guard, padded to 256 bytes
+    # (N = 5120: 40 panels -> 450 words -> 2048 bytes); then the largest of
+    # the split-K GEMM's fp32 partials [S][M][N], the stream-K kernels' per-CTA
     # panel partials [512 CTAs][2][128 rows][token tile] and the integer
     # path's digits + int32 partials (smaller than the stream-K GEMM's here)
-    assert wq.wq_workspace_bytes(128, 5120, 5120, 32) == 1536 + 32 * 128 * 5120 * 4
-    assert wq.wq_workspace_bytes(64, 5120, 5120, 1) == 1536 + 512 * 2 * 128 * 64 * 4
-    assert wq.wq_workspace_bytes(16, 5120, 5120, 1) == 1536 + 512 * 2 * 128 * 16 * 4
+    assert wq.wq_workspace_bytes(128, 5120, 5120, 32) == 2048 + 32 * 128 * 5120 * 4
+    assert wq.wq_workspace_bytes(64, 5120, 5120, 1) == 2048 + 512 * 2 * 128 * 64 * 4
+    assert wq.wq_workspace_bytes(16, 5120, 5120, 1) == 2048 + 512 * 2 * 128 * 16 * 4
     # M = 8: the integer GEMV's per-warp partials 448 CTAs x 8 warps x 2 x 16 rows x 24 x 4 bytes
-    assert wq.wq_workspace_bytes(8, 5120, 5120, 1) == 1536 + 448 * 8 * 2 * 16 * 24 * 4
-    assert wq.wq_workspace_bytes(1, 5120, 17408, 1) == 4608 + 512 * 2 * 128 * 16 * 4  # 136 panels -> 1090 words -> 4608 bytes
+    assert wq.wq_workspace_bytes(8, 5120, 5120, 1) == 2048 + 448 * 8 * 2 * 16 * 24 * 4
+    assert wq.wq_workspace_bytes(1, 5120, 17408, 1) == 5120 + 512 * 2 * 128 * 16 * 4  # 136 panels -> 1218 words
     # integer path, M = 1 (16 digit rows): int32 partials 160 CTAs x 2 x 16 x 128
     assert 160 * 2 * 16 * 128 * 4 < 512 * 2 * 128 * 16 * 4
     assert wq.wq_workspace_bytes(0, 5120, 5120, 4) == 0

@@ -19,8 +19,8 @@ import torch
 import oracle
 import wq_inputs as gen
 import weight_only_quantized_02_b200 as wq
-from wqtest_helpers import (assert_parity, bf16_dev, dev, i8_fixed_point, oracle_linear, pack_canonical_int4,
-                            pack_canonical_int8, quantize_and_pack, to_dev, workspace, y_host)
+from wqtest_helpers import (assert_parity, bf16_dev, dev, extreme_rows, i8_fixed_point, oracle_linear, outlier_rows,
+                            pack_canonical_int4, pack_canonical_int8, quantize_and_pack, to_dev, workspace, y_host)
 
 pytestmark = pytest.mark.gpu
 
@@ -96,12 +96,22 @@ def test_repeated_dispatch_resets_tickets(weight, ws):
             (I8, 5, 1), (I8, 40 if bits == 8 else 30, 1), (GEMV, 3, 2), (I8, 1, 1), (GI, 1, 2), (GI, 8, 1),
             (GEMM_SK, 7, 1), (GI, 4, 1), (I8, 3, 1), (GI, 6, 2)]
     runs += [(GEMM, 16, 2)]
+    # a workspace of its own inside a larger buffer: 4 KiB of canaries on each
+    # side catch any partial or counter written outside the declared size (the
+    # stream-K fix-ups index partials by computed contributor ids)
+    need = wq.wq_workspace_bytes(128, K, N, 32)
+    buf = torch.full((need + 8192,), 0xA5, dtype=torch.uint8, device=dev())
+    own = buf[4096:4096 + need]
+    own.zero_()
     for variant, M, split in runs:
         x = gen.x_bf16(M, K)
-        y = wq.wq_linear_forced(bf16_dev(x), pw, variant, split)
+        y = wq.wq_linear_ex(bf16_dev(x), pw, variant, split, ws=own)
         assert_parity(y_host(y), oracle_linear(x, canon, bits), f"variant={variant} M={M} split={split}")
-    counters = ws[: 4 * (8 * ((N + 127) // 128) + 2)].view(torch.int32)  # tickets + the integer path's grid counters
+    torch.cuda.synchronize()
+    # tickets, the integer path's grid counters and its residual sums (one 64-bit word per token row)
+    counters = own[: 4 * (8 * ((N + 127) // 128) + 2 + 2 * 64)].view(torch.int32)
     assert int(counters.abs().sum()) == 0
+    assert bool((buf[:4096] == 0xA5).all()) and bool((buf[4096 + need:] == 0xA5).all())
 
 
 # ---------------------------------------------------------------------------
@@ -151,8 +161,10 @@ def test_one_hot_int8_weights_exact(ws):
     for variant, split in _all_cases(M, K, 8):
         y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
         if variant in INTEGER:
-            # exact on its fixed-point activations, and within the layer's tolerance of the oracle
-            assert np.array_equal(y, _i8_want_one_hot(x, q, s)), (variant, split)
+            # exact on its fixed-point activations (or, where the exactness guard
+            # recomputed an output, the oracle's value), and within the layer's
+            # tolerance of the oracle
+            assert np.all((y == _i8_want_one_hot(x, q, s)) | (y == want)), (variant, split)
             assert_parity(y, oracle.linear_int8(x, q, s), "one-hot int8 weights, integer path")
         else:
             assert np.array_equal(y, want), (variant, split)
@@ -193,10 +205,10 @@ def test_one_hot_int4_weights_exact(ws):
     for variant, split in _all_cases(M, K, 4):
         y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
         if variant == I8:
-            assert np.array_equal(y, want_i8), (variant, split)
+            assert np.all((y == want_i8) | (y == want)), (variant, split)
             assert_parity(y, oracle.linear_int4(x, q, s, z), "one-hot int4 weights, integer path")
         elif variant == GI:
-            assert np.all((y == want_gi) | (y == want_gi32)), (variant, split)
+            assert np.all((y == want_gi) | (y == want_gi32) | (y == want)), (variant, split)
             assert_parity(y, oracle.linear_int4(x, q, s, z), "one-hot int4 weights, integer GEMV")
         else:
             assert np.array_equal(y, want), (variant, split)
@@ -223,7 +235,41 @@ def test_identity_weights_reproduce_x(bits, ws):
     want_i8 = oracle.bf16_to_f64(oracle.bf16_rne_of(i8_fixed_point(x)))
     for variant, split in _all_cases(M, K, bits):
         y = y_host(wq.wq_linear_forced(bf16_dev(x), pw, variant, split))
-        assert np.array_equal(y, want_i8 if variant in INTEGER else want), (variant, split)
+        if variant in INTEGER:
+            # The integer paths round activations more than 2^14 below their
+            # row's largest to the row's fixed-point grid, so y = x holds
+            # bit for bit only for the others: here y is x on that grid (or
+            # x itself where the exactness guard recomputed the output), and
+            # within the layer's tolerance of the oracle's y = x.
+            assert np.all((y == want_i8) | (y == want)), (variant, split)
+            assert_parity(y, want, f"identity weights, integer path variant={variant} split={split}")
+        else:
+            assert np.array_equal(y, want), (variant, split)
+
+
+@pytest.mark.parametrize("M", [4, 16, 64])
+def test_wide_range_rows_all_variants(weight, ws, M):
+    """Rows with outliers 2^12 .. 2^16 above N(0,1) values, rows around
+    2^-100 and zero rows, through every variant and split; the integer
+    variants also on rows holding bf16's largest and smallest normals (the
+    fp32-accumulating kernels keep x q within the binary32 range, which such
+    rows leave)."""
+    bits, K, N, pw, canon = weight
+    x = outlier_rows(K, M)
+    x[1::4] = gen.f32_to_bf16_bits(oracle.bf16_to_f64(x[1::4]).astype(np.float32) * np.float32(2.0 ** -100))
+    x[3::8] = 0
+    y_ref = oracle_linear(x, canon, bits)
+    xd = bf16_dev(x)
+    for variant, split in _cases(M, K, bits):
+        y = wq.wq_linear_forced(xd, pw, variant, split)
+        assert_parity(y_host(y), y_ref, f"wide range bits={bits} M={M} variant={variant} split={split}")
+    xe = np.concatenate([extreme_rows(K)] * ((M + 3) // 4))[:M]
+    ye_ref = oracle_linear(xe, canon, bits)
+    xed = bf16_dev(xe)
+    for variant, split in _cases(M, K, bits):
+        if variant in INTEGER:
+            y = wq.wq_linear_forced(xed, pw, variant, split)
+            assert_parity(y_host(y), ye_ref, f"extremes bits={bits} M={M} variant={variant} split={split}")
 
 
 @pytest.mark.parametrize("bits", [8, 4])

@@ -96,3 +96,37 @@ def test_trailer_mismatch_is_reported():
     assert wq.wq_check_packed(bad) == -5  # WQ_ERR_HEADER
     bad = wq.PackedWeight(pw.wq, pw.scales, None, 8, K - 32, N, 0)
     assert wq.wq_check_packed(bad) == -5
+
+
+def _trailer_word(pw, i):
+    """32-bit word i of the 64-byte trailer after the packed weights."""
+    wb = pw.wq.numel() - 64
+    return int(pw.wq[wb + 4 * i: wb + 4 * i + 4].cpu().numpy().view(np.uint32)[0])
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_trailer_weight_bound(bits):
+    """The trailer's bound on max |w| that the integer paths' exactness guard
+    reads: INT8 the largest 128 s, INT4 the largest max(z, 15 - z) s of any
+    group; either way at least the largest dequantized magnitude."""
+    K, N = (1024, 272) if bits == 8 else (1152, 272)
+    W = _adversarial(K, N)
+    Wd = torch.from_numpy(W).to(dev())
+    if bits == 8:
+        q, s = wq.wq_quantize_int8(Wd)
+        pw = wq.wq_pack_int8(q, s)
+        s_h = oracle.bf16_to_f64(bits_u16(s))
+        want = np.float32(np.max(128.0 * s_h))
+        w = oracle.dequant_int8(q.cpu().numpy(), bits_u16(s))
+    else:
+        q, s, z = wq.wq_quantize_int4(Wd)
+        pw = wq.wq_pack_int4(q, s, z)
+        s_h = oracle.bf16_to_f64(bits_u16(s))
+        zw = bits_u32(z)
+        zs = np.stack([(zw[:, g // 8] >> np.uint32(4 * (g % 8))) & 0xF for g in range(K // 128)], axis=1)
+        want = np.float32(np.max(s_h * np.maximum(zs, 15 - zs)))
+        w = oracle.dequant_int4(bits_u32(q), bits_u16(s), zw, K)
+    got = np.uint32(_trailer_word(pw, 8)).view(np.float32)
+    assert got == want
+    assert np.max(np.abs(w)) <= float(got)
+    assert _trailer_word(pw, 1) == 3  # layout version

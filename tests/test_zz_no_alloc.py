@@ -10,8 +10,8 @@ This file is collected last so that a run stopping at its first failure has
 already run every other test. It passes both alone in a fresh process and
 after the other tests: the first call on the device sets the array up, and
 the array keeps the previous call's contents. So two calls in a row are
-checked, each against the existing entry point wq_linear, within the
-tolerance the other tests use.
+checked, each against the existing entry point wq_linear and against the
+CPU oracle, within the tolerance the other tests use.
 """
 import numpy as np
 import pytest
@@ -19,7 +19,7 @@ import torch
 
 import wq_inputs as gen
 import weight_only_quantized_02_b200 as wq
-from wqtest_helpers import REL_TOL, assert_parity, bf16_dev, dev, quantize_and_pack, y_host
+from wqtest_helpers import REL_TOL, assert_parity, bf16_dev, dev, oracle_linear, quantize_and_pack, y_host
 
 pytestmark = pytest.mark.gpu
 
@@ -28,13 +28,16 @@ pytestmark = pytest.mark.gpu
                                         (4, 5120, 25600, 1)])
 def test_noalloc_matches_wq_linear_twice(bits, K, N, M):
     W = gen.W_f32(0, N, K)
-    pw, _ = quantize_and_pack(W, bits)
-    x = bf16_dev(gen.x_bf16(M, K))
-    y_ref = y_host(wq.wq_linear(x, pw))  # the existing entry point
+    pw, canon = quantize_and_pack(W, bits)
+    xb = gen.x_bf16(M, K)
+    x = bf16_dev(xb)
+    y_lin = y_host(wq.wq_linear(x, pw))  # the existing entry point
+    y_orc = oracle_linear(xb, canon, bits)  # the CPU oracle
     for call in range(2):
         y = wq.wq_linear_noalloc(x, pw)
         torch.cuda.synchronize()
-        assert_parity(y_host(y), y_ref, f"noalloc call {call} bits={bits} M={M}")
+        assert_parity(y_host(y), y_lin, f"noalloc call {call} bits={bits} M={M} vs wq_linear")
+        assert_parity(y_host(y), y_orc, f"noalloc call {call} bits={bits} M={M} vs the oracle")
     assert REL_TOL == 1e-2
     assert wq.wq_device_error() == 0
 

@@ -9,6 +9,7 @@ import torch
 
 import oracle
 import weight_only_quantized_02_b200 as wq
+import wq_inputs as gen
 
 # The layer's parity bar: |y_gpu - y_ref| <= 1e-2 * max(|y_ref|, 1) elementwise,
 # y_ref the fp64 oracle, y_gpu the bf16 output (fp32 accumulation).
@@ -110,3 +111,45 @@ def i8_fixed_point(x_bits: np.ndarray, with_exponents: bool = False):
         es[m] = e
         out[m] = np.rint(np.ldexp(x[m], e)) * np.ldexp(1.0, -e)  # exact: |X| < 2^22
     return (out, es) if with_exponents else out
+
+
+# ---------------------------------------------------------------------------
+# activation rows of wide dynamic range (the integer paths' exactness guard)
+# ---------------------------------------------------------------------------
+BF16_MAX = 0x7F7F      # largest finite bf16, 3.3895e38
+BF16_MIN_NORMAL = 0x0080
+BF16_MIN_SUB = 0x0001
+
+
+def _bits_of(v: np.ndarray) -> np.ndarray:
+    return gen.f32_to_bf16_bits(np.asarray(v, np.float32))
+
+
+def outlier_rows(K: int, M: int = 4) -> np.ndarray:
+    """M N(0,1) rows, row m with one element at +-2^(12, 14, 15, 16)[m % 4]."""
+    x = oracle.bf16_to_f64(gen.x_bf16(M, K)).astype(np.float32)
+    for m in range(M):
+        p = (12, 14, 15, 16)[m % 4]
+        x[m, (977 * m + 5) % K] = (-1.0) ** m * 2.0 ** p
+    return _bits_of(x)
+
+
+def extreme_rows(K: int) -> np.ndarray:
+    """Row 0: N(0,1) with one element at bf16 max and a few at the smallest
+    normal and subnormals.  Row 1: N(0,1) scaled by 2^-100.  Row 2: zero but
+    for one element at the smallest normal.  Row 3: N(0,1) with one element at
+    -bf16 max.  One huge element per row: two of opposite products would
+    cancel, and the sum of what is left then depends on the order of the
+    binary64 additions (the oracle's among them) by more than the tolerance."""
+    base = gen.x_bf16(4, K)
+    x = base.copy()
+    x[0, 11] = BF16_MAX
+    for j, b in enumerate((BF16_MIN_NORMAL, BF16_MIN_SUB, BF16_MIN_NORMAL | 0x8000, 0x0003)):
+        x[0, 100 + 37 * j] = b
+    x[1] = _bits_of(oracle.bf16_to_f64(base[1:2]).astype(np.float32) * np.float32(2.0 ** -100))[0]
+    x[2] = 0
+    x[2, K - 1] = BF16_MIN_NORMAL
+    x[3, 7] = BF16_MAX | 0x8000
+    return x
+
+

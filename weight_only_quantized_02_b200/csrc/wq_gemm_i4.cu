@@ -63,6 +63,8 @@ struct I4Params {
     float *part;            // [G][2 slots][NR/3 tokens][128 rows] fp32
     uint32_t *cnt;          // [panels][4] tickets
     uint32_t *grid;         // [2]: digit blocks written, CTAs exited
+    unsigned long long *res; // [M] residual sums of the exactness guard
+    const uint32_t *wmax;   // max |s (q - z)| over the weight (binary32 bits, packed trailer)
 };
 
 template <int NR>
@@ -96,7 +98,8 @@ constexpr size_t i4_smem_bytes()
     // digit stage; afull, aempty per A tile; accfull, accempty per
     // accumulator) + tensor-memory slot + row maxima / exponents
     return 1024 + (size_t)C::kRingBytes +
-           (2 * C::kPStages + 2 * C::kDStages + 2 * C::kAStages + 2 * C::kTB) * 8 + 16 + 2 * kI8MaxM * 4;
+           (2 * C::kPStages + 2 * C::kDStages + 2 * C::kAStages + 2 * C::kTB) * 8 + 16 + 2 * kI8MaxM * 4 +
+           kI8MaxM * 8;
 }
 
 // Eight nibbles of one packed word (runs a, b of one row; positions
@@ -147,6 +150,7 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(accempty + TB);
     uint32_t *s_amax = s_tmem + 4;                        // [kI8MaxM]
     int *s_e = reinterpret_cast<int *>(s_amax + kI8MaxM); // [kI8MaxM]
+    double *s_rb = reinterpret_cast<double *>(s_e + kI8MaxM); // [kI8MaxM] residual bounds (8-byte aligned)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, c = blockIdx.x;
@@ -327,7 +331,9 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
         pdl_wait(); // x, y and the workspace may come from / be in use by the preceding kernel
         const int et = threadIdx.x - 64; // 0..127
         const int quad = warp & 3;
-        imma_digit_phase<NR, true>(p.x, M, p.K, KB, c, G, et, p.xd, s_amax, s_e, p.grid);
+        imma_digit_phase<NR, true>(p.x, M, p.K, KB, c, G, et, p.xd, s_amax, s_e, p.grid, p.res);
+        ok = imma_residual_bounds(M, G, et, p.grid, p.res, s_e, s_rb) && ok;
+        const double wmax = (double)__uint_as_float(__ldg(p.wmax));
 
         // ---------------- epilogue: one thread per output channel ----------------
         const int row = 32 * quad + lane;
@@ -377,15 +383,13 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
                 // panel pnl done: y when this CTA covered it whole, else partial + ticket
                 do {
                     const int lo = max(u0, pnl * KB), hi = min(u1, (pnl + 1) * KB);
-                    const int nrow = pnl * kPanelRows + row;
                     if (lo == pnl * KB && hi == (pnl + 1) * KB) {
-                        if (nrow < p.N) {
 #pragma unroll
-                            for (int m = 0; m < MM; ++m)
-                                if (m < M)
-                                    p.y[(size_t)m * p.N + nrow] =
-                                        __bfloat16_as_ushort(__float2bfloat16_rn(ldexpf(acc[m], -s_e[m])));
-                        }
+                        for (int m = 0; m < MM; ++m)
+                            if (m < M) // the same across the warp
+                                imma_emit_rows<4>(p.x, p.wq, p.scales, p.zeros, p.y, p.K, KB, p.N,
+                                                  pnl * kPanelRows + 32 * quad, m, (double)acc[m] * pow2_of(-s_e[m]),
+                                                  wmax * s_rb[m], lane);
                         break;
                     }
                     const int slot = (pnl == u0 / KB) ? 0 : 1;
@@ -418,13 +422,12 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
                         for (int m = 0; m < MM; ++m)
                             tot[m] += v[m];
                     }
-                    if (nrow < p.N) {
 #pragma unroll
-                        for (int m = 0; m < MM; ++m)
-                            if (m < M)
-                                p.y[(size_t)m * p.N + nrow] =
-                                    __bfloat16_as_ushort(__float2bfloat16_rn(ldexpf(tot[m], -s_e[m])));
-                    }
+                    for (int m = 0; m < MM; ++m)
+                        if (m < M) // the same across the warp
+                            imma_emit_rows<4>(p.x, p.wq, p.scales, p.zeros, p.y, p.K, KB, p.N,
+                                              pnl * kPanelRows + 32 * quad, m, (double)tot[m] * pow2_of(-s_e[m]),
+                                              wmax * s_rb[m], lane);
                     if (lane == 0)
                         atomicExch(&p.cnt[pnl * 4 + quad], 0u);
                 } while (false);
@@ -444,10 +447,16 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
         tc_fence_after();
         tmem_dealloc(tmem, TCOLS);
     }
-    // the last CTA out resets the grid counters for the next call
-    if (threadIdx.x == 0 && atomicAdd(&p.grid[1], 1u) == (uint32_t)(G - 1)) {
-        atomicExch(&p.grid[0], 0u);
-        atomicExch(&p.grid[1], 0u);
+    // the last CTA out resets the grid counters and the residual sums for the
+    // next call (every CTA has read them before counting itself out)
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&p.grid[1], 1u) == (uint32_t)(G - 1)) {
+            for (int m = 0; m < M; ++m)
+                p.res[m] = 0ull;
+            atomicExch(&p.grid[0], 0u);
+            atomicExch(&p.grid[1], 0u);
+        }
     }
 }
 
@@ -487,6 +496,8 @@ static cudaError_t launch_i4_t(const LinearArgs &a, void *ws, int sm_count, cuda
     p.y = a.y;
     p.cnt = (uint32_t *)ws;
     p.grid = p.cnt + ws_grid_counter(a.N);
+    p.res = reinterpret_cast<unsigned long long *>(p.cnt + ws_res_counter(a.N));
+    p.wmax = trailer_wmax(a.wq, sh);
     p.xd = (uint8_t *)ws + ws_counter_bytes(a.N);
     p.part = (float *)(p.xd + (size_t)p.KB * NR * 128);
     int G = sm_count < kI8MaxCtas ? sm_count : kI8MaxCtas;

@@ -69,6 +69,7 @@ struct I8Params {
     int32_t *part;  // [G][2 slots][NR][128 rows] int32
     uint32_t *cnt;  // [panels][4] tickets
     uint32_t *grid; // [2]: digit blocks written, CTAs exited
+    unsigned long long *res; // [M] residual sums of the exactness guard
 };
 
 // Per digit-row count NR (the MMA's N): ring depth, tensor-memory columns and
@@ -96,9 +97,9 @@ template <int NR>
 constexpr size_t i8_smem_bytes()
 {
     // ring + barriers (full, empty per stage; accfull, accempty x 2) +
-    // tensor-memory slot + row maxima / exponents
+    // tensor-memory slot + row maxima / exponents + residual bounds
     return 1024 + (size_t)I8Cfg<NR>::kStages * I8Cfg<NR>::kStageBytes + (2 * I8Cfg<NR>::kStages + 4) * 8 + 16 +
-           2 * kI8MaxM * 4;
+           2 * kI8MaxM * 4 + kI8MaxM * 8;
 }
 
 template <int NR>
@@ -118,6 +119,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(accempty + 2);
     uint32_t *s_amax = s_tmem + 4;                        // [kI8MaxM] row maxima (bf16 magnitude bits)
     int *s_e = reinterpret_cast<int *>(s_amax + kI8MaxM); // [kI8MaxM] exponents e_m
+    double *s_rb = reinterpret_cast<double *>(s_e + kI8MaxM); // [kI8MaxM] residual bounds (8-byte aligned)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, c = blockIdx.x;
@@ -229,7 +231,8 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
         const int quad = warp & 3;
         const int K = p.K;
         // ---------------- activations: row maxima, then 1/G of the digit blocks ----------------
-        imma_digit_phase<NR>(p.x, M, K, KB, c, G, et, p.xd, s_amax, s_e, p.grid);
+        imma_digit_phase<NR>(p.x, M, K, KB, c, G, et, p.xd, s_amax, s_e, p.grid, p.res);
+        ok = imma_residual_bounds(M, G, et, p.grid, p.res, s_e, s_rb) && ok;
         // ---------------- epilogue: one thread per output channel ----------------
         const int row = 32 * quad + lane;
         const uint32_t tq = (uint32_t)(32 * quad) << 16;
@@ -303,14 +306,13 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
                         for (int j = 0; j < CG; ++j)
                             v[j] += pre[j];
                     }
-                    if (nrow < p.N) {
 #pragma unroll
-                        for (int t = 0; t < CG / 3; ++t) {
-                            const int m = c0 / 3 + t;
-                            if (m < M)
-                                p.y[(size_t)m * p.N + nrow] =
-                                    i8_output(v[3 * t], v[3 * t + 1], v[3 * t + 2], s_n * pow2_of(-s_e[m]));
-                        }
+                    for (int t = 0; t < CG / 3; ++t) {
+                        const int m = c0 / 3 + t; // the same across the warp
+                        if (m < M)
+                            imma_emit_rows<8>(p.x, p.wq, p.scales, nullptr, p.y, K, KB, p.N, pnl * kPanelRows + 32 * quad,
+                                              m, i8_value(v[3 * t], v[3 * t + 1], v[3 * t + 2], s_n * pow2_of(-s_e[m])),
+                                              128.0 * s_n * s_rb[m], lane);
                     }
                 } else {
 #pragma unroll
@@ -353,14 +355,13 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
                     for (int j = 0; j < CG; ++j)
                         tot[j] += v[j];
                 }
-                if (nrow < p.N) {
 #pragma unroll
-                    for (int t = 0; t < CG / 3; ++t) {
-                        const int m = c0 / 3 + t;
-                        if (m < M)
-                            p.y[(size_t)m * p.N + nrow] =
-                                i8_output(tot[3 * t], tot[3 * t + 1], tot[3 * t + 2], s_n * pow2_of(-s_e[m]));
-                    }
+                for (int t = 0; t < CG / 3; ++t) {
+                    const int m = c0 / 3 + t; // the same across the warp
+                    if (m < M)
+                        imma_emit_rows<8>(p.x, p.wq, p.scales, nullptr, p.y, K, KB, p.N, pnl * kPanelRows + 32 * quad, m,
+                                          i8_value(tot[3 * t], tot[3 * t + 1], tot[3 * t + 2], s_n * pow2_of(-s_e[m])),
+                                          128.0 * s_n * s_rb[m], lane);
                 }
             }
             if (lane == 0)
@@ -377,10 +378,16 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
         tc_fence_after();
         tmem_dealloc(tmem, TCOLS);
     }
-    // the last CTA out resets the grid counters for the next call
-    if (threadIdx.x == 0 && atomicAdd(&p.grid[1], 1u) == (uint32_t)(G - 1)) {
-        atomicExch(&p.grid[0], 0u);
-        atomicExch(&p.grid[1], 0u);
+    // the last CTA out resets the grid counters and the residual sums for the
+    // next call (every CTA has read them before counting itself out)
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&p.grid[1], 1u) == (uint32_t)(G - 1)) {
+            for (int m = 0; m < M; ++m)
+                p.res[m] = 0ull;
+            atomicExch(&p.grid[0], 0u);
+            atomicExch(&p.grid[1], 0u);
+        }
     }
 }
 
@@ -422,6 +429,7 @@ static cudaError_t launch_i8_t(const LinearArgs &a, void *ws, int sm_count, cuda
     p.y = a.y;
     p.cnt = (uint32_t *)ws;
     p.grid = p.cnt + ws_grid_counter(a.N);
+    p.res = reinterpret_cast<unsigned long long *>(p.cnt + ws_res_counter(a.N));
     p.xd = (uint8_t *)ws + ws_counter_bytes(a.N);
     p.part = (int32_t *)(p.xd + (size_t)p.KB * NR * 128);
     int G = sm_count < kI8MaxCtas ? sm_count : kI8MaxCtas;

@@ -63,6 +63,7 @@ struct GiParams {
     uint16_t *y;
     uint32_t *part; // [kGiMaxWarps][2 slots][16 rows][NR] partials
     uint32_t *cnt;  // one ticket per 16-row block
+    const uint32_t *wmax; // INT4: max |s (q - z)| over the whole weight (binary32 bits, packed trailer)
 };
 
 // Prefetch depth (items in flight per warp) by weight format.
@@ -104,7 +105,7 @@ __host__ __device__ constexpr int gi_row_stride(int K)
 //         so a lane's 32 bytes of a block are its four steps' B fragments.
 template <int BITS, int NR, int NTH>
 __device__ __forceinline__ void gi_digits(const GiParams &p, uint8_t *sd, int32_t *s_dsum, uint32_t *s_amax,
-                                          int *s_e)
+                                          int *s_e, unsigned long long *s_res)
 {
     const int et = threadIdx.x, ch = et & 7;
     const int M = p.M, K = p.K, KB = p.KB;
@@ -163,11 +164,15 @@ __device__ __forceinline__ void gi_digits(const GiParams &p, uint8_t *sd, int32_
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 pl[i][j] = 0u;
+        uint32_t units = 0;
         if (act) {
             const float sc = __uint_as_float((uint32_t)(127 + s_e[m]) << 23); // 2^e
             const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-            digit_planes(w, sc, pl);
+            float res = 0.f;
+            digit_planes(w, sc, pl, res);
+            units = residual_units(res);
         }
+        residual_add(s_res, m, units);
         if constexpr (BITS == 8) {
             if (act) {
 #pragma unroll
@@ -304,24 +309,59 @@ __host__ __device__ __forceinline__ bool gi_contrib_at(const GiParams &p, int G,
     return i == 0 || o == s0;
 }
 
+// The outputs of 16-row block n0 / 16 for every token (q = 16 m + r, row
+// n0 + r): value(q) is the integer path's y in binary64.  The exactness
+// guard (wq_imma.cuh) vouches for it or the warp recomputes that output in
+// binary64 from x and the packed codes.  All 32 lanes call it together.
+template <int BITS, class Value>
+__device__ __forceinline__ void gi_emit(const GiParams &p, int n0, const int *s_e, const unsigned long long *s_res,
+                                        Value value, int lane)
+{
+    const int M = p.M, N = p.N;
+    const float wmax4 = BITS == 4 ? __uint_as_float(__ldg(p.wmax)) : 0.f;
+    for (int q0 = 0; q0 < 16 * M; q0 += 32) {
+        const int q = q0 + lane, r = q & 15, m = q >> 4;
+        bool redo = false;
+        if (q < 16 * M) {
+            const double v = value(q);
+            const double wmax =
+                BITS == 8 ? 128.0 * (double)bf16_bits_to_float(p.scales[n0 + r]) : (double)wmax4;
+            redo = !exact_enough(v, wmax * residual_bound(s_res[m], s_e[m]));
+            if (!redo)
+                p.y[(size_t)m * N + n0 + r] = __bfloat16_as_ushort(__double2bfloat16(v));
+        }
+        for (uint32_t mask = __ballot_sync(0xffffffffu, redo); mask; mask &= mask - 1) {
+            const int src = __ffs(mask) - 1, qq = q0 + src, rr = qq & 15, mm = qq >> 4;
+            double v = packed_row_dot<BITS>(p.wq, p.scales, p.zeros, p.K, p.KB, n0 + rr, p.x + (size_t)mm * p.K, lane);
+            if constexpr (BITS == 8)
+                v *= (double)bf16_bits_to_float(p.scales[n0 + rr]);
+            if (lane == src)
+                p.y[(size_t)mm * N + n0 + rr] = __bfloat16_as_ushort(__double2bfloat16(v));
+        }
+    }
+}
+
 // One segment's output, its accumulators in red ([16 rows][NR]; INT8 int32
 // digit sums D_i, INT4 fp32 group-scaled sums A_i): y of the 16 x M outputs.
 template <int BITS, int NR>
-__device__ __forceinline__ void gi_write_y(const GiParams &p, int rb, const uint32_t *red, const int *s_e, int lane)
+__device__ __forceinline__ void gi_write_y(const GiParams &p, int rb, const uint32_t *red, const int *s_e,
+                                           const unsigned long long *s_res, int lane)
 {
-    const int M = p.M, N = p.N, n0 = 16 * rb;
-    for (int q = lane; q < 16 * M; q += 32) {
-        const int r = q & 15, m = q >> 4;
-        if constexpr (BITS == 8) {
-            const int32_t *d = reinterpret_cast<const int32_t *>(red) + r * NR + 3 * m;
-            const double sc = (double)bf16_bits_to_float(p.scales[n0 + r]) * pow2_of(-s_e[m]);
-            p.y[(size_t)m * N + n0 + r] = i8_output(d[0], d[1], d[2], sc);
-        } else {
-            const float *a = reinterpret_cast<const float *>(red) + r * NR + 3 * m;
-            const double v = ((double)a[2] * 65536.0 + (double)a[1] * 256.0 + (double)a[0]) * pow2_of(-s_e[m]);
-            p.y[(size_t)m * N + n0 + r] = __bfloat16_as_ushort(__double2bfloat16(v));
-        }
-    }
+    const int n0 = 16 * rb;
+    gi_emit<BITS>(
+        p, n0, s_e, s_res,
+        [&](int q) -> double {
+            const int r = q & 15, m = q >> 4;
+            if constexpr (BITS == 8) {
+                const int32_t *d = reinterpret_cast<const int32_t *>(red) + r * NR + 3 * m;
+                return ((double)d[2] * 65536.0 + (double)d[1] * 256.0 + (double)d[0]) *
+                       ((double)bf16_bits_to_float(p.scales[n0 + r]) * pow2_of(-s_e[m]));
+            } else {
+                const float *a = reinterpret_cast<const float *>(red) + r * NR + 3 * m;
+                return ((double)a[2] * 65536.0 + (double)a[1] * 256.0 + (double)a[0]) * pow2_of(-s_e[m]);
+            }
+        },
+        lane);
 }
 
 // A partial segment of shared row block rb ended: the warp's partial into
@@ -360,10 +400,10 @@ __device__ __forceinline__ uint32_t gi_shared_partial(const GiParams &p, int rb,
 // list: this warp's scratch of at least CPR words (partial offsets).
 template <int BITS, int NT, int WARPS>
 __device__ __forceinline__ void gi_shared_fixup(const GiParams &p, int rb, uint32_t ticket, int G, const int *s_e,
-                                                uint32_t *list, int lane)
+                                                const unsigned long long *s_res, uint32_t *list, int lane)
 {
     constexpr int NR = 8 * NT;
-    const int M = p.M, N = p.N, n0 = 16 * rb, CPR = p.CPR;
+    const int n0 = 16 * rb, CPR = p.CPR;
     int nc = 0;
     for (int base = 0; base < CPR; base += 32) {
         const int i = base + lane;
@@ -382,47 +422,52 @@ __device__ __forceinline__ void gi_shared_fixup(const GiParams &p, int rb, uint3
     __syncwarp();
     if (ticket != (uint32_t)(nc - 1))
         return;
-    for (int q = lane; q < 16 * M; q += 32) {
-        const int r = q & 15, m = q >> 4;
-        if constexpr (BITS == 8) {
-            int32_t t0 = 0, t1 = 0, t2 = 0;
-            for (int k0 = 0; k0 < nc; k0 += 4) {
-                int32_t v[4][3];
+    gi_emit<BITS>(
+        p, n0, s_e, s_res,
+        [&](int q) -> double {
+            const int r = q & 15, m = q >> 4;
+            if constexpr (BITS == 8) {
+                int32_t t0 = 0, t1 = 0, t2 = 0;
+                for (int k0 = 0; k0 < nc; k0 += 4) {
+                    int32_t v[4][3];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    v[u][0] = v[u][1] = v[u][2] = 0;
-                    if (k0 + u < nc) {
-                        const int32_t *src = reinterpret_cast<const int32_t *>(p.part + list[k0 + u]) + r * NR + 3 * m;
-                        v[u][0] = __ldcg(src);
-                        v[u][1] = __ldcg(src + 1);
-                        v[u][2] = __ldcg(src + 2);
+                    for (int u = 0; u < 4; ++u) {
+                        v[u][0] = v[u][1] = v[u][2] = 0;
+                        if (k0 + u < nc) {
+                            const int32_t *src =
+                                reinterpret_cast<const int32_t *>(p.part + list[k0 + u]) + r * NR + 3 * m;
+                            v[u][0] = __ldcg(src);
+                            v[u][1] = __ldcg(src + 1);
+                            v[u][2] = __ldcg(src + 2);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        t0 += v[u][0];
+                        t1 += v[u][1];
+                        t2 += v[u][2];
                     }
                 }
+                return ((double)t2 * 65536.0 + (double)t1 * 256.0 + (double)t0) *
+                       ((double)bf16_bits_to_float(p.scales[n0 + r]) * pow2_of(-s_e[m]));
+            } else {
+                float tot = 0.f;
+                for (int k0 = 0; k0 < nc; k0 += 4) {
+                    float v[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    t0 += v[u][0];
-                    t1 += v[u][1];
-                    t2 += v[u][2];
+                    for (int u = 0; u < 4; ++u)
+                        v[u] = k0 + u < nc
+                                   ? __ldcg(reinterpret_cast<const float *>(p.part + list[k0 + u]) + r * NR + m)
+                                   : 0.f;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (k0 + u < nc)
+                            tot += v[u];
                 }
+                return (double)tot;
             }
-            const double sc = (double)bf16_bits_to_float(p.scales[n0 + r]) * pow2_of(-s_e[m]);
-            p.y[(size_t)m * N + n0 + r] = i8_output(t0, t1, t2, sc);
-        } else {
-            float tot = 0.f;
-            for (int k0 = 0; k0 < nc; k0 += 4) {
-                float v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    v[u] = k0 + u < nc ? __ldcg(reinterpret_cast<const float *>(p.part + list[k0 + u]) + r * NR + m)
-                                       : 0.f;
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    if (k0 + u < nc)
-                        tot += v[u];
-            }
-            p.y[(size_t)m * N + n0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(tot));
-        }
-    }
+        },
+        lane);
     __syncwarp();
     if (lane == 0)
         atomicExch(&p.cnt[rb], 0u); // ready for the next call
@@ -434,39 +479,41 @@ __device__ __forceinline__ void gi_shared_fixup(const GiParams &p, int rb, uint3
 // summed in binary64) and written to y.
 template <int BITS, int NT, int WARPS>
 __device__ __forceinline__ void gi_local_out(const GiParams &p, const GiCta &ct, int c, const uint32_t *stash,
-                                             const int *s_e, int warp, int lane)
+                                             const int *s_e, const unsigned long long *s_res, int warp, int lane)
 {
     constexpr int NR = 8 * NT;
-    const int M = p.M, N = p.N, CPR = p.CPR;
+    const int CPR = p.CPR;
     const int own = p.LB * CPR, wo = WARPS - ct.ws; // own chunks and the warps that take them
     for (int j = warp; j < p.LB; j += WARPS) {
         const int wf = ct.ws + gi_owner(own, wo, j * CPR), wl = ct.ws + gi_owner(own, wo, j * CPR + CPR - 1);
         if (wf == wl)
             continue; // one warp had it whole and wrote y
         const int n0 = 16 * (c * p.LB + j);
-        for (int q = lane; q < 16 * M; q += 32) {
-            const int r = q & 15, m = q >> 4;
-            int32_t t0 = 0, t1 = 0, t2 = 0;
-            double v = 0.0;
-            for (int wi = wf; wi <= wl; ++wi) {
-                const int sl = gi_start(own, wo, wi - ct.ws) / CPR == j ? 0 : 1; // j is the warp's first row block?
-                const uint32_t *a = stash + ((size_t)wi * 2 + sl) * 16 * NR + r * NR + 3 * m;
-                if constexpr (BITS == 8) {
-                    t0 += (int32_t)a[0];
-                    t1 += (int32_t)a[1];
-                    t2 += (int32_t)a[2];
-                } else {
-                    v += (double)__uint_as_float(a[2]) * 65536.0 + (double)__uint_as_float(a[1]) * 256.0 +
-                         (double)__uint_as_float(a[0]);
+        gi_emit<BITS>(
+            p, n0, s_e, s_res,
+            [&](int q) -> double {
+                const int r = q & 15, m = q >> 4;
+                int32_t t0 = 0, t1 = 0, t2 = 0;
+                double v = 0.0;
+                for (int wi = wf; wi <= wl; ++wi) {
+                    const int sl = gi_start(own, wo, wi - ct.ws) / CPR == j ? 0 : 1; // j: the warp's first row block?
+                    const uint32_t *a = stash + ((size_t)wi * 2 + sl) * 16 * NR + r * NR + 3 * m;
+                    if constexpr (BITS == 8) {
+                        t0 += (int32_t)a[0];
+                        t1 += (int32_t)a[1];
+                        t2 += (int32_t)a[2];
+                    } else {
+                        v += (double)__uint_as_float(a[2]) * 65536.0 + (double)__uint_as_float(a[1]) * 256.0 +
+                             (double)__uint_as_float(a[0]);
+                    }
                 }
-            }
-            if constexpr (BITS == 8) {
-                const double sc = (double)bf16_bits_to_float(p.scales[n0 + r]) * pow2_of(-s_e[m]);
-                p.y[(size_t)m * N + n0 + r] = i8_output(t0, t1, t2, sc);
-            } else {
-                p.y[(size_t)m * N + n0 + r] = __bfloat16_as_ushort(__double2bfloat16(v * pow2_of(-s_e[m])));
-            }
-        }
+                if constexpr (BITS == 8)
+                    return ((double)t2 * 65536.0 + (double)t1 * 256.0 + (double)t0) *
+                           ((double)bf16_bits_to_float(p.scales[n0 + r]) * pow2_of(-s_e[m]));
+                else
+                    return v * pow2_of(-s_e[m]);
+            },
+            lane);
     }
 }
 
@@ -483,6 +530,7 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
     extern __shared__ __align__(16) uint8_t sd[];
     __shared__ uint32_t s_amax[kGiMaxM];
     __shared__ int s_e[kGiMaxM];
+    __shared__ unsigned long long s_res[kGiMaxM]; // residual bound per token row (units of 2^-24)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int G = gridDim.x, c = blockIdx.x;
@@ -561,11 +609,13 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
     }
 
     // ---------------- activations: this CTA's digit rows ----------------
-    if (threadIdx.x < kGiMaxM)
+    if (threadIdx.x < kGiMaxM) {
         s_amax[threadIdx.x] = 0u;
+        s_res[threadIdx.x] = 0ull;
+    }
     __syncthreads();
     pdl_wait(); // x, y and the workspace may come from / be in use by the preceding kernel
-    gi_digits<BITS, NR, WARPS * 32>(p, sd, s_dsum, s_amax, s_e);
+    gi_digits<BITS, NR, WARPS * 32>(p, sd, s_dsum, s_amax, s_e, s_res);
 
     // ---------------- stream the warp's chunks ----------------
     int32_t acc_i[NT][4];
@@ -706,7 +756,7 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
                 ++npend;
             } else if (whole) {
                 __syncwarp();
-                gi_write_y<BITS, NR>(p, crb, red, s_e, lane);
+                gi_write_y<BITS, NR>(p, crb, red, s_e, s_res, lane);
                 __syncwarp(); // red is rewritten by the next segment
             }
             ++crb;
@@ -717,11 +767,11 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
         }
     }
     if (npend > 0)
-        gi_shared_fixup<BITS, NT, WARPS>(p, pend_rb0, pend_t0, G, s_e, st0, lane);
+        gi_shared_fixup<BITS, NT, WARPS>(p, pend_rb0, pend_t0, G, s_e, s_res, st0, lane);
     if (npend > 1)
-        gi_shared_fixup<BITS, NT, WARPS>(p, pend_rb1, pend_t1, G, s_e, st0, lane);
+        gi_shared_fixup<BITS, NT, WARPS>(p, pend_rb1, pend_t1, G, s_e, s_res, st0, lane);
     __syncthreads(); // every warp's stash is complete
-    gi_local_out<BITS, NT, WARPS>(p, ct, c, stash, s_e, warp, lane);
+    gi_local_out<BITS, NT, WARPS>(p, ct, c, stash, s_e, s_res, warp, lane);
     pdl_launch_dependents();
 }
 
@@ -797,6 +847,7 @@ static cudaError_t launch_gi_t(const LinearArgs &a, void *ws, int sm_count, cuda
     p.y = a.y;
     p.cnt = (uint32_t *)ws;
     p.part = (uint32_t *)((uint8_t *)ws + ws_counter_bytes(a.N));
+    p.wmax = trailer_wmax(a.wq, sh);
     int G = per_sm * sm_count;
     if (G * WARPS > kGiMaxWarps)
         G = kGiMaxWarps / WARPS;

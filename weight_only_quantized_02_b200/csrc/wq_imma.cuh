@@ -45,6 +45,11 @@ __device__ __forceinline__ void umma_ss_i8(uint32_t d_tmem, uint64_t a_desc, uin
 // 2^e as a binary64, built from its exponent field (|e| < 1000 here).
 __device__ __forceinline__ double pow2_of(int e) { return __longlong_as_double((long long)(1023 + e) << 52); }
 
+__device__ __forceinline__ double i8_value(int32_t d0, int32_t d1, int32_t d2, double scale_pow2)
+{
+    return ((double)d2 * 65536.0 + (double)d1 * 256.0 + (double)d0) * scale_pow2;
+}
+
 __device__ __forceinline__ uint16_t i8_output(int32_t d0, int32_t d1, int32_t d2, double scale_pow2)
 {
     const double v = ((double)d2 * 65536.0 + (double)d1 * 256.0 + (double)d0) * scale_pow2;
@@ -87,6 +92,169 @@ __device__ __forceinline__ void digit_planes(const uint32_t (&w)[8], float s, ui
         p[0][j] = __byte_perm(a01, a23, 0x5410u) ^ 0x80808080u; // biased -> two's complement
         p[1][j] = __byte_perm(a01, a23, 0x7632u) ^ 0x80808080u;
         p[2][j] = __byte_perm(b01, b23, 0x5410u) ^ 0x80808080u;
+    }
+}
+
+// As digit_planes, and adds to `res` the sum over the 16 elements of the
+// rounding residual |x * 2^e - X|: x * 2^e is exact in binary32 (a power-of-
+// two scale of an 8-bit significand), X = F - 1.5 * 2^23 is exact, and the
+// fused multiply-add x * 2^e - X rounds nothing (|r| <= 1/2 and its bits lie
+// within those of x * 2^e).
+__device__ __forceinline__ void digit_planes(const uint32_t (&w)[8], float s, uint32_t (&p)[3][4], float &res)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
+        const float xl = fmaf(lo, s, 12582912.0f) - 12582912.0f, xh = fmaf(hi, s, 12582912.0f) - 12582912.0f;
+        res += fabsf(fmaf(lo, s, -xl)) + fabsf(fmaf(hi, s, -xh));
+    }
+    digit_planes(w, s, p);
+}
+
+// ---------------------------------------------------------------------------
+// Exactness guard of the integer path.
+//
+// Rounding x to X = round(x 2^e) changes y[m][n] by
+//     |sum_k w[n][k] (x[m][k] - X[m][k] 2^-e_m)| <= max_k |w[n][k]| * 2^-e_m * R_m,
+// R_m = sum_k |x[m][k] 2^e_m - X[m][k]| (each term <= 1/2; zero for every
+// element within 2^14 of the row's largest).  The digit phases accumulate an
+// upper bound of R_m in units of 2^-24 (an integer sum, the same in any
+// order, so every CTA takes the same decisions on every run); the epilogues
+// compare the bound with the output's tolerance and recompute, in binary64
+// straight from x and the packed codes, every output where the bound does not
+// show |y - y_exact| <= 2^-9 max(|y|, 1).  With the bf16 rounding of the
+// output that keeps every output within 2^-8 max(|y_exact|, 1) of the exact
+// sum, inside the 1e-2 relative tolerance of the layer.  A row of ordinary
+// dynamic range never takes the binary64 path; a row holding elements far
+// below its largest (an outlier 2^12 above the rest) can take it for many
+// outputs, which is slow but exact.
+// ---------------------------------------------------------------------------
+constexpr double kExactTol = 1.0 / 512.0;
+
+// A 16-element residual sum (binary32, each term <= 1/2) as an upper bound in
+// units of 2^-24: the float sum's relative error is below 2^-19, and one
+// unit more covers the ceiling.
+__device__ __forceinline__ uint32_t residual_units(float res)
+{
+    return res > 0.f ? (uint32_t)ceilf(res * 16777216.0f * 1.00001f) + 1u : 0u;
+}
+
+// Adds `units` to counter[m]: one atomic per warp when the whole warp works
+// on the same token row m (the usual case), else one per lane.  All 32
+// lanes call it together.
+__device__ __forceinline__ void residual_add(unsigned long long *counter, int m, uint32_t units)
+{
+    const int m0 = __shfl_sync(0xffffffffu, m, 0);
+    if (__all_sync(0xffffffffu, m == m0)) {
+        unsigned long long u = units;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            u += __shfl_xor_sync(0xffffffffu, u, o);
+        if ((threadIdx.x & 31) == 0 && u)
+            atomicAdd(&counter[m0], u);
+    } else if (units) {
+        atomicAdd(&counter[m], (unsigned long long)units);
+    }
+}
+
+// Bound on |y - y_exact| per unit of max|w| for token row m: units * 2^-24 * 2^-e_m.
+__device__ __forceinline__ double residual_bound(unsigned long long units, int e_m)
+{
+    return (double)units * __longlong_as_double((long long)(1023 - 24 - e_m) << 52);
+}
+
+__device__ __forceinline__ bool exact_enough(double y, double bound)
+{
+    return bound <= kExactTol * fmax(fabs(y), 1.0); // false for NaN: recomputed
+}
+
+// Binary64 dot product of token row xm (bf16, K elements) with packed weight
+// row n, dequantized from the codes (INT8: sum x q, the caller applies s[n];
+// INT4: sum_g s[n][g] sum_{k in g} x (q - z[n][g])).  All 32 lanes of the
+// warp call it together and all receive the same sum (fixed order: lane
+// partial sums, then a butterfly).  The recompute of the exactness guard.
+// Kept out of line: it runs only for the outputs the guard rejects, and the
+// callers' streaming loops stay as small as without it.
+template <int BITS>
+__device__ __noinline__ double packed_row_dot(const uint8_t *__restrict__ wq, const uint16_t *__restrict__ scales,
+                                 const uint8_t *__restrict__ zeros, int K, int KB, int n,
+                                 const uint16_t *__restrict__ xm, int lane)
+{
+    const int p = n >> 7, r = n & 127;
+    double acc = 0.0;
+    // 8 items of 16 k per 128-k block
+    for (int it = lane; it < KB * 8; it += 32) {
+        const int kb = it >> 3;
+        const size_t blk = (size_t)p * KB + kb;
+        if constexpr (BITS == 8) {
+            const int k0 = kb * kBlockK + 16 * (it & 7);
+            if (k0 >= K)
+                continue; // codes past K are zero
+            const uint4 qv = __ldg(reinterpret_cast<const uint4 *>(wq + (blk << 14) + int8_chunk_in_block(r, it & 7)));
+            const uint4 xa = __ldg(reinterpret_cast<const uint4 *>(xm + k0));
+            const uint4 xb = __ldg(reinterpret_cast<const uint4 *>(xm + k0 + 8));
+            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+            const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int q = (int)(int8_t)((qw[i >> 2] >> (8 * (i & 3))) & 0xFFu);
+                const uint32_t xb16 = (xw[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
+                acc = fma((double)q, (double)bf16_bits_to_float((uint16_t)xb16), acc);
+            }
+        } else {
+            const int tau = (it >> 2) & 1, t = it & 3;
+            const int j = r >> 4, rr = r & 15, g = rr & 7, h = rr >> 3;
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(wq + (blk << 13) + (size_t)j * 1024 + tau * 512 +
+                                                                   16 * (4 * g + t)));
+            const uint32_t w0 = h ? v.y : v.x, w1 = h ? v.w : v.z; // runs (a, b) and (c, d)
+            const int kt = kb * kBlockK + 64 * tau;
+            const double sg = (double)bf16_bits_to_float(scales[blk * kPanelRows + r]);
+            const int z = (int)((zeros[blk * 64 + (r >> 1)] >> (4 * (r & 1))) & 0xFu);
+            const int kr[4] = {kt + 4 * t, kt + 16 + 4 * t, kt + 32 + 4 * t, kt + 48 + 4 * t};
+            double part = 0.0;
+#pragma unroll
+            for (int run = 0; run < 4; ++run) {
+                const uint32_t w = run < 2 ? w0 : w1;
+                const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(xm + kr[run]));
+                const uint32_t xw[2] = {xv.x, xv.y};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int pos = int4_nibble_pos((run & 1) * 4 + e);
+                    const int q = (int)((w >> (4 * pos)) & 0xFu);
+                    const uint32_t xb16 = (xw[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+                    part = fma((double)(q - z), (double)bf16_bits_to_float((uint16_t)xb16), part);
+                }
+            }
+            acc = fma(sg, part, acc);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    return acc;
+}
+
+// Writes y[m][n] = v for the warp's 32 consecutive weight rows n = nb + lane
+// (token m the same across the warp; rows at or past N write nothing).  An
+// output whose bound the exactness guard cannot accept is recomputed by the
+// whole warp in binary64 (packed_row_dot; INT8 times s[n]).
+template <int BITS>
+__device__ __forceinline__ void imma_emit_rows(const uint16_t *__restrict__ x, const uint8_t *__restrict__ wq,
+                                               const uint16_t *__restrict__ scales, const uint8_t *__restrict__ zeros,
+                                               uint16_t *y, int K, int KB, int N, int nb, int m, double v,
+                                               double bound, int lane)
+{
+    const int n = nb + lane;
+    const bool redo = n < N && !exact_enough(v, bound);
+    if (n < N && !redo)
+        y[(size_t)m * N + n] = __bfloat16_as_ushort(__double2bfloat16(v));
+    for (uint32_t mask = __ballot_sync(0xffffffffu, redo); mask; mask &= mask - 1) {
+        const int src = __ffs(mask) - 1, nn = nb + src;
+        double r = packed_row_dot<BITS>(wq, scales, zeros, K, KB, nn, x + (size_t)m * K, lane);
+        if constexpr (BITS == 8)
+            r *= (double)bf16_bits_to_float(scales[nn]);
+        if (lane == src)
+            y[(size_t)m * N + nn] = __bfloat16_as_ushort(__double2bfloat16(r));
     }
 }
 
@@ -177,7 +345,8 @@ __device__ __forceinline__ void imma_row_maxima(const uint16_t *__restrict__ x, 
 // 16-k chunks interleaved).  An item is then a whole 32-k step.
 template <int NR, bool PAIRED = false>
 __device__ __forceinline__ void imma_digit_phase(const uint16_t *__restrict__ x, int M, int K, int KB, int c, int G,
-                                                 int et, uint8_t *xd, uint32_t *s_amax, int *s_e, uint32_t *grid)
+                                                 int et, uint8_t *xd, uint32_t *s_amax, int *s_e, uint32_t *grid,
+                                                 unsigned long long *g_res)
 {
     constexpr int BB = NR * 128;
     constexpr int W = PAIRED ? 32 : 16;  // k per item
@@ -227,12 +396,17 @@ __device__ __forceinline__ void imma_digit_phase(const uint16_t *__restrict__ x,
                     pl[h][d][q] = 0u;
         if (m < M) {
             const float sc = __uint_as_float((uint32_t)(127 + s_e[m]) << 23); // 2^e, -106 <= e <= 127
+            uint32_t units = 0;
 #pragma unroll
             for (int h = 0; h < NV / 2; ++h) {
                 const uint4 &a = v[2 * h], &b = v[2 * h + 1];
                 const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-                digit_planes(w, sc, pl[h]);
+                float res = 0.f;
+                digit_planes(w, sc, pl[h], res);
+                units += residual_units(res);
             }
+            if (units) // this CTA's share of the row's residual sum (exactness guard)
+                atomicAdd(&g_res[m], (unsigned long long)units);
         }
         uint8_t *blk = xd + (size_t)kb * BB;
 #pragma unroll
@@ -259,6 +433,27 @@ __device__ __forceinline__ void imma_digit_phase(const uint16_t *__restrict__ x,
     named_barrier_sync(1, 128);
     if (et == 0)
         red_release_gpu_add(&grid[0], 1u); // cumulative over the 128 threads' stores
+}
+
+// After the digit phase, by the same 128 threads: once every CTA has counted
+// itself on grid[0] (acquire, bounded), the residual bound of every token row
+// into s_rb (residual_bound of the grid-wide sum).  False if the wait gave up.
+__device__ __forceinline__ bool imma_residual_bounds(int M, int G, int et, const uint32_t *grid,
+                                                     const unsigned long long *g_res, const int *s_e, double *s_rb)
+{
+    bool ok = true;
+    if (et < M) {
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu(grid) < (uint32_t)G) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                ok = false;
+                break;
+            }
+        }
+        s_rb[et] = ok ? residual_bound(__ldcg(g_res + et), s_e[et]) : 0.0;
+    }
+    named_barrier_sync(1, 128);
+    return ok;
 }
 
 } // namespace wq

@@ -23,10 +23,14 @@ struct LinearArgs {
 // path (ws_grid_counter).  Every kernel leaves the counters it used at zero.
 // GEMM with S splits: partials [S][M][N].  Stream-K GEMV: partials
 // [CTAs <= kSkMaxCtas][2][128 rows][8 * ceil(M/8) tokens].
+// After the two grid counters: kResRows 64-bit residual sums of the integer
+// tensor-core path's exactness guard (one per token row), left at zero too.
 constexpr int kSkMaxCtas = 512;
-inline size_t ws_counter_words(int N) { return (size_t)((N + 127) / 128) * 8 + 2; }
+constexpr int kResRows = 64;
+inline size_t ws_counter_words(int N) { return (size_t)((N + 127) / 128) * 8 + 2 + 2 * kResRows; }
 inline size_t ws_counter_bytes(int N) { return (ws_counter_words(N) * 4 + 255) / 256 * 256; }
 inline size_t ws_grid_counter(int N) { return (size_t)((N + 127) / 128) * 8; } // word index of the first
+inline size_t ws_res_counter(int N) { return ws_grid_counter(N) + 2; }          // word index, 8-byte aligned
 inline size_t ws_bytes(int M, int N, int S)
 {
     return ws_counter_bytes(N) + (S > 1 ? (size_t)S * M * N * sizeof(float) : 0);
@@ -47,6 +51,7 @@ inline size_t ws_bytes_gemv_sk(int M, int N)
 // KB x NR x 128][partials: INT8 int32 kI8MaxCtas x 2 x NR x 128, INT4 fp32
 // kI8MaxCtas x 2 x NR/3 x 128].
 constexpr int kI8MaxM = 64;
+static_assert(kI8MaxM <= kResRows, "one residual sum per token row");
 constexpr int kI4MaxM = 32; // W4A16 on the integer path
 constexpr int kI8MaxK = 65536;
 constexpr int kI8MaxCtas = 160;

@@ -57,7 +57,7 @@ constexpr int kBlockK = 128;
 constexpr int kTileBytes = 512;
 constexpr int kTrailerBytes = 64;
 constexpr uint32_t kMagic = 0x32425157u; // "WQB2"
-constexpr uint32_t kLayoutVersion = 2;
+constexpr uint32_t kLayoutVersion = 3;
 
 struct Shape {
     int bits;  // 4 or 8
@@ -98,11 +98,23 @@ WQ_HD int int8_in_block(int r, int kk)
 // INT8: byte offset of the 16-byte chunk c of row r inside its block.
 WQ_HD int int8_chunk_in_block(int r, int c) { return (r >> 3) * 1024 + (r & 7) * 128 + (((c ^ (r & 7)) & 7) << 4); }
 
+// wmax_bits: binary32 bits of an upper bound of max |w| over the whole
+// weight, the bound the integer path's exactness guard uses: for INT4 the
+// largest max(z, 15 - z) s over the groups (the largest |q - z| a group's
+// zero point allows, times its scale), for INT8 the largest 128 s.
 struct Trailer {
     uint32_t magic, version, bits, K, N, group, layout_bytes_lo, layout_bytes_hi;
-    uint32_t reserved[8];
+    uint32_t wmax_bits;
+    uint32_t reserved[7];
 };
 static_assert(sizeof(Trailer) == kTrailerBytes, "trailer is 64 bytes");
+
+// Device address of the trailer's wmax_bits word of packed weights wq.
+inline const uint32_t *trailer_wmax(const void *wq, const Shape &sh)
+{
+    return reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(wq) + sh.weight_bytes() +
+                                              8 * sizeof(uint32_t));
+}
 
 // Position of element k (0..7 relative to the word's 8-k group) inside an
 // INT4 word: runs a = k 0..3, b = k 4..7 -> nibble positions.

@@ -202,27 +202,48 @@ __global__ void pack_int4_kernel(const uint32_t *__restrict__ q, int K, int N, u
     out[idx] = v;
 }
 
+// Folds a nonnegative binary32 value into the trailer's wmax_bits word
+// (nonnegative floats order like their bit patterns): one atomic per warp.
+__device__ __forceinline__ void wmax_fold(uint32_t *wmax_bits, float v)
+{
+    uint32_t b = __float_as_uint(v);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        b = max(b, __shfl_xor_sync(0xffffffffu, b, o));
+    if ((threadIdx.x & 31) == 0)
+        atomicMax(wmax_bits, b);
+}
+
 __global__ void pack_scales_int8_kernel(const uint16_t *__restrict__ s, int N, uint16_t *__restrict__ out,
-                                        int total)
+                                        int total, uint32_t *wmax_bits)
 {
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    const uint16_t v = (i < total && i < N) ? s[i] : 0;
     if (i < total)
-        out[i] = i < N ? s[i] : 0;
+        out[i] = v;
+    wmax_fold(wmax_bits, 128.f * fabsf(__uint_as_float((uint32_t)v << 16)));
 }
 
 __global__ void pack_sz_int4_kernel(const uint16_t *__restrict__ s, const uint32_t *__restrict__ z, int K,
                                     int N, uint16_t *__restrict__ s_out, uint8_t *__restrict__ z_out,
-                                    Shape sh)
+                                    Shape sh, uint32_t *wmax_bits)
 {
     const int KG = K / 128, ZW = (KG + 7) / 8;
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long total = (long long)sh.panels() * KG * kPanelRows;
-    if (idx >= total)
-        return;
     const int i = (int)(idx % kPanelRows);
     const long long pg = idx / kPanelRows;
     const int g = (int)(pg % KG), p = (int)(pg / KG);
     const int row = p * kPanelRows + i;
+    // largest |q - z| the zero point allows, times the scale
+    float wm = 0.f;
+    if (idx < total && row < N) {
+        const uint32_t zz = (z[(size_t)row * ZW + g / 8] >> (4 * (g % 8))) & 0xFu;
+        wm = fabsf(__uint_as_float((uint32_t)s[(size_t)row * KG + g] << 16)) * (float)max(zz, 15u - zz);
+    }
+    wmax_fold(wmax_bits, wm);
+    if (idx >= total)
+        return;
     s_out[idx] = row < N ? s[(size_t)row * KG + g] : 0;
     if ((i & 1) == 0) {
         uint32_t z0 = 0, z1 = 0;
@@ -338,10 +359,11 @@ cudaError_t launch_pack_int8(const int8_t *q, const uint16_t *s, int K, int N, v
 {
     const Shape sh{8, K, N, 0};
     const size_t n_vec = sh.weight_bytes() / 16;
+    write_trailer_kernel<<<1, 1, 0, st>>>((uint8_t *)wq, sh); // first: wmax_bits starts at 0
     pack_int8_kernel<<<nblk((long long)n_vec, 256), 256, 0, st>>>(q, K, N, (uint4 *)wq, n_vec, sh);
     const int total = sh.panels() * kPanelRows;
-    pack_scales_int8_kernel<<<nblk(total, 256), 256, 0, st>>>(s, N, (uint16_t *)s_out, total);
-    write_trailer_kernel<<<1, 1, 0, st>>>((uint8_t *)wq, sh);
+    pack_scales_int8_kernel<<<nblk(total, 256), 256, 0, st>>>(s, N, (uint16_t *)s_out, total,
+                                                              const_cast<uint32_t *>(trailer_wmax(wq, sh)));
     return cudaGetLastError();
 }
 
@@ -350,10 +372,11 @@ cudaError_t launch_pack_int4(const uint32_t *q, const uint16_t *s, const uint32_
 {
     const Shape sh{4, K, N, 128};
     const size_t n_vec = sh.weight_bytes() / 16;
+    write_trailer_kernel<<<1, 1, 0, st>>>((uint8_t *)wq, sh); // first: wmax_bits starts at 0
     pack_int4_kernel<<<nblk((long long)n_vec, 256), 256, 0, st>>>(q, K, N, (uint4 *)wq, n_vec, sh);
     const long long total = (long long)sh.panels() * (K / 128) * kPanelRows;
-    pack_sz_int4_kernel<<<nblk(total, 256), 256, 0, st>>>(s, z, K, N, (uint16_t *)s_out, (uint8_t *)z_out, sh);
-    write_trailer_kernel<<<1, 1, 0, st>>>((uint8_t *)wq, sh);
+    pack_sz_int4_kernel<<<nblk(total, 256), 256, 0, st>>>(s, z, K, N, (uint16_t *)s_out, (uint8_t *)z_out, sh,
+                                                          const_cast<uint32_t *>(trailer_wmax(wq, sh)));
     return cudaGetLastError();
 }
 

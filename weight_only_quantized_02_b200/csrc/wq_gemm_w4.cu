@@ -66,8 +66,6 @@ struct GemmW4Params {
     uint32_t *cnt; // [panels][8] tickets
 };
 
-constexpr int kW4Threads = 512;
-constexpr int kW4Warps = kW4Threads / 32;
 
 template <int NT>
 struct W4Cfg {
@@ -78,9 +76,15 @@ struct W4Cfg {
     static constexpr int kACC = NT <= 32 ? 128 / NT : 256 / NT; // group accumulators
     static constexpr int kA0 = kACC * NT;                // first A column
     static constexpr int kAS = (512 - kA0) / 64;         // A stages, 64 columns each
+    // 16 warps, except 20 at 64 tokens: eight retire warps (their totals fill
+    // the registers) then leave eight dequant warps, one per 16-row block;
+    // with four, dequantization paced the whole pipeline
+    static constexpr int kWarps = NT == 64 ? 20 : 16;
+    static constexpr int kThreads = 32 * kWarps;
     static constexpr int kRW = NT >= 64 ? 8 : 4;         // retire warps
     static constexpr int kCW = NT * 4 / kRW;             // token columns per retire warp
-    static constexpr int kDW = kW4Warps - 4 - kRW;       // dequant warps
+    static constexpr int kDW = kWarps - 4 - kRW;         // dequant warps
+    static constexpr int kRetireCols = kWarps == 20 ? 16 : 32; // accumulator columns per tensor-memory wait
     static constexpr int kBPW = 8 / kDW;                 // 16-row blocks per dequant warp
     static constexpr int kSlot = kBPW * 1024 + 16;       // a unit's blocks + its 16-byte zero-point segment
     static_assert(kA0 + 64 * kAS == 512, "tensor memory plan");
@@ -127,7 +131,7 @@ __device__ __forceinline__ void w4_fixup(const GemmW4Params &p, long long U, int
     const int nrow = pnl * kPanelRows + r;
     // contributors whose partials are in flight together (a panel usually has <= 5; fewer at NT = 128,
     // where the retire warps already hold 64 totals and more would spill)
-    constexpr int CG = NT == 128 ? 2 : 5;
+    constexpr int CG = (NT == 128 || W4Cfg<NT>::kWarps == 20) ? 2 : 5;
     for (int j0 = 0; j0 < CW; j0 += 16) {
         float acc[16];
 #pragma unroll
@@ -172,7 +176,7 @@ __device__ __forceinline__ void w4_fixup(const GemmW4Params &p, long long U, int
 }
 
 template <int NT>
-__global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_constant__ CUtensorMap tmx,
+__global__ void __launch_bounds__(W4Cfg<NT>::kThreads, 1) gemm_w4_kernel(const __grid_constant__ CUtensorMap tmx,
                                                                 const GemmW4Params p)
 {
     using C = W4Cfg<NT>;
@@ -359,16 +363,17 @@ __global__ void __launch_bounds__(kW4Threads, 1) gemm_w4_kernel(const __grid_con
             tc_fence_after();
             const float s = bf16_bits_to_float(reinterpret_cast<const uint16_t *>(sS + ss * 256)[r]);
             const uint32_t ta = tmem + tq + ac * NT + c * CW;
+            constexpr int RC = C::kRetireCols; // columns per wait
 #pragma unroll
-            for (int j0 = 0; j0 < CW; j0 += 32) { // up to 32 columns per wait
-                float v[2][16];
+            for (int j0 = 0; j0 < CW; j0 += RC) {
+                float v[RC / 16][16];
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
+                for (int h = 0; h < RC / 16; ++h)
                     if (j0 + 16 * h < CW)
                         tmem_ld_32x32b_x16(ta + j0 + 16 * h, v[h]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
+                for (int h = 0; h < RC / 16; ++h)
                     if (j0 + 16 * h < CW)
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
@@ -510,7 +515,7 @@ static cudaError_t launch_gemm_w4_t(const LinearArgs &a, void *ws, int sm_count,
         G = p.U;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
-    cfg.blockDim = dim3(kW4Threads);
+    cfg.blockDim = dim3(W4Cfg<NT>::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

@@ -57,8 +57,9 @@ def workload_names(spec):
     """'all' (every workload, in the order of wq_inputs.WORKLOADS) or one name."""
     if spec == "all":
         return list(gen.WORKLOADS)
-    if spec not in gen.WORKLOADS:
-        raise SystemExit(f"unknown workload {spec!r}; choose 'all' or one of {list(gen.WORKLOADS)}")
+    known = list(gen.WORKLOADS) + list(gen.EXTRA_WORKLOADS)
+    if spec not in known:
+        raise SystemExit(f"unknown workload {spec!r}; choose 'all' or one of {known}")
     return [spec]
 
 
@@ -245,7 +246,7 @@ def build_weights(name, device, copies):
     import torch
 
     import weight_only_quantized_02_b200 as wq
-    cfg = gen.WORKLOADS[name]
+    cfg = gen.workload(name)
     K, N, bits = cfg["K"], cfg["N"], cfg["bits"]
     if cfg.get("direct"):
         q, s = gen.direct_int8(K, N)
@@ -296,7 +297,7 @@ def bench_ours(args, device, rank, world):
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     works = []  # one dict per workload
     for name in names:
-        cfg0 = gen.WORKLOADS[name]
+        cfg0 = gen.workload(name)
         K, N, bits, group = cfg0["K"], cfg0["N"], cfg0["bits"], cfg0["group"]
         Ms = list(args.ms) if args.ms else list(cfg0["Ms"])
         wbytes = weight_bytes(bits, K, N, group)
@@ -546,7 +547,7 @@ class OracleSample:
     def __init__(self, name, rows=None):
         import oracle
         self.oracle = oracle
-        cfg = gen.WORKLOADS[name]
+        cfg = gen.workload(name)
         self.name = name
         self.K, self.N, self.bits, self.group = cfg["K"], cfg["N"], cfg["bits"], cfg["group"]
         self.Ms = list(cfg["Ms"])
@@ -662,7 +663,7 @@ def run_config(names):
     """The run's workloads, named by what they are."""
     ws = []
     for name in names:
-        c = gen.WORKLOADS[name]
+        c = gen.workload(name)
         ws.append({"name": name, "bits": c["bits"], "group": c["group"], "K": c["K"], "N": c["N"],
                    "Ms": list(c["Ms"])})
     label = ("all five workloads: " if len(names) == len(gen.WORKLOADS) else "") + ", ".join(names)

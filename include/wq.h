@@ -56,7 +56,9 @@
  *     says "synchronizes".
  *   - bf16 values are passed as their uint16_t bit patterns.
  *   - Shape rules: 1 <= N, N % 16 == 0. W8A16: K % 32 == 0.
- *     W4A16: group == 128, K % 128 == 0. 1 <= M <= 128.
+ *     W4A16: group == 128, K % 128 == 0. 1 <= M <= 65536; a kernel takes
+ *     at most 128 tokens, and wq_linear runs a larger M (prefill) as
+ *     consecutive chunks of 128 tokens.
  *     x, y and every packed buffer must be 16-byte aligned.
  *   - Packed buffers are written by wq_pack_int8 / wq_pack_int4 and are
  *     opaque. wq_packed_bytes gives their sizes. Their layout is described
@@ -183,7 +185,11 @@ int wq_check_packed(const void *Wq, int bits, int K, int N, int group, cudaStrea
  *   y       device, bf16 [M][N], row-major, 16-byte aligned. Every element
  *           is written: bf16_rne of the fp32-accumulated sum.
  * The kernel and split factor come from the dispatcher (tuned table, else
- * the default rule). The stream-K kernels, the integer path and a GEMM
+ * the default rule).  M > 128 runs as chunks of 128 tokens (the last one
+ * ragged), one kernel each, in order on the stream, each streaming the
+ * weights once and each with the dispatcher's choice for its own size; if a
+ * chunk fails its status is returned and the chunks before it stay
+ * enqueued. The stream-K kernels, the integer path and a GEMM
  * split > 1 use the workspace registered with wq_set_workspace for the
  * current device. With no workspace (or too small a one), decode-sized M
  * falls back to the row-block GEMV and the GEMM runs unsplit, so wq_linear
@@ -232,7 +238,8 @@ int wq_linear_noalloc(const uint16_t *x, int M, int K, const void *Wq, const voi
                       const void *zeros, int group, int N, uint16_t *y, cudaStream_t stream);
 
 /* Bytes of workspace for M tokens, a K x N weight and GEMM splits up to
- * max_split: enough for every variant of that shape. It holds eight ticket
+ * max_split: enough for every variant of that shape (M > 128: of its
+ * 128-token chunks, which share the workspace one after another). It holds eight ticket
  * counters per 128-channel panel and the largest of the GEMM's fp32
  * partials [split][M][N], the stream-K kernels' per-CTA panel partials,
  * the integer path's int32 per-CTA partials, and the integer GEMV's
@@ -258,12 +265,14 @@ int wq_set_workspace(void *ws, size_t bytes);
  * keeps the fastest by the mean of the middle half of its sorted times. On an exact tie the later, larger
  * split wins, as in the split_k auto-tune loop of Mit han lab Llm awq Kernel
  * Selection Thresholds, The Insight. Overwrites y. Synchronizes `stream`.
- * Needs a registered workspace that fits split 32 to try every split. */
+ * Needs a registered workspace that fits split 32 to try every split.
+ * M > 128 tunes the 128-token chunk shape on the first 128 rows of x. */
 int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
             const void *zeros, int group, int N, uint16_t *y, int warmup, int iters,
             cudaStream_t stream);
 
-/* The (variant, split) that wq_linear would use for this shape now. Host. */
+/* The (variant, split) that wq_linear would use for this shape now (M > 128:
+ * for its full 128-token chunks). Host. */
 int wq_get_choice(int M, int K, int N, int bits, int group, int *variant, int *split);
 
 /* Sets one table entry by hand (for tests and offline tables). Host. */

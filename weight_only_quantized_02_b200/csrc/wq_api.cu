@@ -192,8 +192,10 @@ int lookup_choice(const DeviceInfo &d, int M, int K, int N, int bits, int group,
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
 
-int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros, int group,
-                int N, uint16_t *y, int variant, int split, void *ws, size_t ws_bytes_given, cudaStream_t stream)
+// One call of at most kChunkTokens tokens: the dispatcher's (or the forced)
+// kernel for this M.
+int linear_chunk(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros, int group,
+                 int N, uint16_t *y, int variant, int split, void *ws, size_t ws_bytes_given, cudaStream_t stream)
 {
     int bits = 0;
     int st = bits_of_group(group, &bits);
@@ -203,7 +205,7 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
         return WQ_ERR_NULL;
     if ((st = check_weight_shape(bits, K, N, group)) != WQ_OK)
         return st;
-    if (M < 1 || M > 128)
+    if (M < 1 || M > kChunkTokens)
         return WQ_ERR_SHAPE;
     if (!aligned16(x) || !aligned16(y) || !aligned16(Wq) || !aligned16(scales) || (zeros && !aligned16(zeros)))
         return WQ_ERR_ALIGN;
@@ -298,6 +300,31 @@ int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *sca
     if (c.split > 1 && (!w || have < ws_bytes(M, N, c.split)))
         return WQ_ERR_WORKSPACE;
     return cuda_status(launch_gemm(a, c.split, c.split > 1 ? w : nullptr, d.sm_count, stream));
+}
+
+// The layer for any M up to kMaxTokens: runs of kChunkTokens tokens, one
+// kernel each, in order on the stream (x and y advance by whole token rows,
+// so every chunk keeps their 16-byte alignment).  Each chunk streams the
+// weights once; the chunks share the workspace one after another.  A
+// failing chunk returns its status; the chunks before it are already
+// enqueued.
+int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros, int group,
+                int N, uint16_t *y, int variant, int split, void *ws, size_t ws_bytes_given, cudaStream_t stream)
+{
+    if (M <= kChunkTokens)
+        return linear_chunk(x, M, K, Wq, scales, zeros, group, N, y, variant, split, ws, ws_bytes_given, stream);
+    if (M > kMaxTokens)
+        return WQ_ERR_SHAPE;
+    if (!x || !y)
+        return WQ_ERR_NULL;
+    for (int m0 = 0; m0 < M; m0 += kChunkTokens) {
+        const int mc = std::min(kChunkTokens, M - m0);
+        const int st = linear_chunk(x + (size_t)m0 * K, mc, K, Wq, scales, zeros, group, N, y + (size_t)m0 * N,
+                                    variant, split, ws, ws_bytes_given, stream);
+        if (st != WQ_OK)
+            return st;
+    }
+    return WQ_OK;
 }
 
 } // namespace
@@ -504,6 +531,7 @@ size_t wq_workspace_bytes(int M, int K, int N, int max_split)
 {
     if (M < 1 || K < 1 || N < 1 || max_split < 1)
         return 0;
+    M = std::min(M, kChunkTokens); // longer inputs run in chunks that share the workspace
     size_t b = std::max(ws_bytes(M, N, max_split), ws_bytes_gemm_sk(M, N));
     if (M <= 32)
         b = std::max(b, ws_bytes_gemv_sk(M, N));
@@ -546,8 +574,9 @@ int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
     DeviceInfo d;
     if ((st = current_device_info(&d)) != WQ_OK)
         return st;
-    if (warmup < 0 || iters < 1)
+    if (warmup < 0 || iters < 1 || M < 1 || M > kMaxTokens)
         return WQ_ERR_SHAPE;
+    M = std::min(M, kChunkTokens); // longer inputs: the chunk shape, timed on the first chunk
     std::vector<std::pair<int, int>> cands;
     if (M <= 32) {
         for (int c : {1, 2, 3})
@@ -679,7 +708,7 @@ int wq_get_choice(int M, int K, int N, int bits, int group, int *variant, int *s
     if (st != WQ_OK)
         return st;
     Choice c;
-    lookup_choice(d, M, K, N, bits, group, &c);
+    lookup_choice(d, std::min(M, kChunkTokens), K, N, bits, group, &c);
     *variant = c.variant;
     *split = c.split;
     return WQ_OK;

@@ -9,6 +9,11 @@
 
 namespace wq {
 
+// Tokens per kernel launch; wq_linear takes up to kMaxTokens and runs longer
+// inputs as consecutive chunks of kChunkTokens.
+constexpr int kChunkTokens = 128;
+constexpr int kMaxTokens = 65536;
+
 struct LinearArgs {
     const uint16_t *x;
     int M, K, N;

@@ -41,6 +41,18 @@ WORKLOADS = {
 }
 
 
+# Beyond the five decode workloads: the same W4A16 layer at prefill-sized M
+# (the larger-M regime; wq_linear runs M > 128 in chunks of 128 tokens).
+EXTRA_WORKLOADS = {
+    "w4g128_prefill_17408x5120": dict(bits=4, K=17408, N=5120, group=128, Ms=(256, 2048)),
+}
+
+
+def workload(name: str) -> dict:
+    """The workload of that name, from WORKLOADS or EXTRA_WORKLOADS."""
+    return WORKLOADS[name] if name in WORKLOADS else EXTRA_WORKLOADS[name]
+
+
 def generator(stream: str, chunk: int = 0, seed: int = SEED) -> np.random.Generator:
     ss = np.random.SeedSequence(entropy=seed, spawn_key=(_STREAMS[stream], int(chunk)))
     return np.random.Generator(np.random.PCG64(ss))

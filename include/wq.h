@@ -237,6 +237,27 @@ int wq_linear_ex(const uint16_t *x, int M, int K, const void *Wq, const void *sc
 int wq_linear_noalloc(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
                       const void *zeros, int group, int N, uint16_t *y, cudaStream_t stream);
 
+/* The vocabulary head's top-k for sampling ("Fused LM Head + Top-k",
+ * tileInfer README, Features list): for every token row m the k largest
+ * logits of y = x . dequant(Wq)^T and their indices, without returning y.
+ *   vals    device, bf16 [M][k]: the k largest logits of row m, descending
+ *   idx     device, int32 [M][k]: their output indices; among equal logits
+ *           the lower index comes first, so the result is unique
+ *   ws      device scratch of at least wq_topk_workspace_bytes(M, N, k)
+ *           bytes, 16-byte aligned, owned by the caller (the logits pass
+ *           through it as bf16, then the candidates of the selection)
+ *   1 <= M <= 128, 1 <= k <= 64, k <= N; other arguments as wq_linear.
+ * The logits come from the dispatcher's kernel (with the workspace
+ * registered by wq_set_workspace, as wq_linear); two selection kernels
+ * follow on the same stream.  Returns WQ_ERR_SHAPE outside the limits,
+ * WQ_ERR_WORKSPACE for a scratch that is too small. */
+int wq_linear_topk(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
+                   const void *zeros, int group, int N, int k, uint16_t *vals, int32_t *idx,
+                   void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Scratch bytes of wq_linear_topk; 0 for arguments out of its limits. Host. */
+size_t wq_topk_workspace_bytes(int M, int N, int k);
+
 /* Bytes of workspace for M tokens, a K x N weight and GEMM splits up to
  * max_split: enough for every variant of that shape (M > 128: of its
  * 128-token chunks, which share the workspace one after another). It holds eight ticket

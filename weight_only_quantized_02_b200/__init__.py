@@ -65,6 +65,8 @@ def _load():
         "wq_linear_forced": (I, [P, I, I, P, P, P, I, I, P, I, I, P]),
         "wq_linear_ex": (I, [P, I, I, P, P, P, I, I, P, I, I, P, SZ, P]),
         "wq_linear_noalloc": (I, [P, I, I, P, P, P, I, I, P, P]),
+        "wq_linear_topk": (I, [P, I, I, P, P, P, I, I, I, P, P, P, SZ, P]),
+        "wq_topk_workspace_bytes": (SZ, [I, I, I]),
         "wq_workspace_bytes": (SZ, [I, I, I, I]),
         "wq_set_workspace": (I, [P, SZ]),
         "wq_tune": (I, [P, I, I, P, P, P, I, I, P, I, I, P]),
@@ -254,6 +256,22 @@ def wq_linear_noalloc(x: torch.Tensor, pw: PackedWeight, y: Optional[torch.Tenso
     _check(lib.wq_linear_noalloc(_p(x), M, K, _p(pw.wq), _p(pw.scales), _p(pw.zeros), pw.group, pw.N, _p(y),
                                  _s(stream)), "wq_linear_noalloc")
     return y
+
+
+def wq_topk_workspace_bytes(M: int, N: int, k: int) -> int:
+    return int(lib.wq_topk_workspace_bytes(M, N, k))
+
+
+def wq_linear_topk(x: torch.Tensor, pw: PackedWeight, k: int, ws: torch.Tensor, stream=None):
+    """The k largest logits of every token row and their indices: (vals bf16
+    [M][k] descending, idx int32 [M][k]); ws a device scratch of at least
+    wq_topk_workspace_bytes(M, N, k) bytes."""
+    M, K = x.shape
+    vals = torch.empty((M, k), dtype=torch.bfloat16, device=x.device)
+    idx = torch.empty((M, k), dtype=torch.int32, device=x.device)
+    _check(lib.wq_linear_topk(_p(x), M, K, _p(pw.wq), _p(pw.scales), _p(pw.zeros), pw.group, pw.N, k, _p(vals),
+                              _p(idx), _p(ws), ws.numel() * ws.element_size(), _s(stream)), "wq_linear_topk")
+    return vals, idx
 
 
 def wq_linear_status(x, pw: PackedWeight, y, variant=WQ_VARIANT_AUTO, split=0, stream=None) -> int:

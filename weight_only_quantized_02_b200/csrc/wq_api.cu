@@ -527,6 +527,36 @@ int wq_linear_noalloc(const uint16_t *x, int M, int K, const void *Wq, const voi
     return cuda_status(launch_gemv_sk_noalloc(a, d.sm_count, stream));
 }
 
+size_t wq_topk_workspace_bytes(int M, int N, int k)
+{
+    if (M > kChunkTokens)
+        return 0;
+    return topk_ws_bytes(M, N, k);
+}
+
+int wq_linear_topk(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros, int group,
+                   int N, int k, uint16_t *vals, int32_t *idx, void *ws, size_t ws_bytes_given, cudaStream_t stream)
+{
+    if (M < 1 || M > kChunkTokens || k < 1 || k > kTopkMaxK || k > N)
+        return WQ_ERR_SHAPE;
+    if (!vals || !idx || !ws)
+        return WQ_ERR_NULL;
+    const size_t need = topk_ws_bytes(M, N, k);
+    if (need == 0)
+        return WQ_ERR_SHAPE;
+    if (!aligned16(ws))
+        return WQ_ERR_ALIGN;
+    if (ws_bytes_given < need)
+        return WQ_ERR_WORKSPACE;
+    // the logits, into the scratch, by the dispatcher's kernel
+    uint16_t *logits = static_cast<uint16_t *>(ws);
+    const int st = linear_impl(x, M, K, Wq, scales, zeros, group, N, logits, WQ_VARIANT_AUTO, 0, nullptr, 0, stream);
+    if (st != WQ_OK)
+        return st;
+    void *cand = static_cast<uint8_t *>(ws) + ((size_t)M * N * 2 + 255) / 256 * 256;
+    return cuda_status(launch_topk(logits, M, N, k, cand, vals, idx, stream));
+}
+
 size_t wq_workspace_bytes(int M, int K, int N, int max_split)
 {
     if (M < 1 || K < 1 || N < 1 || max_split < 1)

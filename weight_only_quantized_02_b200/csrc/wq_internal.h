@@ -122,6 +122,16 @@ bool gi_fits(int bits, int M, int K);
 size_t ws_bytes_gemv_i8(int M, int K, int N);
 cudaError_t launch_gemv_i8(const LinearArgs &a, int split, void *ws, int sm_count, cudaStream_t st);
 
+// Top-k of the vocabulary head (wq_topk.cu): k <= kTopkMaxK.  topk_plan
+// picks the slice S (P slices, merge of T keys); topk_ws_bytes is the
+// scratch of wq_linear_topk (bf16 logits M x N, then M x P x k candidates);
+// launch_topk selects from logits already in that scratch.
+constexpr int kTopkMaxK = 64;
+bool topk_plan(int N, int k, int *S, int *P, int *T);
+size_t topk_ws_bytes(int M, int N, int k);
+cudaError_t launch_topk(const uint16_t *logits, int M, int N, int k, void *cand_ws, uint16_t *vals, int32_t *idx,
+                        cudaStream_t st);
+
 // Launch preparation of one kernel on the current device: raises its
 // dynamic shared-memory limit to smem_optin bytes (0: leave it) the first
 // time it is launched on that device, and returns in *occ (if not NULL) its

@@ -42,6 +42,14 @@ def lib():
         L.wqo_dequant_int4.argtypes = [P, P, P, I64, I64, I64, P, I64, P]
         L.wqo_linear_int8.argtypes = [P, I64, I64, P, P, I64, P, I64, P]
         L.wqo_linear_int4.argtypes = [P, I64, I64, P, P, P, I64, I64, P, I64, P]
+        L.wqo_linear_int8_fmt.argtypes = [P, ctypes.c_int, I64, I64, P, P, I64, P, I64, P]
+        L.wqo_linear_int4_fmt.argtypes = [P, ctypes.c_int, I64, I64, P, P, P, I64, I64, P, I64, P]
+        L.wqo_f16_to_f64.restype = ctypes.c_double
+        L.wqo_f16_to_f64.argtypes = [ctypes.c_uint16]
+        L.wqo_f64_to_f16_rne.restype = ctypes.c_uint16
+        L.wqo_f64_to_f16_rne.argtypes = [ctypes.c_double]
+        L.wqo_f16_to_f64_array.argtypes = [P, I64, P]
+        L.wqo_f16_round_array.argtypes = [P, I64, P]
         L.wqo_quant_int8.argtypes = [P, I64, I64, P, P]
         L.wqo_quant_int4.argtypes = [P, I64, I64, I64, P, P, P]
         _lib = L
@@ -126,8 +134,28 @@ def dequant_int4(q_words, s, z_words, K, G=128, rows=None):
 
 # ---- linear ---------------------------------------------------------------
 
-def linear_int8(x_bf16, q, s, rows=None):
-    """y[m][i] = sum_k x[m][k] * s[n] * q[n][k], n = rows[i]; binary64 [M][len(rows)]."""
+def f16_to_f64(h):
+    """IEEE binary16 bit patterns -> binary64 (exact)."""
+    h, ph = _c(h, np.uint16)
+    out = np.empty(h.shape, np.float64)
+    lib().wqo_f16_to_f64_array(ph, h.size, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def f64_to_f16(v):
+    """binary64 -> IEEE binary16 bit patterns, round to nearest even."""
+    v, pv = _c(v, np.float64)
+    out = np.empty(v.shape, np.uint16)
+    lib().wqo_f16_round_array(pv, v.size, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+_FMT = {"bf16": 0, "fp16": 1}
+
+
+def linear_int8(x_bf16, q, s, rows=None, act="bf16"):
+    """y[m][i] = sum_k x[m][k] * s[n] * q[n][k], n = rows[i]; binary64 [M][len(rows)].
+    x: bf16 bit patterns, or fp16 ones with act='fp16'."""
     x, px = _c(x_bf16, np.uint16)
     q, pq = _c(q, np.int8)
     s, ps = _c(s, np.uint16)
@@ -136,11 +164,11 @@ def linear_int8(x_bf16, q, s, rows=None):
     assert q.shape[1] == K
     r, pr, nr = _rows_arg(rows, N)
     y = np.empty((M, nr), np.float64)
-    lib().wqo_linear_int8(px, M, K, pq, ps, N, pr, nr, y.ctypes.data_as(ctypes.c_void_p))
+    lib().wqo_linear_int8_fmt(px, _FMT[act], M, K, pq, ps, N, pr, nr, y.ctypes.data_as(ctypes.c_void_p))
     return y
 
 
-def linear_int4(x_bf16, q_words, s, z_words, G=128, rows=None):
+def linear_int4(x_bf16, q_words, s, z_words, G=128, rows=None, act="bf16"):
     x, px = _c(x_bf16, np.uint16)
     q_words, pq = _c(q_words, np.uint32)
     s, ps = _c(s, np.uint16)
@@ -150,7 +178,7 @@ def linear_int4(x_bf16, q_words, s, z_words, G=128, rows=None):
     assert q_words.shape[1] * 8 == K
     r, pr, nr = _rows_arg(rows, N)
     y = np.empty((M, nr), np.float64)
-    lib().wqo_linear_int4(px, M, K, pq, ps, pz, G, N, pr, nr, y.ctypes.data_as(ctypes.c_void_p))
+    lib().wqo_linear_int4_fmt(px, _FMT[act], M, K, pq, ps, pz, G, N, pr, nr, y.ctypes.data_as(ctypes.c_void_p))
     return y
 
 

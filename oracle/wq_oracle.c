@@ -32,6 +32,11 @@
  *   - INT4 zero points: uint32 words [N][ceil((K/G)/8)]; nibble j of word
  *     (n, c) is z[n][8c + j], the zero of group 8c + j.
  *   - INT4 scales: bf16 [N][K/G].   INT8: q int8 [N][K], scales bf16 [N].
+ *   - G (INT4) is the group: 32, 64, 128, or K for one scale and zero point
+ *     per output channel ("per-channel and groups 32/64/128" in the
+ *     validation matrix of the Marlin register and launch scheduling
+ *     benchmark, "Validation and limits").
+ *   - Activations x are bf16, or IEEE binary16 in the *_fmt entry points.
  *
  * Parity pins: every function here is pinned by the tests in
  * tests/test_oracle_pins.py against closed forms, brute force in exact
@@ -45,6 +50,13 @@
 #ifdef _OPENMP
 #include <omp.h>
 #endif
+
+double wqo_f16_to_f64(uint16_t h);
+void wqo_linear_int8_fmt(const uint16_t *x, int fmt, int64_t M, int64_t K, const int8_t *q, const uint16_t *s,
+                         int64_t N, const int64_t *rows, int64_t n_rows, double *y);
+void wqo_linear_int4_fmt(const uint16_t *x, int fmt, int64_t M, int64_t K, const uint32_t *q_words,
+                         const uint16_t *s, const uint32_t *z_words, int64_t G, int64_t N, const int64_t *rows,
+                         int64_t n_rows, double *y);
 
 /* ------------------------------------------------------------------ */
 /* bf16 <-> binary64                                                   */
@@ -117,6 +129,70 @@ void wqo_bf16_round_array(const double *v, int64_t n, int mode, uint16_t *out)
 {
     for (int64_t i = 0; i < n; ++i)
         out[i] = round_to_bf16(v[i], mode);
+}
+
+/* ------------------------------------------------------------------ */
+/* IEEE binary16 (fp16) <-> binary64: the FP16 activations of the      */
+/* validation matrix (Marlin register and launch scheduling benchmark,  */
+/* "Validation and limits").                                            */
+/* ------------------------------------------------------------------ */
+
+/* binary16: sign, 5 exponent bits (bias 15), 10 fraction bits.  Normal:
+ * (1024 + f) 2^(e - 25); subnormal (e = 0): f 2^-24; e = 31: inf / NaN.
+ * Exact in binary64. */
+double wqo_f16_to_f64(uint16_t h)
+{
+    const int sign = h >> 15, e = (h >> 10) & 0x1F, f = h & 0x3FF;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + f), e - 25);
+    return sign ? -v : v;
+}
+
+/* binary64 -> binary16, round to nearest, ties to even: the quantum of the
+ * binade of |v| (11 significant bits; 2^-24 below the smallest normal
+ * 2^-14), the exact count of quanta rounded, overflow to infinity at
+ * 65520 = 65504 + half a quantum. */
+uint16_t wqo_f64_to_f16_rne(double v)
+{
+    const int neg = signbit(v) ? 1 : 0;
+    const double a = fabs(v);
+    if (a == 0.0)
+        return neg ? 0x8000 : 0;
+    int e2;
+    frexp(a, &e2); /* a = m 2^e2, m in [0.5, 1): binade 2^(e2 - 1) */
+    const int qe = (e2 - 1 >= -14) ? (e2 - 1) - 10 : -24;
+    const double r = nearbyint(ldexp(a, -qe)); /* default rounding: to nearest even */
+    const double res = ldexp(r, qe);
+    if (res >= 65520.0 || res > 65504.0)
+        return (uint16_t)(neg ? 0xFC00 : 0x7C00);
+    uint16_t out;
+    if (res < ldexp(1.0, -14)) {
+        out = (uint16_t)r; /* subnormal (or the smallest normal when r = 1024) */
+    } else {
+        int e3;
+        const double m = frexp(res, &e3); /* res = m 2^e3 */
+        const int biased = (e3 - 1) + 15;
+        const int frac = (int)(ldexp(m, 11) - 1024.0);
+        out = (uint16_t)((biased << 10) | frac);
+    }
+    return (uint16_t)(out | (neg ? 0x8000 : 0));
+}
+
+void wqo_f16_to_f64_array(const uint16_t *h, int64_t n, double *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = wqo_f16_to_f64(h[i]);
+}
+
+void wqo_f16_round_array(const double *v, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = wqo_f64_to_f16_rne(v[i]);
 }
 
 void wqo_bf16_to_f64_array(const uint16_t *b, int64_t n, double *out)
@@ -254,11 +330,12 @@ static void linear_rows(const double *xd, int64_t M, int64_t K, int64_t n_rows, 
     }
 }
 
-static double *bf16_matrix_to_f64(const uint16_t *x, int64_t n)
+/* x as binary64: bf16 (fmt 0) or IEEE binary16 (fmt 1) bit patterns. */
+static double *act_matrix_to_f64(const uint16_t *x, int64_t n, int fmt)
 {
     double *xd = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
     for (int64_t i = 0; i < n; ++i)
-        xd[i] = wqo_bf16_to_f64(x[i]);
+        xd[i] = fmt ? wqo_f16_to_f64(x[i]) : wqo_bf16_to_f64(x[i]);
     return xd;
 }
 
@@ -297,9 +374,17 @@ void wqo_linear_int8(const uint16_t *x, int64_t M, int64_t K, const int8_t *q,
                      const uint16_t *s, int64_t N, const int64_t *rows, int64_t n_rows,
                      double *y)
 {
+    wqo_linear_int8_fmt(x, 0, M, K, q, s, N, rows, n_rows, y);
+}
+
+/* As wqo_linear_int8, x in activation format fmt (0 bf16, 1 fp16). */
+void wqo_linear_int8_fmt(const uint16_t *x, int fmt, int64_t M, int64_t K, const int8_t *q,
+                         const uint16_t *s, int64_t N, const int64_t *rows, int64_t n_rows,
+                         double *y)
+{
     if (!rows)
         n_rows = N;
-    double *xd = bf16_matrix_to_f64(x, M * K);
+    double *xd = act_matrix_to_f64(x, M * K, fmt);
     struct int8_ctx ctx = {q, s, K, rows};
     linear_rows(xd, M, K, n_rows, y, int8_row, &ctx);
     free(xd);
@@ -309,9 +394,17 @@ void wqo_linear_int4(const uint16_t *x, int64_t M, int64_t K, const uint32_t *q_
                      const uint16_t *s, const uint32_t *z_words, int64_t G, int64_t N,
                      const int64_t *rows, int64_t n_rows, double *y)
 {
+    wqo_linear_int4_fmt(x, 0, M, K, q_words, s, z_words, G, N, rows, n_rows, y);
+}
+
+/* As wqo_linear_int4, x in activation format fmt (0 bf16, 1 fp16). */
+void wqo_linear_int4_fmt(const uint16_t *x, int fmt, int64_t M, int64_t K, const uint32_t *q_words,
+                         const uint16_t *s, const uint32_t *z_words, int64_t G, int64_t N,
+                         const int64_t *rows, int64_t n_rows, double *y)
+{
     if (!rows)
         n_rows = N;
-    double *xd = bf16_matrix_to_f64(x, M * K);
+    double *xd = act_matrix_to_f64(x, M * K, fmt);
     struct int4_ctx ctx = {q_words, s, z_words, K, G, rows};
     linear_rows(xd, M, K, n_rows, y, int4_row, &ctx);
     free(xd);

@@ -423,3 +423,78 @@ def test_generator_rows_are_addressable():
     assert q.min() >= -127 and q.max() <= 127
     sd = oracle.bf16_to_f64(s)
     assert np.all((sd >= 1e-3 * (1 - 2**-8)) & (sd <= 2e-2 * (1 + 2**-8)))
+
+
+# ---------------------------------------------------------------------------
+# groups of 32 and 64 k and one pair per channel (G = K); fp16 activations
+# (the validation matrix of the Marlin register and launch scheduling
+# benchmark, "Validation and limits")
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("G", [32, 64, 512])
+def test_quant_int4_error_bound_groups(G):
+    K = 512  # G = K: one scale and zero point per row
+    W = np.concatenate([gen.W_f32(0, 64, K), _adversarial_rows(K)])
+    q, s, z = oracle.quant_int4(W, G)
+    assert s.shape == (W.shape[0], K // G)
+    w = oracle.dequant_int4(q, s, z, K, G)
+    sd = np.repeat(oracle.bf16_to_f64(s), G, axis=1)
+    err = np.abs(w - W.astype(np.float64))
+    assert np.all((err <= sd / 2 * (1 + 2.0 ** -40)) | ((sd == 0) & (W == 0)))
+
+
+@pytest.mark.parametrize("G", [32, 64, 256])
+def test_linear_int4_exact_bruteforce_groups(G):
+    g = np.random.default_rng(50 + G)
+    M, K, N = 2, 256, 8
+    x = gen.f32_to_bf16_bits(g.normal(0, 1, (M, K)).astype(np.float32))
+    q, s, z = _rand_int4(g, N, K, G)
+    y = oracle.linear_int4(x, q, s, z, G)
+    exact = _exact_int4(x, q, s, z, G)
+    w = oracle.dequant_int4(q, s, z, K, G)
+    _check_against_exact(y, exact, x, np.abs(oracle.bf16_to_f64(x)) @ np.abs(w).T)
+
+
+def test_f16_decode_every_pattern():
+    """binary16 -> binary64 on all 65536 patterns against numpy's float16."""
+    h = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.f16_to_f64(h)
+    ref = h.view(np.float16).astype(np.float64)
+    both_nan = np.isnan(ours) & np.isnan(ref)
+    assert np.all(both_nan | (ours == ref))
+    assert np.all(np.signbit(ours[~both_nan]) == np.signbit(ref[~both_nan]))
+
+
+def test_f16_rounding_against_numpy():
+    """binary64 -> binary16 round to nearest even against numpy's float16
+    conversion: random values over the whole range, exact ties between
+    neighbours (normal and subnormal), and the overflow edge."""
+    g = np.random.default_rng(60)
+    v = np.concatenate([
+        g.normal(0, 1, 20000), g.normal(0, 3e4, 20000), g.normal(0, 1e-5, 20000), g.normal(0, 1e-7, 5000),
+        np.ldexp(g.integers(0, 4096, 20000) + 0.5, -12),           # ties at quantum 2^-11 .. (normal)
+        np.ldexp(g.integers(0, 1024, 4000) + 0.5, -24),            # ties between subnormals
+        [65504.0, 65519.999, 65520.0, 65536.0, 1e9, 2.0 ** -24, 2.0 ** -25, 2.0 ** -25 * 1.0001, 0.0, -0.0],
+    ])
+    v = np.concatenate([v, -v])
+    ours = oracle.f64_to_f16(v)
+    ref = v.astype(np.float16).view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_linear_fp16_activations_match_numpy():
+    """fp16 activations: the oracle's linear against numpy's float16 decode
+    and fp64 matmul on the oracle's own dequantized weights, both formats."""
+    g = np.random.default_rng(70)
+    M, K, N = 3, 512, 32
+    xh = g.normal(0, 1, (M, K)).astype(np.float16).view(np.uint16)
+    xd = xh.view(np.float16).astype(np.float64)
+    q8 = g.integers(-127, 128, size=(N, K), dtype=np.int8)
+    s8 = gen.f32_to_bf16_bits(g.uniform(1e-3, 2e-2, N).astype(np.float32))
+    w8 = oracle.dequant_int8(q8, s8)
+    y8 = oracle.linear_int8(xh, q8, s8, act="fp16")
+    assert np.all(np.abs(y8 - xd @ w8.T) <= 2 * K * 2.0 ** -53 * (np.abs(xd) @ np.abs(w8).T))
+    q4, s4, z4 = _rand_int4(g, N, K, 64)
+    w4 = oracle.dequant_int4(q4, s4, z4, K, 64)
+    y4 = oracle.linear_int4(xh, q4, s4, z4, 64, act="fp16")
+    assert np.all(np.abs(y4 - xd @ w4.T) <= 2 * K * 2.0 ** -53 * (np.abs(xd) @ np.abs(w4).T))

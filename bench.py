@@ -463,14 +463,57 @@ def bench_ours(args, device, rank, world):
                      "traffic_source": f"profiles/{summary}" if traffic is not None else None,
                      "algorithmic_bytes_per_launch": b_dom})
 
+    topk = bench_topk(args, device, works, stream, per_call_us, points)
     e2e = bench_e2e(args, device, works, stream)
     wq.wq_set_workspace(None)
     return {
         "value": value_bps / 1e9, "ms_per_step": tmax / args.steps * 1e3, "per_shape": per_shape,
-        "roofline": roofline, "clocks": clocks, "e2e": e2e, "works": works,
+        "roofline": roofline, "clocks": clocks, "e2e": e2e, "works": works, "topk": topk,
         "gpu_launches": args.steps * sum(w["copies"] for w, _ in points),
         "tflops": step_flops * args.steps * world / tmax / 1e12, "l2_bytes": l2,
     }
+
+
+TOPK_K = 64
+
+
+def bench_topk(args, device, works, stream, per_call_us, points):
+    """The vocabulary head's top-k (wq_linear_topk, k = 64) on every
+    vocabulary-sized workload: the per-call time of the logits plus the
+    selection, beside the plain layer's time from the timed region."""
+    import torch
+
+    import weight_only_quantized_02_b200 as wq
+    out = []
+    for w in works:
+        if w["N"] < 100000:
+            continue
+        for M in w["Ms"]:
+            ws = torch.zeros(wq.wq_topk_workspace_bytes(M, w["N"], TOPK_K), dtype=torch.uint8, device=device)
+            with torch.cuda.stream(stream):
+                for c in range(w["copies"]):
+                    wq.wq_linear_topk(w["xs"][M], w["pws"][c], TOPK_K, ws, stream=stream)
+            torch.cuda.synchronize(device)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for c in range(w["copies"]):
+                    wq.wq_linear_topk(w["xs"][M], w["pws"][c], TOPK_K, ws, stream=stream)
+            reps = max(3, min(args.steps, 20))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                g.replay()
+                a.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                b.record(stream)
+            torch.cuda.synchronize(device)
+            us = a.elapsed_time(b) * 1000.0 / (reps * w["copies"])
+            i = next(j for j, (pw_, pm) in enumerate(points) if pw_ is w and pm == M)
+            plain = statistics.mean(per_call_us[i])
+            out.append({"workload": w["name"], "M": M, "k": TOPK_K, "us_per_call": round(us, 3),
+                        "layer_us_per_call": round(plain, 3), "selection_us": round(us - plain, 3)})
+            del g, ws
+    return out
 
 
 def bench_e2e(args, device, works, stream):
@@ -726,7 +769,7 @@ def main():
                     "W8A16 case draws its codes and scales)",
             "config": conf,
             "tflops": round(r["tflops"], 2), "per_shape": r["per_shape"], "roofline": r["roofline"],
-            "clocks": r["clocks"], "e2e": r["e2e"], "gpu_launches": r["gpu_launches"],
+            "clocks": r["clocks"], "e2e": r["e2e"], "gpu_launches": r["gpu_launches"], "topk": r["topk"],
             "dispatch": {f"{w['name']} M={M}": list(w["choices"][M]) for w in r["works"] for M in w["Ms"]},
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -10,7 +10,8 @@
  *          ("Per-channel W8A16 quantization", tileInfer README, Features
  *          table.)
  *   W4A16  unsigned 4-bit weights q in [0,15] with a bf16 scale and a 4-bit
- *          zero point per (group of `group` consecutive k, output channel):
+ *          zero point per (group of `group` consecutive k, output channel;
+ *          group 32, 64, 128, or K for one pair per output channel):
  *          w[n][k] = s[n][k/group] * (q[n][k] - z[n][k/group])
  *          (A WnA16 kernel shared by several checkpoint formats needs the same
  *          layout, scales, zero points and group size. This is the review of
@@ -55,10 +56,12 @@
  *     after the enqueue, with no implicit synchronization, unless the entry
  *     says "synchronizes".
  *   - bf16 values are passed as their uint16_t bit patterns.
- *   - Shape rules: 1 <= N, N % 16 == 0. W8A16: K % 32 == 0.
- *     W4A16: group == 128, K % 128 == 0. 1 <= M <= 65536; a kernel takes
- *     at most 128 tokens, and wq_linear runs a larger M (prefill) as
- *     consecutive chunks of 128 tokens.
+ *   - Shape rules: 1 <= N, N % 16 == 0. W8A16: group == 0, K % 32 == 0.
+ *     W4A16: K % 128 == 0 and group 32, 64, 128 or K (per channel: one
+ *     scale and zero point per output row). 1 <= M <= 65536; a kernel takes
+ *     at most 128 tokens (32 for groups of 32 and 64 k, which run on the
+ *     row-block GEMV only), and wq_linear runs a larger M (prefill) as
+ *     consecutive chunks.
  *     x, y and every packed buffer must be 16-byte aligned.
  *   - Packed buffers are written by wq_pack_int8 / wq_pack_int4 and are
  *     opaque. wq_packed_bytes gives their sizes. Their layout is described
@@ -116,7 +119,9 @@ const char *wq_strerror(int status);
 int wq_version(void);
 
 /* Byte sizes of the three packed buffers for a weight of shape [N][K].
- * bits = 8 (group must be 0) or 4 (group must be 128). zero_bytes is 0 for
+ * bits = 8 (group must be 0) or 4 (group 32, 64, 128 or K; per channel,
+ * group K, is stored as group 128 with each row's scale and zero point
+ * repeated in every 128-k block, so it runs on every kernel). zero_bytes is 0 for
  * INT8. Any output pointer may be NULL. Host, no device work. */
 int wq_packed_bytes(int bits, int K, int N, int group, size_t *wq_bytes,
                     size_t *scale_bytes, size_t *zero_bytes);
@@ -197,6 +202,16 @@ int wq_check_packed(const void *Wq, int bits, int K, int N, int group, cudaStrea
  * GPU (keep them on one stream). */
 int wq_linear(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
               const void *zeros, int group, int N, uint16_t *y, cudaStream_t stream);
+
+/* wq_linear with fp16 activations and fp16 outputs (x fp16 [M][K], y fp16
+ * [M][N], as their uint16_t bit patterns; the packed weights and their bf16
+ * scales are the same).  Runs the row-block GEMV, 32 tokens per launch, with
+ * the dequantized weights as exact fp16 integers and fp32 accumulation; y is
+ * rounded to fp16, to nearest even.  The FP16 half of the validation matrix
+ * of the Marlin register and launch scheduling benchmark, "Validation and
+ * limits".  1 <= M <= 65536; other rules as wq_linear.  Needs no workspace. */
+int wq_linear_f16(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
+                  const void *zeros, int group, int N, uint16_t *y, cudaStream_t stream);
 
 /* wq_linear with an explicit kernel variant (WQ_VARIANT_*) and split factor.
  * variant = WQ_VARIANT_AUTO, or split = 0, leaves that choice to the dispatcher.

@@ -49,11 +49,18 @@ def test_packed_bytes():
     # ragged: N not a multiple of the 128-row panel, K not a multiple of the 128-k block
     wb, sb, zb = wq.wq_packed_bytes(8, 1120, 400, 0)
     assert wb == 512 * 1152 + 64 and sb == 512 * 2
+    # INT4 groups of 32 and 64 k: one scale and zero point per group; per-channel
+    # (group = K) is stored as group 128 with the row's pair repeated
+    for g in (32, 64):
+        wb, sb, zb = wq.wq_packed_bytes(4, 5120, 25600, g)
+        assert wb == 5120 * 25600 // 2 + 64 and sb == 25600 * (5120 // g) * 2 and zb == 25600 * (5120 // g) // 2
+    assert wq.wq_packed_bytes(4, 5120, 25600, 5120) == wq.wq_packed_bytes(4, 5120, 25600, 128)
 
 
 @pytest.mark.parametrize("bits,K,N,group,status", [
     (8, 1024, 1024, 128, -4),   # INT8 takes no group
-    (4, 1024, 1024, 64, -4),    # only group 128
+    (4, 1024, 1024, 48, -4),    # groups: 32, 64, 128 or K
+    (4, 1024, 1024, 256, -4),   # neither a listed group nor K
     (4, 1000, 1024, 128, -2),   # K not a multiple of the group
     (8, 1000, 1024, 0, -2),     # K not a multiple of 32
     (8, 1024, 1000, 0, -2),     # N not a multiple of 16

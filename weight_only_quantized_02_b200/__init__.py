@@ -66,6 +66,7 @@ def _load():
         "wq_linear_ex": (I, [P, I, I, P, P, P, I, I, P, I, I, P, SZ, P]),
         "wq_linear_noalloc": (I, [P, I, I, P, P, P, I, I, P, P]),
         "wq_linear_topk": (I, [P, I, I, P, P, P, I, I, I, P, P, P, SZ, P]),
+        "wq_linear_f16": (I, [P, I, I, P, P, P, I, I, P, P]),
         "wq_topk_workspace_bytes": (SZ, [I, I, I]),
         "wq_workspace_bytes": (SZ, [I, I, I, I]),
         "wq_set_workspace": (I, [P, SZ]),
@@ -255,6 +256,16 @@ def wq_linear_noalloc(x: torch.Tensor, pw: PackedWeight, y: Optional[torch.Tenso
     y = _y_for(x, pw.N, y)
     _check(lib.wq_linear_noalloc(_p(x), M, K, _p(pw.wq), _p(pw.scales), _p(pw.zeros), pw.group, pw.N, _p(y),
                                  _s(stream)), "wq_linear_noalloc")
+    return y
+
+
+def wq_linear_f16(x: torch.Tensor, pw: PackedWeight, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """y = x . dequant(W)^T with fp16 activations and outputs; x fp16 [M][K]."""
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, pw.N), dtype=torch.float16, device=x.device)
+    _check(lib.wq_linear_f16(_p(x), M, K, _p(pw.wq), _p(pw.scales), _p(pw.zeros), pw.group, pw.N, _p(y),
+                             _s(stream)), "wq_linear_f16")
     return y
 
 

@@ -78,24 +78,21 @@ std::map<Key, Choice> g_table;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// group 0: INT8 per channel; otherwise INT4 with `group` k per scale (32,
+// 64, 128, or K for per channel; check_weight_shape has the rules).
 int bits_of_group(int group, int *bits)
 {
-    if (group == 0) {
-        *bits = 8;
-        return WQ_OK;
-    }
-    if (group == 128) {
-        *bits = 4;
-        return WQ_OK;
-    }
-    return WQ_ERR_GROUP;
+    if (group < 0)
+        return WQ_ERR_GROUP;
+    *bits = group == 0 ? 8 : 4;
+    return WQ_OK;
 }
 
 int check_weight_shape(int bits, int K, int N, int group)
 {
     if (bits == 8 && group != 0)
         return WQ_ERR_GROUP;
-    if (bits == 4 && group != 128)
+    if (bits == 4 && group != 32 && group != 64 && group != 128 && !(group == K && K > 0))
         return WQ_ERR_GROUP;
     if (bits != 4 && bits != 8)
         return WQ_ERR_GROUP;
@@ -121,8 +118,16 @@ size_t ws_bytes_imma(int bits, int M, int K, int N)
     return bits == 8 ? ws_bytes_gemm_i8(M, K, N) : ws_bytes_gemm_i4(M, K, N);
 }
 
-bool choice_valid(int variant, int split, int M, int K, int bits)
+// The INT4 layout group of the caller's group (0 for INT8).
+int lgroup_of(int bits, int K, int group) { return bits == 8 ? 0 : layout_group(K, group); }
+
+// Tokens per kernel launch: groups of 32 or 64 k run on the row-block GEMV only.
+int chunk_tokens(int bits, int lgroup) { return (bits == 4 && lgroup != 128) ? 32 : kChunkTokens; }
+
+bool choice_valid(int variant, int split, int M, int K, int bits, int lgroup = 128)
 {
+    if (bits == 4 && lgroup != 128) // the row-block GEMV is the one kernel with 32- and 64-k groups
+        return variant == WQ_VARIANT_GEMV_RB && M <= 32 && (split == 1 || split == 2 || split == 4 || split == 8);
     if (variant == WQ_VARIANT_I8MMA)
         return i8_fits(bits, M, K) && split == 1;
     if (variant == WQ_VARIANT_GEMV_I8)
@@ -160,8 +165,10 @@ int default_rb_slices(int K, int N, int sm_count)
 // Without a workspace: the row-block GEMV, else the pages' split_k = 8 GEMM
 // (run unsplit when no workspace holds its partials).
 Choice default_choice(int M, int K, int N, int bits, int sm_count, bool have_ws = true, bool have_i8_ws = true,
-                      bool have_gi_ws = true, bool have_w4_ws = true)
+                      bool have_gi_ws = true, bool have_w4_ws = true, int lgroup = 128)
 {
+    if (bits == 4 && lgroup != 128)
+        return {WQ_VARIANT_GEMV_RB, default_rb_slices(K, N, sm_count), 0.f};
     if (M < 8) {
         if (gi_fits(bits, M, K) && have_gi_ws)
             return {WQ_VARIANT_GEMV_I8, 1, 0.f};
@@ -178,6 +185,7 @@ Choice default_choice(int M, int K, int N, int bits, int sm_count, bool have_ws 
 
 int lookup_choice(const DeviceInfo &d, int M, int K, int N, int bits, int group, Choice *c)
 {
+    const int lg = lgroup_of(bits, K, group);
     {
         std::lock_guard<std::mutex> lk(g_mu);
         auto it = g_table.find(Key{device_key(d), M, K, N, bits, group});
@@ -186,7 +194,7 @@ int lookup_choice(const DeviceInfo &d, int M, int K, int N, int bits, int group,
             return WQ_OK;
         }
     }
-    *c = default_choice(M, K, N, bits, d.sm_count);
+    *c = default_choice(M, K, N, bits, d.sm_count, true, true, true, true, lg);
     return WQ_OK;
 }
 
@@ -205,7 +213,8 @@ int linear_chunk(const uint16_t *x, int M, int K, const void *Wq, const void *sc
         return WQ_ERR_NULL;
     if ((st = check_weight_shape(bits, K, N, group)) != WQ_OK)
         return st;
-    if (M < 1 || M > kChunkTokens)
+    const int lg = lgroup_of(bits, K, group);
+    if (M < 1 || M > chunk_tokens(bits, lg))
         return WQ_ERR_SHAPE;
     if (!aligned16(x) || !aligned16(y) || !aligned16(Wq) || !aligned16(scales) || (zeros && !aligned16(zeros)))
         return WQ_ERR_ALIGN;
@@ -253,9 +262,9 @@ int linear_chunk(const uint16_t *x, int M, int K, const void *Wq, const void *sc
         c.split = split;
     if (variant == WQ_VARIANT_AUTO) {
         const bool w4_ws_ok = w && have >= ws_bytes_gemm_sk(M, N);
-        if (!choice_valid(c.variant, c.split, M, K, bits) || (c.variant == WQ_VARIANT_I8MMA && !i8_ws_ok) ||
+        if (!choice_valid(c.variant, c.split, M, K, bits, lg) || (c.variant == WQ_VARIANT_I8MMA && !i8_ws_ok) ||
             (c.variant == WQ_VARIANT_GEMV_I8 && !gi_ws_ok) || (c.variant == WQ_VARIANT_GEMM_W4 && !w4_ws_ok))
-            c = default_choice(M, K, N, bits, d.sm_count, sk_ws_ok, i8_ws_ok, gi_ws_ok, w4_ws_ok);
+            c = default_choice(M, K, N, bits, d.sm_count, sk_ws_ok, i8_ws_ok, gi_ws_ok, w4_ws_ok, lg);
         if (c.variant == WQ_VARIANT_GEMV && !sk_ws_ok)
             c = {WQ_VARIANT_GEMV_RB, default_rb_slices(K, N, d.sm_count), 0.f};
         // an automatic choice never fails for lack of workspace: split-K GEMM
@@ -265,10 +274,10 @@ int linear_chunk(const uint16_t *x, int M, int K, const void *Wq, const void *sc
         if (c.variant == WQ_VARIANT_GEMM_SK && (!w || have < ws_bytes_gemm_sk(M, N)))
             c = {WQ_VARIANT_GEMM, 1, 0.f};
     }
-    if (!choice_valid(c.variant, c.split, M, K, bits))
+    if (!choice_valid(c.variant, c.split, M, K, bits, lg))
         return WQ_ERR_VARIANT;
 
-    LinearArgs a{x, M, K, N, Wq, scales, zeros, bits, group, y};
+    LinearArgs a{x, M, K, N, Wq, scales, zeros, bits, bits == 8 ? 0 : lg, y};
     if (c.variant == WQ_VARIANT_GEMV_I8) {
         if (!gi_ws_ok)
             return WQ_ERR_WORKSPACE;
@@ -311,14 +320,18 @@ int linear_chunk(const uint16_t *x, int M, int K, const void *Wq, const void *sc
 int linear_impl(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros, int group,
                 int N, uint16_t *y, int variant, int split, void *ws, size_t ws_bytes_given, cudaStream_t stream)
 {
-    if (M <= kChunkTokens)
+    int bits = 0;
+    if (bits_of_group(group, &bits) != WQ_OK)
+        return WQ_ERR_GROUP;
+    const int chunk = chunk_tokens(bits, lgroup_of(bits, K, group));
+    if (M <= chunk)
         return linear_chunk(x, M, K, Wq, scales, zeros, group, N, y, variant, split, ws, ws_bytes_given, stream);
     if (M > kMaxTokens)
         return WQ_ERR_SHAPE;
     if (!x || !y)
         return WQ_ERR_NULL;
-    for (int m0 = 0; m0 < M; m0 += kChunkTokens) {
-        const int mc = std::min(kChunkTokens, M - m0);
+    for (int m0 = 0; m0 < M; m0 += chunk) {
+        const int mc = std::min(chunk, M - m0);
         const int st = linear_chunk(x + (size_t)m0 * K, mc, K, Wq, scales, zeros, group, N, y + (size_t)m0 * N,
                                     variant, split, ws, ws_bytes_given, stream);
         if (st != WQ_OK)
@@ -407,7 +420,7 @@ int wq_packed_bytes(int bits, int K, int N, int group, size_t *wq_bytes, size_t 
     const int st = check_weight_shape(bits, K, N, group);
     if (st != WQ_OK)
         return st;
-    const Shape sh{bits, K, N, group};
+    const Shape sh{bits, K, N, lgroup_of(bits, K, group)};
     if (wq_bytes)
         *wq_bytes = sh.wq_bytes();
     if (scale_bytes)
@@ -431,11 +444,11 @@ int wq_quantize_int4(const float *W, int K, int N, int group, uint32_t *q_out, u
 {
     if (!W || !q_out || !s_out || !z_out)
         return WQ_ERR_NULL;
-    if (group != 128)
-        return WQ_ERR_GROUP;
     if (K <= 0 || N <= 0 || K % 128 != 0)
         return WQ_ERR_SHAPE;
-    return cuda_status(launch_quantize_int4(W, K, N, q_out, s_out, z_out, stream));
+    if (group != 32 && group != 64 && group != 128 && group != K)
+        return WQ_ERR_GROUP;
+    return cuda_status(launch_quantize_int4(W, K, N, group, q_out, s_out, z_out, stream));
 }
 
 int wq_pack_int8(const int8_t *q, const uint16_t *scales, int K, int N, void *wq_out, void *scales_out,
@@ -461,7 +474,7 @@ int wq_pack_int4(const uint32_t *q, const uint16_t *scales, const uint32_t *zero
         return st;
     if (!aligned16(wq_out) || !aligned16(scales_out) || !aligned16(zeros_out))
         return WQ_ERR_ALIGN;
-    return cuda_status(launch_pack_int4(q, scales, zeros, K, N, wq_out, scales_out, zeros_out, stream));
+    return cuda_status(launch_pack_int4(q, scales, zeros, K, N, group, wq_out, scales_out, zeros_out, stream));
 }
 
 int wq_check_packed(const void *Wq, int bits, int K, int N, int group, cudaStream_t stream)
@@ -471,7 +484,7 @@ int wq_check_packed(const void *Wq, int bits, int K, int N, int group, cudaStrea
     int st = check_weight_shape(bits, K, N, group);
     if (st != WQ_OK)
         return st;
-    const Shape sh{bits, K, N, group};
+    const Shape sh{bits, K, N, lgroup_of(bits, K, group)};
     Trailer t;
     if (cudaMemcpyAsync(&t, (const uint8_t *)Wq + sh.weight_bytes(), sizeof t, cudaMemcpyDeviceToHost, stream) !=
             cudaSuccess ||
@@ -514,6 +527,8 @@ int wq_linear_noalloc(const uint16_t *x, int M, int K, const void *Wq, const voi
         return WQ_ERR_NULL;
     if ((st = check_weight_shape(bits, K, N, group)) != WQ_OK)
         return st;
+    if (bits == 4 && lgroup_of(bits, K, group) != 128)
+        return WQ_ERR_GROUP; // the stream-K GEMV reads the group-128 layout
     if (M < 1 || M > noalloc_max_m() || N > noalloc_max_n())
         return WQ_ERR_SHAPE;
     if (!aligned16(x) || !aligned16(y) || !aligned16(Wq) || !aligned16(scales) || (zeros && !aligned16(zeros)))
@@ -523,8 +538,38 @@ int wq_linear_noalloc(const uint16_t *x, int M, int K, const void *Wq, const voi
         return st;
     if (d.major != 10)
         return WQ_ERR_ARCH;
-    LinearArgs a{x, M, K, N, Wq, scales, zeros, bits, group, y};
+    LinearArgs a{x, M, K, N, Wq, scales, zeros, bits, bits == 8 ? 0 : 128, y};
     return cuda_status(launch_gemv_sk_noalloc(a, d.sm_count, stream));
+}
+
+int wq_linear_f16(const uint16_t *x, int M, int K, const void *Wq, const void *scales, const void *zeros, int group,
+                  int N, uint16_t *y, cudaStream_t stream)
+{
+    int bits = 0;
+    int st = bits_of_group(group, &bits);
+    if (st != WQ_OK)
+        return st;
+    if (!x || !Wq || !scales || !y || (bits == 4 && !zeros))
+        return WQ_ERR_NULL;
+    if ((st = check_weight_shape(bits, K, N, group)) != WQ_OK)
+        return st;
+    if (M < 1 || M > kMaxTokens)
+        return WQ_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(Wq) || !aligned16(scales) || (zeros && !aligned16(zeros)))
+        return WQ_ERR_ALIGN;
+    DeviceInfo d;
+    if ((st = current_device_info(&d)) != WQ_OK)
+        return st;
+    if (d.major != 10)
+        return WQ_ERR_ARCH;
+    const int lg = lgroup_of(bits, K, group), ks = default_rb_slices(K, N, d.sm_count);
+    for (int m0 = 0; m0 < M; m0 += 32) { // the row-block GEMV: 32 tokens per launch
+        const int mc = std::min(32, M - m0);
+        LinearArgs a{x + (size_t)m0 * K, mc, K, N, Wq, scales, zeros, bits, bits == 8 ? 0 : lg, y + (size_t)m0 * N};
+        if ((st = cuda_status(launch_gemv(a, ks, d.sm_count, stream, true))) != WQ_OK)
+            return st;
+    }
+    return WQ_OK;
 }
 
 size_t wq_topk_workspace_bytes(int M, int N, int k)
@@ -606,9 +651,15 @@ int wq_tune(const uint16_t *x, int M, int K, const void *Wq, const void *scales,
         return st;
     if (warmup < 0 || iters < 1 || M < 1 || M > kMaxTokens)
         return WQ_ERR_SHAPE;
-    M = std::min(M, kChunkTokens); // longer inputs: the chunk shape, timed on the first chunk
+    if ((st = check_weight_shape(bits, K, N, group)) != WQ_OK)
+        return st;
+    const int lg = lgroup_of(bits, K, group);
+    M = std::min(M, chunk_tokens(bits, lg)); // longer inputs: the chunk shape, timed on the first chunk
     std::vector<std::pair<int, int>> cands;
-    if (M <= 32) {
+    if (bits == 4 && lg != 128) {
+        for (int ks : {1, 2, 4, 8})
+            cands.push_back({WQ_VARIANT_GEMV_RB, ks});
+    } else if (M <= 32) {
         for (int c : {1, 2, 3})
             cands.push_back({WQ_VARIANT_GEMV, c});
         for (int ks : {1, 2, 4, 8})
@@ -738,7 +789,7 @@ int wq_get_choice(int M, int K, int N, int bits, int group, int *variant, int *s
     if (st != WQ_OK)
         return st;
     Choice c;
-    lookup_choice(d, std::min(M, kChunkTokens), K, N, bits, group, &c);
+    lookup_choice(d, std::min(M, chunk_tokens(bits, lgroup_of(bits, K, group))), K, N, bits, group, &c);
     *variant = c.variant;
     *split = c.split;
     return WQ_OK;
@@ -750,7 +801,7 @@ int wq_set_choice(int M, int K, int N, int bits, int group, int variant, int spl
     int st = current_device_info(&d);
     if (st != WQ_OK)
         return st;
-    if (!choice_valid(variant, split, M, K, bits))
+    if (check_weight_shape(bits, K, N, group) != WQ_OK || !choice_valid(variant, split, M, K, bits, lgroup_of(bits, K, group)))
         return WQ_ERR_VARIANT;
     std::lock_guard<std::mutex> lk(g_mu);
     g_table[Key{device_key(d), M, K, N, bits, group}] = Choice{variant, split, 0.f};
@@ -820,7 +871,7 @@ int wq_load_tuning(const char *path)
         const int n = sscanf(rest, " %d %d %d %d %d %d %d %f %c", &M, &K, &N, &bits, &group, &variant, &split, &us,
                              &tail);
         if (n != 8 || check_weight_shape(bits, K, N, group) != WQ_OK || M < 1 || M > 128 ||
-            !choice_valid(variant, split, M, K, bits)) {
+            !choice_valid(variant, split, M, K, bits, lgroup_of(bits, K, group))) {
             bad = true;
             break;
         }
@@ -846,7 +897,8 @@ int wq_unpack_debug(const void *Wq, const void *zeros, int bits, int K, int N, i
     const int st = check_weight_shape(bits, K, N, group);
     if (st != WQ_OK)
         return st;
-    return cuda_status(launch_unpack_debug(Wq, zeros, Shape{bits, K, N, group}, q_out, z_out, stream));
+    return cuda_status(
+        launch_unpack_debug(Wq, zeros, Shape{bits, K, N, lgroup_of(bits, K, group)}, group, q_out, z_out, stream));
 }
 
 int wq_dequant_debug(const void *Wq, const void *scales, const void *zeros, int bits, int K, int N, int group,
@@ -857,7 +909,8 @@ int wq_dequant_debug(const void *Wq, const void *scales, const void *zeros, int 
     const int st = check_weight_shape(bits, K, N, group);
     if (st != WQ_OK)
         return st;
-    return cuda_status(launch_dequant_debug(Wq, scales, zeros, Shape{bits, K, N, group}, w_out, stream));
+    return cuda_status(
+        launch_dequant_debug(Wq, scales, zeros, Shape{bits, K, N, lgroup_of(bits, K, group)}, w_out, stream));
 }
 
 int wq_wait_selftest(int limit_us, cudaStream_t stream)

@@ -64,19 +64,20 @@ int i8_digit_rows(int M);
 size_t ws_bytes_gemm_i8(int M, int K, int N);
 
 cudaError_t launch_quantize_int8(const float *W, int K, int N, int8_t *q, uint16_t *s, cudaStream_t st);
-cudaError_t launch_quantize_int4(const float *W, int K, int N, uint32_t *q, uint16_t *s, uint32_t *z,
+cudaError_t launch_quantize_int4(const float *W, int K, int N, int G, uint32_t *q, uint16_t *s, uint32_t *z,
                                  cudaStream_t st);
 cudaError_t launch_pack_int8(const int8_t *q, const uint16_t *s, int K, int N, void *wq, void *s_out,
                              cudaStream_t st);
-cudaError_t launch_pack_int4(const uint32_t *q, const uint16_t *s, const uint32_t *z, int K, int N, void *wq,
-                             void *s_out, void *z_out, cudaStream_t st);
-cudaError_t launch_unpack_debug(const void *wq, const void *zeros, const Shape &sh, int8_t *q_out,
+cudaError_t launch_pack_int4(const uint32_t *q, const uint16_t *s, const uint32_t *z, int K, int N, int G,
+                             void *wq, void *s_out, void *z_out, cudaStream_t st);
+cudaError_t launch_unpack_debug(const void *wq, const void *zeros, const Shape &sh, int G, int8_t *q_out,
                                 int8_t *z_out, cudaStream_t st);
 cudaError_t launch_dequant_debug(const void *wq, const void *scales, const void *zeros, const Shape &sh,
                                  float *w_out, cudaStream_t st);
 
-// GEMV: ks = K slices per 16-row block (1, 2, 4, 8); M <= 32.
-cudaError_t launch_gemv(const LinearArgs &a, int ks, int sm_count, cudaStream_t st);
+// GEMV: ks = K slices per 16-row block (1, 2, 4, 8); M <= 32; f16: fp16
+// activations and outputs instead of bf16.
+cudaError_t launch_gemv(const LinearArgs &a, int ks, int sm_count, cudaStream_t st, bool f16 = false);
 
 // Stream-K GEMV: ctas_per_sm = 0 (occupancy) or 1/2; ws >= ws_bytes_gemv_sk.
 cudaError_t launch_gemv_sk(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st);

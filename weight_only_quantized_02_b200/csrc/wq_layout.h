@@ -36,9 +36,13 @@
 // one contiguous 512-byte segment.
 //
 // Rows past N and k past K are zero in both formats.
-// Scales: INT8 bf16 [P*128] (s[n], zero past N).  INT4 bf16 [P][K/128][128].
-// Zeros (INT4): [P][K/128][128 nibbles = 64 bytes], row i at nibble i
-// (low nibble first).  A 64-byte trailer follows the packed weights.
+// Scales: INT8 bf16 [P*128] (s[n], zero past N).  INT4 bf16 [P][K/L][128]
+// for the layout group L = 32, 64 or 128 (k = L g .. L g + L - 1 share one
+// scale and zero point).  Zeros (INT4): [P][K/L][128 nibbles = 64 bytes],
+// row i at nibble i (low nibble first).  Per-channel INT4 (one scale and
+// zero point per row, group = K) is stored as L = 128 with the row's pair
+// repeated in every 128-k block, so it runs on every group-128 kernel.
+// A 64-byte trailer follows the packed weights.
 #pragma once
 
 #include <cstddef>
@@ -62,7 +66,7 @@ constexpr uint32_t kLayoutVersion = 3;
 struct Shape {
     int bits;  // 4 or 8
     int K, N;
-    int group; // 128 (INT4) or 0 (INT8)
+    int group; // INT4: the layout group L (32, 64 or 128); INT8: 0
     WQ_HD int panels() const { return (N + kPanelRows - 1) / kPanelRows; }
     WQ_HD int kblocks() const { return (K + kBlockK - 1) / kBlockK; }
     WQ_HD int tile_k() const { return bits == 4 ? 64 : 32; }
@@ -71,12 +75,13 @@ struct Shape {
     WQ_HD int block_bytes() const { return 8 * rb_bytes(); }                       // one panel, 128 k
     WQ_HD size_t weight_bytes() const { return (size_t)panels() * kblocks() * block_bytes(); }
     WQ_HD size_t wq_bytes() const { return weight_bytes() + kTrailerBytes; }
+    WQ_HD int groups() const { return bits == 8 ? 0 : K / group; } // INT4 scale groups per row
     WQ_HD size_t scale_bytes() const
     {
         return bits == 8 ? (size_t)panels() * kPanelRows * 2
-                         : (size_t)panels() * kblocks() * kPanelRows * 2;
+                         : (size_t)panels() * groups() * kPanelRows * 2;
     }
-    WQ_HD size_t zero_bytes() const { return bits == 8 ? 0 : (size_t)panels() * kblocks() * 64; }
+    WQ_HD size_t zero_bytes() const { return bits == 8 ? 0 : (size_t)panels() * groups() * 64; }
     // INT4: byte offset of tile (row-block rb = 16-row index, k tile index kt)
     WQ_HD size_t tile_offset(int rb, int kt) const
     {
@@ -87,6 +92,10 @@ struct Shape {
     }
     WQ_HD size_t block_offset(int p, int kb) const { return (size_t)(p * kblocks() + kb) * block_bytes(); }
 };
+
+// The layout group of an INT4 weight quantized with `group` consecutive k per
+// scale: per-channel (group == K > 128) is stored as 128.
+WQ_HD int layout_group(int K, int group) { return (group == K && K > 128) ? 128 : group; }
 
 // INT8: byte offset of element (r, kk) inside its block (r = row in the
 // panel 0..127, kk = k in the block 0..127).

@@ -84,36 +84,31 @@ __global__ void __launch_bounds__(256) quant_int8_kernel(const float *__restrict
 }
 
 // ---------------------------------------------------------------------------
-// INT4 asymmetric group quantizer: a half-warp per (row, group of 128), each
-// lane owning 8 consecutive k (one canonical word).
+// INT4 asymmetric group quantizer: a warp per (row, group of G), each lane
+// taking words of 8 consecutive k (one canonical word) in turn.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) quant_int4_kernel(const float *__restrict__ W, int K, int N,
+__global__ void __launch_bounds__(256) quant_int4_kernel(const float *__restrict__ W, int K, int N, int G,
                                                          uint32_t *__restrict__ q,
                                                          uint16_t *__restrict__ s,
                                                          uint32_t *__restrict__ z)
 {
-    const int KG = K / 128, ZW = (KG + 7) / 8;
-    const long long unit = (long long)blockIdx.x * 16 + (threadIdx.x >> 4);
-    const int l16 = threadIdx.x & 15;
-    const bool active = unit < (long long)N * KG;
-    const int n = active ? (int)(unit / KG) : 0;
-    const int g = active ? (int)(unit % KG) : 0;
-    float v[8];
-    const float *src = W + (size_t)n * K + (size_t)g * 128 + 8 * l16;
+    const int KG = K / G, ZW = (KG + 7) / 8;
+    const long long unit = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (unit >= (long long)N * KG)
+        return; // the whole warp
+    const int n = (int)(unit / KG), g = (int)(unit % KG);
+    const float *src = W + (size_t)n * K + (size_t)g * G;
     float mn = 0.f, mx = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        v[e] = active ? src[e] : 0.f;
-        mn = fminf(mn, v[e]);
-        mx = fmaxf(mx, v[e]);
+    for (int k = lane; k < G; k += 32) {
+        mn = fminf(mn, src[k]);
+        mx = fmaxf(mx, src[k]);
     }
 #pragma unroll
-    for (int o = 8; o; o >>= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o, 16));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o, 16));
+    for (int o = 16; o; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
-    if (!active)
-        return;
     const double lo = (double)mn, hi = (double)mx; // lo <= 0 <= hi
     uint16_t sb = 0;
     double sd = 0.0;
@@ -123,16 +118,18 @@ __global__ void __launch_bounds__(256) quant_int4_kernel(const float *__restrict
         sd = (double)bf16_bits_to_float(sb);
         zq = (uint32_t)fmin(fmax(rint(-lo / sd), 0.0), 15.0);
     }
-    uint32_t word = 0;
+    for (int wi = lane; wi < G / 8; wi += 32) {
+        uint32_t word = 0;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        uint32_t qe = 0;
-        if (sd != 0.0)
-            qe = (uint32_t)fmin(fmax(rint((double)v[e] / sd) + (double)zq, 0.0), 15.0);
-        word |= qe << (4 * e);
+        for (int e = 0; e < 8; ++e) {
+            uint32_t qe = 0;
+            if (sd != 0.0)
+                qe = (uint32_t)fmin(fmax(rint((double)src[8 * wi + e] / sd) + (double)zq, 0.0), 15.0);
+            word |= qe << (4 * e);
+        }
+        q[(size_t)n * (K / 8) + (size_t)g * (G / 8) + wi] = word;
     }
-    q[(size_t)n * (K / 8) + (size_t)g * 16 + l16] = word;
-    if (l16 == 0) {
+    if (lane == 0) {
         s[(size_t)n * KG + g] = sb;
         if (zq)
             atomicOr(&z[(size_t)n * ZW + g / 8], zq << (4 * (g % 8)));
@@ -224,16 +221,20 @@ __global__ void pack_scales_int8_kernel(const uint16_t *__restrict__ s, int N, u
     wmax_fold(wmax_bits, 128.f * fabsf(__uint_as_float((uint32_t)v << 16)));
 }
 
+// Layout group gl of row `row` takes canonical group gl * L / G (G = the
+// quantization group: equal to L, or K for per-channel, repeated per block).
 __global__ void pack_sz_int4_kernel(const uint16_t *__restrict__ s, const uint32_t *__restrict__ z, int K,
-                                    int N, uint16_t *__restrict__ s_out, uint8_t *__restrict__ z_out,
+                                    int N, int G, uint16_t *__restrict__ s_out, uint8_t *__restrict__ z_out,
                                     Shape sh, uint32_t *wmax_bits)
 {
-    const int KG = K / 128, ZW = (KG + 7) / 8;
+    const int L = sh.group, KL = K / L;         // layout groups per row
+    const int KG = K / G, ZW = (KG + 7) / 8;     // canonical groups per row, zero-point words
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long total = (long long)sh.panels() * KG * kPanelRows;
+    const long long total = (long long)sh.panels() * KL * kPanelRows;
     const int i = (int)(idx % kPanelRows);
     const long long pg = idx / kPanelRows;
-    const int g = (int)(pg % KG), p = (int)(pg / KG);
+    const int gl = (int)(pg % KL), p = (int)(pg / KL);
+    const int g = (int)((long long)gl * L / G);
     const int row = p * kPanelRows + i;
     // largest |q - z| the zero point allows, times the scale
     float wm = 0.f;
@@ -255,7 +256,9 @@ __global__ void pack_sz_int4_kernel(const uint16_t *__restrict__ s, const uint32
     }
 }
 
-__global__ void write_trailer_kernel(uint8_t *wq, Shape sh)
+// group: the quantization group the caller packed (0 for INT8, K for
+// per-channel INT4), recorded for wq_check_packed.
+__global__ void write_trailer_kernel(uint8_t *wq, Shape sh, int group)
 {
     Trailer t{};
     t.magic = kMagic;
@@ -263,7 +266,7 @@ __global__ void write_trailer_kernel(uint8_t *wq, Shape sh)
     t.bits = (uint32_t)sh.bits;
     t.K = (uint32_t)sh.K;
     t.N = (uint32_t)sh.N;
-    t.group = (uint32_t)sh.group;
+    t.group = (uint32_t)group;
     const size_t wb = sh.weight_bytes();
     t.layout_bytes_lo = (uint32_t)(wb & 0xffffffffu);
     t.layout_bytes_hi = (uint32_t)(wb >> 32);
@@ -293,14 +296,16 @@ __device__ int packed_q(const uint8_t *wq, const Shape &sh, int n, int k)
     return (int)((w >> (4 * int4_nibble_pos(e))) & 0xFu);
 }
 
-__device__ int packed_z(const uint8_t *zeros, const Shape &sh, int n, int g)
+// Zero point of row n in layout group gl.
+__device__ int packed_z(const uint8_t *zeros, const Shape &sh, int n, int gl)
 {
     const int p = n / kPanelRows, i = n % kPanelRows;
-    const uint8_t b = zeros[((size_t)p * sh.kblocks() + g) * 64 + i / 2];
+    const uint8_t b = zeros[((size_t)p * sh.groups() + gl) * 64 + i / 2];
     return (i & 1) ? (b >> 4) : (b & 0xF);
 }
 
-__global__ void unpack_debug_kernel(const uint8_t *wq, const uint8_t *zeros, Shape sh, int8_t *q_out,
+// z_out: one zero point per quantization group G of the caller ([N][K/G]).
+__global__ void unpack_debug_kernel(const uint8_t *wq, const uint8_t *zeros, Shape sh, int G, int8_t *q_out,
                                     int8_t *z_out)
 {
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -309,8 +314,8 @@ __global__ void unpack_debug_kernel(const uint8_t *wq, const uint8_t *zeros, Sha
         return;
     const int n = (int)(idx / sh.K), k = (int)(idx % sh.K);
     q_out[idx] = (int8_t)packed_q(wq, sh, n, k);
-    if (sh.bits == 4 && z_out && (k % 128) == 0)
-        z_out[(size_t)n * (sh.K / 128) + k / 128] = (int8_t)packed_z(zeros, sh, n, k / 128);
+    if (sh.bits == 4 && z_out && (k % G) == 0)
+        z_out[(size_t)n * (sh.K / G) + k / G] = (int8_t)packed_z(zeros, sh, n, k / sh.group);
 }
 
 __global__ void dequant_debug_kernel(const uint8_t *wq, const uint16_t *scales, const uint8_t *zeros,
@@ -325,9 +330,9 @@ __global__ void dequant_debug_kernel(const uint8_t *wq, const uint16_t *scales, 
     if (sh.bits == 8) {
         w_out[idx] = bf16_bits_to_float(scales[n]) * (float)q;
     } else {
-        const int p = n / kPanelRows, i = n % kPanelRows, g = k / 128;
-        const float s = bf16_bits_to_float(scales[((size_t)p * sh.kblocks() + g) * kPanelRows + i]);
-        w_out[idx] = s * (float)(q - packed_z(zeros, sh, n, g));
+        const int p = n / kPanelRows, i = n % kPanelRows, gl = k / sh.group;
+        const float s = bf16_bits_to_float(scales[((size_t)p * sh.groups() + gl) * kPanelRows + i]);
+        w_out[idx] = s * (float)(q - packed_z(zeros, sh, n, gl));
     }
 }
 
@@ -342,15 +347,15 @@ cudaError_t launch_quantize_int8(const float *W, int K, int N, int8_t *q, uint16
     return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_int4(const float *W, int K, int N, uint32_t *q, uint16_t *s, uint32_t *z,
+cudaError_t launch_quantize_int4(const float *W, int K, int N, int G, uint32_t *q, uint16_t *s, uint32_t *z,
                                  cudaStream_t st)
 {
-    const int KG = K / 128, ZW = (KG + 7) / 8;
+    const int KG = K / G, ZW = (KG + 7) / 8;
     cudaError_t e = cudaMemsetAsync(z, 0, (size_t)N * ZW * sizeof(uint32_t), st);
     if (e != cudaSuccess)
         return e;
     const long long units = (long long)N * KG;
-    quant_int4_kernel<<<nblk(units, 16), 256, 0, st>>>(W, K, N, q, s, z);
+    quant_int4_kernel<<<nblk(units, 8), 256, 0, st>>>(W, K, N, G, q, s, z);
     return cudaGetLastError();
 }
 
@@ -359,7 +364,7 @@ cudaError_t launch_pack_int8(const int8_t *q, const uint16_t *s, int K, int N, v
 {
     const Shape sh{8, K, N, 0};
     const size_t n_vec = sh.weight_bytes() / 16;
-    write_trailer_kernel<<<1, 1, 0, st>>>((uint8_t *)wq, sh); // first: wmax_bits starts at 0
+    write_trailer_kernel<<<1, 1, 0, st>>>((uint8_t *)wq, sh, 0); // first: wmax_bits starts at 0
     pack_int8_kernel<<<nblk((long long)n_vec, 256), 256, 0, st>>>(q, K, N, (uint4 *)wq, n_vec, sh);
     const int total = sh.panels() * kPanelRows;
     pack_scales_int8_kernel<<<nblk(total, 256), 256, 0, st>>>(s, N, (uint16_t *)s_out, total,
@@ -367,24 +372,24 @@ cudaError_t launch_pack_int8(const int8_t *q, const uint16_t *s, int K, int N, v
     return cudaGetLastError();
 }
 
-cudaError_t launch_pack_int4(const uint32_t *q, const uint16_t *s, const uint32_t *z, int K, int N,
+cudaError_t launch_pack_int4(const uint32_t *q, const uint16_t *s, const uint32_t *z, int K, int N, int G,
                              void *wq, void *s_out, void *z_out, cudaStream_t st)
 {
-    const Shape sh{4, K, N, 128};
+    const Shape sh{4, K, N, layout_group(K, G)};
     const size_t n_vec = sh.weight_bytes() / 16;
-    write_trailer_kernel<<<1, 1, 0, st>>>((uint8_t *)wq, sh); // first: wmax_bits starts at 0
+    write_trailer_kernel<<<1, 1, 0, st>>>((uint8_t *)wq, sh, G); // first: wmax_bits starts at 0
     pack_int4_kernel<<<nblk((long long)n_vec, 256), 256, 0, st>>>(q, K, N, (uint4 *)wq, n_vec, sh);
-    const long long total = (long long)sh.panels() * (K / 128) * kPanelRows;
-    pack_sz_int4_kernel<<<nblk(total, 256), 256, 0, st>>>(s, z, K, N, (uint16_t *)s_out, (uint8_t *)z_out, sh,
+    const long long total = (long long)sh.panels() * sh.groups() * kPanelRows;
+    pack_sz_int4_kernel<<<nblk(total, 256), 256, 0, st>>>(s, z, K, N, G, (uint16_t *)s_out, (uint8_t *)z_out, sh,
                                                           const_cast<uint32_t *>(trailer_wmax(wq, sh)));
     return cudaGetLastError();
 }
 
-cudaError_t launch_unpack_debug(const void *wq, const void *zeros, const Shape &sh, int8_t *q_out,
+cudaError_t launch_unpack_debug(const void *wq, const void *zeros, const Shape &sh, int G, int8_t *q_out,
                                 int8_t *z_out, cudaStream_t st)
 {
     const long long total = (long long)sh.N * sh.K;
-    unpack_debug_kernel<<<nblk(total, 256), 256, 0, st>>>((const uint8_t *)wq, (const uint8_t *)zeros, sh,
+    unpack_debug_kernel<<<nblk(total, 256), 256, 0, st>>>((const uint8_t *)wq, (const uint8_t *)zeros, sh, G,
                                                          q_out, z_out);
     return cudaGetLastError();
 }

@@ -63,7 +63,8 @@ def test_packed_bytes():
     (4, 1024, 1024, 256, -4),   # neither a listed group nor K
     (4, 1000, 1024, 128, -2),   # K not a multiple of the group
     (8, 1000, 1024, 0, -2),     # K not a multiple of 32
-    (8, 1024, 1000, 0, -2),     # N not a multiple of 16
+    (8, 1040, 1024, 0, -2),     # INT8: K % 32 (a multiple of 16 is not enough: 32-k integer MMA steps)
+    (8, 1024, 1000, 0, -2),     # N not a multiple of 16 (a multiple of 8 is not enough: 16-row blocks)
     (8, 0, 1024, 0, -2),
     (3, 1024, 1024, 0, -4),
 ])

@@ -6,14 +6,17 @@
 // The logits come from the layer's own kernels into a scratch buffer (bf16,
 // M x N, L2-resident at decode sizes: 4.9 MB for 16 tokens of a 152064-entry
 // vocabulary, against 779 MB of INT8 weights); two small kernels then select:
-//   part   grid (P, M): CTA (p, m) takes logits [p S, p S + S) of token m,
-//          sorts them in shared memory and keeps its k largest;
-//   merge  grid M: CTA m sorts the P k candidates of token m and writes the
-//          k largest, descending.
-// Keys are 64-bit: an order-preserving image of the binary32 value in the high
-// half and the complement of the index in the low half, so a descending sort
-// puts larger values first and, among equal values, the lower index first:
-// the result is unique and deterministic.
+//   part   grid (P, M): CTA (p, m) takes logits [p S, p S + S) of token m and
+//          keeps its k largest, in index order;
+//   merge  grid M: CTA m takes the P k candidates of token m (in index
+//          order, since the slices are) and writes the k largest, descending.
+// Both select with a radix select on 16-bit order-preserving keys (a bf16
+// logit has 16 bits): two passes of an 8-bit histogram find the k-th
+// largest key t exactly; every key above t is kept, and of the keys equal
+// to t the ones with the lowest indices, found by an order-preserving
+// compaction.  The k survivors of the merge are sorted (descending value,
+// then ascending index), so the result is unique and deterministic: ties
+// between equal logits go to the lower index.
 #include <cstdint>
 
 #include <cuda_bf16.h>
@@ -26,109 +29,227 @@ namespace wq {
 namespace {
 
 constexpr int kTopkThreads = 512;
+constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kPartSlice = 4096; // logits per part CTA
 
-__device__ __forceinline__ unsigned long long topk_key(uint16_t bf16_bits, uint32_t index)
+// bf16 bits -> a 16-bit key that orders like the value (-0 and +0 equal).
+__device__ __forceinline__ uint32_t order16(uint16_t b)
 {
-    uint32_t u = (uint32_t)bf16_bits << 16;
-    if ((u << 1) == 0u)
-        u = 0u; // -0 and +0 are one value (and tie on the index)
-    const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u); // monotone in the value
-    return ((unsigned long long)ord << 32) | (uint32_t)~index;
+    if ((b & 0x7FFFu) == 0)
+        b = 0;
+    return (b & 0x8000u) ? (uint32_t)(~b & 0xFFFFu) : (uint32_t)(b | 0x8000u);
 }
 
-__device__ __forceinline__ uint16_t key_value(unsigned long long key)
+__device__ __forceinline__ uint16_t value16(uint32_t key16)
 {
-    const uint32_t ord = (uint32_t)(key >> 32);
-    const uint32_t u = (ord & 0x80000000u) ? (ord ^ 0x80000000u) : ~ord;
-    return (uint16_t)(u >> 16);
+    return (uint16_t)((key16 & 0x8000u) ? (key16 & 0x7FFFu) : (~key16 & 0xFFFFu));
 }
 
-__device__ __forceinline__ int32_t key_index(unsigned long long key) { return (int32_t)~(uint32_t)key; }
-
-// Bitonic sort of n = 2^j keys in shared memory, descending; all threads of
-// the CTA call it.
-__device__ void bitonic_desc(unsigned long long *s, int n)
+// Exact k-th largest of the n keys in s (16-bit keys in uint32), by two
+// 8-bit passes; every thread of the CTA calls it.  Returns t and, in *ties,
+// how many keys equal to t belong to the k largest.
+__device__ uint32_t radix_select16(const uint32_t *s, int n, int k, uint32_t *hist, int *ties)
 {
-    for (int size = 2; size <= n; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = threadIdx.x; i < (n >> 1); i += blockDim.x) {
-                const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
-                const bool desc = (lo & size) == 0;
-                const unsigned long long a = s[lo], b = s[hi];
-                if ((a < b) == desc) {
-                    s[lo] = b;
-                    s[hi] = a;
-                }
+    __shared__ uint32_t s_prefix;
+    __shared__ int s_rank;
+    uint32_t *wh = hist + (threadIdx.x >> 5) * 256; // one 256-bin histogram per warp
+    if (threadIdx.x == 0) {
+        s_prefix = 0;
+        s_rank = k;
+    }
+    for (int pass = 1; pass >= 0; --pass) {
+        for (int i = threadIdx.x; i < kTopkWarps * 256; i += blockDim.x)
+            hist[i] = 0;
+        __syncthreads();
+        const uint32_t prefix = s_prefix, shift = 8 * pass;
+        const uint32_t hi_mask = pass == 1 ? 0u : 0xFF00u;
+        // logits crowd into a few bins: lanes with the same bin add once
+        // (their count) instead of contending for the same word
+        for (int i0 = 0; i0 < n; i0 += blockDim.x) {
+            const int i = i0 + threadIdx.x;
+            const uint32_t key = i < n ? s[i] : 0u;
+            const bool in = i < n && (key & hi_mask) == prefix;
+            const uint32_t bin = in ? (key >> shift) & 0xFFu : 256u;
+            const uint32_t same = __match_any_sync(0xffffffffu, bin);
+            if (in && (threadIdx.x & 31) == (uint32_t)(__ffs(same) - 1))
+                atomicAdd(&wh[bin], (uint32_t)__popc(same));
+        }
+        __syncthreads();
+        if (threadIdx.x < 256) { // fold the warp histograms
+            uint32_t c = 0;
+            for (int w = 0; w < kTopkWarps; ++w)
+                c += hist[w * 256 + threadIdx.x];
+            hist[threadIdx.x] = c;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) { // the digit holding the rank-th largest, from the top
+            int rank = s_rank, d = 255;
+            for (; d > 0; --d) {
+                if ((int)hist[d] >= rank)
+                    break;
+                rank -= (int)hist[d];
             }
-            __syncthreads();
+            s_rank = rank;
+            s_prefix = prefix | ((uint32_t)d << shift);
+        }
+        __syncthreads();
+    }
+    *ties = s_rank;
+    return s_prefix;
+}
+
+// Exclusive prefix sums over the CTA's threads, in thread order, of two
+// per-thread counts (warp shuffles, then the warp totals); every thread
+// calls it.  scratch: 2 * kTopkWarps ints.
+__device__ __forceinline__ void block_scan2(int a, int b, int &ea, int &eb, int *scratch)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int ia = a, ib = b; // inclusive within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int ua = __shfl_up_sync(0xffffffffu, ia, o), ub = __shfl_up_sync(0xffffffffu, ib, o);
+        if (lane >= o) {
+            ia += ua;
+            ib += ub;
         }
     }
-}
-
-// CTA (p, m): the k largest keys among logits[m][p S .. min(N, p S + S)).
-__global__ void __launch_bounds__(kTopkThreads) topk_part_kernel(const uint16_t *__restrict__ logits, int N, int S,
-                                                                 int k, unsigned long long *__restrict__ cand)
-{
-    extern __shared__ unsigned long long sk[];
-    const int p = blockIdx.x, m = blockIdx.y, P = gridDim.x;
-    const int n0 = p * S;
-    const uint16_t *row = logits + (size_t)m * N;
-    for (int i = threadIdx.x; i < S; i += blockDim.x) {
-        const int n = n0 + i;
-        sk[i] = n < N ? topk_key(row[n], (uint32_t)n) : 0ull; // 0: below every real key
+    if (lane == 31) {
+        scratch[warp] = ia;
+        scratch[kTopkWarps + warp] = ib;
     }
     __syncthreads();
-    bitonic_desc(sk, S);
-    unsigned long long *out = cand + ((size_t)m * P + p) * k;
-    for (int i = threadIdx.x; i < k; i += blockDim.x)
-        out[i] = sk[i];
+    int oa = 0, ob = 0; // totals of the warps before this one
+    for (int w = 0; w < warp; ++w) {
+        oa += scratch[w];
+        ob += scratch[kTopkWarps + w];
+    }
+    ea = oa + ia - a;
+    eb = ob + ib - b;
+    __syncthreads(); // scratch reusable
 }
 
-// CTA m: the k largest of the P k candidates of token m (padded to T = 2^j).
+// Keeps the k largest of the n keys of s (index i of s is global index
+// gidx[i], or base + i when gidx is null), in index order: the keys above t
+// and the first `ties` keys equal to t.  Writes 64-bit keys (value key << 48
+// | ~index) to out[0..k).  Each thread scans a contiguous run of s, so the
+// exclusive scans of the per-thread counts give every survivor its position
+// in index order.
+__device__ void compact_topk(const uint32_t *s, int n, int k, uint32_t t, int ties, const uint32_t *gidx,
+                             uint32_t base, unsigned long long *out, int *scratch)
+{
+    const int per = (n + blockDim.x - 1) / blockDim.x;
+    const int i0 = min(n, (int)threadIdx.x * per), i1 = min(n, i0 + per);
+    int above = 0, equal = 0;
+    for (int i = i0; i < i1; ++i) {
+        above += s[i] > t;
+        equal += s[i] == t;
+    }
+    int pa, pe;
+    block_scan2(above, equal, pa, pe, scratch);
+    for (int i = i0; i < i1; ++i) {
+        const uint32_t key = s[i];
+        int pos = -1;
+        if (key > t) {
+            // above-t keys and the kept ties interleave in index order: the
+            // slot counts both kinds before this key
+            pos = pa + min(pe, ties);
+            ++pa;
+        } else if (key == t) {
+            if (pe < ties)
+                pos = pa + pe;
+            ++pe;
+        }
+        if (pos >= 0 && pos < k)
+            out[pos] = ((unsigned long long)key << 48) | (uint32_t)~(gidx ? gidx[i] : base + (uint32_t)i);
+    }
+}
+
+// CTA (p, m): the k largest logits of token m among [p S, p S + S) -> cand.
+__global__ void __launch_bounds__(kTopkThreads) topk_part_kernel(const uint16_t *__restrict__ logits, int N, int k,
+                                                                 unsigned long long *__restrict__ cand)
+{
+    __shared__ uint32_t s_key[kPartSlice];
+    __shared__ uint32_t s_hist[kTopkWarps * 256];
+    __shared__ int s_scan[2 * kTopkWarps];
+    const int p = blockIdx.x, m = blockIdx.y, P = gridDim.x;
+    const int n0 = p * kPartSlice, n = min(kPartSlice, N - n0);
+    const uint16_t *row = logits + (size_t)m * N + n0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+        s_key[i] = order16(row[i]);
+    __syncthreads();
+    unsigned long long *out = cand + ((size_t)m * P + p) * k;
+    const int kk = min(k, n);
+    int ties = 0;
+    const uint32_t t = radix_select16(s_key, n, kk, s_hist, &ties);
+    compact_topk(s_key, n, kk, t, ties, nullptr, (uint32_t)n0, out, s_scan);
+    for (int i = kk + threadIdx.x; i < k; i += blockDim.x)
+        out[i] = 0ull; // a slice shorter than k: padding below every real key
+}
+
+// CTA m: the k largest of the P k candidates of token m, sorted.
 __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(const unsigned long long *__restrict__ cand, int P,
-                                                                  int k, int T, uint16_t *__restrict__ vals,
+                                                                  int k, uint16_t *__restrict__ vals,
                                                                   int32_t *__restrict__ idx)
 {
-    extern __shared__ unsigned long long sk[];
+    extern __shared__ uint32_t sm[];
+    const int C = P * k;
+    uint32_t *s_key = sm, *s_idx = sm + C;                              // [C] each
+    uint32_t *s_hist = s_idx + C;                                       // [kTopkWarps * 256]
+    int *s_scan = reinterpret_cast<int *>(s_hist + kTopkWarps * 256); // [2 * kTopkWarps]
+    __shared__ unsigned long long s_best[kTopkMaxK];
     const int m = blockIdx.x;
-    const unsigned long long *src = cand + (size_t)m * P * k;
-    for (int i = threadIdx.x; i < T; i += blockDim.x)
-        sk[i] = i < P * k ? src[i] : 0ull;
+    const unsigned long long *src = cand + (size_t)m * C;
+    for (int i = threadIdx.x; i < C; i += blockDim.x) {
+        const unsigned long long c = src[i];
+        s_key[i] = (uint32_t)(c >> 48); // padding (0) is below every real key
+        s_idx[i] = ~(uint32_t)c;
+    }
+    for (int i = threadIdx.x; i < kTopkMaxK; i += blockDim.x)
+        s_best[i] = 0ull; // slots past k: below every real key, so the sort below keeps them last
     __syncthreads();
-    bitonic_desc(sk, T);
+    int ties = 0;
+    const uint32_t t = radix_select16(s_key, C, k, s_hist, &ties);
+    compact_topk(s_key, C, k, t, ties, s_idx, 0u, s_best, s_scan);
+    __syncthreads();
+    if (threadIdx.x < 32) { // bitonic sort of the 64 slots, descending, one warp
+        for (int size = 2; size <= kTopkMaxK; size <<= 1)
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                const int i = threadIdx.x; // 32 pairs
+                const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
+                const bool desc = (lo & size) == 0;
+                const unsigned long long a = s_best[lo], b = s_best[hi];
+                if ((a < b) == desc) {
+                    s_best[lo] = b;
+                    s_best[hi] = a;
+                }
+                __syncwarp();
+            }
+    }
+    __syncthreads();
     for (int i = threadIdx.x; i < k; i += blockDim.x) {
-        vals[(size_t)m * k + i] = key_value(sk[i]);
-        idx[(size_t)m * k + i] = key_index(sk[i]);
+        const unsigned long long key = s_best[i];
+        vals[(size_t)m * k + i] = value16((uint32_t)(key >> 48));
+        idx[(size_t)m * k + i] = (int32_t)~(uint32_t)key;
     }
 }
 
-int pow2_at_least(long long v)
-{
-    int p = 1;
-    while (p < v)
-        p <<= 1;
-    return p;
-}
+size_t merge_smem(int P, int k) { return (size_t)2 * P * k * 4 + kTopkWarps * 256 * 4 + 2 * kTopkWarps * 4; }
 
 } // namespace
 
-// Slice S (a power of two, 2048 .. 16384) such that the merge of the
-// ceil(N / S) slices' k candidates fits 16384 keys (128 KB of shared memory).
+// P slices of kPartSlice logits; the merge holds P k candidates in shared
+// memory (at most 200 KB).
 bool topk_plan(int N, int k, int *S, int *P, int *T)
 {
     if (N < 1 || k < 1 || k > kTopkMaxK || k > N)
         return false;
-    for (int s = 2048; s <= 16384; s <<= 1) {
-        const int p = (N + s - 1) / s;
-        const int t = pow2_at_least((long long)p * k);
-        if (t <= 16384) {
-            *S = s;
-            *P = p;
-            *T = t;
-            return true;
-        }
-    }
-    return false;
+    const int p = (N + kPartSlice - 1) / kPartSlice;
+    if (merge_smem(p, k) > 200 * 1024)
+        return false;
+    *S = kPartSlice;
+    *P = p;
+    *T = p * k;
+    return true;
 }
 
 size_t topk_ws_bytes(int M, int N, int k)
@@ -146,15 +267,13 @@ cudaError_t launch_topk(const uint16_t *logits, int M, int N, int k, void *cand_
     int S, P, T;
     if (!topk_plan(N, k, &S, &P, &T))
         return cudaErrorInvalidValue;
-    cudaError_t e = kernel_setup((const void *)topk_part_kernel, (size_t)S * 8, 0, 0, nullptr);
-    if (e != cudaSuccess)
-        return e;
-    e = kernel_setup((const void *)topk_merge_kernel, (size_t)T * 8, 0, 0, nullptr);
+    const size_t msm = merge_smem(P, k);
+    cudaError_t e = kernel_setup((const void *)topk_merge_kernel, msm, 0, 0, nullptr);
     if (e != cudaSuccess)
         return e;
     unsigned long long *cand = static_cast<unsigned long long *>(cand_ws);
-    topk_part_kernel<<<dim3(P, M), kTopkThreads, (size_t)S * 8, st>>>(logits, N, S, k, cand);
-    topk_merge_kernel<<<M, kTopkThreads, (size_t)T * 8, st>>>(cand, P, k, T, vals, idx);
+    topk_part_kernel<<<dim3(P, M), kTopkThreads, 0, st>>>(logits, N, k, cand);
+    topk_merge_kernel<<<M, kTopkThreads, msm, st>>>(cand, P, k, vals, idx);
     return cudaGetLastError();
 }
 

@@ -62,7 +62,7 @@ struct GemmW4Params {
     const uint16_t *scales;
     const uint8_t *zeros;
     uint16_t *y;
-    float *part;   // [CTAs][2 slots][128 rows][NT]
+    float *part;   // [CTAs][2 slots][NT tokens][128 rows]
     uint32_t *cnt; // [panels][8] tickets
 };
 
@@ -114,53 +114,67 @@ constexpr size_t gemm_w4_smem_bytes()
 {
     using C = W4Cfg<NT>;
     return 1024 + (size_t)C::kXS * C::kXB + (size_t)C::kSS * 256 + (size_t)C::kDW * C::kDepth * C::kSlot +
-           (size_t)(2 * C::kXS + 2 * C::kSS + 2 * C::kAS + 2 * C::kACC) * 8 + 16;
+           (size_t)(2 * C::kXS + 2 * C::kSS + 2 * C::kAS + 2 * C::kACC) * 8 + 16 +
+           (size_t)2 * (kSkMaxCtas + 1) * sizeof(int);
 }
+
+// The stream-K cuts of the grid, computed once per CTA (one 64-bit division
+// per thread) so that the flushes and fix-ups look them up instead of
+// dividing: start[c] is the first unit of CTA c, first[c] its first panel.
+struct SkTable {
+    const int *start, *first;
+    // CTA whose range holds unit u: the largest c with start[c] <= u (ranges
+    // may be empty; the largest such c has start[c + 1] > u)
+    __device__ __forceinline__ int owner(int u, int G) const
+    {
+        int lo = 0, hi = G - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (start[mid] <= u)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        return lo;
+    }
+};
 
 // The last contributor to a split panel: sums the fp32 partials of CTAs
 // cf .. cl for its row r and tokens t0 .. t0 + CW - 1 in CTA order and
-// writes y.  The partials of up to five contributors are loaded together
-// (one round trip to L2 per 16 columns, not one per contributor: this runs
-// at the very end of the call, on the critical path).  Called after the
-// retire loop, whose register totals are dead by then.
+// writes y.  The partials are token-major, so every load is one coalesced
+// 128-byte row segment per warp; CG contributors x 16 tokens are in flight
+// together (this runs at the very end of the call, on its critical path).
+// Called after the retire loop, whose register totals are dead by then.
 template <int NT, int CW>
-__device__ __forceinline__ void w4_fixup(const GemmW4Params &p, long long U, int G, int pnl, int cf, int cl, int r,
-                                      int t0)
+__device__ __forceinline__ void w4_fixup(const GemmW4Params &p, const SkTable &sk, int pnl, int cf, int cl, int r,
+                                         int t0)
 {
-    const int KB = p.KB;
     const int nrow = pnl * kPanelRows + r;
-    // contributors whose partials are in flight together (a panel usually has <= 5; fewer at NT = 128,
-    // where the retire warps already hold 64 totals and more would spill)
-    constexpr int CG = (NT == 128 || W4Cfg<NT>::kWarps == 20) ? 2 : 5;
+    constexpr int CG = 4;
     for (int j0 = 0; j0 < CW; j0 += 16) {
         float acc[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             acc[j] = 0.f;
         for (int c0 = cf; c0 <= cl; c0 += CG) {
-            float4 v[CG][4];
+            float v[CG][16];
 #pragma unroll
             for (int u = 0; u < CG; ++u) {
                 const int cc = c0 + u;
                 if (cc <= cl) {
-                    const int sl = (pnl == sk_start(U, G, cc) / KB) ? 0 : 1;
-                    const float4 *src =
-                        reinterpret_cast<const float4 *>(p.part + ((size_t)(cc * 2 + sl) * kPanelRows + r) * NT + t0 + j0);
+                    const int sl = pnl == sk.first[cc] ? 0 : 1;
+                    const float *src = p.part + ((size_t)(cc * 2 + sl) * NT + t0 + j0) * kPanelRows + r;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        v[u][j] = __ldcg(src + j);
+                    for (int j = 0; j < 16; ++j)
+                        v[u][j] = __ldcg(src + j * kPanelRows);
                 }
             }
 #pragma unroll
             for (int u = 0; u < CG; ++u) // in CTA order
                 if (c0 + u <= cl)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        acc[4 * j] += v[u][j].x;
-                        acc[4 * j + 1] += v[u][j].y;
-                        acc[4 * j + 2] += v[u][j].z;
-                        acc[4 * j + 3] += v[u][j].w;
-                    }
+                    for (int j = 0; j < 16; ++j)
+                        acc[j] += v[u][j];
         }
         if (nrow < p.N) {
             const int jn = min(16, p.M - t0 - j0);
@@ -195,11 +209,19 @@ __global__ void __launch_bounds__(W4Cfg<NT>::kThreads, 1) gemm_w4_kernel(const _
     uint64_t *afull = sempty + SS, *aempty = afull + AS;
     uint64_t *accfull = aempty + AS, *accempty = accfull + ACC;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(accempty + ACC);
+    int *s_start = reinterpret_cast<int *>(s_tmem + 4); // [kSkMaxCtas + 1]
+    int *s_first = s_start + kSkMaxCtas + 1;            // [kSkMaxCtas + 1]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, cta = blockIdx.x;
     const long long U = p.U;
     const int KB = p.KB;
+    for (int c = threadIdx.x; c <= G; c += blockDim.x) {
+        const int st = sk_start(U, G, c);
+        s_start[c] = st;
+        s_first[c] = st / KB;
+    }
+    const SkTable sk{s_start, s_first};
     const int u0 = sk_start(U, G, cta), u1 = sk_start(U, G, cta + 1);
     const int n = u1 - u0;
 
@@ -334,17 +356,17 @@ __global__ void __launch_bounds__(W4Cfg<NT>::kThreads, 1) gemm_w4_kernel(const _
                 return;
             }
             const int slot = (pnl == u0 / KB) ? 0 : 1;
-            float *mine = p.part + ((size_t)(cta * 2 + slot) * kPanelRows + r) * NT + t0;
+            float *mine = p.part + ((size_t)(cta * 2 + slot) * NT + t0) * kPanelRows + r;
 #pragma unroll
-            for (int j = 0; j < CW; j += 4)
-                *reinterpret_cast<float4 *>(mine + j) = make_float4(tot[j], tot[j + 1], tot[j + 2], tot[j + 3]);
+            for (int j = 0; j < CW; ++j)
+                mine[j * kPanelRows] = tot[j]; // token-major: the warp writes 128 contiguous bytes
             __threadfence(); // every lane's partial is visible before lane 0's ticket
             __syncwarp();
             uint32_t ticket = 0;
             if (lane == 0)
                 ticket = ticket_take_acq_rel(&p.cnt[pnl * 8 + dw]);
             ticket = __shfl_sync(0xffffffffu, ticket, 0);
-            const int cf = sk_owner(U, G, pnl * KB), cl = sk_owner(U, G, (pnl + 1) * KB - 1);
+            const int cf = sk.owner(pnl * KB, G), cl = sk.owner((pnl + 1) * KB - 1, G);
             if (ticket != (uint32_t)(cl - cf))
                 return;
             // the last contributor: sum the partials once the loop is done
@@ -394,7 +416,7 @@ __global__ void __launch_bounds__(W4Cfg<NT>::kThreads, 1) gemm_w4_kernel(const _
         }
         __syncwarp(); // lane 0's acquire (the tickets) orders every lane's reads below
         for (int f = 0; f < nfix && ok; ++f) {
-            w4_fixup<NT, CW>(p, U, G, fix_pnl[f], fix_cf[f], fix_cl[f], r, c * CW);
+            w4_fixup<NT, CW>(p, sk, fix_pnl[f], fix_cf[f], fix_cl[f], r, c * CW);
             if (lane == 0)
                 atomicExch(&p.cnt[fix_pnl[f] * 8 + dw], 0u); // ready for the next call
         }

@@ -52,6 +52,7 @@ __device__ uint32_t radix_select16(const uint32_t *s, int n, int k, uint32_t *hi
 {
     __shared__ uint32_t s_prefix;
     __shared__ int s_rank;
+    __shared__ int s_wsum[8], c_bin[256], c_inc[256];
     uint32_t *wh = hist + (threadIdx.x >> 5) * 256; // one 256-bin histogram per warp
     if (threadIdx.x == 0) {
         s_prefix = 0;
@@ -75,22 +76,39 @@ __device__ uint32_t radix_select16(const uint32_t *s, int n, int k, uint32_t *hi
                 atomicAdd(&wh[bin], (uint32_t)__popc(same));
         }
         __syncthreads();
-        if (threadIdx.x < 256) { // fold the warp histograms
-            uint32_t c = 0;
+        // fold the warp histograms and find the digit holding the rank-th
+        // largest key: thread j takes bin 255 - j, so an inclusive scan over
+        // the threads counts the keys at or above each bin, and exactly one
+        // bin has the rank-th largest between its exclusive and inclusive
+        // counts (the selected keys number at least the rank)
+        const int rank = s_rank;
+        if (threadIdx.x < 256) {
+            const int d = 255 - (int)threadIdx.x, lane = threadIdx.x & 31;
+            int c = 0;
             for (int w = 0; w < kTopkWarps; ++w)
-                c += hist[w * 256 + threadIdx.x];
-            hist[threadIdx.x] = c;
+                c += (int)hist[w * 256 + d];
+            int inc = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o)
+                    inc += u;
+            }
+            if (lane == 31)
+                s_wsum[threadIdx.x >> 5] = inc;
+            c_bin[threadIdx.x] = c;
+            c_inc[threadIdx.x] = inc;
         }
         __syncthreads();
-        if (threadIdx.x == 0) { // the digit holding the rank-th largest, from the top
-            int rank = s_rank, d = 255;
-            for (; d > 0; --d) {
-                if ((int)hist[d] >= rank)
-                    break;
-                rank -= (int)hist[d];
+        if (threadIdx.x < 256) {
+            int inc = c_inc[threadIdx.x];
+            for (int w = 0; w < (int)(threadIdx.x >> 5); ++w)
+                inc += s_wsum[w];
+            const int exc = inc - c_bin[threadIdx.x];
+            if (exc < rank && inc >= rank) {
+                s_rank = rank - exc;
+                s_prefix = prefix | ((uint32_t)(255 - threadIdx.x) << shift);
             }
-            s_rank = rank;
-            s_prefix = prefix | ((uint32_t)d << shift);
         }
         __syncthreads();
     }

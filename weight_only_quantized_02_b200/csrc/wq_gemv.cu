@@ -356,6 +356,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvParams 
     const int nrb = p.N >> 4;
     const int units = (nrb + rbs_per_cta - 1) / rbs_per_cta;
     const int ks_i = warp % ks;
+    // The next kernel on the stream may launch now (this grid is one wave,
+    // every CTA resident); x and y wait for the preceding kernel.
+    pdl_launch_dependents();
+    pdl_wait();
 
     for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
         const int rb = unit * rbs_per_cta + warp / ks;
@@ -428,8 +432,16 @@ static cudaError_t launch_gemv_t(const GemvParams &p, int sm_count, cudaStream_t
     int grid = occ * sm_count;
     if (grid > units)
         grid = units;
-    gemv_kernel<BITS, MT, LG, F16><<<grid, kGemvWarps * 32, 0, st>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kGemvWarps * 32);
+    cfg.stream = st;
+    return cudaLaunchKernelEx(&cfg, gemv_kernel<BITS, MT, LG, F16>, p);
 }
 
 template <bool F16>

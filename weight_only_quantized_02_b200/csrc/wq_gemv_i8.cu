@@ -614,6 +614,11 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
         s_res[threadIdx.x] = 0ull;
     }
     __syncthreads();
+    // The next kernel on the stream may launch now: its CTAs take the SMs
+    // this grid leaves and prefetch their weights while its last CTAs
+    // finish; whatever it shares with this grid waits behind its own launch
+    // wait.  (Every CTA of this grid is resident by then: one wave.)
+    pdl_launch_dependents();
     pdl_wait(); // x, y and the workspace may come from / be in use by the preceding kernel
     gi_digits<BITS, NR, WARPS * 32>(p, sd, s_dsum, s_amax, s_e, s_res);
 
@@ -772,7 +777,6 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
         gi_shared_fixup<BITS, NT, WARPS>(p, pend_rb1, pend_t1, G, s_e, s_res, st0, lane);
     __syncthreads(); // every warp's stash is complete
     gi_local_out<BITS, NT, WARPS>(p, ct, c, stash, s_e, s_res, warp, lane);
-    pdl_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------

@@ -22,6 +22,7 @@
 #include <cuda_bf16.h>
 
 #include "wq.h"
+#include "wq_device.cuh"
 #include "wq_internal.h"
 
 namespace wq {
@@ -192,6 +193,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_part_kernel(const uint16_t 
     const int p = blockIdx.x, m = blockIdx.y, P = gridDim.x;
     const int n0 = p * kPartSlice, n = min(kPartSlice, N - n0);
     const uint16_t *row = logits + (size_t)m * N + n0;
+    pdl_launch_dependents(); // the merge may launch; it waits for this grid before reading
+    pdl_wait();              // the logits come from the preceding kernel
     for (int i = threadIdx.x; i < n; i += blockDim.x)
         s_key[i] = order16(row[i]);
     __syncthreads();
@@ -217,6 +220,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(const unsigned
     __shared__ unsigned long long s_best[kTopkMaxK];
     const int m = blockIdx.x;
     const unsigned long long *src = cand + (size_t)m * C;
+    pdl_launch_dependents();
+    pdl_wait(); // the candidates come from the part kernel
     for (int i = threadIdx.x; i < C; i += blockDim.x) {
         const unsigned long long c = src[i];
         s_key[i] = (uint32_t)(c >> 48); // padding (0) is below every real key
@@ -290,9 +295,21 @@ cudaError_t launch_topk(const uint16_t *logits, int M, int N, int k, void *cand_
     if (e != cudaSuccess)
         return e;
     unsigned long long *cand = static_cast<unsigned long long *>(cand_ws);
-    topk_part_kernel<<<dim3(P, M), kTopkThreads, 0, st>>>(logits, N, k, cand);
-    topk_merge_kernel<<<M, kTopkThreads, msm, st>>>(cand, P, k, vals, idx);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.stream = st;
+    cfg.gridDim = dim3(P, M);
+    cfg.blockDim = dim3(kTopkThreads);
+    e = cudaLaunchKernelEx(&cfg, topk_part_kernel, logits, N, k, cand);
+    if (e != cudaSuccess)
+        return e;
+    cfg.gridDim = dim3(M);
+    cfg.dynamicSmemBytes = msm;
+    return cudaLaunchKernelEx(&cfg, topk_merge_kernel, (const unsigned long long *)cand, P, k, vals, idx);
 }
 
 } // namespace wq

@@ -128,7 +128,7 @@ cudaError_t launch_gemv_i8(const LinearArgs &a, int split, void *ws, int sm_coun
 // scratch of wq_linear_topk (bf16 logits M x N, then M x P x k candidates);
 // launch_topk selects from logits already in that scratch.
 constexpr int kTopkMaxK = 64;
-bool topk_plan(int N, int k, int *S, int *P, int *T);
+bool topk_plan(int M, int N, int k, int *S, int *P, int *T);
 size_t topk_ws_bytes(int M, int N, int k);
 cudaError_t launch_topk(const uint16_t *logits, int M, int N, int k, void *cand_ws, uint16_t *vals, int32_t *idx,
                         cudaStream_t st);

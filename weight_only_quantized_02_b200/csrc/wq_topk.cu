@@ -31,7 +31,10 @@ namespace {
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kPartSlice = 4096; // logits per part CTA
+// Logits per part CTA: 4096, or 8192 where the grid of 4096-logit slices
+// would not fit the GPU at once (four CTAs per SM).
+constexpr int kPartSlice = 4096, kPartSliceWide = 8192;
+constexpr long long kTopkWaveCtas = 4 * 148; // four 512-thread CTAs on each of a B200's 148 SMs
 
 // bf16 bits -> a 16-bit key that orders like the value (-0 and +0 equal).
 __device__ __forceinline__ uint32_t order16(uint16_t b)
@@ -46,10 +49,11 @@ __device__ __forceinline__ uint16_t value16(uint32_t key16)
     return (uint16_t)((key16 & 0x8000u) ? (key16 & 0x7FFFu) : (~key16 & 0xFFFFu));
 }
 
-// Exact k-th largest of the n keys in s (16-bit keys in uint32), by two
-// 8-bit passes; every thread of the CTA calls it.  Returns t and, in *ties,
-// how many keys equal to t belong to the k largest.
-__device__ uint32_t radix_select16(const uint32_t *s, int n, int k, uint32_t *hist, int *ties)
+// Exact k-th largest of the n keys in s (16-bit keys), by two 8-bit passes;
+// every thread of the CTA calls it.  Returns t and, in *ties, how many keys
+// equal to t belong to the k largest.
+template <typename Key>
+__device__ uint32_t radix_select16(const Key *s, int n, int k, uint32_t *hist, int *ties)
 {
     __shared__ uint32_t s_prefix;
     __shared__ int s_rank;
@@ -65,16 +69,12 @@ __device__ uint32_t radix_select16(const uint32_t *s, int n, int k, uint32_t *hi
         __syncthreads();
         const uint32_t prefix = s_prefix, shift = 8 * pass;
         const uint32_t hi_mask = pass == 1 ? 0u : 0xFF00u;
-        // logits crowd into a few bins: lanes with the same bin add once
-        // (their count) instead of contending for the same word
-        for (int i0 = 0; i0 < n; i0 += blockDim.x) {
-            const int i = i0 + threadIdx.x;
-            const uint32_t key = i < n ? s[i] : 0u;
-            const bool in = i < n && (key & hi_mask) == prefix;
-            const uint32_t bin = in ? (key >> shift) & 0xFFu : 256u;
-            const uint32_t same = __match_any_sync(0xffffffffu, bin);
-            if (in && (threadIdx.x & 31) == (uint32_t)(__ffs(same) - 1))
-                atomicAdd(&wh[bin], (uint32_t)__popc(same));
+        // one histogram per warp spreads the contention of the few bins
+        // that logits crowd into
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            const uint32_t key = s[i];
+            if ((key & hi_mask) == prefix)
+                atomicAdd(&wh[(key >> shift) & 0xFFu], 1u);
         }
         __syncthreads();
         // fold the warp histograms and find the digit holding the rank-th
@@ -117,86 +117,86 @@ __device__ uint32_t radix_select16(const uint32_t *s, int n, int k, uint32_t *hi
     return s_prefix;
 }
 
-// Exclusive prefix sums over the CTA's threads, in thread order, of two
-// per-thread counts (warp shuffles, then the warp totals); every thread
-// calls it.  scratch: 2 * kTopkWarps ints.
-__device__ __forceinline__ void block_scan2(int a, int b, int &ea, int &eb, int *scratch)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int ia = a, ib = b; // inclusive within the warp
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int ua = __shfl_up_sync(0xffffffffu, ia, o), ub = __shfl_up_sync(0xffffffffu, ib, o);
-        if (lane >= o) {
-            ia += ua;
-            ib += ub;
-        }
-    }
-    if (lane == 31) {
-        scratch[warp] = ia;
-        scratch[kTopkWarps + warp] = ib;
-    }
-    __syncthreads();
-    int oa = 0, ob = 0; // totals of the warps before this one
-    for (int w = 0; w < warp; ++w) {
-        oa += scratch[w];
-        ob += scratch[kTopkWarps + w];
-    }
-    ea = oa + ia - a;
-    eb = ob + ib - b;
-    __syncthreads(); // scratch reusable
-}
-
 // Keeps the k largest of the n keys of s (index i of s is global index
 // gidx[i], or base + i when gidx is null), in index order: the keys above t
 // and the first `ties` keys equal to t.  Writes 64-bit keys (value key << 48
-// | ~index) to out[0..k).  Each thread scans a contiguous run of s, so the
-// exclusive scans of the per-thread counts give every survivor its position
-// in index order.
-__device__ void compact_topk(const uint32_t *s, int n, int k, uint32_t t, int ties, const uint32_t *gidx,
+// | ~index) to out[0..k).  Warp w takes the keys [w span, (w + 1) span), 32
+// consecutive keys at a time, so the ballots of the lanes, the chunks in
+// turn and the warp totals scanned in warp order give every survivor its
+// position in index order; lanes read consecutive keys (no bank conflicts).
+// scratch: 2 * kTopkWarps ints.
+template <typename Key>
+__device__ void compact_topk(const Key *s, int n, int k, uint32_t t, int ties, const uint32_t *gidx,
                              uint32_t base, unsigned long long *out, int *scratch)
 {
-    const int per = (n + blockDim.x - 1) / blockDim.x;
-    const int i0 = min(n, (int)threadIdx.x * per), i1 = min(n, i0 + per);
-    int above = 0, equal = 0;
-    for (int i = i0; i < i1; ++i) {
-        above += s[i] > t;
-        equal += s[i] == t;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int span = (n + kTopkWarps - 1) / kTopkWarps;
+    const int w0 = min(n, warp * span), w1 = min(n, w0 + span);
+    int ca = 0, ce = 0;
+    for (int i0 = w0; i0 < w1; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t key = i < w1 ? (uint32_t)s[i] : 0u;
+        ca += __popc(__ballot_sync(0xffffffffu, i < w1 && key > t));
+        ce += __popc(__ballot_sync(0xffffffffu, i < w1 && key == t));
     }
-    int pa, pe;
-    block_scan2(above, equal, pa, pe, scratch);
-    for (int i = i0; i < i1; ++i) {
-        const uint32_t key = s[i];
+    if (lane == 0) {
+        scratch[warp] = ca;
+        scratch[kTopkWarps + warp] = ce;
+    }
+    __syncthreads();
+    int pa = 0, pe = 0; // keys above t / equal to t before this warp's range
+    for (int w = 0; w < warp; ++w) {
+        pa += scratch[w];
+        pe += scratch[kTopkWarps + w];
+    }
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int i0 = w0; i0 < w1; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t key = i < w1 ? (uint32_t)s[i] : 0u;
+        const bool above = i < w1 && key > t, equal = i < w1 && key == t;
+        const uint32_t ma = __ballot_sync(0xffffffffu, above), me = __ballot_sync(0xffffffffu, equal);
+        const int ra = pa + __popc(ma & lt), re = pe + __popc(me & lt);
         int pos = -1;
-        if (key > t) {
-            // above-t keys and the kept ties interleave in index order: the
-            // slot counts both kinds before this key
-            pos = pa + min(pe, ties);
-            ++pa;
-        } else if (key == t) {
-            if (pe < ties)
-                pos = pa + pe;
-            ++pe;
-        }
+        if (above) // above-t keys and the kept ties interleave in index order
+            pos = ra + min(re, ties);
+        else if (equal && re < ties)
+            pos = ra + re;
         if (pos >= 0 && pos < k)
             out[pos] = ((unsigned long long)key << 48) | (uint32_t)~(gidx ? gidx[i] : base + (uint32_t)i);
+        pa += __popc(ma);
+        pe += __popc(me);
     }
+    __syncthreads(); // scratch reusable
 }
 
 // CTA (p, m): the k largest logits of token m among [p S, p S + S) -> cand.
+template <int S>
 __global__ void __launch_bounds__(kTopkThreads) topk_part_kernel(const uint16_t *__restrict__ logits, int N, int k,
                                                                  unsigned long long *__restrict__ cand)
 {
-    __shared__ uint32_t s_key[kPartSlice];
+    __shared__ uint16_t s_key[S];
     __shared__ uint32_t s_hist[kTopkWarps * 256];
     __shared__ int s_scan[2 * kTopkWarps];
     const int p = blockIdx.x, m = blockIdx.y, P = gridDim.x;
-    const int n0 = p * kPartSlice, n = min(kPartSlice, N - n0);
+    const int n0 = p * S, n = min(S, N - n0);
     const uint16_t *row = logits + (size_t)m * N + n0;
     pdl_launch_dependents(); // the merge may launch; it waits for this grid before reading
     pdl_wait();              // the logits come from the preceding kernel
-    for (int i = threadIdx.x; i < n; i += blockDim.x)
-        s_key[i] = order16(row[i]);
+    { // every thread's logits in flight together, then their keys
+        constexpr int J = S / kTopkThreads;
+        uint16_t v[J];
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int i = threadIdx.x + j * kTopkThreads;
+            v[j] = i < n ? row[i] : (uint16_t)0;
+        }
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int i = threadIdx.x + j * kTopkThreads;
+            if (i < n)
+                s_key[i] = (uint16_t)order16(v[j]);
+        }
+    }
     __syncthreads();
     unsigned long long *out = cand + ((size_t)m * P + p) * k;
     const int kk = min(k, n);
@@ -222,8 +222,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(const unsigned
     const unsigned long long *src = cand + (size_t)m * C;
     pdl_launch_dependents();
     pdl_wait(); // the candidates come from the part kernel
+#pragma unroll 4
     for (int i = threadIdx.x; i < C; i += blockDim.x) {
-        const unsigned long long c = src[i];
+        const unsigned long long c = __ldcg(src + i);
         s_key[i] = (uint32_t)(c >> 48); // padding (0) is below every real key
         s_idx[i] = ~(uint32_t)c;
     }
@@ -260,16 +261,18 @@ size_t merge_smem(int P, int k) { return (size_t)2 * P * k * 4 + kTopkWarps * 25
 
 } // namespace
 
-// P slices of kPartSlice logits; the merge holds P k candidates in shared
-// memory (at most 200 KB).
-bool topk_plan(int N, int k, int *S, int *P, int *T)
+// P slices of S logits; the merge holds P k candidates in shared memory (at
+// most 200 KB).
+bool topk_plan(int M, int N, int k, int *S, int *P, int *T)
 {
-    if (N < 1 || k < 1 || k > kTopkMaxK || k > N)
+    if (M < 1 || N < 1 || k < 1 || k > kTopkMaxK || k > N)
         return false;
-    const int p = (N + kPartSlice - 1) / kPartSlice;
+    const int narrow = (N + kPartSlice - 1) / kPartSlice;
+    const int sl = (long long)narrow * M <= kTopkWaveCtas ? kPartSlice : kPartSliceWide;
+    const int p = (N + sl - 1) / sl;
     if (merge_smem(p, k) > 200 * 1024)
         return false;
-    *S = kPartSlice;
+    *S = sl;
     *P = p;
     *T = p * k;
     return true;
@@ -278,7 +281,7 @@ bool topk_plan(int N, int k, int *S, int *P, int *T)
 size_t topk_ws_bytes(int M, int N, int k)
 {
     int S, P, T;
-    if (M < 1 || !topk_plan(N, k, &S, &P, &T))
+    if (!topk_plan(M, N, k, &S, &P, &T))
         return 0;
     const size_t logits = ((size_t)M * N * 2 + 255) / 256 * 256;
     return logits + (size_t)M * P * k * sizeof(unsigned long long);
@@ -288,7 +291,7 @@ cudaError_t launch_topk(const uint16_t *logits, int M, int N, int k, void *cand_
                         cudaStream_t st)
 {
     int S, P, T;
-    if (!topk_plan(N, k, &S, &P, &T))
+    if (!topk_plan(M, N, k, &S, &P, &T))
         return cudaErrorInvalidValue;
     const size_t msm = merge_smem(P, k);
     cudaError_t e = kernel_setup((const void *)topk_merge_kernel, msm, 0, 0, nullptr);
@@ -304,7 +307,8 @@ cudaError_t launch_topk(const uint16_t *logits, int M, int N, int k, void *cand_
     cfg.stream = st;
     cfg.gridDim = dim3(P, M);
     cfg.blockDim = dim3(kTopkThreads);
-    e = cudaLaunchKernelEx(&cfg, topk_part_kernel, logits, N, k, cand);
+    e = S == kPartSlice ? cudaLaunchKernelEx(&cfg, topk_part_kernel<kPartSlice>, logits, N, k, cand)
+                        : cudaLaunchKernelEx(&cfg, topk_part_kernel<kPartSliceWide>, logits, N, k, cand);
     if (e != cudaSuccess)
         return e;
     cfg.gridDim = dim3(M);

@@ -56,7 +56,8 @@
  *     after the enqueue, with no implicit synchronization, unless the entry
  *     says "synchronizes".
  *   - bf16 values are passed as their uint16_t bit patterns.
- *   - Shape rules: 1 <= N, N % 16 == 0. W8A16: group == 0, K % 32 == 0.
+ *   - Shape rules: 1 <= N <= 1048576, N % 16 == 0. W8A16: group == 0,
+ *     K % 32 == 0.
  *     W4A16: K % 128 == 0 and group 32, 64, 128 or K (per channel: one
  *     scale and zero point per output row). 1 <= M <= 65536; a kernel takes
  *     at most 128 tokens (32 for groups of 32 and 64 k, which run on the
@@ -275,12 +276,15 @@ size_t wq_topk_workspace_bytes(int M, int N, int k);
 
 /* Bytes of workspace for M tokens, a K x N weight and GEMM splits up to
  * max_split: enough for every variant of that shape (M > 128: of its
- * 128-token chunks, which share the workspace one after another). It holds eight ticket
- * counters per 128-channel panel and the largest of the GEMM's fp32
- * partials [split][M][N], the stream-K kernels' per-CTA panel partials,
- * the integer path's int32 per-CTA partials, and the integer GEMV's
- * per-warp partials. Returns 0 for M, K, N or
- * max_split < 1. Host. */
+ * 128-token chunks, which share the workspace one after another). It holds
+ * a counter region of the same size for every shape (257 KiB: eight ticket
+ * counters per 128-channel panel of the largest N, then the integer path's
+ * grid counters and residual sums), so one workspace sized for the largest
+ * of several layers serves them all in turn, and after it the largest of
+ * the GEMM's fp32 partials [split][M][N], the stream-K kernels' per-CTA
+ * panel partials, the integer path's int32 per-CTA partials, and the
+ * integer GEMV's per-warp partials. Returns 0 for M, K, N or max_split < 1.
+ * Host. */
 size_t wq_workspace_bytes(int M, int K, int N, int max_split);
 
 /* Registers a caller-owned device workspace for the current device, used by

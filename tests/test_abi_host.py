@@ -65,6 +65,7 @@ def test_packed_bytes():
     (8, 1000, 1024, 0, -2),     # K not a multiple of 32
     (8, 1040, 1024, 0, -2),     # INT8: K % 32 (a multiple of 16 is not enough: 32-k integer MMA steps)
     (8, 1024, 1000, 0, -2),     # N not a multiple of 16 (a multiple of 8 is not enough: 16-row blocks)
+    (8, 32, (1 << 20) + 16, 0, -2),  # N beyond the workspace's fixed counter region (2^20 channels)
     (8, 0, 1024, 0, -2),
     (3, 1024, 1024, 0, -4),
 ])
@@ -74,18 +75,20 @@ def test_packed_bytes_rejects(bits, K, N, group, status):
 
 
 def test_workspace_bytes():
-    # counters: 8 tickets per 128-row panel + 2 grid counters + 64 two-word
-    # residual sums of the integer path's exactness guard, padded to 256 bytes
-    # (N = 5120: 40 panels -> 450 words -> 2048 bytes); then the largest of
-    # the split-K GEMM's fp32 partials [S][M][N], the stream-K kernels' per-CTA
+    # counters: a region of one size for every shape -- 8 tickets per
+    # 128-row panel of the largest N (2^20: 8192 panels) + 2 grid counters +
+    # 64 two-word residual sums of the integer path's exactness guard, padded
+    # to 256 bytes (65666 words -> 262912 bytes); then the largest of the
+    # split-K GEMM's fp32 partials [S][M][N], the stream-K kernels' per-CTA
     # panel partials [512 CTAs][2][128 rows][token tile] and the integer
     # path's digits + int32 partials (smaller than the stream-K GEMM's here)
-    assert wq.wq_workspace_bytes(128, 5120, 5120, 32) == 2048 + 32 * 128 * 5120 * 4
-    assert wq.wq_workspace_bytes(64, 5120, 5120, 1) == 2048 + 512 * 2 * 128 * 64 * 4
-    assert wq.wq_workspace_bytes(16, 5120, 5120, 1) == 2048 + 512 * 2 * 128 * 16 * 4
+    C = 262912
+    assert wq.wq_workspace_bytes(128, 5120, 5120, 32) == C + 32 * 128 * 5120 * 4
+    assert wq.wq_workspace_bytes(64, 5120, 5120, 1) == C + 512 * 2 * 128 * 64 * 4
+    assert wq.wq_workspace_bytes(16, 5120, 5120, 1) == C + 512 * 2 * 128 * 16 * 4
     # M = 8: the integer GEMV's per-warp partials 448 CTAs x 8 warps x 2 x 16 rows x 24 x 4 bytes
-    assert wq.wq_workspace_bytes(8, 5120, 5120, 1) == 2048 + 448 * 8 * 2 * 16 * 24 * 4
-    assert wq.wq_workspace_bytes(1, 5120, 17408, 1) == 5120 + 512 * 2 * 128 * 16 * 4  # 136 panels -> 1218 words
+    assert wq.wq_workspace_bytes(8, 5120, 5120, 1) == C + 448 * 8 * 2 * 16 * 24 * 4
+    assert wq.wq_workspace_bytes(1, 5120, 17408, 1) == C + 512 * 2 * 128 * 16 * 4
     # integer path, M = 1 (16 digit rows): int32 partials 160 CTAs x 2 x 16 x 128
     assert 160 * 2 * 16 * 128 * 4 < 512 * 2 * 128 * 16 * 4
     assert wq.wq_workspace_bytes(0, 5120, 5120, 4) == 0

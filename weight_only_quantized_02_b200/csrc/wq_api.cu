@@ -96,7 +96,7 @@ int check_weight_shape(int bits, int K, int N, int group)
         return WQ_ERR_GROUP;
     if (bits != 4 && bits != 8)
         return WQ_ERR_GROUP;
-    if (K <= 0 || N <= 0 || N % 16 != 0)
+    if (K <= 0 || N <= 0 || N % 16 != 0 || N > kMaxN)
         return WQ_ERR_SHAPE;
     if (bits == 8 && K % 32 != 0)
         return WQ_ERR_SHAPE;

@@ -417,7 +417,7 @@ static cudaError_t launch_gemm_t(const LinearArgs &a, int S, void *ws, cudaStrea
     p.zeros = (const uint8_t *)a.zeros;
     p.y = a.y;
     p.cnt = (uint32_t *)ws;
-    p.part = ws ? (float *)((uint8_t *)ws + ws_counter_bytes(a.N)) : nullptr;
+    p.part = ws ? (float *)((uint8_t *)ws + ws_counter_bytes()) : nullptr;
     dim3 grid(sh.panels(), S);
     gemm_kernel<BITS, NT><<<grid, 192, smem, st>>>(map, p);
     return cudaGetLastError();

@@ -469,7 +469,7 @@ size_t ws_bytes_gemm_i4(int M, int K, int N)
         return 0;
     const int NR = i8_digit_rows(M);
     const size_t KB = (size_t)(K + kBlockK - 1) / kBlockK;
-    return ws_counter_bytes(N) + KB * NR * 128 + (size_t)kI8MaxCtas * 2 * (NR / 3) * 128 * sizeof(float);
+    return ws_counter_bytes() + KB * NR * 128 + (size_t)kI8MaxCtas * 2 * (NR / 3) * 128 * sizeof(float);
 }
 
 template <int NR>
@@ -495,10 +495,10 @@ static cudaError_t launch_i4_t(const LinearArgs &a, void *ws, int sm_count, cuda
     p.zeros = (const uint8_t *)a.zeros;
     p.y = a.y;
     p.cnt = (uint32_t *)ws;
-    p.grid = p.cnt + ws_grid_counter(a.N);
-    p.res = reinterpret_cast<unsigned long long *>(p.cnt + ws_res_counter(a.N));
+    p.grid = p.cnt + ws_grid_counter();
+    p.res = reinterpret_cast<unsigned long long *>(p.cnt + ws_res_counter());
     p.wmax = trailer_wmax(a.wq, sh);
-    p.xd = (uint8_t *)ws + ws_counter_bytes(a.N);
+    p.xd = (uint8_t *)ws + ws_counter_bytes();
     p.part = (float *)(p.xd + (size_t)p.KB * NR * 128);
     int G = sm_count < kI8MaxCtas ? sm_count : kI8MaxCtas;
     if (G > p.U)

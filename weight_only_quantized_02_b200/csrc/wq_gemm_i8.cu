@@ -402,7 +402,7 @@ size_t ws_bytes_gemm_i8(int M, int K, int N)
         return 0;
     const int NR = i8_digit_rows(M);
     const size_t KB = (size_t)(K + kBlockK - 1) / kBlockK;
-    return ws_counter_bytes(N) + KB * NR * 128 + (size_t)kI8MaxCtas * 2 * NR * 128 * sizeof(int32_t);
+    return ws_counter_bytes() + KB * NR * 128 + (size_t)kI8MaxCtas * 2 * NR * 128 * sizeof(int32_t);
 }
 
 template <int NR>
@@ -428,9 +428,9 @@ static cudaError_t launch_i8_t(const LinearArgs &a, void *ws, int sm_count, cuda
     p.scales = (const uint16_t *)a.scales;
     p.y = a.y;
     p.cnt = (uint32_t *)ws;
-    p.grid = p.cnt + ws_grid_counter(a.N);
-    p.res = reinterpret_cast<unsigned long long *>(p.cnt + ws_res_counter(a.N));
-    p.xd = (uint8_t *)ws + ws_counter_bytes(a.N);
+    p.grid = p.cnt + ws_grid_counter();
+    p.res = reinterpret_cast<unsigned long long *>(p.cnt + ws_res_counter());
+    p.xd = (uint8_t *)ws + ws_counter_bytes();
     p.part = (int32_t *)(p.xd + (size_t)p.KB * NR * 128);
     int G = sm_count < kI8MaxCtas ? sm_count : kI8MaxCtas;
     if (G > p.U)

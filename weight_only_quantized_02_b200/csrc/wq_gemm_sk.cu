@@ -491,7 +491,7 @@ static cudaError_t launch_gemm_sk_t(const LinearArgs &a, int ctas_per_sm, void *
     p.zeros = (const uint8_t *)a.zeros;
     p.y = a.y;
     p.cnt = (uint32_t *)ws;
-    p.part = (float *)((uint8_t *)ws + ws_counter_bytes(a.N));
+    p.part = (float *)((uint8_t *)ws + ws_counter_bytes());
     const int per_sm = (ctas_per_sm >= 1 && ctas_per_sm < C::kOcc) ? ctas_per_sm : C::kOcc;
     int G = per_sm * sm_count;
     if (G > kSkMaxCtas)

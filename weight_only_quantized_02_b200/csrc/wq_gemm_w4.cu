@@ -529,7 +529,7 @@ static cudaError_t launch_gemm_w4_t(const LinearArgs &a, void *ws, int sm_count,
     p.zeros = (const uint8_t *)a.zeros;
     p.y = a.y;
     p.cnt = (uint32_t *)ws;
-    p.part = (float *)((uint8_t *)ws + ws_counter_bytes(a.N));
+    p.part = (float *)((uint8_t *)ws + ws_counter_bytes());
     int G = sm_count;
     if (G > kSkMaxCtas)
         G = kSkMaxCtas;

@@ -806,7 +806,7 @@ size_t ws_bytes_gemv_i8(int M, int K, int N)
     if (M < 1 || M > kGiMaxM || K < 1 || K > kI8MaxK)
         return 0;
     const size_t NR = 8 * gi_ntiles(M);
-    return ws_counter_bytes(N) + (size_t)kGiMaxWarps * 2 * 16 * NR * 4;
+    return ws_counter_bytes() + (size_t)kGiMaxWarps * 2 * 16 * NR * 4;
 }
 
 // The work split of a grid of G CTAs of `warps` warps: chunks per row block,
@@ -850,7 +850,7 @@ static cudaError_t launch_gi_t(const LinearArgs &a, void *ws, int sm_count, cuda
     p.zeros = (const uint8_t *)a.zeros;
     p.y = a.y;
     p.cnt = (uint32_t *)ws;
-    p.part = (uint32_t *)((uint8_t *)ws + ws_counter_bytes(a.N));
+    p.part = (uint32_t *)((uint8_t *)ws + ws_counter_bytes());
     p.wmax = trailer_wmax(a.wq, sh);
     int G = per_sm * sm_count;
     if (G * WARPS > kGiMaxWarps)

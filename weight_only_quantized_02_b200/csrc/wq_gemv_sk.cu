@@ -429,7 +429,7 @@ static cudaError_t launch_sk_t(const LinearArgs &a, void *ws, int sm_count, cuda
     p.KB = sh.kblocks();
     p.U = sh.panels() * sh.kblocks();
     p.cnt = (uint32_t *)ws;
-    p.part = (float *)((uint8_t *)ws + ws_counter_bytes(a.N));
+    p.part = (float *)((uint8_t *)ws + ws_counter_bytes());
     int G = per_sm * sm_count;
     if (G > kSkMaxCtas)
         G = kSkMaxCtas;

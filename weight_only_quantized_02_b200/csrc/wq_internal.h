@@ -23,32 +23,37 @@ struct LinearArgs {
 };
 
 // Split-K workspace: [counters, 256-byte padded][partials].
-// Counters: 8 tickets per 128-row panel (one per 16-row block; the GEMM uses
-// the first panel-count entries), then two grid counters of the integer
-// path (ws_grid_counter).  Every kernel leaves the counters it used at zero.
-// GEMM with S splits: partials [S][M][N].  Stream-K GEMV: partials
-// [CTAs <= kSkMaxCtas][2][128 rows][8 * ceil(M/8) tokens].
-// After the two grid counters: kResRows 64-bit residual sums of the integer
-// tensor-core path's exactness guard (one per token row), left at zero too.
+// Counters: a region of fixed size, the same for every shape, so that one
+// workspace serves layers of any N in turn (a smaller layer's partials never
+// land on a larger layer's counters): 8 tickets per 128-row panel for up to
+// kMaxN output channels (one per 16-row block; the GEMM uses the first
+// panel-count entries), then two grid counters of the integer path
+// (ws_grid_counter), then kResRows 64-bit residual sums of the integer
+// tensor-core path's exactness guard (one per token row).  Every kernel
+// leaves the counters it used at zero.  GEMM with S splits: partials
+// [S][M][N].  Stream-K GEMV: partials [CTAs <= kSkMaxCtas][2][128 rows][8 *
+// ceil(M/8) tokens].
 constexpr int kSkMaxCtas = 512;
 constexpr int kResRows = 64;
-inline size_t ws_counter_words(int N) { return (size_t)((N + 127) / 128) * 8 + 2 + 2 * kResRows; }
-inline size_t ws_counter_bytes(int N) { return (ws_counter_words(N) * 4 + 255) / 256 * 256; }
-inline size_t ws_grid_counter(int N) { return (size_t)((N + 127) / 128) * 8; } // word index of the first
-inline size_t ws_res_counter(int N) { return ws_grid_counter(N) + 2; }          // word index, 8-byte aligned
+constexpr int kMaxN = 1 << 20;                     // output channels of a layer
+constexpr int kCounterPanels = kMaxN / 128;
+inline size_t ws_counter_words() { return (size_t)kCounterPanels * 8 + 2 + 2 * kResRows; }
+inline size_t ws_counter_bytes() { return (ws_counter_words() * 4 + 255) / 256 * 256; }
+inline size_t ws_grid_counter() { return (size_t)kCounterPanels * 8; } // word index of the first
+inline size_t ws_res_counter() { return ws_grid_counter() + 2; }       // word index, 8-byte aligned
 inline size_t ws_bytes(int M, int N, int S)
 {
-    return ws_counter_bytes(N) + (S > 1 ? (size_t)S * M * N * sizeof(float) : 0);
+    return ws_counter_bytes() + (S > 1 ? (size_t)S * M * N * sizeof(float) : 0);
 }
 inline int gemm_token_tile(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
 inline size_t ws_bytes_gemm_sk(int M, int N)
 {
-    return ws_counter_bytes(N) + (size_t)kSkMaxCtas * 2 * 128 * gemm_token_tile(M) * sizeof(float);
+    return ws_counter_bytes() + (size_t)kSkMaxCtas * 2 * 128 * gemm_token_tile(M) * sizeof(float);
 }
 inline size_t ws_bytes_gemv_sk(int M, int N)
 {
     const int tok = 8 * ((M + 7) / 8);
-    return ws_counter_bytes(N) + (size_t)kSkMaxCtas * 2 * 128 * tok * sizeof(float);
+    return ws_counter_bytes() + (size_t)kSkMaxCtas * 2 * 128 * tok * sizeof(float);
 }
 
 // Integer tensor-core GEMMs (W8A16 and W4A16): M <= kI8MaxM, K <= kI8MaxK, at

@@ -85,7 +85,9 @@ def test_workspace_bytes():
     C = 262912
     assert wq.wq_workspace_bytes(128, 5120, 5120, 32) == C + 32 * 128 * 5120 * 4
     assert wq.wq_workspace_bytes(64, 5120, 5120, 1) == C + 512 * 2 * 128 * 64 * 4
-    assert wq.wq_workspace_bytes(16, 5120, 5120, 1) == C + 512 * 2 * 128 * 16 * 4
+    # M = 16: the integer tensor-core GEMM's digit blocks (40 k-blocks x 48 digit rows x 128) and int32
+    # partials [2 CTAs per SM x 160][2][48][128]
+    assert wq.wq_workspace_bytes(16, 5120, 5120, 1) == C + 40 * 48 * 128 + 320 * 2 * 48 * 128 * 4
     # M = 8: the integer GEMV's per-warp partials 448 CTAs x 8 warps x 2 x 16 rows x 24 x 4 bytes
     assert wq.wq_workspace_bytes(8, 5120, 5120, 1) == C + 448 * 8 * 2 * 16 * 24 * 4
     assert wq.wq_workspace_bytes(1, 5120, 17408, 1) == C + 512 * 2 * 128 * 16 * 4

@@ -24,7 +24,8 @@
 // MMA reads it, and the SM's threads never touch the weights.
 //
 // Work split: stream-K.  The (panel, k-block) units form one stream; CTA c of
-// G (one per SM) takes units [U*c/G, U*(c+1)/G).  Warp roles (192 threads):
+// G (two per SM where two rings fit, for NR <= 48, else one) takes units
+// [U*c/G, U*(c+1)/G).  Warp roles (192 threads):
 //   warp 0     producer: per unit one 16 KB bulk copy of the weight block and
 //              one of the unit's digit block (L2-resident) into a ring; the
 //              first stages' weights are issued before the programmatic-launch
@@ -41,10 +42,11 @@
 //              whole panel, else store int32 partials and take a ticket; the
 //              last arriver for a panel's rows sums every contributor's
 //              partial (integer sums: exact in any order) and writes y.
-// All G CTAs are resident at once (one per SM, G <= SMs), so the grid
-// counter wait always ends; the last CTA to exit resets it.  For small M the
-// ring fits two CTAs per SM, so the next call's CTAs can stream their first
-// weights while this call's last CTAs finish.
+// The grid is one wave (G <= CTAs per SM x SMs), so every CTA becomes
+// resident (a dependent kernel launches only after every CTA of this grid
+// has started) and the grid counter wait always ends; the last CTA to exit
+// resets it.  For small M (NR <= 48) two CTAs share an SM, each with its own
+// ring and producer thread: twice the weight copies in flight per SM.
 // Every wait is bounded (2 s); on a timeout the device error word is set and
 // the CTA winds down.
 #include <cstdint>
@@ -402,7 +404,8 @@ size_t ws_bytes_gemm_i8(int M, int K, int N)
         return 0;
     const int NR = i8_digit_rows(M);
     const size_t KB = (size_t)(K + kBlockK - 1) / kBlockK;
-    return ws_counter_bytes() + KB * NR * 128 + (size_t)kI8MaxCtas * 2 * NR * 128 * sizeof(int32_t);
+    const size_t ctas = (size_t)(NR <= 48 ? 2 : 1) * kI8MaxCtas; // the grid: CTAs per SM x at most kI8MaxCtas SMs
+    return ws_counter_bytes() + KB * NR * 128 + ctas * 2 * NR * 128 * sizeof(int32_t);
 }
 
 template <int NR>
@@ -432,7 +435,11 @@ static cudaError_t launch_i8_t(const LinearArgs &a, void *ws, int sm_count, cuda
     p.res = reinterpret_cast<unsigned long long *>(p.cnt + ws_res_counter());
     p.xd = (uint8_t *)ws + ws_counter_bytes();
     p.part = (int32_t *)(p.xd + (size_t)p.KB * NR * 128);
-    int G = sm_count < kI8MaxCtas ? sm_count : kI8MaxCtas;
+    // two CTAs per SM where they fit: twice the weight copies in flight per
+    // SM (one producer thread and its ring per CTA)
+    constexpr int occ = I8Cfg<NR>::kOcc;
+    static_assert(occ == (NR <= 48 ? 2 : 1), "workspace sizing (ws_bytes_gemm_i8) follows the occupancy");
+    int G = occ * (sm_count < kI8MaxCtas ? sm_count : kI8MaxCtas);
     if (G > p.U)
         G = p.U;
     cudaLaunchConfig_t cfg = {};

@@ -97,6 +97,17 @@ struct W4Cfg {
     static_assert(kXS % 2 == 0 && kAS % 2 == 0 && kACC % 2 == 0, "rings the MMA issuers wait on are even");
 };
 
+// d0 += a b0, d1 += a b1: one packed fp32 FMA (each half rounded as fmaf).
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float a, float b0, float b1)
+{
+    unsigned long long d, aa, bb;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(d0), "f"(d1));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(aa) : "f"(a));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(bb) : "f"(b0), "f"(b1));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(aa), "l"(bb));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+}
+
 // 16-byte asynchronous global -> shared copy (L2 only) and its groups.
 __device__ __forceinline__ void cp_async_cg16(uint32_t dst, const void *src)
 {
@@ -398,8 +409,8 @@ __global__ void __launch_bounds__(W4Cfg<NT>::kThreads, 1) gemm_w4_kernel(const _
                 for (int h = 0; h < RC / 16; ++h)
                     if (j0 + 16 * h < CW)
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            tot[j0 + 16 * h + j] = fmaf(s, v[h][j], tot[j0 + 16 * h + j]);
+                        for (int j = 0; j < 16; j += 2)
+                            ffma2(tot[j0 + 16 * h + j], tot[j0 + 16 * h + j + 1], s, v[h][j], v[h][j + 1]);
             }
             tc_fence_before();
             __syncwarp();

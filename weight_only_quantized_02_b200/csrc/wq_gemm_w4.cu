@@ -271,7 +271,6 @@ __global__ void __launch_bounds__(W4Cfg<NT>::kThreads, 1) gemm_w4_kernel(const _
     bool ok = true;
 
     auto panel_of = [&](int i) { return (u0 + i) / KB; };
-    auto last_of_panel = [&](int i) { return i == n - 1 || panel_of(i + 1) != panel_of(i); };
 
     if (warp == 0) {
         // ---------------- scale producer ----------------
@@ -387,6 +386,7 @@ __global__ void __launch_bounds__(W4Cfg<NT>::kThreads, 1) gemm_w4_kernel(const _
             ++nfix;
         };
 
+        int kb = u0 % KB; // k-block of unit i, kept without dividing
         for (int i = 0; i < n; ++i) {
             const int ac = i % ACC, ss = i % SS;
             if (!mbar_wait_warp(&accfull[ac], (i / ACC) & 1) || !mbar_wait_warp(&sfull[ss], (i / SS) & 1)) {
@@ -418,12 +418,13 @@ __global__ void __launch_bounds__(W4Cfg<NT>::kThreads, 1) gemm_w4_kernel(const _
                 mbar_arrive(&accempty[ac]);
                 mbar_arrive(&sempty[ss]);
             }
-            if (last_of_panel(i)) {
+            if (i == n - 1 || kb == KB - 1) { // the last unit of a panel
                 flush(panel_of(i));
 #pragma unroll
                 for (int j = 0; j < CW; ++j)
                     tot[j] = 0.f;
             }
+            kb = kb + 1 == KB ? 0 : kb + 1;
         }
         __syncwarp(); // lane 0's acquire (the tickets) orders every lane's reads below
         for (int f = 0; f < nfix && ok; ++f) {

@@ -160,9 +160,11 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
                 mbar_arrive_expect_tx(&full[st], C::kStageBytes);
                 bulk_g2s(ring + st * C::kStageBytes, p.wq + (size_t)(u0 + i) * C::kAB, C::kAB, &full[st], pol_w);
             };
+            int xkb = u0 % KB; // k-block of the next digit block issued, kept without dividing
             auto issue_x = [&](int i, int st) {
-                const int kb = (u0 + i) % KB;
-                bulk_g2s(ring + st * C::kStageBytes + C::kAB, p.xd + (size_t)kb * C::kBB, C::kBB, &full[st], pol_x);
+                (void)i;
+                bulk_g2s(ring + st * C::kStageBytes + C::kAB, p.xd + (size_t)xkb * C::kBB, C::kBB, &full[st], pol_x);
+                xkb = xkb + 1 == KB ? 0 : xkb + 1;
             };
             const int pre = n < STAGES ? n : STAGES;
             for (int i = 0; i < pre; ++i) // weights never depend on the preceding kernel
@@ -196,9 +198,8 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = umma_idesc_s8(NR);
-            int seg = -1;
-            for (int i = 0; i < n; ++i) {
-                const int u = u0 + i, kb = u % KB;
+            int seg = -1, kb = u0 % KB; // k-block of unit i, kept without dividing
+            for (int i = 0; i < n; ++i, kb = kb + 1 == KB ? 0 : kb + 1) {
                 const bool first = (i == 0 || kb == 0), last = (i == n - 1 || kb == KB - 1);
                 const int st = i % STAGES, use = i / STAGES;
                 if (first) {

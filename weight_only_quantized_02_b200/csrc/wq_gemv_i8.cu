@@ -607,14 +607,6 @@ __global__ void __launch_bounds__(WARPS * 32, 16 / WARPS) gemv_i8_kernel(const G
                 load_slot(s, wb[s], sz[s]);
         next_chunk();
     }
-    if (n > 1) { // the warp's next chunk into L2 while the preceding kernel ends (its
-                 // registers hold the first one; two chunks ahead measured slower)
-        const size_t blk = (size_t)(lrb >> 3) * KB + D * lq;
-        const int j = lrb & 7;
-        const uint8_t *b = BITS == 8 ? p.wq + (blk << 14) + (j << 11) + 64 * lane : p.wq + ((blk * 8 + j) << 10) + 32 * lane;
-        for (int s = 0; s < D && D * lq + s < KB; ++s)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(b + (size_t)s * kWStep));
-    }
 
     // ---------------- activations: this CTA's digit rows ----------------
     if (threadIdx.x < kGiMaxM) {

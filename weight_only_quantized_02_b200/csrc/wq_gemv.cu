@@ -254,14 +254,16 @@ __device__ __forceinline__ void gemv_int4_slice(const GemvParams &p, int rb, int
     const int g = lane >> 2, t = lane & 3;
     const int KL = p.K / LG;     // groups per row
     const int pnl = rb >> 3, rowp = 16 * (rb & 7) + g; // row inside the panel
-    const uint8_t *base = p.wq + 16 * lane;
+    // this lane's 16 bytes of the row block's tiles: (rb, k-block bi) is 1 KB
+    // at ((panel KB + bi) 8 + rb % 8) KB, its two 64-k tiles 512 B apart
+    const uint8_t *base = p.wq + ((size_t)pnl * p.sh.kblocks() * 8 + (rb & 7)) * 1024 + 16 * lane;
     uint4 cw[UG][2], nw[UG][2];
     uint16_t cs[UG][NG][2], ns[UG][NG][2];
     uint8_t cz[UG][NG][2], nz[UG][NG][2];
     auto load = [&](int bi, uint4 (&w)[2], uint16_t (&sc)[NG][2], uint8_t (&z)[NG][2]) {
         if (bi < b1) {
-            w[0] = ldg_stream(base + p.sh.tile_offset(rb, 2 * bi));
-            w[1] = ldg_stream(base + p.sh.tile_offset(rb, 2 * bi + 1));
+            w[0] = ldg_stream(base + (size_t)bi * 8192);
+            w[1] = ldg_stream(base + (size_t)bi * 8192 + 512);
 #pragma unroll
             for (int j = 0; j < NG; ++j) {
                 const size_t grp = (size_t)pnl * KL + (size_t)bi * NG + j;

@@ -390,6 +390,27 @@ __device__ __forceinline__ int sk_owner(long long U, int G, int u)
     return c;
 }
 
+// The stream-K cuts of the grid, computed once per CTA (one 64-bit division
+// per thread) so that the flushes and fix-ups look them up instead of
+// dividing: start[c] is the first unit of CTA c, first[c] its first panel.
+struct SkTable {
+    const int *start, *first;
+    // CTA whose range holds unit u: the largest c with start[c] <= u (ranges
+    // may be empty; the largest such c has start[c + 1] > u)
+    __device__ __forceinline__ int owner(int u, int G) const
+    {
+        int lo = 0, hi = G - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (start[mid] <= u)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        return lo;
+    }
+};
+
 // ---------------------------------------------------------------------------
 // Integer -> bf16 conversions (exact; written from the IEEE-754 encodings).
 // ---------------------------------------------------------------------------

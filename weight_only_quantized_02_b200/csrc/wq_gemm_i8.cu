@@ -101,7 +101,7 @@ constexpr size_t i8_smem_bytes()
     // ring + barriers (full, empty per stage; accfull, accempty x 2) +
     // tensor-memory slot + row maxima / exponents + residual bounds
     return 1024 + (size_t)I8Cfg<NR>::kStages * I8Cfg<NR>::kStageBytes + (2 * I8Cfg<NR>::kStages + 4) * 8 + 16 +
-           2 * kI8MaxM * 4 + kI8MaxM * 8;
+           2 * kI8MaxM * 4 + kI8MaxM * 8 + (size_t)2 * (2 * kI8MaxCtas + 1) * 4;
 }
 
 template <int NR>
@@ -122,6 +122,8 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
     uint32_t *s_amax = s_tmem + 4;                        // [kI8MaxM] row maxima (bf16 magnitude bits)
     int *s_e = reinterpret_cast<int *>(s_amax + kI8MaxM); // [kI8MaxM] exponents e_m
     double *s_rb = reinterpret_cast<double *>(s_e + kI8MaxM); // [kI8MaxM] residual bounds (8-byte aligned)
+    int *s_start = reinterpret_cast<int *>(s_rb + kI8MaxM);    // [G + 1] stream-K cuts
+    int *s_first = s_start + 2 * kI8MaxCtas + 1;              // [G + 1] first panel of each range
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, c = blockIdx.x;
@@ -143,6 +145,11 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
     }
     if (threadIdx.x < kI8MaxM)
         s_amax[threadIdx.x] = 0u;
+    for (int i = threadIdx.x; i <= G; i += blockDim.x) {
+        const int st = sk_start(U, G, i);
+        s_start[i] = st;
+        s_first[i] = st / KB;
+    }
     if (warp == 1) {
         tmem_alloc(s_tmem, TCOLS);
         tmem_relinquish();
@@ -151,6 +158,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+    const SkTable sk{s_start, s_first};
     bool ok = true;
 
     if (warp == 0) {
@@ -244,7 +252,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
             const int lo = max(u0, pnl * KB), hi = min(u1, (pnl + 1) * KB);
             const bool whole = (lo == pnl * KB && hi == (pnl + 1) * KB);
             const int b = seg & 1;
-            const int cf = sk_owner(U, G, pnl * KB), cl = sk_owner(U, G, (pnl + 1) * KB - 1);
+            const int cf = sk.owner(pnl * KB, G), cl = sk.owner((pnl + 1) * KB - 1, G);
             // A split panel whose other contributors have all taken their tickets
             // (typically the last segment of the range: its partner did its part
             // first): this warp is the last arriver.  It reads their partials now,
@@ -264,7 +272,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
                     for (int cc = cf; cc <= cl; ++cc) {
                         if (cc == c)
                             continue;
-                        const int sl = (pnl == sk_start(U, G, cc) / KB) ? 0 : 1;
+                        const int sl = (pnl == sk.first[cc]) ? 0 : 1;
                         const int32_t *src = p.part + (size_t)(cc * 2 + sl) * NR * 128 + row;
                         int32_t v[CG];
 #pragma unroll
@@ -283,7 +291,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
             tc_fence_after();
             const int nrow = pnl * kPanelRows + row;
             const double s_n = nrow < p.N ? (double)bf16_bits_to_float(p.scales[nrow]) : 0.0;
-            const int slot = (pnl == u0 / KB) ? 0 : 1;
+            const int slot = (pnl == sk.first[c]) ? 0 : 1;
             int32_t *mine = p.part + (size_t)(c * 2 + slot) * NR * 128;
 #pragma unroll
             for (int c0 = 0; c0 < NR; c0 += CG) {
@@ -348,7 +356,7 @@ __global__ void __launch_bounds__(kI8Threads, I8Cfg<NR>::kOcc) gemm_i8_kernel(co
                 for (int j = 0; j < CG; ++j)
                     tot[j] = 0;
                 for (int cc = cf; cc <= cl; ++cc) { // all CG loads of a contributor in flight together
-                    const int sl = (pnl == sk_start(U, G, cc) / KB) ? 0 : 1;
+                    const int sl = (pnl == sk.first[cc]) ? 0 : 1;
                     const int32_t *src = p.part + (size_t)(cc * 2 + sl) * NR * 128 + row;
                     int32_t v[CG];
 #pragma unroll

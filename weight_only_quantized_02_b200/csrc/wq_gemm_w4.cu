@@ -129,27 +129,6 @@ constexpr size_t gemm_w4_smem_bytes()
            (size_t)2 * (kSkMaxCtas + 1) * sizeof(int);
 }
 
-// The stream-K cuts of the grid, computed once per CTA (one 64-bit division
-// per thread) so that the flushes and fix-ups look them up instead of
-// dividing: start[c] is the first unit of CTA c, first[c] its first panel.
-struct SkTable {
-    const int *start, *first;
-    // CTA whose range holds unit u: the largest c with start[c] <= u (ranges
-    // may be empty; the largest such c has start[c + 1] > u)
-    __device__ __forceinline__ int owner(int u, int G) const
-    {
-        int lo = 0, hi = G - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (start[mid] <= u)
-                lo = mid;
-            else
-                hi = mid - 1;
-        }
-        return lo;
-    }
-};
-
 // The last contributor to a split panel: sums the fp32 partials of CTAs
 // cf .. cl for its row r and tokens t0 .. t0 + CW - 1 in CTA order and
 // writes y.  The partials are token-major, so every load is one coalesced

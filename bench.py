@@ -206,18 +206,27 @@ class ClockSampler:
 def profile_traffic(src_file: str, summary_name: str, M: int):
     """DRAM bytes per launch (read + write) of this kernel at this M, from the
     committed ncu summary -- only if it was captured on the current kernel
-    source (its sha256 is recorded in the summary)."""
+    source: the summary records a sha256 for every source file it covers
+    (the kernel's own file among them), and each must match the file now."""
     path = os.path.join(ROOT, "profiles", summary_name)
-    src = os.path.join(ROOT, "weight_only_quantized_02_b200", "csrc", src_file)
+    csrc = os.path.join(ROOT, "weight_only_quantized_02_b200", "csrc")
     try:
-        text = open(path).read()
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        lines = [ln.strip().lstrip("- ") for ln in open(path).read().splitlines()]
     except OSError:
         return None
-    if f"source_sha256: {sha}" not in text:
+    covered = {}
+    for a, b in zip(lines, lines[1:]):
+        if a.startswith("source_sha256:") and b.startswith("source:"):
+            covered[os.path.basename(b.split(":", 1)[1].strip().strip("`"))] = a.split(":", 1)[1].strip()
+    if src_file not in covered:
         return None
-    for line in text.splitlines():
-        line = line.strip().lstrip("- ")
+    for name, sha in covered.items():
+        try:
+            if hashlib.sha256(open(os.path.join(csrc, name), "rb").read()).hexdigest() != sha:
+                return None
+        except OSError:
+            return None
+    for line in lines:
         if line.startswith(f"traffic_bytes_per_launch M={M}:"):
             try:
                 return float(line.split(":", 1)[1])

@@ -24,3 +24,34 @@ def test_reference_arm_prints_one_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_profile_traffic_needs_every_listed_source_current(tmp_path, monkeypatch):
+    """The roofline's traffic comes from a committed ncu summary only while
+    every source file the summary lists (the kernel's own file among them)
+    still has the sha256 recorded there."""
+    import hashlib
+    sys.path.insert(0, ROOT)
+    import bench
+    csrc = tmp_path / "weight_only_quantized_02_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (csrc / "k.cu").write_text("kernel\n")
+    (csrc / "h.cuh").write_text("header\n")
+
+    def summary(files):
+        body = ["# k", "", "- traffic_bytes_per_launch M=16: 1234", ""]
+        for f in files:
+            sha = hashlib.sha256((csrc / f).read_bytes()).hexdigest()
+            body += [f"- source_sha256: {sha}", f"- source: `weight_only_quantized_02_b200/csrc/{f}`"]
+        (tmp_path / "profiles" / "k.md").write_text("\n".join(body) + "\n")
+
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    summary(["k.cu", "h.cuh"])
+    assert bench.profile_traffic("k.cu", "k.md", 16) == 1234.0
+    assert bench.profile_traffic("k.cu", "k.md", 1) is None  # no figure for this M
+    assert bench.profile_traffic("other.cu", "k.md", 16) is None  # the kernel's file is not covered
+    (csrc / "h.cuh").write_text("header, changed\n")
+    assert bench.profile_traffic("k.cu", "k.md", 16) is None  # a listed header changed since the capture
+    summary(["h.cuh"])
+    assert bench.profile_traffic("k.cu", "k.md", 16) is None  # the kernel's own file unlisted

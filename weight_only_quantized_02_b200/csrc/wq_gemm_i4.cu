@@ -96,10 +96,11 @@ constexpr size_t i4_smem_bytes()
     using C = I4Cfg<NR>;
     // rings + barriers (pfull, pempty per packed stage; xfull, xempty per
     // digit stage; afull, aempty per A tile; accfull, accempty per
-    // accumulator) + tensor-memory slot + row maxima / exponents
+    // accumulator) + tensor-memory slot + row maxima / exponents + residual
+    // bounds + the stream-K table
     return 1024 + (size_t)C::kRingBytes +
            (2 * C::kPStages + 2 * C::kDStages + 2 * C::kAStages + 2 * C::kTB) * 8 + 16 + 2 * kI8MaxM * 4 +
-           kI8MaxM * 8;
+           kI8MaxM * 8 + (size_t)2 * (kI8MaxCtas + 1) * 4;
 }
 
 // Eight nibbles of one packed word (runs a, b of one row; positions
@@ -151,6 +152,8 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
     uint32_t *s_amax = s_tmem + 4;                        // [kI8MaxM]
     int *s_e = reinterpret_cast<int *>(s_amax + kI8MaxM); // [kI8MaxM]
     double *s_rb = reinterpret_cast<double *>(s_e + kI8MaxM); // [kI8MaxM] residual bounds (8-byte aligned)
+    int *s_start = reinterpret_cast<int *>(s_rb + kI8MaxM);    // [G + 1] stream-K cuts
+    int *s_first = s_start + kI8MaxCtas + 1;                  // [G + 1] first panel of each range
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, c = blockIdx.x;
@@ -180,6 +183,11 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
     }
     if (threadIdx.x < kI8MaxM)
         s_amax[threadIdx.x] = 0u;
+    for (int i = threadIdx.x; i <= G; i += blockDim.x) {
+        const int st = sk_start(U, G, i);
+        s_start[i] = st;
+        s_first[i] = st / KB;
+    }
     if (warp == 1) {
         tmem_alloc(s_tmem, TCOLS);
         tmem_relinquish();
@@ -188,6 +196,7 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+    const SkTable sk{s_start, s_first};
     bool ok = true;
 
     if (warp == 0) {
@@ -206,10 +215,12 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
                 bulk_g2s(dst + C::kPB, p.zeros + u * 64, 64, &pfull[st], pol_w);
                 bulk_g2s(dst + C::kPB + 64, p.scales + u * kPanelRows, 256, &pfull[st], pol_w);
             };
+            int xkb = u0 % KB; // k-block of the next digit block issued (units in order), kept without dividing
             auto issue_x = [&](int i) {
-                const int sd = i % SD, kb = (u0 + i) % KB;
+                const int sd = i % SD;
                 mbar_arrive_expect_tx(&xfull[sd], C::kBB);
-                bulk_g2s(dring + sd * C::kBB, p.xd + (size_t)kb * C::kBB, C::kBB, &xfull[sd], pol_x);
+                bulk_g2s(dring + sd * C::kBB, p.xd + (size_t)xkb * C::kBB, C::kBB, &xfull[sd], pol_x);
+                xkb = xkb + 1 == KB ? 0 : xkb + 1;
             };
             const int pre = n < SP ? n : SP;
             for (int i = 0; i < pre; ++i) // weights never depend on the preceding kernel
@@ -342,8 +353,8 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
 #pragma unroll
         for (int m = 0; m < MM; ++m)
             acc[m] = 0.f;
+        int pnl = u0 / KB, kb = u0 - pnl * KB; // panel and k-block of unit i, kept without dividing
         for (int i = 0; i < n && ok; ++i) {
-            const int u = u0 + i, pnl = u / KB, kb = u - pnl * KB;
             const int b = i % TB;
             if (!mbar_wait_warp(&accfull[b], (i / TB) & 1)) {
                 ok = false;
@@ -392,7 +403,7 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
                                                   wmax * s_rb[m], lane);
                         break;
                     }
-                    const int slot = (pnl == u0 / KB) ? 0 : 1;
+                    const int slot = (pnl == sk.first[c]) ? 0 : 1;
                     float *mine = p.part + (size_t)(c * 2 + slot) * MM * 128 + row;
 #pragma unroll
                     for (int m = 0; m < MM; ++m)
@@ -403,7 +414,7 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
                     if (lane == 0)
                         ticket = ticket_take_acq_rel(&p.cnt[pnl * 4 + quad]);
                     ticket = __shfl_sync(0xffffffffu, ticket, 0);
-                    const int cf = sk_owner(U, G, pnl * KB), cl = sk_owner(U, G, (pnl + 1) * KB - 1);
+                    const int cf = sk.owner(pnl * KB, G), cl = sk.owner((pnl + 1) * KB - 1, G);
                     if (ticket != (uint32_t)(cl - cf))
                         break;
                     __syncwarp(); // lane 0's acquire orders every lane's reads below
@@ -412,7 +423,7 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
                     for (int m = 0; m < MM; ++m)
                         tot[m] = 0.f;
                     for (int cc = cf; cc <= cl; ++cc) { // contributors in CTA order: deterministic
-                        const int sl = (pnl == sk_start(U, G, cc) / KB) ? 0 : 1;
+                        const int sl = (pnl == sk.first[cc]) ? 0 : 1;
                         const float *src = p.part + (size_t)(cc * 2 + sl) * MM * 128 + row;
                         float v[MM];
 #pragma unroll
@@ -434,6 +445,10 @@ __global__ void __maxnreg__(128) gemm_i4_kernel(const I4Params p)
 #pragma unroll
                 for (int m = 0; m < MM; ++m)
                     acc[m] = 0.f;
+            }
+            if (++kb == KB) {
+                kb = 0;
+                ++pnl;
             }
         }
         pdl_launch_dependents();

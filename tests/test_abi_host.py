@@ -97,6 +97,32 @@ def test_workspace_bytes():
     assert wq.wq_workspace_bytes(1, 0, 5120, 4) == 0
 
 
+def test_topk_workspace_bytes():
+    # the bf16 logits M x N (padded to 256 bytes), then P candidates of k
+    # 64-bit (key, index) words per token; P slices of 4096 logits, or of
+    # 8192 when the 4096-logit grid (P x M CTAs) would not fit the GPU at
+    # once (4 CTAs x 148 SMs = 592)
+    def expect(M, N, k, S):
+        P = -(-N // S)
+        return -(-(M * N * 2) // 256) * 256 + M * P * k * 8
+    V = 152064  # the vocabulary head: 38 slices of 4096, or 19 of 8192
+    assert wq.wq_topk_workspace_bytes(1, V, 64) == expect(1, V, 64, 4096) == 304128 + 38 * 64 * 8
+    assert wq.wq_topk_workspace_bytes(4, V, 64) == expect(4, V, 64, 4096)
+    assert wq.wq_topk_workspace_bytes(15, V, 64) == expect(15, V, 64, 4096)  # 570 CTAs: one wave
+    assert wq.wq_topk_workspace_bytes(16, V, 64) == expect(16, V, 64, 8192)  # 608 CTAs: wider slices
+    assert wq.wq_topk_workspace_bytes(128, V, 1) == expect(128, V, 1, 8192)
+    assert wq.wq_topk_workspace_bytes(1, 1, 1) == 256 + 8
+    assert wq.wq_topk_workspace_bytes(2, 4097, 3) == 256 * 65 + 2 * 2 * 3 * 8  # a ragged last slice
+    # outside the limits: no scratch
+    assert wq.wq_topk_workspace_bytes(0, V, 64) == 0
+    assert wq.wq_topk_workspace_bytes(1, V, 65) == 0  # k > 64
+    assert wq.wq_topk_workspace_bytes(1, 8, 9) == 0   # k > N
+    assert wq.wq_topk_workspace_bytes(1, V, 0) == 0
+    # the merge keeps P k candidates (two 32-bit words each) in shared memory, at most 200 KB
+    assert wq.wq_topk_workspace_bytes(1, 367 * 4096, 64) == expect(1, 367 * 4096, 64, 4096)
+    assert wq.wq_topk_workspace_bytes(1, 368 * 4096, 64) == 0
+
+
 def test_null_pointer_checks_need_no_device():
     assert wq.lib.wq_linear(None, 1, 1024, None, None, None, 0, 1024, None, None) == -1
     assert wq.lib.wq_pack_int8(None, None, 1024, 1024, None, None, None) == -1

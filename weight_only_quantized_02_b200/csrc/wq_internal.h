@@ -56,10 +56,11 @@ inline size_t ws_bytes_gemv_sk(int M, int N)
     return ws_counter_bytes() + (size_t)kSkMaxCtas * 2 * 128 * tok * sizeof(float);
 }
 
-// Integer tensor-core GEMMs (W8A16 and W4A16): M <= kI8MaxM, K <= kI8MaxK, at
-// most kI8MaxCtas persistent CTAs.  Workspace: [counters][digit blocks
-// KB x NR x 128][partials: INT8 int32 kI8MaxCtas x 2 x NR x 128, INT4 fp32
-// kI8MaxCtas x 2 x NR/3 x 128].
+// Integer tensor-core GEMMs (W8A16 and W4A16): M <= kI8MaxM, K <= kI8MaxK,
+// persistent CTAs: INT8 two per SM up to 48 digit rows (16 tokens), else one,
+// INT4 one, with at most kI8MaxCtas per CTA-per-SM.  Workspace: [counters]
+// [digit blocks KB x NR x 128][partials: INT8 int32 (2 or 1) kI8MaxCtas x 2 x
+// NR x 128, INT4 fp32 kI8MaxCtas x 2 x NR/3 x 128].
 constexpr int kI8MaxM = 64;
 static_assert(kI8MaxM <= kResRows, "one residual sum per token row");
 constexpr int kI4MaxM = 32; // W4A16 on the integer path
@@ -101,8 +102,8 @@ cudaError_t launch_gemm(const LinearArgs &a, int split, void *ws, int sm_count, 
 cudaError_t launch_gemm_sk(const LinearArgs &a, int ctas_per_sm, void *ws, int sm_count, cudaStream_t st);
 cudaError_t read_gemm_sk_error(int *code, cudaStream_t st);
 
-// W4A16 stream-K GEMM (the GEMM_SK variant for 4-bit weights): one
-// 512-thread CTA per SM; ws >= ws_bytes_gemm_sk.
+// Role-split W4A16 stream-K GEMM (GEMM_W4): one CTA per SM (16 warps; 20 at
+// 64 tokens); ws >= ws_bytes_gemm_sk.
 cudaError_t launch_gemm_w4(const LinearArgs &a, void *ws, int sm_count, cudaStream_t st);
 cudaError_t read_gemm_w4_error(int *code, cudaStream_t st);
 

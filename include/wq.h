@@ -383,6 +383,23 @@ int wq_gemv_i8_plan(int bits, int K, int N, int G, int warps, int *meta, int *ru
 int wq_gemv_i8_contributors(int bits, int K, int N, int G, int warps, int rb, int *warp_ids, int *slots,
                             int *count);
 
+/* Debug view of the stream-K cuts shared by the persistent kernels (the
+ * stream-K GEMV and GEMM, GEMM_W4, the integer tensor-core GEMMs), computed
+ * by the kernels' own partition code on the host (no GPU). The pages have
+ * no counterpart beyond naming stream-K ("Marlin register and launch
+ * scheduling benchmark"); the tests check the partition with it.
+ * The weights are U units (128-row panel x 128-k block, panel-major, KB
+ * k-blocks per panel); CTA c of G takes units [start[c], start[c + 1]).
+ *   start[G + 1]    each CTA's first unit (start[G] = U)
+ *   first[G + 1]    each CTA's first panel, start[c] / KB
+ *   owner_table[U]  the CTA whose range holds unit u, by the binary search
+ *                   over the per-CTA table (the fix-ups' lookup)
+ *   owner_div[U]    the same by the division form
+ * Host buffers owned by the caller. Returns WQ_ERR_NULL for a null pointer,
+ * WQ_ERR_SHAPE unless 1 <= G <= U <= 2^31 - 1 and KB >= 1 (every launcher
+ * caps its grid at the unit count). */
+int wq_stream_k_plan(long long U, int G, int KB, int *start, int *first, int *owner_table, int *owner_div);
+
 #ifdef __cplusplus
 }
 #endif

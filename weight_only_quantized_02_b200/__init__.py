@@ -82,6 +82,7 @@ def _load():
         "wq_wait_selftest": (I, [I, P]),
         "wq_gemv_i8_plan": (I, [I, I, I, I, I, P, P]),
         "wq_gemv_i8_contributors": (I, [I, I, I, I, I, I, P, P, P]),
+        "wq_stream_k_plan": (I, [ctypes.c_longlong, I, I, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -371,6 +372,18 @@ def wq_gemv_i8_plan(bits: int, K: int, N: int, G: int, warps: int = 16):
     _check(lib.wq_gemv_i8_plan(bits, K, N, G, warps, meta, runs), "wq_gemv_i8_plan")
     return dict(CPR=meta[0], LB=meta[1], RB0=meta[2], RL=meta[3]), \
         [[tuple(runs[(c * warps + w) * 4:(c * warps + w) * 4 + 4]) for w in range(warps)] for c in range(G)]
+
+
+def wq_stream_k_plan(U: int, G: int, KB: int):
+    """The stream-K cuts of U units over G CTAs (KB k-blocks per panel), host
+    only: (start [G + 1], first panel [G + 1], owner of every unit by the
+    per-CTA table, the same by the division form)."""
+    start = (ctypes.c_int * (G + 1))()
+    first = (ctypes.c_int * (G + 1))()
+    own_t = (ctypes.c_int * max(U, 1))()
+    own_d = (ctypes.c_int * max(U, 1))()
+    _check(lib.wq_stream_k_plan(U, G, KB, start, first, own_t, own_d), "wq_stream_k_plan")
+    return list(start), list(first), list(own_t)[:U], list(own_d)[:U]
 
 
 def wq_gemv_i8_contributors(bits: int, K: int, N: int, G: int, warps: int, rb: int, cpr: int):

@@ -23,7 +23,7 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libwq.so")
 
 SOURCES = ["wq_api.cu", "wq_pack.cu", "wq_gemv.cu", "wq_gemv_sk.cu", "wq_gemv_i8.cu", "wq_gemm.cu", "wq_gemm_sk.cu",
-           "wq_gemm_i8.cu", "wq_gemm_i4.cu", "wq_gemm_w4.cu", "wq_topk.cu"]
+           "wq_gemm_i8.cu", "wq_gemm_i4.cu", "wq_gemm_w4.cu", "wq_topk.cu", "wq_sk_debug.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

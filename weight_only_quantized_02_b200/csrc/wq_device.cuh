@@ -375,10 +375,10 @@ __device__ __forceinline__ uint32_t ticket_take_acq_rel(uint32_t *counter)
 // Stream-K partition: U units cut into G contiguous ranges [start(c),
 // start(c+1)); a panel of consecutive units may span several ranges.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int sk_start(long long U, int G, int c) { return (int)(U * c / G); }
+WQ_HD int sk_start(long long U, int G, int c) { return (int)(U * c / G); }
 
 // CTA that owns unit u (ranges [start(c), start(c+1)); empty ranges skipped)
-__device__ __forceinline__ int sk_owner(long long U, int G, int u)
+WQ_HD int sk_owner(long long U, int G, int u)
 {
     int c = (int)(((long long)u * G) / U);
     if (c >= G)
@@ -397,7 +397,7 @@ struct SkTable {
     const int *start, *first;
     // CTA whose range holds unit u: the largest c with start[c] <= u (ranges
     // may be empty; the largest such c has start[c + 1] > u)
-    __device__ __forceinline__ int owner(int u, int G) const
+    WQ_HD int owner(int u, int G) const
     {
         int lo = 0, hi = G - 1;
         while (lo < hi) {

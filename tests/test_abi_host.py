@@ -129,6 +129,25 @@ def test_null_pointer_checks_need_no_device():
     assert wq.lib.wq_quantize_int4(None, 1024, 16, 128, None, None, None, None) == -1
 
 
+def test_topk_argument_checks_need_no_device():
+    # every check of wq_linear_topk runs before its first CUDA call; the
+    # pointers here are never dereferenced
+    f = wq.lib.wq_linear_topk
+    P = ctypes.c_void_p
+    x, w, s, z, v, i = (P(0x10000 * n) for n in range(1, 7))
+    ws = P(0x100000)
+    V = 152064
+    need = wq.wq_topk_workspace_bytes(4, V, 64)
+
+    def call(M=4, N=V, k=64, vals=v, idx=i, scratch=ws, nbytes=need):
+        return f(x, M, 5120, w, s, z, 0, N, k, vals, idx, scratch, nbytes, None)
+    for kw in (dict(M=0), dict(M=129), dict(k=0), dict(k=65), dict(N=32, k=33), dict(M=1, N=368 * 4096)):
+        assert call(**kw) == -2, kw  # WQ_ERR_SHAPE
+    assert call(vals=None) == -1 and call(idx=None) == -1 and call(scratch=None) == -1  # WQ_ERR_NULL
+    assert call(scratch=P(0x100008)) == -3  # WQ_ERR_ALIGN: the scratch must be 16-byte aligned
+    assert call(nbytes=need - 1) == -6  # WQ_ERR_WORKSPACE
+
+
 def test_tuning_file_parse_errors(tmp_path):
     good = tmp_path / "good.txt"
     good.write_text("# comment\nNVIDIA B200|148 1 5120 17408 8 0 0 4 12.500\n"

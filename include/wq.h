@@ -109,8 +109,8 @@ typedef enum {
                                 3 * M * K bytes of digits plus 16-48 KB of partial sums <= 226 KB;
                                 split 1 = one 16-warp CTA per SM, 2 = two 8-warp CTAs per SM; needs
                                 the workspace */
-#define WQ_VARIANT_GEMM_W4 6 /* W4A16 only, M <= 128: stream-K tcgen05 GEMM with one 512-thread CTA
-                                per SM, every role (weight and x loads, dequantization, MMA, group
+#define WQ_VARIANT_GEMM_W4 6 /* W4A16 only, M <= 128: stream-K tcgen05 GEMM with one CTA per SM
+                                (16 warps; 20 at 64 tokens), every role (weight and x loads, dequantization, MMA, group
                                 rescale) on its own warps with its own ring; needs the workspace */
 
 /* Static description of a status code. Host. Never NULL. */
